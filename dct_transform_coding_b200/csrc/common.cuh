@@ -1,0 +1,173 @@
+// Shared device code of the TACT-KV codec kernels (internal header).
+//
+// The method is the one of the TACT-KV summary page ("TACT-KV: Tri-Axis Cosine Transform for
+// Compressing Volumetric KV Caches in Medical VLMs"), "Methodology in Plain English"; the C ABI,
+// payload format and calling rules are in include/tactkv.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include <cstdint>
+
+#include "tactkv.h"
+
+namespace tactkv {
+
+constexpr uint32_t kMagic = 0x31564B54u;   // "TKV1"
+constexpr int kVersion = 1;
+constexpr int kMaxUnits = 64;              // units per launch (descriptors travel as kernel parameters)
+constexpr int kHeaderBytes = 64;
+constexpr int kChunk = 32;                 // channels per H/W-axis CTA
+constexpr int kPairs = kChunk / 2;         // channel pairs: every pencil carries two channels (float2)
+constexpr int kHwThreads = 256;
+constexpr int kAllocThreads = 1024;
+constexpr size_t kStatusBytes = 256;       // status word at the start of the workspace
+constexpr int kMaxHW = 1024;               // H*W limit of the H/W-axis kernels
+
+enum HwMode { kStats = 0, kQuant = 1, kRaw = 2 };
+
+// ------------------------------------------------------------------------ launch descriptors ---
+struct UnitDev {
+  const void* in;
+  void* out;
+  unsigned char* payload;
+  long long tok_stride, head_stride;   // elements
+  int layer, kv;
+};
+struct UnitList {
+  UnitDev u[kMaxUnits];
+};
+struct Geom {
+  int S, H, W, HW, T, heads, head_dim, n, nch, N, bits, flags;
+  int off_sigma, off_codes;     // payload byte offsets
+  long long capacity;           // payload bytes available (minimum over the launch)
+};
+
+__host__ __device__ inline long long pad16(long long x) { return (x + 15) / 16 * 16; }
+
+// Codebook b (1..8) has 2^b - 1 thresholds and 2^b levels, stored for b = 1, 2, ... in turn.
+__host__ __device__ constexpr int lm_thr_offset(int b) { return (1 << b) - b - 1; }
+__host__ __device__ constexpr int lm_lv_offset(int b) { return (1 << b) - 2; }
+constexpr int kLmThrTotal = lm_thr_offset(9);   // 502
+constexpr int kLmLvTotal = lm_lv_offset(9);     // 510
+
+// Length classes: a kernel instantiated for class C holds pencils of up to C values in
+// registers and dispatches only the generated lengths of that class.
+inline bool supported_length(int L) {
+  if (L >= 1 && L <= 16) return true;
+  switch (L) {
+    case 20: case 24: case 28: case 32: case 40: case 48: case 56: case 64: return true;
+    default: return false;
+  }
+}
+inline int length_class(int L) { return L <= 16 ? 16 : (L <= 32 ? 32 : 64); }
+
+// Shared memory of the H/W-axis kernels.
+__host__ __device__ inline int stream_words_per_slab(int HW) { return (8 * HW + 31) / 32 + 2; }
+__host__ __device__ inline size_t hw_smem_bytes(int HW) {
+  const size_t w = stream_words_per_slab(HW);
+  return (size_t)HW * kPairs * 8 + (size_t)(kLmThrTotal + kLmLvTotal) * 4 + (size_t)HW * 4 * 3 +
+         (size_t)kChunk * w * 4 + kChunk * 4 + 33 * 4 + 64;
+}
+
+// --------------------------------------------------------------------------------- launchers ---
+cudaError_t launch_axis_s(int cls, bool inverse, const Geom& g, const UnitList& ul, int nu, float* buf,
+                          cudaStream_t st);
+cudaError_t launch_axis_hw(int hcls, int wcls, bool inverse, int mode, const Geom& g, const UnitList& ul, int nu, float* buf,
+                           float* partial, unsigned int* status, cudaStream_t st);
+cudaError_t launch_allocate(const Geom& g, const UnitList& ul, int nu, const float* partial, double* var,
+                            cudaStream_t st);
+
+#ifdef __CUDACC__
+// ------------------------------------------------------------------ float2 value operations ---
+// Every pencil carries two channels; the packed f32x2 instructions issue both halves at once.
+__device__ __forceinline__ float2 vadd(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 vsub(float2 a, float2 b) { return __ffma2_rn(b, make_float2(-1.f, -1.f), a); }
+__device__ __forceinline__ float2 vneg(float2 a) { return make_float2(-a.x, -a.y); }
+__device__ __forceinline__ float2 vmul(float2 a, float c) { return __fmul2_rn(a, make_float2(c, c)); }
+__device__ __forceinline__ float2 vfma(float2 a, float c, float2 b) { return __ffma2_rn(a, make_float2(c, c), b); }
+
+// the generated pencil transforms (templates over the value type) live in this namespace too
+#include "dct_gen.cuh"
+
+// Orthonormal DCT-II (INV = false) or DCT-III (INV = true) of x[0..L) held in registers.
+template <int CLASS, bool INV>
+__device__ __forceinline__ void dct_pencil(float2* x, int L) {
+#define TACTKV_CASE(n)                          \
+  case n:                                       \
+    if constexpr (INV) idct_##n(x);             \
+    else fdct_##n(x);                           \
+    break;
+  if constexpr (CLASS == 16) {
+    switch (L) {
+      TACTKV_CASE(1) TACTKV_CASE(2) TACTKV_CASE(3) TACTKV_CASE(4) TACTKV_CASE(5) TACTKV_CASE(6)
+      TACTKV_CASE(7) TACTKV_CASE(8) TACTKV_CASE(9) TACTKV_CASE(10) TACTKV_CASE(11) TACTKV_CASE(12)
+      TACTKV_CASE(13) TACTKV_CASE(14) TACTKV_CASE(15) TACTKV_CASE(16)
+      default: break;
+    }
+  } else if constexpr (CLASS == 32) {
+    switch (L) {
+      TACTKV_CASE(20) TACTKV_CASE(24) TACTKV_CASE(28) TACTKV_CASE(32)
+      default: break;
+    }
+  } else {
+    switch (L) {
+      TACTKV_CASE(40) TACTKV_CASE(48) TACTKV_CASE(56) TACTKV_CASE(64)
+      default: break;
+    }
+  }
+#undef TACTKV_CASE
+}
+
+__device__ __forceinline__ void set_status(unsigned int* status, unsigned int code) { atomicCAS(status, 0u, code); }
+
+__device__ __forceinline__ float2 load_pair(const void* base, long long elem, bool fp32) {
+  if (fp32) return *reinterpret_cast<const float2*>(static_cast<const float*>(base) + elem);
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(static_cast<const __nv_bfloat16*>(base) + elem));
+}
+__device__ __forceinline__ void store_pair(void* base, long long elem, float2 v, bool fp32) {
+  if (fp32) *reinterpret_cast<float2*>(static_cast<float*>(base) + elem) = v;
+  else *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(base) + elem) = __float22bfloat162_rn(v);
+}
+
+// In place exclusive scan of a[0..n) in shared memory; blockDim.x a multiple of 32; returns the total.
+__device__ inline uint32_t block_exclusive_scan(uint32_t* a, int n, uint32_t* s_warp /* 33 entries */) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int per = (n + blockDim.x - 1) / blockDim.x;
+  const int beg = min(n, (int)threadIdx.x * per), end = min(n, beg + per);
+  uint32_t sum = 0;
+  for (int i = beg; i < end; ++i) sum += a[i];
+  uint32_t incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t w = lane < nwarps ? s_warp[lane] : 0u;
+    uint32_t wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += t;
+    }
+    s_warp[lane] = wi - w;
+    if (lane == 31) s_warp[32] = wi;
+  }
+  __syncthreads();
+  uint32_t run = s_warp[warp] + incl - sum;
+  for (int i = beg; i < end; ++i) {
+    const uint32_t v = a[i];
+    a[i] = run;
+    run += v;
+  }
+  const uint32_t total = s_warp[32];
+  __syncthreads();
+  return total;
+}
+#endif  // __CUDACC__
+
+}  // namespace tactkv

@@ -1,0 +1,262 @@
+// TACT-KV codec C ABI (host side): argument checks, grouping of units into waves, launches.
+//
+// A compress wave (up to kMaxUnits units of identical shape) runs four kernels on the
+// caller's stream: the forward DCT along S (axis_s.cu), the forward DCT along H and W with
+// per-bin energy sums (axis_hw.cu, kStats), the per-unit allocation and payload header
+// (allocate.cu) and the H/W pass again with quantization and packing (axis_hw.cu, kQuant),
+// which reads the S-transformed volume kept in the workspace.  A decompress wave runs the
+// inverse H/W pass (dequantize + inverse DCT along W and H) and the inverse DCT along S.
+#include <algorithm>
+#include <cstring>
+
+#include "common.cuh"
+#include "lloyd_max_tables.inc"
+
+namespace tactkv {
+
+cudaError_t launch_axis_s_16(bool, const Geom&, const UnitList&, int, float*, cudaStream_t);
+cudaError_t launch_axis_s_32(bool, const Geom&, const UnitList&, int, float*, cudaStream_t);
+cudaError_t launch_axis_s_64(bool, const Geom&, const UnitList&, int, float*, cudaStream_t);
+#define TACTKV_DECL_HW(h, w)                                                                                   \
+  cudaError_t launch_axis_hw_##h##_##w(bool, int, const Geom&, const UnitList&, int, float*, float*, unsigned int*, \
+                                       cudaStream_t);
+TACTKV_DECL_HW(16, 16)
+TACTKV_DECL_HW(16, 32)
+TACTKV_DECL_HW(32, 16)
+TACTKV_DECL_HW(32, 32)
+#undef TACTKV_DECL_HW
+
+cudaError_t launch_axis_s(int cls, bool inverse, const Geom& g, const UnitList& ul, int nu, float* buf,
+                          cudaStream_t st) {
+  if (cls == 16) return launch_axis_s_16(inverse, g, ul, nu, buf, st);
+  if (cls == 32) return launch_axis_s_32(inverse, g, ul, nu, buf, st);
+  return launch_axis_s_64(inverse, g, ul, nu, buf, st);
+}
+
+cudaError_t launch_axis_hw(int hcls, int wcls, bool inverse, int mode, const Geom& g, const UnitList& ul, int nu,
+                           float* buf, float* partial, unsigned int* status, cudaStream_t st) {
+  if (hcls == 16 && wcls == 16) return launch_axis_hw_16_16(inverse, mode, g, ul, nu, buf, partial, status, st);
+  if (hcls == 16) return launch_axis_hw_16_32(inverse, mode, g, ul, nu, buf, partial, status, st);
+  if (wcls == 16) return launch_axis_hw_32_16(inverse, mode, g, ul, nu, buf, partial, status, st);
+  return launch_axis_hw_32_32(inverse, mode, g, ul, nu, buf, partial, status, st);
+}
+
+namespace {
+
+tactkv_status make_geom(const tactkv_unit& u, Geom& g) {
+  if (u.bits < 1 || u.bits > 8) return TACTKV_INVALID_ARG;
+  if (u.flags & ~(TACTKV_NO_QUANT | TACTKV_FP32_IO)) return TACTKV_INVALID_ARG;
+  if (u.S < 1 || u.H < 1 || u.W < 1 || u.heads < 1 || u.head_dim < 1) return TACTKV_INVALID_ARG;
+  if (!supported_length(u.S) || !supported_length(u.H) || !supported_length(u.W)) return TACTKV_UNSUPPORTED_SHAPE;
+  if (u.H > 32 || u.W > 32 || u.H * u.W > kMaxHW) return TACTKV_UNSUPPORTED_SHAPE;
+  const long long n = (long long)u.heads * u.head_dim;
+  if (n % kChunk != 0 || u.head_dim % 2 != 0 || n > (1 << 16)) return TACTKV_UNSUPPORTED_SHAPE;
+  const long long N = (long long)u.S * u.H * u.W;
+  g.S = u.S;
+  g.H = u.H;
+  g.W = u.W;
+  g.HW = u.H * u.W;
+  g.T = (int)N;
+  g.heads = u.heads;
+  g.head_dim = u.head_dim;
+  g.n = (int)n;
+  g.nch = (int)(n / kChunk);
+  g.N = (int)N;
+  g.bits = u.bits;
+  g.flags = (int)u.flags;
+  g.off_sigma = (int)(kHeaderBytes + pad16(g.N));
+  g.off_codes = (int)(g.off_sigma + pad16(4LL * g.N));
+  g.capacity = 0;
+  return TACTKV_OK;
+}
+
+size_t payload_bytes_geom(const Geom& g) {
+  const long long bits_per_chan = (g.flags & TACTKV_NO_QUANT) ? 32LL * g.N : (long long)g.bits * g.N;
+  return (size_t)(g.off_codes + (long long)g.n * pad16((bits_per_chan + 7) / 8));
+}
+
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+// workspace of one unit: the S-transformed volume (fp32), per-chunk energy sums, fp64 variances
+size_t unit_ws_bytes(const Geom& g) {
+  return round256((size_t)g.T * g.n * 4) + round256((size_t)g.nch * g.N * 4) + round256((size_t)g.N * 8);
+}
+
+struct WsView {
+  unsigned int* status;
+  float* big;      // nu * T * n floats: Y (compress) or V (decompress)
+  float* partial;  // nu * nch * N floats
+  double* var;     // nu * N doubles
+};
+
+WsView view(unsigned char* ws, const Geom& g, int nu) {
+  WsView v;
+  v.status = reinterpret_cast<unsigned int*>(ws);
+  size_t off = kStatusBytes;
+  v.big = reinterpret_cast<float*>(ws + off);
+  off += round256((size_t)nu * g.T * g.n * 4);
+  v.partial = reinterpret_cast<float*>(ws + off);
+  off += round256((size_t)nu * g.nch * g.N * 4);
+  v.var = reinterpret_cast<double*>(ws + off);
+  return v;
+}
+
+bool same_group(const tactkv_unit& a, const tactkv_unit& b) {
+  return a.S == b.S && a.H == b.H && a.W == b.W && a.heads == b.heads && a.head_dim == b.head_dim &&
+         a.bits == b.bits && a.flags == b.flags;
+}
+
+tactkv_status check_unit(const tactkv_unit& u, const Geom& g, bool compress) {
+  const size_t elem = (u.flags & TACTKV_FP32_IO) ? 4 : 2;
+  const void* io = compress ? u.kv_in : static_cast<const void*>(u.kv_out);
+  if (!io || !u.payload) return TACTKV_INVALID_ARG;
+  if (u.token_stride <= 0 || u.head_stride < 0) return TACTKV_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(io) % (2 * elem)) || (u.token_stride % 2) || (u.head_stride % 2))
+    return TACTKV_ALIGNMENT;
+  if (reinterpret_cast<uintptr_t>(u.payload) % 16) return TACTKV_ALIGNMENT;
+  if (u.payload_capacity < payload_bytes_geom(g)) return TACTKV_CAPACITY;
+  return TACTKV_OK;
+}
+
+template <class F>
+tactkv_status for_each_wave(const tactkv_unit* units, int n_units, void* ws, size_t ws_bytes, bool compress,
+                            F&& fn) {
+  if (n_units < 0 || (n_units > 0 && !units)) return TACTKV_INVALID_ARG;
+  if (n_units == 0) return TACTKV_OK;
+  if (!ws || ws_bytes < kStatusBytes || reinterpret_cast<uintptr_t>(ws) % 256) return TACTKV_WORKSPACE;
+  int i = 0;
+  while (i < n_units) {
+    int j = i + 1;
+    while (j < n_units && same_group(units[i], units[j])) ++j;
+    Geom g;
+    tactkv_status st = make_geom(units[i], g);
+    if (st != TACTKV_OK) return st;
+    long long cap = -1;
+    for (int k = i; k < j; ++k) {
+      st = check_unit(units[k], g, compress);
+      if (st != TACTKV_OK) return st;
+      cap = cap < 0 ? (long long)units[k].payload_capacity : std::min(cap, (long long)units[k].payload_capacity);
+    }
+    g.capacity = cap;
+    const size_t per = unit_ws_bytes(g);
+    const int wave = (int)std::min<size_t>(kMaxUnits, (ws_bytes - kStatusBytes) / per);
+    if (wave < 1) return TACTKV_WORKSPACE;
+    for (int k = i; k < j; k += wave) {
+      const int nu = std::min(wave, j - k);
+      UnitList ul;
+      memset(&ul, 0, sizeof(ul));
+      for (int q = 0; q < nu; ++q) {
+        const tactkv_unit& s = units[k + q];
+        ul.u[q].in = s.kv_in;
+        ul.u[q].out = s.kv_out;
+        ul.u[q].payload = static_cast<unsigned char*>(s.payload);
+        ul.u[q].tok_stride = s.token_stride;
+        ul.u[q].head_stride = s.head_stride;
+        ul.u[q].layer = s.layer;
+        ul.u[q].kv = s.kv;
+      }
+      st = fn(g, ul, nu, static_cast<unsigned char*>(ws));
+      if (st != TACTKV_OK) return st;
+    }
+    i = j;
+  }
+  return TACTKV_OK;
+}
+
+}  // namespace
+}  // namespace tactkv
+
+using namespace tactkv;
+
+extern "C" {
+
+size_t tactkv_payload_bytes(const tactkv_unit* unit) {
+  if (!unit) return 0;
+  Geom g;
+  if (make_geom(*unit, g) != TACTKV_OK) return 0;
+  return payload_bytes_geom(g);
+}
+
+size_t tactkv_workspace_bytes(const tactkv_unit* units, int n_units) {
+  size_t best = 0;
+  int i = 0;
+  while (units && i < n_units) {
+    int j = i + 1;
+    while (j < n_units && same_group(units[i], units[j])) ++j;
+    Geom g;
+    if (make_geom(units[i], g) == TACTKV_OK)
+      best = std::max(best, (size_t)std::min(kMaxUnits, j - i) * unit_ws_bytes(g));
+    i = j;
+  }
+  return kStatusBytes + best;
+}
+
+tactkv_status tactkv_compress(const tactkv_unit* units, int n_units, void* workspace, size_t workspace_bytes,
+                              struct CUstream_st* stream) {
+  cudaStream_t st = stream;
+  return for_each_wave(units, n_units, workspace, workspace_bytes, true,
+                       [&](const Geom& g, const UnitList& ul, int nu, unsigned char* ws) -> tactkv_status {
+                         const WsView w = view(ws, g, nu);
+                         const int cs = length_class(g.S), ch = length_class(g.H), cw = length_class(g.W);
+                         const int mode2 = (g.flags & TACTKV_NO_QUANT) ? kRaw : kQuant;
+                         if (launch_axis_s(cs, false, g, ul, nu, w.big, st) != cudaSuccess) return TACTKV_CUDA;
+                         if (launch_axis_hw(ch, cw, false, kStats, g, ul, nu, w.big, w.partial, w.status, st) !=
+                             cudaSuccess)
+                           return TACTKV_CUDA;
+                         if (launch_allocate(g, ul, nu, w.partial, w.var, st) != cudaSuccess) return TACTKV_CUDA;
+                         if (launch_axis_hw(ch, cw, false, mode2, g, ul, nu, w.big, w.partial, w.status, st) !=
+                             cudaSuccess)
+                           return TACTKV_CUDA;
+                         return TACTKV_OK;
+                       });
+}
+
+tactkv_status tactkv_decompress(const tactkv_unit* units, int n_units, void* workspace, size_t workspace_bytes,
+                                struct CUstream_st* stream) {
+  cudaStream_t st = stream;
+  return for_each_wave(units, n_units, workspace, workspace_bytes, false,
+                       [&](const Geom& g, const UnitList& ul, int nu, unsigned char* ws) -> tactkv_status {
+                         const WsView w = view(ws, g, nu);
+                         const int cs = length_class(g.S), ch = length_class(g.H), cw = length_class(g.W);
+                         const int mode = (g.flags & TACTKV_NO_QUANT) ? kRaw : kQuant;
+                         if (launch_axis_hw(ch, cw, true, mode, g, ul, nu, w.big, nullptr, w.status, st) != cudaSuccess)
+                           return TACTKV_CUDA;
+                         if (launch_axis_s(cs, true, g, ul, nu, w.big, st) != cudaSuccess) return TACTKV_CUDA;
+                         return TACTKV_OK;
+                       });
+}
+
+tactkv_status tactkv_device_status(void* workspace, size_t workspace_bytes, struct CUstream_st* stream) {
+  if (!workspace || workspace_bytes < kStatusBytes) return TACTKV_WORKSPACE;
+  unsigned int v = 0;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return TACTKV_CUDA;
+  if (cudaMemcpy(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return TACTKV_CUDA;
+  if (cudaMemset(workspace, 0, sizeof(v)) != cudaSuccess) return TACTKV_CUDA;
+  return static_cast<tactkv_status>(v);
+}
+
+const char* tactkv_status_string(tactkv_status s) {
+  switch (s) {
+    case TACTKV_OK: return "ok";
+    case TACTKV_INVALID_ARG: return "invalid argument";
+    case TACTKV_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case TACTKV_CAPACITY: return "payload capacity too small";
+    case TACTKV_ALIGNMENT: return "misaligned pointer or stride";
+    case TACTKV_CORRUPT_PAYLOAD: return "corrupt payload";
+    case TACTKV_CUDA: return "CUDA error";
+    case TACTKV_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+int tactkv_lloyd_max_table(int bits, double* levels, double* thresholds) {
+  if (bits < 1 || bits > 8) return 0;
+  const int L = 1 << bits;
+  if (levels) memcpy(levels, kLmLevels + lm_lv_offset(bits), sizeof(double) * L);
+  if (thresholds) memcpy(thresholds, kLmThresholds + lm_thr_offset(bits), sizeof(double) * (L - 1));
+  return L;
+}
+
+int tactkv_format_version(void) { return kVersion; }
+
+}  // extern "C"

@@ -1,0 +1,221 @@
+"""Thin Python binding of libtactkv.so (include/tactkv.h): argument marshalling only.
+
+Every step of compression and decompression runs in the library's CUDA kernels.  PyTorch is
+used for device memory and streams: the helpers below allocate payload, output and workspace
+tensors and pass their device pointers to the C ABI.  If the shared library is missing the
+import fails; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import List, Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtactkv.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m dct_transform_coding_b200.build` "
+                      "(or __graft_entry__.build()); the codec has no CPU path")
+_lib = ctypes.CDLL(LIB_PATH)
+
+TACTKV_OK = 0
+TACTKV_INVALID_ARG = 1
+TACTKV_UNSUPPORTED_SHAPE = 2
+TACTKV_CAPACITY = 3
+TACTKV_ALIGNMENT = 4
+TACTKV_CORRUPT_PAYLOAD = 5
+TACTKV_CUDA = 6
+TACTKV_WORKSPACE = 7
+
+TACTKV_NO_QUANT = 1
+TACTKV_FP32_IO = 2
+
+HEADER_BYTES = 64
+EXPORTED = ("tactkv_payload_bytes", "tactkv_workspace_bytes", "tactkv_compress", "tactkv_decompress",
+            "tactkv_device_status", "tactkv_status_string", "tactkv_lloyd_max_table", "tactkv_format_version")
+
+
+class tactkv_unit(ctypes.Structure):
+    _fields_ = [
+        ("layer", ctypes.c_int32), ("kv", ctypes.c_int32),
+        ("S", ctypes.c_int32), ("H", ctypes.c_int32), ("W", ctypes.c_int32),
+        ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+        ("bits", ctypes.c_int32), ("flags", ctypes.c_uint32),
+        ("kv_in", ctypes.c_void_p), ("kv_out", ctypes.c_void_p),
+        ("token_stride", ctypes.c_int64), ("head_stride", ctypes.c_int64),
+        ("payload", ctypes.c_void_p), ("payload_capacity", ctypes.c_size_t),
+    ]
+
+
+_P = ctypes.POINTER(tactkv_unit)
+_lib.tactkv_payload_bytes.restype = ctypes.c_size_t
+_lib.tactkv_payload_bytes.argtypes = [_P]
+_lib.tactkv_workspace_bytes.restype = ctypes.c_size_t
+_lib.tactkv_workspace_bytes.argtypes = [_P, ctypes.c_int]
+for _name in ("tactkv_compress", "tactkv_decompress"):
+    getattr(_lib, _name).restype = ctypes.c_int
+    getattr(_lib, _name).argtypes = [_P, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+_lib.tactkv_device_status.restype = ctypes.c_int
+_lib.tactkv_device_status.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+_lib.tactkv_status_string.restype = ctypes.c_char_p
+_lib.tactkv_status_string.argtypes = [ctypes.c_int]
+_lib.tactkv_lloyd_max_table.restype = ctypes.c_int
+_lib.tactkv_lloyd_max_table.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]
+_lib.tactkv_format_version.restype = ctypes.c_int
+_lib.tactkv_format_version.argtypes = []
+
+
+class TactkvError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {tactkv_status_string(status)} ({status})")
+
+
+# ------------------------------------------------------------------------- raw C entry points ---
+def tactkv_payload_bytes(unit: tactkv_unit) -> int:
+    return int(_lib.tactkv_payload_bytes(ctypes.byref(unit)))
+
+
+def tactkv_workspace_bytes(units) -> int:
+    arr = _as_array(units)
+    return int(_lib.tactkv_workspace_bytes(arr, len(arr)))
+
+
+def tactkv_compress(units, workspace_ptr: int, workspace_bytes: int, stream_ptr: int) -> int:
+    arr = _as_array(units)
+    return int(_lib.tactkv_compress(arr, len(arr), ctypes.c_void_p(workspace_ptr), workspace_bytes,
+                                    ctypes.c_void_p(stream_ptr)))
+
+
+def tactkv_decompress(units, workspace_ptr: int, workspace_bytes: int, stream_ptr: int) -> int:
+    arr = _as_array(units)
+    return int(_lib.tactkv_decompress(arr, len(arr), ctypes.c_void_p(workspace_ptr), workspace_bytes,
+                                      ctypes.c_void_p(stream_ptr)))
+
+
+def tactkv_device_status(workspace_ptr: int, workspace_bytes: int, stream_ptr: int) -> int:
+    return int(_lib.tactkv_device_status(ctypes.c_void_p(workspace_ptr), workspace_bytes, ctypes.c_void_p(stream_ptr)))
+
+
+def tactkv_status_string(status: int) -> str:
+    return _lib.tactkv_status_string(int(status)).decode()
+
+
+def tactkv_lloyd_max_table(bits: int):
+    """The library's own codebook: (levels, thresholds) as lists of floats (host only)."""
+    L = 1 << bits
+    lv = (ctypes.c_double * L)()
+    th = (ctypes.c_double * max(1, L - 1))()
+    n = _lib.tactkv_lloyd_max_table(bits, lv, th)
+    if n != L:
+        raise ValueError("bits must be 1..8")
+    return list(lv), list(th)[:L - 1]
+
+
+def tactkv_format_version() -> int:
+    return int(_lib.tactkv_format_version())
+
+
+def _as_array(units):
+    if isinstance(units, ctypes.Array):
+        return units
+    units = list(units)
+    arr = (tactkv_unit * len(units))(*units)
+    return arr
+
+
+# ------------------------------------------------------------------------------ torch helpers ---
+def _stream_ptr(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def make_units(x: Optional[torch.Tensor], S: int, H: int, W: int, bits: int, *, heads: int, head_dim: int,
+               payload: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+               layers: Optional[Sequence[int]] = None, kvs: Optional[Sequence[int]] = None,
+               flags: int = 0, n_units: Optional[int] = None):
+    """Descriptors for a batch laid out as [units, tokens, heads, head_dim] (strided views allowed).
+
+    x is the compress input (or None for decompress), out the decompress output, payload a
+    [units, capacity] uint8 tensor."""
+    ref = x if x is not None else out
+    U = ref.shape[0] if n_units is None else n_units
+    arr = (tactkv_unit * U)()
+    for i in range(U):
+        u = arr[i]
+        u.layer = int(layers[i]) if layers is not None else i
+        u.kv = int(kvs[i]) if kvs is not None else 0
+        u.S, u.H, u.W, u.heads, u.head_dim, u.bits, u.flags = S, H, W, heads, head_dim, bits, flags
+        if x is not None:
+            u.kv_in = x[i].data_ptr()
+            u.token_stride, u.head_stride = x.stride(1), x.stride(2)
+        if out is not None:
+            u.kv_out = out[i].data_ptr()
+            u.token_stride, u.head_stride = out.stride(1), out.stride(2)
+        if payload is not None:
+            u.payload = payload[i].data_ptr()
+            u.payload_capacity = payload.shape[1]
+    return arr
+
+
+def payload_capacity(S: int, H: int, W: int, heads: int, head_dim: int, bits: int, flags: int = 0) -> int:
+    u = tactkv_unit(S=S, H=H, W=W, heads=heads, head_dim=head_dim, bits=bits, flags=flags)
+    cap = tactkv_payload_bytes(u)
+    if cap == 0:
+        raise TactkvError(TACTKV_UNSUPPORTED_SHAPE, "payload_capacity")
+    return cap
+
+
+def alloc_workspace(units, device) -> torch.Tensor:
+    nbytes = tactkv_workspace_bytes(units)
+    ws = torch.zeros(nbytes + 256, dtype=torch.uint8, device=device)
+    off = (-ws.data_ptr()) % 256
+    return ws[off:off + nbytes]
+
+
+def compress(x: torch.Tensor, S: int, H: int, W: int, bits: int, *, layers=None, kvs=None, flags: int = 0,
+             payload: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+             stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Compress x [units, S*H*W, heads, head_dim] (bf16, or fp32 with TACTKV_FP32_IO) on its device.
+    Returns the [units, capacity] uint8 payload tensor (asynchronous on the stream)."""
+    U, T, heads, D = x.shape
+    if x.dtype == torch.float32:
+        flags |= TACTKV_FP32_IO
+    cap = payload_capacity(S, H, W, heads, D, bits, flags)
+    if payload is None:
+        payload = torch.empty((U, (cap + 15) // 16 * 16), dtype=torch.uint8, device=x.device)
+    units = make_units(x, S, H, W, bits, heads=heads, head_dim=D, payload=payload, layers=layers, kvs=kvs,
+                       flags=flags)
+    if workspace is None:
+        workspace = alloc_workspace(units, x.device)
+    st = tactkv_compress(units, workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+    if st != TACTKV_OK:
+        raise TactkvError(st, "tactkv_compress")
+    return payload
+
+
+def decompress(payload: torch.Tensor, S: int, H: int, W: int, bits: int, *, heads: int, head_dim: int,
+               layers=None, kvs=None, flags: int = 0, dtype=torch.bfloat16, out: Optional[torch.Tensor] = None,
+               workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None,
+               check: bool = False) -> torch.Tensor:
+    """Decompress [units, capacity] payloads into [units, S*H*W, heads, head_dim]."""
+    U = payload.shape[0]
+    if dtype == torch.float32:
+        flags |= TACTKV_FP32_IO
+    if out is None:
+        out = torch.empty((U, S * H * W, heads, head_dim), dtype=dtype, device=payload.device)
+    units = make_units(None, S, H, W, bits, heads=heads, head_dim=head_dim, payload=payload, out=out,
+                       layers=layers, kvs=kvs, flags=flags, n_units=U)
+    if workspace is None:
+        workspace = alloc_workspace(units, payload.device)
+    st = tactkv_decompress(units, workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+    if st != TACTKV_OK:
+        raise TactkvError(st, "tactkv_decompress")
+    if check:
+        ds = tactkv_device_status(workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+        if ds != TACTKV_OK:
+            raise TactkvError(ds, "tactkv_decompress (device)")
+    return out

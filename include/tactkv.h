@@ -1,0 +1,128 @@
+/*
+ * tactkv.h -- C ABI of the B200 TACT-KV visual-KV transform codec.
+ *
+ * The operations are those of the TACT-KV summary page ("TACT-KV: Tri-Axis Cosine Transform for
+ * Compressing Volumetric KV Caches in Medical VLMs"), section "Methodology in Plain English":
+ *   stage 1  the visual K or V of one layer of one sequence is laid out on its (S, H, W) grid;
+ *   stage 2  a separable orthonormal 3D DCT-II runs along S, H and W (features untouched);
+ *   stage 3  per-bin variances (over all heads x head_dim channels) drive a reverse
+ *            water-filling split of the layer's bit budget: b_i = max(0, 1/2 log2(s_i^2/theta)),
+ *            theta by bisection, integer rounding, +-1 greedy fix to hit the budget, cap 8 bits;
+ *   stage 4  each surviving bin is scaled by its own gain s_i and every coordinate is quantized
+ *            with a fixed Lloyd-Max table of a unit Gaussian at the bin's bit width;
+ *   decoding reverses the stages (paragraph after stage 4).
+ *
+ * Terms.  A UNIT is one (sequence, layer, K|V) volume: T = S*H*W tokens by n = heads*head_dim
+ * channels.  Token t = (s*H + h)*W + w; channel c = head*head_dim + d.  Frequency bin
+ * i = (k_s*H + k_h)*W + k_w, N = T bins.  Nominal budget: bits*N bit slots per channel.
+ *
+ * Memory.  Every pointer in a unit descriptor and the workspace are DEVICE pointers owned by
+ * the caller.  The library allocates nothing, keeps no state other than constant tables in the
+ * CUDA module, and is safe to call from several host threads on different streams provided
+ * each call has its own workspace.  Calls are asynchronous on `stream`; a status other than
+ * TACTKV_OK means nothing was launched for the failing group of units (earlier groups of the
+ * same call may already be queued).  Errors found by the kernels (a corrupt payload) are
+ * recorded in the workspace and read back with tactkv_device_status().
+ *
+ * Payload format (version 1, little-endian), one self-describing blob per unit:
+ *   [0, 64)             header: u32 magic 0x31564B54 ("TKV1"), u16 version = 1, u16 flags,
+ *                       i32 layer, kv, S, H, W, heads, head_dim, bits, u32 code_bits (sum b_i,
+ *                       or 32*N with TACTKV_NO_QUANT), u32 chan_stride (bytes), u64 total_bytes,
+ *                       u32 0, u32 0
+ *   [64, +pad16(N))     u8 b[N]          bits of every bin (0..8; 0 = dropped)
+ *   then pad16(4N)      f32 sigma[N]     gain of every bin, float32(sqrt(sigma^2))
+ *   then n streams      channel c at offset off_codes + c*chan_stride, chan_stride =
+ *                       pad16(ceil(code_bits/8)); stream bit P_i + k is bit k (LSB first) of bin
+ *                       i's code, P_i = sum_{j<i} b_j; stream bit q is bit (q&7) of byte q>>3.
+ *                       With TACTKV_NO_QUANT a stream holds the N float32 coefficients instead.
+ * pad16(x) rounds x up to a multiple of 16.  The gain/rate part is the pages' sum(b_i*d + 32)
+ * bits per layer; the b[] bytes are its "small index overhead".
+ */
+#ifndef TACTKV_H_
+#define TACTKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st; /* cudaStream_t is `struct CUstream_st*`; NULL is the legacy default stream */
+
+typedef enum {
+  TACTKV_OK = 0,
+  TACTKV_INVALID_ARG = 1,        /* null pointer, n_units < 0, bits outside 1..8, bad flags */
+  TACTKV_UNSUPPORTED_SHAPE = 2,  /* an axis length or channel layout the kernels do not cover */
+  TACTKV_CAPACITY = 3,           /* payload_capacity below tactkv_payload_bytes() */
+  TACTKV_ALIGNMENT = 4,          /* a pointer or stride breaks the alignment rules below */
+  TACTKV_CORRUPT_PAYLOAD = 5,    /* (device status) a payload header or allocation is invalid */
+  TACTKV_CUDA = 6,               /* a CUDA launch or copy failed */
+  TACTKV_WORKSPACE = 7           /* workspace null or smaller than one unit needs */
+} tactkv_status;
+
+/* flags */
+#define TACTKV_NO_QUANT 1u /* transform only: store float32 coefficients (lossless round trip) */
+#define TACTKV_FP32_IO  2u /* K/V are float32 instead of bfloat16 */
+
+typedef struct {
+  int32_t layer;          /* recorded in the header, checked by decompress */
+  int32_t kv;             /* 0 = K, 1 = V; recorded and checked like layer */
+  int32_t S, H, W;        /* token grid; each axis 1..64 from the supported set (see below) */
+  int32_t heads, head_dim;/* n = heads*head_dim channels, n a multiple of 32, head_dim even */
+  int32_t bits;           /* nominal bits per element, 1..8 */
+  uint32_t flags;         /* TACTKV_NO_QUANT | TACTKV_FP32_IO */
+  const void* kv_in;      /* compress input: element (t, head, d) at
+                             kv_in + t*token_stride + head*head_stride + d (elements) */
+  void* kv_out;           /* decompress output, same indexing as kv_in */
+  int64_t token_stride;   /* in elements; even, > 0 */
+  int64_t head_stride;    /* in elements; even */
+  void* payload;          /* compress writes, decompress reads; 16-byte aligned */
+  size_t payload_capacity;/* bytes available at payload */
+} tactkv_unit;
+
+/* Supported axis lengths S, H, W: 1..16, 20, 24, 28, 32, 40, 48, 56, 64, with H*W <= 1024.
+   kv_in / kv_out must be 4-byte aligned (8-byte with TACTKV_FP32_IO).  */
+
+/* Worst-case payload size of one unit (every bin budget used): the capacity to provide. */
+size_t tactkv_payload_bytes(const tactkv_unit* unit);
+
+/* Workspace bytes that let compress/decompress process all `n_units` in one wave.  Any size of
+   at least tactkv_workspace_bytes(units, 1) works; the units are then processed in waves. */
+size_t tactkv_workspace_bytes(const tactkv_unit* units, int n_units);
+
+/* Compress every unit: read kv_in, write the payload.  Units with identical shape, bits and
+   flags that are adjacent in the array are batched into one set of launches.  Steps: forward
+   DCT along S; forward DCT along H and W with per-bin energy sums; per-unit bit allocation and
+   gains; the forward DCT again with quantization and bit packing. */
+tactkv_status tactkv_compress(const tactkv_unit* units, int n_units, void* workspace,
+                              size_t workspace_bytes, struct CUstream_st* stream);
+
+/* Decompress every unit: read the payload, write kv_out (bfloat16, or float32 with
+   TACTKV_FP32_IO) with the descriptor's strides.  The payload header must match the
+   descriptor (layer, kv, shape, bits, flags); a mismatch or an invalid allocation is recorded
+   as TACTKV_CORRUPT_PAYLOAD in the workspace and that unit's output is zero-filled. */
+tactkv_status tactkv_decompress(const tactkv_unit* units, int n_units, void* workspace,
+                                size_t workspace_bytes, struct CUstream_st* stream);
+
+/* Synchronizes `stream`, returns the first error the kernels recorded in `workspace` since the
+   previous call (TACTKV_OK if none), and clears it. */
+tactkv_status tactkv_device_status(void* workspace, size_t workspace_bytes,
+                                   struct CUstream_st* stream);
+
+/* Human-readable status name. */
+const char* tactkv_status_string(tactkv_status status);
+
+/* The library's own Lloyd-Max codebook for `bits` (1..8): 2^bits levels and 2^bits - 1
+   thresholds, increasing, written to the host arrays given.  Returns the number of levels, or
+   0 for bits outside 1..8.  Host-only; needs no GPU. */
+int tactkv_lloyd_max_table(int bits, double* levels, double* thresholds);
+
+/* Version of the payload format this library writes and reads. */
+int tactkv_format_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TACTKV_H_ */

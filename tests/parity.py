@@ -1,0 +1,92 @@
+"""Parity checks of the CUDA codec against the CPU oracle (shared by the GPU tests and smoke()).
+
+Acceptance, per unit (the codec's stated tolerances, with the readings needed to apply them):
+* bit allocations equal the oracle's exactly.  A differing bin is tolerated only as a tie
+  artefact: its deciding key sigma^2 4^-k lies within 1e-6 (relative) of the oracle's selection
+  threshold, where fp32-vs-fp64 variance estimates may legitimately swap the order;
+* quantization codes equal the oracle's, except where the oracle's scaled coefficient
+  u = X / sigma lies within 1e-5 * max(1, |t|) of a decision threshold t (distance taken in
+  sigma-scaled units, because the middle threshold is 0);
+* reconstructions: ||y_gpu - y_oracle|| / ||y_oracle|| <= 1e-3, both rounded to the I/O type;
+* with TACTKV_NO_QUANT the round trip matches the input within 1e-5 relative RMS.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from oracle import tactkv_oracle as O
+
+CODE_BAND = 1e-5
+RECON_TOL = 1e-3
+ROUNDTRIP_TOL = 1e-5
+TIE_TOL = 1e-6
+
+
+def rel_rms(a, b) -> float:
+    a = np.asarray(a, dtype=np.float64).ravel()
+    b = np.asarray(b, dtype=np.float64).ravel()
+    nb = np.linalg.norm(b)
+    return float(np.linalg.norm(a - b) / nb) if nb > 0 else float(np.linalg.norm(a - b))
+
+
+def selection_threshold(var: np.ndarray, bits: int) -> float:
+    """The B-th largest key sigma_i^2 4^-k of the oracle's allocation (inf if all active bins saturate)."""
+    act = var > 0
+    B = bits * var.size
+    if 8 * int(act.sum()) <= B:
+        return np.inf
+    keys = (var[act][:, None] * 4.0 ** -np.arange(8)[None, :]).ravel()
+    return float(np.partition(keys, keys.size - B)[keys.size - B])
+
+
+def compare_unit(x: np.ndarray, gpu_payload: bytes, gpu_recon: np.ndarray, *, S, H, W, heads, head_dim, bits,
+                 layer=0, kv=0, flags=0, io_round=O.to_bf16, report=None):
+    """Check one unit.  x: the input exactly as the GPU saw it; gpu_recon: the GPU decode of gpu_payload."""
+    no_quant = bool(flags & 1)
+    p_o, info = O.compress_unit(x, S, H, W, heads, head_dim, bits, layer=layer, kv=kv, no_quant=no_quant,
+                                return_info=True)
+    g = O.parse_payload(gpu_payload)
+    assert (g["layer"], g["kv"], g["S"], g["H"], g["W"], g["heads"], g["head_dim"], g["bits"]) == \
+        (layer, kv, S, H, W, heads, head_dim, bits)
+    assert bool(g["flags"] & 1) == no_quant
+    N = S * H * W
+    var = info["var"]
+    # gains: float32(sqrt(sigma^2)) from fp32 coefficients and fp64 sums
+    sig_o = info["sigma"].astype(np.float64)
+    sig_g = g["sigma"].astype(np.float64)
+    big = var > 1e-12 * max(var.max(), 1e-300)
+    assert np.all(np.abs(sig_g[big] - sig_o[big]) <= 2e-5 * sig_o[big]), "gain mismatch"
+    out = dict(tie_bins=0, code_mismatch_band=0, codes=0)
+    if no_quant:
+        Xg = g["streams"][:, :4 * N].copy().view("<f4").astype(np.float64).T
+        assert rel_rms(Xg, info["X"]) <= ROUNDTRIP_TOL
+    else:
+        b_o, b_g = info["b"], g["b"]
+        differ = np.nonzero(b_o != b_g)[0]
+        if differ.size:
+            thr = selection_threshold(var, bits)
+            for i in differ:
+                k = min(b_o[i], b_g[i])                     # the key that decides the extra bit
+                key = var[i] * 4.0 ** -k
+                assert abs(key / thr - 1) < TIE_TOL, f"allocation differs at bin {i}: {b_o[i]} vs {b_g[i]}"
+            out["tie_bins"] = int(differ.size)
+        assert b_g.sum() == g["code_bits"]
+        _, codes_g = O.codes_of(gpu_payload)
+        codes_o = info["codes"]
+        X = info["X"]
+        same = np.nonzero((b_o == b_g) & (b_o > 0))[0]
+        for i in same:
+            bad = codes_g[i] != codes_o[i]
+            out["codes"] += codes_o.shape[1]
+            if bad.any():
+                u = X[i, bad] / sig_o[i]
+                d = O.threshold_distance(u, int(b_o[i]))
+                assert np.all(d <= CODE_BAND), f"code mismatch outside the band at bin {i}: {d.max()}"
+                out["code_mismatch_band"] += int(bad.sum())
+    y_o = io_round(O.decompress_unit(p_o)).reshape(gpu_recon.shape)
+    err = rel_rms(gpu_recon, y_o)
+    out["recon_rel_rms"] = err
+    assert err <= (ROUNDTRIP_TOL if no_quant else RECON_TOL), f"reconstruction rel RMS {err}"
+    if report is not None:
+        report.append(out)
+    return out

@@ -1,0 +1,235 @@
+"""GPU parity of the CUDA codec (through the C ABI) against the CPU oracle.
+
+Every case generates its input once (seeded), hands the same tensor to the CUDA path and to
+the oracle, and applies the acceptance rules of tests/parity.py.  Sizes: small cases that span
+several 32-channel chunks and S slabs with ragged (non power of two) axes, the exact shapes of
+every benchmark workload on sampled units, and the degenerate inputs of the method.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import tactkv_oracle as O
+from dct_transform_coding_b200.workloads import WORKLOADS, make_unit, make_workload_unit
+
+from parity import compare_unit, rel_rms
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    from dct_transform_coding_b200 import tactkv as T
+
+DEV = "cuda:0"
+
+
+def _round_trip(x_dev, S, H, W, bits, layers=None, kvs=None, flags=0, workspace=None):
+    U, _, heads, D = x_dev.shape
+    pay = T.compress(x_dev, S, H, W, bits, layers=layers, kvs=kvs, flags=flags, workspace=workspace)
+    out_dtype = x_dev.dtype
+    y = T.decompress(pay, S, H, W, bits, heads=heads, head_dim=D, layers=layers, kvs=kvs, flags=flags,
+                     dtype=out_dtype, workspace=workspace, check=True)
+    torch.cuda.synchronize()
+    return pay, y
+
+
+def _check_batch(x_dev, S, H, W, bits, layers=None, kvs=None, flags=0, units=None, workspace=None):
+    U, _, heads, D = x_dev.shape
+    pay, y = _round_trip(x_dev, S, H, W, bits, layers, kvs, flags, workspace)
+    fp32 = x_dev.dtype == torch.float32
+    io_round = (lambda v: np.asarray(v, np.float32).astype(np.float64)) if fp32 else O.to_bf16
+    reports = []
+    for i in (range(U) if units is None else units):
+        x = x_dev[i].double().cpu().numpy()
+        gp = pay[i].cpu().numpy().tobytes()
+        yr = y[i].double().cpu().numpy()
+        compare_unit(x, gp, yr, S=S, H=H, W=W, heads=heads, head_dim=D, bits=bits,
+                     layer=layers[i] if layers is not None else i, kv=kvs[i] if kvs is not None else 0,
+                     flags=flags, io_round=io_round, report=reports)
+    return reports, pay, y
+
+
+# ------------------------------------------------------------------------------ small cases ---
+def test_tiny_config_fp32_io():
+    """The 8x8x8, 1 x 64, fp32, 2-bit oracle workload."""
+    w = WORKLOADS["tiny"]
+    x = make_workload_unit(w, 0, 0, 0, device=DEV)[None]
+    reports, _, _ = _check_batch(x, w.S, w.H, w.W, 2)
+    assert reports[0]["codes"] > 0
+
+
+@pytest.mark.parametrize("shape,bits", [
+    ((5, 7, 3, 2, 32), 3),      # ragged axes, two chunks
+    ((12, 6, 10, 1, 96), 1),    # three chunks, odd-ish lengths
+    ((16, 16, 16, 2, 64), 4),
+    ((3, 14, 14, 4, 16), 2),    # the video grid's H, W with a short S; head_dim 16 < 32
+    ((24, 5, 9, 1, 32), 8),     # 8 bits: every active bin saturates
+    ((32, 2, 24, 1, 64), 2),    # S in the 32 class, W in the 32 class
+    ((1, 1, 1, 1, 32), 5),      # a single token
+])
+def test_small_shapes_bf16(shape, bits):
+    S, H, W, heads, D = shape
+    x = torch.stack([make_unit(S, H, W, heads, D, rho=(0.9, 0.8, 0.85), nu=4.0, seed=10 * i + bits, device=DEV)
+                     for i in range(2)])
+    reports, _, _ = _check_batch(x, S, H, W, bits, layers=[3, 4], kvs=[0, 1])
+    assert all(r["recon_rel_rms"] <= 1e-3 for r in reports)
+
+
+def test_no_quant_round_trip_is_lossless():
+    S, H, W, heads, D = 16, 8, 12, 2, 32
+    x = torch.stack([make_unit(S, H, W, heads, D, rho=(0.9, 0.9, 0.9), nu=4.0, seed=i, device=DEV) for i in range(3)])
+    reports, pay, y = _check_batch(x, S, H, W, 2, flags=T.TACTKV_NO_QUANT)
+    assert rel_rms(y.double().cpu(), x.double().cpu()) <= 1e-5
+    # bf16 in, fp32 transform, bf16 out: all but the tiniest elements come back bit for bit
+    # (an fp32 round-trip error of ~1e-7 can move a value of ~1e-5 across a bf16 rounding boundary)
+    assert (y == x).double().mean().item() > 0.999
+
+
+def test_no_quant_fp32_io():
+    S, H, W, heads, D = 8, 8, 8, 1, 64
+    x = make_unit(S, H, W, heads, D, rho=(0.9, 0.9, 0.9), seed=3, dtype=torch.float32, device=DEV)[None]
+    _, _, y = _check_batch(x, S, H, W, 4, flags=T.TACTKV_NO_QUANT)
+    assert rel_rms(y.double().cpu(), x.double().cpu()) <= 1e-6
+
+
+def test_strided_input_and_output():
+    """kv_in as a view into a larger [tokens, heads_total, head_dim] cache (only 2 of 4 heads)."""
+    S, H, W, D = 8, 6, 6, 32
+    big = make_unit(S, H, W, 4, D, rho=(0.9, 0.9, 0.9), nu=4.0, seed=5, device=DEV)
+    x = big[:, 1:3, :][None]                          # stride(2) = D, stride(1) = 4 * D
+    assert not x.is_contiguous()
+    reports, pay, y = _check_batch(x, S, H, W, 2)
+    # decode into a strided output as well
+    out_big = torch.zeros_like(big)[None]
+    T.decompress(pay, S, H, W, 2, heads=2, head_dim=D, out=out_big[:, :, 1:3, :], check=True)
+    torch.cuda.synchronize()
+    assert torch.equal(out_big[0, :, 1:3, :], y[0])
+    assert not out_big[0, :, 0, :].any() and not out_big[0, :, 3, :].any()
+
+
+# --------------------------------------------------------------------------- degenerate inputs ---
+def test_all_zero_input():
+    S, H, W, heads, D = 8, 4, 4, 1, 32
+    x = torch.zeros((1, S * H * W, heads, D), dtype=torch.bfloat16, device=DEV)
+    pay, y = _round_trip(x, S, H, W, 2)
+    p = O.parse_payload(pay[0].cpu().numpy().tobytes())
+    assert p["code_bits"] == 0 and not p["b"].any() and not p["sigma"].any()
+    assert not y.any()
+
+
+def test_constant_field_keeps_dc():
+    """A constant field has all its energy in the DC bin; the other bins hold only rounding noise
+    (fp32 on the GPU, fp64 in the oracle) whose allocation is meaningless, so the DC allocation
+    and the reconstruction are compared.  The DC coefficient scaled by its own gain is exactly 1
+    in every channel, so even 8 bits leave the Lloyd-Max error of u = 1 (about 1%) on both sides."""
+    S, H, W, heads, D = 8, 8, 8, 1, 32
+    x = torch.full((1, S * H * W, heads, D), 0.75, dtype=torch.bfloat16, device=DEV)
+    pay, y = _round_trip(x, S, H, W, 1)
+    p = O.parse_payload(pay[0].cpu().numpy().tobytes())
+    assert p["b"][0] == 8
+    p_o = O.compress_unit(x[0].double().cpu().numpy(), S, H, W, heads, D, 1)
+    assert O.parse_payload(p_o)["b"][0] == 8
+    y_o = O.to_bf16(O.decompress_unit(p_o))
+    assert rel_rms(y[0].double().cpu().numpy(), y_o) <= 1e-3
+    assert rel_rms(y.double().cpu(), x.double().cpu()) < 0.02
+
+
+# ---------------------------------------------------------------------- batching and waves ---
+def test_many_units_and_small_workspace():
+    """More units than one launch carries (64), processed again with a workspace of one unit."""
+    S, H, W, heads, D = 4, 4, 4, 1, 32
+    U = 70
+    x = torch.stack([make_unit(S, H, W, heads, D, rho=(0.8, 0.8, 0.8), seed=i, device=DEV) for i in range(U)])
+    pay_a, y_a = _round_trip(x, S, H, W, 3)
+    units = T.make_units(x, S, H, W, 3, heads=heads, head_dim=D, payload=pay_a)
+    one = T.tactkv_workspace_bytes(units[:1])
+    ws = torch.zeros(one + 256, dtype=torch.uint8, device=DEV)
+    off = (-ws.data_ptr()) % 256
+    pay_b, y_b = _round_trip(x, S, H, W, 3, workspace=ws[off:off + one])
+    assert torch.equal(pay_a, pay_b) and torch.equal(y_a, y_b)
+    _check_batch(x, S, H, W, 3, units=[0, 33, 64, 69])
+
+
+def test_deterministic():
+    S, H, W, heads, D = 16, 8, 8, 2, 64
+    x = make_unit(S, H, W, heads, D, rho=(0.9, 0.9, 0.9), nu=4.0, seed=1, device=DEV)[None]
+    a, _ = _round_trip(x, S, H, W, 2)
+    b, _ = _round_trip(x, S, H, W, 2)
+    assert torch.equal(a, b)
+
+
+def test_cross_decode_oracle_payload_on_gpu():
+    """The GPU decoder reads a payload written by the oracle (same format, independent writers)."""
+    S, H, W, heads, D = 8, 6, 10, 1, 64
+    x = make_unit(S, H, W, heads, D, rho=(0.9, 0.85, 0.8), nu=4.0, seed=9, device=DEV)
+    p_o = O.compress_unit(x.double().cpu().numpy(), S, H, W, heads, D, 3, layer=0, kv=0)
+    cap = T.payload_capacity(S, H, W, heads, D, 3)
+    pay = torch.zeros((1, (cap + 15) // 16 * 16), dtype=torch.uint8)
+    pay[0, :len(p_o)] = torch.frombuffer(bytearray(p_o), dtype=torch.uint8)
+    y = T.decompress(pay.to(DEV), S, H, W, 3, heads=heads, head_dim=D, layers=[0], kvs=[0], check=True)
+    ref = O.to_bf16(O.decompress_unit(p_o))
+    assert rel_rms(y[0].double().cpu().numpy(), ref) <= 1e-3
+
+
+def test_payload_bytes_match_oracle_format():
+    """Where allocations and codes agree, the GPU payload is byte-identical to the oracle's."""
+    S, H, W, heads, D = 8, 8, 8, 1, 64
+    x = make_unit(S, H, W, heads, D, rho=(0.9, 0.9, 0.9), nu=4.0, seed=21, device=DEV)[None]
+    pay, _ = _round_trip(x, S, H, W, 2, layers=[0], kvs=[0])
+    p_o, info = O.compress_unit(x[0].double().cpu().numpy(), S, H, W, heads, D, 2, return_info=True)
+    g = pay[0].cpu().numpy().tobytes()[:len(p_o)]
+    po = np.frombuffer(p_o, np.uint8)
+    gg = np.frombuffer(g, np.uint8)
+    lay = O.payload_layout(S * H * W, heads * D, int(info["b"].sum()))
+    # header + bit allocation identical
+    assert np.array_equal(gg[:lay["off_sigma"]], po[:lay["off_sigma"]])
+    # code area: identical unless a code sits inside the tolerance band
+    _, codes_g = O.codes_of(g)
+    if np.array_equal(codes_g, info["codes"]):
+        assert np.array_equal(gg[lay["off_codes"]:], po[lay["off_codes"]:])
+
+
+# ------------------------------------------------------------------------------- full sizes ---
+@pytest.mark.parametrize("name,bits,pick", [
+    ("med4b", 1, [0, 67]),
+    ("med4b_b8", 2, [5, 300]),
+    ("med4b_b8", 4, [77, 543]),
+    ("med32b", 1, [0, 511]),
+    ("video", 1, [0, 895]),
+])
+def test_full_size_sampled_units(name, bits, pick):
+    """The benchmark workloads' exact shapes; the oracle checks sampled units of the batch."""
+    w = WORKLOADS[name]
+    all_units = list(w.units())
+    x = torch.stack([make_workload_unit(w, *all_units[u], device=DEV) for u in pick])
+    layers = [all_units[u][1] for u in pick]
+    kvs = [all_units[u][2] for u in pick]
+    reports, _, _ = _check_batch(x, w.S, w.H, w.W, bits, layers=layers, kvs=kvs)
+    for r in reports:
+        print(name, bits, r)
+
+
+# ------------------------------------------------------------------------------ error paths ---
+def test_corrupt_header_is_reported_and_zero_filled():
+    S, H, W, heads, D = 8, 4, 4, 1, 32
+    x = make_unit(S, H, W, heads, D, seed=2, device=DEV)[None]
+    pay = T.compress(x, S, H, W, 2)
+    bad = pay.clone()
+    bad[0, 16] ^= 1                                   # S field of the header
+    units = T.make_units(None, S, H, W, 2, heads=heads, head_dim=D, payload=bad,
+                         out=torch.ones_like(x), n_units=1)
+    ws = T.alloc_workspace(units, DEV)
+    out = torch.ones_like(x)
+    T.decompress(bad, S, H, W, 2, heads=heads, head_dim=D, out=out, workspace=ws)
+    st = T.tactkv_device_status(ws.data_ptr(), ws.numel(), torch.cuda.current_stream().cuda_stream)
+    assert st == T.TACTKV_CORRUPT_PAYLOAD
+    assert not out.any()
+    # status is cleared once read; a good payload decodes cleanly afterwards
+    T.decompress(pay, S, H, W, 2, heads=heads, head_dim=D, workspace=ws, check=True)
+
+
+def test_wrong_layer_is_rejected():
+    S, H, W, heads, D = 8, 4, 4, 1, 32
+    x = make_unit(S, H, W, heads, D, seed=2, device=DEV)[None]
+    pay = T.compress(x, S, H, W, 2, layers=[7])
+    with pytest.raises(T.TactkvError):
+        T.decompress(pay, S, H, W, 2, heads=heads, head_dim=D, layers=[8], check=True)

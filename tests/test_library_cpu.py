@@ -1,0 +1,105 @@
+"""The C ABI library on a machine without a GPU: it loads, exports every symbol include/tactkv.h
+declares, and its host-only functions and argument checks behave (no kernel is launched)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import tactkv_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def T():
+    from dct_transform_coding_b200 import tactkv
+    return tactkv
+
+
+def test_exports_every_declared_symbol(T):
+    header = open(os.path.join(ROOT, "include", "tactkv.h")).read()
+    declared = set(re.findall(r"^\w[\w\s\*]*?\b(tactkv_\w+)\s*\(", header, flags=re.M))
+    assert declared >= set(T.EXPORTED)
+    lib = ctypes.CDLL(T.LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_format_version_and_status_strings(T):
+    assert T.tactkv_format_version() == O.VERSION
+    assert T.tactkv_status_string(T.TACTKV_OK) == "ok"
+    assert T.tactkv_status_string(T.TACTKV_CORRUPT_PAYLOAD) == "corrupt payload"
+    assert T.tactkv_status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("bits", range(1, 9))
+def test_library_codebooks_match_oracle(T, bits):
+    """Two independent Lloyd-Max solvers (library build step vs oracle) agree to 1e-12."""
+    lv, th = T.tactkv_lloyd_max_table(bits)
+    y, t = O.table(bits)
+    assert np.max(np.abs(np.array(lv) - y)) < 1e-12
+    assert np.max(np.abs(np.array(th) - t)) < 1e-12
+
+
+def test_codebook_rejects_bad_bits(T):
+    with pytest.raises(ValueError):
+        T.tactkv_lloyd_max_table(0)
+    with pytest.raises(ValueError):
+        T.tactkv_lloyd_max_table(9)
+
+
+@pytest.mark.parametrize("shape,bits,flags", [((64, 16, 16, 4, 256), 1, 0), ((32, 24, 24, 8, 128), 1, 0),
+                                              ((64, 14, 14, 4, 128), 4, 0), ((8, 8, 8, 1, 64), 2, 0),
+                                              ((8, 8, 8, 1, 64), 2, 1), ((5, 7, 3, 2, 32), 8, 0)])
+def test_payload_capacity_matches_oracle_layout(T, shape, bits, flags):
+    S, H, W, heads, D = shape
+    cap = T.payload_capacity(S, H, W, heads, D, bits, flags)
+    assert cap == O.payload_capacity(S, H, W, heads, D, bits, no_quant=bool(flags & 1))
+
+
+def test_unsupported_shapes_report_zero_capacity(T):
+    for S, H, W, heads, D in [(17, 8, 8, 1, 32), (8, 33, 8, 1, 32), (8, 8, 8, 1, 30), (8, 8, 8, 1, 48),
+                              (65, 8, 8, 1, 32), (8, 32, 40, 1, 32)]:
+        u = T.tactkv_unit(S=S, H=H, W=W, heads=heads, head_dim=D, bits=2)
+        assert T.tactkv_payload_bytes(u) == 0, (S, H, W, heads, D)
+
+
+def _unit(T, **kw):
+    d = dict(S=8, H=8, W=8, heads=1, head_dim=32, bits=2, flags=0, kv_in=4096, kv_out=4096,
+             token_stride=32, head_stride=32, payload=8192, payload_capacity=1 << 20)
+    d.update(kw)
+    return T.tactkv_unit(**d)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(bits=0), "TACTKV_INVALID_ARG"), (dict(bits=9), "TACTKV_INVALID_ARG"),
+    (dict(flags=8), "TACTKV_INVALID_ARG"), (dict(S=0), "TACTKV_INVALID_ARG"),
+    (dict(kv_in=None), "TACTKV_INVALID_ARG"), (dict(payload=None), "TACTKV_INVALID_ARG"),
+    (dict(token_stride=0), "TACTKV_INVALID_ARG"),
+    (dict(S=17), "TACTKV_UNSUPPORTED_SHAPE"), (dict(head_dim=30), "TACTKV_UNSUPPORTED_SHAPE"),
+    (dict(kv_in=4098), "TACTKV_ALIGNMENT"), (dict(token_stride=33), "TACTKV_ALIGNMENT"),
+    (dict(payload=8200), "TACTKV_ALIGNMENT"), (dict(payload_capacity=100), "TACTKV_CAPACITY"),
+])
+def test_compress_argument_checks_without_gpu(T, kw, status):
+    units = [_unit(T, **kw)]
+    st = T.tactkv_compress(units, 1 << 20, 1 << 30, 0)
+    assert st == getattr(T, status)
+
+
+def test_workspace_checks_without_gpu(T):
+    units = [_unit(T)]
+    assert T.tactkv_compress(units, 0, 1 << 30, 0) == T.TACTKV_WORKSPACE
+    assert T.tactkv_compress(units, 1 << 20, 16, 0) == T.TACTKV_WORKSPACE
+    assert T.tactkv_compress(units, (1 << 20) + 8, 1 << 30, 0) == T.TACTKV_WORKSPACE
+    assert T.tactkv_compress([], 1 << 20, 1 << 30, 0) == T.TACTKV_OK
+    need = T.tactkv_workspace_bytes(units)
+    assert need >= 8 * 8 * 8 * 32 * 4
+    # a workspace one byte short of a single unit is refused before anything is launched
+    assert T.tactkv_compress(units, 1 << 20, need - 1, 0) == T.TACTKV_WORKSPACE
+
+
+def test_decompress_checks_output_pointer(T):
+    units = [_unit(T, kv_out=None)]
+    assert T.tactkv_decompress(units, 1 << 20, 1 << 30, 0) == T.TACTKV_INVALID_ARG
