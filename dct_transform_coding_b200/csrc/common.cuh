@@ -16,7 +16,7 @@ namespace tactkv {
 
 constexpr uint32_t kMagic = 0x31564B54u;   // "TKV1"
 constexpr int kVersion = 1;
-constexpr int kMaxUnits = 64;              // units per launch (descriptors travel as kernel parameters)
+constexpr int kMaxUnits = 256;             // units per launch (descriptors travel as kernel parameters, 12 KB)
 constexpr int kHeaderBytes = 64;
 constexpr int kChunk = 32;                 // channels per H/W-axis CTA
 constexpr int kPairs = kChunk / 2;         // channel pairs: every pencil carries two channels (float2)

@@ -191,39 +191,71 @@ size_t tactkv_workspace_bytes(const tactkv_unit* units, int n_units) {
   return kStatusBytes + best;
 }
 
-tactkv_status tactkv_compress(const tactkv_unit* units, int n_units, void* workspace, size_t workspace_bytes,
-                              struct CUstream_st* stream) {
-  cudaStream_t st = stream;
+static tactkv_status compress_impl(const tactkv_unit* units, int n_units, void* workspace, size_t workspace_bytes,
+                                   cudaStream_t st, void* const* events) {
+  auto mark = [&](int k) {
+    if (events && events[k]) cudaEventRecord(static_cast<cudaEvent_t>(events[k]), st);
+  };
   return for_each_wave(units, n_units, workspace, workspace_bytes, true,
                        [&](const Geom& g, const UnitList& ul, int nu, unsigned char* ws) -> tactkv_status {
                          const WsView w = view(ws, g, nu);
                          const int cs = length_class(g.S), ch = length_class(g.H), cw = length_class(g.W);
                          const int mode2 = (g.flags & TACTKV_NO_QUANT) ? kRaw : kQuant;
+                         mark(0);
                          if (launch_axis_s(cs, false, g, ul, nu, w.big, st) != cudaSuccess) return TACTKV_CUDA;
+                         mark(1);
                          if (launch_axis_hw(ch, cw, false, kStats, g, ul, nu, w.big, w.partial, w.status, st) !=
                              cudaSuccess)
                            return TACTKV_CUDA;
+                         mark(2);
                          if (launch_allocate(g, ul, nu, w.partial, w.var, st) != cudaSuccess) return TACTKV_CUDA;
+                         mark(3);
                          if (launch_axis_hw(ch, cw, false, mode2, g, ul, nu, w.big, w.partial, w.status, st) !=
                              cudaSuccess)
                            return TACTKV_CUDA;
+                         mark(4);
                          return TACTKV_OK;
                        });
 }
 
-tactkv_status tactkv_decompress(const tactkv_unit* units, int n_units, void* workspace, size_t workspace_bytes,
-                                struct CUstream_st* stream) {
-  cudaStream_t st = stream;
+static tactkv_status decompress_impl(const tactkv_unit* units, int n_units, void* workspace, size_t workspace_bytes,
+                                     cudaStream_t st, void* const* events) {
+  auto mark = [&](int k) {
+    if (events && events[k]) cudaEventRecord(static_cast<cudaEvent_t>(events[k]), st);
+  };
   return for_each_wave(units, n_units, workspace, workspace_bytes, false,
                        [&](const Geom& g, const UnitList& ul, int nu, unsigned char* ws) -> tactkv_status {
                          const WsView w = view(ws, g, nu);
                          const int cs = length_class(g.S), ch = length_class(g.H), cw = length_class(g.W);
                          const int mode = (g.flags & TACTKV_NO_QUANT) ? kRaw : kQuant;
+                         mark(0);
                          if (launch_axis_hw(ch, cw, true, mode, g, ul, nu, w.big, nullptr, w.status, st) != cudaSuccess)
                            return TACTKV_CUDA;
+                         mark(1);
                          if (launch_axis_s(cs, true, g, ul, nu, w.big, st) != cudaSuccess) return TACTKV_CUDA;
+                         mark(2);
                          return TACTKV_OK;
                        });
+}
+
+tactkv_status tactkv_compress(const tactkv_unit* units, int n_units, void* workspace, size_t workspace_bytes,
+                              struct CUstream_st* stream) {
+  return compress_impl(units, n_units, workspace, workspace_bytes, stream, nullptr);
+}
+
+tactkv_status tactkv_decompress(const tactkv_unit* units, int n_units, void* workspace, size_t workspace_bytes,
+                                struct CUstream_st* stream) {
+  return decompress_impl(units, n_units, workspace, workspace_bytes, stream, nullptr);
+}
+
+tactkv_status tactkv_compress_profiled(const tactkv_unit* units, int n_units, void* workspace,
+                                       size_t workspace_bytes, struct CUstream_st* stream, void* const* events) {
+  return compress_impl(units, n_units, workspace, workspace_bytes, stream, events);
+}
+
+tactkv_status tactkv_decompress_profiled(const tactkv_unit* units, int n_units, void* workspace,
+                                         size_t workspace_bytes, struct CUstream_st* stream, void* const* events) {
+  return decompress_impl(units, n_units, workspace, workspace_bytes, stream, events);
 }
 
 tactkv_status tactkv_device_status(void* workspace, size_t workspace_bytes, struct CUstream_st* stream) {

@@ -35,7 +35,8 @@ TACTKV_FP32_IO = 2
 
 HEADER_BYTES = 64
 EXPORTED = ("tactkv_payload_bytes", "tactkv_workspace_bytes", "tactkv_compress", "tactkv_decompress",
-            "tactkv_device_status", "tactkv_status_string", "tactkv_lloyd_max_table", "tactkv_format_version")
+            "tactkv_compress_profiled", "tactkv_decompress_profiled", "tactkv_device_status",
+            "tactkv_status_string", "tactkv_lloyd_max_table", "tactkv_format_version")
 
 
 class tactkv_unit(ctypes.Structure):
@@ -58,6 +59,10 @@ _lib.tactkv_workspace_bytes.argtypes = [_P, ctypes.c_int]
 for _name in ("tactkv_compress", "tactkv_decompress"):
     getattr(_lib, _name).restype = ctypes.c_int
     getattr(_lib, _name).argtypes = [_P, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+for _name in ("tactkv_compress_profiled", "tactkv_decompress_profiled"):
+    getattr(_lib, _name).restype = ctypes.c_int
+    getattr(_lib, _name).argtypes = [_P, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+                                     ctypes.POINTER(ctypes.c_void_p)]
 _lib.tactkv_device_status.restype = ctypes.c_int
 _lib.tactkv_device_status.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
 _lib.tactkv_status_string.restype = ctypes.c_char_p
@@ -94,6 +99,26 @@ def tactkv_decompress(units, workspace_ptr: int, workspace_bytes: int, stream_pt
     arr = _as_array(units)
     return int(_lib.tactkv_decompress(arr, len(arr), ctypes.c_void_p(workspace_ptr), workspace_bytes,
                                       ctypes.c_void_p(stream_ptr)))
+
+
+def _events_array(events):
+    if events is None:
+        return None
+    return (ctypes.c_void_p * len(events))(*[int(e) if e else None for e in events])
+
+
+def tactkv_compress_profiled(units, workspace_ptr: int, workspace_bytes: int, stream_ptr: int, events) -> int:
+    """events: sequence of 5 cudaEvent_t handles (ints, e.g. torch.cuda.Event().cuda_event) or None."""
+    arr = _as_array(units)
+    return int(_lib.tactkv_compress_profiled(arr, len(arr), ctypes.c_void_p(workspace_ptr), workspace_bytes,
+                                             ctypes.c_void_p(stream_ptr), _events_array(events)))
+
+
+def tactkv_decompress_profiled(units, workspace_ptr: int, workspace_bytes: int, stream_ptr: int, events) -> int:
+    """events: sequence of 3 cudaEvent_t handles or None."""
+    arr = _as_array(units)
+    return int(_lib.tactkv_decompress_profiled(arr, len(arr), ctypes.c_void_p(workspace_ptr), workspace_bytes,
+                                               ctypes.c_void_p(stream_ptr), _events_array(events)))
 
 
 def tactkv_device_status(workspace_ptr: int, workspace_bytes: int, stream_ptr: int) -> int:

@@ -68,7 +68,7 @@ typedef enum {
 typedef struct {
   int32_t layer;          /* recorded in the header, checked by decompress */
   int32_t kv;             /* 0 = K, 1 = V; recorded and checked like layer */
-  int32_t S, H, W;        /* token grid; each axis 1..64 from the supported set (see below) */
+  int32_t S, H, W;        /* token grid; lengths from the supported set below */
   int32_t heads, head_dim;/* n = heads*head_dim channels, n a multiple of 32, head_dim even */
   int32_t bits;           /* nominal bits per element, 1..8 */
   uint32_t flags;         /* TACTKV_NO_QUANT | TACTKV_FP32_IO */
@@ -81,14 +81,17 @@ typedef struct {
   size_t payload_capacity;/* bytes available at payload */
 } tactkv_unit;
 
-/* Supported axis lengths S, H, W: 1..16, 20, 24, 28, 32, 40, 48, 56, 64, with H*W <= 1024.
-   kv_in / kv_out must be 4-byte aligned (8-byte with TACTKV_FP32_IO).  */
+/* Supported shapes: S in {1..16, 20, 24, 28, 32, 40, 48, 56, 64}; H and W in {1..16, 20, 24, 28,
+   32} with H*W <= 1024; heads*head_dim a multiple of 32 and at most 65536.  kv_in / kv_out must
+   be 4-byte aligned (8-byte with TACTKV_FP32_IO); strides even.  Other shapes return
+   TACTKV_UNSUPPORTED_SHAPE. */
 
 /* Worst-case payload size of one unit (every bin budget used): the capacity to provide. */
 size_t tactkv_payload_bytes(const tactkv_unit* unit);
 
-/* Workspace bytes that let compress/decompress process all `n_units` in one wave.  Any size of
-   at least tactkv_workspace_bytes(units, 1) works; the units are then processed in waves. */
+/* Workspace bytes that let compress/decompress process the units in as few waves as possible
+   (a wave is up to 256 units of one shape).  Any size of at least tactkv_workspace_bytes(units,
+   1) works; the units are then processed in more, smaller waves. */
 size_t tactkv_workspace_bytes(const tactkv_unit* units, int n_units);
 
 /* Compress every unit: read kv_in, write the payload.  Units with identical shape, bits and
@@ -104,6 +107,20 @@ tactkv_status tactkv_compress(const tactkv_unit* units, int n_units, void* works
    as TACTKV_CORRUPT_PAYLOAD in the workspace and that unit's output is zero-filled. */
 tactkv_status tactkv_decompress(const tactkv_unit* units, int n_units, void* workspace,
                                 size_t workspace_bytes, struct CUstream_st* stream);
+
+/* Profiling variants: the same work as tactkv_compress / tactkv_decompress, and, when `events`
+   is not NULL, cudaEventRecord(events[k], stream) at the stage boundaries of every wave (so for
+   a call that fits in one wave the events bracket each kernel).  events[k] are cudaEvent_t
+   handles created by the caller; a NULL entry is skipped.
+   compress:   0 before the S-axis DCT, 1 after it, 2 after the H/W DCT with energy sums,
+               3 after the allocation, 4 after the H/W DCT with quantization and packing.
+   decompress: 0 before the inverse H/W pass, 1 after it, 2 after the inverse S-axis pass. */
+tactkv_status tactkv_compress_profiled(const tactkv_unit* units, int n_units, void* workspace,
+                                       size_t workspace_bytes, struct CUstream_st* stream,
+                                       void* const* events);
+tactkv_status tactkv_decompress_profiled(const tactkv_unit* units, int n_units, void* workspace,
+                                         size_t workspace_bytes, struct CUstream_st* stream,
+                                         void* const* events);
 
 /* Synchronizes `stream`, returns the first error the kernels recorded in `workspace` since the
    previous call (TACTKV_OK if none), and clears it. */

@@ -135,9 +135,9 @@ def test_constant_field_keeps_dc():
 
 # ---------------------------------------------------------------------- batching and waves ---
 def test_many_units_and_small_workspace():
-    """More units than one launch carries (64), processed again with a workspace of one unit."""
+    """More units than one launch carries (256), processed again with a workspace of one unit."""
     S, H, W, heads, D = 4, 4, 4, 1, 32
-    U = 70
+    U = 260
     x = torch.stack([make_unit(S, H, W, heads, D, rho=(0.8, 0.8, 0.8), seed=i, device=DEV) for i in range(U)])
     pay_a, y_a = _round_trip(x, S, H, W, 3)
     units = T.make_units(x, S, H, W, 3, heads=heads, head_dim=D, payload=pay_a)
@@ -146,7 +146,7 @@ def test_many_units_and_small_workspace():
     off = (-ws.data_ptr()) % 256
     pay_b, y_b = _round_trip(x, S, H, W, 3, workspace=ws[off:off + one])
     assert torch.equal(pay_a, pay_b) and torch.equal(y_a, y_b)
-    _check_batch(x, S, H, W, 3, units=[0, 33, 64, 69])
+    _check_batch(x, S, H, W, 3, units=[0, 130, 256, 259])
 
 
 def test_deterministic():
