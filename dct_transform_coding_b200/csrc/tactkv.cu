@@ -8,6 +8,7 @@
 // inverse H/W pass (dequantize + inverse DCT along W and H) and the inverse DCT along S.
 #include <algorithm>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "lloyd_max_tables.inc"
@@ -164,6 +165,37 @@ tactkv_status for_each_wave(const tactkv_unit* units, int n_units, void* ws, siz
 }
 
 }  // namespace
+
+// ------------------------------------------------------------- allocation-free compress scratch ---
+// Scratch of tactkv_compress_noalloc: a fixed array in the library's device image, so the call
+// needs no allocation from its caller.  Every device that loads the library holds it until exit.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+constexpr int kMaxDevices = 64;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device.  In host code the symbol names a
+// host-side stand-in, not device memory, so the address is looked up once per device (with that
+// device current) and cached.
+cudaError_t noalloc_scratch(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return cudaSuccess;
+}
+}  // namespace
 }  // namespace tactkv
 
 using namespace tactkv;
@@ -258,6 +290,22 @@ tactkv_status tactkv_decompress_profiled(const tactkv_unit* units, int n_units, 
   return decompress_impl(units, n_units, workspace, workspace_bytes, stream, events);
 }
 
+tactkv_status tactkv_compress_noalloc(const tactkv_unit* units, int n_units, struct CUstream_st* stream) {
+  if (n_units < 0 || (n_units > 0 && !units)) return TACTKV_INVALID_ARG;
+  if (n_units == 0) return TACTKV_OK;
+  for (int i = 0; i < n_units; ++i) {   // every unit must fit the fixed scratch on its own
+    Geom g;
+    const tactkv_status st = make_geom(units[i], g);
+    if (st != TACTKV_OK) return st;
+    if (kStatusBytes + unit_ws_bytes(g) > kNoAllocScratchBytes) return TACTKV_SCRATCH_LIMIT;
+  }
+  void* ws = nullptr;
+  if (noalloc_scratch(&ws) != cudaSuccess) return TACTKV_CUDA;
+  // the scratch keeps the previous call's contents: the status word is the part that must start at 0
+  if (cudaMemsetAsync(ws, 0, kStatusBytes, stream) != cudaSuccess) return TACTKV_CUDA;
+  return compress_impl(units, n_units, ws, kNoAllocScratchBytes, stream, nullptr);
+}
+
 tactkv_status tactkv_device_status(void* workspace, size_t workspace_bytes, struct CUstream_st* stream) {
   if (!workspace || workspace_bytes < kStatusBytes) return TACTKV_WORKSPACE;
   unsigned int v = 0;
@@ -277,6 +325,7 @@ const char* tactkv_status_string(tactkv_status s) {
     case TACTKV_CORRUPT_PAYLOAD: return "corrupt payload";
     case TACTKV_CUDA: return "CUDA error";
     case TACTKV_WORKSPACE: return "workspace missing or too small";
+    case TACTKV_SCRATCH_LIMIT: return "unit larger than the fixed scratch of tactkv_compress_noalloc";
     default: return "unknown status";
   }
 }

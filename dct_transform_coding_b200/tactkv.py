@@ -29,13 +29,15 @@ TACTKV_ALIGNMENT = 4
 TACTKV_CORRUPT_PAYLOAD = 5
 TACTKV_CUDA = 6
 TACTKV_WORKSPACE = 7
+TACTKV_SCRATCH_LIMIT = 8
 
 TACTKV_NO_QUANT = 1
 TACTKV_FP32_IO = 2
 
 HEADER_BYTES = 64
 EXPORTED = ("tactkv_payload_bytes", "tactkv_workspace_bytes", "tactkv_compress", "tactkv_decompress",
-            "tactkv_compress_profiled", "tactkv_decompress_profiled", "tactkv_device_status",
+            "tactkv_compress_profiled", "tactkv_decompress_profiled", "tactkv_compress_noalloc",
+            "tactkv_device_status",
             "tactkv_status_string", "tactkv_lloyd_max_table", "tactkv_format_version")
 
 
@@ -63,6 +65,8 @@ for _name in ("tactkv_compress_profiled", "tactkv_decompress_profiled"):
     getattr(_lib, _name).restype = ctypes.c_int
     getattr(_lib, _name).argtypes = [_P, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
                                      ctypes.POINTER(ctypes.c_void_p)]
+_lib.tactkv_compress_noalloc.restype = ctypes.c_int
+_lib.tactkv_compress_noalloc.argtypes = [_P, ctypes.c_int, ctypes.c_void_p]
 _lib.tactkv_device_status.restype = ctypes.c_int
 _lib.tactkv_device_status.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
 _lib.tactkv_status_string.restype = ctypes.c_char_p
@@ -119,6 +123,14 @@ def tactkv_decompress_profiled(units, workspace_ptr: int, workspace_bytes: int, 
     arr = _as_array(units)
     return int(_lib.tactkv_decompress_profiled(arr, len(arr), ctypes.c_void_p(workspace_ptr), workspace_bytes,
                                                ctypes.c_void_p(stream_ptr), _events_array(events)))
+
+
+def tactkv_compress_noalloc(units, stream_ptr: int) -> int:
+    """Compress with the library's fixed device scratch instead of a caller workspace (for callers
+    that cannot allocate, e.g. while recording a CUDA graph).  Calls share that scratch: serialize
+    calls that could overlap on the GPU."""
+    arr = _as_array(units)
+    return int(_lib.tactkv_compress_noalloc(arr, len(arr), ctypes.c_void_p(stream_ptr)))
 
 
 def tactkv_device_status(workspace_ptr: int, workspace_bytes: int, stream_ptr: int) -> int:

@@ -58,7 +58,8 @@ typedef enum {
   TACTKV_ALIGNMENT = 4,          /* a pointer or stride breaks the alignment rules below */
   TACTKV_CORRUPT_PAYLOAD = 5,    /* (device status) a payload header or allocation is invalid */
   TACTKV_CUDA = 6,               /* a CUDA launch or copy failed */
-  TACTKV_WORKSPACE = 7           /* workspace null or smaller than one unit needs */
+  TACTKV_WORKSPACE = 7,          /* workspace null or smaller than one unit needs */
+  TACTKV_SCRATCH_LIMIT = 8       /* a unit needs more scratch than tactkv_compress_noalloc has */
 } tactkv_status;
 
 /* flags */
@@ -121,6 +122,23 @@ tactkv_status tactkv_compress_profiled(const tactkv_unit* units, int n_units, vo
 tactkv_status tactkv_decompress_profiled(const tactkv_unit* units, int n_units, void* workspace,
                                          size_t workspace_bytes, struct CUstream_st* stream,
                                          void* const* events);
+
+/* tactkv_compress without a workspace argument, for callers that cannot allocate device memory
+   at the point where they compress: code recording a CUDA graph (a cudaMalloc there fails or
+   breaks the capture), engines whose device memory is all handed out by their own pool, and
+   latency-critical loops where an allocation could synchronize the device.  The TACT-KV pages
+   have no counterpart of this call; it only changes where the scratch lives.
+   The scratch is a fixed 16 MiB array inside the library's device image, which every GPU that
+   loads the library holds until the process exits.  Each unit on its own must fit in it (its
+   workspace, tactkv_workspace_bytes of that one unit, at most 16 MiB: e.g. 8x8x8 x 64 channels or
+   64x16x16 x 128 channels, not 64x16x16 x 1024); otherwise TACTKV_SCRATCH_LIMIT is returned and
+   nothing is launched.  The first call on a device looks the array's address up
+   (cudaGetSymbolAddress), so make that first call before any stream capture.  All calls share
+   the one array: calls that may overlap on the GPU (different streams, or several host threads)
+   race on it and must be serialized by the caller.  Allocates nothing; output is identical to
+   tactkv_compress. */
+tactkv_status tactkv_compress_noalloc(const tactkv_unit* units, int n_units,
+                                      struct CUstream_st* stream);
 
 /* Synchronizes `stream`, returns the first error the kernels recorded in `workspace` since the
    previous call (TACTKV_OK if none), and clears it. */
