@@ -1,7 +1,7 @@
 // Per-unit bit allocation (TACT-KV stage 3) and payload header, one CTA per unit.
 //
 // sigma_i^2 = (1/n) sum_c X[i, c]^2 is assembled in fp64 from the per-chunk fp32 energy sums in
-// a fixed order (deterministic).  The pages allocate by reverse water-filling,
+// a fixed order (deterministic) by reduce_var_kernel, spread over the whole GPU.  The pages allocate by reverse water-filling,
 // b_i = max(0, 1/2 log2(sigma_i^2 / theta)) with theta from bisection, rounding, a +-1 greedy
 // fix to hit the budget B = bits * N exactly and a cap of 8 bits.  Rounding at theta keeps the
 // keys sigma_i^2 4^-k (k = 0..7) that are >= 2 theta, and each greedy step adds the largest
@@ -17,6 +17,8 @@
 
 namespace tactkv {
 namespace {
+
+constexpr size_t kAllocSmemVar = 200 * 1024;   // variances kept in shared memory up to N = 25600 bins
 
 // Number of keys var * 4^-k (k = 0..7) that are >= v, exactly; var > 0, v >= 0.
 __device__ __forceinline__ int key_count(double var, double v) {
@@ -63,30 +65,44 @@ __device__ double block_max(double v, double* s_red) {
   return r;
 }
 
+// sigma_i^2 = (1/n) sum over the channel chunks of the fp32 per-chunk energy sums, in fp64 and
+// in a fixed order; one thread per bin across the whole GPU.
+__global__ void __launch_bounds__(256) reduce_var_kernel(const __grid_constant__ Geom g, const float* __restrict__ partial,
+                                                         double* __restrict__ var_ws) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  const int u = blockIdx.y;
+  if (i >= g.N) return;
+  const float* p = partial + (size_t)u * g.nch * g.N + i;
+  double acc = 0.0;
+#pragma unroll 8
+  for (int q = 0; q < g.nch; ++q) acc += (double)__ldcs(p + (size_t)q * g.N);
+  var_ws[(size_t)u * g.N + i] = acc / (double)g.n;
+}
+
 __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_constant__ Geom g,
                                                                  const __grid_constant__ UnitList ul,
-                                                                 const float* __restrict__ partial,
-                                                                 double* __restrict__ var_ws) {
+                                                                 double* __restrict__ var_ws, bool var_in_smem) {
   __shared__ long long s_ll[32];
   __shared__ double s_d[32];
   __shared__ uint32_t s_scan[33];
   __shared__ uint32_t s_cnt[kAllocThreads];
+  extern __shared__ __align__(16) unsigned char smem_var[];
   const int u = blockIdx.x;
   const UnitDev& ud = ul.u[u];
   unsigned char* pay = ud.payload;
-  double* var = var_ws + (size_t)u * g.N;
+  // the bisection reads every variance ~64 times: keep them in shared memory when they fit
+  double* var = var_in_smem ? reinterpret_cast<double*>(smem_var) : var_ws + (size_t)u * g.N;
   const bool raw = g.flags & TACTKV_NO_QUANT;
   // each thread owns a contiguous range of bins, so thread order is bin order
   const int per = (g.N + blockDim.x - 1) / blockDim.x;
   const int beg = min(g.N, (int)threadIdx.x * per), end = min(g.N, beg + per);
 
-  // 1. sigma^2 in fp64 from the per-chunk fp32 sums, in a fixed order
+  // 1. sigma^2 (reduced over the channel chunks by reduce_var_kernel)
   long long act = 0;
   double vmax = 0.0;
+  const double* var_g = var_ws + (size_t)u * g.N;
   for (int i = beg; i < end; ++i) {
-    double acc = 0.0;
-    for (int q = 0; q < g.nch; ++q) acc += (double)partial[((size_t)u * g.nch + q) * g.N + i];
-    const double v = acc / (double)g.n;
+    const double v = var_g[i];
     var[i] = v;
     act += v > 0.0;
     vmax = fmax(vmax, v);
@@ -184,7 +200,11 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
 
 cudaError_t launch_allocate(const Geom& g, const UnitList& ul, int nu, const float* partial, double* var,
                             cudaStream_t st) {
-  allocate_kernel<<<nu, kAllocThreads, 0, st>>>(g, ul, partial, var);
+  const size_t var_bytes = (size_t)g.N * sizeof(double);
+  const bool in_smem = var_bytes <= kAllocSmemVar;
+  if (in_smem) cudaFuncSetAttribute(allocate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)var_bytes);
+  reduce_var_kernel<<<dim3((g.N + 255) / 256, nu), 256, 0, st>>>(g, partial, var);
+  allocate_kernel<<<nu, kAllocThreads, in_smem ? var_bytes : 0, st>>>(g, ul, var, in_smem);
   return cudaGetLastError();
 }
 

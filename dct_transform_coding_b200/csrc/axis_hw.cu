@@ -8,8 +8,12 @@
 //   kRaw    float32 coefficients into the streams (TACTKV_NO_QUANT)
 // Because a CTA owns its channels' streams from the first bit to the last, each output word is
 // assembled in shared memory and stored exactly once; the word that straddles two slabs is
-// carried to the next slab.  Decoding (idct_hw) reads the same words, dequantizes and applies
-// the inverse DCTs along W and H.
+// carried to the next slab.  The next slab's coefficients are fetched with cp.async into a
+// second buffer while the current one is transformed (when two buffers fit in shared memory).
+//
+// Both directions first compute the stream offset of every (k_s, k_h) pencil from the bit
+// allocation, so no per-slab scan is needed; decoding (idct_hw) prefetches the stream words of
+// slab k_s+1 while slab k_s is dequantized and put through the inverse DCTs along W and H.
 //
 // Compiled once per pair of length classes (TACTKV_HCLASS, TACTKV_WCLASS: 16 or 32 each).
 #include "common.cuh"
@@ -22,35 +26,47 @@
 namespace tactkv {
 namespace {
 
-struct HwSmem {
-  float2* tile;       // [HW][16] channel pairs of one S slab
-  float* thr;         // all Lloyd-Max thresholds
-  float* lv;          // all Lloyd-Max levels
-  float* gain;        // [HW] 1/sigma (encode) or sigma (decode) of the slab's bins
-  uint32_t* b;        // [HW] bits of the slab's bins
-  uint32_t* off;      // [HW] bit offset of each bin, relative to the word holding the slab's first bit
-  uint32_t* sbuf;     // [32][words] stream words of the slab, per channel
-  uint32_t* carry;    // [32]
-  uint32_t* warp;     // [33] scan scratch
-  int words;          // stride of sbuf rows
+constexpr size_t kSmemBudget = 220 * 1024;
+constexpr int kEnergyStride = kPairs + 1;   // padded row of per-pair energies: conflict-free both ways
+constexpr int kMaxSlabs = 64;
+
+__host__ __device__ inline int stream_words_per_slab(int HW) { return (8 * HW + 31) / 32 + 2; }
+
+struct HwLayout {
+  size_t tile, thr, lv, meta_b, meta_g, off, uni, carry, warp, slab, total;
+  int nbuf;
+  int words;
 };
 
-__device__ HwSmem carve(unsigned char* sm, int HW) {
-  HwSmem s;
-  s.words = stream_words_per_slab(HW);
-  s.tile = reinterpret_cast<float2*>(sm); sm += (size_t)HW * kPairs * sizeof(float2);
-  s.thr = reinterpret_cast<float*>(sm); sm += kLmThrTotal * 4;
-  s.lv = reinterpret_cast<float*>(sm); sm += kLmLvTotal * 4;
-  s.gain = reinterpret_cast<float*>(sm); sm += (size_t)HW * 4;
-  s.b = reinterpret_cast<uint32_t*>(sm); sm += (size_t)HW * 4;
-  s.off = reinterpret_cast<uint32_t*>(sm); sm += (size_t)HW * 4;
-  s.sbuf = reinterpret_cast<uint32_t*>(sm); sm += (size_t)kChunk * s.words * 4;
-  s.carry = reinterpret_cast<uint32_t*>(sm); sm += kChunk * 4;
-  s.warp = reinterpret_cast<uint32_t*>(sm);
-  return s;
+// Shared memory carve-up; `uni` holds the energy rows (kStats) or the stream words (kQuant and
+// decoding) -- never both in one launch.
+__host__ __device__ inline HwLayout hw_layout(int HW, bool decode) {
+  HwLayout L;
+  L.words = stream_words_per_slab(HW);
+  const size_t tile1 = (size_t)HW * kPairs * 8;
+  const size_t energy = (size_t)HW * kEnergyStride * 4;
+  const size_t words = (size_t)kChunk * L.words * 4 * (decode ? 2 : 1);
+  const size_t uni = energy > words ? energy : words;
+  const size_t fixed = (size_t)(kLmThrTotal + kLmLvTotal) * 4 + (size_t)HW * 4 * 3 +
+                       (size_t)(HW > kMaxSlabs * 32 ? HW : kMaxSlabs * 32) * 8 + uni + kChunk * 4 + 33 * 4 +
+                       (kMaxSlabs + 1) * 4 + 256;
+  L.nbuf = (decode || 2 * tile1 + fixed > kSmemBudget) ? 1 : 2;
+  size_t o = 0;
+  L.tile = o; o += tile1 * L.nbuf;
+  L.thr = o; o += kLmThrTotal * 4;
+  L.lv = o; o += kLmLvTotal * 4;
+  L.meta_b = o; o += (size_t)(HW > kMaxSlabs * 32 ? HW : kMaxSlabs * 32) * 4 * 2;
+  L.meta_g = o; o += (size_t)HW * 4 * 2;
+  L.off = o; o += (size_t)HW * 4;
+  L.uni = o; o += (uni + 15) / 16 * 16;
+  L.carry = o; o += kChunk * 4;
+  L.warp = o; o += 33 * 4;
+  L.slab = o; o += (kMaxSlabs + 1) * 4;
+  L.total = o;
+  return L;
 }
 
-// Lloyd-Max code: the number of thresholds t_j <= u (branch-free bisection over 2^b - 1 values).
+// Lloyd-Max code: the number of thresholds t_j <= u (bisection over the 2^b - 1 thresholds).
 __device__ __forceinline__ uint32_t lm_code(float u, int bits, const float* thr) {
   const float* t = thr + lm_thr_offset(bits);
   uint32_t code = 0;
@@ -59,75 +75,98 @@ __device__ __forceinline__ uint32_t lm_code(float u, int bits, const float* thr)
   return code;
 }
 
-// Pencil DCTs along one axis of the tile: along H the pencils are (w, pair) with stride W*16,
-// along W they are (h, pair) with stride 16.
+// Pencil DCTs along H of the tile: pencils (w, pair), stride W*16 between elements.
 template <int CLASS, bool INV>
-__device__ __forceinline__ void tile_pass(const Geom& g, float2* tile, bool along_h) {
-  const int L = along_h ? g.H : g.W;
-  const int npen = (along_h ? g.W : g.H) * kPairs;
-  const int step = along_h ? g.W * kPairs : kPairs;
-  for (int p = threadIdx.x; p < npen; p += blockDim.x) {
-    const int q = p >> 4, pair = p & 15;
-    const int base = along_h ? q * kPairs + pair : q * g.W * kPairs + pair;
+__device__ __forceinline__ void h_pass(const Geom& g, float2* tile) {
+  const int step = g.W * kPairs;
+  for (int p = threadIdx.x; p < g.W * kPairs; p += blockDim.x) {
+    const int base = (p >> 4) * kPairs + (p & 15);
     float2 x[CLASS];
 #pragma unroll
     for (int t = 0; t < CLASS; ++t)
-      if (t < L) x[t] = tile[base + t * step];
-    dct_pencil<CLASS, INV>(x, L);
+      if (t < g.H) x[t] = tile[base + t * step];
+    dct_pencil<CLASS, INV>(x, g.H);
 #pragma unroll
     for (int t = 0; t < CLASS; ++t)
-      if (t < L) tile[base + t * step] = x[t];
+      if (t < g.H) tile[base + t * step] = x[t];
   }
+}
+
+// Copy one S slab of Y (HW rows of 32 channels, 128 bytes each) into a tile, asynchronously.
+__device__ __forceinline__ void issue_tile(const Geom& g, const float4* ysrc_unit, int ks, float2* tile) {
+  const int rowq = g.n / 4;
+  const float4* src = ysrc_unit + (size_t)ks * g.HW * rowq;
+  float4* dst = reinterpret_cast<float4*>(tile);
+  for (int i = threadIdx.x; i < g.HW * (kChunk / 4); i += blockDim.x)
+    cp_async16(dst + i, src + (size_t)(i >> 3) * rowq + (i & 7));
 }
 
 template <int HC, int WC>
 __global__ void __launch_bounds__(kHwThreads) fdct_hw_kernel(const __grid_constant__ Geom g,
                                                              const __grid_constant__ UnitList ul, int mode,
                                                              const float* __restrict__ Y, float* __restrict__ partial) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  HwSmem s = carve(smem_raw, g.HW);
+  extern __shared__ __align__(16) unsigned char smem[];
+  const HwLayout L = hw_layout(g.HW, false);
+  float2* tiles = reinterpret_cast<float2*>(smem + L.tile);
+  float* thr = reinterpret_cast<float*>(smem + L.thr);
+  uint32_t* pen = reinterpret_cast<uint32_t*>(smem + L.meta_b);   // bit offset of every (k_s, k_h) pencil
+  float* energy = reinterpret_cast<float*>(smem + L.uni);
+  uint32_t* sbuf = reinterpret_cast<uint32_t*>(smem + L.uni);
+  uint32_t* carry = reinterpret_cast<uint32_t*>(smem + L.carry);
+  uint32_t* swarp = reinterpret_cast<uint32_t*>(smem + L.warp);
+  const int words = L.words;
   const int chunk = blockIdx.x, u = blockIdx.y;
   const UnitDev& ud = ul.u[u];
   unsigned char* pay = ud.payload;
   uint32_t* words_out = reinterpret_cast<uint32_t*>(pay + g.off_codes);
+  const bool quant = mode == kQuant;
   uint32_t cstride = 0, stride_words = 0;
-  if (mode != kStats) {  // the header was written by the allocation kernel
+  if (mode != kStats) {  // written by the allocation kernel
     cstride = reinterpret_cast<const uint32_t*>(pay)[11];
     stride_words = cstride / 4;
   }
-  if (mode == kQuant) {
-    for (int i = threadIdx.x; i < kLmThrTotal; i += blockDim.x) s.thr[i] = c_lm_thresholds[i];
-    if (threadIdx.x < kChunk) s.carry[threadIdx.x] = 0;
-  }
   const float4* ysrc = reinterpret_cast<const float4*>(Y + (size_t)u * g.S * g.HW * g.n) + chunk * (kChunk / 4);
-  const int rowq = g.n / 4;
-  uint32_t P = 0;  // stream bits written so far, identical for every channel
-  for (int ks = 0; ks < g.S; ++ks) {
-    // stage the slab: HW rows of 32 channels
-    const float4* src = ysrc + (size_t)ks * g.HW * rowq;
-    float4* dst = reinterpret_cast<float4*>(s.tile);
-    for (int i = threadIdx.x; i < g.HW * (kChunk / 4); i += blockDim.x) dst[i] = src[(size_t)(i >> 3) * rowq + (i & 7)];
-    const uint32_t shift0 = P & 31u;
-    uint32_t slab_bits = 0;
-    if (mode == kQuant) {
-      const int i0 = ks * g.HW;
-      for (int j = threadIdx.x; j < g.HW; j += blockDim.x) {
-        const uint32_t b = pay[kHeaderBytes + i0 + j];
-        s.b[j] = b;
-        s.off[j] = b;
-        s.gain[j] = b ? 1.0f / reinterpret_cast<const float*>(pay + g.off_sigma)[i0 + j] : 0.0f;
-      }
-      __syncthreads();
-      slab_bits = block_exclusive_scan(s.off, g.HW, s.warp);
-      for (int j = threadIdx.x; j < g.HW; j += blockDim.x) s.off[j] += shift0;
-      const int nw = (int)((shift0 + slab_bits + 31) >> 5) + 1;
-      for (int i = threadIdx.x; i < kChunk * nw; i += blockDim.x) {
-        const int ch = i / nw, w = i - ch * nw;
-        s.sbuf[ch * s.words + w] = w == 0 ? s.carry[ch] : 0u;
-      }
+  const unsigned char* pay_b = pay + kHeaderBytes;
+  const float* pay_sig = reinterpret_cast<const float*>(pay + g.off_sigma);
+
+  issue_tile(g, ysrc, 0, tiles);
+  cp_async_commit();
+  if (quant) {
+    for (int i = threadIdx.x; i < kLmThrTotal; i += blockDim.x) thr[i] = c_lm_thresholds[i];
+    if (threadIdx.x < kChunk) carry[threadIdx.x] = 0;
+    // every pencil's first stream bit, once: bits of each (k_s, k_h) row, then a scan in bin order
+    const int npen = g.S * g.H;
+    for (int p = threadIdx.x; p < npen; p += blockDim.x) {
+      const unsigned char* b = pay_b + (size_t)p * g.W;
+      uint32_t t = 0;
+      for (int w = 0; w < g.W; ++w) t += b[w];
+      pen[p] = t;
     }
     __syncthreads();
-    tile_pass<HC, false>(g, s.tile, true);
+    block_exclusive_scan(pen, npen, swarp);
+  }
+  uint32_t P = 0;  // stream bits written so far, identical for every channel
+  for (int ks = 0; ks < g.S; ++ks) {
+    const int cur = L.nbuf == 2 ? (ks & 1) : 0;
+    float2* tile = tiles + (size_t)cur * g.HW * kPairs;
+    cp_async_wait_all();
+    __syncthreads();  // slab ks is in place and every thread is done with slab ks - 1
+    if (L.nbuf == 2 && ks + 1 < g.S) {
+      issue_tile(g, ysrc, ks + 1, tiles + (size_t)(cur ^ 1) * g.HW * kPairs);
+      cp_async_commit();
+    }
+    const uint32_t slab_end = quant ? (ks + 1 < g.S ? pen[(ks + 1) * g.H] : (uint32_t)0) : 0u;
+    const uint32_t w0 = P >> 5;                 // first stream word this slab touches
+    uint32_t slab_bits = 0;
+    if (quant) {
+      slab_bits = (ks + 1 < g.S ? slab_end : reinterpret_cast<const uint32_t*>(pay)[10]) - P;
+      const int nw = (int)(((P & 31u) + slab_bits + 31) >> 5) + 1;
+      for (int i = threadIdx.x; i < kChunk * nw; i += blockDim.x) {
+        const int ch = i / nw, w = i - ch * nw;
+        sbuf[ch * words + w] = w == 0 ? carry[ch] : 0u;
+      }
+    }
+    h_pass<HC, false>(g, tile);
     __syncthreads();
     // W pass fused with the per-bin epilogue
     for (int p = threadIdx.x; p < g.H * kPairs; p += blockDim.x) {
@@ -136,12 +175,12 @@ __global__ void __launch_bounds__(kHwThreads) fdct_hw_kernel(const __grid_consta
       float2 x[WC];
 #pragma unroll
       for (int t = 0; t < WC; ++t)
-        if (t < g.W) x[t] = s.tile[base + t * kPairs];
+        if (t < g.W) x[t] = tile[base + t * kPairs];
       dct_pencil<WC, false>(x, g.W);
       if (mode == kStats) {
 #pragma unroll
         for (int t = 0; t < WC; ++t)
-          if (t < g.W) s.tile[base + t * kPairs].x = x[t].x * x[t].x + x[t].y * x[t].y;
+          if (t < g.W) energy[(kh * g.W + t) * kEnergyStride + pair] = x[t].x * x[t].x + x[t].y * x[t].y;
       } else if (mode == kRaw) {
         const int c = chunk * kChunk + 2 * pair;
         float* s0 = reinterpret_cast<float*>(pay + g.off_codes + (size_t)c * cstride) + ks * g.HW + kh * g.W;
@@ -153,26 +192,36 @@ __global__ void __launch_bounds__(kHwThreads) fdct_hw_kernel(const __grid_consta
             s1[t] = x[t].y;
           }
       } else {
-        uint32_t* r0 = s.sbuf + (2 * pair) * s.words;
-        uint32_t* r1 = r0 + s.words;
+        // codes of the pencil's W bins are contiguous in each channel stream: pack them in a
+        // 64-bit register and flush whole words into the slab's stream buffer
+        const int i0 = (ks * g.H + kh) * g.W;
+        const uint32_t o0 = pen[ks * g.H + kh] - (w0 << 5);
+        uint32_t* r0 = sbuf + (2 * pair) * words + (o0 >> 5);
+        uint32_t* r1 = r0 + words;
+        unsigned long long a0 = 0, a1 = 0;
+        uint32_t apos = o0 & 31u;
 #pragma unroll
         for (int t = 0; t < WC; ++t) {
           if (t < g.W) {
-            const int j = kh * g.W + t;
-            const int bits = (int)s.b[j];
+            const int bits = pay_b[i0 + t];
             if (bits) {
-              const float inv = s.gain[j];
-              const uint32_t c0 = lm_code(x[t].x * inv, bits, s.thr);
-              const uint32_t c1 = lm_code(x[t].y * inv, bits, s.thr);
-              const uint32_t off = s.off[j], wi = off >> 5, sh = off & 31u;
-              atomicOr(r0 + wi, c0 << sh);
-              atomicOr(r1 + wi, c1 << sh);
-              if (sh + bits > 32) {
-                atomicOr(r0 + wi + 1, c0 >> (32 - sh));
-                atomicOr(r1 + wi + 1, c1 >> (32 - sh));
+              const float inv = __frcp_rn(pay_sig[i0 + t]);
+              a0 |= (unsigned long long)lm_code(x[t].x * inv, bits, thr) << apos;
+              a1 |= (unsigned long long)lm_code(x[t].y * inv, bits, thr) << apos;
+              apos += bits;
+              if (apos >= 32) {
+                atomicOr(r0++, (uint32_t)a0);
+                atomicOr(r1++, (uint32_t)a1);
+                a0 >>= 32;
+                a1 >>= 32;
+                apos -= 32;
               }
             }
           }
+        }
+        if (apos) {
+          atomicOr(r0, (uint32_t)a0);
+          atomicOr(r1, (uint32_t)a1);
         }
       }
     }
@@ -180,33 +229,38 @@ __global__ void __launch_bounds__(kHwThreads) fdct_hw_kernel(const __grid_consta
     if (mode == kStats) {
       float* dst = partial + ((size_t)u * g.nch + chunk) * g.N + (size_t)ks * g.HW;
       for (int j = threadIdx.x; j < g.HW; j += blockDim.x) {
+        const float* e = energy + j * kEnergyStride;
         float acc = 0.f;
 #pragma unroll
-        for (int q = 0; q < kPairs; ++q) acc += s.tile[j * kPairs + q].x;
+        for (int q = 0; q < kPairs; ++q) acc += e[q];
         dst[j] = acc;
       }
-    } else if (mode == kQuant) {
+    } else if (quant) {
       // complete words go out now; the word holding the run's last bits carries over
-      const uint32_t endbit = shift0 + slab_bits;
+      const uint32_t endbit = (P & 31u) + slab_bits;
       const int full = (int)(endbit >> 5);
-      const uint32_t w0 = P >> 5;
       for (int i = threadIdx.x; i < kChunk * full; i += blockDim.x) {
         const int ch = i / full, w = i - ch * full;
-        words_out[(size_t)(chunk * kChunk + ch) * stride_words + w0 + w] = s.sbuf[ch * s.words + w];
+        words_out[(size_t)(chunk * kChunk + ch) * stride_words + w0 + w] = sbuf[ch * words + w];
       }
-      __syncthreads();
-      if (threadIdx.x < kChunk) s.carry[threadIdx.x] = (endbit & 31u) ? s.sbuf[threadIdx.x * s.words + full] : 0u;
+      if (threadIdx.x < kChunk) carry[threadIdx.x] = (endbit & 31u) ? sbuf[threadIdx.x * words + full] : 0u;
       P += slab_bits;
     }
-    __syncthreads();
+    if (L.nbuf == 1 && ks + 1 < g.S) {
+      __syncthreads();  // everyone is done with the only tile
+      issue_tile(g, ysrc, ks + 1, tiles);
+      cp_async_commit();
+    }
   }
-  if (mode == kQuant) {
+  cp_async_wait_all();
+  if (quant) {
+    __syncthreads();
     // the last partial word, then zero padding up to the channel stride
     const uint32_t wlast = P >> 5;
     const int tail = (int)stride_words - (int)wlast;
     for (int i = threadIdx.x; i < kChunk * tail; i += blockDim.x) {
       const int ch = i / tail, w = i - ch * tail;
-      words_out[(size_t)(chunk * kChunk + ch) * stride_words + wlast + w] = (w == 0) ? s.carry[ch] : 0u;
+      words_out[(size_t)(chunk * kChunk + ch) * stride_words + wlast + w] = (w == 0) ? carry[ch] : 0u;
     }
   } else if (mode == kRaw) {
     const int pad = (int)cstride - 4 * g.N;
@@ -217,123 +271,154 @@ __global__ void __launch_bounds__(kHwThreads) fdct_hw_kernel(const __grid_consta
   }
 }
 
+// ----------------------------------------------------------------------------------- decode ---
 template <int HC, int WC>
 __global__ void __launch_bounds__(kHwThreads) idct_hw_kernel(const __grid_constant__ Geom g,
                                                              const __grid_constant__ UnitList ul, int mode,
                                                              float* __restrict__ V, unsigned int* status) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  HwSmem s = carve(smem_raw, g.HW);
+  extern __shared__ __align__(16) unsigned char smem[];
+  const HwLayout L = hw_layout(g.HW, true);
+  float2* tile = reinterpret_cast<float2*>(smem + L.tile);
+  float* lvs = reinterpret_cast<float*>(smem + L.lv);
+  uint32_t* pen = reinterpret_cast<uint32_t*>(smem + L.meta_b);   // first stream bit of every pencil
+  uint32_t* sbufs = reinterpret_cast<uint32_t*>(smem + L.uni);
+  uint32_t* swarp = reinterpret_cast<uint32_t*>(smem + L.warp);
   __shared__ int s_ok;
-  __shared__ unsigned int s_bad_b;
+  __shared__ unsigned int s_bad;
+  const int words = L.words;
   const int chunk = blockIdx.x, u = blockIdx.y;
   const UnitDev& ud = ul.u[u];
   const unsigned char* pay = ud.payload;
   const bool raw = mode == kRaw;
+  uint32_t code_bits = 0;
   if (threadIdx.x == 0) {
     // the header must describe exactly the unit the caller asked for
     const uint32_t* h32 = reinterpret_cast<const uint32_t*>(pay);
     const int32_t* i32 = reinterpret_cast<const int32_t*>(pay);
-    const uint32_t ver_flags = h32[1], code_bits = h32[10], cstride = h32[11];
+    const uint32_t ver_flags = h32[1], cb = h32[10], cs = h32[11];
     const unsigned long long total = *reinterpret_cast<const unsigned long long*>(pay + 48);
     bool ok = h32[0] == kMagic && (ver_flags & 0xffffu) == (uint32_t)kVersion &&
               ((ver_flags >> 16) & TACTKV_NO_QUANT) == (raw ? TACTKV_NO_QUANT : 0u) && i32[2] == ud.layer &&
               i32[3] == ud.kv && i32[4] == g.S && i32[5] == g.H && i32[6] == g.W && i32[7] == g.heads &&
               i32[8] == g.head_dim && i32[9] == g.bits;
     if (ok) {
-      ok = (raw ? code_bits == 32u * (uint32_t)g.N : code_bits <= (uint32_t)g.bits * (uint32_t)g.N) &&
-           (long long)cstride == pad16(((long long)code_bits + 7) / 8) &&
-           (long long)total == (long long)g.off_codes + (long long)g.n * cstride && (long long)total <= g.capacity;
+      ok = (raw ? cb == 32u * (uint32_t)g.N : cb <= (uint32_t)g.bits * (uint32_t)g.N) &&
+           (long long)cs == pad16(((long long)cb + 7) / 8) &&
+           (long long)total == (long long)g.off_codes + (long long)g.n * cs && (long long)total <= g.capacity;
     }
     s_ok = ok;
-    s_bad_b = 0;
-    if (!ok && chunk == 0) set_status(status, TACTKV_CORRUPT_PAYLOAD);
+    s_bad = 0;
   }
-  for (int i = threadIdx.x; i < kLmLvTotal; i += blockDim.x) s.lv[i] = c_lm_levels[i];
+  for (int i = threadIdx.x; i < kLmLvTotal; i += blockDim.x) lvs[i] = c_lm_levels[i];
+  __syncthreads();
+  const bool ok0 = s_ok;
+  const uint32_t stride_words = ok0 ? reinterpret_cast<const uint32_t*>(pay)[11] / 4 : 0u;
+  if (ok0) code_bits = reinterpret_cast<const uint32_t*>(pay)[10];
+  const uint32_t* streams = reinterpret_cast<const uint32_t*>(pay + g.off_codes);
+  const unsigned char* pay_b = pay + kHeaderBytes;
+  const float* pay_sig = reinterpret_cast<const float*>(pay + g.off_sigma);
+  const int npen = g.S * g.H;
+  // every pencil's first stream bit: bits of each (k_s, k_h) row, then a scan in bin order
+  if (ok0 && !raw) {
+    for (int p = threadIdx.x; p < npen; p += blockDim.x) {
+      const unsigned char* b = pay_b + (size_t)p * g.W;
+      uint32_t t = 0;
+      for (int w = 0; w < g.W; ++w) {
+        const uint32_t v = b[w];
+        if (v > 8) s_bad = 1;
+        t += v;
+      }
+      pen[p] = t;
+    }
+    __syncthreads();
+    const uint32_t total = block_exclusive_scan(pen, npen, swarp);
+    if (threadIdx.x == 0 && (total != code_bits || s_bad)) s_ok = 0;
+  }
   __syncthreads();
   const bool ok = s_ok;
-  const uint32_t stride_words = ok ? reinterpret_cast<const uint32_t*>(pay)[11] / 4 : 0u;
-  const uint32_t* streams = reinterpret_cast<const uint32_t*>(pay + g.off_codes);
+  if (threadIdx.x == 0 && !ok && chunk == 0) set_status(status, TACTKV_CORRUPT_PAYLOAD);
+  const int ch0 = chunk * kChunk;
+  auto slab_begin = [&](int ks) -> uint32_t { return ks < g.S ? pen[ks * g.H] : code_bits; };
+
+  auto issue_words = [&](int ks, uint32_t* sb) {  // stream words of slab ks for the 32 channels
+    const uint32_t p0 = slab_begin(ks), p1 = slab_begin(ks + 1);
+    const uint32_t w0 = p0 >> 5;
+    const int nw = (int)(((p0 & 31u) + (p1 - p0) + 31) >> 5);
+    for (int i = threadIdx.x; i < kChunk * (nw + 1); i += blockDim.x) {
+      const int ch = i / (nw + 1), w = i - ch * (nw + 1);
+      const uint32_t word = w0 + w;
+      if (w < nw && word < stride_words) cp_async4(sb + ch * words + w, streams + (size_t)(ch0 + ch) * stride_words + word);
+      else sb[ch * words + w] = 0u;
+    }
+  };
+
+  if (ok && !raw) {
+    issue_words(0, sbufs);
+    cp_async_commit();
+  }
   float4* vdst = reinterpret_cast<float4*>(V + (size_t)u * g.S * g.HW * g.n) + chunk * (kChunk / 4);
   const int rowq = g.n / 4;
-  uint32_t P = 0;
   for (int ks = 0; ks < g.S; ++ks) {
-    const int i0 = ks * g.HW;
-    const uint32_t shift0 = P & 31u;
-    uint32_t slab_bits = 0;
-    if (ok) {
-      for (int j = threadIdx.x; j < g.HW; j += blockDim.x) {
-        const uint32_t b = raw ? 0u : pay[kHeaderBytes + i0 + j];
-        if (b > 8) s_bad_b = 1;
-        s.b[j] = b > 8 ? 0u : b;
-        s.off[j] = s.b[j];
-        s.gain[j] = reinterpret_cast<const float*>(pay + g.off_sigma)[i0 + j];
-      }
-      __syncthreads();
-      if (!raw) {
-        slab_bits = block_exclusive_scan(s.off, g.HW, s.warp);
-        for (int j = threadIdx.x; j < g.HW; j += blockDim.x) s.off[j] += shift0;
-        const int nw = (int)((shift0 + slab_bits + 31) >> 5);
-        const uint32_t w0 = P >> 5;
-        for (int i = threadIdx.x; i < kChunk * (nw + 1); i += blockDim.x) {
-          const int ch = i / (nw + 1), w = i - ch * (nw + 1);
-          const uint32_t word = w0 + w;
-          s.sbuf[ch * s.words + w] =
-              (w < nw && word < stride_words) ? streams[(size_t)(chunk * kChunk + ch) * stride_words + word] : 0u;
-        }
-      }
-      __syncthreads();
+    const int mc = ks & 1;
+    const uint32_t* sb = sbufs + (size_t)mc * kChunk * words;
+    cp_async_wait_all();
+    __syncthreads();  // slab ks's stream words are in place; slab ks - 1 is done
+    if (ok && !raw && ks + 1 < g.S) {
+      issue_words(ks + 1, sbufs + (size_t)(mc ^ 1) * kChunk * words);
+      cp_async_commit();
     }
+    const int i0s = ks * g.HW;
+    const uint32_t wbase = raw ? 0u : (slab_begin(ks) >> 5) << 5;
     // inverse DCT along W from the dequantized coefficients
     for (int p = threadIdx.x; p < g.H * kPairs; p += blockDim.x) {
       const int kh = p >> 4, pair = p & 15;
       const int base = kh * g.W * kPairs + pair;
-      const int c = chunk * kChunk + 2 * pair;
+      const int c = ch0 + 2 * pair;
+      const int i0 = i0s + kh * g.W;
       float2 x[WC];
+      if (!ok) {
 #pragma unroll
-      for (int t = 0; t < WC; ++t) {
-        if (t < g.W) {
-          float2 v = make_float2(0.f, 0.f);
-          if (ok) {
-            const int j = kh * g.W + t;
-            if (raw) {
-              const float* st = reinterpret_cast<const float*>(streams);
-              v.x = st[(size_t)c * stride_words + i0 + j];
-              v.y = st[(size_t)(c + 1) * stride_words + i0 + j];
-            } else {
-              const int bits = (int)s.b[j];
-              if (bits) {
-                const uint32_t off = s.off[j], wi = off >> 5, sh = off & 31u, mask = (1u << bits) - 1u;
-                const uint32_t* r0 = s.sbuf + (2 * pair) * s.words + wi;
-                const uint32_t* r1 = r0 + s.words;
-                const uint32_t c0 = (uint32_t)(((((unsigned long long)r0[1]) << 32) | r0[0]) >> sh) & mask;
-                const uint32_t c1 = (uint32_t)(((((unsigned long long)r1[1]) << 32) | r1[0]) >> sh) & mask;
-                const float* lv = s.lv + lm_lv_offset(bits);
-                const float sg = s.gain[j];
-                v = make_float2(sg * lv[c0], sg * lv[c1]);
-              }
+        for (int t = 0; t < WC; ++t) x[t] = make_float2(0.f, 0.f);
+      } else if (raw) {
+        const float* st = reinterpret_cast<const float*>(streams);
+#pragma unroll
+        for (int t = 0; t < WC; ++t)
+          if (t < g.W) x[t] = make_float2(st[(size_t)c * stride_words + i0 + t], st[(size_t)(c + 1) * stride_words + i0 + t]);
+      } else {
+        uint32_t o = pen[ks * g.H + kh] - wbase;
+        const uint32_t* r0 = sb + (2 * pair) * words;
+        const uint32_t* r1 = r0 + words;
+#pragma unroll
+        for (int t = 0; t < WC; ++t) {
+          if (t < g.W) {
+            const int bits = pay_b[i0 + t];
+            float2 v = make_float2(0.f, 0.f);
+            if (bits) {
+              const uint32_t wi = o >> 5, sh = o & 31u, mask = (1u << bits) - 1u;
+              const uint32_t c0 = (uint32_t)(((((unsigned long long)r0[wi + 1]) << 32) | r0[wi]) >> sh) & mask;
+              const uint32_t c1 = (uint32_t)(((((unsigned long long)r1[wi + 1]) << 32) | r1[wi]) >> sh) & mask;
+              const float* lv = lvs + lm_lv_offset(bits);
+              const float sg = pay_sig[i0 + t];
+              v = make_float2(sg * lv[c0], sg * lv[c1]);
+              o += bits;
             }
+            x[t] = v;
           }
-          x[t] = v;
         }
       }
       dct_pencil<WC, true>(x, g.W);
 #pragma unroll
       for (int t = 0; t < WC; ++t)
-        if (t < g.W) s.tile[base + t * kPairs] = x[t];
+        if (t < g.W) tile[base + t * kPairs] = x[t];
     }
     __syncthreads();
-    tile_pass<HC, true>(g, s.tile, true);
+    h_pass<HC, true>(g, tile);
     __syncthreads();
     float4* dst = vdst + (size_t)ks * g.HW * rowq;
-    const float4* src = reinterpret_cast<const float4*>(s.tile);
+    const float4* src = reinterpret_cast<const float4*>(tile);
     for (int i = threadIdx.x; i < g.HW * (kChunk / 4); i += blockDim.x) dst[(size_t)(i >> 3) * rowq + (i & 7)] = src[i];
-    P += slab_bits;
-    __syncthreads();
   }
-  if (threadIdx.x == 0 && ok && !raw) {
-    const uint32_t code_bits = reinterpret_cast<const uint32_t*>(pay)[10];
-    if (P != code_bits || s_bad_b) set_status(status, TACTKV_CORRUPT_PAYLOAD);
-  }
+  cp_async_wait_all();
 }
 
 }  // namespace
@@ -342,16 +427,18 @@ __global__ void __launch_bounds__(kHwThreads) idct_hw_kernel(const __grid_consta
 #define TACTKV_CAT(a, b) TACTKV_CAT2(a, b)
 #define TACTKV_LAUNCHER(h, w) TACTKV_CAT(TACTKV_CAT(TACTKV_CAT(launch_axis_hw_, h), _), w)
 cudaError_t TACTKV_LAUNCHER(TACTKV_HCLASS, TACTKV_WCLASS)(bool inverse, int mode, const Geom& g, const UnitList& ul,
-                                                      int nu, float* buf, float* partial, unsigned int* status,
-                                                      cudaStream_t st) {
-  const size_t sm = hw_smem_bytes(g.HW);
+                                                          int nu, float* buf, float* partial, unsigned int* status,
+                                                          cudaStream_t st) {
+  const HwLayout L = hw_layout(g.HW, inverse);
   const dim3 grid(g.nch, nu);
   if (inverse) {
-    cudaFuncSetAttribute(idct_hw_kernel<TACTKV_HCLASS, TACTKV_WCLASS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    idct_hw_kernel<TACTKV_HCLASS, TACTKV_WCLASS><<<grid, kHwThreads, sm, st>>>(g, ul, mode, buf, status);
+    cudaFuncSetAttribute(idct_hw_kernel<TACTKV_HCLASS, TACTKV_WCLASS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)L.total);
+    idct_hw_kernel<TACTKV_HCLASS, TACTKV_WCLASS><<<grid, kHwThreads, L.total, st>>>(g, ul, mode, buf, status);
   } else {
-    cudaFuncSetAttribute(fdct_hw_kernel<TACTKV_HCLASS, TACTKV_WCLASS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    fdct_hw_kernel<TACTKV_HCLASS, TACTKV_WCLASS><<<grid, kHwThreads, sm, st>>>(g, ul, mode, buf, partial);
+    cudaFuncSetAttribute(fdct_hw_kernel<TACTKV_HCLASS, TACTKV_WCLASS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)L.total);
+    fdct_hw_kernel<TACTKV_HCLASS, TACTKV_WCLASS><<<grid, kHwThreads, L.total, st>>>(g, ul, mode, buf, partial);
   }
   return cudaGetLastError();
 }

@@ -63,13 +63,6 @@ inline bool supported_length(int L) {
 }
 inline int length_class(int L) { return L <= 16 ? 16 : (L <= 32 ? 32 : 64); }
 
-// Shared memory of the H/W-axis kernels.
-__host__ __device__ inline int stream_words_per_slab(int HW) { return (8 * HW + 31) / 32 + 2; }
-__host__ __device__ inline size_t hw_smem_bytes(int HW) {
-  const size_t w = stream_words_per_slab(HW);
-  return (size_t)HW * kPairs * 8 + (size_t)(kLmThrTotal + kLmLvTotal) * 4 + (size_t)HW * 4 * 3 +
-         (size_t)kChunk * w * 4 + kChunk * 4 + 33 * 4 + 64;
-}
 
 // --------------------------------------------------------------------------------- launchers ---
 cudaError_t launch_axis_s(int cls, bool inverse, const Geom& g, const UnitList& ul, int nu, float* buf,
@@ -88,12 +81,19 @@ __device__ __forceinline__ float2 vneg(float2 a) { return make_float2(-a.x, -a.y
 __device__ __forceinline__ float2 vmul(float2 a, float c) { return __fmul2_rn(a, make_float2(c, c)); }
 __device__ __forceinline__ float2 vfma(float2 a, float c, float2 b) { return __ffma2_rn(a, make_float2(c, c), b); }
 
+// one-channel pencils use plain fp32 operations
+__device__ __forceinline__ float vadd(float a, float b) { return a + b; }
+__device__ __forceinline__ float vsub(float a, float b) { return a - b; }
+__device__ __forceinline__ float vneg(float a) { return -a; }
+__device__ __forceinline__ float vmul(float a, float c) { return a * c; }
+__device__ __forceinline__ float vfma(float a, float c, float b) { return fmaf(a, c, b); }
+
 // the generated pencil transforms (templates over the value type) live in this namespace too
 #include "dct_gen.cuh"
 
 // Orthonormal DCT-II (INV = false) or DCT-III (INV = true) of x[0..L) held in registers.
-template <int CLASS, bool INV>
-__device__ __forceinline__ void dct_pencil(float2* x, int L) {
+template <int CLASS, bool INV, class V>
+__device__ __forceinline__ void dct_pencil(V* x, int L) {
 #define TACTKV_CASE(n)                          \
   case n:                                       \
     if constexpr (INV) idct_##n(x);             \
@@ -122,6 +122,14 @@ __device__ __forceinline__ void dct_pencil(float2* x, int L) {
 
 __device__ __forceinline__ void set_status(unsigned int* status, unsigned int code) { atomicCAS(status, 0u, code); }
 
+__device__ __forceinline__ float load_one(const void* base, long long elem, bool fp32) {
+  if (fp32) return static_cast<const float*>(base)[elem];
+  return __bfloat162float(static_cast<const __nv_bfloat16*>(base)[elem]);
+}
+__device__ __forceinline__ void store_one(void* base, long long elem, float v, bool fp32) {
+  if (fp32) static_cast<float*>(base)[elem] = v;
+  else static_cast<__nv_bfloat16*>(base)[elem] = __float2bfloat16_rn(v);
+}
 __device__ __forceinline__ float2 load_pair(const void* base, long long elem, bool fp32) {
   if (fp32) return *reinterpret_cast<const float2*>(static_cast<const float*>(base) + elem);
   return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(static_cast<const __nv_bfloat16*>(base) + elem));
@@ -130,6 +138,18 @@ __device__ __forceinline__ void store_pair(void* base, long long elem, float2 v,
   if (fp32) *reinterpret_cast<float2*>(static_cast<float*>(base) + elem) = v;
   else *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(base) + elem) = __float22bfloat162_rn(v);
 }
+
+// Asynchronous global -> shared copies (LDGSTS): issued now, waited for with cp_async_wait_all.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
+  const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
 
 // In place exclusive scan of a[0..n) in shared memory; blockDim.x a multiple of 32; returns the total.
 __device__ inline uint32_t block_exclusive_scan(uint32_t* a, int n, uint32_t* s_warp /* 33 entries */) {

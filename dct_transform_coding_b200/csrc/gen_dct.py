@@ -8,7 +8,8 @@ and their inverses for decoding.  The oracle does not use this file.
 Algorithm (for the un-normalised Z[k] = sum_t x[t] cos(pi (2t+1) k / (2L))):
   * even L: u[t] = x[t] + x[L-1-t], v[t] = x[t] - x[L-1-t] (t < L/2); the even outputs are the
     length-L/2 DCT-II of u and the odd outputs Z[2k+1] are the length-L/2 DCT-IV of v;
-  * the DCT-IV halves and odd-length DCT-IIs: the definition, one multiply-add per term.
+  * DCT-IV halves of power-of-two length >= 8: pre-twiddle, complex FFT of half the length,
+    post-twiddle (see dct4_unnorm); other DCT-IV halves and odd-length DCT-IIs: the definition.
 Orthonormal scaling a_0 = sqrt(1/L), a_k = sqrt(2/L) is applied to the outputs.  The inverse
 (DCT-III) is emitted as the exact transpose of the forward flow graph (reverse-mode accumulation
 of the same linear statements), so forward and inverse use the same constants.
@@ -71,34 +72,91 @@ def dct2_unnorm(g: Graph, x: List[int]) -> List[int]:
     return dense(g, x, lambda k, t: math.cos(math.pi * (2 * t + 1) * k / (2 * L)))
 
 
-def dct4_unnorm(g: Graph, v: List[int]) -> List[int]:
-    """DCT-IV by its definition.  (The shorter route through a pre-scaled DCT-II and the running
-    difference Y[k] = Z'[k] - Y[k-1] carries the rounding error of the large low-frequency terms
-    into the small high-frequency ones and is ~14x less accurate in float32, too much for the
-    code-level parity the codec needs.)"""
-    M = len(v)
-    return dense(g, v, lambda k, t: math.cos(math.pi * (2 * t + 1) * (2 * k + 1) / (4 * M)))
+def cmul_const(g: Graph, z, w: complex):
+    """z * w for a complex constant w (z a pair of nodes)."""
+    a, b = z
+    c, d = w.real, w.imag
+    if abs(d) < 1e-15 and abs(c - 1) < 1e-15:
+        return z
+    if abs(c) < 1e-15:                                  # w = i d: (a + ib) i d = -b d + i a d
+        return (g.scale(b, -d), g.scale(a, d))
+    if abs(d) < 1e-15:
+        return (g.scale(a, c), g.scale(b, c))
+    return (g.lin([(c, a), (-d, b)]), g.lin([(d, a), (c, b)]))
 
 
-def dense(g: Graph, x: List[int], coef) -> List[int]:
-    L = len(x)
-    out = []
-    for k in range(L):
-        acc = g.scale(x[0], coef(k, 0))
-        for t in range(1, L):
-            c = coef(k, t)
-            if abs(c) < 1e-15:
-                continue
-            acc = g.lin([(c, x[t]), (1.0, acc)])
-        out.append(acc)
+def fft(g: Graph, z, sign: int):
+    """Z[p] = sum_m z[m] exp(sign 2 pi i m p / M), radix 2 (len(z) a power of two)."""
+    M = len(z)
+    if M == 1:
+        return list(z)
+    E = fft(g, z[0::2], sign)
+    O = fft(g, z[1::2], sign)
+    out = [None] * M
+    for p in range(M // 2):
+        t = cmul_const(g, O[p], complex(math.cos(2 * math.pi * p / M), sign * math.sin(2 * math.pi * p / M)))
+        out[p] = (g.add(E[p][0], t[0]), g.add(E[p][1], t[1]))
+        out[p + M // 2] = (g.sub(E[p][0], t[0]), g.sub(E[p][1], t[1]))
     return out
 
 
+def dct4_unnorm(g: Graph, v: List[int]) -> List[int]:
+    """DCT-IV, Y[k] = sum_t v[t] cos(pi (2t+1)(2k+1) / (4N)).
+
+    N a power of two >= 8: with a_m = v[2m], b_m = v[N-1-2m] (m < N/2),
+        sum_m (a_m - i b_m) exp(i pi (4m+1)(4p+1) / (4N)) = Y[2p] + i Y[N-1-2p],
+    and the exponent splits into exp(i pi m/N) (pre-twiddle), exp(2 pi i m p / (N/2)) (an
+    N/2-point DFT, by FFT) and exp(i pi (p + 1/4)/N) (post-twiddle).  Every step is a rotation or
+    a butterfly, so float32 rounding stays at the level of the dense product.  Other lengths: the
+    definition.  (The shorter route through a pre-scaled DCT-II and the running difference
+    Y[k] = Z'[k] - Y[k-1] carries the rounding error of the large low-frequency terms into the
+    small high-frequency ones and is ~14x less accurate in float32: not used.)"""
+    N = len(v)
+    if N >= 8 and N & (N - 1) == 0:
+        M = N // 2
+        d = []
+        for m in range(M):
+            a, b = v[2 * m], v[N - 1 - 2 * m]
+            al = math.pi * m / N
+            ca, sa = math.cos(al), math.sin(al)
+            if m == 0:
+                d.append((a, g.scale(b, -1.0)))
+            else:                                       # (a - i b)(cos al + i sin al)
+                d.append((g.lin([(ca, a), (sa, b)]), g.lin([(sa, a), (-ca, b)])))
+        D = fft(g, d, +1)
+        Y = [None] * N
+        for p in range(M):
+            be = math.pi * (p + 0.25) / N
+            re, im = cmul_const(g, D[p], complex(math.cos(be), math.sin(be)))
+            Y[2 * p] = re
+            Y[N - 1 - 2 * p] = im
+        return Y
+    return dense(g, v, lambda k, t: math.cos(math.pi * (2 * t + 1) * (2 * k + 1) / (4 * N)))
+
+
+def dense(g: Graph, x: List[int], coef) -> List[int]:
+    """Matrix-vector product, emitted term-major: every output advances by one multiply-add per
+    step, so neighbouring statements are independent (L chains in flight, not one)."""
+    L = len(x)
+    acc = [g.scale(x[0], coef(k, 0)) for k in range(L)]
+    for t in range(1, L):
+        for k in range(L):
+            c = coef(k, t)
+            if abs(c) < 1e-15:
+                continue
+            acc[k] = g.lin([(c, x[t]), (1.0, acc[k])])
+    return acc
+
+
 def build_forward(L: int) -> Tuple[Graph, List[int]]:
+    """Forward orthonormal DCT-II flow graph.  The recursion is built once, then transposed twice:
+    the second transpose computes the same map with the scale factors folded into the
+    multiply-adds (see transpose_graph), a few percent fewer statements."""
     g = Graph(L)
     Z = dct2_unnorm(g, list(range(L)))
     out = [g.scale(Z[k], math.sqrt((1.0 if k == 0 else 2.0) / L)) for k in range(L)]
-    return g, out
+    tg, touts = transpose_graph(g, out)
+    return transpose_graph(tg, touts)
 
 
 def evaluate(g: Graph, outs: List[int], x: np.ndarray, dtype=np.float64) -> np.ndarray:
@@ -164,26 +222,34 @@ def emit_program(g: Graph, inputs: List[str], outs: List[int], out_names: List[s
 
 
 def transpose_graph(g: Graph, outs: List[int]) -> Tuple[Graph, List[int]]:
-    """Adjoint program: inputs are the forward outputs' adjoints, outputs the inputs' adjoints."""
+    """Adjoint program: inputs are the forward outputs' adjoints, outputs the inputs' adjoints.
+
+    Adjoints are carried as (coefficient, node) pairs meaning coefficient * node, so a scale is
+    only materialized when two contributions meet (c1 n1 + c2 n2 = c1 (n1 + (c2/c1) n2), one
+    fused multiply-add) or at an output."""
     L = len(outs)
     tg = Graph(L)
-    adj: Dict[int, int] = {}
+    adj: Dict[int, List[Tuple[float, int]]] = {}
 
-    def acc(node: int, src: int, c: float):
-        if node not in adj:
-            adj[node] = src if c == 1.0 else tg.scale(src, c)
-        else:
-            adj[node] = tg.lin([(1.0, adj[node]), (c, src)])     # one fused statement
+    def combine(terms: List[Tuple[float, int]]) -> Tuple[float, int]:
+        c0, n0 = terms[0]
+        for c, n in terms[1:]:
+            n0 = tg.lin([(1.0, n0), (c / c0, n)])
+        return c0, n0
 
     for j, o in enumerate(outs):
-        acc(o, j, 1.0)
+        adj.setdefault(o, []).append((1.0, j))
     for idx in range(len(g.ops) - 1, g.n_in - 1, -1):
         if idx not in adj:
             continue
-        a = adj.pop(idx)
-        for c, s in g.ops[idx]:
-            acc(s, a, c)
-    return tg, [adj[i] for i in range(g.n_in)]
+        c, n = combine(adj.pop(idx))
+        for cop, src in g.ops[idx]:
+            adj.setdefault(src, []).append((c * cop, n))
+    res = []
+    for i in range(g.n_in):
+        c, n = combine(adj[i])
+        res.append(n if c == 1.0 else tg.scale(n, c))
+    return tg, res
 
 
 def generate(lengths=FAST_LENGTHS) -> str:
