@@ -33,35 +33,45 @@ constexpr int kMaxSlabs = 64;
 __host__ __device__ inline int stream_words_per_slab(int HW) { return (8 * HW + 31) / 32 + 2; }
 
 struct HwLayout {
-  size_t tile, thr, lv, meta_b, meta_g, off, uni, carry, warp, slab, total;
+  size_t tile, thr, lv, pen, meta, off, uni, carry, warp, bsl, sig2, total;
+  size_t bsl_stride;
   int nbuf;
   int words;
 };
 
-// Shared memory carve-up; `uni` holds the energy rows (kStats) or the stream words (kQuant and
-// decoding) -- never both in one launch.
-__host__ __device__ inline HwLayout hw_layout(int HW, bool decode) {
+enum LayoutKind { kLayStats = 0, kLayQuant = 1, kLayDecode = 2 };
+
+// Shared memory carve-up of one launch.  stats: slab tiles and padded energy rows; quant: slab
+// tiles, thresholds, pencil offsets, per-bin metadata, the bit widths and sigmas of two slabs
+// and the stream words of a slab; decode: one tile, levels, the same metadata and two slabs of
+// stream words.  Regions a kind does not use have size 0.
+__host__ __device__ inline HwLayout hw_layout(int HW, int N, int S, int H, int kind) {
   HwLayout L;
   L.words = stream_words_per_slab(HW);
+  const bool st = kind == kLayStats, qu = kind == kLayQuant, de = kind == kLayDecode;
   const size_t tile1 = (size_t)HW * kPairs * 8;
-  const size_t energy = (size_t)HW * kEnergyStride * 4;
-  const size_t words = (size_t)kChunk * L.words * 4 * (decode ? 2 : 1);
-  const size_t uni = energy > words ? energy : words;
-  const size_t fixed = (size_t)(kLmThrTotal + kLmLvTotal) * 4 + (size_t)HW * 4 * 3 +
-                       (size_t)(HW > kMaxSlabs * 32 ? HW : kMaxSlabs * 32) * 8 + uni + kChunk * 4 + 33 * 4 +
-                       (kMaxSlabs + 1) * 4 + 256;
-  L.nbuf = (decode || 2 * tile1 + fixed > kSmemBudget) ? 1 : 2;
+  const size_t energy = st ? (size_t)HW * kEnergyStride * 4 : 0;
+  const size_t words = st ? 0 : (size_t)kChunk * L.words * 4 * (de ? 2 : 1);
+  const size_t thr = qu ? kLmThrTotal * 4 : 0, lv = de ? kLmLvTotal * 4 : 0;
+  const size_t pen = st ? 0 : ((size_t)S * H * 4 + 15) / 16 * 16;
+  const size_t meta = st ? 0 : (size_t)HW * 8, off = st ? 0 : ((size_t)HW * 4 + 15) / 16 * 16;
+  // a slab's bit widths are fetched as the 16-byte aligned window around them
+  L.bsl_stride = ((size_t)HW + 15) / 16 * 16 + 32;
+  const size_t bsl = st ? 0 : 2 * L.bsl_stride, sig2 = st ? 0 : (size_t)HW * 8;
+  const size_t fixed = thr + lv + pen + meta + off + energy + words + kChunk * 4 + 33 * 4 + bsl + sig2 + 256;
+  L.nbuf = (de || 2 * tile1 + fixed > kSmemBudget) ? 1 : 2;
   size_t o = 0;
   L.tile = o; o += tile1 * L.nbuf;
-  L.thr = o; o += kLmThrTotal * 4;
-  L.lv = o; o += kLmLvTotal * 4;
-  L.meta_b = o; o += (size_t)(HW > kMaxSlabs * 32 ? HW : kMaxSlabs * 32) * 4 * 2;
-  L.meta_g = o; o += (size_t)HW * 4 * 2;
-  L.off = o; o += (size_t)HW * 4;
-  L.uni = o; o += (uni + 15) / 16 * 16;
+  L.uni = o; o += ((energy > words ? energy : words) + 15) / 16 * 16;
+  L.bsl = o; o += bsl;
+  L.thr = o; o += thr;
+  L.lv = o; o += lv;
+  L.pen = o; o += pen;
+  L.meta = o; o += meta;
+  L.off = o; o += off;
+  L.sig2 = o; o += sig2;
   L.carry = o; o += kChunk * 4;
   L.warp = o; o += 33 * 4;
-  L.slab = o; o += (kMaxSlabs + 1) * 4;
   L.total = o;
   return L;
 }
@@ -73,6 +83,17 @@ __device__ __forceinline__ uint32_t lm_code(float u, int bits, const float* thr)
   for (int step = 1 << (bits - 1); step > 0; step >>= 1)
     if (u >= t[code + step - 1]) code += step;
   return code;
+}
+
+// Code for u at 1, 2 or more bits (the count of thresholds t <= u).  The 1- and 2-bit codebooks
+// have thresholds {0} and {-t, 0, t}: a sign test and three compares; wider ones use bisection.
+__device__ __forceinline__ uint32_t quant_code(float u, int bits, const float* thr) {
+  if (bits == 1) return u >= 0.f;
+  if (bits == 2) {
+    const float t = thr[lm_thr_offset(2) + 2];
+    return (uint32_t)(u >= -t) + (uint32_t)(u >= 0.f) + (uint32_t)(u >= t);
+  }
+  return lm_code(u, bits, thr);
 }
 
 // Pencil DCTs along H of the tile: pencils (w, pair), stride W*16 between elements.
@@ -101,15 +122,84 @@ __device__ __forceinline__ void issue_tile(const Geom& g, const float4* ysrc_uni
     cp_async16(dst + i, src + (size_t)(i >> 3) * rowq + (i & 7));
 }
 
-template <int HC, int WC>
+// The unit's bit widths into shared memory (16-byte copies: the payload and its b[] array are
+// 16-byte aligned and padded), used once to compute the pencil offsets.
+__device__ __forceinline__ void issue_bits(const Geom& g, const unsigned char* pay_b, unsigned char* dst) {
+  for (int i = threadIdx.x; i < (g.N + 15) / 16; i += blockDim.x) cp_async16(dst + 16 * i, pay_b + 16 * i);
+}
+// The bit widths of slab ks as the 16-byte aligned window that holds them; they start at byte
+// (ks * HW) % 16 of dst.  The window ends inside the padded b[] array.
+__device__ __forceinline__ void issue_slab_bits(const Geom& g, const unsigned char* pay_b, int ks, unsigned char* dst) {
+  const size_t a0 = (size_t)ks * g.HW, q0 = a0 / 16, q1 = (a0 + g.HW + 15) / 16;
+  for (int i = threadIdx.x; i < (int)(q1 - q0); i += blockDim.x) cp_async16(dst + 16 * i, pay_b + 16 * (q0 + i));
+}
+// The sigmas of slab ks (4-byte copies).
+__device__ __forceinline__ void issue_sigma(const Geom& g, const float* pay_sig, int ks, float* dst) {
+  for (int j = threadIdx.x; j < g.HW; j += blockDim.x) cp_async4(dst + j, pay_sig + (size_t)ks * g.HW + j);
+}
+
+// Stream bit offset of every (k_s, k_h) pencil: the bits of each row of W bins, then an exclusive
+// scan in bin order.  bfull: the unit's bit widths in shared memory.  Returns the total; sets
+// *bad when a width exceeds 8.
+__device__ __forceinline__ uint32_t pencil_offsets(const Geom& g, const unsigned char* bfull, uint32_t* pen,
+                                                   uint32_t* swarp, unsigned int* bad) {
+  const int npen = g.S * g.H;
+  for (int p = threadIdx.x; p < npen; p += blockDim.x) {
+    const unsigned char* b = bfull + (size_t)p * g.W;
+    uint32_t t = 0;
+    bool over = false;
+    for (int w = 0; w < g.W; ++w) {
+      const uint32_t v = b[w];
+      over |= v > 8;
+      t += v;
+    }
+    if (over) *bad = 1;
+    pen[p] = t;
+  }
+  __syncthreads();
+  return block_exclusive_scan(pen, npen, swarp);
+}
+
+// Bits, gain and stream bit offset of every bin of slab ks: one warp per (k_s, k_h) row of at most
+// 32 bins, the offset being the row's start (pen) plus a shuffle scan of the row's bit widths.
+// gain_inv: store 1/sigma (encoding) instead of sigma (decoding).
+// bsl: this slab's bit widths in shared memory; sig: its sigmas.
+__device__ __forceinline__ void slab_meta(const Geom& g, int ks, const unsigned char* bsl, const float* sig,
+                                          const uint32_t* pen, uint32_t wbase, bool gain_inv, uint32_t* sb_bits,
+                                          float* sb_gain, uint32_t* sb_off) {
+  const int lane = threadIdx.x & 31, nwarp = blockDim.x >> 5;
+  for (int kh = threadIdx.x >> 5; kh < g.H; kh += nwarp) {
+    const int j = kh * g.W + lane;
+    const uint32_t b = lane < g.W ? bsl[j] : 0u;
+    uint32_t incl = b;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    if (lane < g.W) {
+      sb_bits[j] = b;
+      sb_off[j] = pen[ks * g.H + kh] - wbase + incl - b;
+      const float sg = sig[j];
+      sb_gain[j] = gain_inv ? (b ? __frcp_rn(sg) : 0.f) : sg;
+    }
+  }
+}
+
+template <int HC, int WC, int MODE>
 __global__ void __launch_bounds__(kHwThreads) fdct_hw_kernel(const __grid_constant__ Geom g,
-                                                             const __grid_constant__ UnitList ul, int mode,
+                                                             const __grid_constant__ UnitList ul,
                                                              const float* __restrict__ Y, float* __restrict__ partial) {
   extern __shared__ __align__(16) unsigned char smem[];
-  const HwLayout L = hw_layout(g.HW, false);
+  const HwLayout L = hw_layout(g.HW, g.N, g.S, g.H, MODE == kStats ? kLayStats : kLayQuant);
   float2* tiles = reinterpret_cast<float2*>(smem + L.tile);
   float* thr = reinterpret_cast<float*>(smem + L.thr);
-  uint32_t* pen = reinterpret_cast<uint32_t*>(smem + L.meta_b);   // bit offset of every (k_s, k_h) pencil
+  uint32_t* pen = reinterpret_cast<uint32_t*>(smem + L.pen);   // bit offset of every (k_s, k_h) pencil
+  uint32_t* sb_bits = reinterpret_cast<uint32_t*>(smem + L.meta);  // this slab: bits of every bin
+  float* sb_gain = reinterpret_cast<float*>(smem + L.meta) + g.HW;   // 1/sigma of every bin
+  uint32_t* sb_off = reinterpret_cast<uint32_t*>(smem + L.off);      // bit offset in the slab's words
+  unsigned char* bsl = smem + L.bsl;                                   // bit widths of two slabs
+  float* sig2 = reinterpret_cast<float*>(smem + L.sig2);               // sigmas of two slabs
   float* energy = reinterpret_cast<float*>(smem + L.uni);
   uint32_t* sbuf = reinterpret_cast<uint32_t*>(smem + L.uni);
   uint32_t* carry = reinterpret_cast<uint32_t*>(smem + L.carry);
@@ -119,9 +209,9 @@ __global__ void __launch_bounds__(kHwThreads) fdct_hw_kernel(const __grid_consta
   const UnitDev& ud = ul.u[u];
   unsigned char* pay = ud.payload;
   uint32_t* words_out = reinterpret_cast<uint32_t*>(pay + g.off_codes);
-  const bool quant = mode == kQuant;
+  const bool quant = MODE == kQuant;
   uint32_t cstride = 0, stride_words = 0;
-  if (mode != kStats) {  // written by the allocation kernel
+  if (MODE != kStats) {  // written by the allocation kernel
     cstride = reinterpret_cast<const uint32_t*>(pay)[11];
     stride_words = cstride / 4;
   }
@@ -129,21 +219,27 @@ __global__ void __launch_bounds__(kHwThreads) fdct_hw_kernel(const __grid_consta
   const unsigned char* pay_b = pay + kHeaderBytes;
   const float* pay_sig = reinterpret_cast<const float*>(pay + g.off_sigma);
 
-  issue_tile(g, ysrc, 0, tiles);
+  // The unit's bit widths, needed once for the pencil offsets, go to the tile buffer that slab 0
+  // does not use; with a single buffer they go there first and slab 0 follows.
+  unsigned char* bstage = reinterpret_cast<unsigned char*>(tiles + (L.nbuf == 2 ? (size_t)g.HW * kPairs : 0));
+  if (!quant || L.nbuf == 2) issue_tile(g, ysrc, 0, tiles);
+  if (quant) {
+    issue_bits(g, pay_b, bstage);
+    issue_slab_bits(g, pay_b, 0, bsl);
+    issue_sigma(g, pay_sig, 0, sig2);
+  }
   cp_async_commit();
   if (quant) {
+    __shared__ unsigned int s_unused;
     for (int i = threadIdx.x; i < kLmThrTotal; i += blockDim.x) thr[i] = c_lm_thresholds[i];
     if (threadIdx.x < kChunk) carry[threadIdx.x] = 0;
-    // every pencil's first stream bit, once: bits of each (k_s, k_h) row, then a scan in bin order
-    const int npen = g.S * g.H;
-    for (int p = threadIdx.x; p < npen; p += blockDim.x) {
-      const unsigned char* b = pay_b + (size_t)p * g.W;
-      uint32_t t = 0;
-      for (int w = 0; w < g.W; ++w) t += b[w];
-      pen[p] = t;
-    }
+    cp_async_wait_all();
     __syncthreads();
-    block_exclusive_scan(pen, npen, swarp);
+    pencil_offsets(g, bstage, pen, swarp, &s_unused);   // widths come from the allocation: all <= 8
+    if (L.nbuf == 1) {  // every read of bstage is done
+      issue_tile(g, ysrc, 0, tiles);
+      cp_async_commit();
+    }
   }
   uint32_t P = 0;  // stream bits written so far, identical for every channel
   for (int ks = 0; ks < g.S; ++ks) {
@@ -151,10 +247,12 @@ __global__ void __launch_bounds__(kHwThreads) fdct_hw_kernel(const __grid_consta
     float2* tile = tiles + (size_t)cur * g.HW * kPairs;
     cp_async_wait_all();
     __syncthreads();  // slab ks is in place and every thread is done with slab ks - 1
-    if (L.nbuf == 2 && ks + 1 < g.S) {
-      issue_tile(g, ysrc, ks + 1, tiles + (size_t)(cur ^ 1) * g.HW * kPairs);
-      cp_async_commit();
+    if (L.nbuf == 2 && ks + 1 < g.S) issue_tile(g, ysrc, ks + 1, tiles + (size_t)(cur ^ 1) * g.HW * kPairs);
+    if (quant && ks + 1 < g.S) {
+      issue_slab_bits(g, pay_b, ks + 1, bsl + ((ks + 1) & 1) * L.bsl_stride);
+      issue_sigma(g, pay_sig, ks + 1, sig2 + ((ks + 1) & 1) * g.HW);
     }
+    if (ks + 1 < g.S && (L.nbuf == 2 || quant)) cp_async_commit();
     const uint32_t slab_end = quant ? (ks + 1 < g.S ? pen[(ks + 1) * g.H] : (uint32_t)0) : 0u;
     const uint32_t w0 = P >> 5;                 // first stream word this slab touches
     uint32_t slab_bits = 0;
@@ -165,23 +263,27 @@ __global__ void __launch_bounds__(kHwThreads) fdct_hw_kernel(const __grid_consta
         const int ch = i / nw, w = i - ch * nw;
         sbuf[ch * words + w] = w == 0 ? carry[ch] : 0u;
       }
+      slab_meta(g, ks, bsl + (ks & 1) * L.bsl_stride + (((size_t)ks * g.HW) & 15), sig2 + (ks & 1) * g.HW, pen,
+                w0 << 5, true, sb_bits, sb_gain, sb_off);
     }
     h_pass<HC, false>(g, tile);
     __syncthreads();
-    // W pass fused with the per-bin epilogue
+    // W pass fused with the per-bin epilogue.  Rows are dealt so that warp w takes k_h = w and
+    // k_h = H-1-w: the low-frequency rows, which carry most of the code bits, pair with light ones.
     for (int p = threadIdx.x; p < g.H * kPairs; p += blockDim.x) {
-      const int kh = p >> 4, pair = p & 15;
+      const int r = p >> 4, pair = p & 15;
+      const int kh = (r & 1) ? g.H - 1 - (r >> 1) : (r >> 1);
       const int base = kh * g.W * kPairs + pair;
       float2 x[WC];
 #pragma unroll
       for (int t = 0; t < WC; ++t)
         if (t < g.W) x[t] = tile[base + t * kPairs];
       dct_pencil<WC, false>(x, g.W);
-      if (mode == kStats) {
+      if (MODE == kStats) {
 #pragma unroll
         for (int t = 0; t < WC; ++t)
           if (t < g.W) energy[(kh * g.W + t) * kEnergyStride + pair] = x[t].x * x[t].x + x[t].y * x[t].y;
-      } else if (mode == kRaw) {
+      } else if (MODE == kRaw) {
         const int c = chunk * kChunk + 2 * pair;
         float* s0 = reinterpret_cast<float*>(pay + g.off_codes + (size_t)c * cstride) + ks * g.HW + kh * g.W;
         float* s1 = reinterpret_cast<float*>(pay + g.off_codes + (size_t)(c + 1) * cstride) + ks * g.HW + kh * g.W;
@@ -192,10 +294,10 @@ __global__ void __launch_bounds__(kHwThreads) fdct_hw_kernel(const __grid_consta
             s1[t] = x[t].y;
           }
       } else {
-        // codes of the pencil's W bins are contiguous in each channel stream: pack them in a
-        // 64-bit register and flush whole words into the slab's stream buffer
-        const int i0 = (ks * g.H + kh) * g.W;
-        const uint32_t o0 = pen[ks * g.H + kh] - (w0 << 5);
+        // the pencil's codes are contiguous in both channel streams: pack them in 64-bit
+        // registers and OR whole words into the slab's stream buffer
+        const int i0 = kh * g.W;
+        const uint32_t o0 = sb_off[i0];
         uint32_t* r0 = sbuf + (2 * pair) * words + (o0 >> 5);
         uint32_t* r1 = r0 + words;
         unsigned long long a0 = 0, a1 = 0;
@@ -203,11 +305,11 @@ __global__ void __launch_bounds__(kHwThreads) fdct_hw_kernel(const __grid_consta
 #pragma unroll
         for (int t = 0; t < WC; ++t) {
           if (t < g.W) {
-            const int bits = pay_b[i0 + t];
+            const int bits = (int)sb_bits[i0 + t];
             if (bits) {
-              const float inv = __frcp_rn(pay_sig[i0 + t]);
-              a0 |= (unsigned long long)lm_code(x[t].x * inv, bits, thr) << apos;
-              a1 |= (unsigned long long)lm_code(x[t].y * inv, bits, thr) << apos;
+              const float inv = sb_gain[i0 + t];
+              a0 |= (unsigned long long)quant_code(x[t].x * inv, bits, thr) << apos;
+              a1 |= (unsigned long long)quant_code(x[t].y * inv, bits, thr) << apos;
               apos += bits;
               if (apos >= 32) {
                 atomicOr(r0++, (uint32_t)a0);
@@ -219,14 +321,14 @@ __global__ void __launch_bounds__(kHwThreads) fdct_hw_kernel(const __grid_consta
             }
           }
         }
-        if (apos) {
+        if (a0 | a1) {
           atomicOr(r0, (uint32_t)a0);
           atomicOr(r1, (uint32_t)a1);
         }
       }
     }
     __syncthreads();
-    if (mode == kStats) {
+    if (MODE == kStats) {
       float* dst = partial + ((size_t)u * g.nch + chunk) * g.N + (size_t)ks * g.HW;
       for (int j = threadIdx.x; j < g.HW; j += blockDim.x) {
         const float* e = energy + j * kEnergyStride;
@@ -262,7 +364,7 @@ __global__ void __launch_bounds__(kHwThreads) fdct_hw_kernel(const __grid_consta
       const int ch = i / tail, w = i - ch * tail;
       words_out[(size_t)(chunk * kChunk + ch) * stride_words + wlast + w] = (w == 0) ? carry[ch] : 0u;
     }
-  } else if (mode == kRaw) {
+  } else if (MODE == kRaw) {
     const int pad = (int)cstride - 4 * g.N;
     for (int i = threadIdx.x; i < kChunk * pad; i += blockDim.x) {
       const int ch = i / pad, b = i - ch * pad;
@@ -272,24 +374,29 @@ __global__ void __launch_bounds__(kHwThreads) fdct_hw_kernel(const __grid_consta
 }
 
 // ----------------------------------------------------------------------------------- decode ---
-template <int HC, int WC>
+template <int HC, int WC, int MODE>
 __global__ void __launch_bounds__(kHwThreads) idct_hw_kernel(const __grid_constant__ Geom g,
-                                                             const __grid_constant__ UnitList ul, int mode,
+                                                             const __grid_constant__ UnitList ul,
                                                              float* __restrict__ V, unsigned int* status) {
   extern __shared__ __align__(16) unsigned char smem[];
-  const HwLayout L = hw_layout(g.HW, true);
+  const HwLayout L = hw_layout(g.HW, g.N, g.S, g.H, kLayDecode);
   float2* tile = reinterpret_cast<float2*>(smem + L.tile);
   float* lvs = reinterpret_cast<float*>(smem + L.lv);
-  uint32_t* pen = reinterpret_cast<uint32_t*>(smem + L.meta_b);   // first stream bit of every pencil
+  uint32_t* pen = reinterpret_cast<uint32_t*>(smem + L.pen);   // first stream bit of every pencil
   uint32_t* sbufs = reinterpret_cast<uint32_t*>(smem + L.uni);
   uint32_t* swarp = reinterpret_cast<uint32_t*>(smem + L.warp);
+  uint32_t* sb_bits = reinterpret_cast<uint32_t*>(smem + L.meta);  // this slab: bits of every bin
+  float* sb_gain = reinterpret_cast<float*>(smem + L.meta) + g.HW;   // sigma of every bin
+  uint32_t* sb_off = reinterpret_cast<uint32_t*>(smem + L.off);      // bit offset in the slab's words
+  unsigned char* bsl = smem + L.bsl;                                   // bit widths of two slabs
+  float* sig2 = reinterpret_cast<float*>(smem + L.sig2);               // sigmas of two slabs
   __shared__ int s_ok;
   __shared__ unsigned int s_bad;
   const int words = L.words;
   const int chunk = blockIdx.x, u = blockIdx.y;
   const UnitDev& ud = ul.u[u];
   const unsigned char* pay = ud.payload;
-  const bool raw = mode == kRaw;
+  const bool raw = MODE == kRaw;
   uint32_t code_bits = 0;
   if (threadIdx.x == 0) {
     // the header must describe exactly the unit the caller asked for
@@ -317,21 +424,17 @@ __global__ void __launch_bounds__(kHwThreads) idct_hw_kernel(const __grid_consta
   const uint32_t* streams = reinterpret_cast<const uint32_t*>(pay + g.off_codes);
   const unsigned char* pay_b = pay + kHeaderBytes;
   const float* pay_sig = reinterpret_cast<const float*>(pay + g.off_sigma);
-  const int npen = g.S * g.H;
-  // every pencil's first stream bit: bits of each (k_s, k_h) row, then a scan in bin order
+  // every pencil's first stream bit, from the unit's bit widths staged in the (still unused) tile
   if (ok0 && !raw) {
-    for (int p = threadIdx.x; p < npen; p += blockDim.x) {
-      const unsigned char* b = pay_b + (size_t)p * g.W;
-      uint32_t t = 0;
-      for (int w = 0; w < g.W; ++w) {
-        const uint32_t v = b[w];
-        if (v > 8) s_bad = 1;
-        t += v;
-      }
-      pen[p] = t;
-    }
+    unsigned char* bstage = reinterpret_cast<unsigned char*>(tile);
+    issue_bits(g, pay_b, bstage);
+    issue_slab_bits(g, pay_b, 0, bsl);
+    issue_sigma(g, pay_sig, 0, sig2);
+    cp_async_commit();
+    cp_async_wait_all();
     __syncthreads();
-    const uint32_t total = block_exclusive_scan(pen, npen, swarp);
+    const uint32_t total = pencil_offsets(g, bstage, pen, swarp, &s_bad);
+    __syncthreads();
     if (threadIdx.x == 0 && (total != code_bits || s_bad)) s_ok = 0;
   }
   __syncthreads();
@@ -365,42 +468,61 @@ __global__ void __launch_bounds__(kHwThreads) idct_hw_kernel(const __grid_consta
     __syncthreads();  // slab ks's stream words are in place; slab ks - 1 is done
     if (ok && !raw && ks + 1 < g.S) {
       issue_words(ks + 1, sbufs + (size_t)(mc ^ 1) * kChunk * words);
+      issue_slab_bits(g, pay_b, ks + 1, bsl + (mc ^ 1) * L.bsl_stride);
+      issue_sigma(g, pay_sig, ks + 1, sig2 + (mc ^ 1) * g.HW);
       cp_async_commit();
     }
     const int i0s = ks * g.HW;
     const uint32_t wbase = raw ? 0u : (slab_begin(ks) >> 5) << 5;
-    // inverse DCT along W from the dequantized coefficients
+    if (ok && !raw) {
+      slab_meta(g, ks, bsl + mc * L.bsl_stride + (((size_t)ks * g.HW) & 15), sig2 + mc * g.HW, pen, wbase, false,
+                sb_bits, sb_gain, sb_off);
+      __syncthreads();
+    }
+    // dequantize in registers, fused with the inverse DCT along W: a thread takes one pencil (a
+    // k_h row of W bins, two channels), whose codes are contiguous in both streams and are read
+    // through 64-bit windows; rows are dealt as in encoding (k_h = w with k_h = H-1-w)
     for (int p = threadIdx.x; p < g.H * kPairs; p += blockDim.x) {
-      const int kh = p >> 4, pair = p & 15;
+      const int r = p >> 4, pair = p & 15;
+      const int kh = (r & 1) ? g.H - 1 - (r >> 1) : (r >> 1);
       const int base = kh * g.W * kPairs + pair;
-      const int c = ch0 + 2 * pair;
-      const int i0 = i0s + kh * g.W;
+      const int i0 = kh * g.W;
       float2 x[WC];
       if (!ok) {
 #pragma unroll
         for (int t = 0; t < WC; ++t) x[t] = make_float2(0.f, 0.f);
       } else if (raw) {
         const float* st = reinterpret_cast<const float*>(streams);
+        const int c = ch0 + 2 * pair;
 #pragma unroll
         for (int t = 0; t < WC; ++t)
-          if (t < g.W) x[t] = make_float2(st[(size_t)c * stride_words + i0 + t], st[(size_t)(c + 1) * stride_words + i0 + t]);
+          if (t < g.W)
+            x[t] = make_float2(st[(size_t)c * stride_words + i0s + i0 + t], st[(size_t)(c + 1) * stride_words + i0s + i0 + t]);
       } else {
-        uint32_t o = pen[ks * g.H + kh] - wbase;
-        const uint32_t* r0 = sb + (2 * pair) * words;
-        const uint32_t* r1 = r0 + words;
+        const uint32_t* row0 = sb + (2 * pair) * words;
+        const uint32_t* row1 = row0 + words;
+        const uint32_t o0 = sb_off[i0];
+        uint32_t wi = o0 >> 5, pos = o0 & 31u;
+        unsigned long long w0v = (unsigned long long)row0[wi] | ((unsigned long long)row0[wi + 1] << 32);
+        unsigned long long w1v = (unsigned long long)row1[wi] | ((unsigned long long)row1[wi + 1] << 32);
 #pragma unroll
         for (int t = 0; t < WC; ++t) {
           if (t < g.W) {
-            const int bits = pay_b[i0 + t];
+            const int bits = (int)sb_bits[i0 + t];
             float2 v = make_float2(0.f, 0.f);
             if (bits) {
-              const uint32_t wi = o >> 5, sh = o & 31u, mask = (1u << bits) - 1u;
-              const uint32_t c0 = (uint32_t)(((((unsigned long long)r0[wi + 1]) << 32) | r0[wi]) >> sh) & mask;
-              const uint32_t c1 = (uint32_t)(((((unsigned long long)r1[wi + 1]) << 32) | r1[wi]) >> sh) & mask;
+              const uint32_t mask = (1u << bits) - 1u;
               const float* lv = lvs + lm_lv_offset(bits);
-              const float sg = pay_sig[i0 + t];
-              v = make_float2(sg * lv[c0], sg * lv[c1]);
-              o += bits;
+              const float sg = sb_gain[i0 + t];
+              v = make_float2(sg * lv[(uint32_t)(w0v >> pos) & mask], sg * lv[(uint32_t)(w1v >> pos) & mask]);
+              pos += bits;
+              if (pos >= 32) {
+                ++wi;
+                const bool in = wi + 1 < (uint32_t)words;
+                w0v = (w0v >> 32) | ((unsigned long long)(in ? row0[wi + 1] : 0u) << 32);
+                w1v = (w1v >> 32) | ((unsigned long long)(in ? row1[wi + 1] : 0u) << 32);
+                pos -= 32;
+              }
             }
             x[t] = v;
           }
@@ -429,16 +551,27 @@ __global__ void __launch_bounds__(kHwThreads) idct_hw_kernel(const __grid_consta
 cudaError_t TACTKV_LAUNCHER(TACTKV_HCLASS, TACTKV_WCLASS)(bool inverse, int mode, const Geom& g, const UnitList& ul,
                                                           int nu, float* buf, float* partial, unsigned int* status,
                                                           cudaStream_t st) {
-  const HwLayout L = hw_layout(g.HW, inverse);
+  const HwLayout L = hw_layout(g.HW, g.N, g.S, g.H, inverse ? kLayDecode : (mode == kStats ? kLayStats : kLayQuant));
   const dim3 grid(g.nch, nu);
+  constexpr int H = TACTKV_HCLASS, W = TACTKV_WCLASS;
+  const int sm = (int)L.total;
   if (inverse) {
-    cudaFuncSetAttribute(idct_hw_kernel<TACTKV_HCLASS, TACTKV_WCLASS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)L.total);
-    idct_hw_kernel<TACTKV_HCLASS, TACTKV_WCLASS><<<grid, kHwThreads, L.total, st>>>(g, ul, mode, buf, status);
+    if (mode == kRaw) {
+      cudaFuncSetAttribute(idct_hw_kernel<H, W, kRaw>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+      idct_hw_kernel<H, W, kRaw><<<grid, kHwThreads, sm, st>>>(g, ul, buf, status);
+    } else {
+      cudaFuncSetAttribute(idct_hw_kernel<H, W, kQuant>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+      idct_hw_kernel<H, W, kQuant><<<grid, kHwThreads, sm, st>>>(g, ul, buf, status);
+    }
+  } else if (mode == kStats) {
+    cudaFuncSetAttribute(fdct_hw_kernel<H, W, kStats>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    fdct_hw_kernel<H, W, kStats><<<grid, kHwThreads, sm, st>>>(g, ul, buf, partial);
+  } else if (mode == kRaw) {
+    cudaFuncSetAttribute(fdct_hw_kernel<H, W, kRaw>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    fdct_hw_kernel<H, W, kRaw><<<grid, kHwThreads, sm, st>>>(g, ul, buf, partial);
   } else {
-    cudaFuncSetAttribute(fdct_hw_kernel<TACTKV_HCLASS, TACTKV_WCLASS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)L.total);
-    fdct_hw_kernel<TACTKV_HCLASS, TACTKV_WCLASS><<<grid, kHwThreads, L.total, st>>>(g, ul, mode, buf, partial);
+    cudaFuncSetAttribute(fdct_hw_kernel<H, W, kQuant>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    fdct_hw_kernel<H, W, kQuant><<<grid, kHwThreads, sm, st>>>(g, ul, buf, partial);
   }
   return cudaGetLastError();
 }

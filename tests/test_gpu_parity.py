@@ -74,6 +74,16 @@ def test_small_shapes_bf16(shape, bits):
     assert all(r["recon_rel_rms"] <= 1e-3 for r in reports)
 
 
+@pytest.mark.parametrize("bits,flags", [(1, 0), (8, 0), (2, 1)])
+def test_maximum_grid(bits, flags):
+    """S = 64 slabs of a 32 x 32 grid (the largest unit the codec takes): the shared-memory
+    footprint of every kernel is at its largest here.  flags = 1 is TACTKV_NO_QUANT."""
+    S, H, W, heads, D = 64, 32, 32, 1, 32
+    x = make_unit(S, H, W, heads, D, rho=(0.95, 0.9, 0.9), nu=4.0, seed=7 + bits, device=DEV)[None]
+    reports, _, _ = _check_batch(x, S, H, W, bits, flags=flags)
+    assert reports[0]["recon_rel_rms"] <= (1e-5 if flags else 1e-3)
+
+
 def test_no_quant_round_trip_is_lossless():
     S, H, W, heads, D = 16, 8, 12, 2, 32
     x = torch.stack([make_unit(S, H, W, heads, D, rho=(0.9, 0.9, 0.9), nu=4.0, seed=i, device=DEV) for i in range(3)])
