@@ -131,6 +131,27 @@ def oracle_round_trip_seconds(x_np, w, bits, n_units=1):
     return time.perf_counter() - t
 
 
+# ---------------------------------------------------------------------- multi-rank host logic ---
+def rank_workload(w, rank: int):
+    """The batch rank `rank` compresses: same shape and size on every rank, independent seeds
+    (units are independent, so N ranks process N batches: weak scaling)."""
+    import dataclasses
+    return dataclasses.replace(w, seed=w.seed + 1000 * rank)
+
+
+def max_over_ranks(ms: float, dist, device) -> float:
+    """The slowest rank's time: every rank must call this (one all-reduce MAX)."""
+    import torch
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbs(world: int, bytes_per_rank: int, ms: float) -> float:
+    """Whole-job throughput: the bytes all ranks processed over the slowest rank's time."""
+    return world * bytes_per_rank / (ms * 1e-3) / 1e9
+
+
 # ---------------------------------------------------------------------------- reference arm ---
 def run_reference(args, w, bits, rank):
     """The base contract's reference arm for this codec: the CPU oracle on the host cores."""
@@ -202,7 +223,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     # every rank compresses its own batch (independent seeds per rank): weak scaling
-    wr = dataclasses.replace(w, seed=w.seed + 1000 * rank)
+    wr = rank_workload(w, rank)
     x = make_batch(wr, device=dev, units=list(range(args.units)) if args.units else None)
     U, Tk, heads, D = x.shape
     all_units = list(wr.units())
@@ -262,9 +283,7 @@ def main():
     clocks = sampler.stop() if sampler else None
     elapsed_ms = t0.elapsed_time(t1)
     if world > 1:
-        tt = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(tt.item())
+        elapsed_ms = max_over_ranks(elapsed_ms, dist, dev)
     ms_step = elapsed_ms / args.steps
 
     # per-kernel averages from the bracketing events
@@ -284,7 +303,7 @@ def main():
     alg_c = in_bytes + pay_bytes                     # read bf16 K/V, write payloads
     alg_d = pay_bytes + in_bytes                     # read payloads, write bf16 K/V
     peak, peak_kind = measured_peaks()
-    value = world * in_bytes / (ms_step * 1e-3) / 1e9
+    value = job_gbs(world, in_bytes, ms_step)
     if args.units:
         w = dataclasses.replace(w, sequences=1, layers=U, kv=(0,))   # describe what actually ran
     achieved = (alg_c + alg_d) / (ms_step * 1e-3) / 1e9
@@ -365,11 +384,9 @@ def e2e_run(args, T, x, payload, out, cu, du, ws, stream, world):
     torch.cuda.synchronize(dev)
     ms = a.elapsed_time(b) / args.e2e_steps
     if world > 1:
-        tt = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+        ms = max_over_ranks(ms, dist, dev)
     in_bytes = x.numel() * x.element_size()
-    return {"value": round(world * in_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+    return {"value": round(job_gbs(world, in_bytes, ms), 2), "unit": "GB/s",
             "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": payload.numel() + out.numel() * out.element_size(),
             "ms_per_step": round(ms, 3)}
 

@@ -1,0 +1,71 @@
+"""The oracle's pins catch plausible mistakes.
+
+Each case plants one mistake in a copy of the oracle, on the CPU:
+- a dropped normalisation factor;
+- a transposed operand;
+- a wrong tie order;
+- a wrong rounding;
+- a shifted bit;
+- ...
+
+It then runs the pin suite (tests/test_oracle.py) against that copy, which must fail. The real oracle
+is never modified. Together these show that the pins pin the oracle to the pages and the
+mathematics, not to itself.
+"""
+import os
+import shutil
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+# (name, text in oracle/tactkv_oracle.py, replacement)
+MUTATIONS = [
+    ("dct: a_k = sqrt(1/L) for every k", "math.sqrt(1.0 / L), math.sqrt(2.0 / L))",
+     "math.sqrt(1.0 / L), math.sqrt(1.0 / L))"),
+    ("dct: half-sample shift dropped", "np.cos(np.pi * (2.0 * t + 1.0) * k / (2.0 * L))",
+     "np.cos(np.pi * (2.0 * t) * k / (2.0 * L))"),
+    ("dct3: H-axis matrix transposed", 'np.einsum("kh,shwc->skwc", dct_matrix(H), y)',
+     'np.einsum("hk,shwc->skwc", dct_matrix(H), y)'),
+    ("variance: mean removed", "return np.mean(Xf * Xf, axis=1)",
+     "return np.var(Xf, axis=1)"),
+    # (rounding down instead of to nearest is NOT a mistake: the +-1 greedy reaches the same top-B
+    #  set from any rounding, so that change is equivalent and left out)
+    ("allocation: 8-bit cap ignored by the greedy", "cand = act & (b < MAX_BITS)", "cand = act"),
+    ("allocation: budget one bit short", "B = int(bits) * N\n    act", "B = int(bits) * N - 1\n    act"),
+    ("allocation: greedy adds the least valuable bit", "m = key.max()",
+     "m = key[np.isfinite(key)].min()"),
+    ("allocation: add-ties to the highest index", "i = idx[key == m].min()                     # ties -> lowest index",
+     "i = idx[key == m].max()"),
+    ("quantize: ties go down", 'np.asarray(u, dtype=np.float32), side="right")',
+     'np.asarray(u, dtype=np.float32), side="left")'),
+    ("pack: MSB-first bit order", "out[:, q >> 3] |= (bit << (q & 7)).astype(np.uint8)",
+     "out[:, q >> 3] |= (bit << (7 - (q & 7))).astype(np.uint8)"),
+    ("lloyd-max: thresholds not midpoints", "return y, 0.5 * (y[1:] + y[:-1])",
+     "return y, 0.45 * (y[1:] + y[:-1])"),
+]
+
+
+def _copy_tree(dst):
+    shutil.copytree(os.path.join(ROOT, "oracle"), os.path.join(dst, "oracle"))
+    os.makedirs(os.path.join(dst, "tests"))
+    for f in ("conftest.py", "test_oracle.py"):
+        shutil.copy(os.path.join(ROOT, "tests", f), os.path.join(dst, "tests", f))
+    shutil.copytree(os.path.join(ROOT, "tests", "golden"), os.path.join(dst, "tests", "golden"))
+    shutil.copytree(os.path.join(ROOT, "dct_transform_coding_b200"), os.path.join(dst, "dct_transform_coding_b200"),
+                    ignore=shutil.ignore_patterns("*.so", "_build", "csrc", "__pycache__"))
+    shutil.copy(os.path.join(ROOT, "pytest.ini"), os.path.join(dst, "pytest.ini"))
+
+
+@pytest.mark.parametrize("name,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_planted_mistake_fails_a_pin(tmp_path, name, old, new):
+    _copy_tree(str(tmp_path))
+    path = tmp_path / "oracle" / "tactkv_oracle.py"
+    src = path.read_text()
+    assert src.count(old) >= 1, f"mutation anchor not found: {old}"
+    path.write_text(src.replace(old, new, 1))
+    r = subprocess.run([sys.executable, "-m", "pytest", "tests/test_oracle.py", "-x", "-q", "-m", "not gpu",
+                        "-p", "no:cacheprovider"], cwd=str(tmp_path), capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"no pin caught the planted mistake '{name}':\n{r.stdout[-2000:]}"
