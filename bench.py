@@ -332,13 +332,13 @@ def main():
         "decompress_gbs": round(in_bytes / (ms_d * 1e-3) / 1e9, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "kernel": "compress+decompress step (7 kernels per wave)",
+                     "kernel": "compress+decompress step (8 kernels per wave)",
                      "algorithmic_bytes_per_step": alg_c + alg_d, "peak_kind": peak_kind,
                      "compress_frac": round(alg_c / (ms_c * 1e-3) / 1e9 / peak, 4),
                      "decompress_frac": round(alg_d / (ms_d * 1e-3) / 1e9 / peak, 4),
                      "dominant_kernel": dominant},
         "kernels": kernels,
-        "gpu_launches": 7 * waves * args.steps,
+        "gpu_launches": 8 * waves * args.steps,
         "clocks": clocks,
     }
 

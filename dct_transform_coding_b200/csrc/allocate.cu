@@ -13,6 +13,11 @@
 //     (monotone in value), ~62 steps of one block-wide count;
 //   * keys equal to that value are handed out in bin order until the budget is met.
 // If the active bins cannot absorb B (8 * #active <= B) every active bin gets 8 bits.
+//
+// The kernel also writes the first stream bit P(k_s) of every S slab (the same for every
+// channel) into the workspace and zeroes the stream word holding each P(k_s): the packing kernel
+// ORs the words it shares with a neighbouring slab range into those.  decode_index_kernel
+// rebuilds P from a payload before decoding and checks the header and the bit widths.
 #include "common.cuh"
 
 namespace tactkv {
@@ -79,13 +84,34 @@ __global__ void __launch_bounds__(256) reduce_var_kernel(const __grid_constant__
   var_ws[(size_t)u * g.N + i] = acc / (double)g.n;
 }
 
+// Exclusive scan of s_slab[0..S) into out[0..S] (out[S] = total), by one warp.
+__device__ void slab_scan(const uint32_t* s_slab, int S, uint32_t* out) {
+  const int lane = threadIdx.x & 31;
+  uint32_t run = 0;
+  for (int k0 = 0; k0 < S; k0 += 32) {
+    const uint32_t v = k0 + lane < S ? s_slab[k0 + lane] : 0u;
+    uint32_t incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    if (k0 + lane < S) out[k0 + lane] = run + incl - v;
+    run += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) out[S] = run;
+}
+
 __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_constant__ Geom g,
                                                                  const __grid_constant__ UnitList ul,
-                                                                 double* __restrict__ var_ws, bool var_in_smem) {
+                                                                 double* __restrict__ var_ws, bool var_in_smem,
+                                                                 uint32_t* __restrict__ slab_off) {
   __shared__ long long s_ll[32];
   __shared__ double s_d[32];
   __shared__ uint32_t s_scan[33];
   __shared__ uint32_t s_cnt[kAllocThreads];
+  __shared__ uint32_t s_slab[kMaxSlabs];
+  __shared__ uint32_t s_P[kMaxSlabs + 1];
   extern __shared__ __align__(16) unsigned char smem_var[];
   const int u = blockIdx.x;
   const UnitDev& ud = ul.u[u];
@@ -151,6 +177,10 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
   block_exclusive_scan(s_cnt, blockDim.x, s_scan);
   long long rank = s_cnt[threadIdx.x];
   long long code_bits_local = 0;
+  for (int k = threadIdx.x; k < g.S; k += blockDim.x) s_slab[k] = 0;
+  __syncthreads();
+  int ks = beg / g.HW, in_slab = beg - ks * g.HW;   // slab of bin i, walked incrementally
+  uint32_t slab_sum = 0;
   for (int i = beg; i < end; ++i) {
     const double x = var[i];
     int b = 0;
@@ -168,13 +198,35 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
     pay[kHeaderBytes + i] = (unsigned char)b;
     reinterpret_cast<float*>(pay + g.off_sigma)[i] = (float)sqrt(x);
     code_bits_local += b;
+    slab_sum += b;
+    if (++in_slab == g.HW || i + 1 == end) {
+      if (slab_sum) atomicAdd(&s_slab[ks], slab_sum);
+      slab_sum = 0;
+      in_slab = 0;
+      ++ks;
+    }
   }
   // zero padding after the b[] and sigma[] arrays
   for (int i = kHeaderBytes + g.N + threadIdx.x; i < g.off_sigma; i += blockDim.x) pay[i] = 0;
   for (int i = g.off_sigma + 4 * g.N + threadIdx.x; i < g.off_codes; i += blockDim.x) pay[i] = 0;
   const long long code_bits = raw ? 32LL * g.N : block_sum<long long>(code_bits_local, s_ll);
+  const long long cstride = pad16((code_bits + 7) / 8);
+  // slab offsets P(k_s), and a zero in the stream word at every P(k_s) of every channel
+  __syncthreads();
+  if (threadIdx.x < 32) slab_scan(s_slab, g.S, s_P);
+  __syncthreads();
+  uint32_t* P = slab_off + (size_t)u * (g.S + 2);
+  for (int k = threadIdx.x; k <= g.S; k += blockDim.x) P[k] = raw ? 0u : s_P[k];
+  if (!raw) {
+    const uint32_t sw = (uint32_t)(cstride / 4);
+    uint32_t* words = reinterpret_cast<uint32_t*>(pay + g.off_codes);
+    for (int k = 0; k <= g.S; ++k) {
+      const uint32_t w = s_P[k] >> 5;
+      if (w < sw)
+        for (int c = threadIdx.x; c < g.n; c += blockDim.x) words[(size_t)c * sw + w] = 0u;
+    }
+  }
   if (threadIdx.x == 0) {
-    const long long cstride = pad16((code_bits + 7) / 8);
     uint32_t* h32 = reinterpret_cast<uint32_t*>(pay);
     int32_t* i32 = reinterpret_cast<int32_t*>(pay);
     h32[0] = kMagic;
@@ -196,15 +248,81 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
   }
 }
 
+// ----------------------------------------------------------------------------- decode index ---
+// One CTA per unit: the header must describe exactly the unit the caller asked for, every bit
+// width must be <= 8 and their sum must equal the header's code_bits; then P(k_s) is rebuilt.
+__global__ void __launch_bounds__(256) decode_index_kernel(const __grid_constant__ Geom g,
+                                                           const __grid_constant__ UnitList ul,
+                                                           uint32_t* __restrict__ slab_off, unsigned int* status) {
+  __shared__ int s_ok;
+  __shared__ uint32_t s_slab[kMaxSlabs];
+  __shared__ uint32_t s_P[kMaxSlabs + 1];
+  const int u = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const UnitDev& ud = ul.u[u];
+  const unsigned char* pay = ud.payload;
+  const bool raw = g.flags & TACTKV_NO_QUANT;
+  if (threadIdx.x == 0) {
+    const uint32_t* h32 = reinterpret_cast<const uint32_t*>(pay);
+    const int32_t* i32 = reinterpret_cast<const int32_t*>(pay);
+    const uint32_t ver_flags = h32[1], cb = h32[10], cs = h32[11];
+    const unsigned long long total = *reinterpret_cast<const unsigned long long*>(pay + 48);
+    bool ok = h32[0] == kMagic && (ver_flags & 0xffffu) == (uint32_t)kVersion &&
+              ((ver_flags >> 16) & TACTKV_NO_QUANT) == (raw ? TACTKV_NO_QUANT : 0u) && i32[2] == ud.layer &&
+              i32[3] == ud.kv && i32[4] == g.S && i32[5] == g.H && i32[6] == g.W && i32[7] == g.heads &&
+              i32[8] == g.head_dim && i32[9] == g.bits;
+    if (ok) {
+      ok = (raw ? cb == 32u * (uint32_t)g.N : cb <= (uint32_t)g.bits * (uint32_t)g.N) &&
+           (long long)cs == pad16(((long long)cb + 7) / 8) &&
+           (long long)total == (long long)g.off_codes + (long long)g.n * cs && (long long)total <= g.capacity;
+    }
+    s_ok = ok;
+  }
+  __syncthreads();
+  bool ok = s_ok;
+  if (ok && !raw) {
+    const unsigned char* b = pay + kHeaderBytes;
+    bool bad = false;
+    for (int k = warp; k < g.S; k += nwarps) {
+      uint32_t sum = 0;
+      for (int i = lane; i < g.HW; i += 32) {
+        const uint32_t v = b[(size_t)k * g.HW + i];
+        bad |= v > 8;
+        sum += v;
+      }
+      sum = __reduce_add_sync(0xffffffffu, sum);
+      if (lane == 0) s_slab[k] = sum;
+    }
+    if (bad) s_ok = 0;
+    __syncthreads();
+    if (warp == 0) slab_scan(s_slab, g.S, s_P);
+    __syncthreads();
+    if (threadIdx.x == 0 && s_P[g.S] != reinterpret_cast<const uint32_t*>(pay)[10]) s_ok = 0;
+    __syncthreads();
+    ok = s_ok;
+  }
+  uint32_t* P = slab_off + (size_t)u * (g.S + 2);
+  for (int k = threadIdx.x; k <= g.S; k += blockDim.x) P[k] = (ok && !raw) ? s_P[k] : 0u;
+  if (threadIdx.x == 0) {
+    P[g.S + 1] = ok ? 1u : 0u;
+    if (!ok) set_status(status, TACTKV_CORRUPT_PAYLOAD);
+  }
+}
+
 }  // namespace
 
+cudaError_t launch_decode_index(const Geom& g, const UnitList& ul, int nu, uint32_t* slab_off, unsigned int* status,
+                                cudaStream_t st) {
+  decode_index_kernel<<<nu, 256, 0, st>>>(g, ul, slab_off, status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_allocate(const Geom& g, const UnitList& ul, int nu, const float* partial, double* var,
-                            cudaStream_t st) {
+                            uint32_t* slab_off, cudaStream_t st) {
   const size_t var_bytes = (size_t)g.N * sizeof(double);
   const bool in_smem = var_bytes <= kAllocSmemVar;
   if (in_smem) cudaFuncSetAttribute(allocate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)var_bytes);
   reduce_var_kernel<<<dim3((g.N + 255) / 256, nu), 256, 0, st>>>(g, partial, var);
-  allocate_kernel<<<nu, kAllocThreads, in_smem ? var_bytes : 0, st>>>(g, ul, var, in_smem);
+  allocate_kernel<<<nu, kAllocThreads, in_smem ? var_bytes : 0, st>>>(g, ul, var, in_smem, slab_off);
   return cudaGetLastError();
 }
 

@@ -1,19 +1,32 @@
 // DCT along the H and W axes plus the per-bin epilogues (TACT-KV stages 2-4 and their inverse).
 //
-// One CTA owns one (unit, 32-channel chunk) and walks the S frequency slabs k_s in order.  Per
-// slab it stages the H*W x 32 coefficients in shared memory (16 channel pairs per row), runs
-// the pencil DCTs along H and then along W, and finishes with one of:
-//   kStats  per-bin energy sum_c X^2 over its 32 channels -> partial[u][chunk][bin] (pass 1)
-//   kQuant  u = X / sigma_i, Lloyd-Max code at b_i bits, packed into the 32 channel streams
-//   kRaw    float32 coefficients into the streams (TACTKV_NO_QUANT)
-// Because a CTA owns its channels' streams from the first bit to the last, each output word is
-// assembled in shared memory and stored exactly once; the word that straddles two slabs is
-// carried to the next slab.  The next slab's coefficients are fetched with cp.async into a
-// second buffer while the current one is transformed (when two buffers fit in shared memory).
+// A CTA owns one (unit, 32-channel chunk, range of S slabs) and walks its slabs in order.  Lane l
+// of every warp is channel l of the chunk, and a thread's float2 holds two pencils of that
+// channel: two columns (w, w+1) in the pass along H, two rows (h, h+1) in the pass along W.  All
+// lanes of a warp therefore work on the same frequency bins at the same time, and everything that
+// depends on a bin (its bit width, its gain, where its code goes in the stream) is uniform across
+// the warp: no lane waits for another lane's branch.
 //
-// Both directions first compute the stream offset of every (k_s, k_h) pencil from the bit
-// allocation, so no per-slab scan is needed; decoding (idct_hw) prefetches the stream words of
-// slab k_s+1 while slab k_s is dequantized and put through the inverse DCTs along W and H.
+// Forward, per slab k_s:
+//   1. the slab's H*W x 32 coefficients of the S-transformed volume Y arrive by cp.async, and the
+//      next slab's coefficients, bit widths and gains are fetched meanwhile;
+//   2. DCT along H in place: a warp reads a column pair, transforms it and writes it back into the
+//      same bytes as row pairs (float2 = rows 2i, 2i+1 of one column and channel);
+//   3. DCT along W: warp j takes row pair j, then
+//        kStats  squares, sums over the 32 channels -> partial[u][chunk][bin]   (pass 1)
+//        kQuant  u = X * (1/sigma_i), Lloyd-Max code at b_i bits, appended to the channel's stream
+//        kRaw    float32 coefficients into the streams (TACTKV_NO_QUANT)
+// A channel's codes of slab k_s occupy stream bits [P(k_s), P(k_s+1)) (the allocation writes P);
+// a warp finds its rows' offsets by summing the slab's bit widths before them.  Words are
+// assembled in shared memory and complete words are stored once; the word that straddles two
+// slabs is carried to the next slab.  The first and the last word of the CTA's slab range may
+// hold bits of the neighbouring ranges and are ORed into the payload atomically (the allocation
+// zeroes the word at every P(k_s) first).
+//
+// Inverse (idct_hw), per slab: the slab's stream words arrive by cp.async (next slab prefetched);
+// warp j decodes rows 2j and 2j+1 (unpack + dequantize in registers), runs the inverse DCT along W
+// and writes column pairs; warp j then runs the inverse DCT along H on column pair j and stores
+// the result into the fp32 volume V.
 //
 // Compiled once per pair of length classes (TACTKV_HCLASS, TACTKV_WCLASS: 16 or 32 each).
 #include "common.cuh"
@@ -27,518 +40,540 @@ namespace tactkv {
 namespace {
 
 constexpr size_t kSmemBudget = 220 * 1024;
-constexpr int kEnergyStride = kPairs + 1;   // padded row of per-pair energies: conflict-free both ways
-constexpr int kMaxSlabs = 64;
-
-__host__ __device__ inline int stream_words_per_slab(int HW) { return (8 * HW + 31) / 32 + 2; }
-
-struct HwLayout {
-  size_t tile, thr, lv, pen, meta, off, uni, carry, warp, bsl, sig2, total;
-  size_t bsl_stride;
-  int nbuf;
-  int words;
-};
 
 enum LayoutKind { kLayStats = 0, kLayQuant = 1, kLayDecode = 2 };
 
-// Shared memory carve-up of one launch.  stats: slab tiles and padded energy rows; quant: slab
-// tiles, thresholds, pencil offsets, per-bin metadata, the bit widths and sigmas of two slabs
-// and the stream words of a slab; decode: one tile, levels, the same metadata and two slabs of
-// stream words.  Regions a kind does not use have size 0.
-__host__ __device__ inline HwLayout hw_layout(int HW, int N, int S, int H, int kind) {
+struct HwLayout {
+  size_t tile, tile_bytes, sbuf, meta, bsl, bsl_stride, sig, thr, qcell, lv, carry, total;
+  int nbuf, words;
+};
+
+__host__ __device__ inline int row_pairs(int L) { return (L + 1) >> 1; }
+
+// One warp per column pair (pass along H) and per row pair (pass along W), at most 8 warps; with
+// more pairs than warps, a warp takes several in turn.
+constexpr int kMaxHwThreads = 256;
+__host__ __device__ inline int hw_threads(int H, int W) {
+  const int HP = row_pairs(H), WP = row_pairs(W), m = 32 * (HP > WP ? HP : WP);
+  return m < kMaxHwThreads ? m : kMaxHwThreads;
+}
+
+// Thresholds of width b padded with two +inf, stored for b = 1, 2, ... in turn.
+__device__ __forceinline__ int thr_pad_offset(int b) { return (1 << b) + b - 3; }
+
+// Shared memory of one launch.  A tile buffer holds a slab as cells of 32 floats on a grid of
+// 2*ceil(H/2) rows of Wp = 2*ceil(W/2) cells (the padding row and column are never read), which
+// also holds its row-pair (forward) or column-pair (inverse) rearrangement.  stats: the slab
+// tiles only (the energies reuse the rearranged tile).  quant: tiles, one
+// slab of stream words, per-bin records, bit widths and sigmas of two slabs, padded thresholds,
+// code table, carried words.  decode: one tile, two slabs of stream words, records, widths and
+// sigmas of two slabs, levels.  words (the stride of a channel's word row) is odd, so the 32 lanes
+// writing 32 channels' rows hit 32 different banks.
+__host__ __device__ inline HwLayout hw_layout(int H, int W, int kind) {
   HwLayout L;
-  L.words = stream_words_per_slab(HW);
+  const int HP = row_pairs(H), WP = row_pairs(W), HW = H * W;
   const bool st = kind == kLayStats, qu = kind == kLayQuant, de = kind == kLayDecode;
-  const size_t tile1 = (size_t)HW * kPairs * 8;
-  const size_t energy = st ? (size_t)HW * kEnergyStride * 4 : 0;
-  const size_t words = st ? 0 : (size_t)kChunk * L.words * 4 * (de ? 2 : 1);
-  const size_t thr = qu ? kLmThrTotal * 4 : 0, lv = de ? kLmLvTotal * 4 : 0;
-  const size_t pen = st ? 0 : ((size_t)S * H * 4 + 15) / 16 * 16;
-  const size_t meta = st ? 0 : (size_t)HW * 8, off = st ? 0 : ((size_t)HW * 4 + 15) / 16 * 16;
-  // a slab's bit widths are fetched as the 16-byte aligned window around them
+  L.tile_bytes = (size_t)(2 * HP) * (2 * WP) * 32 * 4;
+  L.words = ((8 * HW + 31) / 32 + 3) | 1;
+  const size_t words = st ? 0 : (size_t)32 * L.words * 4 * (de ? 2 : 1);
+  const size_t meta = st ? 0 : (size_t)HP * W * 16;
   L.bsl_stride = ((size_t)HW + 15) / 16 * 16 + 32;
-  const size_t bsl = st ? 0 : 2 * L.bsl_stride, sig2 = st ? 0 : (size_t)HW * 8;
-  const size_t fixed = thr + lv + pen + meta + off + energy + words + kChunk * 4 + 33 * 4 + bsl + sig2 + 256;
-  L.nbuf = (de || 2 * tile1 + fixed > kSmemBudget) ? 1 : 2;
+  const size_t bsl = st ? 0 : 2 * L.bsl_stride;
+  const size_t sig = st ? 0 : (size_t)2 * HW * 4;
+  const size_t thr = qu ? TACTKV_THR_PAD_TOTAL * 4 : 0;
+  const size_t qcell = qu ? ((size_t)6 * TACTKV_Q_CELLS + 15) / 16 * 16 : 0;
+  const size_t lv = de ? kLmLvTotal * 4 : 0;
+  const size_t carry = qu ? kChunk * 4 : 0;
+  const size_t rest = words + meta + bsl + sig + thr + qcell + lv + carry + 256;
+  L.nbuf = (de || 2 * L.tile_bytes + rest > kSmemBudget) ? 1 : 2;
+  // every region starts on a 16-byte boundary (cp.async of 16 bytes, 16-byte record loads)
+  auto p16 = [](size_t x) { return (x + 15) / 16 * 16; };
   size_t o = 0;
-  L.tile = o; o += tile1 * L.nbuf;
-  L.uni = o; o += ((energy > words ? energy : words) + 15) / 16 * 16;
-  L.bsl = o; o += bsl;
-  L.thr = o; o += thr;
-  L.lv = o; o += lv;
-  L.pen = o; o += pen;
-  L.meta = o; o += meta;
-  L.off = o; o += off;
-  L.sig2 = o; o += sig2;
-  L.carry = o; o += kChunk * 4;
-  L.warp = o; o += 33 * 4;
+  L.tile = o; o += p16(L.tile_bytes * L.nbuf);
+  L.sbuf = o; o += p16(words);
+  L.meta = o; o += p16(meta);
+  L.sig = o; o += p16(sig);
+  L.thr = o; o += p16(thr);
+  L.lv = o; o += p16(lv);
+  L.carry = o; o += p16(carry);
+  L.bsl = o; o += p16(bsl);
+  L.qcell = o; o += p16(qcell);
   L.total = o;
   return L;
 }
 
-// Lloyd-Max code: the number of thresholds t_j <= u (bisection over the 2^b - 1 thresholds).
-__device__ __forceinline__ uint32_t lm_code(float u, int bits, const float* thr) {
-  const float* t = thr + lm_thr_offset(bits);
-  uint32_t code = 0;
-  for (int step = 1 << (bits - 1); step > 0; step >>= 1)
-    if (u >= t[code + step - 1]) code += step;
+
+// Grid sizes of a launch.  HX, WX > 0 are exact lengths fixed at compile time (the common grids
+// get their own kernels: straight-line transforms, no bounds tests); 0 takes them from the Geom.
+template <int HX, int WX>
+struct Dims {
+  static constexpr int hx = HX, wx = WX;
+  int H, W, HW, n;
+  __device__ __forceinline__ explicit Dims(const Geom& g)
+      : H(HX ? HX : g.H), W(WX ? WX : g.W), HW((HX ? HX : g.H) * (WX ? WX : g.W)), n(g.n) {}
+};
+
+// Pencil transform of length L (= EXACT when EXACT > 0) from length class CLASS.
+template <int CLASS, int EXACT, bool INV, class V>
+__device__ __forceinline__ void pencil(V* x, int L) {
+  if constexpr (EXACT > 0) dct_exact<EXACT, INV>(x);
+  else dct_pencil<CLASS, INV>(x, L);
+}
+
+// Code of u at b bits: the number of thresholds t_j <= u (float32 compares, ties go up).  b = 1:
+// the sign test; b = 2: three compares against {-t, 0, t}; b >= 3: the cell of u in a uniform grid
+// gives the count c of thresholds below the cell, and two compares finish it (a cell holds at most
+// two thresholds; the thresholds are padded with +inf).
+__device__ __forceinline__ uint32_t quant_code(float u, int b, const float* thr, const unsigned char* qcell) {
+  if (b == 1) return u >= 0.f;
+  if (b == 2) {
+    const float t = thr[thr_pad_offset(2) + 2];
+    return (uint32_t)(u >= -t) + (uint32_t)(u >= 0.f) + (uint32_t)(u >= t);
+  }
+  int j = __float2int_rd(fmaf(u, TACTKV_Q_SCALE, TACTKV_Q_OFFSET));
+  j = min(max(j, 0), TACTKV_Q_CELLS - 1);
+  const uint32_t c = qcell[(b - 3) * TACTKV_Q_CELLS + j];
+  const float* t = thr + thr_pad_offset(b) + c;
+  return c + (uint32_t)(u >= t[0]) + (uint32_t)(u >= t[1]);
+}
+
+// Append a b-bit code (b >= 1) at stream position p of a channel's word row; full words are ORed
+// into shared memory (a word may be shared with the neighbouring row, which another warp fills).
+__device__ __forceinline__ void put_code(uint32_t& acc, uint32_t& p, uint32_t code, int b, uint32_t* row) {
+  const uint32_t s = p & 31u;
+  acc |= code << s;
+  if (s + b >= 32) {          // b <= 8, so s >= 24 here and the shift below is 1..8
+    atomicOr(row + (p >> 5), acc);
+    acc = code >> (32 - s);
+  }
+  p += b;
+}
+
+// Read a b-bit code (b >= 1) at the reader's position and advance (64-bit window lo:hi).
+__device__ __forceinline__ uint32_t get_code(uint32_t& lo, uint32_t& hi, uint32_t& s, uint32_t& wi, int b,
+                                             const uint32_t* row) {
+  const uint32_t code = __funnelshift_r(lo, hi, s) & ((1u << b) - 1u);
+  s += b;
+  if (s >= 32) {
+    s -= 32;
+    lo = hi;
+    ++wi;
+    hi = row[wi + 1];
+  }
   return code;
 }
 
-// Code for u at 1, 2 or more bits (the count of thresholds t <= u).  The 1- and 2-bit codebooks
-// have thresholds {0} and {-t, 0, t}: a sign test and three compares; wider ones use bisection.
-__device__ __forceinline__ uint32_t quant_code(float u, int bits, const float* thr) {
-  if (bits == 1) return u >= 0.f;
-  if (bits == 2) {
-    const float t = thr[lm_thr_offset(2) + 2];
-    return (uint32_t)(u >= -t) + (uint32_t)(u >= 0.f) + (uint32_t)(u >= t);
-  }
-  return lm_code(u, bits, thr);
+// Copy one S slab of Y (H*W cells of 32 channels, 128 bytes each) into a tile with rows of Wp
+// cells, asynchronously.
+template <class D>
+__device__ __forceinline__ void issue_tile(const D& g, const float* slab_src, float* tile) {
+  const int Wp = 2 * row_pairs(g.W);
+  for (int r = threadIdx.x >> 3; r < g.H; r += blockDim.x >> 3)      // blockDim.x is a multiple of 32
+    for (int w = 0; w < g.W; ++w)
+      cp_async16(tile + (r * Wp + w) * 32 + (threadIdx.x & 7) * 4,
+                 slab_src + (size_t)(r * g.W + w) * g.n + (threadIdx.x & 7) * 4);
 }
-
-// Pencil DCTs along H of the tile: pencils (w, pair), stride W*16 between elements.
-template <int CLASS, bool INV>
-__device__ __forceinline__ void h_pass(const Geom& g, float2* tile) {
-  const int step = g.W * kPairs;
-  for (int p = threadIdx.x; p < g.W * kPairs; p += blockDim.x) {
-    const int base = (p >> 4) * kPairs + (p & 15);
-    float2 x[CLASS];
-#pragma unroll
-    for (int t = 0; t < CLASS; ++t)
-      if (t < g.H) x[t] = tile[base + t * step];
-    dct_pencil<CLASS, INV>(x, g.H);
-#pragma unroll
-    for (int t = 0; t < CLASS; ++t)
-      if (t < g.H) tile[base + t * step] = x[t];
-  }
-}
-
-// Copy one S slab of Y (HW rows of 32 channels, 128 bytes each) into a tile, asynchronously.
-__device__ __forceinline__ void issue_tile(const Geom& g, const float4* ysrc_unit, int ks, float2* tile) {
-  const int rowq = g.n / 4;
-  const float4* src = ysrc_unit + (size_t)ks * g.HW * rowq;
-  float4* dst = reinterpret_cast<float4*>(tile);
-  for (int i = threadIdx.x; i < g.HW * (kChunk / 4); i += blockDim.x)
-    cp_async16(dst + i, src + (size_t)(i >> 3) * rowq + (i & 7));
-}
-
-// The unit's bit widths into shared memory (16-byte copies: the payload and its b[] array are
-// 16-byte aligned and padded), used once to compute the pencil offsets.
-__device__ __forceinline__ void issue_bits(const Geom& g, const unsigned char* pay_b, unsigned char* dst) {
-  for (int i = threadIdx.x; i < (g.N + 15) / 16; i += blockDim.x) cp_async16(dst + 16 * i, pay_b + 16 * i);
-}
-// The bit widths of slab ks as the 16-byte aligned window that holds them; they start at byte
-// (ks * HW) % 16 of dst.  The window ends inside the padded b[] array.
-__device__ __forceinline__ void issue_slab_bits(const Geom& g, const unsigned char* pay_b, int ks, unsigned char* dst) {
+// The bit widths of slab ks as the 16-byte aligned window around them (the payload and its b[]
+// array are 16-byte aligned and padded); they start at byte (ks * HW) % 16 of dst.
+template <class D>
+__device__ __forceinline__ void issue_slab_bits(const D& g, const unsigned char* pay_b, int ks, unsigned char* dst) {
   const size_t a0 = (size_t)ks * g.HW, q0 = a0 / 16, q1 = (a0 + g.HW + 15) / 16;
   for (int i = threadIdx.x; i < (int)(q1 - q0); i += blockDim.x) cp_async16(dst + 16 * i, pay_b + 16 * (q0 + i));
 }
-// The sigmas of slab ks (4-byte copies).
-__device__ __forceinline__ void issue_sigma(const Geom& g, const float* pay_sig, int ks, float* dst) {
+template <class D>
+__device__ __forceinline__ void issue_sigma(const D& g, const float* pay_sig, int ks, float* dst) {
   for (int j = threadIdx.x; j < g.HW; j += blockDim.x) cp_async4(dst + j, pay_sig + (size_t)ks * g.HW + j);
 }
 
-// Stream bit offset of every (k_s, k_h) pencil: the bits of each row of W bins, then an exclusive
-// scan in bin order.  bfull: the unit's bit widths in shared memory.  Returns the total; sets
-// *bad when a width exceeds 8.
-__device__ __forceinline__ uint32_t pencil_offsets(const Geom& g, const unsigned char* bfull, uint32_t* pen,
-                                                   uint32_t* swarp, unsigned int* bad) {
-  const int npen = g.S * g.H;
-  for (int p = threadIdx.x; p < npen; p += blockDim.x) {
-    const unsigned char* b = bfull + (size_t)p * g.W;
-    uint32_t t = 0;
-    bool over = false;
-    for (int w = 0; w < g.W; ++w) {
-      const uint32_t v = b[w];
-      over |= v > 8;
-      t += v;
+// Per-bin records of slab ks, one 16-byte record per (row pair, w): {gain of row 2i, gain of row
+// 2i+1, bits of row 2i | bits of row 2i+1 << 8}.  gain = 1/sigma (encoding) or sigma (decoding);
+// rows past H (odd H) get 0 bits.
+template <class D>
+__device__ __forceinline__ void slab_records(const D& g, const unsigned char* bs, const float* sig, bool inv,
+                                             unsigned char* meta) {
+  const int lane = threadIdx.x & 31, nwarps = blockDim.x >> 5, HP2 = 2 * row_pairs(g.H);
+  for (int kh = threadIdx.x >> 5; kh < HP2; kh += nwarps)
+    for (int t = lane; t < g.W; t += 32) {
+      const int i = kh * g.W + t;
+      const uint32_t b = kh < g.H ? bs[i] : 0u;
+      float gv = 0.f;
+      if (b) gv = inv ? __frcp_rn(sig[i]) : sig[i];
+      unsigned char* rec = meta + ((size_t)(kh >> 1) * g.W + t) * 16;
+      reinterpret_cast<float*>(rec)[kh & 1] = gv;
+      rec[8 + (kh & 1)] = (unsigned char)b;
     }
-    if (over) *bad = 1;
-    pen[p] = t;
-  }
-  __syncthreads();
-  return block_exclusive_scan(pen, npen, swarp);
 }
 
-// Bits, gain and stream bit offset of every bin of slab ks: one warp per (k_s, k_h) row of at most
-// 32 bins, the offset being the row's start (pen) plus a shuffle scan of the row's bit widths.
-// gain_inv: store 1/sigma (encoding) instead of sigma (decoding).
-// bsl: this slab's bit widths in shared memory; sig: its sigmas.
-__device__ __forceinline__ void slab_meta(const Geom& g, int ks, const unsigned char* bsl, const float* sig,
-                                          const uint32_t* pen, uint32_t wbase, bool gain_inv, uint32_t* sb_bits,
-                                          float* sb_gain, uint32_t* sb_off) {
-  const int lane = threadIdx.x & 31, nwarp = blockDim.x >> 5;
-  for (int kh = threadIdx.x >> 5; kh < g.H; kh += nwarp) {
-    const int j = kh * g.W + lane;
-    const uint32_t b = lane < g.W ? bsl[j] : 0u;
-    uint32_t incl = b;
+// Stream positions (relative to the slab's first word) of rows 2kp and 2kp+1, for one warp.
+template <class D>
+__device__ __forceinline__ void row_positions(const D& g, const unsigned char* bs, int kp, uint32_t base,
+                                              uint32_t& p0, uint32_t& p1) {
+  const int lane = threadIdx.x & 31, lim = 2 * kp * g.W;
+  uint32_t before = 0, row0 = 0;
+  for (int i = lane; i < lim; i += 32) before += bs[i];
+  for (int i = lane; i < g.W; i += 32) row0 += bs[lim + i];
+  before = __reduce_add_sync(0xffffffffu, before);
+  row0 = __reduce_add_sync(0xffffffffu, row0);
+  p0 = base + before;
+  p1 = p0 + row0;
+}
+
+// Forward rearrangement.  The tile's cells (h, w) sit at cell index h*Wp + w.  After the pass
+// along H, element (row pair kp, column w, channel c) = {X[2kp][w], X[2kp+1][w]} (float2) sits at
+// float2 index ((2kp + (w & 1))*Wp + (w & ~1))*16 + c: the 256 bytes of cells (2kp + d, w0) and
+// (2kp + d, w0 + 1) hold row pair kp of column w0 + d.  Those are bytes that column pair w0 itself
+// read, so a warp rewrites its own column pair in place with no other warp involved.
+__device__ __forceinline__ int rp_index(int Wp, int kp, int w) { return ((2 * kp + (w & 1)) * Wp + (w & ~1)) * 16; }
+
+// Column pair (w0, w0+1): read, DCT along H, written back in place as row pairs.
+template <int HC, class D>
+__device__ __forceinline__ void h_pass_fwd(const D& g, float* tile, int w0, int lane) {
+  const int Wp = 2 * row_pairs(g.W), HP = row_pairs(g.H);
+  float2 xh[HC];
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
+  for (int h = 0; h < HC; ++h)
+    if (h < g.H) {
+      const float* cell = tile + (h * Wp + w0) * kChunk + lane;
+      xh[h] = make_float2(cell[0], cell[kChunk]);   // column W (odd W) is padding: read, never used
     }
-    if (lane < g.W) {
-      sb_bits[j] = b;
-      sb_off[j] = pen[ks * g.H + kh] - wbase + incl - b;
-      const float sg = sig[j];
-      sb_gain[j] = gain_inv ? (b ? __frcp_rn(sg) : 0.f) : sg;
+  __syncwarp();   // the whole column pair is read before any lane rewrites it
+  pencil<HC, D::hx, false>(xh, g.H);
+  float2* t2 = reinterpret_cast<float2*>(tile);
+#pragma unroll
+  for (int kp = 0; kp < (HC + 1) / 2; ++kp)
+    if (kp < HP) {
+      const float2 a = xh[2 * kp];
+      const float2 b = (2 * kp + 1 < g.H) ? xh[2 * kp + 1] : make_float2(0.f, 0.f);
+      t2[rp_index(Wp, kp, w0) + lane] = make_float2(a.x, b.x);
+      t2[rp_index(Wp, kp, w0 + 1) + lane] = make_float2(a.y, b.y);
     }
-  }
+}
+// Row pair kp -> DCT along W.
+template <int WC, class D>
+__device__ __forceinline__ void w_load_fdct(const D& g, const float2* t2, int kp, int lane, float2 (&x)[WC]) {
+  const int Wp = 2 * row_pairs(g.W);
+#pragma unroll
+  for (int t = 0; t < WC; ++t)
+    if (t < g.W) x[t] = t2[rp_index(Wp, kp, t) + lane];
+  pencil<WC, D::wx, false>(x, g.W);
+}
+// Energies of row pair kp, written over its own (already read) elements: channel c of record
+// (kp, t) at rp_index(kp, t) + (c ^ (p & 15)) with p = kp*W + t, conflict-free for the 32 channels
+// writing a record and for the 16 records that a half warp reads at once.
+template <int WC, class D>
+__device__ __forceinline__ void put_energy(const D& g, float2* t2, int kp, int lane, const float2 (&x)[WC]) {
+  const int Wp = 2 * row_pairs(g.W);
+#pragma unroll
+  for (int t = 0; t < WC; ++t)
+    if (t < g.W) {
+      const int p = kp * g.W + t;
+      t2[rp_index(Wp, kp, t) + (lane ^ (p & 15))] = __fmul2_rn(x[t], x[t]);
+    }
 }
 
-template <int HC, int WC, int MODE>
-__global__ void __launch_bounds__(kHwThreads) fdct_hw_kernel(const __grid_constant__ Geom g,
-                                                             const __grid_constant__ UnitList ul,
-                                                             const float* __restrict__ Y, float* __restrict__ partial) {
+// ---------------------------------------------------------------------------------- forward ---
+// Register budget: class-16 pencils fit two CTAs of 256 threads per SM; class-32 float2 pencils
+// need more than 128 registers.
+constexpr int kHwMinBlocks = (TACTKV_HCLASS == 16 && TACTKV_WCLASS == 16) ? 2 : 1;
+
+template <int HC, int WC, int HX, int WX, int MODE>
+__global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) fdct_hw_kernel(const __grid_constant__ Geom g, const __grid_constant__ UnitList ul,
+                                                      const float* __restrict__ Y, float* __restrict__ partial,
+                                                      const uint32_t* __restrict__ slab_off, int spc) {
   extern __shared__ __align__(16) unsigned char smem[];
-  const HwLayout L = hw_layout(g.HW, g.N, g.S, g.H, MODE == kStats ? kLayStats : kLayQuant);
-  float2* tiles = reinterpret_cast<float2*>(smem + L.tile);
-  float* thr = reinterpret_cast<float*>(smem + L.thr);
-  uint32_t* pen = reinterpret_cast<uint32_t*>(smem + L.pen);   // bit offset of every (k_s, k_h) pencil
-  uint32_t* sb_bits = reinterpret_cast<uint32_t*>(smem + L.meta);  // this slab: bits of every bin
-  float* sb_gain = reinterpret_cast<float*>(smem + L.meta) + g.HW;   // 1/sigma of every bin
-  uint32_t* sb_off = reinterpret_cast<uint32_t*>(smem + L.off);      // bit offset in the slab's words
-  unsigned char* bsl = smem + L.bsl;                                   // bit widths of two slabs
-  float* sig2 = reinterpret_cast<float*>(smem + L.sig2);               // sigmas of two slabs
-  float* energy = reinterpret_cast<float*>(smem + L.uni);
-  uint32_t* sbuf = reinterpret_cast<uint32_t*>(smem + L.uni);
-  uint32_t* carry = reinterpret_cast<uint32_t*>(smem + L.carry);
-  uint32_t* swarp = reinterpret_cast<uint32_t*>(smem + L.warp);
-  const int words = L.words;
-  const int chunk = blockIdx.x, u = blockIdx.y;
+  const Dims<HX, WX> D(g);
+  constexpr bool quant = MODE == kQuant, raw = MODE == kRaw, stats = MODE == kStats;
+  const HwLayout L = hw_layout(D.H, D.W, stats ? kLayStats : kLayQuant);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int HP = row_pairs(D.H), WP = row_pairs(D.W);
+  const int chunk = blockIdx.x, u = blockIdx.z;
+  const int ks0 = blockIdx.y * spc, ks1 = min(g.S, ks0 + spc);
   const UnitDev& ud = ul.u[u];
   unsigned char* pay = ud.payload;
-  uint32_t* words_out = reinterpret_cast<uint32_t*>(pay + g.off_codes);
-  const bool quant = MODE == kQuant;
-  uint32_t cstride = 0, stride_words = 0;
-  if (MODE != kStats) {  // written by the allocation kernel
-    cstride = reinterpret_cast<const uint32_t*>(pay)[11];
-    stride_words = cstride / 4;
-  }
-  const float4* ysrc = reinterpret_cast<const float4*>(Y + (size_t)u * g.S * g.HW * g.n) + chunk * (kChunk / 4);
+  const float* ysrc = Y + (size_t)u * g.S * D.HW * g.n + chunk * kChunk;
+  uint32_t* sbuf = reinterpret_cast<uint32_t*>(smem + L.sbuf);
+  const uint4* meta = reinterpret_cast<const uint4*>(smem + L.meta);
+  float* thr = reinterpret_cast<float*>(smem + L.thr);
+  unsigned char* qcell = smem + L.qcell;
+  uint32_t* carry = reinterpret_cast<uint32_t*>(smem + L.carry);
   const unsigned char* pay_b = pay + kHeaderBytes;
   const float* pay_sig = reinterpret_cast<const float*>(pay + g.off_sigma);
+  const uint32_t* P = slab_off + (size_t)u * (g.S + 2);
+  uint32_t cstride = 0, sw = 0;
+  if (!stats) {  // written by the allocation kernel
+    cstride = reinterpret_cast<const uint32_t*>(pay)[11];
+    sw = cstride / 4;
+  }
+  uint32_t* words_out = reinterpret_cast<uint32_t*>(pay + g.off_codes) + (size_t)chunk * kChunk * sw;
 
-  // The unit's bit widths, needed once for the pencil offsets, go to the tile buffer that slab 0
-  // does not use; with a single buffer they go there first and slab 0 follows.
-  unsigned char* bstage = reinterpret_cast<unsigned char*>(tiles + (L.nbuf == 2 ? (size_t)g.HW * kPairs : 0));
-  if (!quant || L.nbuf == 2) issue_tile(g, ysrc, 0, tiles);
+  auto tile_of = [&](int ks) {
+    return reinterpret_cast<float*>(smem + L.tile + (L.nbuf == 2 ? (ks & 1) : 0) * L.tile_bytes);
+  };
+  auto bsl_of = [&](int ks) { return smem + L.bsl + (ks & 1) * L.bsl_stride; };
+  auto sig_of = [&](int ks) { return reinterpret_cast<float*>(smem + L.sig) + (ks & 1) * D.HW; };
+
+  issue_tile(D, ysrc + (size_t)ks0 * D.HW * g.n, tile_of(ks0));
   if (quant) {
-    issue_bits(g, pay_b, bstage);
-    issue_slab_bits(g, pay_b, 0, bsl);
-    issue_sigma(g, pay_sig, 0, sig2);
+    issue_slab_bits(D, pay_b, ks0, bsl_of(ks0));
+    issue_sigma(D, pay_sig, ks0, sig_of(ks0));
+    for (int i = threadIdx.x; i < TACTKV_THR_PAD_TOTAL; i += blockDim.x) thr[i] = c_thr_pad[i];
+    for (int i = threadIdx.x; i < 6 * TACTKV_Q_CELLS; i += blockDim.x) qcell[i] = c_qcell[i];
+    if (threadIdx.x < kChunk) carry[threadIdx.x] = 0;
   }
   cp_async_commit();
-  if (quant) {
-    __shared__ unsigned int s_unused;
-    for (int i = threadIdx.x; i < kLmThrTotal; i += blockDim.x) thr[i] = c_lm_thresholds[i];
-    if (threadIdx.x < kChunk) carry[threadIdx.x] = 0;
+  const uint32_t A = quant ? P[ks0] : 0u;   // first stream bit of the range
+
+  for (int ks = ks0; ks < ks1; ++ks) {
+    float* tile = tile_of(ks);
+    const unsigned char* bs = bsl_of(ks) + (((size_t)ks * D.HW) & 15);
     cp_async_wait_all();
-    __syncthreads();
-    pencil_offsets(g, bstage, pen, swarp, &s_unused);   // widths come from the allocation: all <= 8
-    if (L.nbuf == 1) {  // every read of bstage is done
-      issue_tile(g, ysrc, 0, tiles);
+    __syncthreads();  // slab ks is in place; every thread is done with slab ks - 1
+    if (ks + 1 < ks1) {
+      if (L.nbuf == 2) issue_tile(D, ysrc + (size_t)(ks + 1) * D.HW * g.n, tile_of(ks + 1));
+      if (quant) {
+        issue_slab_bits(D, pay_b, ks + 1, bsl_of(ks + 1));
+        issue_sigma(D, pay_sig, ks + 1, sig_of(ks + 1));
+      }
       cp_async_commit();
     }
-  }
-  uint32_t P = 0;  // stream bits written so far, identical for every channel
-  for (int ks = 0; ks < g.S; ++ks) {
-    const int cur = L.nbuf == 2 ? (ks & 1) : 0;
-    float2* tile = tiles + (size_t)cur * g.HW * kPairs;
-    cp_async_wait_all();
-    __syncthreads();  // slab ks is in place and every thread is done with slab ks - 1
-    if (L.nbuf == 2 && ks + 1 < g.S) issue_tile(g, ysrc, ks + 1, tiles + (size_t)(cur ^ 1) * g.HW * kPairs);
-    if (quant && ks + 1 < g.S) {
-      issue_slab_bits(g, pay_b, ks + 1, bsl + ((ks + 1) & 1) * L.bsl_stride);
-      issue_sigma(g, pay_sig, ks + 1, sig2 + ((ks + 1) & 1) * g.HW);
-    }
-    if (ks + 1 < g.S && (L.nbuf == 2 || quant)) cp_async_commit();
-    const uint32_t slab_end = quant ? (ks + 1 < g.S ? pen[(ks + 1) * g.H] : (uint32_t)0) : 0u;
-    const uint32_t w0 = P >> 5;                 // first stream word this slab touches
-    uint32_t slab_bits = 0;
+    uint32_t pstart = 0, slab_bits = 0;
     if (quant) {
-      slab_bits = (ks + 1 < g.S ? slab_end : reinterpret_cast<const uint32_t*>(pay)[10]) - P;
-      const int nw = (int)(((P & 31u) + slab_bits + 31) >> 5) + 1;
-      for (int i = threadIdx.x; i < kChunk * nw; i += blockDim.x) {
-        const int ch = i / nw, w = i - ch * nw;
-        sbuf[ch * words + w] = w == 0 ? carry[ch] : 0u;
-      }
-      slab_meta(g, ks, bsl + (ks & 1) * L.bsl_stride + (((size_t)ks * g.HW) & 15), sig2 + (ks & 1) * g.HW, pen,
-                w0 << 5, true, sb_bits, sb_gain, sb_off);
+      pstart = P[ks];
+      slab_bits = P[ks + 1] - pstart;
+      slab_records(D, bs, sig_of(ks), true, smem + L.meta);
+      const int nw = (int)(((pstart & 31u) + slab_bits + 31) >> 5) + 1;
+      for (int c = warp; c < kChunk; c += nwarps)
+        for (int w = lane; w < nw; w += 32) sbuf[c * L.words + w] = w == 0 ? carry[c] : 0u;
     }
-    h_pass<HC, false>(g, tile);
+
+    // DCT along H, in place, one column pair at a time per warp
+    for (int wp = warp; wp < WP; wp += nwarps) h_pass_fwd<HC>(D, tile, 2 * wp, lane);
     __syncthreads();
-    // W pass fused with the per-bin epilogue.  Rows are dealt so that warp w takes k_h = w and
-    // k_h = H-1-w: the low-frequency rows, which carry most of the code bits, pair with light ones.
-    for (int p = threadIdx.x; p < g.H * kPairs; p += blockDim.x) {
-      const int r = p >> 4, pair = p & 15;
-      const int kh = (r & 1) ? g.H - 1 - (r >> 1) : (r >> 1);
-      const int base = kh * g.W * kPairs + pair;
-      float2 x[WC];
+    float2* t2 = reinterpret_cast<float2*>(tile);
+    const int Wp = 2 * WP;
+
+    // DCT along W on row pair kp, fused with the epilogue
+    if (stats) {
+      for (int kp = warp; kp < HP; kp += nwarps) {
+        float2 x[WC];
+        w_load_fdct<WC>(D, t2, kp, lane, x);
+        __syncwarp();   // the row pair is read before its energies overwrite it
+        put_energy<WC>(D, t2, kp, lane, x);
+      }
+      __syncthreads();
+      float* dst = partial + ((size_t)u * g.nch + chunk) * g.N + (size_t)ks * D.HW;
+      for (int p = threadIdx.x; p < HP * D.W; p += blockDim.x) {
+        const int r = p / D.W, t = p - r * D.W;
+        const float2* e = t2 + rp_index(Wp, r, t);
+        const int sw15 = p & 15;
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll 8
+        for (int c = 0; c < kChunk; ++c) acc = __fadd2_rn(acc, e[c ^ sw15]);
+        dst[2 * r * D.W + t] = acc.x;
+        if (2 * r + 1 < D.H) dst[(2 * r + 1) * D.W + t] = acc.y;
+      }
+    } else {
+      for (int kp = warp; kp < HP; kp += nwarps) {
+        float2 x[WC];
+        w_load_fdct<WC>(D, t2, kp, lane, x);
+        if (raw) {
+          float* s = reinterpret_cast<float*>(pay + g.off_codes + (size_t)(chunk * kChunk + lane) * cstride) +
+                     (size_t)ks * D.HW + 2 * kp * D.W;
+          const bool second = 2 * kp + 1 < D.H;
 #pragma unroll
-      for (int t = 0; t < WC; ++t)
-        if (t < g.W) x[t] = tile[base + t * kPairs];
-      dct_pencil<WC, false>(x, g.W);
-      if (MODE == kStats) {
-#pragma unroll
-        for (int t = 0; t < WC; ++t)
-          if (t < g.W) energy[(kh * g.W + t) * kEnergyStride + pair] = x[t].x * x[t].x + x[t].y * x[t].y;
-      } else if (MODE == kRaw) {
-        const int c = chunk * kChunk + 2 * pair;
-        float* s0 = reinterpret_cast<float*>(pay + g.off_codes + (size_t)c * cstride) + ks * g.HW + kh * g.W;
-        float* s1 = reinterpret_cast<float*>(pay + g.off_codes + (size_t)(c + 1) * cstride) + ks * g.HW + kh * g.W;
-#pragma unroll
-        for (int t = 0; t < WC; ++t)
-          if (t < g.W) {
-            s0[t] = x[t].x;
-            s1[t] = x[t].y;
-          }
-      } else {
-        // the pencil's codes are contiguous in both channel streams: pack them in 64-bit
-        // registers and OR whole words into the slab's stream buffer
-        const int i0 = kh * g.W;
-        const uint32_t o0 = sb_off[i0];
-        uint32_t* r0 = sbuf + (2 * pair) * words + (o0 >> 5);
-        uint32_t* r1 = r0 + words;
-        unsigned long long a0 = 0, a1 = 0;
-        uint32_t apos = o0 & 31u;
-#pragma unroll
-        for (int t = 0; t < WC; ++t) {
-          if (t < g.W) {
-            const int bits = (int)sb_bits[i0 + t];
-            if (bits) {
-              const float inv = sb_gain[i0 + t];
-              a0 |= (unsigned long long)quant_code(x[t].x * inv, bits, thr) << apos;
-              a1 |= (unsigned long long)quant_code(x[t].y * inv, bits, thr) << apos;
-              apos += bits;
-              if (apos >= 32) {
-                atomicOr(r0++, (uint32_t)a0);
-                atomicOr(r1++, (uint32_t)a1);
-                a0 >>= 32;
-                a1 >>= 32;
-                apos -= 32;
-              }
+          for (int t = 0; t < WC; ++t)
+            if (t < D.W) {
+              s[t] = x[t].x;
+              if (second) s[D.W + t] = x[t].y;
             }
-          }
-        }
-        if (a0 | a1) {
-          atomicOr(r0, (uint32_t)a0);
-          atomicOr(r1, (uint32_t)a1);
-        }
-      }
-    }
-    __syncthreads();
-    if (MODE == kStats) {
-      float* dst = partial + ((size_t)u * g.nch + chunk) * g.N + (size_t)ks * g.HW;
-      for (int j = threadIdx.x; j < g.HW; j += blockDim.x) {
-        const float* e = energy + j * kEnergyStride;
-        float acc = 0.f;
+        } else {
+          uint32_t p0, p1;
+          row_positions(D, bs, kp, pstart & 31u, p0, p1);
+          uint32_t* row = sbuf + lane * L.words;
+          uint32_t acc0 = 0, acc1 = 0;
 #pragma unroll
-        for (int q = 0; q < kPairs; ++q) acc += e[q];
-        dst[j] = acc;
+          for (int t = 0; t < WC; ++t)
+            if (t < D.W) {
+              const uint4 m = meta[kp * D.W + t];
+              const float2 uu = __fmul2_rn(x[t], make_float2(__uint_as_float(m.x), __uint_as_float(m.y)));
+              const int b0 = m.z & 0xff, b1 = (m.z >> 8) & 0xff;
+              if (b0) put_code(acc0, p0, quant_code(uu.x, b0, thr, qcell), b0, row);
+              if (b1) put_code(acc1, p1, quant_code(uu.y, b1, thr, qcell), b1, row);
+            }
+          if (p0 & 31u) atomicOr(row + (p0 >> 5), acc0);
+          if (p1 & 31u) atomicOr(row + (p1 >> 5), acc1);
+        }
       }
-    } else if (quant) {
-      // complete words go out now; the word holding the run's last bits carries over
-      const uint32_t endbit = (P & 31u) + slab_bits;
-      const int full = (int)(endbit >> 5);
-      for (int i = threadIdx.x; i < kChunk * full; i += blockDim.x) {
-        const int ch = i / full, w = i - ch * full;
-        words_out[(size_t)(chunk * kChunk + ch) * stride_words + w0 + w] = sbuf[ch * words + w];
+      if (quant) {
+        __syncthreads();
+        // complete words go out; the first word of the range may be shared with the previous range
+        const uint32_t endbit = (pstart & 31u) + slab_bits;
+        const int full = (int)(endbit >> 5);
+        const uint32_t wbase = pstart >> 5, wA = A >> 5;
+        const bool shared_first = (A & 31u) != 0;
+        for (int c = warp; c < kChunk; c += nwarps) {
+          uint32_t* out = words_out + (size_t)c * sw;
+          for (int w = lane; w < full; w += 32) {
+            const uint32_t v = sbuf[c * L.words + w];
+            if (shared_first && wbase + w == wA) atomicOr(out + wA, v);
+            else out[wbase + w] = v;
+          }
+          if (lane == 0) carry[c] = (endbit & 31u) ? sbuf[c * L.words + full] : 0u;
+        }
       }
-      if (threadIdx.x < kChunk) carry[threadIdx.x] = (endbit & 31u) ? sbuf[threadIdx.x * words + full] : 0u;
-      P += slab_bits;
     }
-    if (L.nbuf == 1 && ks + 1 < g.S) {
+    if (L.nbuf == 1 && ks + 1 < ks1) {
       __syncthreads();  // everyone is done with the only tile
-      issue_tile(g, ysrc, ks + 1, tiles);
+      issue_tile(D, ysrc + (size_t)(ks + 1) * D.HW * g.n, tile_of(ks + 1));
       cp_async_commit();
     }
   }
   cp_async_wait_all();
   if (quant) {
     __syncthreads();
-    // the last partial word, then zero padding up to the channel stride
-    const uint32_t wlast = P >> 5;
-    const int tail = (int)stride_words - (int)wlast;
-    for (int i = threadIdx.x; i < kChunk * tail; i += blockDim.x) {
-      const int ch = i / tail, w = i - ch * tail;
-      words_out[(size_t)(chunk * kChunk + ch) * stride_words + wlast + w] = (w == 0) ? carry[ch] : 0u;
+    // the range's last partial word (shared with the next range), then the stream's zero padding
+    const uint32_t B = P[ks1];
+    if (threadIdx.x < kChunk && (B & 31u))
+      atomicOr(words_out + (size_t)threadIdx.x * sw + (B >> 5), carry[threadIdx.x]);
+    if (ks1 == g.S) {
+      const uint32_t first = (B + 31) >> 5;
+      for (int c = warp; c < kChunk; c += nwarps)
+        for (uint32_t w = first + lane; w < sw; w += 32) words_out[(size_t)c * sw + w] = 0u;
     }
-  } else if (MODE == kRaw) {
+  } else if (raw && ks1 == g.S) {
     const int pad = (int)cstride - 4 * g.N;
     for (int i = threadIdx.x; i < kChunk * pad; i += blockDim.x) {
-      const int ch = i / pad, b = i - ch * pad;
-      pay[g.off_codes + (size_t)(chunk * kChunk + ch) * cstride + 4 * g.N + b] = 0;
+      const int c = i / pad, b = i - c * pad;
+      pay[g.off_codes + (size_t)(chunk * kChunk + c) * cstride + 4 * g.N + b] = 0;
     }
   }
 }
 
-// ----------------------------------------------------------------------------------- decode ---
-template <int HC, int WC, int MODE>
-__global__ void __launch_bounds__(kHwThreads) idct_hw_kernel(const __grid_constant__ Geom g,
-                                                             const __grid_constant__ UnitList ul,
-                                                             float* __restrict__ V, unsigned int* status) {
+// ---------------------------------------------------------------------------------- inverse ---
+template <int HC, int WC, int HX, int WX, int MODE>
+__global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) idct_hw_kernel(const __grid_constant__ Geom g, const __grid_constant__ UnitList ul,
+                                                      float* __restrict__ V, const uint32_t* __restrict__ slab_off,
+                                                      int spc) {
   extern __shared__ __align__(16) unsigned char smem[];
-  const HwLayout L = hw_layout(g.HW, g.N, g.S, g.H, kLayDecode);
-  float2* tile = reinterpret_cast<float2*>(smem + L.tile);
-  float* lvs = reinterpret_cast<float*>(smem + L.lv);
-  uint32_t* pen = reinterpret_cast<uint32_t*>(smem + L.pen);   // first stream bit of every pencil
-  uint32_t* sbufs = reinterpret_cast<uint32_t*>(smem + L.uni);
-  uint32_t* swarp = reinterpret_cast<uint32_t*>(smem + L.warp);
-  uint32_t* sb_bits = reinterpret_cast<uint32_t*>(smem + L.meta);  // this slab: bits of every bin
-  float* sb_gain = reinterpret_cast<float*>(smem + L.meta) + g.HW;   // sigma of every bin
-  uint32_t* sb_off = reinterpret_cast<uint32_t*>(smem + L.off);      // bit offset in the slab's words
-  unsigned char* bsl = smem + L.bsl;                                   // bit widths of two slabs
-  float* sig2 = reinterpret_cast<float*>(smem + L.sig2);               // sigmas of two slabs
-  __shared__ int s_ok;
-  __shared__ unsigned int s_bad;
-  const int words = L.words;
-  const int chunk = blockIdx.x, u = blockIdx.y;
+  const Dims<HX, WX> D(g);
+  constexpr bool raw = MODE == kRaw;
+  const HwLayout L = hw_layout(D.H, D.W, kLayDecode);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int HP = row_pairs(D.H), WP = row_pairs(D.W);
+  const int chunk = blockIdx.x, u = blockIdx.z;
+  const int ks0 = blockIdx.y * spc, ks1 = min(g.S, ks0 + spc);
   const UnitDev& ud = ul.u[u];
   const unsigned char* pay = ud.payload;
-  const bool raw = MODE == kRaw;
-  uint32_t code_bits = 0;
-  if (threadIdx.x == 0) {
-    // the header must describe exactly the unit the caller asked for
-    const uint32_t* h32 = reinterpret_cast<const uint32_t*>(pay);
-    const int32_t* i32 = reinterpret_cast<const int32_t*>(pay);
-    const uint32_t ver_flags = h32[1], cb = h32[10], cs = h32[11];
-    const unsigned long long total = *reinterpret_cast<const unsigned long long*>(pay + 48);
-    bool ok = h32[0] == kMagic && (ver_flags & 0xffffu) == (uint32_t)kVersion &&
-              ((ver_flags >> 16) & TACTKV_NO_QUANT) == (raw ? TACTKV_NO_QUANT : 0u) && i32[2] == ud.layer &&
-              i32[3] == ud.kv && i32[4] == g.S && i32[5] == g.H && i32[6] == g.W && i32[7] == g.heads &&
-              i32[8] == g.head_dim && i32[9] == g.bits;
-    if (ok) {
-      ok = (raw ? cb == 32u * (uint32_t)g.N : cb <= (uint32_t)g.bits * (uint32_t)g.N) &&
-           (long long)cs == pad16(((long long)cb + 7) / 8) &&
-           (long long)total == (long long)g.off_codes + (long long)g.n * cs && (long long)total <= g.capacity;
-    }
-    s_ok = ok;
-    s_bad = 0;
-  }
-  for (int i = threadIdx.x; i < kLmLvTotal; i += blockDim.x) lvs[i] = c_lm_levels[i];
-  __syncthreads();
-  const bool ok0 = s_ok;
-  const uint32_t stride_words = ok0 ? reinterpret_cast<const uint32_t*>(pay)[11] / 4 : 0u;
-  if (ok0) code_bits = reinterpret_cast<const uint32_t*>(pay)[10];
-  const uint32_t* streams = reinterpret_cast<const uint32_t*>(pay + g.off_codes);
+  const uint32_t* P = slab_off + (size_t)u * (g.S + 2);
+  const bool ok = P[g.S + 1] != 0;   // the index kernel checked the header and the bit widths
+  const uint32_t cstride = ok ? reinterpret_cast<const uint32_t*>(pay)[11] : 0u, sw = cstride / 4;
+  const uint32_t* streams = reinterpret_cast<const uint32_t*>(pay + g.off_codes) + (size_t)chunk * kChunk * sw;
   const unsigned char* pay_b = pay + kHeaderBytes;
   const float* pay_sig = reinterpret_cast<const float*>(pay + g.off_sigma);
-  // every pencil's first stream bit, from the unit's bit widths staged in the (still unused) tile
-  if (ok0 && !raw) {
-    unsigned char* bstage = reinterpret_cast<unsigned char*>(tile);
-    issue_bits(g, pay_b, bstage);
-    issue_slab_bits(g, pay_b, 0, bsl);
-    issue_sigma(g, pay_sig, 0, sig2);
-    cp_async_commit();
-    cp_async_wait_all();
-    __syncthreads();
-    const uint32_t total = pencil_offsets(g, bstage, pen, swarp, &s_bad);
-    __syncthreads();
-    if (threadIdx.x == 0 && (total != code_bits || s_bad)) s_ok = 0;
-  }
-  __syncthreads();
-  const bool ok = s_ok;
-  if (threadIdx.x == 0 && !ok && chunk == 0) set_status(status, TACTKV_CORRUPT_PAYLOAD);
-  const int ch0 = chunk * kChunk;
-  auto slab_begin = [&](int ks) -> uint32_t { return ks < g.S ? pen[ks * g.H] : code_bits; };
+  float2* tile = reinterpret_cast<float2*>(smem + L.tile);
+  const uint4* meta = reinterpret_cast<const uint4*>(smem + L.meta);
+  float* lvs = reinterpret_cast<float*>(smem + L.lv);
+  auto sbuf_of = [&](int ks) { return reinterpret_cast<uint32_t*>(smem + L.sbuf) + (ks & 1) * kChunk * L.words; };
+  auto bsl_of = [&](int ks) { return smem + L.bsl + (ks & 1) * L.bsl_stride; };
+  auto sig_of = [&](int ks) { return reinterpret_cast<float*>(smem + L.sig) + (ks & 1) * D.HW; };
 
-  auto issue_words = [&](int ks, uint32_t* sb) {  // stream words of slab ks for the 32 channels
-    const uint32_t p0 = slab_begin(ks), p1 = slab_begin(ks + 1);
+  // stream words of slab ks for the 32 channels, from word P(ks) >> 5 on, then two zero words
+  // that the readers' look-ahead may touch
+  auto issue_words = [&](int ks) {
+    uint32_t* sb = sbuf_of(ks);
+    const uint32_t p0 = P[ks], p1 = P[ks + 1];
     const uint32_t w0 = p0 >> 5;
     const int nw = (int)(((p0 & 31u) + (p1 - p0) + 31) >> 5);
-    for (int i = threadIdx.x; i < kChunk * (nw + 1); i += blockDim.x) {
-      const int ch = i / (nw + 1), w = i - ch * (nw + 1);
-      const uint32_t word = w0 + w;
-      if (w < nw && word < stride_words) cp_async4(sb + ch * words + w, streams + (size_t)(ch0 + ch) * stride_words + word);
-      else sb[ch * words + w] = 0u;
-    }
+    for (int c = warp; c < kChunk; c += nwarps)
+      for (int w = lane; w < nw + 2; w += 32) {
+        if (w < nw) cp_async4(sb + c * L.words + w, streams + (size_t)c * sw + w0 + w);
+        else sb[c * L.words + w] = 0u;
+      }
   };
-
-  if (ok && !raw) {
-    issue_words(0, sbufs);
+  if (!raw) {
+    for (int i = threadIdx.x; i < kLmLvTotal; i += blockDim.x) lvs[i] = c_lm_levels[i];
+    if (ok) {
+      issue_words(ks0);
+      issue_slab_bits(D, pay_b, ks0, bsl_of(ks0));
+      issue_sigma(D, pay_sig, ks0, sig_of(ks0));
+    }
     cp_async_commit();
   }
-  float4* vdst = reinterpret_cast<float4*>(V + (size_t)u * g.S * g.HW * g.n) + chunk * (kChunk / 4);
-  const int rowq = g.n / 4;
-  for (int ks = 0; ks < g.S; ++ks) {
-    const int mc = ks & 1;
-    const uint32_t* sb = sbufs + (size_t)mc * kChunk * words;
+  float* vunit = V + (size_t)u * g.S * D.HW * g.n + chunk * kChunk + lane;
+
+  for (int ks = ks0; ks < ks1; ++ks) {
+    const unsigned char* bs = bsl_of(ks) + (((size_t)ks * D.HW) & 15);
     cp_async_wait_all();
-    __syncthreads();  // slab ks's stream words are in place; slab ks - 1 is done
-    if (ok && !raw && ks + 1 < g.S) {
-      issue_words(ks + 1, sbufs + (size_t)(mc ^ 1) * kChunk * words);
-      issue_slab_bits(g, pay_b, ks + 1, bsl + (mc ^ 1) * L.bsl_stride);
-      issue_sigma(g, pay_sig, ks + 1, sig2 + (mc ^ 1) * g.HW);
-      cp_async_commit();
-    }
-    const int i0s = ks * g.HW;
-    const uint32_t wbase = raw ? 0u : (slab_begin(ks) >> 5) << 5;
+    __syncthreads();  // slab ks's words are in place; slab ks - 1 is done
     if (ok && !raw) {
-      slab_meta(g, ks, bsl + mc * L.bsl_stride + (((size_t)ks * g.HW) & 15), sig2 + mc * g.HW, pen, wbase, false,
-                sb_bits, sb_gain, sb_off);
+      if (ks + 1 < ks1) {
+        issue_words(ks + 1);
+        issue_slab_bits(D, pay_b, ks + 1, bsl_of(ks + 1));
+        issue_sigma(D, pay_sig, ks + 1, sig_of(ks + 1));
+        cp_async_commit();
+      }
+      slab_records(D, bs, sig_of(ks), false, smem + L.meta);
       __syncthreads();
     }
-    // dequantize in registers, fused with the inverse DCT along W: a thread takes one pencil (a
-    // k_h row of W bins, two channels), whose codes are contiguous in both streams and are read
-    // through 64-bit windows; rows are dealt as in encoding (k_h = w with k_h = H-1-w)
-    for (int p = threadIdx.x; p < g.H * kPairs; p += blockDim.x) {
-      const int r = p >> 4, pair = p & 15;
-      const int kh = (r & 1) ? g.H - 1 - (r >> 1) : (r >> 1);
-      const int base = kh * g.W * kPairs + pair;
-      const int i0 = kh * g.W;
+    // decode rows 2j, 2j+1 of warp j and run the inverse DCT along W; write column pairs
+    for (int kp = warp; kp < HP; kp += nwarps) {
       float2 x[WC];
       if (!ok) {
 #pragma unroll
         for (int t = 0; t < WC; ++t) x[t] = make_float2(0.f, 0.f);
       } else if (raw) {
-        const float* st = reinterpret_cast<const float*>(streams);
-        const int c = ch0 + 2 * pair;
+        const float* s = reinterpret_cast<const float*>(pay + g.off_codes + (size_t)(chunk * kChunk + lane) * cstride) +
+                         (size_t)ks * D.HW + 2 * kp * D.W;
+        const bool second = 2 * kp + 1 < D.H;
 #pragma unroll
         for (int t = 0; t < WC; ++t)
-          if (t < g.W)
-            x[t] = make_float2(st[(size_t)c * stride_words + i0s + i0 + t], st[(size_t)(c + 1) * stride_words + i0s + i0 + t]);
+          if (t < D.W) x[t] = make_float2(s[t], second ? s[D.W + t] : 0.f);
       } else {
-        const uint32_t* row0 = sb + (2 * pair) * words;
-        const uint32_t* row1 = row0 + words;
-        const uint32_t o0 = sb_off[i0];
-        uint32_t wi = o0 >> 5, pos = o0 & 31u;
-        unsigned long long w0v = (unsigned long long)row0[wi] | ((unsigned long long)row0[wi + 1] << 32);
-        unsigned long long w1v = (unsigned long long)row1[wi] | ((unsigned long long)row1[wi + 1] << 32);
+        uint32_t p0, p1;
+        row_positions(D, bs, kp, P[ks] & 31u, p0, p1);
+        const uint32_t* row = sbuf_of(ks) + lane * L.words;
+        uint32_t wi0 = p0 >> 5, s0 = p0 & 31u, wi1 = p1 >> 5, s1 = p1 & 31u;
+        uint32_t lo0 = row[wi0], hi0 = row[wi0 + 1], lo1 = row[wi1], hi1 = row[wi1 + 1];
 #pragma unroll
-        for (int t = 0; t < WC; ++t) {
-          if (t < g.W) {
-            const int bits = (int)sb_bits[i0 + t];
-            float2 v = make_float2(0.f, 0.f);
-            if (bits) {
-              const uint32_t mask = (1u << bits) - 1u;
-              const float* lv = lvs + lm_lv_offset(bits);
-              const float sg = sb_gain[i0 + t];
-              v = make_float2(sg * lv[(uint32_t)(w0v >> pos) & mask], sg * lv[(uint32_t)(w1v >> pos) & mask]);
-              pos += bits;
-              if (pos >= 32) {
-                ++wi;
-                const bool in = wi + 1 < (uint32_t)words;
-                w0v = (w0v >> 32) | ((unsigned long long)(in ? row0[wi + 1] : 0u) << 32);
-                w1v = (w1v >> 32) | ((unsigned long long)(in ? row1[wi + 1] : 0u) << 32);
-                pos -= 32;
-              }
-            }
-            x[t] = v;
+        for (int t = 0; t < WC; ++t)
+          if (t < D.W) {
+            const uint4 m = meta[kp * D.W + t];
+            const int b0 = m.z & 0xff, b1 = (m.z >> 8) & 0xff;
+            float l0 = 0.f, l1 = 0.f;
+            if (b0) l0 = lvs[lm_lv_offset(b0) + get_code(lo0, hi0, s0, wi0, b0, row)];
+            if (b1) l1 = lvs[lm_lv_offset(b1) + get_code(lo1, hi1, s1, wi1, b1, row)];
+            x[t] = __fmul2_rn(make_float2(l0, l1), make_float2(__uint_as_float(m.x), __uint_as_float(m.y)));
           }
-        }
       }
-      dct_pencil<WC, true>(x, g.W);
+      pencil<WC, WX, true>(x, D.W);
+      const bool second = 2 * kp + 1 < D.H;
 #pragma unroll
-      for (int t = 0; t < WC; ++t)
-        if (t < g.W) tile[base + t * kPairs] = x[t];
+      for (int wp = 0; wp < (WC + 1) / 2; ++wp)
+        if (wp < WP) {
+          const float2 a = x[2 * wp];
+          const float2 b = (2 * wp + 1 < D.W) ? x[2 * wp + 1] : make_float2(0.f, 0.f);
+          tile[((2 * kp) * WP + wp) * kChunk + lane] = make_float2(a.x, b.x);
+          if (second) tile[((2 * kp + 1) * WP + wp) * kChunk + lane] = make_float2(a.y, b.y);
+        }
     }
     __syncthreads();
-    h_pass<HC, true>(g, tile);
-    __syncthreads();
-    float4* dst = vdst + (size_t)ks * g.HW * rowq;
-    const float4* src = reinterpret_cast<const float4*>(tile);
-    for (int i = threadIdx.x; i < g.HW * (kChunk / 4); i += blockDim.x) dst[(size_t)(i >> 3) * rowq + (i & 7)] = src[i];
+    // inverse DCT along H on column pair (2j, 2j+1) of warp j; store to V
+    for (int wp = warp; wp < WP; wp += nwarps) {
+      float2 xh[HC];
+#pragma unroll
+      for (int h = 0; h < HC; ++h)
+        if (h < D.H) xh[h] = tile[(h * WP + wp) * kChunk + lane];
+      pencil<HC, HX, true>(xh, D.H);
+      float* v = vunit + ((size_t)ks * D.HW + 2 * wp) * g.n;
+      const bool two = 2 * wp + 1 < D.W;
+#pragma unroll
+      for (int h = 0; h < HC; ++h)
+        if (h < D.H) {
+          float* cell = v + (size_t)h * D.W * g.n;
+          cell[0] = xh[h].x;
+          if (two) cell[g.n] = xh[h].y;
+        }
+    }
   }
   cp_async_wait_all();
 }
@@ -547,33 +582,59 @@ __global__ void __launch_bounds__(kHwThreads) idct_hw_kernel(const __grid_consta
 
 #define TACTKV_CAT2(a, b) a##b
 #define TACTKV_CAT(a, b) TACTKV_CAT2(a, b)
-#define TACTKV_LAUNCHER(h, w) TACTKV_CAT(TACTKV_CAT(TACTKV_CAT(launch_axis_hw_, h), _), w)
-cudaError_t TACTKV_LAUNCHER(TACTKV_HCLASS, TACTKV_WCLASS)(bool inverse, int mode, const Geom& g, const UnitList& ul,
-                                                          int nu, float* buf, float* partial, unsigned int* status,
-                                                          cudaStream_t st) {
-  const HwLayout L = hw_layout(g.HW, g.N, g.S, g.H, inverse ? kLayDecode : (mode == kStats ? kLayStats : kLayQuant));
-  const dim3 grid(g.nch, nu);
+#define TACTKV_HWNAME(base) TACTKV_CAT(TACTKV_CAT(TACTKV_CAT(base, TACTKV_HCLASS), _), TACTKV_WCLASS)
+namespace {
+template <int HX, int WX>
+cudaError_t launch_hw(bool inverse, int mode, const Geom& g, const UnitList& ul, int nu, float* buf, float* partial,
+                      const uint32_t* slab_off, int spc, cudaStream_t st) {
+  const HwLayout L = hw_layout(g.H, g.W, inverse ? kLayDecode : (mode == kStats ? kLayStats : kLayQuant));
+  const dim3 grid(g.nch, (g.S + spc - 1) / spc, nu);
+  const int threads = hw_threads(g.H, g.W);
   constexpr int H = TACTKV_HCLASS, W = TACTKV_WCLASS;
   const int sm = (int)L.total;
+  const size_t regions[] = {L.tile, L.sbuf, L.meta, L.sig, L.thr, L.lv, L.carry, L.bsl, L.qcell, L.tile_bytes,
+                            L.bsl_stride};
+  for (size_t r : regions)
+    if (r % 16) return cudaErrorMisalignedAddress;   // never launch a misaligned layout
+  if (L.total > 227 * 1024) return cudaErrorInvalidConfiguration;
+#define TACTKV_GO(kern, ...)                                                           \
+  do {                                                                                 \
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);       \
+    kern<<<grid, threads, sm, st>>>(__VA_ARGS__);                                      \
+  } while (0)
   if (inverse) {
-    if (mode == kRaw) {
-      cudaFuncSetAttribute(idct_hw_kernel<H, W, kRaw>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
-      idct_hw_kernel<H, W, kRaw><<<grid, kHwThreads, sm, st>>>(g, ul, buf, status);
-    } else {
-      cudaFuncSetAttribute(idct_hw_kernel<H, W, kQuant>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
-      idct_hw_kernel<H, W, kQuant><<<grid, kHwThreads, sm, st>>>(g, ul, buf, status);
-    }
+    if (mode == kRaw) TACTKV_GO((idct_hw_kernel<H, W, HX, WX, kRaw>), g, ul, buf, slab_off, spc);
+    else TACTKV_GO((idct_hw_kernel<H, W, HX, WX, kQuant>), g, ul, buf, slab_off, spc);
   } else if (mode == kStats) {
-    cudaFuncSetAttribute(fdct_hw_kernel<H, W, kStats>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
-    fdct_hw_kernel<H, W, kStats><<<grid, kHwThreads, sm, st>>>(g, ul, buf, partial);
+    TACTKV_GO((fdct_hw_kernel<H, W, HX, WX, kStats>), g, ul, buf, partial, slab_off, spc);
   } else if (mode == kRaw) {
-    cudaFuncSetAttribute(fdct_hw_kernel<H, W, kRaw>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
-    fdct_hw_kernel<H, W, kRaw><<<grid, kHwThreads, sm, st>>>(g, ul, buf, partial);
+    TACTKV_GO((fdct_hw_kernel<H, W, HX, WX, kRaw>), g, ul, buf, partial, slab_off, spc);
   } else {
-    cudaFuncSetAttribute(fdct_hw_kernel<H, W, kQuant>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
-    fdct_hw_kernel<H, W, kQuant><<<grid, kHwThreads, sm, st>>>(g, ul, buf, partial);
+    TACTKV_GO((fdct_hw_kernel<H, W, HX, WX, kQuant>), g, ul, buf, partial, slab_off, spc);
   }
+#undef TACTKV_GO
   return cudaGetLastError();
+}
+}  // namespace
+
+// The grids of the common layouts (medical volumes 16x16 and 24x24, video frames 14x14, the 8x8
+// test volume) have their own exact-size kernels; every other grid of the class runs the generic one.
+cudaError_t TACTKV_HWNAME(launch_axis_hw_)(bool inverse, int mode, const Geom& g, const UnitList& ul, int nu, float* buf,
+                                           float* partial, const uint32_t* slab_off, int spc, cudaStream_t st) {
+#if TACTKV_HCLASS == 16 && TACTKV_WCLASS == 16
+  if (g.H == 16 && g.W == 16) return launch_hw<16, 16>(inverse, mode, g, ul, nu, buf, partial, slab_off, spc, st);
+  if (g.H == 14 && g.W == 14) return launch_hw<14, 14>(inverse, mode, g, ul, nu, buf, partial, slab_off, spc, st);
+  if (g.H == 8 && g.W == 8) return launch_hw<8, 8>(inverse, mode, g, ul, nu, buf, partial, slab_off, spc, st);
+#elif TACTKV_HCLASS == 32 && TACTKV_WCLASS == 32
+  if (g.H == 24 && g.W == 24) return launch_hw<24, 24>(inverse, mode, g, ul, nu, buf, partial, slab_off, spc, st);
+#endif
+  return launch_hw<0, 0>(inverse, mode, g, ul, nu, buf, partial, slab_off, spc, st);
+}
+
+// Shared memory and threads of one CTA (host queries used to size the slab ranges).
+void TACTKV_HWNAME(axis_hw_shape_)(const Geom& g, bool inverse, int mode, size_t* smem, int* threads) {
+  *smem = hw_layout(g.H, g.W, inverse ? kLayDecode : (mode == kStats ? kLayStats : kLayQuant)).total;
+  *threads = hw_threads(g.H, g.W);
 }
 
 }  // namespace tactkv

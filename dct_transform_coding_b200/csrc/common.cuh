@@ -20,10 +20,10 @@ constexpr int kMaxUnits = 256;             // units per launch (descriptors trav
 constexpr int kHeaderBytes = 64;
 constexpr int kChunk = 32;                 // channels per H/W-axis CTA
 constexpr int kPairs = kChunk / 2;         // channel pairs: every pencil carries two channels (float2)
-constexpr int kHwThreads = 256;
 constexpr int kAllocThreads = 1024;
 constexpr size_t kStatusBytes = 256;       // status word at the start of the workspace
 constexpr int kMaxHW = 1024;               // H*W limit of the H/W-axis kernels
+constexpr int kMaxSlabs = 64;              // S limit
 
 enum HwMode { kStats = 0, kQuant = 1, kRaw = 2 };
 
@@ -68,9 +68,16 @@ inline int length_class(int L) { return L <= 16 ? 16 : (L <= 32 ? 32 : 64); }
 cudaError_t launch_axis_s(int cls, bool inverse, const Geom& g, const UnitList& ul, int nu, float* buf,
                           cudaStream_t st);
 cudaError_t launch_axis_hw(int hcls, int wcls, bool inverse, int mode, const Geom& g, const UnitList& ul, int nu, float* buf,
-                           float* partial, unsigned int* status, cudaStream_t st);
+                           float* partial, const uint32_t* slab_off, int spc, cudaStream_t st);
+void axis_hw_shape(int hcls, int wcls, const Geom& g, bool inverse, int mode, size_t* smem, int* threads);
+// Per-unit bit allocation: writes b, sigma, the header, the slab offsets P(k_s) (slab_off[u][0..S])
+// and zeroes the stream word at every P(k_s).
 cudaError_t launch_allocate(const Geom& g, const UnitList& ul, int nu, const float* partial, double* var,
-                            cudaStream_t st);
+                            uint32_t* slab_off, cudaStream_t st);
+// Decoding index: checks every unit's header and bit widths, writes slab_off[u][0..S] and the
+// unit's ok flag slab_off[u][S+1]; a bad unit sets TACTKV_CORRUPT_PAYLOAD in *status.
+cudaError_t launch_decode_index(const Geom& g, const UnitList& ul, int nu, uint32_t* slab_off, unsigned int* status,
+                                cudaStream_t st);
 
 #ifdef __CUDACC__
 // ------------------------------------------------------------------ float2 value operations ---
@@ -118,6 +125,21 @@ __device__ __forceinline__ void dct_pencil(V* x, int L) {
     }
   }
 #undef TACTKV_CASE
+}
+
+// Orthonormal DCT-II (INV = false) or DCT-III (INV = true) of exactly L values in registers.
+template <int L, bool INV, class V>
+__device__ __forceinline__ void dct_exact(V* x) {
+#define TACTKV_EXACT(n)              \
+  if constexpr (L == n) {            \
+    if constexpr (INV) idct_##n(x);  \
+    else fdct_##n(x);                \
+  }
+  TACTKV_EXACT(1) TACTKV_EXACT(2) TACTKV_EXACT(3) TACTKV_EXACT(4) TACTKV_EXACT(5) TACTKV_EXACT(6) TACTKV_EXACT(7)
+  TACTKV_EXACT(8) TACTKV_EXACT(9) TACTKV_EXACT(10) TACTKV_EXACT(11) TACTKV_EXACT(12) TACTKV_EXACT(13)
+  TACTKV_EXACT(14) TACTKV_EXACT(15) TACTKV_EXACT(16) TACTKV_EXACT(20) TACTKV_EXACT(24) TACTKV_EXACT(28)
+  TACTKV_EXACT(32) TACTKV_EXACT(40) TACTKV_EXACT(48) TACTKV_EXACT(56) TACTKV_EXACT(64)
+#undef TACTKV_EXACT
 }
 
 __device__ __forceinline__ void set_status(unsigned int* status, unsigned int code) { atomicCAS(status, 0u, code); }

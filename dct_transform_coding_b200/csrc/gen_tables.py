@@ -108,6 +108,42 @@ def f32(v: float) -> str:
     return repr(struct.unpack("<f", struct.pack("<f", v))[0]) + "f"
 
 
+# Code lookup for b >= 3.  The range [-G, G) of u is cut into K equal cells; cell j of u is
+# clamp(floor(fmaf(u, QSCALE, QOFFSET)), 0, K-1) in float32.  The table holds, per cell, the
+# number c of thresholds below the cell's lower edge minus DELTA; the code of u is then
+# c + [u >= t_c] + [u >= t_{c+1}], exact as long as every cell, widened by DELTA on both sides,
+# holds at most two thresholds (checked here).  DELTA covers the float32 rounding of the cell
+# index (|error| < 1e-4 cell widths).  Thresholds are padded with two +inf after the last one.
+QK = 512
+QG = 4.5
+QDELTA = 1e-4
+
+
+def f32v(v: float) -> float:
+    return struct.unpack("<f", struct.pack("<f", v))[0]
+
+
+def code_table(th32):
+    """Per-cell count of thresholds below (cell edge - DELTA), with the two-threshold check."""
+    scale = f32v(QK / (2.0 * QG))
+    offset = f32v(QK / 2.0)
+    out = []
+    for j in range(QK):
+        lo = (j - offset) / scale
+        hi = (j + 1 - offset) / scale
+        c = sum(1 for t in th32 if t < lo - QDELTA)
+        if j == 0:
+            inside = [t for t in th32 if t < hi + QDELTA]
+        elif j == QK - 1:
+            inside = [t for t in th32 if t >= lo - QDELTA]
+        else:
+            inside = [t for t in th32 if lo - QDELTA <= t < hi + QDELTA]
+        assert len(inside) <= 2, (len(th32), j, inside)
+        assert c <= 255
+        out.append(c)
+    return out, scale, offset
+
+
 def generate() -> str:
     lv_all, th_all, lv_off, th_off = [], [], [], []
     for b in range(1, 9):
@@ -130,6 +166,26 @@ def generate() -> str:
     lines += ["  " + ", ".join(f32(v) for v in lv_all[i:i + 4]) + "," for i in range(0, len(lv_all), 4)]
     lines += ["};", "static __constant__ float c_lm_thresholds[] = {"]
     lines += ["  " + ", ".join(f32(v) for v in th_all[i:i + 4]) + "," for i in range(0, len(th_all), 4)]
+    lines += ["};"]
+    # thresholds of each width followed by two +inf (width b starts at 2^b + b - 3), and the
+    # per-cell code table for b >= 3
+    pad_all, qtab = [], []
+    for b in range(1, 9):
+        th32 = [f32v(v) for v in th_all[th_off[b - 1]:th_off[b - 1] + (1 << b) - 1]]
+        assert len(pad_all) == (1 << b) + b - 3
+        pad_all += th32 + [math.inf, math.inf]
+        if b >= 3:
+            tab, scale, offset = code_table(th32)
+            qtab += tab
+    lines += [f"#define TACTKV_Q_CELLS {QK}",
+              f"#define TACTKV_Q_SCALE {f32(scale)}",
+              f"#define TACTKV_Q_OFFSET {f32(offset)}",
+              f"#define TACTKV_THR_PAD_TOTAL {len(pad_all)}",
+              "static __constant__ float c_thr_pad[] = {"]
+    lit = lambda v: "INFINITY" if math.isinf(v) else f32(v)
+    lines += ["  " + ", ".join(lit(v) for v in pad_all[i:i + 4]) + "," for i in range(0, len(pad_all), 4)]
+    lines += ["};", "static __constant__ unsigned char c_qcell[] = {"]
+    lines += ["  " + ", ".join(str(v) for v in qtab[i:i + 32]) + "," for i in range(0, len(qtab), 32)]
     lines += ["};", "#endif", ""]
     return "\n".join(lines)
 

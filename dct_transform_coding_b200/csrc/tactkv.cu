@@ -1,11 +1,12 @@
 // TACT-KV codec C ABI (host side): argument checks, grouping of units into waves, launches.
 //
-// A compress wave (up to kMaxUnits units of identical shape) runs four kernels on the
-// caller's stream: the forward DCT along S (axis_s.cu), the forward DCT along H and W with
-// per-bin energy sums (axis_hw.cu, kStats), the per-unit allocation and payload header
-// (allocate.cu) and the H/W pass again with quantization and packing (axis_hw.cu, kQuant),
-// which reads the S-transformed volume kept in the workspace.  A decompress wave runs the
-// inverse H/W pass (dequantize + inverse DCT along W and H) and the inverse DCT along S.
+// A compress wave (up to kMaxUnits units of identical shape) runs five kernels on the caller's
+// stream: the forward DCT along S (axis_s.cu), the forward DCT along H and W with per-bin energy
+// sums (axis_hw.cu, kStats), the variance reduction and the per-unit allocation with the payload
+// header and slab offsets (allocate.cu), and the H/W pass again with quantization and packing
+// (axis_hw.cu, kQuant), which reads the S-transformed volume kept in the workspace.  A decompress
+// wave runs the decoding index (allocate.cu: header checks, slab offsets), the inverse H/W pass
+// (dequantize + inverse DCT along W and H) and the inverse DCT along S.
 #include <algorithm>
 #include <cstring>
 #include <mutex>
@@ -18,9 +19,10 @@ namespace tactkv {
 cudaError_t launch_axis_s_16(bool, const Geom&, const UnitList&, int, float*, cudaStream_t);
 cudaError_t launch_axis_s_32(bool, const Geom&, const UnitList&, int, float*, cudaStream_t);
 cudaError_t launch_axis_s_64(bool, const Geom&, const UnitList&, int, float*, cudaStream_t);
-#define TACTKV_DECL_HW(h, w)                                                                                   \
-  cudaError_t launch_axis_hw_##h##_##w(bool, int, const Geom&, const UnitList&, int, float*, float*, unsigned int*, \
-                                       cudaStream_t);
+#define TACTKV_DECL_HW(h, w)                                                                                 \
+  cudaError_t launch_axis_hw_##h##_##w(bool, int, const Geom&, const UnitList&, int, float*, float*, const uint32_t*, \
+                                       int, cudaStream_t);                                                            \
+  void axis_hw_shape_##h##_##w(const Geom&, bool, int, size_t*, int*);
 TACTKV_DECL_HW(16, 16)
 TACTKV_DECL_HW(16, 32)
 TACTKV_DECL_HW(32, 16)
@@ -35,11 +37,18 @@ cudaError_t launch_axis_s(int cls, bool inverse, const Geom& g, const UnitList& 
 }
 
 cudaError_t launch_axis_hw(int hcls, int wcls, bool inverse, int mode, const Geom& g, const UnitList& ul, int nu,
-                           float* buf, float* partial, unsigned int* status, cudaStream_t st) {
-  if (hcls == 16 && wcls == 16) return launch_axis_hw_16_16(inverse, mode, g, ul, nu, buf, partial, status, st);
-  if (hcls == 16) return launch_axis_hw_16_32(inverse, mode, g, ul, nu, buf, partial, status, st);
-  if (wcls == 16) return launch_axis_hw_32_16(inverse, mode, g, ul, nu, buf, partial, status, st);
-  return launch_axis_hw_32_32(inverse, mode, g, ul, nu, buf, partial, status, st);
+                           float* buf, float* partial, const uint32_t* slab_off, int spc, cudaStream_t st) {
+  if (hcls == 16 && wcls == 16) return launch_axis_hw_16_16(inverse, mode, g, ul, nu, buf, partial, slab_off, spc, st);
+  if (hcls == 16) return launch_axis_hw_16_32(inverse, mode, g, ul, nu, buf, partial, slab_off, spc, st);
+  if (wcls == 16) return launch_axis_hw_32_16(inverse, mode, g, ul, nu, buf, partial, slab_off, spc, st);
+  return launch_axis_hw_32_32(inverse, mode, g, ul, nu, buf, partial, slab_off, spc, st);
+}
+
+void axis_hw_shape(int hcls, int wcls, const Geom& g, bool inverse, int mode, size_t* smem, int* threads) {
+  if (hcls == 16 && wcls == 16) return axis_hw_shape_16_16(g, inverse, mode, smem, threads);
+  if (hcls == 16) return axis_hw_shape_16_32(g, inverse, mode, smem, threads);
+  if (wcls == 16) return axis_hw_shape_32_16(g, inverse, mode, smem, threads);
+  return axis_hw_shape_32_32(g, inverse, mode, smem, threads);
 }
 
 namespace {
@@ -78,16 +87,19 @@ size_t payload_bytes_geom(const Geom& g) {
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
-// workspace of one unit: the S-transformed volume (fp32), per-chunk energy sums, fp64 variances
+// workspace of one unit: the S-transformed volume (fp32), per-chunk energy sums, fp64 variances,
+// slab offsets P(0..S) and the decoder's ok flag
 size_t unit_ws_bytes(const Geom& g) {
-  return round256((size_t)g.T * g.n * 4) + round256((size_t)g.nch * g.N * 4) + round256((size_t)g.N * 8);
+  return round256((size_t)g.T * g.n * 4) + round256((size_t)g.nch * g.N * 4) + round256((size_t)g.N * 8) +
+         round256((size_t)(g.S + 2) * 4);
 }
 
 struct WsView {
   unsigned int* status;
-  float* big;      // nu * T * n floats: Y (compress) or V (decompress)
-  float* partial;  // nu * nch * N floats
-  double* var;     // nu * N doubles
+  float* big;         // nu * T * n floats: Y (compress) or V (decompress)
+  float* partial;     // nu * nch * N floats
+  double* var;        // nu * N doubles
+  uint32_t* slab_off; // nu * (S + 2) words
 };
 
 WsView view(unsigned char* ws, const Geom& g, int nu) {
@@ -99,7 +111,26 @@ WsView view(unsigned char* ws, const Geom& g, int nu) {
   v.partial = reinterpret_cast<float*>(ws + off);
   off += round256((size_t)nu * g.nch * g.N * 4);
   v.var = reinterpret_cast<double*>(ws + off);
+  off += round256((size_t)nu * g.N * 8);
+  v.slab_off = reinterpret_cast<uint32_t*>(ws + off);
   return v;
+}
+
+// Slabs per CTA of the H/W passes: whole units when the batch alone fills the GPU a couple of
+// times over, shorter slab ranges (more CTAs) for small batches.
+int slabs_per_cta(const Geom& g, int nu, bool inverse, int mode) {
+  size_t smem = 0;
+  int threads = 32;
+  axis_hw_shape(length_class(g.H), length_class(g.W), g, inverse, mode, &smem, &threads);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int by_smem = (int)((228 * 1024) / (smem + 1024));
+  const int by_threads = 2048 / threads;
+  const int occ = std::max(1, std::min(by_smem, by_threads));
+  const long long target = 2LL * sms * occ;
+  const long long have = (long long)g.nch * nu;
+  const int ranges = (int)std::min<long long>(g.S, std::max<long long>(1, (target + have - 1) / have));
+  return (g.S + ranges - 1) / ranges;
 }
 
 bool same_group(const tactkv_unit& a, const tactkv_unit& b) {
@@ -236,14 +267,15 @@ static tactkv_status compress_impl(const tactkv_unit* units, int n_units, void* 
                          mark(0);
                          if (launch_axis_s(cs, false, g, ul, nu, w.big, st) != cudaSuccess) return TACTKV_CUDA;
                          mark(1);
-                         if (launch_axis_hw(ch, cw, false, kStats, g, ul, nu, w.big, w.partial, w.status, st) !=
-                             cudaSuccess)
+                         if (launch_axis_hw(ch, cw, false, kStats, g, ul, nu, w.big, w.partial, w.slab_off,
+                                            slabs_per_cta(g, nu, false, kStats), st) != cudaSuccess)
                            return TACTKV_CUDA;
                          mark(2);
-                         if (launch_allocate(g, ul, nu, w.partial, w.var, st) != cudaSuccess) return TACTKV_CUDA;
+                         if (launch_allocate(g, ul, nu, w.partial, w.var, w.slab_off, st) != cudaSuccess)
+                           return TACTKV_CUDA;
                          mark(3);
-                         if (launch_axis_hw(ch, cw, false, mode2, g, ul, nu, w.big, w.partial, w.status, st) !=
-                             cudaSuccess)
+                         if (launch_axis_hw(ch, cw, false, mode2, g, ul, nu, w.big, w.partial, w.slab_off,
+                                            slabs_per_cta(g, nu, false, mode2), st) != cudaSuccess)
                            return TACTKV_CUDA;
                          mark(4);
                          return TACTKV_OK;
@@ -261,7 +293,10 @@ static tactkv_status decompress_impl(const tactkv_unit* units, int n_units, void
                          const int cs = length_class(g.S), ch = length_class(g.H), cw = length_class(g.W);
                          const int mode = (g.flags & TACTKV_NO_QUANT) ? kRaw : kQuant;
                          mark(0);
-                         if (launch_axis_hw(ch, cw, true, mode, g, ul, nu, w.big, nullptr, w.status, st) != cudaSuccess)
+                         if (launch_decode_index(g, ul, nu, w.slab_off, w.status, st) != cudaSuccess)
+                           return TACTKV_CUDA;
+                         if (launch_axis_hw(ch, cw, true, mode, g, ul, nu, w.big, nullptr, w.slab_off,
+                                            slabs_per_cta(g, nu, true, mode), st) != cudaSuccess)
                            return TACTKV_CUDA;
                          mark(1);
                          if (launch_axis_s(cs, true, g, ul, nu, w.big, st) != cudaSuccess) return TACTKV_CUDA;

@@ -103,3 +103,42 @@ def test_workspace_checks_without_gpu(T):
 def test_decompress_checks_output_pointer(T):
     units = [_unit(T, kv_out=None)]
     assert T.tactkv_decompress(units, 1 << 20, 1 << 30, 0) == T.TACTKV_INVALID_ARG
+
+
+# ------------------------------------------------------------ code lookup of the quantizer ---
+def _gen_tables():
+    import importlib.util
+    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                        "dct_transform_coding_b200", "csrc", "gen_tables.py")
+    spec = importlib.util.spec_from_file_location("gen_tables", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+@pytest.mark.parametrize("bits", range(3, 9))
+def test_cell_table_code_lookup_equals_threshold_count(bits):
+    """The kernels' code lookup for b >= 3 (cell of u, table count, two compares), emulated in
+    float32 exactly as the device computes it, equals the number of float32 thresholds <= u for
+    values on, next to and between every threshold, far outside the range, and at +-0."""
+    G = _gen_tables()
+    lv, th = G.codebook(bits)
+    th32 = np.array(th, dtype=np.float32)
+    tab, scale, offset = G.code_table([float(t) for t in th32])
+    tab = np.array(tab)
+    padded = np.concatenate([th32, np.array([np.inf, np.inf], np.float32)])
+    rng = np.random.default_rng(bits)
+    u = [th32, np.nextafter(th32, np.float32(np.inf)), np.nextafter(th32, np.float32(-np.inf)),
+         rng.uniform(-6, 6, 200000).astype(np.float32), rng.standard_normal(200000).astype(np.float32) * 3,
+         np.array([0.0, -0.0, 4.5, -4.5, 1e30, -1e30, 1e-40, -1e-40], np.float32)]
+    for k in range(2, 6):   # a few ulps on both sides of every threshold
+        u.append(th32 + np.float32(k) * np.spacing(th32))
+        u.append(th32 - np.float32(k) * np.spacing(th32))
+    u = np.concatenate(u).astype(np.float32)
+    # fmaf(u, scale, offset): u*scale + offset is exact in float64, so one rounding to float32
+    jf = (u.astype(np.float64) * np.float64(np.float32(scale)) + np.float64(np.float32(offset))).astype(np.float32)
+    j = np.clip(np.floor(jf.astype(np.float64)), 0, G.QK - 1).astype(np.int64)
+    c = tab[j]
+    code = c + (u >= padded[c]) + (u >= padded[c + 1])
+    want = np.searchsorted(th32, u, side="right")
+    assert np.array_equal(code, want)
