@@ -287,7 +287,7 @@ def main():
     ms_step = elapsed_ms / args.steps
 
     # per-kernel averages from the bracketing events
-    names_c = ["fdct_s", "fdct_hw_stats", "reduce_var+allocate", "fdct_hw_quant"]
+    names_c = ["fdct_s", "fdct_hw_stats", "reduce_var+allocate", "pack"]
     names_d = ["idct_hw", "idct_s"]
     kern = {n: statistics.mean(evs_c[k][i].elapsed_time(evs_c[k][i + 1]) for k in range(args.steps))
             for i, n in enumerate(names_c)}
@@ -308,9 +308,12 @@ def main():
         w = dataclasses.replace(w, sequences=1, layers=U, kv=(0,))   # describe what actually ran
     achieved = (alg_c + alg_d) / (ms_step * 1e-3) / 1e9
     n_el = U * Tk * heads * D
-    # the kernels' own DRAM needs in this design (fp32 scratch between the axis passes)
-    own = {"fdct_s": n_el * (2 + 4), "fdct_hw_stats": n_el * 4 + U * (heads * D // 32) * Tk * 4,
-           "reduce_var+allocate": U * (heads * D // 32) * Tk * 4, "fdct_hw_quant": n_el * 4 + pay_bytes,
+    # the kernels' own DRAM needs in this design (fp32 volume between the axis passes; the packing
+    # kernel reads the coefficients of the bins with bits only)
+    nz_bins = int((payload[:, 64:64 + Tk] > 0).sum().item())
+    chunk_partials = U * (heads * D // 32) * Tk * 4
+    own = {"fdct_s": n_el * (2 + 4), "fdct_hw_stats": n_el * (4 + 4) + chunk_partials,
+           "reduce_var+allocate": chunk_partials + U * Tk * 16, "pack": nz_bins * heads * D * 4 + pay_bytes,
            "idct_hw": pay_bytes + n_el * 4, "idct_s": n_el * (4 + 2)}
     dominant = max(kern, key=kern.get)
     kernels = {n: {"ms": round(kern[n], 4), "share": round(kern[n] / (ms_c + ms_d), 4),

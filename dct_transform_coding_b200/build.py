@@ -30,6 +30,7 @@ UNITS = [
     ("axis_hw_32_16", "axis_hw.cu", ["-DTACTKV_HCLASS=32", "-DTACTKV_WCLASS=16"]),
     ("axis_hw_32_32", "axis_hw.cu", ["-DTACTKV_HCLASS=32", "-DTACTKV_WCLASS=32"]),
     ("allocate", "allocate.cu", []),
+    ("pack", "pack.cu", []),
     ("tactkv", "tactkv.cu", []),
 ]
 

@@ -15,8 +15,9 @@
 // If the active bins cannot absorb B (8 * #active <= B) every active bin gets 8 bits.
 //
 // The kernel also writes the first stream bit P(k_s) of every S slab (the same for every
-// channel) into the workspace and zeroes the stream word holding each P(k_s): the packing kernel
-// ORs the words it shares with a neighbouring slab range into those.  decode_index_kernel
+// channel) and the list of bins with bits (records {bin, bits, first stream bit, 1/sigma}, in bin
+// order) into the workspace, and zeroes the stream word where each packing range of kPackRecs
+// records starts: the packing kernel ORs the words it shares with a neighbouring range into those.  decode_index_kernel
 // rebuilds P from a payload before decoding and checks the header and the bit widths.
 #include "common.cuh"
 
@@ -105,13 +106,16 @@ __device__ void slab_scan(const uint32_t* s_slab, int S, uint32_t* out) {
 __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_constant__ Geom g,
                                                                  const __grid_constant__ UnitList ul,
                                                                  double* __restrict__ var_ws, bool var_in_smem,
-                                                                 uint32_t* __restrict__ slab_off) {
+                                                                 uint32_t* __restrict__ index, uint4* __restrict__ recs) {
   __shared__ long long s_ll[32];
   __shared__ double s_d[32];
   __shared__ uint32_t s_scan[33];
   __shared__ uint32_t s_cnt[kAllocThreads];
   __shared__ uint32_t s_slab[kMaxSlabs];
+  __shared__ uint32_t s_nzslab[kMaxSlabs];
   __shared__ uint32_t s_P[kMaxSlabs + 1];
+  __shared__ uint32_t s_NZ[kMaxSlabs + 1];
+  __shared__ uint32_t s_bpos[kMaxN / kPackRecs + 1];
   extern __shared__ __align__(16) unsigned char smem_var[];
   const int u = blockIdx.x;
   const UnitDev& ud = ul.u[u];
@@ -127,7 +131,9 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
   long long act = 0;
   double vmax = 0.0;
   const double* var_g = var_ws + (size_t)u * g.N;
-  for (int i = beg; i < end; ++i) {
+  // the counting passes take bins interleaved across threads (bin i to thread i mod blockDim):
+  // consecutive threads read consecutive variances, without bank conflicts
+  for (int i = threadIdx.x; i < g.N; i += blockDim.x) {
     const double v = var_g[i];
     var[i] = v;
     act += v > 0.0;
@@ -146,7 +152,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
       const unsigned long long mid = lo + (hi - lo) / 2;
       const double v = __longlong_as_double((long long)mid);
       long long c = 0;
-      for (int i = beg; i < end; ++i) {
+      for (int i = threadIdx.x; i < g.N; i += blockDim.x) {
         const double x = var[i];
         if (x > 0.0) c += key_count(x, v);
       }
@@ -177,10 +183,13 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
   block_exclusive_scan(s_cnt, blockDim.x, s_scan);
   long long rank = s_cnt[threadIdx.x];
   long long code_bits_local = 0;
-  for (int k = threadIdx.x; k < g.S; k += blockDim.x) s_slab[k] = 0;
+  for (int k = threadIdx.x; k < g.S; k += blockDim.x) {
+    s_slab[k] = 0;
+    s_nzslab[k] = 0;
+  }
   __syncthreads();
   int ks = beg / g.HW, in_slab = beg - ks * g.HW;   // slab of bin i, walked incrementally
-  uint32_t slab_sum = 0;
+  uint32_t slab_sum = 0, slab_nz = 0, my_nz = 0;
   for (int i = beg; i < end; ++i) {
     const double x = var[i];
     int b = 0;
@@ -199,9 +208,13 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
     reinterpret_cast<float*>(pay + g.off_sigma)[i] = (float)sqrt(x);
     code_bits_local += b;
     slab_sum += b;
+    slab_nz += b > 0;
+    my_nz += b > 0;
     if (++in_slab == g.HW || i + 1 == end) {
       if (slab_sum) atomicAdd(&s_slab[ks], slab_sum);
+      if (slab_nz) atomicAdd(&s_nzslab[ks], slab_nz);
       slab_sum = 0;
+      slab_nz = 0;
       in_slab = 0;
       ++ks;
     }
@@ -211,12 +224,51 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
   for (int i = g.off_sigma + 4 * g.N + threadIdx.x; i < g.off_codes; i += blockDim.x) pay[i] = 0;
   const long long code_bits = raw ? 32LL * g.N : block_sum<long long>(code_bits_local, s_ll);
   const long long cstride = pad16((code_bits + 7) / 8);
-  // slab offsets P(k_s), and a zero in the stream word at every P(k_s) of every channel
+  // slab offsets P(k_s) and record offsets NZ(k_s), and a zero in the stream word at every P(k_s)
+  // of every channel
   __syncthreads();
   if (threadIdx.x < 32) slab_scan(s_slab, g.S, s_P);
+  else if (threadIdx.x < 64) slab_scan(s_nzslab, g.S, s_NZ);
   __syncthreads();
-  uint32_t* P = slab_off + (size_t)u * (g.S + 2);
-  for (int k = threadIdx.x; k <= g.S; k += blockDim.x) P[k] = raw ? 0u : s_P[k];
+  uint32_t* P = index + (size_t)u * unit_index_words(g.S);
+  uint32_t* NZ = P + g.S + 2;
+  for (int k = threadIdx.x; k <= g.S; k += blockDim.x) {
+    P[k] = raw ? 0u : s_P[k];
+    NZ[k] = raw ? 0u : s_NZ[k];
+  }
+  // the records of the bins with bits, in bin order: {bin, bits, P_i, 1/sigma_i}
+  if (!raw) {
+    s_cnt[threadIdx.x] = my_nz;
+    __syncthreads();
+    block_exclusive_scan(s_cnt, blockDim.x, s_scan);
+    uint32_t slot = s_cnt[threadIdx.x];
+    __syncthreads();
+    s_cnt[threadIdx.x] = (uint32_t)code_bits_local;
+    __syncthreads();
+    block_exclusive_scan(s_cnt, blockDim.x, s_scan);
+    uint32_t pos = s_cnt[threadIdx.x];
+    uint4* urecs = recs + (size_t)u * g.N;
+    const float* sig = reinterpret_cast<const float*>(pay + g.off_sigma);
+    for (int i = beg; i < end; ++i) {
+      const uint32_t b = pay[kHeaderBytes + i];
+      if (b) {
+        if (slot % kPackRecs == 0) s_bpos[slot / kPackRecs] = pos;   // a packing range starts here
+        urecs[slot++] = make_uint4((uint32_t)i, b, pos, __float_as_uint(__frcp_rn(sig[i])));
+        pos += b;
+      }
+    }
+    __syncthreads();
+    // zero the stream word where each packing range starts and the word holding the last code bit:
+    // neighbouring ranges OR their bits into them
+    const uint32_t sw = (uint32_t)(cstride / 4), nrec = s_NZ[g.S];
+    const uint32_t nb = (nrec + kPackRecs - 1) / kPackRecs;
+    uint32_t* words = reinterpret_cast<uint32_t*>(pay + g.off_codes);
+    for (uint32_t k = 0; k <= nb; ++k) {
+      const uint32_t w = (k < nb ? s_bpos[k] : s_P[g.S]) >> 5;
+      if (w < sw)
+        for (int c = threadIdx.x; c < g.n; c += blockDim.x) words[(size_t)c * sw + w] = 0u;
+    }
+  }
   if (!raw) {
     const uint32_t sw = (uint32_t)(cstride / 4);
     uint32_t* words = reinterpret_cast<uint32_t*>(pay + g.off_codes);
@@ -253,7 +305,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
 // width must be <= 8 and their sum must equal the header's code_bits; then P(k_s) is rebuilt.
 __global__ void __launch_bounds__(256) decode_index_kernel(const __grid_constant__ Geom g,
                                                            const __grid_constant__ UnitList ul,
-                                                           uint32_t* __restrict__ slab_off, unsigned int* status) {
+                                                           uint32_t* __restrict__ index, unsigned int* status) {
   __shared__ int s_ok;
   __shared__ uint32_t s_slab[kMaxSlabs];
   __shared__ uint32_t s_P[kMaxSlabs + 1];
@@ -300,7 +352,7 @@ __global__ void __launch_bounds__(256) decode_index_kernel(const __grid_constant
     __syncthreads();
     ok = s_ok;
   }
-  uint32_t* P = slab_off + (size_t)u * (g.S + 2);
+  uint32_t* P = index + (size_t)u * unit_index_words(g.S);
   for (int k = threadIdx.x; k <= g.S; k += blockDim.x) P[k] = (ok && !raw) ? s_P[k] : 0u;
   if (threadIdx.x == 0) {
     P[g.S + 1] = ok ? 1u : 0u;
@@ -310,19 +362,19 @@ __global__ void __launch_bounds__(256) decode_index_kernel(const __grid_constant
 
 }  // namespace
 
-cudaError_t launch_decode_index(const Geom& g, const UnitList& ul, int nu, uint32_t* slab_off, unsigned int* status,
+cudaError_t launch_decode_index(const Geom& g, const UnitList& ul, int nu, uint32_t* index, unsigned int* status,
                                 cudaStream_t st) {
-  decode_index_kernel<<<nu, 256, 0, st>>>(g, ul, slab_off, status);
+  decode_index_kernel<<<nu, 256, 0, st>>>(g, ul, index, status);
   return cudaGetLastError();
 }
 
 cudaError_t launch_allocate(const Geom& g, const UnitList& ul, int nu, const float* partial, double* var,
-                            uint32_t* slab_off, cudaStream_t st) {
+                            uint32_t* index, uint4* recs, cudaStream_t st) {
   const size_t var_bytes = (size_t)g.N * sizeof(double);
   const bool in_smem = var_bytes <= kAllocSmemVar;
   if (in_smem) cudaFuncSetAttribute(allocate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)var_bytes);
   reduce_var_kernel<<<dim3((g.N + 255) / 256, nu), 256, 0, st>>>(g, partial, var);
-  allocate_kernel<<<nu, kAllocThreads, in_smem ? var_bytes : 0, st>>>(g, ul, var, in_smem, slab_off);
+  allocate_kernel<<<nu, kAllocThreads, in_smem ? var_bytes : 0, st>>>(g, ul, var, in_smem, index, recs);
   return cudaGetLastError();
 }
 

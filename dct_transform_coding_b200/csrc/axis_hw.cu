@@ -1,32 +1,23 @@
-// DCT along the H and W axes plus the per-bin epilogues (TACT-KV stages 2-4 and their inverse).
+// DCT along the H and W axes (TACT-KV stage 2, after the S pass) with the per-bin energies of
+// stage 3, and the inverse with unpacking and dequantization (the decoding paragraph).
 //
 // A CTA owns one (unit, 32-channel chunk, range of S slabs) and walks its slabs in order.  Lane l
 // of every warp is channel l of the chunk, and a thread's float2 holds two pencils of that
 // channel: two columns (w, w+1) in the pass along H, two rows (h, h+1) in the pass along W.  All
 // lanes of a warp therefore work on the same frequency bins at the same time, and everything that
-// depends on a bin (its bit width, its gain, where its code goes in the stream) is uniform across
-// the warp: no lane waits for another lane's branch.
+// depends on a bin (its bit width, its gain, where its code sits in the stream) is uniform across
+// the warp.
 //
-// Forward, per slab k_s:
-//   1. the slab's H*W x 32 coefficients of the S-transformed volume Y arrive by cp.async, and the
-//      next slab's coefficients, bit widths and gains are fetched meanwhile;
-//   2. DCT along H in place: a warp reads a column pair, transforms it and writes it back into the
-//      same bytes as row pairs (float2 = rows 2i, 2i+1 of one column and channel);
-//   3. DCT along W: warp j takes row pair j, then
-//        kStats  squares, sums over the 32 channels -> partial[u][chunk][bin]   (pass 1)
-//        kQuant  u = X * (1/sigma_i), Lloyd-Max code at b_i bits, appended to the channel's stream
-//        kRaw    float32 coefficients into the streams (TACTKV_NO_QUANT)
-// A channel's codes of slab k_s occupy stream bits [P(k_s), P(k_s+1)) (the allocation writes P);
-// a warp finds its rows' offsets by summing the slab's bit widths before them.  Words are
-// assembled in shared memory and complete words are stored once; the word that straddles two
-// slabs is carried to the next slab.  The first and the last word of the CTA's slab range may
-// hold bits of the neighbouring ranges and are ORed into the payload atomically (the allocation
-// zeroes the word at every P(k_s) first).
+// Forward (fdct_hw), per slab k_s: the slab's H*W x 32 coefficients of the S-transformed volume
+// arrive by cp.async (the next slab's meanwhile); the DCT along H runs in place (a warp reads a
+// column pair and writes it back into the same bytes as row pairs); the DCT along W runs on row
+// pairs, writes the finished coefficients X back over the slab in global memory and sums X^2 over
+// the 32 channels into partial[u][chunk][bin].
 //
 // Inverse (idct_hw), per slab: the slab's stream words arrive by cp.async (next slab prefetched);
-// warp j decodes rows 2j and 2j+1 (unpack + dequantize in registers), runs the inverse DCT along W
-// and writes column pairs; warp j then runs the inverse DCT along H on column pair j and stores
-// the result into the fp32 volume V.
+// per-bin records give each bin's bits, gain and stream position; warp j decodes rows 2j and 2j+1
+// (unpack + dequantize in registers), runs the inverse DCT along W and writes column pairs; then
+// runs the inverse DCT along H on column pair j and stores the result into the fp32 volume V.
 //
 // Compiled once per pair of length classes (TACTKV_HCLASS, TACTKV_WCLASS: 16 or 32 each).
 #include "common.cuh"
@@ -41,10 +32,10 @@ namespace {
 
 constexpr size_t kSmemBudget = 220 * 1024;
 
-enum LayoutKind { kLayStats = 0, kLayQuant = 1, kLayDecode = 2 };
+enum LayoutKind { kLayStats = 0, kLayDecode = 2 };
 
 struct HwLayout {
-  size_t tile, tile_bytes, sbuf, meta, bsl, bsl_stride, sig, thr, qcell, lv, carry, total;
+  size_t tile, tile_bytes, sbuf, meta, bsl, bsl_stride, sig, lv, total;
   int nbuf, words;
 };
 
@@ -58,33 +49,26 @@ __host__ __device__ inline int hw_threads(int H, int W) {
   return m < kMaxHwThreads ? m : kMaxHwThreads;
 }
 
-// Thresholds of width b padded with two +inf, stored for b = 1, 2, ... in turn.
-__device__ __forceinline__ int thr_pad_offset(int b) { return (1 << b) + b - 3; }
-
 // Shared memory of one launch.  A tile buffer holds a slab as cells of 32 floats on a grid of
 // 2*ceil(H/2) rows of Wp = 2*ceil(W/2) cells (the padding row and column are never read), which
-// also holds its row-pair (forward) or column-pair (inverse) rearrangement.  stats: the slab
-// tiles only (the energies reuse the rearranged tile).  quant: tiles, one
-// slab of stream words, per-bin records, bit widths and sigmas of two slabs, padded thresholds,
-// code table, carried words.  decode: one tile, two slabs of stream words, records, widths and
-// sigmas of two slabs, levels.  words (the stride of a channel's word row) is odd, so the 32 lanes
-// writing 32 channels' rows hit 32 different banks.
+// also holds its row-pair (forward) or column-pair (inverse) rearrangement.  stats: the slab tiles
+// (two when they fit, so the next slab loads while this one is transformed; the energies reuse
+// the rearranged tile).  decode: one tile, two slabs of stream words, per-bin records, bit widths
+// and sigmas of two slabs, levels.  words (the stride of a channel's word row) is odd, so the 32
+// lanes reading 32 channels' rows hit 32 different banks.
 __host__ __device__ inline HwLayout hw_layout(int H, int W, int kind) {
   HwLayout L;
   const int HP = row_pairs(H), WP = row_pairs(W), HW = H * W;
-  const bool st = kind == kLayStats, qu = kind == kLayQuant, de = kind == kLayDecode;
+  const bool de = kind == kLayDecode;
   L.tile_bytes = (size_t)(2 * HP) * (2 * WP) * 32 * 4;
   L.words = ((8 * HW + 31) / 32 + 3) | 1;
-  const size_t words = st ? 0 : (size_t)32 * L.words * 4 * (de ? 2 : 1);
-  const size_t meta = st ? 0 : (size_t)HP * W * 16;
+  const size_t words = de ? (size_t)32 * L.words * 4 * 2 : 0;
+  const size_t meta = de ? (size_t)HP * W * 16 : 0;
   L.bsl_stride = ((size_t)HW + 15) / 16 * 16 + 32;
-  const size_t bsl = st ? 0 : 2 * L.bsl_stride;
-  const size_t sig = st ? 0 : (size_t)2 * HW * 4;
-  const size_t thr = qu ? TACTKV_THR_PAD_TOTAL * 4 : 0;
-  const size_t qcell = qu ? ((size_t)6 * TACTKV_Q_CELLS + 15) / 16 * 16 : 0;
+  const size_t bsl = de ? 2 * L.bsl_stride : 0;
+  const size_t sig = de ? (size_t)2 * HW * 4 : 0;
   const size_t lv = de ? kLmLvTotal * 4 : 0;
-  const size_t carry = qu ? kChunk * 4 : 0;
-  const size_t rest = words + meta + bsl + sig + thr + qcell + lv + carry + 256;
+  const size_t rest = words + meta + bsl + sig + lv + 256;
   L.nbuf = (de || 2 * L.tile_bytes + rest > kSmemBudget) ? 1 : 2;
   // every region starts on a 16-byte boundary (cp.async of 16 bytes, 16-byte record loads)
   auto p16 = [](size_t x) { return (x + 15) / 16 * 16; };
@@ -93,11 +77,8 @@ __host__ __device__ inline HwLayout hw_layout(int H, int W, int kind) {
   L.sbuf = o; o += p16(words);
   L.meta = o; o += p16(meta);
   L.sig = o; o += p16(sig);
-  L.thr = o; o += p16(thr);
   L.lv = o; o += p16(lv);
-  L.carry = o; o += p16(carry);
   L.bsl = o; o += p16(bsl);
-  L.qcell = o; o += p16(qcell);
   L.total = o;
   return L;
 }
@@ -118,49 +99,6 @@ template <int CLASS, int EXACT, bool INV, class V>
 __device__ __forceinline__ void pencil(V* x, int L) {
   if constexpr (EXACT > 0) dct_exact<EXACT, INV>(x);
   else dct_pencil<CLASS, INV>(x, L);
-}
-
-// Code of u at b bits: the number of thresholds t_j <= u (float32 compares, ties go up).  b = 1:
-// the sign test; b = 2: three compares against {-t, 0, t}; b >= 3: the cell of u in a uniform grid
-// gives the count c of thresholds below the cell, and two compares finish it (a cell holds at most
-// two thresholds; the thresholds are padded with +inf).
-__device__ __forceinline__ uint32_t quant_code(float u, int b, const float* thr, const unsigned char* qcell) {
-  if (b == 1) return u >= 0.f;
-  if (b == 2) {
-    const float t = thr[thr_pad_offset(2) + 2];
-    return (uint32_t)(u >= -t) + (uint32_t)(u >= 0.f) + (uint32_t)(u >= t);
-  }
-  int j = __float2int_rd(fmaf(u, TACTKV_Q_SCALE, TACTKV_Q_OFFSET));
-  j = min(max(j, 0), TACTKV_Q_CELLS - 1);
-  const uint32_t c = qcell[(b - 3) * TACTKV_Q_CELLS + j];
-  const float* t = thr + thr_pad_offset(b) + c;
-  return c + (uint32_t)(u >= t[0]) + (uint32_t)(u >= t[1]);
-}
-
-// Append a b-bit code (b >= 1) at stream position p of a channel's word row; full words are ORed
-// into shared memory (a word may be shared with the neighbouring row, which another warp fills).
-__device__ __forceinline__ void put_code(uint32_t& acc, uint32_t& p, uint32_t code, int b, uint32_t* row) {
-  const uint32_t s = p & 31u;
-  acc |= code << s;
-  if (s + b >= 32) {          // b <= 8, so s >= 24 here and the shift below is 1..8
-    atomicOr(row + (p >> 5), acc);
-    acc = code >> (32 - s);
-  }
-  p += b;
-}
-
-// Read a b-bit code (b >= 1) at the reader's position and advance (64-bit window lo:hi).
-__device__ __forceinline__ uint32_t get_code(uint32_t& lo, uint32_t& hi, uint32_t& s, uint32_t& wi, int b,
-                                             const uint32_t* row) {
-  const uint32_t code = __funnelshift_r(lo, hi, s) & ((1u << b) - 1u);
-  s += b;
-  if (s >= 32) {
-    s -= 32;
-    lo = hi;
-    ++wi;
-    hi = row[wi + 1];
-  }
-  return code;
 }
 
 // Copy one S slab of Y (H*W cells of 32 channels, 128 bytes each) into a tile with rows of Wp
@@ -186,36 +124,42 @@ __device__ __forceinline__ void issue_sigma(const D& g, const float* pay_sig, in
 }
 
 // Per-bin records of slab ks, one 16-byte record per (row pair, w): {gain of row 2i, gain of row
-// 2i+1, bits of row 2i | bits of row 2i+1 << 8}.  gain = 1/sigma (encoding) or sigma (decoding);
-// rows past H (odd H) get 0 bits.
+// 2i+1, stream position of row 2i's code << 4 | its bits, the same for row 2i+1}.  gain = 1/sigma
+// (encoding) or sigma (decoding).  The position counts from bit pbase of the slab's first word:
+// the bits of every bin before it in the slab, found by a sum over the earlier rows and a warp scan
+// along the row.  Rows past H (odd H) get 0 bits.
 template <class D>
 __device__ __forceinline__ void slab_records(const D& g, const unsigned char* bs, const float* sig, bool inv,
-                                             unsigned char* meta) {
+                                             unsigned char* meta, uint32_t pbase) {
   const int lane = threadIdx.x & 31, nwarps = blockDim.x >> 5, HP2 = 2 * row_pairs(g.H);
-  for (int kh = threadIdx.x >> 5; kh < HP2; kh += nwarps)
-    for (int t = lane; t < g.W; t += 32) {
-      const int i = kh * g.W + t;
-      const uint32_t b = kh < g.H ? bs[i] : 0u;
+  for (int kh = threadIdx.x >> 5; kh < HP2; kh += nwarps) {
+    const bool real = kh < g.H;
+    const int i = kh * g.W + lane;
+    const uint32_t b = (real && lane < g.W) ? bs[i] : 0u;
+    uint32_t before = 0;
+    const int lim = real ? kh * g.W : 0;
+    for (int q = lane; q < lim; q += 32) before += bs[q];
+    before = __reduce_add_sync(0xffffffffu, before);
+    uint32_t incl = b;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    if (lane < g.W) {
       float gv = 0.f;
       if (b) gv = inv ? __frcp_rn(sig[i]) : sig[i];
-      unsigned char* rec = meta + ((size_t)(kh >> 1) * g.W + t) * 16;
-      reinterpret_cast<float*>(rec)[kh & 1] = gv;
-      rec[8 + (kh & 1)] = (unsigned char)b;
+      uint32_t* rec = reinterpret_cast<uint32_t*>(meta + ((size_t)(kh >> 1) * g.W + lane) * 16);
+      rec[kh & 1] = __float_as_uint(gv);
+      rec[2 + (kh & 1)] = ((pbase + before + incl - b) << 4) | b;
     }
+  }
 }
 
-// Stream positions (relative to the slab's first word) of rows 2kp and 2kp+1, for one warp.
-template <class D>
-__device__ __forceinline__ void row_positions(const D& g, const unsigned char* bs, int kp, uint32_t base,
-                                              uint32_t& p0, uint32_t& p1) {
-  const int lane = threadIdx.x & 31, lim = 2 * kp * g.W;
-  uint32_t before = 0, row0 = 0;
-  for (int i = lane; i < lim; i += 32) before += bs[i];
-  for (int i = lane; i < g.W; i += 32) row0 += bs[lim + i];
-  before = __reduce_add_sync(0xffffffffu, before);
-  row0 = __reduce_add_sync(0xffffffffu, row0);
-  p0 = base + before;
-  p1 = p0 + row0;
+// The b-bit code at bit position off of a channel's word row (b >= 1).
+__device__ __forceinline__ uint32_t read_code(const uint32_t* row, uint32_t off, uint32_t b) {
+  const uint32_t w = off >> 5;
+  return __funnelshift_r(row[w], row[w + 1], off & 31u) & ((1u << b) - 1u);
 }
 
 // Forward rearrangement.  The tile's cells (h, w) sit at cell index h*Wp + w.  After the pass
@@ -271,182 +215,82 @@ __device__ __forceinline__ void put_energy(const D& g, float2* t2, int kp, int l
     }
 }
 
-// ---------------------------------------------------------------------------------- forward ---
 // Register budget: class-16 pencils fit two CTAs of 256 threads per SM; class-32 float2 pencils
 // need more than 128 registers.
 constexpr int kHwMinBlocks = (TACTKV_HCLASS == 16 && TACTKV_WCLASS == 16) ? 2 : 1;
 
-template <int HC, int WC, int HX, int WX, int MODE>
-__global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) fdct_hw_kernel(const __grid_constant__ Geom g, const __grid_constant__ UnitList ul,
-                                                      const float* __restrict__ Y, float* __restrict__ partial,
-                                                      const uint32_t* __restrict__ slab_off, int spc) {
+// ---------------------------------------------------------------------------------- forward ---
+// Pass 1 of compression: the 3D DCT is completed (H and W after the S pass) and written back over
+// the S-transformed slab, and the per-bin energies are summed over the CTA's 32 channels.  The
+// packing kernel then quantizes the finished coefficients without transforming anything.
+template <int HC, int WC, int HX, int WX>
+__global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) fdct_hw_kernel(const __grid_constant__ Geom g,
+                                                                              const __grid_constant__ UnitList ul,
+                                                                              float* __restrict__ Y,
+                                                                              float* __restrict__ partial, int spc) {
   extern __shared__ __align__(16) unsigned char smem[];
   const Dims<HX, WX> D(g);
-  constexpr bool quant = MODE == kQuant, raw = MODE == kRaw, stats = MODE == kStats;
-  const HwLayout L = hw_layout(D.H, D.W, stats ? kLayStats : kLayQuant);
+  const HwLayout L = hw_layout(D.H, D.W, kLayStats);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const int HP = row_pairs(D.H), WP = row_pairs(D.W);
   const int chunk = blockIdx.x, u = blockIdx.z;
   const int ks0 = blockIdx.y * spc, ks1 = min(g.S, ks0 + spc);
-  const UnitDev& ud = ul.u[u];
-  unsigned char* pay = ud.payload;
-  const float* ysrc = Y + (size_t)u * g.S * D.HW * g.n + chunk * kChunk;
-  uint32_t* sbuf = reinterpret_cast<uint32_t*>(smem + L.sbuf);
-  const uint4* meta = reinterpret_cast<const uint4*>(smem + L.meta);
-  float* thr = reinterpret_cast<float*>(smem + L.thr);
-  unsigned char* qcell = smem + L.qcell;
-  uint32_t* carry = reinterpret_cast<uint32_t*>(smem + L.carry);
-  const unsigned char* pay_b = pay + kHeaderBytes;
-  const float* pay_sig = reinterpret_cast<const float*>(pay + g.off_sigma);
-  const uint32_t* P = slab_off + (size_t)u * (g.S + 2);
-  uint32_t cstride = 0, sw = 0;
-  if (!stats) {  // written by the allocation kernel
-    cstride = reinterpret_cast<const uint32_t*>(pay)[11];
-    sw = cstride / 4;
-  }
-  uint32_t* words_out = reinterpret_cast<uint32_t*>(pay + g.off_codes) + (size_t)chunk * kChunk * sw;
-
+  float* yunit = Y + (size_t)u * g.S * D.HW * g.n + chunk * kChunk;
   auto tile_of = [&](int ks) {
     return reinterpret_cast<float*>(smem + L.tile + (L.nbuf == 2 ? (ks & 1) : 0) * L.tile_bytes);
   };
-  auto bsl_of = [&](int ks) { return smem + L.bsl + (ks & 1) * L.bsl_stride; };
-  auto sig_of = [&](int ks) { return reinterpret_cast<float*>(smem + L.sig) + (ks & 1) * D.HW; };
 
-  issue_tile(D, ysrc + (size_t)ks0 * D.HW * g.n, tile_of(ks0));
-  if (quant) {
-    issue_slab_bits(D, pay_b, ks0, bsl_of(ks0));
-    issue_sigma(D, pay_sig, ks0, sig_of(ks0));
-    for (int i = threadIdx.x; i < TACTKV_THR_PAD_TOTAL; i += blockDim.x) thr[i] = c_thr_pad[i];
-    for (int i = threadIdx.x; i < 6 * TACTKV_Q_CELLS; i += blockDim.x) qcell[i] = c_qcell[i];
-    if (threadIdx.x < kChunk) carry[threadIdx.x] = 0;
-  }
+  issue_tile(D, yunit + (size_t)ks0 * D.HW * g.n, tile_of(ks0));
   cp_async_commit();
-  const uint32_t A = quant ? P[ks0] : 0u;   // first stream bit of the range
-
   for (int ks = ks0; ks < ks1; ++ks) {
     float* tile = tile_of(ks);
-    const unsigned char* bs = bsl_of(ks) + (((size_t)ks * D.HW) & 15);
+    float* yslab = yunit + (size_t)ks * D.HW * g.n + lane;
     cp_async_wait_all();
     __syncthreads();  // slab ks is in place; every thread is done with slab ks - 1
-    if (ks + 1 < ks1) {
-      if (L.nbuf == 2) issue_tile(D, ysrc + (size_t)(ks + 1) * D.HW * g.n, tile_of(ks + 1));
-      if (quant) {
-        issue_slab_bits(D, pay_b, ks + 1, bsl_of(ks + 1));
-        issue_sigma(D, pay_sig, ks + 1, sig_of(ks + 1));
-      }
+    if (L.nbuf == 2 && ks + 1 < ks1) {
+      issue_tile(D, yunit + (size_t)(ks + 1) * D.HW * g.n, tile_of(ks + 1));
       cp_async_commit();
     }
-    uint32_t pstart = 0, slab_bits = 0;
-    if (quant) {
-      pstart = P[ks];
-      slab_bits = P[ks + 1] - pstart;
-      slab_records(D, bs, sig_of(ks), true, smem + L.meta);
-      const int nw = (int)(((pstart & 31u) + slab_bits + 31) >> 5) + 1;
-      for (int c = warp; c < kChunk; c += nwarps)
-        for (int w = lane; w < nw; w += 32) sbuf[c * L.words + w] = w == 0 ? carry[c] : 0u;
-    }
-
     // DCT along H, in place, one column pair at a time per warp
     for (int wp = warp; wp < WP; wp += nwarps) h_pass_fwd<HC>(D, tile, 2 * wp, lane);
     __syncthreads();
     float2* t2 = reinterpret_cast<float2*>(tile);
     const int Wp = 2 * WP;
-
-    // DCT along W on row pair kp, fused with the epilogue
-    if (stats) {
-      for (int kp = warp; kp < HP; kp += nwarps) {
-        float2 x[WC];
-        w_load_fdct<WC>(D, t2, kp, lane, x);
-        __syncwarp();   // the row pair is read before its energies overwrite it
-        put_energy<WC>(D, t2, kp, lane, x);
-      }
-      __syncthreads();
-      float* dst = partial + ((size_t)u * g.nch + chunk) * g.N + (size_t)ks * D.HW;
-      for (int p = threadIdx.x; p < HP * D.W; p += blockDim.x) {
-        const int r = p / D.W, t = p - r * D.W;
-        const float2* e = t2 + rp_index(Wp, r, t);
-        const int sw15 = p & 15;
-        float2 acc = make_float2(0.f, 0.f);
+    // DCT along W on row pair kp; the coefficients go back over the slab of Y (this CTA's own
+    // bytes), their squares over the row pair's own elements of the tile
+    for (int kp = warp; kp < HP; kp += nwarps) {
+      float2 x[WC];
+      w_load_fdct<WC>(D, t2, kp, lane, x);
+      const bool second = 2 * kp + 1 < D.H;
+      float* y0 = yslab + (size_t)(2 * kp * D.W) * g.n;
+#pragma unroll
+      for (int t = 0; t < WC; ++t)
+        if (t < D.W) {
+          y0[(size_t)t * g.n] = x[t].x;
+          if (second) y0[(size_t)(D.W + t) * g.n] = x[t].y;
+        }
+      __syncwarp();   // the row pair is read before its energies overwrite it
+      put_energy<WC>(D, t2, kp, lane, x);
+    }
+    __syncthreads();
+    float* dst = partial + ((size_t)u * g.nch + chunk) * g.N + (size_t)ks * D.HW;
+    for (int p = threadIdx.x; p < HP * D.W; p += blockDim.x) {
+      const int r = p / D.W, t = p - r * D.W;
+      const float2* e = t2 + rp_index(Wp, r, t);
+      const int sw15 = p & 15;
+      float2 acc = make_float2(0.f, 0.f);
 #pragma unroll 8
-        for (int c = 0; c < kChunk; ++c) acc = __fadd2_rn(acc, e[c ^ sw15]);
-        dst[2 * r * D.W + t] = acc.x;
-        if (2 * r + 1 < D.H) dst[(2 * r + 1) * D.W + t] = acc.y;
-      }
-    } else {
-      for (int kp = warp; kp < HP; kp += nwarps) {
-        float2 x[WC];
-        w_load_fdct<WC>(D, t2, kp, lane, x);
-        if (raw) {
-          float* s = reinterpret_cast<float*>(pay + g.off_codes + (size_t)(chunk * kChunk + lane) * cstride) +
-                     (size_t)ks * D.HW + 2 * kp * D.W;
-          const bool second = 2 * kp + 1 < D.H;
-#pragma unroll
-          for (int t = 0; t < WC; ++t)
-            if (t < D.W) {
-              s[t] = x[t].x;
-              if (second) s[D.W + t] = x[t].y;
-            }
-        } else {
-          uint32_t p0, p1;
-          row_positions(D, bs, kp, pstart & 31u, p0, p1);
-          uint32_t* row = sbuf + lane * L.words;
-          uint32_t acc0 = 0, acc1 = 0;
-#pragma unroll
-          for (int t = 0; t < WC; ++t)
-            if (t < D.W) {
-              const uint4 m = meta[kp * D.W + t];
-              const float2 uu = __fmul2_rn(x[t], make_float2(__uint_as_float(m.x), __uint_as_float(m.y)));
-              const int b0 = m.z & 0xff, b1 = (m.z >> 8) & 0xff;
-              if (b0) put_code(acc0, p0, quant_code(uu.x, b0, thr, qcell), b0, row);
-              if (b1) put_code(acc1, p1, quant_code(uu.y, b1, thr, qcell), b1, row);
-            }
-          if (p0 & 31u) atomicOr(row + (p0 >> 5), acc0);
-          if (p1 & 31u) atomicOr(row + (p1 >> 5), acc1);
-        }
-      }
-      if (quant) {
-        __syncthreads();
-        // complete words go out; the first word of the range may be shared with the previous range
-        const uint32_t endbit = (pstart & 31u) + slab_bits;
-        const int full = (int)(endbit >> 5);
-        const uint32_t wbase = pstart >> 5, wA = A >> 5;
-        const bool shared_first = (A & 31u) != 0;
-        for (int c = warp; c < kChunk; c += nwarps) {
-          uint32_t* out = words_out + (size_t)c * sw;
-          for (int w = lane; w < full; w += 32) {
-            const uint32_t v = sbuf[c * L.words + w];
-            if (shared_first && wbase + w == wA) atomicOr(out + wA, v);
-            else out[wbase + w] = v;
-          }
-          if (lane == 0) carry[c] = (endbit & 31u) ? sbuf[c * L.words + full] : 0u;
-        }
-      }
+      for (int c = 0; c < kChunk; ++c) acc = __fadd2_rn(acc, e[c ^ sw15]);
+      dst[2 * r * D.W + t] = acc.x;
+      if (2 * r + 1 < D.H) dst[(2 * r + 1) * D.W + t] = acc.y;
     }
     if (L.nbuf == 1 && ks + 1 < ks1) {
       __syncthreads();  // everyone is done with the only tile
-      issue_tile(D, ysrc + (size_t)(ks + 1) * D.HW * g.n, tile_of(ks + 1));
+      issue_tile(D, yunit + (size_t)(ks + 1) * D.HW * g.n, tile_of(ks + 1));
       cp_async_commit();
     }
   }
   cp_async_wait_all();
-  if (quant) {
-    __syncthreads();
-    // the range's last partial word (shared with the next range), then the stream's zero padding
-    const uint32_t B = P[ks1];
-    if (threadIdx.x < kChunk && (B & 31u))
-      atomicOr(words_out + (size_t)threadIdx.x * sw + (B >> 5), carry[threadIdx.x]);
-    if (ks1 == g.S) {
-      const uint32_t first = (B + 31) >> 5;
-      for (int c = warp; c < kChunk; c += nwarps)
-        for (uint32_t w = first + lane; w < sw; w += 32) words_out[(size_t)c * sw + w] = 0u;
-    }
-  } else if (raw && ks1 == g.S) {
-    const int pad = (int)cstride - 4 * g.N;
-    for (int i = threadIdx.x; i < kChunk * pad; i += blockDim.x) {
-      const int c = i / pad, b = i - c * pad;
-      pay[g.off_codes + (size_t)(chunk * kChunk + c) * cstride + 4 * g.N + b] = 0;
-    }
-  }
 }
 
 // ---------------------------------------------------------------------------------- inverse ---
@@ -464,7 +308,7 @@ __global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) idct_hw_kernel(co
   const int ks0 = blockIdx.y * spc, ks1 = min(g.S, ks0 + spc);
   const UnitDev& ud = ul.u[u];
   const unsigned char* pay = ud.payload;
-  const uint32_t* P = slab_off + (size_t)u * (g.S + 2);
+  const uint32_t* P = slab_off + (size_t)u * unit_index_words(g.S);
   const bool ok = P[g.S + 1] != 0;   // the index kernel checked the header and the bit widths
   const uint32_t cstride = ok ? reinterpret_cast<const uint32_t*>(pay)[11] : 0u, sw = cstride / 4;
   const uint32_t* streams = reinterpret_cast<const uint32_t*>(pay + g.off_codes) + (size_t)chunk * kChunk * sw;
@@ -512,7 +356,7 @@ __global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) idct_hw_kernel(co
         issue_sigma(D, pay_sig, ks + 1, sig_of(ks + 1));
         cp_async_commit();
       }
-      slab_records(D, bs, sig_of(ks), false, smem + L.meta);
+      slab_records(D, bs, sig_of(ks), false, smem + L.meta, P[ks] & 31u);
       __syncthreads();
     }
     // decode rows 2j, 2j+1 of warp j and run the inverse DCT along W; write column pairs
@@ -529,19 +373,15 @@ __global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) idct_hw_kernel(co
         for (int t = 0; t < WC; ++t)
           if (t < D.W) x[t] = make_float2(s[t], second ? s[D.W + t] : 0.f);
       } else {
-        uint32_t p0, p1;
-        row_positions(D, bs, kp, P[ks] & 31u, p0, p1);
         const uint32_t* row = sbuf_of(ks) + lane * L.words;
-        uint32_t wi0 = p0 >> 5, s0 = p0 & 31u, wi1 = p1 >> 5, s1 = p1 & 31u;
-        uint32_t lo0 = row[wi0], hi0 = row[wi0 + 1], lo1 = row[wi1], hi1 = row[wi1 + 1];
 #pragma unroll
         for (int t = 0; t < WC; ++t)
           if (t < D.W) {
             const uint4 m = meta[kp * D.W + t];
-            const int b0 = m.z & 0xff, b1 = (m.z >> 8) & 0xff;
+            const uint32_t b0 = m.z & 15u, b1 = m.w & 15u;
             float l0 = 0.f, l1 = 0.f;
-            if (b0) l0 = lvs[lm_lv_offset(b0) + get_code(lo0, hi0, s0, wi0, b0, row)];
-            if (b1) l1 = lvs[lm_lv_offset(b1) + get_code(lo1, hi1, s1, wi1, b1, row)];
+            if (b0) l0 = lvs[lm_lv_offset((int)b0) + read_code(row, m.z >> 4, b0)];
+            if (b1) l1 = lvs[lm_lv_offset((int)b1) + read_code(row, m.w >> 4, b1)];
             x[t] = __fmul2_rn(make_float2(l0, l1), make_float2(__uint_as_float(m.x), __uint_as_float(m.y)));
           }
       }
@@ -587,13 +427,12 @@ namespace {
 template <int HX, int WX>
 cudaError_t launch_hw(bool inverse, int mode, const Geom& g, const UnitList& ul, int nu, float* buf, float* partial,
                       const uint32_t* slab_off, int spc, cudaStream_t st) {
-  const HwLayout L = hw_layout(g.H, g.W, inverse ? kLayDecode : (mode == kStats ? kLayStats : kLayQuant));
+  const HwLayout L = hw_layout(g.H, g.W, inverse ? kLayDecode : kLayStats);
   const dim3 grid(g.nch, (g.S + spc - 1) / spc, nu);
   const int threads = hw_threads(g.H, g.W);
   constexpr int H = TACTKV_HCLASS, W = TACTKV_WCLASS;
   const int sm = (int)L.total;
-  const size_t regions[] = {L.tile, L.sbuf, L.meta, L.sig, L.thr, L.lv, L.carry, L.bsl, L.qcell, L.tile_bytes,
-                            L.bsl_stride};
+  const size_t regions[] = {L.tile, L.sbuf, L.meta, L.sig, L.lv, L.bsl, L.tile_bytes, L.bsl_stride};
   for (size_t r : regions)
     if (r % 16) return cudaErrorMisalignedAddress;   // never launch a misaligned layout
   if (L.total > 227 * 1024) return cudaErrorInvalidConfiguration;
@@ -605,12 +444,8 @@ cudaError_t launch_hw(bool inverse, int mode, const Geom& g, const UnitList& ul,
   if (inverse) {
     if (mode == kRaw) TACTKV_GO((idct_hw_kernel<H, W, HX, WX, kRaw>), g, ul, buf, slab_off, spc);
     else TACTKV_GO((idct_hw_kernel<H, W, HX, WX, kQuant>), g, ul, buf, slab_off, spc);
-  } else if (mode == kStats) {
-    TACTKV_GO((fdct_hw_kernel<H, W, HX, WX, kStats>), g, ul, buf, partial, slab_off, spc);
-  } else if (mode == kRaw) {
-    TACTKV_GO((fdct_hw_kernel<H, W, HX, WX, kRaw>), g, ul, buf, partial, slab_off, spc);
   } else {
-    TACTKV_GO((fdct_hw_kernel<H, W, HX, WX, kQuant>), g, ul, buf, partial, slab_off, spc);
+    TACTKV_GO((fdct_hw_kernel<H, W, HX, WX>), g, ul, buf, partial, spc);
   }
 #undef TACTKV_GO
   return cudaGetLastError();
@@ -633,7 +468,7 @@ cudaError_t TACTKV_HWNAME(launch_axis_hw_)(bool inverse, int mode, const Geom& g
 
 // Shared memory and threads of one CTA (host queries used to size the slab ranges).
 void TACTKV_HWNAME(axis_hw_shape_)(const Geom& g, bool inverse, int mode, size_t* smem, int* threads) {
-  *smem = hw_layout(g.H, g.W, inverse ? kLayDecode : (mode == kStats ? kLayStats : kLayQuant)).total;
+  *smem = hw_layout(g.H, g.W, inverse ? kLayDecode : kLayStats).total;
   *threads = hw_threads(g.H, g.W);
 }
 

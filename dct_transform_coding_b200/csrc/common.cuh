@@ -24,6 +24,8 @@ constexpr int kAllocThreads = 1024;
 constexpr size_t kStatusBytes = 256;       // status word at the start of the workspace
 constexpr int kMaxHW = 1024;               // H*W limit of the H/W-axis kernels
 constexpr int kMaxSlabs = 64;              // S limit
+constexpr int kMaxN = kMaxSlabs * kMaxHW;  // bins per unit limit
+constexpr int kPackRecs = 1024;            // records per packing range (one CTA)
 
 enum HwMode { kStats = 0, kQuant = 1, kRaw = 2 };
 
@@ -45,6 +47,11 @@ struct Geom {
 };
 
 __host__ __device__ inline long long pad16(long long x) { return (x + 15) / 16 * 16; }
+
+// Per-unit index block in the workspace: P(k_s) for k_s = 0..S (first stream bit of each slab,
+// P(S) = code_bits), the decoder's ok flag, then NZ(k_s) for k_s = 0..S (first record of each slab
+// in the unit's list of bins with bits).
+__host__ __device__ inline int unit_index_words(int S) { return 2 * S + 3; }
 
 // Codebook b (1..8) has 2^b - 1 thresholds and 2^b levels, stored for b = 1, 2, ... in turn.
 __host__ __device__ constexpr int lm_thr_offset(int b) { return (1 << b) - b - 1; }
@@ -70,13 +77,17 @@ cudaError_t launch_axis_s(int cls, bool inverse, const Geom& g, const UnitList& 
 cudaError_t launch_axis_hw(int hcls, int wcls, bool inverse, int mode, const Geom& g, const UnitList& ul, int nu, float* buf,
                            float* partial, const uint32_t* slab_off, int spc, cudaStream_t st);
 void axis_hw_shape(int hcls, int wcls, const Geom& g, bool inverse, int mode, size_t* smem, int* threads);
-// Per-unit bit allocation: writes b, sigma, the header, the slab offsets P(k_s) (slab_off[u][0..S])
-// and zeroes the stream word at every P(k_s).
+// Per-unit bit allocation: writes b, sigma and the header into the payload, P and NZ into the
+// unit's index block, the records {bin, bits, P_i, 1/sigma_i} of the bins with bits into recs
+// (N per unit), and zeroes the stream word at every P(k_s).
 cudaError_t launch_allocate(const Geom& g, const UnitList& ul, int nu, const float* partial, double* var,
-                            uint32_t* slab_off, cudaStream_t st);
-// Decoding index: checks every unit's header and bit widths, writes slab_off[u][0..S] and the
-// unit's ok flag slab_off[u][S+1]; a bad unit sets TACTKV_CORRUPT_PAYLOAD in *status.
-cudaError_t launch_decode_index(const Geom& g, const UnitList& ul, int nu, uint32_t* slab_off, unsigned int* status,
+                            uint32_t* index, uint4* recs, cudaStream_t st);
+// Quantization and packing of the finished coefficients X (workspace volume) into the payloads.
+cudaError_t launch_pack(const Geom& g, const UnitList& ul, int nu, const float* X, const uint4* recs,
+                        const uint32_t* index, cudaStream_t st);
+// Decoding index: checks every unit's header and bit widths, writes P(0..S) and the unit's ok
+// flag into its index block; a bad unit sets TACTKV_CORRUPT_PAYLOAD in *status.
+cudaError_t launch_decode_index(const Geom& g, const UnitList& ul, int nu, uint32_t* index, unsigned int* status,
                                 cudaStream_t st);
 
 #ifdef __CUDACC__

@@ -1,0 +1,188 @@
+// Quantization and bit packing (TACT-KV stage 4: gain-shape scalar quantization with the fixed
+// Lloyd-Max codebook at each bin's bit width), on the finished 3D-DCT coefficients X.
+//
+// The allocation kernel lists, once per unit, every bin that received bits, in bin order, as a
+// 16-byte record {bin, bits, first stream bit P_i, 1/sigma_i}; P_i = sum of the bits of every
+// earlier bin, the same in every channel's stream.  A CTA owns one (unit, 32-channel chunk, range
+// of kPackRecs records); lane l of a warp is channel l, so every decision about a record is
+// uniform across the warp and only the 32 coefficient values differ.  Bins without bits are never
+// read.
+//
+// The CTA loads its records with cp.async, clears the word rows of its bit span in shared memory,
+// and each warp takes blocks of 8 records: it loads the 8 coefficient rows (128 bytes each, all
+// in flight at once), computes u = X * (1/sigma) and the code, and ORs the code into the channel's
+// word row at its stream position (records are independent of each other).  The span's words are
+// then stored once; its first and last words may hold bits of the neighbouring ranges and are
+// ORed into the payload atomically (the allocation zeroes those words first).  The CTA with the
+// last record also writes the zero padding of the channel streams.
+//
+// NO_QUANT (raw) copies X into the channel streams as float32.
+#include "common.cuh"
+#include "lloyd_max_tables.inc"
+
+namespace tactkv {
+namespace {
+
+constexpr int kPackThreads = 256;
+constexpr int kPackBlock = 8;   // records per warp step
+
+// Thresholds of width b padded with two +inf, stored for b = 1, 2, ... in turn.
+__device__ __forceinline__ int thr_pad_offset(int b) { return (1 << b) + b - 3; }
+
+// Code of u at b bits: the number of thresholds t_j <= u (float32 compares, ties go up).  b = 1:
+// the sign test; b = 2: three compares against {-t, 0, t}; b >= 3: the cell of u in a uniform grid
+// gives the count c of thresholds below the cell, and two compares finish it (a cell holds at most
+// two thresholds; the thresholds are padded with +inf).
+__device__ __forceinline__ uint32_t quant_code(float u, int b, const float* thr, const unsigned char* qcell) {
+  if (b == 1) return u >= 0.f;
+  if (b == 2) {
+    const float t = thr[thr_pad_offset(2) + 2];
+    return (uint32_t)(u >= -t) + (uint32_t)(u >= 0.f) + (uint32_t)(u >= t);
+  }
+  int j = __float2int_rd(fmaf(u, TACTKV_Q_SCALE, TACTKV_Q_OFFSET));
+  j = min(max(j, 0), TACTKV_Q_CELLS - 1);
+  const uint32_t c = qcell[(b - 3) * TACTKV_Q_CELLS + j];
+  const float* t = thr + thr_pad_offset(b) + c;
+  return c + (uint32_t)(u >= t[0]) + (uint32_t)(u >= t[1]);
+}
+
+// OR a b-bit code into a channel's word row at bit position off (b >= 1); codes of other records
+// in the same word come from other warps, so words are combined atomically.
+__device__ __forceinline__ void emit_code(uint32_t* row, uint32_t off, uint32_t b, uint32_t code) {
+  const uint32_t w = off >> 5, sh = off & 31u;
+  atomicOr(row + w, code << sh);
+  if (sh + b > 32) atomicOr(row + w + 1, code >> (32 - sh));   // sh >= 25 here
+}
+
+struct PackLayout {
+  size_t rec, sbuf, thr, qcell, total;
+  int words;
+};
+__host__ __device__ inline PackLayout pack_layout() {
+  PackLayout L;
+  auto p16 = [](size_t x) { return (x + 15) / 16 * 16; };
+  L.words = ((8 * kPackRecs + 31) / 32 + 3) | 1;   // odd: 32 channels' rows in 32 different banks
+  size_t o = 0;
+  L.rec = o; o += p16((size_t)kPackRecs * 16);
+  L.sbuf = o; o += p16((size_t)kChunk * L.words * 4);
+  L.thr = o; o += p16((size_t)TACTKV_THR_PAD_TOTAL * 4);
+  L.qcell = o; o += p16((size_t)6 * TACTKV_Q_CELLS);
+  L.total = o;
+  return L;
+}
+
+__global__ void __launch_bounds__(kPackThreads) pack_kernel(const __grid_constant__ Geom g,
+                                                            const __grid_constant__ UnitList ul,
+                                                            const float* __restrict__ X, const uint4* __restrict__ recs,
+                                                            const uint32_t* __restrict__ index) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const PackLayout L = pack_layout();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int chunk = blockIdx.x, u = blockIdx.z;
+  const uint32_t* P = index + (size_t)u * unit_index_words(g.S);
+  const uint32_t nrec = P[2 * g.S + 2], code_bits = P[g.S];      // NZ(S) and P(S)
+  const uint32_t r0 = blockIdx.y * kPackRecs;
+  if (r0 >= nrec && !(r0 == 0 && nrec == 0)) return;             // (range 0 also pads an empty unit)
+  const uint32_t r1 = min(nrec, r0 + kPackRecs);
+  const int m = (int)(r1 - r0);
+  unsigned char* pay = ul.u[u].payload;
+  const uint4* urecs = recs + (size_t)u * g.N;
+  const float* xu = X + (size_t)u * g.N * g.n + chunk * kChunk + lane;
+  uint4* rs = reinterpret_cast<uint4*>(smem + L.rec);
+  uint32_t* sbuf = reinterpret_cast<uint32_t*>(smem + L.sbuf);
+  float* thr = reinterpret_cast<float*>(smem + L.thr);
+  unsigned char* qcell = smem + L.qcell;
+  const uint32_t cstride = reinterpret_cast<const uint32_t*>(pay)[11], sw = cstride / 4;
+  uint32_t* words_out = reinterpret_cast<uint32_t*>(pay + g.off_codes) + (size_t)chunk * kChunk * sw;
+
+  for (int e = threadIdx.x; e < m; e += blockDim.x) cp_async16(rs + e, urecs + r0 + e);
+  cp_async_commit();
+  for (int i = threadIdx.x; i < TACTKV_THR_PAD_TOTAL; i += blockDim.x) thr[i] = c_thr_pad[i];
+  for (int i = threadIdx.x; i < 6 * TACTKV_Q_CELLS; i += blockDim.x) qcell[i] = c_qcell[i];
+  // bit span [A, B) of the range; its words from word A >> 5 on are assembled in shared memory
+  const uint32_t A = m > 0 ? urecs[r0].z : code_bits;
+  const uint32_t B = r1 < nrec ? urecs[r1].z : code_bits;
+  const uint32_t base = A & ~31u;
+  const int nw = (int)((B - base + 31) >> 5);
+  for (int c = warp; c < kChunk; c += nwarps)
+    for (int w = lane; w <= nw; w += 32) sbuf[c * L.words + w] = 0u;
+  cp_async_wait_all();
+  __syncthreads();
+
+  uint32_t* row = sbuf + lane * L.words;
+  for (int e0 = warp * kPackBlock; e0 < m; e0 += nwarps * kPackBlock) {
+    uint4 r[kPackBlock];
+    float x[kPackBlock];
+#pragma unroll
+    for (int j = 0; j < kPackBlock; ++j)
+      if (e0 + j < m) {
+        r[j] = rs[e0 + j];
+        x[j] = __ldcs(xu + (size_t)r[j].x * g.n);
+      }
+#pragma unroll
+    for (int j = 0; j < kPackBlock; ++j)
+      if (e0 + j < m) {
+        const int b = (int)r[j].y;
+        const float uq = x[j] * __uint_as_float(r[j].w);
+        emit_code(row, r[j].z - base, (uint32_t)b, quant_code(uq, b, thr, qcell));
+      }
+  }
+  __syncthreads();
+  // the span's words; the first and the last may be shared with the neighbouring ranges
+  const uint32_t wbase = base >> 5, wlast = (B - 1) >> 5;
+  const bool first_shared = (A & 31u) != 0, last_shared = (B & 31u) != 0;
+  for (int c = warp; c < kChunk; c += nwarps) {
+    uint32_t* out = words_out + (size_t)c * sw;
+    for (int w = lane; w < nw; w += 32) {
+      const uint32_t gw = wbase + w, v = sbuf[c * L.words + w];
+      if ((gw == wbase && first_shared) || (gw == wlast && last_shared)) atomicOr(out + gw, v);
+      else out[gw] = v;
+    }
+  }
+  if (r1 == nrec) {   // zero padding of the streams after the last code bit
+    const uint32_t first = (code_bits + 31) >> 5;
+    for (int c = warp; c < kChunk; c += nwarps)
+      for (uint32_t w = first + lane; w < sw; w += 32) words_out[(size_t)c * sw + w] = 0u;
+  }
+}
+
+// NO_QUANT: the float32 coefficients of every bin into the channel streams (stream c holds X[i, c]
+// at byte 4i), then the zero padding up to the channel stride.
+__global__ void __launch_bounds__(kPackThreads) pack_raw_kernel(const __grid_constant__ Geom g,
+                                                                const __grid_constant__ UnitList ul,
+                                                                const float* __restrict__ X, int spc) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int chunk = blockIdx.x, u = blockIdx.z;
+  const int ks0 = blockIdx.y * spc, ks1 = min(g.S, ks0 + spc);
+  unsigned char* pay = ul.u[u].payload;
+  const uint32_t cstride = reinterpret_cast<const uint32_t*>(pay)[11];
+  float* stream = reinterpret_cast<float*>(pay + g.off_codes + (size_t)(chunk * kChunk + lane) * cstride);
+  const float* xu = X + (size_t)u * g.N * g.n + chunk * kChunk + lane;
+  for (int i = ks0 * g.HW + warp; i < ks1 * g.HW; i += nwarps) stream[i] = xu[(size_t)i * g.n];
+  if (ks1 == g.S) {
+    const int pad = (int)cstride - 4 * g.N;
+    for (int i = threadIdx.x; i < kChunk * pad; i += blockDim.x) {
+      const int c = i / pad, b = i - c * pad;
+      pay[g.off_codes + (size_t)(chunk * kChunk + c) * cstride + 4 * g.N + b] = 0;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_pack(const Geom& g, const UnitList& ul, int nu, const float* X, const uint4* recs,
+                        const uint32_t* index, cudaStream_t st) {
+  if (g.flags & TACTKV_NO_QUANT) {
+    const int spc = 1;
+    pack_raw_kernel<<<dim3(g.nch, g.S, nu), kPackThreads, 0, st>>>(g, ul, X, spc);
+  } else {
+    const PackLayout L = pack_layout();
+    cudaFuncSetAttribute(pack_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
+    // ranges of kPackRecs records; a unit has at most N records, CTAs past its last record exit
+    const dim3 grid(g.nch, (g.N + kPackRecs - 1) / kPackRecs, nu);
+    pack_kernel<<<grid, kPackThreads, L.total, st>>>(g, ul, X, recs, index);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace tactkv

@@ -1,10 +1,11 @@
 // TACT-KV codec C ABI (host side): argument checks, grouping of units into waves, launches.
 //
 // A compress wave (up to kMaxUnits units of identical shape) runs five kernels on the caller's
-// stream: the forward DCT along S (axis_s.cu), the forward DCT along H and W with per-bin energy
-// sums (axis_hw.cu, kStats), the variance reduction and the per-unit allocation with the payload
-// header and slab offsets (allocate.cu), and the H/W pass again with quantization and packing
-// (axis_hw.cu, kQuant), which reads the S-transformed volume kept in the workspace.  A decompress
+// stream: the forward DCT along S (axis_s.cu), the forward DCT along H and W, which writes the
+// finished coefficients back into the workspace volume and sums the per-bin energies (axis_hw.cu),
+// the variance reduction and the per-unit allocation with the payload header, slab offsets and
+// the records of the bins with bits (allocate.cu), and the quantization and packing of those bins
+// (pack.cu).  A decompress
 // wave runs the decoding index (allocate.cu: header checks, slab offsets), the inverse H/W pass
 // (dequantize + inverse DCT along W and H) and the inverse DCT along S.
 #include <algorithm>
@@ -87,19 +88,21 @@ size_t payload_bytes_geom(const Geom& g) {
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
-// workspace of one unit: the S-transformed volume (fp32), per-chunk energy sums, fp64 variances,
-// slab offsets P(0..S) and the decoder's ok flag
+// workspace of one unit: the transformed volume (fp32; Y and then X when compressing, V when
+// decompressing), per-chunk energy sums, fp64 variances, the index block (P, ok, NZ) and the
+// records of the bins with bits
 size_t unit_ws_bytes(const Geom& g) {
   return round256((size_t)g.T * g.n * 4) + round256((size_t)g.nch * g.N * 4) + round256((size_t)g.N * 8) +
-         round256((size_t)(g.S + 2) * 4);
+         round256((size_t)unit_index_words(g.S) * 4) + round256((size_t)g.N * 16);
 }
 
 struct WsView {
   unsigned int* status;
-  float* big;         // nu * T * n floats: Y (compress) or V (decompress)
+  float* big;         // nu * T * n floats: Y/X (compress) or V (decompress)
   float* partial;     // nu * nch * N floats
   double* var;        // nu * N doubles
-  uint32_t* slab_off; // nu * (S + 2) words
+  uint32_t* index;    // nu * unit_index_words(S) words
+  uint4* recs;        // nu * N records
 };
 
 WsView view(unsigned char* ws, const Geom& g, int nu) {
@@ -112,16 +115,15 @@ WsView view(unsigned char* ws, const Geom& g, int nu) {
   off += round256((size_t)nu * g.nch * g.N * 4);
   v.var = reinterpret_cast<double*>(ws + off);
   off += round256((size_t)nu * g.N * 8);
-  v.slab_off = reinterpret_cast<uint32_t*>(ws + off);
+  v.index = reinterpret_cast<uint32_t*>(ws + off);
+  off += round256((size_t)nu * unit_index_words(g.S) * 4);
+  v.recs = reinterpret_cast<uint4*>(ws + off);
   return v;
 }
 
-// Slabs per CTA of the H/W passes: whole units when the batch alone fills the GPU a couple of
-// times over, shorter slab ranges (more CTAs) for small batches.
-int slabs_per_cta(const Geom& g, int nu, bool inverse, int mode) {
-  size_t smem = 0;
-  int threads = 32;
-  axis_hw_shape(length_class(g.H), length_class(g.W), g, inverse, mode, &smem, &threads);
+// Slabs per CTA of the slab-walking kernels: whole units when the batch alone fills the GPU a
+// couple of times over, shorter slab ranges (more CTAs) for small batches.
+int slabs_per_cta_for(const Geom& g, int nu, size_t smem, int threads) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int by_smem = (int)((228 * 1024) / (smem + 1024));
@@ -131,6 +133,12 @@ int slabs_per_cta(const Geom& g, int nu, bool inverse, int mode) {
   const long long have = (long long)g.nch * nu;
   const int ranges = (int)std::min<long long>(g.S, std::max<long long>(1, (target + have - 1) / have));
   return (g.S + ranges - 1) / ranges;
+}
+int slabs_per_cta(const Geom& g, int nu, bool inverse, int mode) {
+  size_t smem = 0;
+  int threads = 32;
+  axis_hw_shape(length_class(g.H), length_class(g.W), g, inverse, mode, &smem, &threads);
+  return slabs_per_cta_for(g, nu, smem, threads);
 }
 
 bool same_group(const tactkv_unit& a, const tactkv_unit& b) {
@@ -267,15 +275,14 @@ static tactkv_status compress_impl(const tactkv_unit* units, int n_units, void* 
                          mark(0);
                          if (launch_axis_s(cs, false, g, ul, nu, w.big, st) != cudaSuccess) return TACTKV_CUDA;
                          mark(1);
-                         if (launch_axis_hw(ch, cw, false, kStats, g, ul, nu, w.big, w.partial, w.slab_off,
+                         if (launch_axis_hw(ch, cw, false, kStats, g, ul, nu, w.big, w.partial, w.index,
                                             slabs_per_cta(g, nu, false, kStats), st) != cudaSuccess)
                            return TACTKV_CUDA;
                          mark(2);
-                         if (launch_allocate(g, ul, nu, w.partial, w.var, w.slab_off, st) != cudaSuccess)
+                         if (launch_allocate(g, ul, nu, w.partial, w.var, w.index, w.recs, st) != cudaSuccess)
                            return TACTKV_CUDA;
                          mark(3);
-                         if (launch_axis_hw(ch, cw, false, mode2, g, ul, nu, w.big, w.partial, w.slab_off,
-                                            slabs_per_cta(g, nu, false, mode2), st) != cudaSuccess)
+                         if (launch_pack(g, ul, nu, w.big, w.recs, w.index, st) != cudaSuccess)
                            return TACTKV_CUDA;
                          mark(4);
                          return TACTKV_OK;
@@ -293,9 +300,9 @@ static tactkv_status decompress_impl(const tactkv_unit* units, int n_units, void
                          const int cs = length_class(g.S), ch = length_class(g.H), cw = length_class(g.W);
                          const int mode = (g.flags & TACTKV_NO_QUANT) ? kRaw : kQuant;
                          mark(0);
-                         if (launch_decode_index(g, ul, nu, w.slab_off, w.status, st) != cudaSuccess)
+                         if (launch_decode_index(g, ul, nu, w.index, w.status, st) != cudaSuccess)
                            return TACTKV_CUDA;
-                         if (launch_axis_hw(ch, cw, true, mode, g, ul, nu, w.big, nullptr, w.slab_off,
+                         if (launch_axis_hw(ch, cw, true, mode, g, ul, nu, w.big, nullptr, w.index,
                                             slabs_per_cta(g, nu, true, mode), st) != cudaSuccess)
                            return TACTKV_CUDA;
                          mark(1);
