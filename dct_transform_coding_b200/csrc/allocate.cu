@@ -302,13 +302,18 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
 
 // ----------------------------------------------------------------------------- decode index ---
 // One CTA per unit: the header must describe exactly the unit the caller asked for, every bit
-// width must be <= 8 and their sum must equal the header's code_bits; then P(k_s) is rebuilt.
+// width must be <= 8 and their sum must equal the header's code_bits; then P(k_s), NZ(k_s) and the
+// records {bin, bits, first stream bit, sigma} of the bins with bits are rebuilt from the payload
+// (one warp per slab: a ballot gives each record's slot, a scan its stream position).
 __global__ void __launch_bounds__(256) decode_index_kernel(const __grid_constant__ Geom g,
                                                            const __grid_constant__ UnitList ul,
-                                                           uint32_t* __restrict__ index, unsigned int* status) {
+                                                           uint32_t* __restrict__ index, uint4* __restrict__ recs,
+                                                           unsigned int* status) {
   __shared__ int s_ok;
   __shared__ uint32_t s_slab[kMaxSlabs];
+  __shared__ uint32_t s_nzslab[kMaxSlabs];
   __shared__ uint32_t s_P[kMaxSlabs + 1];
+  __shared__ uint32_t s_NZ[kMaxSlabs + 1];
   const int u = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const UnitDev& ud = ul.u[u];
   const unsigned char* pay = ud.payload;
@@ -331,40 +336,72 @@ __global__ void __launch_bounds__(256) decode_index_kernel(const __grid_constant
   }
   __syncthreads();
   bool ok = s_ok;
+  const unsigned char* b = pay + kHeaderBytes;
   if (ok && !raw) {
-    const unsigned char* b = pay + kHeaderBytes;
     bool bad = false;
     for (int k = warp; k < g.S; k += nwarps) {
-      uint32_t sum = 0;
+      uint32_t sum = 0, nz = 0;
       for (int i = lane; i < g.HW; i += 32) {
         const uint32_t v = b[(size_t)k * g.HW + i];
         bad |= v > 8;
         sum += v;
+        nz += v > 0;
       }
       sum = __reduce_add_sync(0xffffffffu, sum);
-      if (lane == 0) s_slab[k] = sum;
+      nz = __reduce_add_sync(0xffffffffu, nz);
+      if (lane == 0) {
+        s_slab[k] = sum;
+        s_nzslab[k] = nz;
+      }
     }
     if (bad) s_ok = 0;
     __syncthreads();
     if (warp == 0) slab_scan(s_slab, g.S, s_P);
+    else if (warp == 1) slab_scan(s_nzslab, g.S, s_NZ);
     __syncthreads();
     if (threadIdx.x == 0 && s_P[g.S] != reinterpret_cast<const uint32_t*>(pay)[10]) s_ok = 0;
     __syncthreads();
     ok = s_ok;
   }
   uint32_t* P = index + (size_t)u * unit_index_words(g.S);
-  for (int k = threadIdx.x; k <= g.S; k += blockDim.x) P[k] = (ok && !raw) ? s_P[k] : 0u;
+  uint32_t* NZ = P + g.S + 2;
+  for (int k = threadIdx.x; k <= g.S; k += blockDim.x) {
+    P[k] = (ok && !raw) ? s_P[k] : 0u;
+    NZ[k] = (ok && !raw) ? s_NZ[k] : 0u;
+  }
   if (threadIdx.x == 0) {
     P[g.S + 1] = ok ? 1u : 0u;
     if (!ok) set_status(status, TACTKV_CORRUPT_PAYLOAD);
+  }
+  if (ok && !raw) {
+    const float* sig = reinterpret_cast<const float*>(pay + g.off_sigma);
+    uint4* urecs = recs + (size_t)u * g.N;
+    const uint32_t below = (1u << lane) - 1u;
+    for (int k = warp; k < g.S; k += nwarps) {
+      uint32_t slot = s_NZ[k], pos = s_P[k];
+      for (int i0 = 0; i0 < g.HW; i0 += 32) {
+        const int i = k * g.HW + i0 + lane;
+        const uint32_t v = i0 + lane < g.HW ? b[i] : 0u;
+        uint32_t incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += t;
+        }
+        const uint32_t nzmask = __ballot_sync(0xffffffffu, v > 0);
+        if (v) urecs[slot + __popc(nzmask & below)] = make_uint4((uint32_t)i, v, pos + incl - v, __float_as_uint(sig[i]));
+        slot += __popc(nzmask);
+        pos += __shfl_sync(0xffffffffu, incl, 31);
+      }
+    }
   }
 }
 
 }  // namespace
 
-cudaError_t launch_decode_index(const Geom& g, const UnitList& ul, int nu, uint32_t* index, unsigned int* status,
-                                cudaStream_t st) {
-  decode_index_kernel<<<nu, 256, 0, st>>>(g, ul, index, status);
+cudaError_t launch_decode_index(const Geom& g, const UnitList& ul, int nu, uint32_t* index, uint4* recs,
+                                unsigned int* status, cudaStream_t st) {
+  decode_index_kernel<<<nu, 256, 0, st>>>(g, ul, index, recs, status);
   return cudaGetLastError();
 }
 

@@ -37,6 +37,7 @@ enum LayoutKind { kLayStats = 0, kLayDecode = 2 };
 struct HwLayout {
   size_t tile, tile_bytes, sbuf, meta, bsl, bsl_stride, sig, lv, total;
   int nbuf, words;
+  int nslot;   // decode: slabs of stream words and records held at once (2: the next one prefetched)
 };
 
 __host__ __device__ inline int row_pairs(int L) { return (L + 1) >> 1; }
@@ -53,8 +54,7 @@ __host__ __device__ inline int hw_threads(int H, int W) {
 // 2*ceil(H/2) rows of Wp = 2*ceil(W/2) cells (the padding row and column are never read), which
 // also holds its row-pair (forward) or column-pair (inverse) rearrangement.  stats: the slab tiles
 // (two when they fit, so the next slab loads while this one is transformed; the energies reuse
-// the rearranged tile).  decode: one tile, two slabs of stream words, per-bin records, bit widths
-// and sigmas of two slabs, levels.  words (the stride of a channel's word row) is odd, so the 32
+// the rearranged tile).  decode: one tile, the stream words and the records of two slabs, levels.  words (the stride of a channel's word row) is odd, so the 32
 // lanes reading 32 channels' rows hit 32 different banks.
 __host__ __device__ inline HwLayout hw_layout(int H, int W, int kind) {
   HwLayout L;
@@ -62,11 +62,13 @@ __host__ __device__ inline HwLayout hw_layout(int H, int W, int kind) {
   const bool de = kind == kLayDecode;
   L.tile_bytes = (size_t)(2 * HP) * (2 * WP) * 32 * 4;
   L.words = ((8 * HW + 31) / 32 + 3) | 1;
-  const size_t words = de ? (size_t)32 * L.words * 4 * 2 : 0;
-  const size_t meta = de ? (size_t)HP * W * 16 : 0;
-  L.bsl_stride = ((size_t)HW + 15) / 16 * 16 + 32;
-  const size_t bsl = de ? 2 * L.bsl_stride : 0;
-  const size_t sig = de ? (size_t)2 * HW * 4 : 0;
+  const size_t words1 = (size_t)32 * L.words * 4, meta1 = (size_t)HW * 16;
+  L.nslot = (de && (size_t)(2 * HP) * (2 * WP) * 128 + 2 * (words1 + meta1) + kLmLvTotal * 4 + 256 > kSmemBudget) ? 1 : 2;
+  const size_t words = de ? words1 * L.nslot : 0;
+  const size_t meta = de ? meta1 * L.nslot : 0;       // records
+  L.bsl_stride = 0;
+  const size_t bsl = 0;
+  const size_t sig = 0;
   const size_t lv = de ? kLmLvTotal * 4 : 0;
   const size_t rest = words + meta + bsl + sig + lv + 256;
   L.nbuf = (de || 2 * L.tile_bytes + rest > kSmemBudget) ? 1 : 2;
@@ -110,50 +112,6 @@ __device__ __forceinline__ void issue_tile(const D& g, const float* slab_src, fl
     for (int w = 0; w < g.W; ++w)
       cp_async16(tile + (r * Wp + w) * 32 + (threadIdx.x & 7) * 4,
                  slab_src + (size_t)(r * g.W + w) * g.n + (threadIdx.x & 7) * 4);
-}
-// The bit widths of slab ks as the 16-byte aligned window around them (the payload and its b[]
-// array are 16-byte aligned and padded); they start at byte (ks * HW) % 16 of dst.
-template <class D>
-__device__ __forceinline__ void issue_slab_bits(const D& g, const unsigned char* pay_b, int ks, unsigned char* dst) {
-  const size_t a0 = (size_t)ks * g.HW, q0 = a0 / 16, q1 = (a0 + g.HW + 15) / 16;
-  for (int i = threadIdx.x; i < (int)(q1 - q0); i += blockDim.x) cp_async16(dst + 16 * i, pay_b + 16 * (q0 + i));
-}
-template <class D>
-__device__ __forceinline__ void issue_sigma(const D& g, const float* pay_sig, int ks, float* dst) {
-  for (int j = threadIdx.x; j < g.HW; j += blockDim.x) cp_async4(dst + j, pay_sig + (size_t)ks * g.HW + j);
-}
-
-// Per-bin records of slab ks, one 16-byte record per (row pair, w): {gain of row 2i, gain of row
-// 2i+1, stream position of row 2i's code << 4 | its bits, the same for row 2i+1}.  gain = 1/sigma
-// (encoding) or sigma (decoding).  The position counts from bit pbase of the slab's first word:
-// the bits of every bin before it in the slab, found by a sum over the earlier rows and a warp scan
-// along the row.  Rows past H (odd H) get 0 bits.
-template <class D>
-__device__ __forceinline__ void slab_records(const D& g, const unsigned char* bs, const float* sig, bool inv,
-                                             unsigned char* meta, uint32_t pbase) {
-  const int lane = threadIdx.x & 31, nwarps = blockDim.x >> 5, HP2 = 2 * row_pairs(g.H);
-  for (int kh = threadIdx.x >> 5; kh < HP2; kh += nwarps) {
-    const bool real = kh < g.H;
-    const int i = kh * g.W + lane;
-    const uint32_t b = (real && lane < g.W) ? bs[i] : 0u;
-    uint32_t before = 0;
-    const int lim = real ? kh * g.W : 0;
-    for (int q = lane; q < lim; q += 32) before += bs[q];
-    before = __reduce_add_sync(0xffffffffu, before);
-    uint32_t incl = b;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
-    }
-    if (lane < g.W) {
-      float gv = 0.f;
-      if (b) gv = inv ? __frcp_rn(sig[i]) : sig[i];
-      uint32_t* rec = reinterpret_cast<uint32_t*>(meta + ((size_t)(kh >> 1) * g.W + lane) * 16);
-      rec[kh & 1] = __float_as_uint(gv);
-      rec[2 + (kh & 1)] = ((pbase + before + incl - b) << 4) | b;
-    }
-  }
 }
 
 // The b-bit code at bit position off of a channel's word row (b >= 1).
@@ -294,36 +252,46 @@ __global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) fdct_hw_kernel(co
 }
 
 // ---------------------------------------------------------------------------------- inverse ---
+// Column-pair element (h, column pair wp, channel c) = {X[h][2wp], X[h][2wp+1]} at float2 index
+// (h*Wp + 2wp)*16 + c: rows 2kp and 2kp+1 of the cell grid hold row pair kp (forward
+// rearrangement) and its column pairs alike, so the inverse pass along W rewrites its row pair
+// in place.
+__device__ __forceinline__ int cp_index(int Wp, int h, int wp) { return (h * Wp + 2 * wp) * 16; }
+
+// Per slab: the tile is cleared, the slab's records (bins with bits: bin, bits, stream position,
+// sigma) are dequantized into it, then the inverse DCT along W runs on row pairs (in place, to
+// column pairs) and the inverse DCT along H on column pairs, into the fp32 volume V.
 template <int HC, int WC, int HX, int WX, int MODE>
-__global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) idct_hw_kernel(const __grid_constant__ Geom g, const __grid_constant__ UnitList ul,
-                                                      float* __restrict__ V, const uint32_t* __restrict__ slab_off,
-                                                      int spc) {
+__global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) idct_hw_kernel(const __grid_constant__ Geom g,
+                                                                              const __grid_constant__ UnitList ul,
+                                                                              float* __restrict__ V,
+                                                                              const uint32_t* __restrict__ index,
+                                                                              const uint4* __restrict__ recs, int spc) {
   extern __shared__ __align__(16) unsigned char smem[];
   const Dims<HX, WX> D(g);
   constexpr bool raw = MODE == kRaw;
   const HwLayout L = hw_layout(D.H, D.W, kLayDecode);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  const int HP = row_pairs(D.H), WP = row_pairs(D.W);
+  const int HP = row_pairs(D.H), WP = row_pairs(D.W), Wp = 2 * WP;
   const int chunk = blockIdx.x, u = blockIdx.z;
   const int ks0 = blockIdx.y * spc, ks1 = min(g.S, ks0 + spc);
-  const UnitDev& ud = ul.u[u];
-  const unsigned char* pay = ud.payload;
-  const uint32_t* P = slab_off + (size_t)u * unit_index_words(g.S);
+  const unsigned char* pay = ul.u[u].payload;
+  const uint32_t* P = index + (size_t)u * unit_index_words(g.S);
+  const uint32_t* NZ = P + g.S + 2;
   const bool ok = P[g.S + 1] != 0;   // the index kernel checked the header and the bit widths
   const uint32_t cstride = ok ? reinterpret_cast<const uint32_t*>(pay)[11] : 0u, sw = cstride / 4;
   const uint32_t* streams = reinterpret_cast<const uint32_t*>(pay + g.off_codes) + (size_t)chunk * kChunk * sw;
-  const unsigned char* pay_b = pay + kHeaderBytes;
-  const float* pay_sig = reinterpret_cast<const float*>(pay + g.off_sigma);
-  float2* tile = reinterpret_cast<float2*>(smem + L.tile);
-  const uint4* meta = reinterpret_cast<const uint4*>(smem + L.meta);
+  const uint4* urecs = recs + (size_t)u * g.N;
+  float* tilef = reinterpret_cast<float*>(smem + L.tile);
+  float2* tile = reinterpret_cast<float2*>(tilef);
   float* lvs = reinterpret_cast<float*>(smem + L.lv);
-  auto sbuf_of = [&](int ks) { return reinterpret_cast<uint32_t*>(smem + L.sbuf) + (ks & 1) * kChunk * L.words; };
-  auto bsl_of = [&](int ks) { return smem + L.bsl + (ks & 1) * L.bsl_stride; };
-  auto sig_of = [&](int ks) { return reinterpret_cast<float*>(smem + L.sig) + (ks & 1) * D.HW; };
+  auto slot = [&](int ks) { return L.nslot == 2 ? (ks & 1) : 0; };
+  auto sbuf_of = [&](int ks) { return reinterpret_cast<uint32_t*>(smem + L.sbuf) + slot(ks) * kChunk * L.words; };
+  auto rbuf_of = [&](int ks) { return reinterpret_cast<uint4*>(smem + L.meta) + slot(ks) * D.HW; };
 
-  // stream words of slab ks for the 32 channels, from word P(ks) >> 5 on, then two zero words
-  // that the readers' look-ahead may touch
-  auto issue_words = [&](int ks) {
+  // stream words of slab ks for the 32 channels from word P(ks) >> 5 on, then two zero words for
+  // the look-ahead of the code reads; and the slab's records
+  auto issue_slab = [&](int ks) {
     uint32_t* sb = sbuf_of(ks);
     const uint32_t p0 = P[ks], p1 = P[ks + 1];
     const uint32_t w0 = p0 >> 5;
@@ -333,58 +301,68 @@ __global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) idct_hw_kernel(co
         if (w < nw) cp_async4(sb + c * L.words + w, streams + (size_t)c * sw + w0 + w);
         else sb[c * L.words + w] = 0u;
       }
+    const uint32_t e0 = NZ[ks], m = NZ[ks + 1] - e0;
+    uint4* rb = rbuf_of(ks);
+    for (uint32_t e = threadIdx.x; e < m; e += blockDim.x) cp_async16(rb + e, urecs + e0 + e);
   };
   if (!raw) {
     for (int i = threadIdx.x; i < kLmLvTotal; i += blockDim.x) lvs[i] = c_lm_levels[i];
-    if (ok) {
-      issue_words(ks0);
-      issue_slab_bits(D, pay_b, ks0, bsl_of(ks0));
-      issue_sigma(D, pay_sig, ks0, sig_of(ks0));
-    }
+    if (ok) issue_slab(ks0);
     cp_async_commit();
   }
   float* vunit = V + (size_t)u * g.S * D.HW * g.n + chunk * kChunk + lane;
 
   for (int ks = ks0; ks < ks1; ++ks) {
-    const unsigned char* bs = bsl_of(ks) + (((size_t)ks * D.HW) & 15);
     cp_async_wait_all();
-    __syncthreads();  // slab ks's words are in place; slab ks - 1 is done
-    if (ok && !raw) {
-      if (ks + 1 < ks1) {
-        issue_words(ks + 1);
-        issue_slab_bits(D, pay_b, ks + 1, bsl_of(ks + 1));
-        issue_sigma(D, pay_sig, ks + 1, sig_of(ks + 1));
-        cp_async_commit();
-      }
-      slab_records(D, bs, sig_of(ks), false, smem + L.meta, P[ks] & 31u);
-      __syncthreads();
+    __syncthreads();  // slab ks's words and records are in place; slab ks - 1 is done
+    if (L.nslot == 2 && ok && !raw && ks + 1 < ks1) {
+      issue_slab(ks + 1);
+      cp_async_commit();
     }
-    // decode rows 2j, 2j+1 of warp j and run the inverse DCT along W; write column pairs
-    for (int kp = warp; kp < HP; kp += nwarps) {
-      float2 x[WC];
-      if (!ok) {
+    // clear the tile (rows past H and columns past W stay zero), then place the slab's values
+    {
+      float4* t4 = reinterpret_cast<float4*>(tilef);
+      const int n4 = (int)(L.tile_bytes / 16);
+      for (int i = threadIdx.x; i < n4; i += blockDim.x) t4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    __syncthreads();
+    if (ok && raw) {
+      const float* s = reinterpret_cast<const float*>(pay + g.off_codes + (size_t)(chunk * kChunk + lane) * cstride) +
+                       (size_t)ks * D.HW;
+      for (int i = warp; i < D.HW; i += nwarps) {
+        const int kh = i / D.W, t = i - kh * D.W;
+        tilef[(rp_index(Wp, kh >> 1, t) + lane) * 2 + (kh & 1)] = s[i];
+      }
+    } else if (ok) {
+      const uint32_t base = P[ks] & ~31u;
+      const int m = (int)(NZ[ks + 1] - NZ[ks]);
+      const uint4* rs = rbuf_of(ks);
+      const uint32_t* row = sbuf_of(ks) + lane * L.words;
+      const uint32_t slab0 = (uint32_t)ks * D.HW;
+      constexpr int kBlk = 4;   // records per warp step, loaded together
+      for (int e0 = warp * kBlk; e0 < m; e0 += nwarps * kBlk) {
+        uint4 r[kBlk];
 #pragma unroll
-        for (int t = 0; t < WC; ++t) x[t] = make_float2(0.f, 0.f);
-      } else if (raw) {
-        const float* s = reinterpret_cast<const float*>(pay + g.off_codes + (size_t)(chunk * kChunk + lane) * cstride) +
-                         (size_t)ks * D.HW + 2 * kp * D.W;
-        const bool second = 2 * kp + 1 < D.H;
+        for (int j = 0; j < kBlk; ++j)
+          if (e0 + j < m) r[j] = rs[e0 + j];
 #pragma unroll
-        for (int t = 0; t < WC; ++t)
-          if (t < D.W) x[t] = make_float2(s[t], second ? s[D.W + t] : 0.f);
-      } else {
-        const uint32_t* row = sbuf_of(ks) + lane * L.words;
-#pragma unroll
-        for (int t = 0; t < WC; ++t)
-          if (t < D.W) {
-            const uint4 m = meta[kp * D.W + t];
-            const uint32_t b0 = m.z & 15u, b1 = m.w & 15u;
-            float l0 = 0.f, l1 = 0.f;
-            if (b0) l0 = lvs[lm_lv_offset((int)b0) + read_code(row, m.z >> 4, b0)];
-            if (b1) l1 = lvs[lm_lv_offset((int)b1) + read_code(row, m.w >> 4, b1)];
-            x[t] = __fmul2_rn(make_float2(l0, l1), make_float2(__uint_as_float(m.x), __uint_as_float(m.y)));
+        for (int j = 0; j < kBlk; ++j)
+          if (e0 + j < m) {
+            const int b = (int)r[j].y;
+            const int i = (int)(r[j].x - slab0), kh = i / D.W, t = i - kh * D.W;
+            const float v = lvs[lm_lv_offset(b) + read_code(row, r[j].z - base, (uint32_t)b)] * __uint_as_float(r[j].w);
+            tilef[(rp_index(Wp, kh >> 1, t) + lane) * 2 + (kh & 1)] = v;
           }
       }
+    }
+    __syncthreads();
+    // inverse DCT along W on row pair kp, written back in place as column pairs
+    for (int kp = warp; kp < HP; kp += nwarps) {
+      float2 x[WC];
+#pragma unroll
+      for (int t = 0; t < WC; ++t)
+        if (t < D.W) x[t] = tile[rp_index(Wp, kp, t) + lane];
+      __syncwarp();   // the row pair is read before it is rewritten
       pencil<WC, WX, true>(x, D.W);
       const bool second = 2 * kp + 1 < D.H;
 #pragma unroll
@@ -392,17 +370,17 @@ __global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) idct_hw_kernel(co
         if (wp < WP) {
           const float2 a = x[2 * wp];
           const float2 b = (2 * wp + 1 < D.W) ? x[2 * wp + 1] : make_float2(0.f, 0.f);
-          tile[((2 * kp) * WP + wp) * kChunk + lane] = make_float2(a.x, b.x);
-          if (second) tile[((2 * kp + 1) * WP + wp) * kChunk + lane] = make_float2(a.y, b.y);
+          tile[cp_index(Wp, 2 * kp, wp) + lane] = make_float2(a.x, b.x);
+          if (second) tile[cp_index(Wp, 2 * kp + 1, wp) + lane] = make_float2(a.y, b.y);
         }
     }
     __syncthreads();
-    // inverse DCT along H on column pair (2j, 2j+1) of warp j; store to V
+    // inverse DCT along H on column pair wp; store to V
     for (int wp = warp; wp < WP; wp += nwarps) {
       float2 xh[HC];
 #pragma unroll
       for (int h = 0; h < HC; ++h)
-        if (h < D.H) xh[h] = tile[(h * WP + wp) * kChunk + lane];
+        if (h < D.H) xh[h] = tile[cp_index(Wp, h, wp) + lane];
       pencil<HC, HX, true>(xh, D.H);
       float* v = vunit + ((size_t)ks * D.HW + 2 * wp) * g.n;
       const bool two = 2 * wp + 1 < D.W;
@@ -413,6 +391,10 @@ __global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) idct_hw_kernel(co
           cell[0] = xh[h].x;
           if (two) cell[g.n] = xh[h].y;
         }
+    }
+    if (L.nslot == 1 && ok && !raw && ks + 1 < ks1) {   // the single slot is free once the records are used
+      issue_slab(ks + 1);
+      cp_async_commit();
     }
   }
   cp_async_wait_all();
@@ -426,7 +408,7 @@ __global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) idct_hw_kernel(co
 namespace {
 template <int HX, int WX>
 cudaError_t launch_hw(bool inverse, int mode, const Geom& g, const UnitList& ul, int nu, float* buf, float* partial,
-                      const uint32_t* slab_off, int spc, cudaStream_t st) {
+                      const uint32_t* slab_off, const uint4* recs, int spc, cudaStream_t st) {
   const HwLayout L = hw_layout(g.H, g.W, inverse ? kLayDecode : kLayStats);
   const dim3 grid(g.nch, (g.S + spc - 1) / spc, nu);
   const int threads = hw_threads(g.H, g.W);
@@ -442,8 +424,8 @@ cudaError_t launch_hw(bool inverse, int mode, const Geom& g, const UnitList& ul,
     kern<<<grid, threads, sm, st>>>(__VA_ARGS__);                                      \
   } while (0)
   if (inverse) {
-    if (mode == kRaw) TACTKV_GO((idct_hw_kernel<H, W, HX, WX, kRaw>), g, ul, buf, slab_off, spc);
-    else TACTKV_GO((idct_hw_kernel<H, W, HX, WX, kQuant>), g, ul, buf, slab_off, spc);
+    if (mode == kRaw) TACTKV_GO((idct_hw_kernel<H, W, HX, WX, kRaw>), g, ul, buf, slab_off, recs, spc);
+    else TACTKV_GO((idct_hw_kernel<H, W, HX, WX, kQuant>), g, ul, buf, slab_off, recs, spc);
   } else {
     TACTKV_GO((fdct_hw_kernel<H, W, HX, WX>), g, ul, buf, partial, spc);
   }
@@ -455,15 +437,16 @@ cudaError_t launch_hw(bool inverse, int mode, const Geom& g, const UnitList& ul,
 // The grids of the common layouts (medical volumes 16x16 and 24x24, video frames 14x14, the 8x8
 // test volume) have their own exact-size kernels; every other grid of the class runs the generic one.
 cudaError_t TACTKV_HWNAME(launch_axis_hw_)(bool inverse, int mode, const Geom& g, const UnitList& ul, int nu, float* buf,
-                                           float* partial, const uint32_t* slab_off, int spc, cudaStream_t st) {
+                                           float* partial, const uint32_t* slab_off, const uint4* recs, int spc,
+                                           cudaStream_t st) {
 #if TACTKV_HCLASS == 16 && TACTKV_WCLASS == 16
-  if (g.H == 16 && g.W == 16) return launch_hw<16, 16>(inverse, mode, g, ul, nu, buf, partial, slab_off, spc, st);
-  if (g.H == 14 && g.W == 14) return launch_hw<14, 14>(inverse, mode, g, ul, nu, buf, partial, slab_off, spc, st);
-  if (g.H == 8 && g.W == 8) return launch_hw<8, 8>(inverse, mode, g, ul, nu, buf, partial, slab_off, spc, st);
+  if (g.H == 16 && g.W == 16) return launch_hw<16, 16>(inverse, mode, g, ul, nu, buf, partial, slab_off, recs, spc, st);
+  if (g.H == 14 && g.W == 14) return launch_hw<14, 14>(inverse, mode, g, ul, nu, buf, partial, slab_off, recs, spc, st);
+  if (g.H == 8 && g.W == 8) return launch_hw<8, 8>(inverse, mode, g, ul, nu, buf, partial, slab_off, recs, spc, st);
 #elif TACTKV_HCLASS == 32 && TACTKV_WCLASS == 32
-  if (g.H == 24 && g.W == 24) return launch_hw<24, 24>(inverse, mode, g, ul, nu, buf, partial, slab_off, spc, st);
+  if (g.H == 24 && g.W == 24) return launch_hw<24, 24>(inverse, mode, g, ul, nu, buf, partial, slab_off, recs, spc, st);
 #endif
-  return launch_hw<0, 0>(inverse, mode, g, ul, nu, buf, partial, slab_off, spc, st);
+  return launch_hw<0, 0>(inverse, mode, g, ul, nu, buf, partial, slab_off, recs, spc, st);
 }
 
 // Shared memory and threads of one CTA (host queries used to size the slab ranges).

@@ -75,7 +75,7 @@ inline int length_class(int L) { return L <= 16 ? 16 : (L <= 32 ? 32 : 64); }
 cudaError_t launch_axis_s(int cls, bool inverse, const Geom& g, const UnitList& ul, int nu, float* buf,
                           cudaStream_t st);
 cudaError_t launch_axis_hw(int hcls, int wcls, bool inverse, int mode, const Geom& g, const UnitList& ul, int nu, float* buf,
-                           float* partial, const uint32_t* slab_off, int spc, cudaStream_t st);
+                           float* partial, const uint32_t* index, const uint4* recs, int spc, cudaStream_t st);
 void axis_hw_shape(int hcls, int wcls, const Geom& g, bool inverse, int mode, size_t* smem, int* threads);
 // Per-unit bit allocation: writes b, sigma and the header into the payload, P and NZ into the
 // unit's index block, the records {bin, bits, P_i, 1/sigma_i} of the bins with bits into recs
@@ -85,10 +85,11 @@ cudaError_t launch_allocate(const Geom& g, const UnitList& ul, int nu, const flo
 // Quantization and packing of the finished coefficients X (workspace volume) into the payloads.
 cudaError_t launch_pack(const Geom& g, const UnitList& ul, int nu, const float* X, const uint4* recs,
                         const uint32_t* index, cudaStream_t st);
-// Decoding index: checks every unit's header and bit widths, writes P(0..S) and the unit's ok
-// flag into its index block; a bad unit sets TACTKV_CORRUPT_PAYLOAD in *status.
-cudaError_t launch_decode_index(const Geom& g, const UnitList& ul, int nu, uint32_t* index, unsigned int* status,
-                                cudaStream_t st);
+// Decoding index: checks every unit's header and bit widths, writes P, the unit's ok flag and NZ
+// into its index block and the records {bin, bits, first stream bit, sigma} of the bins with bits
+// into recs; a bad unit sets TACTKV_CORRUPT_PAYLOAD in *status.
+cudaError_t launch_decode_index(const Geom& g, const UnitList& ul, int nu, uint32_t* index, uint4* recs,
+                                unsigned int* status, cudaStream_t st);
 
 #ifdef __CUDACC__
 // ------------------------------------------------------------------ float2 value operations ---

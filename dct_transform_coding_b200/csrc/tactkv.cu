@@ -22,7 +22,7 @@ cudaError_t launch_axis_s_32(bool, const Geom&, const UnitList&, int, float*, cu
 cudaError_t launch_axis_s_64(bool, const Geom&, const UnitList&, int, float*, cudaStream_t);
 #define TACTKV_DECL_HW(h, w)                                                                                 \
   cudaError_t launch_axis_hw_##h##_##w(bool, int, const Geom&, const UnitList&, int, float*, float*, const uint32_t*, \
-                                       int, cudaStream_t);                                                            \
+                                       const uint4*, int, cudaStream_t);                                              \
   void axis_hw_shape_##h##_##w(const Geom&, bool, int, size_t*, int*);
 TACTKV_DECL_HW(16, 16)
 TACTKV_DECL_HW(16, 32)
@@ -38,11 +38,12 @@ cudaError_t launch_axis_s(int cls, bool inverse, const Geom& g, const UnitList& 
 }
 
 cudaError_t launch_axis_hw(int hcls, int wcls, bool inverse, int mode, const Geom& g, const UnitList& ul, int nu,
-                           float* buf, float* partial, const uint32_t* slab_off, int spc, cudaStream_t st) {
-  if (hcls == 16 && wcls == 16) return launch_axis_hw_16_16(inverse, mode, g, ul, nu, buf, partial, slab_off, spc, st);
-  if (hcls == 16) return launch_axis_hw_16_32(inverse, mode, g, ul, nu, buf, partial, slab_off, spc, st);
-  if (wcls == 16) return launch_axis_hw_32_16(inverse, mode, g, ul, nu, buf, partial, slab_off, spc, st);
-  return launch_axis_hw_32_32(inverse, mode, g, ul, nu, buf, partial, slab_off, spc, st);
+                           float* buf, float* partial, const uint32_t* index, const uint4* recs, int spc,
+                           cudaStream_t st) {
+  if (hcls == 16 && wcls == 16) return launch_axis_hw_16_16(inverse, mode, g, ul, nu, buf, partial, index, recs, spc, st);
+  if (hcls == 16) return launch_axis_hw_16_32(inverse, mode, g, ul, nu, buf, partial, index, recs, spc, st);
+  if (wcls == 16) return launch_axis_hw_32_16(inverse, mode, g, ul, nu, buf, partial, index, recs, spc, st);
+  return launch_axis_hw_32_32(inverse, mode, g, ul, nu, buf, partial, index, recs, spc, st);
 }
 
 void axis_hw_shape(int hcls, int wcls, const Geom& g, bool inverse, int mode, size_t* smem, int* threads) {
@@ -275,7 +276,7 @@ static tactkv_status compress_impl(const tactkv_unit* units, int n_units, void* 
                          mark(0);
                          if (launch_axis_s(cs, false, g, ul, nu, w.big, st) != cudaSuccess) return TACTKV_CUDA;
                          mark(1);
-                         if (launch_axis_hw(ch, cw, false, kStats, g, ul, nu, w.big, w.partial, w.index,
+                         if (launch_axis_hw(ch, cw, false, kStats, g, ul, nu, w.big, w.partial, w.index, nullptr,
                                             slabs_per_cta(g, nu, false, kStats), st) != cudaSuccess)
                            return TACTKV_CUDA;
                          mark(2);
@@ -300,9 +301,9 @@ static tactkv_status decompress_impl(const tactkv_unit* units, int n_units, void
                          const int cs = length_class(g.S), ch = length_class(g.H), cw = length_class(g.W);
                          const int mode = (g.flags & TACTKV_NO_QUANT) ? kRaw : kQuant;
                          mark(0);
-                         if (launch_decode_index(g, ul, nu, w.index, w.status, st) != cudaSuccess)
+                         if (launch_decode_index(g, ul, nu, w.index, w.recs, w.status, st) != cudaSuccess)
                            return TACTKV_CUDA;
-                         if (launch_axis_hw(ch, cw, true, mode, g, ul, nu, w.big, nullptr, w.index,
+                         if (launch_axis_hw(ch, cw, true, mode, g, ul, nu, w.big, nullptr, w.index, w.recs,
                                             slabs_per_cta(g, nu, true, mode), st) != cudaSuccess)
                            return TACTKV_CUDA;
                          mark(1);
