@@ -159,6 +159,8 @@ tactkv_status check_unit(const tactkv_unit& u, const Geom& g, bool compress) {
   return TACTKV_OK;
 }
 
+thread_local int t_launches = 0;    // kernels launched by this thread's current or last call
+
 template <class F>
 tactkv_status for_each_wave(const tactkv_unit* units, int n_units, void* ws, size_t ws_bytes, bool compress,
                             F&& fn) {
@@ -268,10 +270,12 @@ static tactkv_status compress_impl(const tactkv_unit* units, int n_units, void* 
   auto mark = [&](int k) {
     if (events && events[k]) cudaEventRecord(static_cast<cudaEvent_t>(events[k]), st);
   };
+  t_launches = 0;
   return for_each_wave(units, n_units, workspace, workspace_bytes, true,
                        [&](const Geom& g, const UnitList& ul, int nu, unsigned char* ws) -> tactkv_status {
                          const WsView w = view(ws, g, nu);
                          const int cs = length_class(g.S), ch = length_class(g.H), cw = length_class(g.W);
+                         t_launches += 5;   // fdct_s, fdct_hw, reduce_var, allocate, pack
                          const int mode2 = (g.flags & TACTKV_NO_QUANT) ? kRaw : kQuant;
                          mark(0);
                          if (launch_axis_s(cs, false, g, ul, nu, w.big, st) != cudaSuccess) return TACTKV_CUDA;
@@ -295,10 +299,12 @@ static tactkv_status decompress_impl(const tactkv_unit* units, int n_units, void
   auto mark = [&](int k) {
     if (events && events[k]) cudaEventRecord(static_cast<cudaEvent_t>(events[k]), st);
   };
+  t_launches = 0;
   return for_each_wave(units, n_units, workspace, workspace_bytes, false,
                        [&](const Geom& g, const UnitList& ul, int nu, unsigned char* ws) -> tactkv_status {
                          const WsView w = view(ws, g, nu);
                          const int cs = length_class(g.S), ch = length_class(g.H), cw = length_class(g.W);
+                         t_launches += 3;   // decode_index, idct_hw, idct_s
                          const int mode = (g.flags & TACTKV_NO_QUANT) ? kRaw : kQuant;
                          mark(0);
                          if (launch_decode_index(g, ul, nu, w.index, w.recs, w.status, st) != cudaSuccess)
@@ -380,6 +386,8 @@ int tactkv_lloyd_max_table(int bits, double* levels, double* thresholds) {
   if (thresholds) memcpy(thresholds, kLmThresholds + lm_thr_offset(bits), sizeof(double) * (L - 1));
   return L;
 }
+
+int tactkv_last_launches(void) { return t_launches; }
 
 int tactkv_format_version(void) { return kVersion; }
 

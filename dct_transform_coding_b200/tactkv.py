@@ -38,7 +38,7 @@ HEADER_BYTES = 64
 EXPORTED = ("tactkv_payload_bytes", "tactkv_workspace_bytes", "tactkv_compress", "tactkv_decompress",
             "tactkv_compress_profiled", "tactkv_decompress_profiled", "tactkv_compress_noalloc",
             "tactkv_device_status",
-            "tactkv_status_string", "tactkv_lloyd_max_table", "tactkv_format_version")
+            "tactkv_status_string", "tactkv_lloyd_max_table", "tactkv_format_version", "tactkv_last_launches")
 
 
 class tactkv_unit(ctypes.Structure):
@@ -75,6 +75,8 @@ _lib.tactkv_lloyd_max_table.restype = ctypes.c_int
 _lib.tactkv_lloyd_max_table.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]
 _lib.tactkv_format_version.restype = ctypes.c_int
 _lib.tactkv_format_version.argtypes = []
+_lib.tactkv_last_launches.restype = ctypes.c_int
+_lib.tactkv_last_launches.argtypes = []
 
 
 class TactkvError(RuntimeError):
@@ -154,6 +156,11 @@ def tactkv_lloyd_max_table(bits: int):
 
 def tactkv_format_version() -> int:
     return int(_lib.tactkv_format_version())
+
+
+def tactkv_last_launches() -> int:
+    """Kernels launched by this thread's most recent compress / decompress call."""
+    return int(_lib.tactkv_last_launches())
 
 
 def _as_array(units):

@@ -156,6 +156,11 @@ int tactkv_lloyd_max_table(int bits, double* levels, double* thresholds);
 /* Version of the payload format this library writes and reads. */
 int tactkv_format_version(void);
 
+/* Number of kernels that the calling host thread's most recent tactkv_compress*,
+   tactkv_decompress* call launched (all its waves: 5 per compress wave, 3 per decompress wave;
+   0 after a call that failed before launching). */
+int tactkv_last_launches(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -159,6 +159,27 @@ def test_many_units_and_small_workspace():
     _check_batch(x, S, H, W, 3, units=[0, 130, 256, 259])
 
 
+def test_wave_splitting_and_launch_counts():
+    """12 units in one wave (5 compress kernels, 3 decompress kernels) give the same payloads and
+    outputs as 12 waves of one unit each (a one-unit workspace)."""
+    S, H, W, heads, D = 8, 8, 8, 2, 32
+    U = 12
+    x = torch.stack([make_unit(S, H, W, heads, D, rho=(0.9, 0.8, 0.85), nu=4.0, seed=40 + i, device=DEV)
+                     for i in range(U)])
+    pay = T.compress(x, S, H, W, 2)
+    assert T.tactkv_last_launches() == 5
+    y = T.decompress(pay, S, H, W, 2, heads=heads, head_dim=D, check=False)
+    assert T.tactkv_last_launches() == 3
+    units = T.make_units(x, S, H, W, 2, heads=heads, head_dim=D, payload=pay)
+    one = T.tactkv_workspace_bytes(units[:1])
+    ws = torch.zeros(one + 256, dtype=torch.uint8, device=DEV)
+    off = (-ws.data_ptr()) % 256
+    pay1, y1 = _round_trip(x, S, H, W, 2, workspace=ws[off:off + one])
+    assert T.tactkv_last_launches() == 3 * U
+    torch.cuda.synchronize()
+    assert torch.equal(pay, pay1) and torch.equal(y, y1)
+
+
 def test_deterministic():
     S, H, W, heads, D = 16, 8, 8, 2, 64
     x = make_unit(S, H, W, heads, D, rho=(0.9, 0.9, 0.9), nu=4.0, seed=1, device=DEV)[None]
