@@ -177,7 +177,8 @@ def generate() -> str:
         if b >= 3:
             tab, scale, offset = code_table(th32)
             qtab += tab
-    lines += [f"#define TACTKV_Q_CELLS {QK}",
+    lines += [f"#define TACTKV_LM_T2 {f32(th_all[th_off[1] + 2])}   // the positive 2-bit threshold",
+              f"#define TACTKV_Q_CELLS {QK}",
               f"#define TACTKV_Q_SCALE {f32(scale)}",
               f"#define TACTKV_Q_OFFSET {f32(offset)}",
               f"#define TACTKV_THR_PAD_TOTAL {len(pad_all)}",

@@ -8,10 +8,11 @@
 // uniform across the warp and only the 32 coefficient values differ.  Bins without bits are never
 // read.
 //
-// The CTA loads its records with cp.async, clears the word rows of its bit span in shared memory,
-// and each warp takes blocks of 8 records: it loads the 8 coefficient rows (128 bytes each, all
-// in flight at once), computes u = X * (1/sigma) and the code, and ORs the code into the channel's
-// word row at its stream position (records are independent of each other).  The span's words are
+// The CTA loads its records with cp.async and clears the word rows of its bit span in shared
+// memory.  Each warp takes blocks of 16 records; while it quantizes one block, the 16 coefficient
+// rows (128 bytes each) of its next block are in flight.  For a record it computes
+// u = X * (1/sigma) and the code, and ORs the code into the channel's word row at its stream
+// position (records are independent of each other).  The span's words are
 // then stored once; its first and last words may hold bits of the neighbouring ranges and are
 // ORed into the payload atomically (the allocation zeroes those words first).  The CTA with the
 // last record also writes the zero padding of the channel streams.
@@ -24,7 +25,7 @@ namespace tactkv {
 namespace {
 
 constexpr int kPackThreads = 256;
-constexpr int kPackBlock = 8;   // records per warp step
+constexpr int kPackBlock = 16;  // records per warp step
 
 // Thresholds of width b padded with two +inf, stored for b = 1, 2, ... in turn.
 __device__ __forceinline__ int thr_pad_offset(int b) { return (1 << b) + b - 3; }
@@ -35,10 +36,7 @@ __device__ __forceinline__ int thr_pad_offset(int b) { return (1 << b) + b - 3; 
 // two thresholds; the thresholds are padded with +inf).
 __device__ __forceinline__ uint32_t quant_code(float u, int b, const float* thr, const unsigned char* qcell) {
   if (b == 1) return u >= 0.f;
-  if (b == 2) {
-    const float t = thr[thr_pad_offset(2) + 2];
-    return (uint32_t)(u >= -t) + (uint32_t)(u >= 0.f) + (uint32_t)(u >= t);
-  }
+  if (b == 2) return (uint32_t)(u >= -TACTKV_LM_T2) + (uint32_t)(u >= 0.f) + (uint32_t)(u >= TACTKV_LM_T2);
   int j = __float2int_rd(fmaf(u, TACTKV_Q_SCALE, TACTKV_Q_OFFSET));
   j = min(max(j, 0), TACTKV_Q_CELLS - 1);
   const uint32_t c = qcell[(b - 3) * TACTKV_Q_CELLS + j];
@@ -63,7 +61,7 @@ __host__ __device__ inline PackLayout pack_layout() {
   auto p16 = [](size_t x) { return (x + 15) / 16 * 16; };
   L.words = ((8 * kPackRecs + 31) / 32 + 3) | 1;   // odd: 32 channels' rows in 32 different banks
   size_t o = 0;
-  L.rec = o; o += p16((size_t)kPackRecs * 16);
+  L.rec = o; o += p16((size_t)(kPackRecs + kPackBlock) * 16);   // + padding records
   L.sbuf = o; o += p16((size_t)kChunk * L.words * 4);
   L.thr = o; o += p16((size_t)TACTKV_THR_PAD_TOTAL * 4);
   L.qcell = o; o += p16((size_t)6 * TACTKV_Q_CELLS);
@@ -97,6 +95,13 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const __grid_constan
 
   for (int e = threadIdx.x; e < m; e += blockDim.x) cp_async16(rs + e, urecs + r0 + e);
   cp_async_commit();
+  // the list is padded to whole blocks with records that set one bit of word 257 of a row, which
+  // is past every range's span (at most 8 * kPackRecs + 31 bits = 257 words) and never stored
+  const int m_pad = (m + kPackBlock - 1) / kPackBlock * kPackBlock;
+  {
+    const uint32_t A0 = m > 0 ? urecs[r0].z : 0u;
+    for (int e = m + threadIdx.x; e < m_pad; e += blockDim.x) rs[e] = make_uint4(0u, 1u, (A0 & ~31u) + 32u * 257u, 0u);
+  }
   for (int i = threadIdx.x; i < TACTKV_THR_PAD_TOTAL; i += blockDim.x) thr[i] = c_thr_pad[i];
   for (int i = threadIdx.x; i < 6 * TACTKV_Q_CELLS; i += blockDim.x) qcell[i] = c_qcell[i];
   // bit span [A, B) of the range; its words from word A >> 5 on are assembled in shared memory
@@ -110,22 +115,30 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const __grid_constan
   __syncthreads();
 
   uint32_t* row = sbuf + lane * L.words;
-  for (int e0 = warp * kPackBlock; e0 < m; e0 += nwarps * kPackBlock) {
-    uint4 r[kPackBlock];
-    float x[kPackBlock];
+  // blocks of kPackBlock records per warp; the next block's coefficients are loaded while this
+  // one is quantized
+  const int stride = nwarps * kPackBlock;
+  int e0 = warp * kPackBlock;
+  float x[kPackBlock];
+  if (e0 < m_pad) {
 #pragma unroll
-    for (int j = 0; j < kPackBlock; ++j)
-      if (e0 + j < m) {
-        r[j] = rs[e0 + j];
-        x[j] = __ldcs(xu + (size_t)r[j].x * g.n);
-      }
+    for (int j = 0; j < kPackBlock; ++j) x[j] = __ldcs(xu + (size_t)rs[e0 + j].x * g.n);
+  }
+  for (; e0 < m_pad; e0 += stride) {
+    float xn[kPackBlock];
+    const int e1 = e0 + stride;
+    if (e1 < m_pad) {
 #pragma unroll
-    for (int j = 0; j < kPackBlock; ++j)
-      if (e0 + j < m) {
-        const int b = (int)r[j].y;
-        const float uq = x[j] * __uint_as_float(r[j].w);
-        emit_code(row, r[j].z - base, (uint32_t)b, quant_code(uq, b, thr, qcell));
-      }
+      for (int j = 0; j < kPackBlock; ++j) xn[j] = __ldcs(xu + (size_t)rs[e1 + j].x * g.n);
+    }
+#pragma unroll
+    for (int j = 0; j < kPackBlock; ++j) {
+      const uint4 r = rs[e0 + j];
+      const int b = (int)r.y;
+      emit_code(row, r.z - base, (uint32_t)b, quant_code(x[j] * __uint_as_float(r.w), b, thr, qcell));
+    }
+#pragma unroll
+    for (int j = 0; j < kPackBlock; ++j) x[j] = xn[j];
   }
   __syncthreads();
   // the span's words; the first and the last may be shared with the neighbouring ranges
