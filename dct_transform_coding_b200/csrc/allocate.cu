@@ -303,8 +303,12 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
 // ----------------------------------------------------------------------------- decode index ---
 // One CTA per unit: the header must describe exactly the unit the caller asked for, every bit
 // width must be <= 8 and their sum must equal the header's code_bits; then P(k_s), NZ(k_s) and the
-// records {bin, bits, first stream bit, sigma} of the bins with bits are rebuilt from the payload
-// (one warp per slab: a ballot gives each record's slot, a scan its stream position).
+// records of the bins with bits are rebuilt from the payload (one warp per slab: a ballot gives
+// each record's slot, a scan its stream position).  A decoding record is
+//   {the bin's float offset in the inverse kernel's slab tile (lane 0),
+//    code mask 2^b - 1 | offset of the b-bit levels in the level table << 8,
+//    first stream bit, sigma},
+// so the 32 chunk CTAs that decode a bin do no index arithmetic of their own.
 __global__ void __launch_bounds__(256) decode_index_kernel(const __grid_constant__ Geom g,
                                                            const __grid_constant__ UnitList ul,
                                                            uint32_t* __restrict__ index, uint4* __restrict__ recs,
@@ -389,7 +393,13 @@ __global__ void __launch_bounds__(256) decode_index_kernel(const __grid_constant
           if (lane >= o) incl += t;
         }
         const uint32_t nzmask = __ballot_sync(0xffffffffu, v > 0);
-        if (v) urecs[slot + __popc(nzmask & below)] = make_uint4((uint32_t)i, v, pos + incl - v, __float_as_uint(sig[i]));
+        if (v) {
+          const int j = i0 + lane, kh = j / g.W, t = j - kh * g.W, Wp = 2 * ((g.W + 1) >> 1);
+          const uint32_t cell2 = (uint32_t)(((2 * (kh >> 1) + (t & 1)) * Wp + (t & ~1)) * 16);   // row-pair float2 cell
+          const uint32_t mask_lv = ((1u << v) - 1u) | ((uint32_t)lm_lv_offset((int)v) << 8);
+          urecs[slot + __popc(nzmask & below)] =
+              make_uint4(cell2 * 2 + (uint32_t)(kh & 1), mask_lv, pos + incl - v, __float_as_uint(sig[i]));
+        }
         slot += __popc(nzmask);
         pos += __shfl_sync(0xffffffffu, incl, 31);
       }

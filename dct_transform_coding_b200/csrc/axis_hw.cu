@@ -114,11 +114,6 @@ __device__ __forceinline__ void issue_tile(const D& g, const float* slab_src, fl
                  slab_src + (size_t)(r * g.W + w) * g.n + (threadIdx.x & 7) * 4);
 }
 
-// The b-bit code at bit position off of a channel's word row (b >= 1).
-__device__ __forceinline__ uint32_t read_code(const uint32_t* row, uint32_t off, uint32_t b) {
-  const uint32_t w = off >> 5;
-  return __funnelshift_r(row[w], row[w + 1], off & 31u) & ((1u << b) - 1u);
-}
 
 // Forward rearrangement.  The tile's cells (h, w) sit at cell index h*Wp + w.  After the pass
 // along H, element (row pair kp, column w, channel c) = {X[2kp][w], X[2kp+1][w]} (float2) sits at
@@ -337,9 +332,9 @@ __global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) idct_hw_kernel(co
       const uint32_t base = P[ks] & ~31u;
       const int m = (int)(NZ[ks + 1] - NZ[ks]);
       const uint4* rs = rbuf_of(ks);
-      const uint32_t* row = sbuf_of(ks) + lane * L.words;
-      const uint32_t slab0 = (uint32_t)ks * D.HW;
-      constexpr int kBlk = 4;   // records per warp step, loaded together
+      const uint32_t* row = sbuf_of(ks) + lane * L.words;   // this lane's channel stream
+      float* tl = tilef + 2 * lane;
+      constexpr int kBlk = 8;   // records per warp step, loaded together
       for (int e0 = warp * kBlk; e0 < m; e0 += nwarps * kBlk) {
         uint4 r[kBlk];
 #pragma unroll
@@ -348,10 +343,10 @@ __global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) idct_hw_kernel(co
 #pragma unroll
         for (int j = 0; j < kBlk; ++j)
           if (e0 + j < m) {
-            const int b = (int)r[j].y;
-            const int i = (int)(r[j].x - slab0), kh = i / D.W, t = i - kh * D.W;
-            const float v = lvs[lm_lv_offset(b) + read_code(row, r[j].z - base, (uint32_t)b)] * __uint_as_float(r[j].w);
-            tilef[(rp_index(Wp, kh >> 1, t) + lane) * 2 + (kh & 1)] = v;
+            // record: tile offset, code mask | level offset << 8, stream position, sigma
+            const uint32_t off = r[j].z - base, w = off >> 5;
+            const uint32_t code = __funnelshift_r(row[w], row[w + 1], off) & (r[j].y & 0xffu);
+            tl[r[j].x] = lvs[(r[j].y >> 8) + code] * __uint_as_float(r[j].w);
           }
       }
     }
