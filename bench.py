@@ -249,9 +249,10 @@ def main():
         check(T.tactkv_decompress(du, ws.data_ptr(), ws.numel(), sp), "decompress")
         return n + T.tactkv_last_launches()
 
-    def profiled_step(ev_c, ev_d):
-        check(T.tactkv_compress_profiled(cu, ws.data_ptr(), ws.numel(), sp, [e.cuda_event for e in ev_c]), "compress")
-        check(T.tactkv_decompress_profiled(du, ws.data_ptr(), ws.numel(), sp, [e.cuda_event for e in ev_d]),
+    def profiled_step(cu_p, du_p, ev_c, ev_d):
+        check(T.tactkv_compress_profiled(cu_p, ws.data_ptr(), ws.numel(), sp, [e.cuda_event for e in ev_c]),
+              "compress")
+        check(T.tactkv_decompress_profiled(du_p, ws.data_ptr(), ws.numel(), sp, [e.cuda_event for e in ev_d]),
               "decompress")
 
     for _ in range(args.warmup):
@@ -284,22 +285,27 @@ def main():
 
     # per-kernel attribution: separate profiled steps (the profiled entry points record an event at
     # every kernel boundary); not part of the timed region above
+    # a call records the stage events again in every wave, so the profiled steps run one wave's
+    # worth of units (at most 256) and the times are scaled to the whole batch
+    n_sub = min(U, 256)
+    cu_p, du_p = cu[:n_sub], du[:n_sub]
+    scale = U / n_sub
     n_prof = min(5, args.steps)
     evs_c = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_prof)]
     evs_d = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_prof)]
     for e in [e for es in evs_c + evs_d for e in es]:
         e.record(stream)   # torch creates the CUDA event on its first record
     for k in range(n_prof):
-        profiled_step(evs_c[k], evs_d[k])
+        profiled_step(cu_p, du_p, evs_c[k], evs_d[k])
     torch.cuda.synchronize(dev)
     names_c = ["fdct_s", "fdct_hw_stats", "reduce_var+allocate", "pack"]
     names_d = ["idct_hw", "idct_s"]
-    kern = {n: statistics.mean(evs_c[k][i].elapsed_time(evs_c[k][i + 1]) for k in range(n_prof))
+    kern = {n: scale * statistics.mean(evs_c[k][i].elapsed_time(evs_c[k][i + 1]) for k in range(n_prof))
             for i, n in enumerate(names_c)}
-    kern.update({n: statistics.mean(evs_d[k][i].elapsed_time(evs_d[k][i + 1]) for k in range(n_prof))
+    kern.update({n: scale * statistics.mean(evs_d[k][i].elapsed_time(evs_d[k][i + 1]) for k in range(n_prof))
                  for i, n in enumerate(names_d)})
-    ms_c = statistics.mean(evs_c[k][0].elapsed_time(evs_c[k][4]) for k in range(n_prof))
-    ms_d = statistics.mean(evs_d[k][0].elapsed_time(evs_d[k][2]) for k in range(n_prof))
+    ms_c = scale * statistics.mean(evs_c[k][0].elapsed_time(evs_c[k][4]) for k in range(n_prof))
+    ms_d = scale * statistics.mean(evs_d[k][0].elapsed_time(evs_d[k][2]) for k in range(n_prof))
 
     # bytes: payload sizes actually written (header field total_bytes)
     hdr = payload[:, :64].cpu().numpy()

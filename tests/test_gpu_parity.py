@@ -228,15 +228,26 @@ def test_payload_bytes_match_oracle_format():
     ("video", 1, [0, 895]),
 ])
 def test_full_size_sampled_units(name, bits, pick):
-    """The benchmark workloads' exact shapes; the oracle checks sampled units of the batch."""
+    """The benchmark workloads at full size: the whole batch is compressed and decompressed in the
+    launch configuration the benchmark uses (one call, waves of up to 256 units, workspace sized
+    by tactkv_workspace_bytes), and the oracle checks sampled units of it."""
+    from dct_transform_coding_b200.workloads import make_batch
     w = WORKLOADS[name]
     all_units = list(w.units())
-    x = torch.stack([make_workload_unit(w, *all_units[u], device=DEV) for u in pick])
-    layers = [all_units[u][1] for u in pick]
-    kvs = [all_units[u][2] for u in pick]
-    reports, _, _ = _check_batch(x, w.S, w.H, w.W, bits, layers=layers, kvs=kvs)
-    for r in reports:
-        print(name, bits, r)
+    x = make_batch(w, device=DEV)
+    layers = [u[1] for u in all_units]
+    kvs = [u[2] for u in all_units]
+    pay, y = _round_trip(x, w.S, w.H, w.W, bits, layers=layers, kvs=kvs)
+    heads, D = w.heads, w.head_dim
+    fp32 = x.dtype == torch.float32
+    io_round = (lambda v: np.asarray(v, np.float32).astype(np.float64)) if fp32 else O.to_bf16
+    for u in pick:
+        r = compare_unit(x[u].double().cpu().numpy(), pay[u].cpu().numpy().tobytes(), y[u].double().cpu().numpy(),
+                         S=w.S, H=w.H, W=w.W, heads=heads, head_dim=D, bits=bits, layer=layers[u], kv=kvs[u],
+                         io_round=io_round, report=[])
+        print(name, bits, u, r)
+    del x, y, pay
+    torch.cuda.empty_cache()
 
 
 # ------------------------------------------------------------------------------ error paths ---
