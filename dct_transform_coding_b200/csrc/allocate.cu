@@ -303,12 +303,11 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
 // ----------------------------------------------------------------------------- decode index ---
 // One CTA per unit: the header must describe exactly the unit the caller asked for, every bit
 // width must be <= 8 and their sum must equal the header's code_bits; then P(k_s), NZ(k_s) and the
-// records of the bins with bits are rebuilt from the payload (one warp per slab: a ballot gives
-// each record's slot, a scan its stream position).  A decoding record is
-//   {the bin's float offset in the inverse kernel's slab tile (lane 0),
-//    code mask 2^b - 1 | offset of the b-bit levels in the level table << 8,
-//    first stream bit, sigma},
-// so the 32 chunk CTAs that decode a bin do no index arithmetic of their own.
+// decoding records are rebuilt from the payload (one warp per slab, a scan gives every bin's stream
+// position).  Decoding records are dense, one per (slab, row pair, column), so that the inverse
+// kernel's warp for a row pair reads its two rows' bins in order: sigma and position << 8 | code
+// mask for each of the two rows.  The 32 chunk CTAs that decode a bin do no index arithmetic of
+// their own.
 __global__ void __launch_bounds__(256) decode_index_kernel(const __grid_constant__ Geom g,
                                                            const __grid_constant__ UnitList ul,
                                                            uint32_t* __restrict__ index, uint4* __restrict__ recs,
@@ -378,31 +377,37 @@ __global__ void __launch_bounds__(256) decode_index_kernel(const __grid_constant
     if (!ok) set_status(status, TACTKV_CORRUPT_PAYLOAD);
   }
   if (ok && !raw) {
+    // dense decoding records, one per (slab, row pair kp, column t) at ks*HP*W + kp*W + t:
+    // {sigma of row 2kp, sigma of row 2kp+1, position << 8 | code mask of each row}; a bin without
+    // bits (and the padding row of an odd H) has sigma 0 and mask 0
     const float* sig = reinterpret_cast<const float*>(pay + g.off_sigma);
-    uint4* urecs = recs + (size_t)u * g.N;
-    const uint32_t below = (1u << lane) - 1u;
+    const int HP = (g.H + 1) >> 1, RP = HP * g.W;
+    uint32_t* urec32 = reinterpret_cast<uint32_t*>(recs + (size_t)u * g.N);
     for (int k = warp; k < g.S; k += nwarps) {
-      uint32_t slot = s_NZ[k], pos = s_P[k];
+      uint32_t pos = s_P[k];
       for (int i0 = 0; i0 < g.HW; i0 += 32) {
-        const int i = k * g.HW + i0 + lane;
-        const uint32_t v = i0 + lane < g.HW ? b[i] : 0u;
+        const int j = i0 + lane, i = k * g.HW + j;
+        const uint32_t v = j < g.HW ? b[i] : 0u;
         uint32_t incl = v;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
           const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
           if (lane >= o) incl += t;
         }
-        const uint32_t nzmask = __ballot_sync(0xffffffffu, v > 0);
-        if (v) {
-          const int j = i0 + lane, kh = j / g.W, t = j - kh * g.W, Wp = 2 * ((g.W + 1) >> 1);
-          const uint32_t cell2 = (uint32_t)(((2 * (kh >> 1) + (t & 1)) * Wp + (t & ~1)) * 16);   // row-pair float2 cell
-          const uint32_t mask_lv = ((1u << v) - 1u) | ((uint32_t)lm_lv_offset((int)v) << 8);
-          urecs[slot + __popc(nzmask & below)] =
-              make_uint4(cell2 * 2 + (uint32_t)(kh & 1), mask_lv, pos + incl - v, __float_as_uint(sig[i]));
+        if (j < g.HW) {
+          const int kh = j / g.W, t = j - kh * g.W;
+          uint32_t* rec = urec32 + ((size_t)k * RP + (size_t)(kh >> 1) * g.W + t) * 4;
+          rec[kh & 1] = v ? __float_as_uint(sig[i]) : 0u;
+          rec[2 + (kh & 1)] = ((pos + incl - v) << 8) | ((1u << v) - 1u);
         }
-        slot += __popc(nzmask);
         pos += __shfl_sync(0xffffffffu, incl, 31);
       }
+      if (g.H & 1)   // the padding row H of the last row pair
+        for (int t = lane; t < g.W; t += 32) {
+          uint32_t* rec = urec32 + ((size_t)k * RP + (size_t)(HP - 1) * g.W + t) * 4;
+          rec[1] = 0u;
+          rec[3] = 0u;
+        }
     }
   }
 }

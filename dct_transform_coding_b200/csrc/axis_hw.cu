@@ -253,9 +253,10 @@ __global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) fdct_hw_kernel(co
 // in place.
 __device__ __forceinline__ int cp_index(int Wp, int h, int wp) { return (h * Wp + 2 * wp) * 16; }
 
-// Per slab: the tile is cleared, the slab's records (bins with bits: bin, bits, stream position,
-// sigma) are dequantized into it, then the inverse DCT along W runs on row pairs (in place, to
-// column pairs) and the inverse DCT along H on column pairs, into the fp32 volume V.
+// Per slab: the stream words and the slab's dense records (per row pair and column: sigma and
+// stream position of the two rows' bins) arrive by cp.async, the next slab's meanwhile.  Warp kp
+// decodes rows 2kp and 2kp+1 in registers and runs the inverse DCT along W, writing column pairs;
+// then the inverse DCT along H runs on column pairs, into the fp32 volume V.
 template <int HC, int WC, int HX, int WX, int MODE>
 __global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) idct_hw_kernel(const __grid_constant__ Geom g,
                                                                               const __grid_constant__ UnitList ul,
@@ -272,13 +273,11 @@ __global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) idct_hw_kernel(co
   const int ks0 = blockIdx.y * spc, ks1 = min(g.S, ks0 + spc);
   const unsigned char* pay = ul.u[u].payload;
   const uint32_t* P = index + (size_t)u * unit_index_words(g.S);
-  const uint32_t* NZ = P + g.S + 2;
   const bool ok = P[g.S + 1] != 0;   // the index kernel checked the header and the bit widths
   const uint32_t cstride = ok ? reinterpret_cast<const uint32_t*>(pay)[11] : 0u, sw = cstride / 4;
   const uint32_t* streams = reinterpret_cast<const uint32_t*>(pay + g.off_codes) + (size_t)chunk * kChunk * sw;
   const uint4* urecs = recs + (size_t)u * g.N;
-  float* tilef = reinterpret_cast<float*>(smem + L.tile);
-  float2* tile = reinterpret_cast<float2*>(tilef);
+  float2* tile = reinterpret_cast<float2*>(smem + L.tile);
   float* lvs = reinterpret_cast<float*>(smem + L.lv);
   auto slot = [&](int ks) { return L.nslot == 2 ? (ks & 1) : 0; };
   auto sbuf_of = [&](int ks) { return reinterpret_cast<uint32_t*>(smem + L.sbuf) + slot(ks) * kChunk * L.words; };
@@ -296,9 +295,9 @@ __global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) idct_hw_kernel(co
         if (w < nw) cp_async4(sb + c * L.words + w, streams + (size_t)c * sw + w0 + w);
         else sb[c * L.words + w] = 0u;
       }
-    const uint32_t e0 = NZ[ks], m = NZ[ks + 1] - e0;
+    const int RP = row_pairs(D.H) * D.W;   // dense records of the slab
     uint4* rb = rbuf_of(ks);
-    for (uint32_t e = threadIdx.x; e < m; e += blockDim.x) cp_async16(rb + e, urecs + e0 + e);
+    for (int e = threadIdx.x; e < RP; e += blockDim.x) cp_async16(rb + e, urecs + (size_t)ks * RP + e);
   };
   if (!raw) {
     for (int i = threadIdx.x; i < kLmLvTotal; i += blockDim.x) lvs[i] = c_lm_levels[i];
@@ -314,50 +313,42 @@ __global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) idct_hw_kernel(co
       issue_slab(ks + 1);
       cp_async_commit();
     }
-    // clear the tile (rows past H and columns past W stay zero), then place the slab's values
-    {
-      float4* t4 = reinterpret_cast<float4*>(tilef);
-      const int n4 = (int)(L.tile_bytes / 16);
-      for (int i = threadIdx.x; i < n4; i += blockDim.x) t4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    __syncthreads();
-    if (ok && raw) {
-      const float* s = reinterpret_cast<const float*>(pay + g.off_codes + (size_t)(chunk * kChunk + lane) * cstride) +
-                       (size_t)ks * D.HW;
-      for (int i = warp; i < D.HW; i += nwarps) {
-        const int kh = i / D.W, t = i - kh * D.W;
-        tilef[(rp_index(Wp, kh >> 1, t) + lane) * 2 + (kh & 1)] = s[i];
-      }
-    } else if (ok) {
-      const uint32_t base = P[ks] & ~31u;
-      const int m = (int)(NZ[ks + 1] - NZ[ks]);
-      const uint4* rs = rbuf_of(ks);
-      const uint32_t* row = sbuf_of(ks) + lane * L.words;   // this lane's channel stream
-      float* tl = tilef + 2 * lane;
-      constexpr int kBlk = 8;   // records per warp step, loaded together
-      for (int e0 = warp * kBlk; e0 < m; e0 += nwarps * kBlk) {
-        uint4 r[kBlk];
-#pragma unroll
-        for (int j = 0; j < kBlk; ++j)
-          if (e0 + j < m) r[j] = rs[e0 + j];
-#pragma unroll
-        for (int j = 0; j < kBlk; ++j)
-          if (e0 + j < m) {
-            // record: tile offset, code mask | level offset << 8, stream position, sigma
-            const uint32_t off = r[j].z - base, w = off >> 5;
-            const uint32_t code = __funnelshift_r(row[w], row[w + 1], off) & (r[j].y & 0xffu);
-            tl[r[j].x] = lvs[(r[j].y >> 8) + code] * __uint_as_float(r[j].w);
-          }
-      }
-    }
-    __syncthreads();
-    // inverse DCT along W on row pair kp, written back in place as column pairs
+    // decode rows 2kp, 2kp+1 of warp kp (dequantize in registers) and run the inverse DCT along W;
+    // column pairs go to the tile
+    const uint32_t base = ok && !raw ? (P[ks] & ~31u) : 0u;
+    const uint4* rs = rbuf_of(ks);
+    const uint32_t* row = sbuf_of(ks) + lane * L.words;   // this lane's channel stream
     for (int kp = warp; kp < HP; kp += nwarps) {
       float2 x[WC];
+      if (!ok) {
 #pragma unroll
-      for (int t = 0; t < WC; ++t)
-        if (t < D.W) x[t] = tile[rp_index(Wp, kp, t) + lane];
-      __syncwarp();   // the row pair is read before it is rewritten
+        for (int t = 0; t < WC; ++t) x[t] = make_float2(0.f, 0.f);
+      } else if (raw) {
+        const float* s = reinterpret_cast<const float*>(pay + g.off_codes + (size_t)(chunk * kChunk + lane) * cstride) +
+                         (size_t)ks * D.HW + 2 * kp * D.W;
+        const bool second = 2 * kp + 1 < D.H;
+#pragma unroll
+        for (int t = 0; t < WC; ++t)
+          if (t < D.W) x[t] = make_float2(s[t], second ? s[D.W + t] : 0.f);
+      } else {
+#pragma unroll
+        for (int t = 0; t < WC; ++t)
+          if (t < D.W) {
+            // record: sigma of each row, position << 8 | code mask of each row (mask 0: no bits)
+            const uint4 m = rs[kp * D.W + t];
+            float l0 = 0.f, l1 = 0.f;
+            const uint32_t k0 = m.z & 0xffu, k1 = m.w & 0xffu;
+            if (k0) {
+              const uint32_t off = (m.z >> 8) - base, w = off >> 5;
+              l0 = lvs[k0 - 1u + (__funnelshift_r(row[w], row[w + 1], off) & k0)];
+            }
+            if (k1) {
+              const uint32_t off = (m.w >> 8) - base, w = off >> 5;
+              l1 = lvs[k1 - 1u + (__funnelshift_r(row[w], row[w + 1], off) & k1)];
+            }
+            x[t] = __fmul2_rn(make_float2(l0, l1), make_float2(__uint_as_float(m.x), __uint_as_float(m.y)));
+          }
+      }
       pencil<WC, WX, true>(x, D.W);
       const bool second = 2 * kp + 1 < D.H;
 #pragma unroll
