@@ -7,11 +7,14 @@
 // keys sigma_i^2 4^-k (k = 0..7) that are >= 2 theta, and each greedy step adds the largest
 // missing key or drops the smallest kept one, so the result is the set of the B largest keys
 // (ties to the lower bin index).  This kernel selects that set directly and exactly:
+//   * the B-th largest key K is found by radix selection on its fp64 bit pattern (patterns of
+//     positive doubles order like their values): a histogram of all keys' exponents, then 8-bit
+//     digits of the mantissa among the keys with K's exponent -- 8 passes; if any key would be
+//     subnormal, by bisection over the patterns instead;
 //   * count(v) = #keys >= v is evaluated per bin from the fp64 exponent and mantissa fields
 //     (sigma^2 4^-k >= v  <=>  2k <= e(sigma^2) - e(v) - 1 + [m(sigma^2) >= m(v)]);
-//   * the B-th largest key is found by bisection over the 64-bit patterns of positive doubles
-//     (monotone in value), ~62 steps of one block-wide count;
-//   * keys equal to that value are handed out in bin order until the budget is met.
+//   * keys above K are all taken, keys equal to K are handed out in bin order until the budget
+//     is met.
 // If the active bins cannot absorb B (8 * #active <= B) every active bin gets 8 bits.
 //
 // The kernel also writes the first stream bit P(k_s) of every S slab (the same for every
@@ -24,7 +27,8 @@
 namespace tactkv {
 namespace {
 
-constexpr size_t kAllocSmemVar = 200 * 1024;   // variances kept in shared memory up to N = 25600 bins
+constexpr size_t kAllocSmemVar = 192 * 1024;   // variances kept in shared memory up to N = 24576 bins
+constexpr int kExpBuckets = 2048;                // biased exponents of fp64
 
 // Number of keys var * 4^-k (k = 0..7) that are >= v, exactly; var > 0, v >= 0.
 __device__ __forceinline__ int key_count(double var, double v) {
@@ -103,6 +107,28 @@ __device__ void slab_scan(const uint32_t* s_slab, int S, uint32_t* out) {
   if (lane == 0) out[S] = run;
 }
 
+// Largest bucket D of hist[0..nb) with sum_{d >= D} hist[d] >= need (need >= 1, reached); returns D,
+// puts sum_{d > D} hist[d] in *above and hist[D] in *count.  rev: scratch of nb words (may be the
+// storage of another histogram, not hist itself).  All threads call it.
+__device__ int select_bucket(const uint32_t* hist, int nb, uint32_t need, uint32_t* rev, uint32_t* s_warp,
+                             int* s_pick, uint32_t* s_above, uint32_t* s_count, uint32_t* above, uint32_t* count) {
+  for (int j = threadIdx.x; j < nb; j += blockDim.x) rev[j] = hist[nb - 1 - j];
+  __syncthreads();
+  block_exclusive_scan(rev, nb, s_warp);   // rev[j] = number of keys in buckets above nb-1-j
+  for (int j = threadIdx.x; j < nb; j += blockDim.x) {
+    const uint32_t pre = rev[j], here = hist[nb - 1 - j];
+    if (pre < need && need <= pre + here) {
+      *s_pick = nb - 1 - j;
+      *s_above = pre;
+      *s_count = here;
+    }
+  }
+  __syncthreads();
+  *above = *s_above;
+  *count = *s_count;
+  return *s_pick;
+}
+
 __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_constant__ Geom g,
                                                                  const __grid_constant__ UnitList ul,
                                                                  double* __restrict__ var_ws, bool var_in_smem,
@@ -116,11 +142,15 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
   __shared__ uint32_t s_P[kMaxSlabs + 1];
   __shared__ uint32_t s_NZ[kMaxSlabs + 1];
   __shared__ uint32_t s_bpos[kMaxN / kPackRecs + 1];
+  __shared__ uint32_t s_hist[kExpBuckets], s_rev[kExpBuckets];
+  __shared__ int s_pick, s_emin;
+  __shared__ uint32_t s_above, s_count;
+  __shared__ unsigned long long s_mant;
   extern __shared__ __align__(16) unsigned char smem_var[];
   const int u = blockIdx.x;
   const UnitDev& ud = ul.u[u];
   unsigned char* pay = ud.payload;
-  // the bisection reads every variance ~64 times: keep them in shared memory when they fit
+  // the selection passes read every variance several times: keep them in shared memory when they fit
   double* var = var_in_smem ? reinterpret_cast<double*>(smem_var) : var_ws + (size_t)u * g.N;
   const bool raw = g.flags & TACTKV_NO_QUANT;
   // each thread owns a contiguous range of bins, so thread order is bin order
@@ -130,6 +160,9 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
   // 1. sigma^2 (reduced over the channel chunks by reduce_var_kernel)
   long long act = 0;
   double vmax = 0.0;
+  int emin = 2047;   // smallest biased exponent of a positive variance
+  if (threadIdx.x == 0) s_emin = 2047;
+  __syncthreads();
   const double* var_g = var_ws + (size_t)u * g.N;
   // the counting passes take bins interleaved across threads (bin i to thread i mod blockDim):
   // consecutive threads read consecutive variances, without bank conflicts
@@ -138,27 +171,95 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
     var[i] = v;
     act += v > 0.0;
     vmax = fmax(vmax, v);
+    if (v > 0.0) emin = min(emin, (int)(__double_as_longlong(v) >> 52));
   }
+  atomicMin(&s_emin, emin);   // (block_sum synchronizes the block before s_emin is read)
   act = block_sum<long long>(act, s_ll);
   vmax = block_max(vmax, s_d);
   const long long B = (long long)g.bits * g.N;
   const bool select = !raw && 8 * act > B;
 
-  // 2. the B-th largest key: largest pattern lo with count(lo) >= B; count(lo + 1) < B
+  // 2. the B-th largest key K (counted with multiplicity): the largest pattern lo with
+  // count(lo) >= B, so count(lo + 1) < B.  The keys of bin i are var_i * 4^-k: the mantissa of
+  // var_i with the exponents e_i - 2k.  When every key is a normal number (e_i >= 15), K is found by
+  // radix selection: K's exponent from the histogram of all keys' exponents (the histogram of the
+  // bins' exponents summed over the 8 shifts), then 11-bit digits of K's mantissa from the keys
+  // with that exponent (at most one per bin), until one key is left.  Otherwise (subnormal keys)
+  // by bisection over the 64-bit patterns, which order like the values.
   unsigned long long lo = 0, hi = 0;
   if (select) {
-    hi = (unsigned long long)__double_as_longlong(vmax) + 1ull;   // above every key: count = 0 < B
-    while (hi - lo > 1) {                                         // count(+0) = 8 * act > B
-      const unsigned long long mid = lo + (hi - lo) / 2;
-      const double v = __longlong_as_double((long long)mid);
-      long long c = 0;
-      for (int i = threadIdx.x; i < g.N; i += blockDim.x) {
-        const double x = var[i];
-        if (x > 0.0) c += key_count(x, v);
+    if (s_emin >= 15) {
+      for (int j = threadIdx.x; j < kExpBuckets; j += blockDim.x) s_hist[j] = 0;
+      __syncthreads();
+      const unsigned lt = (1u << (threadIdx.x & 31)) - 1u;
+      for (int i0 = 0; i0 < g.N; i0 += blockDim.x) {   // warp-uniform rounds: bins with one exponent
+        const int i = i0 + (int)threadIdx.x;           // are counted by one atomic per warp
+        const double x = i < g.N ? var[i] : 0.0;
+        const int e = x > 0.0 ? (int)(__double_as_longlong(x) >> 52) : -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        if (e >= 0 && (peers & lt) == 0u) atomicAdd(&s_hist[e], (uint32_t)__popc(peers));
       }
-      c = block_sum<long long>(c, s_ll);
-      if (c >= B) lo = mid;
-      else hi = mid;
+      __syncthreads();
+      for (int j = threadIdx.x; j < kExpBuckets; j += blockDim.x) {
+        uint32_t c = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) c += j + 2 * k < kExpBuckets ? s_hist[j + 2 * k] : 0u;
+        s_rev[j] = c;   // keys with exponent j
+      }
+      __syncthreads();
+      uint32_t above = 0, here = 0;
+      const int E = select_bucket(s_rev, kExpBuckets, (uint32_t)B, s_hist, s_scan, &s_pick, &s_above, &s_count,
+                                  &above, &here);
+      uint32_t need = (uint32_t)B - above;      // K is the need-th largest key with exponent E
+      unsigned long long prefix = 0;            // K's leading mantissa bits selected so far
+      int done = 0;                             // how many of the 52 mantissa bits
+      while (done < 52) {
+        const int width = min(11, 52 - done), shift = 52 - done - width;
+        __syncthreads();
+        for (int j = threadIdx.x; j < (1 << width); j += blockDim.x) s_hist[j] = 0;
+        __syncthreads();
+        for (int i = threadIdx.x; i < g.N; i += blockDim.x) {
+          const unsigned long long bits = (unsigned long long)__double_as_longlong(var[i]);
+          const int d = (int)(bits >> 52) - E;   // (var[i] > 0: its sign bit is 0)
+          const unsigned long long m = bits & 0xFFFFFFFFFFFFFull;
+          if (var[i] > 0.0 && d >= 0 && d <= 14 && !(d & 1) && (m >> (shift + width)) == prefix)
+            atomicAdd(&s_hist[(m >> shift) & ((1u << width) - 1u)], 1u);
+        }
+        __syncthreads();
+        uint32_t above_d = 0;
+        const int digit = select_bucket(s_hist, 1 << width, need, s_rev, s_scan, &s_pick, &s_above, &s_count,
+                                        &above_d, &here);
+        need -= above_d;
+        prefix = (prefix << width) | (unsigned long long)digit;
+        done += width;
+        if (here == 1u && done < 52) {   // a single key has these leading bits: it is K
+          for (int i = threadIdx.x; i < g.N; i += blockDim.x) {
+            const unsigned long long bits = (unsigned long long)__double_as_longlong(var[i]);
+            const int d = (int)(bits >> 52) - E;
+            const unsigned long long m = bits & 0xFFFFFFFFFFFFFull;
+            if (var[i] > 0.0 && d >= 0 && d <= 14 && !(d & 1) && (m >> shift) == prefix) s_mant = m;
+          }
+          __syncthreads();
+          prefix = s_mant;
+          done = 52;
+        }
+      }
+      lo = ((unsigned long long)E << 52) | prefix;
+      hi = lo + 1ull;
+    } else {
+      hi = (unsigned long long)__double_as_longlong(vmax) + 1ull;   // above every key: count = 0 < B
+      while (hi - lo > 1) {                                         // count(+0) = 8 * act > B
+        const unsigned long long mid = lo + (hi - lo) / 2;
+        const double v = __longlong_as_double((long long)mid);
+        long long c = 0;
+        for (int i = threadIdx.x; i < g.N; i += blockDim.x) {
+          const double x = var[i];
+          if (x > 0.0) c += key_count(x, v);
+        }
+        c = block_sum<long long>(c, s_ll);
+        if (c >= B) lo = mid;
+        else hi = mid;
+      }
     }
   }
   const double v_lo = __longlong_as_double((long long)lo), v_hi = __longlong_as_double((long long)hi);
@@ -205,7 +306,9 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
       }
     }
     pay[kHeaderBytes + i] = (unsigned char)b;
-    reinterpret_cast<float*>(pay + g.off_sigma)[i] = (float)sqrt(x);
+    const float sg = (float)sqrt(x);
+    reinterpret_cast<float*>(pay + g.off_sigma)[i] = sg;
+    reinterpret_cast<uint2*>(var)[i] = make_uint2(__float_as_uint(sg), (uint32_t)b);   // for the records
     code_bits_local += b;
     slab_sum += b;
     slab_nz += b > 0;
@@ -248,12 +351,12 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
     block_exclusive_scan(s_cnt, blockDim.x, s_scan);
     uint32_t pos = s_cnt[threadIdx.x];
     uint4* urecs = recs + (size_t)u * g.N;
-    const float* sig = reinterpret_cast<const float*>(pay + g.off_sigma);
     for (int i = beg; i < end; ++i) {
-      const uint32_t b = pay[kHeaderBytes + i];
+      const uint2 sb = reinterpret_cast<const uint2*>(var)[i];   // {sigma_i, b_i} of this thread's bins
+      const uint32_t b = sb.y;
       if (b) {
         if (slot % kPackRecs == 0) s_bpos[slot / kPackRecs] = pos;   // a packing range starts here
-        urecs[slot++] = make_uint4((uint32_t)i, b, pos, __float_as_uint(__frcp_rn(sig[i])));
+        urecs[slot++] = make_uint4((uint32_t)i, b, pos, __float_as_uint(__frcp_rn(__uint_as_float(sb.x))));
         pos += b;
       }
     }

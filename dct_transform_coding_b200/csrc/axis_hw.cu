@@ -171,6 +171,9 @@ __device__ __forceinline__ void put_energy(const D& g, float2* t2, int kp, int l
 // Register budget: class-16 pencils fit two CTAs of 256 threads per SM; class-32 float2 pencils
 // need more than 128 registers.
 constexpr int kHwMinBlocks = (TACTKV_HCLASS == 16 && TACTKV_WCLASS == 16) ? 2 : 1;
+// The exact-size class-16 inverse kernels fit 80 registers without spilling: three CTAs per SM.
+template <int HX>
+constexpr int hw_min_blocks_inv() { return (TACTKV_HCLASS == 16 && TACTKV_WCLASS == 16) ? (HX > 0 ? 3 : 2) : 1; }
 
 // ---------------------------------------------------------------------------------- forward ---
 // Pass 1 of compression: the 3D DCT is completed (H and W after the S pass) and written back over
@@ -186,7 +189,7 @@ __global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) fdct_hw_kernel(co
   const HwLayout L = hw_layout(D.H, D.W, kLayStats);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const int HP = row_pairs(D.H), WP = row_pairs(D.W);
-  const int chunk = blockIdx.x, u = blockIdx.z;
+  const int chunk = blockIdx.x, u = g.unit0 + blockIdx.z;
   const int ks0 = blockIdx.y * spc, ks1 = min(g.S, ks0 + spc);
   float* yunit = Y + (size_t)u * g.S * D.HW * g.n + chunk * kChunk;
   auto tile_of = [&](int ks) {
@@ -258,7 +261,7 @@ __device__ __forceinline__ int cp_index(int Wp, int h, int wp) { return (h * Wp 
 // decodes rows 2kp and 2kp+1 in registers and runs the inverse DCT along W, writing column pairs;
 // then the inverse DCT along H runs on column pairs, into the fp32 volume V.
 template <int HC, int WC, int HX, int WX, int MODE>
-__global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) idct_hw_kernel(const __grid_constant__ Geom g,
+__global__ void __launch_bounds__(kMaxHwThreads, hw_min_blocks_inv<HX>()) idct_hw_kernel(const __grid_constant__ Geom g,
                                                                               const __grid_constant__ UnitList ul,
                                                                               float* __restrict__ V,
                                                                               const uint32_t* __restrict__ index,
@@ -269,7 +272,7 @@ __global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) idct_hw_kernel(co
   const HwLayout L = hw_layout(D.H, D.W, kLayDecode);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const int HP = row_pairs(D.H), WP = row_pairs(D.W), Wp = 2 * WP;
-  const int chunk = blockIdx.x, u = blockIdx.z;
+  const int chunk = blockIdx.x, u = g.unit0 + blockIdx.z;
   const int ks0 = blockIdx.y * spc, ks1 = min(g.S, ks0 + spc);
   const unsigned char* pay = ul.u[u].payload;
   const uint32_t* P = index + (size_t)u * unit_index_words(g.S);

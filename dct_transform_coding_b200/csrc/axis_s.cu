@@ -55,7 +55,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) fdct_s_kernel(const __gr
   const int lane = threadIdx.x & 31, hwl = threadIdx.x >> 5;
   const int hw0 = blockIdx.y * kCells, hw = hw0 + hwl;
   const int c0 = blockIdx.x * 32;
-  const int u = blockIdx.z;
+  const int u = g.unit0 + blockIdx.z;
   const UnitDev& ud = ul.u[u];
   const bool fp32 = g.flags & TACTKV_FP32_IO;
   stage_input<L>(g, ud, hw0, c0, fp32 ? 4 : 2, lg_cpr, tile);
@@ -88,7 +88,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) idct_s_kernel(const __gr
   const int lane = threadIdx.x & 31, hwl = threadIdx.x >> 5;
   const int hw0 = blockIdx.y * kCells, hw = hw0 + hwl;
   const int c0 = blockIdx.x * 32;
-  const int u = blockIdx.z;
+  const int u = g.unit0 + blockIdx.z;
   const UnitDev& ud = ul.u[u];
   {  // 128-byte rows of 32 channels, 8 copies of 16 bytes each; 4 values of s per pass
     const int q = threadIdx.x & 7, cl = (threadIdx.x >> 3) & 3, s0 = threadIdx.x >> 5;
@@ -102,6 +102,14 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) idct_s_kernel(const __gr
   }
   cp_async_wait_all();
   __syncthreads();
+  {  // V is dead once staged: drop its lines from L2 without writing them back to memory
+    const int q = threadIdx.x & 7, cl = (threadIdx.x >> 3) & 3, s0 = threadIdx.x >> 5;
+    if (q == 0 && hw0 + cl < g.HW && s0 < L) {
+      const float* src = V + (((size_t)u * L + s0) * g.HW + hw0 + cl) * g.n + c0;
+      const size_t sstep = (size_t)4 * g.HW * g.n;
+      for (int s = s0; s < L; s += 4, src += sstep) discard_l2_line(src);
+    }
+  }
   if (hw >= g.HW) return;
   float v[L];
   const float* t = vtile + hwl * 32 + lane;
@@ -133,7 +141,7 @@ cudaError_t launch_len(bool inverse, const Geom& g, const UnitList& ul, int nu, 
     // 16-byte copies need every unit's pointer, strides and head_dim on 16-byte boundaries
     const int esz = fp32 ? 4 : 2, per = 16 / esz;
     bool vec16 = g.head_dim % per == 0;
-    for (int i = 0; i < nu && vec16; ++i)
+    for (int i = g.unit0; i < g.unit0 + nu && vec16; ++i)
       vec16 = reinterpret_cast<uintptr_t>(ul.u[i].in) % 16 == 0 && ul.u[i].tok_stride % per == 0 &&
               ul.u[i].head_stride % per == 0;
     // copies per 32-channel row: 64 or 128 bytes in pieces of 16 or 4 bytes

@@ -44,6 +44,7 @@ struct Geom {
   int S, H, W, HW, T, heads, head_dim, n, nch, N, bits, flags;
   int off_sigma, off_codes;     // payload byte offsets
   long long capacity;           // payload bytes available (minimum over the launch)
+  int unit0;                    // the transform kernels: unit of blockIdx.z == 0 within the wave
 };
 
 __host__ __device__ inline long long pad16(long long x) { return (x + 15) / 16 * 16; }
@@ -184,6 +185,11 @@ __device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+// Invalidate the 128-byte L2 line at p (global memory, 128-byte aligned) without writing it back,
+// for scratch data that nothing reads again; its contents become undefined.
+__device__ __forceinline__ void discard_l2_line(const void* p) {
+  asm volatile("discard.global.L2 [%0], 128;\n" ::"l"(__cvta_generic_to_global(p)) : "memory");
+}
 
 // In place exclusive scan of a[0..n) in shared memory; blockDim.x a multiple of 32; returns the total.
 __device__ inline uint32_t block_exclusive_scan(uint32_t* a, int n, uint32_t* s_warp /* 33 entries */) {

@@ -8,12 +8,12 @@
 // uniform across the warp and only the 32 coefficient values differ.  Bins without bits are never
 // read.
 //
-// The CTA loads its records with cp.async and clears the word rows of its bit span in shared
-// memory.  Each warp takes blocks of 16 records; while it quantizes one block, the 16 coefficient
-// rows (128 bytes each) of its next block are in flight.  For a record it computes
-// u = X * (1/sigma) and the code, and ORs the code into the channel's word row at its stream
-// position (records are independent of each other).  The span's words are
-// then stored once; its first and last words may hold bits of the neighbouring ranges and are
+// The CTA clears the word rows of its bit span in shared memory and puts its records there grouped
+// by bit width (records are independent of each other: each carries its stream position), each
+// group padded to whole blocks of 16.  Each warp takes blocks of 16 records of one width; while it
+// quantizes one block, the 16 coefficient rows (128 bytes each) of its next block are in flight.
+// For a record it computes u = X * (1/sigma) and the code, and ORs the code into the channel's
+// word row at its stream position.  The span's words are then stored once; its first and last words may hold bits of the neighbouring ranges and are
 // ORed into the payload atomically (the allocation zeroes those words first).  The CTA with the
 // last record also writes the zero padding of the channel streams.
 //
@@ -30,38 +30,18 @@ constexpr int kPackBlock = 16;  // records per warp step
 // Thresholds of width b padded with two +inf, stored for b = 1, 2, ... in turn.
 __device__ __forceinline__ int thr_pad_offset(int b) { return (1 << b) + b - 3; }
 
-// Code of u at b bits: the number of thresholds t_j <= u (float32 compares, ties go up).  b = 1:
-// the sign test; b = 2: three compares against {-t, 0, t}; b >= 3: the cell of u in a uniform grid
-// gives the count c of thresholds below the cell, and two compares finish it (a cell holds at most
-// two thresholds; the thresholds are padded with +inf).
-__device__ __forceinline__ uint32_t quant_code(float u, int b, const float* thr, const unsigned char* qcell) {
-  if (b == 1) return u >= 0.f;
-  if (b == 2) return (uint32_t)(u >= -TACTKV_LM_T2) + (uint32_t)(u >= 0.f) + (uint32_t)(u >= TACTKV_LM_T2);
-  int j = __float2int_rd(fmaf(u, TACTKV_Q_SCALE, TACTKV_Q_OFFSET));
-  j = min(max(j, 0), TACTKV_Q_CELLS - 1);
-  const uint32_t c = qcell[(b - 3) * TACTKV_Q_CELLS + j];
-  const float* t = thr + thr_pad_offset(b) + c;
-  return c + (uint32_t)(u >= t[0]) + (uint32_t)(u >= t[1]);
-}
-
-// OR a b-bit code into a channel's word row at bit position off (b >= 1); codes of other records
-// in the same word come from other warps, so words are combined atomically.
-__device__ __forceinline__ void emit_code(uint32_t* row, uint32_t off, uint32_t b, uint32_t code) {
-  const uint32_t w = off >> 5, sh = off & 31u;
-  atomicOr(row + w, code << sh);
-  if (sh + b > 32) atomicOr(row + w + 1, code >> (32 - sh));   // sh >= 25 here
-}
-
 struct PackLayout {
   size_t rec, sbuf, thr, qcell, total;
   int words;
 };
+// A range's records grouped by bit width, each group padded to whole blocks of kPackBlock.
+constexpr int kPackRecSlots = kPackRecs + 8 * kPackBlock;
 __host__ __device__ inline PackLayout pack_layout() {
   PackLayout L;
   auto p16 = [](size_t x) { return (x + 15) / 16 * 16; };
   L.words = ((8 * kPackRecs + 31) / 32 + 3) | 1;   // odd: 32 channels' rows in 32 different banks
   size_t o = 0;
-  L.rec = o; o += p16((size_t)(kPackRecs + kPackBlock) * 16);   // + padding records
+  L.rec = o; o += p16((size_t)kPackRecSlots * 16);
   L.sbuf = o; o += p16((size_t)kChunk * L.words * 4);
   L.thr = o; o += p16((size_t)TACTKV_THR_PAD_TOTAL * 4);
   L.qcell = o; o += p16((size_t)6 * TACTKV_Q_CELLS);
@@ -69,13 +49,57 @@ __host__ __device__ inline PackLayout pack_layout() {
   return L;
 }
 
+// Code of u at B bits (B fixed at compile time): the number of thresholds t_j <= u (float32
+// compares, ties go up).  B = 1: the sign test, which needs no gain (1/sigma is positive and
+// finite, so u >= 0 exactly when x >= 0); B = 2: three compares against {-t, 0, t}; B >= 3: the
+// cell of u in a uniform grid gives the count c of thresholds below the cell, and two compares
+// finish it (a cell holds at most two thresholds; the thresholds are padded with +inf).
+template <int B>
+__device__ __forceinline__ uint32_t quant_code_b(float x, float inv_sigma, const float* thr, const unsigned char* qcell) {
+  if constexpr (B == 1) {
+    return x >= 0.f;
+  } else {
+    const float u = x * inv_sigma;
+    if constexpr (B == 2) {
+      return (uint32_t)(u >= -TACTKV_LM_T2) + (uint32_t)(u >= 0.f) + (uint32_t)(u >= TACTKV_LM_T2);
+    } else {
+      int j = __float2int_rd(fmaf(u, TACTKV_Q_SCALE, TACTKV_Q_OFFSET));
+      j = min(max(j, 0), TACTKV_Q_CELLS - 1);
+      const uint32_t c = qcell[(B - 3) * TACTKV_Q_CELLS + j];
+      const float* t = thr + thr_pad_offset(B) + c;
+      return c + (uint32_t)(u >= t[0]) + (uint32_t)(u >= t[1]);
+    }
+  }
+}
+
+// One block of kPackBlock records, all of width B: quantize x[] and OR the codes into the row
+// (a code of B > 1 bits may straddle into the next word).
+template <int B>
+__device__ __forceinline__ void pack_block(const uint4* rs, const float (&x)[kPackBlock], uint32_t* row, uint32_t base,
+                                           const float* thr, const unsigned char* qcell) {
+#pragma unroll
+  for (int j = 0; j < kPackBlock; ++j) {
+    const uint4 r = rs[j];
+    const uint32_t code = quant_code_b<B>(x[j], __uint_as_float(r.w), thr, qcell);
+    const uint32_t off = r.z - base, w = off >> 5, sh = off & 31u;
+    atomicOr(row + w, code << sh);
+    if constexpr (B > 1) {
+      if (sh > 32u - B) atomicOr(row + w + 1, code >> (32u - sh));
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kPackThreads) pack_kernel(const __grid_constant__ Geom g,
                                                             const __grid_constant__ UnitList ul,
                                                             const float* __restrict__ X, const uint4* __restrict__ recs,
                                                             const uint32_t* __restrict__ index) {
   extern __shared__ __align__(16) unsigned char smem[];
+  constexpr int kWarps = kPackThreads / 32;
+  __shared__ uint32_t s_cnt[9][kWarps];   // per bit width and warp: record counts, then first slots
+  __shared__ uint32_t s_fill[9];          // end of each width's records
+  __shared__ uint32_t s_grp[10];          // first slot of each width's group; s_grp[9]: all slots
   const PackLayout L = pack_layout();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int chunk = blockIdx.x, u = blockIdx.z;
   const uint32_t* P = index + (size_t)u * unit_index_words(g.S);
   const uint32_t nrec = P[2 * g.S + 2], code_bits = P[g.S];      // NZ(S) and P(S)
@@ -93,31 +117,73 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const __grid_constan
   const uint32_t cstride = reinterpret_cast<const uint32_t*>(pay)[11], sw = cstride / 4;
   uint32_t* words_out = reinterpret_cast<uint32_t*>(pay + g.off_codes) + (size_t)chunk * kChunk * sw;
 
-  for (int e = threadIdx.x; e < m; e += blockDim.x) cp_async16(rs + e, urecs + r0 + e);
-  cp_async_commit();
-  // the list is padded to whole blocks with records that set one bit of word 257 of a row, which
-  // is past every range's span (at most 8 * kPackRecs + 31 bits = 257 words) and never stored
-  const int m_pad = (m + kPackBlock - 1) / kPackBlock * kPackBlock;
-  {
-    const uint32_t A0 = m > 0 ? urecs[r0].z : 0u;
-    for (int e = m + threadIdx.x; e < m_pad; e += blockDim.x) rs[e] = make_uint4(0u, 1u, (A0 & ~31u) + 32u * 257u, 0u);
+  // Thread t holds records t, t + 256, ... of the range (empty slots past m have width 0).
+  constexpr int kPer = kPackRecs / kPackThreads;
+  uint4 mine[kPer];
+#pragma unroll
+  for (int q = 0; q < kPer; ++q) {
+    const int e = q * kPackThreads + (int)threadIdx.x;
+    mine[q] = e < m ? urecs[r0 + e] : make_uint4(0u, 0u, 0u, 0u);
   }
-  for (int i = threadIdx.x; i < TACTKV_THR_PAD_TOTAL; i += blockDim.x) thr[i] = c_thr_pad[i];
-  for (int i = threadIdx.x; i < 6 * TACTKV_Q_CELLS; i += blockDim.x) qcell[i] = c_qcell[i];
+  if (threadIdx.x < 9 * kWarps) (&s_cnt[0][0])[threadIdx.x] = 0u;
+  for (int i = threadIdx.x; i < TACTKV_THR_PAD_TOTAL; i += kPackThreads) thr[i] = c_thr_pad[i];
+  for (int i = threadIdx.x; i < 6 * TACTKV_Q_CELLS; i += kPackThreads) qcell[i] = c_qcell[i];
   // bit span [A, B) of the range; its words from word A >> 5 on are assembled in shared memory
   const uint32_t A = m > 0 ? urecs[r0].z : code_bits;
   const uint32_t B = r1 < nrec ? urecs[r1].z : code_bits;
   const uint32_t base = A & ~31u;
   const int nw = (int)((B - base + 31) >> 5);
-  for (int c = warp; c < kChunk; c += nwarps)
+  for (int c = warp; c < kChunk; c += kWarps)
     for (int w = lane; w <= nw; w += 32) sbuf[c * L.words + w] = 0u;
-  cp_async_wait_all();
+  __syncthreads();
+
+  // The records are grouped by bit width (each carries its own stream position, so their order
+  // does not matter), and every block of kPackBlock records then has a single width.
+  const uint32_t lt = (1u << lane) - 1u;
+  uint32_t rank[kPer];
+#pragma unroll
+  for (int q = 0; q < kPer; ++q) {
+    const uint32_t b = mine[q].y;
+    const uint32_t peers = __match_any_sync(0xffffffffu, b);
+    rank[q] = s_cnt[b][warp] + __popc(peers & lt);
+    __syncwarp();
+    if ((peers & lt) == 0u) s_cnt[b][warp] += __popc(peers);   // the lowest lane of each width
+    __syncwarp();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t run = 0;
+    for (int b = 1; b <= 8; ++b) {
+      s_grp[b] = run;
+      for (int w = 0; w < kWarps; ++w) {
+        const uint32_t c = s_cnt[b][w];
+        s_cnt[b][w] = run;
+        run += c;
+      }
+      s_fill[b] = run;
+      run = (run + kPackBlock - 1) / kPackBlock * kPackBlock;
+    }
+    s_grp[9] = run;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int q = 0; q < kPer; ++q)
+    if (mine[q].y) rs[s_cnt[mine[q].y][warp] + rank[q]] = mine[q];
+  // padding records fill each group to whole blocks: width b, coefficient row 0, gain 0, code bits
+  // into word 257 of the row, which is past every range's span (at most 8 * kPackRecs + 31 bits =
+  // 257 words) and never stored
+  if (threadIdx.x < 8 * kPackBlock) {
+    const int b = 1 + (int)threadIdx.x / kPackBlock;
+    const uint32_t e = s_fill[b] + threadIdx.x % kPackBlock;
+    if (e < s_grp[b + 1]) rs[e] = make_uint4(0u, (uint32_t)b, base + 32u * 257u, 0u);
+  }
   __syncthreads();
 
   uint32_t* row = sbuf + lane * L.words;
   // blocks of kPackBlock records per warp; the next block's coefficients are loaded while this
   // one is quantized
-  const int stride = nwarps * kPackBlock;
+  const int m_pad = (int)s_grp[9];
+  constexpr int stride = kWarps * kPackBlock;
   int e0 = warp * kPackBlock;
   float x[kPackBlock];
   if (e0 < m_pad) {
@@ -131,11 +197,16 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const __grid_constan
 #pragma unroll
       for (int j = 0; j < kPackBlock; ++j) xn[j] = __ldcs(xu + (size_t)rs[e1 + j].x * g.n);
     }
-#pragma unroll
-    for (int j = 0; j < kPackBlock; ++j) {
-      const uint4 r = rs[e0 + j];
-      const int b = (int)r.y;
-      emit_code(row, r.z - base, (uint32_t)b, quant_code(x[j] * __uint_as_float(r.w), b, thr, qcell));
+    const uint4* blk = rs + e0;
+    switch (blk[0].y) {
+      case 1: pack_block<1>(blk, x, row, base, thr, qcell); break;
+      case 2: pack_block<2>(blk, x, row, base, thr, qcell); break;
+      case 3: pack_block<3>(blk, x, row, base, thr, qcell); break;
+      case 4: pack_block<4>(blk, x, row, base, thr, qcell); break;
+      case 5: pack_block<5>(blk, x, row, base, thr, qcell); break;
+      case 6: pack_block<6>(blk, x, row, base, thr, qcell); break;
+      case 7: pack_block<7>(blk, x, row, base, thr, qcell); break;
+      default: pack_block<8>(blk, x, row, base, thr, qcell); break;
     }
 #pragma unroll
     for (int j = 0; j < kPackBlock; ++j) x[j] = xn[j];
@@ -144,7 +215,7 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const __grid_constan
   // the span's words; the first and the last may be shared with the neighbouring ranges
   const uint32_t wbase = base >> 5, wlast = (B - 1) >> 5;
   const bool first_shared = (A & 31u) != 0, last_shared = (B & 31u) != 0;
-  for (int c = warp; c < kChunk; c += nwarps) {
+  for (int c = warp; c < kChunk; c += kWarps) {
     uint32_t* out = words_out + (size_t)c * sw;
     for (int w = lane; w < nw; w += 32) {
       const uint32_t gw = wbase + w, v = sbuf[c * L.words + w];
@@ -154,7 +225,7 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const __grid_constan
   }
   if (r1 == nrec) {   // zero padding of the streams after the last code bit
     const uint32_t first = (code_bits + 31) >> 5;
-    for (int c = warp; c < kChunk; c += nwarps)
+    for (int c = warp; c < kChunk; c += kWarps)
       for (uint32_t w = first + lane; w < sw; w += 32) words_out[(size_t)c * sw + w] = 0u;
   }
 }

@@ -79,6 +79,7 @@ tactkv_status make_geom(const tactkv_unit& u, Geom& g) {
   g.off_sigma = (int)(kHeaderBytes + pad16(g.N));
   g.off_codes = (int)(g.off_sigma + pad16(4LL * g.N));
   g.capacity = 0;
+  g.unit0 = 0;
   return TACTKV_OK;
 }
 
@@ -275,21 +276,20 @@ static tactkv_status compress_impl(const tactkv_unit* units, int n_units, void* 
                        [&](const Geom& g, const UnitList& ul, int nu, unsigned char* ws) -> tactkv_status {
                          const WsView w = view(ws, g, nu);
                          const int cs = length_class(g.S), ch = length_class(g.H), cw = length_class(g.W);
-                         t_launches += 5;   // fdct_s, fdct_hw, reduce_var, allocate, pack
-                         const int mode2 = (g.flags & TACTKV_NO_QUANT) ? kRaw : kQuant;
+                         t_launches += 2;   // fdct_s, fdct_hw
                          mark(0);
                          if (launch_axis_s(cs, false, g, ul, nu, w.big, st) != cudaSuccess) return TACTKV_CUDA;
-                         mark(1);
                          if (launch_axis_hw(ch, cw, false, kStats, g, ul, nu, w.big, w.partial, w.index, nullptr,
                                             slabs_per_cta(g, nu, false, kStats), st) != cudaSuccess)
                            return TACTKV_CUDA;
-                         mark(2);
+                         mark(1);
+                         t_launches += 3;   // reduce_var, allocate, pack
                          if (launch_allocate(g, ul, nu, w.partial, w.var, w.index, w.recs, st) != cudaSuccess)
                            return TACTKV_CUDA;
-                         mark(3);
+                         mark(2);
                          if (launch_pack(g, ul, nu, w.big, w.recs, w.index, st) != cudaSuccess)
                            return TACTKV_CUDA;
-                         mark(4);
+                         mark(3);
                          return TACTKV_OK;
                        });
 }
@@ -304,15 +304,15 @@ static tactkv_status decompress_impl(const tactkv_unit* units, int n_units, void
                        [&](const Geom& g, const UnitList& ul, int nu, unsigned char* ws) -> tactkv_status {
                          const WsView w = view(ws, g, nu);
                          const int cs = length_class(g.S), ch = length_class(g.H), cw = length_class(g.W);
-                         t_launches += 3;   // decode_index, idct_hw, idct_s
                          const int mode = (g.flags & TACTKV_NO_QUANT) ? kRaw : kQuant;
                          mark(0);
+                         t_launches += 3;   // decode_index, idct_hw, idct_s
                          if (launch_decode_index(g, ul, nu, w.index, w.recs, w.status, st) != cudaSuccess)
                            return TACTKV_CUDA;
+                         mark(1);
                          if (launch_axis_hw(ch, cw, true, mode, g, ul, nu, w.big, nullptr, w.index, w.recs,
                                             slabs_per_cta(g, nu, true, mode), st) != cudaSuccess)
                            return TACTKV_CUDA;
-                         mark(1);
                          if (launch_axis_s(cs, true, g, ul, nu, w.big, st) != cudaSuccess) return TACTKV_CUDA;
                          mark(2);
                          return TACTKV_OK;

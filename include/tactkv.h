@@ -98,7 +98,7 @@ size_t tactkv_workspace_bytes(const tactkv_unit* units, int n_units);
 /* Compress every unit: read kv_in, write the payload.  Units with identical shape, bits and
    flags that are adjacent in the array are batched into one set of launches.  Steps: forward
    DCT along S; forward DCT along H and W with per-bin energy sums; per-unit bit allocation and
-   gains; the forward DCT again with quantization and bit packing. */
+   gains; quantization of the finished coefficients and bit packing. */
 tactkv_status tactkv_compress(const tactkv_unit* units, int n_units, void* workspace,
                               size_t workspace_bytes, struct CUstream_st* stream);
 
@@ -111,11 +111,12 @@ tactkv_status tactkv_decompress(const tactkv_unit* units, int n_units, void* wor
 
 /* Profiling variants: the same work as tactkv_compress / tactkv_decompress, and, when `events`
    is not NULL, cudaEventRecord(events[k], stream) at the stage boundaries of every wave (so for
-   a call that fits in one wave the events bracket each kernel).  events[k] are cudaEvent_t
+   a call that fits in one wave the events bracket each stage).  events[k] are cudaEvent_t
    handles created by the caller; a NULL entry is skipped.
-   compress:   0 before the S-axis DCT, 1 after it, 2 after the H/W DCT with energy sums,
-               3 after the allocation, 4 after the H/W DCT with quantization and packing.
-   decompress: 0 before the inverse H/W pass, 1 after it, 2 after the inverse S-axis pass. */
+   compress:   0 before the transforms, 1 after the DCTs along S and along H and W (with the
+               energy sums) of every unit, 2 after the allocation, 3 after quantization and
+               packing.
+   decompress: 0 before the payload index, 1 after it, 2 after the inverse DCTs of every unit. */
 tactkv_status tactkv_compress_profiled(const tactkv_unit* units, int n_units, void* workspace,
                                        size_t workspace_bytes, struct CUstream_st* stream,
                                        void* const* events);
