@@ -29,6 +29,10 @@ UNITS = [
     ("axis_hw_16_32", "axis_hw.cu", ["-DTACTKV_HCLASS=16", "-DTACTKV_WCLASS=32"]),
     ("axis_hw_32_16", "axis_hw.cu", ["-DTACTKV_HCLASS=32", "-DTACTKV_WCLASS=16"]),
     ("axis_hw_32_32", "axis_hw.cu", ["-DTACTKV_HCLASS=32", "-DTACTKV_WCLASS=32"]),
+    ("fused_8", "fused.cu", ["-DTACTKV_FUSED_S=8"]),
+    ("fused_16", "fused.cu", ["-DTACTKV_FUSED_S=16"]),
+    ("fused_32", "fused.cu", ["-DTACTKV_FUSED_S=32"]),
+    ("fused_64", "fused.cu", ["-DTACTKV_FUSED_S=64"]),
     ("allocate", "allocate.cu", []),
     ("pack", "pack.cu", []),
     ("tactkv", "tactkv.cu", []),

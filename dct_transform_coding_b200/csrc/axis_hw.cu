@@ -1,27 +1,9 @@
-// DCT along the H and W axes (TACT-KV stage 2, after the S pass) with the per-bin energies of
-// stage 3, and the inverse with unpacking and dequantization (the decoding paragraph).
-//
-// A CTA owns one (unit, 32-channel chunk, range of S slabs) and walks its slabs in order.  Lane l
-// of every warp is channel l of the chunk, and a thread's float2 holds two pencils of that
-// channel: two columns (w, w+1) in the pass along H, two rows (h, h+1) in the pass along W.  All
-// lanes of a warp therefore work on the same frequency bins at the same time, and everything that
-// depends on a bin (its bit width, its gain, where its code sits in the stream) is uniform across
-// the warp.
-//
-// Forward (fdct_hw), per slab k_s: the slab's H*W x 32 coefficients of the S-transformed volume
-// arrive by cp.async (the next slab's meanwhile); the DCT along H runs in place (a warp reads a
-// column pair and writes it back into the same bytes as row pairs); the DCT along W runs on row
-// pairs, writes the finished coefficients X back over the slab in global memory and sums X^2 over
-// the 32 channels into partial[u][chunk][bin].
-//
-// Inverse (idct_hw), per slab: the slab's stream words arrive by cp.async (next slab prefetched);
-// per-bin records give each bin's bits, gain and stream position; warp j decodes rows 2j and 2j+1
-// (unpack + dequantize in registers), runs the inverse DCT along W and writes column pairs; then
-// runs the inverse DCT along H on column pair j and stores the result into the fp32 volume V.
+// Kernels for the DCT along the H and W axes with the per-bin energies, and for its inverse with
+// unpacking and dequantization; each CTA walks one range of S slabs of one (unit, 32-channel
+// chunk) with the pieces of axis_hw.cuh.
 //
 // Compiled once per pair of length classes (TACTKV_HCLASS, TACTKV_WCLASS: 16 or 32 each).
-#include "common.cuh"
-#include "lloyd_max_tables.inc"
+#include "axis_hw.cuh"
 
 #if !defined(TACTKV_HCLASS) || !defined(TACTKV_WCLASS)
 #error "TACTKV_HCLASS and TACTKV_WCLASS must be defined"
@@ -30,144 +12,6 @@
 namespace tactkv {
 namespace {
 
-constexpr size_t kSmemBudget = 220 * 1024;
-
-enum LayoutKind { kLayStats = 0, kLayDecode = 2 };
-
-struct HwLayout {
-  size_t tile, tile_bytes, sbuf, meta, bsl, bsl_stride, sig, lv, total;
-  int nbuf, words;
-  int nslot;   // decode: slabs of stream words and records held at once (2: the next one prefetched)
-};
-
-__host__ __device__ inline int row_pairs(int L) { return (L + 1) >> 1; }
-
-// One warp per column pair (pass along H) and per row pair (pass along W), at most 8 warps; with
-// more pairs than warps, a warp takes several in turn.
-constexpr int kMaxHwThreads = 256;
-__host__ __device__ inline int hw_threads(int H, int W) {
-  const int HP = row_pairs(H), WP = row_pairs(W), m = 32 * (HP > WP ? HP : WP);
-  return m < kMaxHwThreads ? m : kMaxHwThreads;
-}
-
-// Shared memory of one launch.  A tile buffer holds a slab as cells of 32 floats on a grid of
-// 2*ceil(H/2) rows of Wp = 2*ceil(W/2) cells (the padding row and column are never read), which
-// also holds its row-pair (forward) or column-pair (inverse) rearrangement.  stats: the slab tiles
-// (two when they fit, so the next slab loads while this one is transformed; the energies reuse
-// the rearranged tile).  decode: one tile, the stream words and the records of two slabs, levels.  words (the stride of a channel's word row) is odd, so the 32
-// lanes reading 32 channels' rows hit 32 different banks.
-__host__ __device__ inline HwLayout hw_layout(int H, int W, int kind) {
-  HwLayout L;
-  const int HP = row_pairs(H), WP = row_pairs(W), HW = H * W;
-  const bool de = kind == kLayDecode;
-  L.tile_bytes = (size_t)(2 * HP) * (2 * WP) * 32 * 4;
-  L.words = ((8 * HW + 31) / 32 + 3) | 1;
-  const size_t words1 = (size_t)32 * L.words * 4, meta1 = (size_t)HW * 16;
-  L.nslot = (de && (size_t)(2 * HP) * (2 * WP) * 128 + 2 * (words1 + meta1) + kLmLvTotal * 4 + 256 > kSmemBudget) ? 1 : 2;
-  const size_t words = de ? words1 * L.nslot : 0;
-  const size_t meta = de ? meta1 * L.nslot : 0;       // records
-  L.bsl_stride = 0;
-  const size_t bsl = 0;
-  const size_t sig = 0;
-  const size_t lv = de ? kLmLvTotal * 4 : 0;
-  const size_t rest = words + meta + bsl + sig + lv + 256;
-  L.nbuf = (de || 2 * L.tile_bytes + rest > kSmemBudget) ? 1 : 2;
-  // every region starts on a 16-byte boundary (cp.async of 16 bytes, 16-byte record loads)
-  auto p16 = [](size_t x) { return (x + 15) / 16 * 16; };
-  size_t o = 0;
-  L.tile = o; o += p16(L.tile_bytes * L.nbuf);
-  L.sbuf = o; o += p16(words);
-  L.meta = o; o += p16(meta);
-  L.sig = o; o += p16(sig);
-  L.lv = o; o += p16(lv);
-  L.bsl = o; o += p16(bsl);
-  L.total = o;
-  return L;
-}
-
-
-// Grid sizes of a launch.  HX, WX > 0 are exact lengths fixed at compile time (the common grids
-// get their own kernels: straight-line transforms, no bounds tests); 0 takes them from the Geom.
-template <int HX, int WX>
-struct Dims {
-  static constexpr int hx = HX, wx = WX;
-  int H, W, HW, n;
-  __device__ __forceinline__ explicit Dims(const Geom& g)
-      : H(HX ? HX : g.H), W(WX ? WX : g.W), HW((HX ? HX : g.H) * (WX ? WX : g.W)), n(g.n) {}
-};
-
-// Pencil transform of length L (= EXACT when EXACT > 0) from length class CLASS.
-template <int CLASS, int EXACT, bool INV, class V>
-__device__ __forceinline__ void pencil(V* x, int L) {
-  if constexpr (EXACT > 0) dct_exact<EXACT, INV>(x);
-  else dct_pencil<CLASS, INV>(x, L);
-}
-
-// Copy one S slab of Y (H*W cells of 32 channels, 128 bytes each) into a tile with rows of Wp
-// cells, asynchronously.
-template <class D>
-__device__ __forceinline__ void issue_tile(const D& g, const float* slab_src, float* tile) {
-  const int Wp = 2 * row_pairs(g.W);
-  for (int r = threadIdx.x >> 3; r < g.H; r += blockDim.x >> 3)      // blockDim.x is a multiple of 32
-    for (int w = 0; w < g.W; ++w)
-      cp_async16(tile + (r * Wp + w) * 32 + (threadIdx.x & 7) * 4,
-                 slab_src + (size_t)(r * g.W + w) * g.n + (threadIdx.x & 7) * 4);
-}
-
-
-// Forward rearrangement.  The tile's cells (h, w) sit at cell index h*Wp + w.  After the pass
-// along H, element (row pair kp, column w, channel c) = {X[2kp][w], X[2kp+1][w]} (float2) sits at
-// float2 index ((2kp + (w & 1))*Wp + (w & ~1))*16 + c: the 256 bytes of cells (2kp + d, w0) and
-// (2kp + d, w0 + 1) hold row pair kp of column w0 + d.  Those are bytes that column pair w0 itself
-// read, so a warp rewrites its own column pair in place with no other warp involved.
-__device__ __forceinline__ int rp_index(int Wp, int kp, int w) { return ((2 * kp + (w & 1)) * Wp + (w & ~1)) * 16; }
-
-// Column pair (w0, w0+1): read, DCT along H, written back in place as row pairs.
-template <int HC, class D>
-__device__ __forceinline__ void h_pass_fwd(const D& g, float* tile, int w0, int lane) {
-  const int Wp = 2 * row_pairs(g.W), HP = row_pairs(g.H);
-  float2 xh[HC];
-#pragma unroll
-  for (int h = 0; h < HC; ++h)
-    if (h < g.H) {
-      const float* cell = tile + (h * Wp + w0) * kChunk + lane;
-      xh[h] = make_float2(cell[0], cell[kChunk]);   // column W (odd W) is padding: read, never used
-    }
-  __syncwarp();   // the whole column pair is read before any lane rewrites it
-  pencil<HC, D::hx, false>(xh, g.H);
-  float2* t2 = reinterpret_cast<float2*>(tile);
-#pragma unroll
-  for (int kp = 0; kp < (HC + 1) / 2; ++kp)
-    if (kp < HP) {
-      const float2 a = xh[2 * kp];
-      const float2 b = (2 * kp + 1 < g.H) ? xh[2 * kp + 1] : make_float2(0.f, 0.f);
-      t2[rp_index(Wp, kp, w0) + lane] = make_float2(a.x, b.x);
-      t2[rp_index(Wp, kp, w0 + 1) + lane] = make_float2(a.y, b.y);
-    }
-}
-// Row pair kp -> DCT along W.
-template <int WC, class D>
-__device__ __forceinline__ void w_load_fdct(const D& g, const float2* t2, int kp, int lane, float2 (&x)[WC]) {
-  const int Wp = 2 * row_pairs(g.W);
-#pragma unroll
-  for (int t = 0; t < WC; ++t)
-    if (t < g.W) x[t] = t2[rp_index(Wp, kp, t) + lane];
-  pencil<WC, D::wx, false>(x, g.W);
-}
-// Energies of row pair kp, written over its own (already read) elements: channel c of record
-// (kp, t) at rp_index(kp, t) + (c ^ (p & 15)) with p = kp*W + t, conflict-free for the 32 channels
-// writing a record and for the 16 records that a half warp reads at once.
-template <int WC, class D>
-__device__ __forceinline__ void put_energy(const D& g, float2* t2, int kp, int lane, const float2 (&x)[WC]) {
-  const int Wp = 2 * row_pairs(g.W);
-#pragma unroll
-  for (int t = 0; t < WC; ++t)
-    if (t < g.W) {
-      const int p = kp * g.W + t;
-      t2[rp_index(Wp, kp, t) + (lane ^ (p & 15))] = __fmul2_rn(x[t], x[t]);
-    }
-}
-
 // Register budget: class-16 pencils fit two CTAs of 256 threads per SM; class-32 float2 pencils
 // need more than 128 registers.
 constexpr int kHwMinBlocks = (TACTKV_HCLASS == 16 && TACTKV_WCLASS == 16) ? 2 : 1;
@@ -175,218 +19,27 @@ constexpr int kHwMinBlocks = (TACTKV_HCLASS == 16 && TACTKV_WCLASS == 16) ? 2 : 
 template <int HX>
 constexpr int hw_min_blocks_inv() { return (TACTKV_HCLASS == 16 && TACTKV_WCLASS == 16) ? (HX > 0 ? 3 : 2) : 1; }
 
-// ---------------------------------------------------------------------------------- forward ---
-// Pass 1 of compression: the 3D DCT is completed (H and W after the S pass) and written back over
-// the S-transformed slab, and the per-bin energies are summed over the CTA's 32 channels.  The
-// packing kernel then quantizes the finished coefficients without transforming anything.
 template <int HC, int WC, int HX, int WX>
 __global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) fdct_hw_kernel(const __grid_constant__ Geom g,
                                                                               const __grid_constant__ UnitList ul,
                                                                               float* __restrict__ Y,
                                                                               float* __restrict__ partial, int spc) {
   extern __shared__ __align__(16) unsigned char smem[];
-  const Dims<HX, WX> D(g);
-  const HwLayout L = hw_layout(D.H, D.W, kLayStats);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  const int HP = row_pairs(D.H), WP = row_pairs(D.W);
-  const int chunk = blockIdx.x, u = g.unit0 + blockIdx.z;
-  const int ks0 = blockIdx.y * spc, ks1 = min(g.S, ks0 + spc);
-  float* yunit = Y + (size_t)u * g.S * D.HW * g.n + chunk * kChunk;
-  auto tile_of = [&](int ks) {
-    return reinterpret_cast<float*>(smem + L.tile + (L.nbuf == 2 ? (ks & 1) : 0) * L.tile_bytes);
-  };
-
-  issue_tile(D, yunit + (size_t)ks0 * D.HW * g.n, tile_of(ks0));
-  cp_async_commit();
-  for (int ks = ks0; ks < ks1; ++ks) {
-    float* tile = tile_of(ks);
-    float* yslab = yunit + (size_t)ks * D.HW * g.n + lane;
-    cp_async_wait_all();
-    __syncthreads();  // slab ks is in place; every thread is done with slab ks - 1
-    if (L.nbuf == 2 && ks + 1 < ks1) {
-      issue_tile(D, yunit + (size_t)(ks + 1) * D.HW * g.n, tile_of(ks + 1));
-      cp_async_commit();
-    }
-    // DCT along H, in place, one column pair at a time per warp
-    for (int wp = warp; wp < WP; wp += nwarps) h_pass_fwd<HC>(D, tile, 2 * wp, lane);
-    __syncthreads();
-    float2* t2 = reinterpret_cast<float2*>(tile);
-    const int Wp = 2 * WP;
-    // DCT along W on row pair kp; the coefficients go back over the slab of Y (this CTA's own
-    // bytes), their squares over the row pair's own elements of the tile
-    for (int kp = warp; kp < HP; kp += nwarps) {
-      float2 x[WC];
-      w_load_fdct<WC>(D, t2, kp, lane, x);
-      const bool second = 2 * kp + 1 < D.H;
-      float* y0 = yslab + (size_t)(2 * kp * D.W) * g.n;
-#pragma unroll
-      for (int t = 0; t < WC; ++t)
-        if (t < D.W) {
-          y0[(size_t)t * g.n] = x[t].x;
-          if (second) y0[(size_t)(D.W + t) * g.n] = x[t].y;
-        }
-      __syncwarp();   // the row pair is read before its energies overwrite it
-      put_energy<WC>(D, t2, kp, lane, x);
-    }
-    __syncthreads();
-    float* dst = partial + ((size_t)u * g.nch + chunk) * g.N + (size_t)ks * D.HW;
-    for (int p = threadIdx.x; p < HP * D.W; p += blockDim.x) {
-      const int r = p / D.W, t = p - r * D.W;
-      const float2* e = t2 + rp_index(Wp, r, t);
-      const int sw15 = p & 15;
-      float2 acc = make_float2(0.f, 0.f);
-#pragma unroll 8
-      for (int c = 0; c < kChunk; ++c) acc = __fadd2_rn(acc, e[c ^ sw15]);
-      dst[2 * r * D.W + t] = acc.x;
-      if (2 * r + 1 < D.H) dst[(2 * r + 1) * D.W + t] = acc.y;
-    }
-    if (L.nbuf == 1 && ks + 1 < ks1) {
-      __syncthreads();  // everyone is done with the only tile
-      issue_tile(D, yunit + (size_t)(ks + 1) * D.HW * g.n, tile_of(ks + 1));
-      cp_async_commit();
-    }
-  }
-  cp_async_wait_all();
+  const int ks0 = blockIdx.y * spc;
+  fdct_hw_slabs<HC, WC, HX, WX, false>(g, Y, partial, g.unit0 + blockIdx.z, blockIdx.x, ks0, min(g.S, ks0 + spc), smem);
 }
 
-// ---------------------------------------------------------------------------------- inverse ---
-// Column-pair element (h, column pair wp, channel c) = {X[h][2wp], X[h][2wp+1]} at float2 index
-// (h*Wp + 2wp)*16 + c: rows 2kp and 2kp+1 of the cell grid hold row pair kp (forward
-// rearrangement) and its column pairs alike, so the inverse pass along W rewrites its row pair
-// in place.
-__device__ __forceinline__ int cp_index(int Wp, int h, int wp) { return (h * Wp + 2 * wp) * 16; }
-
-// Per slab: the stream words and the slab's dense records (per row pair and column: sigma and
-// stream position of the two rows' bins) arrive by cp.async, the next slab's meanwhile.  Warp kp
-// decodes rows 2kp and 2kp+1 in registers and runs the inverse DCT along W, writing column pairs;
-// then the inverse DCT along H runs on column pairs, into the fp32 volume V.
 template <int HC, int WC, int HX, int WX, int MODE>
 __global__ void __launch_bounds__(kMaxHwThreads, hw_min_blocks_inv<HX>()) idct_hw_kernel(const __grid_constant__ Geom g,
-                                                                              const __grid_constant__ UnitList ul,
-                                                                              float* __restrict__ V,
-                                                                              const uint32_t* __restrict__ index,
-                                                                              const uint4* __restrict__ recs, int spc) {
+                                                                                         const __grid_constant__ UnitList ul,
+                                                                                         float* __restrict__ V,
+                                                                                         const uint32_t* __restrict__ index,
+                                                                                         const uint4* __restrict__ recs,
+                                                                                         int spc) {
   extern __shared__ __align__(16) unsigned char smem[];
-  const Dims<HX, WX> D(g);
-  constexpr bool raw = MODE == kRaw;
-  const HwLayout L = hw_layout(D.H, D.W, kLayDecode);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  const int HP = row_pairs(D.H), WP = row_pairs(D.W), Wp = 2 * WP;
-  const int chunk = blockIdx.x, u = g.unit0 + blockIdx.z;
-  const int ks0 = blockIdx.y * spc, ks1 = min(g.S, ks0 + spc);
-  const unsigned char* pay = ul.u[u].payload;
-  const uint32_t* P = index + (size_t)u * unit_index_words(g.S);
-  const bool ok = P[g.S + 1] != 0;   // the index kernel checked the header and the bit widths
-  const uint32_t cstride = ok ? reinterpret_cast<const uint32_t*>(pay)[11] : 0u, sw = cstride / 4;
-  const uint32_t* streams = reinterpret_cast<const uint32_t*>(pay + g.off_codes) + (size_t)chunk * kChunk * sw;
-  const uint4* urecs = recs + (size_t)u * g.N;
-  float2* tile = reinterpret_cast<float2*>(smem + L.tile);
-  float* lvs = reinterpret_cast<float*>(smem + L.lv);
-  auto slot = [&](int ks) { return L.nslot == 2 ? (ks & 1) : 0; };
-  auto sbuf_of = [&](int ks) { return reinterpret_cast<uint32_t*>(smem + L.sbuf) + slot(ks) * kChunk * L.words; };
-  auto rbuf_of = [&](int ks) { return reinterpret_cast<uint4*>(smem + L.meta) + slot(ks) * D.HW; };
-
-  // stream words of slab ks for the 32 channels from word P(ks) >> 5 on, then two zero words for
-  // the look-ahead of the code reads; and the slab's records
-  auto issue_slab = [&](int ks) {
-    uint32_t* sb = sbuf_of(ks);
-    const uint32_t p0 = P[ks], p1 = P[ks + 1];
-    const uint32_t w0 = p0 >> 5;
-    const int nw = (int)(((p0 & 31u) + (p1 - p0) + 31) >> 5);
-    for (int c = warp; c < kChunk; c += nwarps)
-      for (int w = lane; w < nw + 2; w += 32) {
-        if (w < nw) cp_async4(sb + c * L.words + w, streams + (size_t)c * sw + w0 + w);
-        else sb[c * L.words + w] = 0u;
-      }
-    const int RP = row_pairs(D.H) * D.W;   // dense records of the slab
-    uint4* rb = rbuf_of(ks);
-    for (int e = threadIdx.x; e < RP; e += blockDim.x) cp_async16(rb + e, urecs + (size_t)ks * RP + e);
-  };
-  if (!raw) {
-    for (int i = threadIdx.x; i < kLmLvTotal; i += blockDim.x) lvs[i] = c_lm_levels[i];
-    if (ok) issue_slab(ks0);
-    cp_async_commit();
-  }
-  float* vunit = V + (size_t)u * g.S * D.HW * g.n + chunk * kChunk + lane;
-
-  for (int ks = ks0; ks < ks1; ++ks) {
-    cp_async_wait_all();
-    __syncthreads();  // slab ks's words and records are in place; slab ks - 1 is done
-    if (L.nslot == 2 && ok && !raw && ks + 1 < ks1) {
-      issue_slab(ks + 1);
-      cp_async_commit();
-    }
-    // decode rows 2kp, 2kp+1 of warp kp (dequantize in registers) and run the inverse DCT along W;
-    // column pairs go to the tile
-    const uint32_t base = ok && !raw ? (P[ks] & ~31u) : 0u;
-    const uint4* rs = rbuf_of(ks);
-    const uint32_t* row = sbuf_of(ks) + lane * L.words;   // this lane's channel stream
-    for (int kp = warp; kp < HP; kp += nwarps) {
-      float2 x[WC];
-      if (!ok) {
-#pragma unroll
-        for (int t = 0; t < WC; ++t) x[t] = make_float2(0.f, 0.f);
-      } else if (raw) {
-        const float* s = reinterpret_cast<const float*>(pay + g.off_codes + (size_t)(chunk * kChunk + lane) * cstride) +
-                         (size_t)ks * D.HW + 2 * kp * D.W;
-        const bool second = 2 * kp + 1 < D.H;
-#pragma unroll
-        for (int t = 0; t < WC; ++t)
-          if (t < D.W) x[t] = make_float2(s[t], second ? s[D.W + t] : 0.f);
-      } else {
-#pragma unroll
-        for (int t = 0; t < WC; ++t)
-          if (t < D.W) {
-            // record: sigma of each row, position << 8 | code mask of each row (mask 0: no bits)
-            const uint4 m = rs[kp * D.W + t];
-            float l0 = 0.f, l1 = 0.f;
-            const uint32_t k0 = m.z & 0xffu, k1 = m.w & 0xffu;
-            if (k0) {
-              const uint32_t off = (m.z >> 8) - base, w = off >> 5;
-              l0 = lvs[k0 - 1u + (__funnelshift_r(row[w], row[w + 1], off) & k0)];
-            }
-            if (k1) {
-              const uint32_t off = (m.w >> 8) - base, w = off >> 5;
-              l1 = lvs[k1 - 1u + (__funnelshift_r(row[w], row[w + 1], off) & k1)];
-            }
-            x[t] = __fmul2_rn(make_float2(l0, l1), make_float2(__uint_as_float(m.x), __uint_as_float(m.y)));
-          }
-      }
-      pencil<WC, WX, true>(x, D.W);
-      const bool second = 2 * kp + 1 < D.H;
-#pragma unroll
-      for (int wp = 0; wp < (WC + 1) / 2; ++wp)
-        if (wp < WP) {
-          const float2 a = x[2 * wp];
-          const float2 b = (2 * wp + 1 < D.W) ? x[2 * wp + 1] : make_float2(0.f, 0.f);
-          tile[cp_index(Wp, 2 * kp, wp) + lane] = make_float2(a.x, b.x);
-          if (second) tile[cp_index(Wp, 2 * kp + 1, wp) + lane] = make_float2(a.y, b.y);
-        }
-    }
-    __syncthreads();
-    // inverse DCT along H on column pair wp; store to V
-    for (int wp = warp; wp < WP; wp += nwarps) {
-      float2 xh[HC];
-#pragma unroll
-      for (int h = 0; h < HC; ++h)
-        if (h < D.H) xh[h] = tile[cp_index(Wp, h, wp) + lane];
-      pencil<HC, HX, true>(xh, D.H);
-      float* v = vunit + ((size_t)ks * D.HW + 2 * wp) * g.n;
-      const bool two = 2 * wp + 1 < D.W;
-#pragma unroll
-      for (int h = 0; h < HC; ++h)
-        if (h < D.H) {
-          float* cell = v + (size_t)h * D.W * g.n;
-          cell[0] = xh[h].x;
-          if (two) cell[g.n] = xh[h].y;
-        }
-    }
-    if (L.nslot == 1 && ok && !raw && ks + 1 < ks1) {   // the single slot is free once the records are used
-      issue_slab(ks + 1);
-      cp_async_commit();
-    }
-  }
-  cp_async_wait_all();
+  const int ks0 = blockIdx.y * spc;
+  idct_hw_slabs<HC, WC, HX, WX, MODE>(g, ul, V, index, recs, g.unit0 + blockIdx.z, blockIdx.x, ks0,
+                                      min(g.S, ks0 + spc), smem);
 }
 
 }  // namespace

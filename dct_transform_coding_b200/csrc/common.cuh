@@ -185,6 +185,30 @@ __device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+// Streams that pass through L2 once (the input, the finished coefficients, the output) are
+// marked evict-first, so that they give way to the fp32 volume that is read back soon after.
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void cp_async16_ef(void* smem, const void* gmem, uint64_t pol) {
+  const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;\n" ::"r"(sa), "l"(gmem), "l"(pol)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4_ef(void* smem, const void* gmem, uint64_t pol) {
+  const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.ca.shared.global.L2::cache_hint [%0], [%1], 4, %2;\n" ::"r"(sa), "l"(gmem), "l"(pol)
+               : "memory");
+}
+__device__ __forceinline__ void st_ef(float* p, float v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;\n" ::"l"(p), "f"(v), "l"(pol) : "memory");
+}
+__device__ __forceinline__ void st_ef(__nv_bfloat16* p, __nv_bfloat16 v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.b16 [%0], %1, %2;\n" ::"l"(p), "h"(__bfloat16_as_ushort(v)), "l"(pol)
+               : "memory");
+}
 // Invalidate the 128-byte L2 line at p (global memory, 128-byte aligned) without writing it back,
 // for scratch data that nothing reads again; its contents become undefined.
 __device__ __forceinline__ void discard_l2_line(const void* p) {

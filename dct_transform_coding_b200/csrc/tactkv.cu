@@ -37,6 +37,30 @@ cudaError_t launch_axis_s(int cls, bool inverse, const Geom& g, const UnitList& 
   return launch_axis_s_64(inverse, g, ul, nu, buf, st);
 }
 
+#define TACTKV_DECL_FUSED(s) \
+  cudaError_t launch_fused_##s(const Geom&, const UnitList&, int, float*, float*, cudaStream_t);
+TACTKV_DECL_FUSED(8)
+TACTKV_DECL_FUSED(16)
+TACTKV_DECL_FUSED(32)
+TACTKV_DECL_FUSED(64)
+#undef TACTKV_DECL_FUSED
+
+// Grids with a fused three-axis forward kernel (one launch for the S and H/W passes, the volume
+// kept in L2 between them).
+bool fused_grid(const Geom& g) {
+  const bool s = g.S == 8 || g.S == 16 || g.S == 32 || g.S == 64;
+  return s && ((g.H == 16 && g.W == 16) || (g.H == 14 && g.W == 14) || (g.H == 8 && g.W == 8));
+}
+cudaError_t launch_fused(const Geom& g, const UnitList& ul, int nu, float* buf, float* partial, cudaStream_t st) {
+  switch (g.S) {
+    case 8: return launch_fused_8(g, ul, nu, buf, partial, st);
+    case 16: return launch_fused_16(g, ul, nu, buf, partial, st);
+    case 32: return launch_fused_32(g, ul, nu, buf, partial, st);
+    case 64: return launch_fused_64(g, ul, nu, buf, partial, st);
+    default: return cudaErrorNotSupported;
+  }
+}
+
 cudaError_t launch_axis_hw(int hcls, int wcls, bool inverse, int mode, const Geom& g, const UnitList& ul, int nu,
                            float* buf, float* partial, const uint32_t* index, const uint4* recs, int spc,
                            cudaStream_t st) {
@@ -276,12 +300,17 @@ static tactkv_status compress_impl(const tactkv_unit* units, int n_units, void* 
                        [&](const Geom& g, const UnitList& ul, int nu, unsigned char* ws) -> tactkv_status {
                          const WsView w = view(ws, g, nu);
                          const int cs = length_class(g.S), ch = length_class(g.H), cw = length_class(g.W);
-                         t_launches += 2;   // fdct_s, fdct_hw
                          mark(0);
-                         if (launch_axis_s(cs, false, g, ul, nu, w.big, st) != cudaSuccess) return TACTKV_CUDA;
-                         if (launch_axis_hw(ch, cw, false, kStats, g, ul, nu, w.big, w.partial, w.index, nullptr,
-                                            slabs_per_cta(g, nu, false, kStats), st) != cudaSuccess)
-                           return TACTKV_CUDA;
+                         if (fused_grid(g)) {
+                           t_launches += 1;   // fdct3
+                           if (launch_fused(g, ul, nu, w.big, w.partial, st) != cudaSuccess) return TACTKV_CUDA;
+                         } else {
+                           t_launches += 2;   // fdct_s, fdct_hw
+                           if (launch_axis_s(cs, false, g, ul, nu, w.big, st) != cudaSuccess) return TACTKV_CUDA;
+                           if (launch_axis_hw(ch, cw, false, kStats, g, ul, nu, w.big, w.partial, w.index, nullptr,
+                                              slabs_per_cta(g, nu, false, kStats), st) != cudaSuccess)
+                             return TACTKV_CUDA;
+                         }
                          mark(1);
                          t_launches += 3;   // reduce_var, allocate, pack
                          if (launch_allocate(g, ul, nu, w.partial, w.var, w.index, w.recs, st) != cudaSuccess)
@@ -306,10 +335,11 @@ static tactkv_status decompress_impl(const tactkv_unit* units, int n_units, void
                          const int cs = length_class(g.S), ch = length_class(g.H), cw = length_class(g.W);
                          const int mode = (g.flags & TACTKV_NO_QUANT) ? kRaw : kQuant;
                          mark(0);
-                         t_launches += 3;   // decode_index, idct_hw, idct_s
+                         t_launches += 1;   // decode_index
                          if (launch_decode_index(g, ul, nu, w.index, w.recs, w.status, st) != cudaSuccess)
                            return TACTKV_CUDA;
                          mark(1);
+                         t_launches += 2;   // idct_hw, idct_s
                          if (launch_axis_hw(ch, cw, true, mode, g, ul, nu, w.big, nullptr, w.index, w.recs,
                                             slabs_per_cta(g, nu, true, mode), st) != cudaSuccess)
                            return TACTKV_CUDA;

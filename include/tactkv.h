@@ -158,8 +158,10 @@ int tactkv_lloyd_max_table(int bits, double* levels, double* thresholds);
 int tactkv_format_version(void);
 
 /* Number of kernels that the calling host thread's most recent tactkv_compress*,
-   tactkv_decompress* call launched (all its waves: 5 per compress wave, 3 per decompress wave;
-   0 after a call that failed before launching). */
+   tactkv_decompress* call launched, over all its waves (0 after a call that failed before
+   launching).  A compress wave launches 4 kernels when its grid has a fused three-axis forward
+   transform kernel (H x W = 16 x 16, 14 x 14 or 8 x 8 with S = 8, 16, 32 or 64) and 5 otherwise;
+   a decompress wave launches 3. */
 int tactkv_last_launches(void);
 
 #ifdef __cplusplus

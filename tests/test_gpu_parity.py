@@ -65,6 +65,9 @@ def test_tiny_config_fp32_io():
     ((24, 5, 9, 1, 32), 8),     # 8 bits: every active bin saturates
     ((32, 2, 24, 1, 64), 2),    # S in the 32 class, W in the 32 class
     ((1, 1, 1, 1, 32), 5),      # a single token
+    ((8, 14, 14, 1, 64), 3),    # fused three-axis kernels: S = 8 on the 14 x 14 grid
+    ((32, 8, 8, 2, 32), 2),     # fused, S = 32 on the 8 x 8 grid
+    ((64, 8, 8, 1, 32), 1),     # fused, S = 64 on the 8 x 8 grid
 ])
 def test_small_shapes_bf16(shape, bits):
     S, H, W, heads, D = shape
@@ -101,9 +104,10 @@ def test_no_quant_fp32_io():
     assert rel_rms(y.double().cpu(), x.double().cpu()) <= 1e-6
 
 
-def test_strided_input_and_output():
+@pytest.mark.parametrize("S,H,W", [(8, 6, 6), (8, 8, 8)])   # separate and fused transform kernels
+def test_strided_input_and_output(S, H, W):
     """kv_in as a view into a larger [tokens, heads_total, head_dim] cache (only 2 of 4 heads)."""
-    S, H, W, D = 8, 6, 6, 32
+    D = 32
     big = make_unit(S, H, W, 4, D, rho=(0.9, 0.9, 0.9), nu=4.0, seed=5, device=DEV)
     x = big[:, 1:3, :][None]                          # stride(2) = D, stride(1) = 4 * D
     assert not x.is_contiguous()
@@ -160,14 +164,15 @@ def test_many_units_and_small_workspace():
 
 
 def test_wave_splitting_and_launch_counts():
-    """12 units in one wave (5 compress kernels, 3 decompress kernels) give the same payloads and
-    outputs as 12 waves of one unit each (a one-unit workspace)."""
+    """12 units in one wave (4 compress kernels: the 8 x 8 x 8 grid has the fused three-axis forward
+    kernel; 3 decompress kernels) give the same payloads and outputs as 12 waves of one unit each
+    (a one-unit workspace)."""
     S, H, W, heads, D = 8, 8, 8, 2, 32
     U = 12
     x = torch.stack([make_unit(S, H, W, heads, D, rho=(0.9, 0.8, 0.85), nu=4.0, seed=40 + i, device=DEV)
                      for i in range(U)])
     pay = T.compress(x, S, H, W, 2)
-    assert T.tactkv_last_launches() == 5
+    assert T.tactkv_last_launches() == 4
     y = T.decompress(pay, S, H, W, 2, heads=heads, head_dim=D, check=False)
     assert T.tactkv_last_launches() == 3
     units = T.make_units(x, S, H, W, 2, heads=heads, head_dim=D, payload=pay)
