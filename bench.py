@@ -42,6 +42,7 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-groups", type=int, default=16, help="unit groups pipelined over streams in the e2e run")
     ap.add_argument("--units", type=int, default=None, help="use only the first U units of the batch (profiling)")
     return ap.parse_args()
 
@@ -362,22 +363,42 @@ def main():
 
 def e2e_run(args, T, x, payload, out, cu, du, ws, stream, world):
     """The same metric through the C ABI from pinned host memory: each step copies the K/V in,
-    compresses, copies the payloads out, decompresses and copies the reconstruction out."""
+    compresses, copies the payloads out, decompresses and copies the reconstruction out.  The
+    batch goes in groups of units over a few streams (each with its own workspace), so that the
+    host-link copies of one group overlap the kernels of the others."""
     import torch
     import torch.distributed as dist
     dev = x.device
+    U = x.shape[0]
     xh = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
     xh.copy_(x)
     ph = torch.empty(payload.shape, dtype=payload.dtype, pin_memory=True)
     oh = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    sp = int(stream.cuda_stream)
+    G = max(1, min(U, args.e2e_groups))
+    bounds = [(U * g // G, U * (g + 1) // G) for g in range(G)]
+    bounds = [(a, b) for a, b in bounds if b > a]
+    streams = [torch.cuda.Stream(dev) for _ in range(min(3, len(bounds)))]
+    largest = max(b - a for a, b in bounds)
+    wss = [T.alloc_workspace(cu[:largest], dev) for _ in streams]
 
     def one():
-        x.copy_(xh, non_blocking=True)
-        T.tactkv_compress(cu, ws.data_ptr(), ws.numel(), sp)
-        ph.copy_(payload, non_blocking=True)
-        T.tactkv_decompress(du, ws.data_ptr(), ws.numel(), sp)
-        oh.copy_(out, non_blocking=True)
+        start = torch.cuda.Event()
+        start.record(stream)
+        for s in streams:
+            s.wait_event(start)
+        for g, (a, b) in enumerate(bounds):
+            s, wsg = streams[g % len(streams)], wss[g % len(streams)]
+            sp = int(s.cuda_stream)
+            with torch.cuda.stream(s):
+                x[a:b].copy_(xh[a:b], non_blocking=True)
+                T.tactkv_compress(cu[a:b], wsg.data_ptr(), wsg.numel(), sp)
+                ph[a:b].copy_(payload[a:b], non_blocking=True)
+                T.tactkv_decompress(du[a:b], wsg.data_ptr(), wsg.numel(), sp)
+                oh[a:b].copy_(out[a:b], non_blocking=True)
+        for s in streams:
+            done = torch.cuda.Event()
+            done.record(s)
+            stream.wait_event(done)
 
     one()
     torch.cuda.synchronize(dev)
@@ -395,7 +416,7 @@ def e2e_run(args, T, x, payload, out, cu, du, ws, stream, world):
     in_bytes = x.numel() * x.element_size()
     return {"value": round(job_gbs(world, in_bytes, ms), 2), "unit": "GB/s",
             "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": payload.numel() + out.numel() * out.element_size(),
-            "ms_per_step": round(ms, 3)}
+            "ms_per_step": round(ms, 3), "groups": len(bounds), "streams": len(streams)}
 
 
 def cpu_baseline(w, bits, x):

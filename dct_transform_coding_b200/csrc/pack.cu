@@ -10,12 +10,13 @@
 //
 // The CTA clears the word rows of its bit span in shared memory and puts its records there grouped
 // by bit width (records are independent of each other: each carries its stream position), each
-// group padded to whole blocks of 16.  Each warp takes blocks of 16 records of one width; while it
-// quantizes one block, the 16 coefficient rows (128 bytes each) of its next block are in flight.
-// For a record it computes u = X * (1/sigma) and the code, and ORs the code into the channel's
-// word row at its stream position.  The span's words are then stored once; its first and last words may hold bits of the neighbouring ranges and are
-// ORed into the payload atomically (the allocation zeroes those words first).  The CTA with the
-// last record also writes the zero padding of the channel streams.
+// group padded to whole blocks of 16.  Each warp takes blocks of 16 records of one width (quantized
+// by code specialised for 1 bit, 2 bits, or 3 and more bits by table); while it quantizes one
+// block, the 16 coefficient rows (128 bytes each) of its next block are in flight.  For a record
+// it computes u = X * (1/sigma) and the code, and ORs the code into the channel's word row at its
+// stream position.  The span's words are then stored once; its first and last words may hold bits
+// of the neighbouring ranges and are ORed into the payload atomically (the allocation zeroes those
+// words first).  The CTA with the last record also writes the zero padding of the channel streams.
 //
 // NO_QUANT (raw) copies X into the channel streams as float32.
 #include "common.cuh"
@@ -49,13 +50,15 @@ __host__ __device__ inline PackLayout pack_layout() {
   return L;
 }
 
-// Code of u at B bits (B fixed at compile time): the number of thresholds t_j <= u (float32
-// compares, ties go up).  B = 1: the sign test, which needs no gain (1/sigma is positive and
-// finite, so u >= 0 exactly when x >= 0); B = 2: three compares against {-t, 0, t}; B >= 3: the
-// cell of u in a uniform grid gives the count c of thresholds below the cell, and two compares
-// finish it (a cell holds at most two thresholds; the thresholds are padded with +inf).
+// Code of u at b bits: the number of thresholds t_j <= u (float32 compares, ties go up).  B is
+// the width when fixed at compile time (1 or 2), 0 for a width b >= 3 known at run time.  b = 1:
+// the sign test, which needs no gain (1/sigma is positive and finite, so u >= 0 exactly when
+// x >= 0); b = 2: three compares against {-t, 0, t}; b >= 3: the cell of u in a uniform grid gives
+// the count c of thresholds below the cell, and two compares finish it (a cell holds at most two
+// thresholds; the thresholds are padded with +inf).
 template <int B>
-__device__ __forceinline__ uint32_t quant_code_b(float x, float inv_sigma, const float* thr, const unsigned char* qcell) {
+__device__ __forceinline__ uint32_t quant_code_b(float x, float inv_sigma, int b, const float* __restrict__ thr,
+                                                 const unsigned char* __restrict__ qcell) {
   if constexpr (B == 1) {
     return x >= 0.f;
   } else {
@@ -65,26 +68,28 @@ __device__ __forceinline__ uint32_t quant_code_b(float x, float inv_sigma, const
     } else {
       int j = __float2int_rd(fmaf(u, TACTKV_Q_SCALE, TACTKV_Q_OFFSET));
       j = min(max(j, 0), TACTKV_Q_CELLS - 1);
-      const uint32_t c = qcell[(B - 3) * TACTKV_Q_CELLS + j];
-      const float* t = thr + thr_pad_offset(B) + c;
+      const uint32_t c = qcell[(b - 3) * TACTKV_Q_CELLS + j];
+      const float* t = thr + thr_pad_offset(b) + c;
       return c + (uint32_t)(u >= t[0]) + (uint32_t)(u >= t[1]);
     }
   }
 }
 
-// One block of kPackBlock records, all of width B: quantize x[] and OR the codes into the row
-// (a code of B > 1 bits may straddle into the next word).
+// One block of kPackBlock records, all of width b (= B when B > 0): quantize x[] and OR the codes
+// into the row (a code of more than one bit may straddle into the next word).  The records, the
+// word row and the tables do not overlap, so the record loads need not wait for the atomics.
 template <int B>
-__device__ __forceinline__ void pack_block(const uint4* rs, const float (&x)[kPackBlock], uint32_t* row, uint32_t base,
-                                           const float* thr, const unsigned char* qcell) {
+__device__ __forceinline__ void pack_block(const uint4* __restrict__ rs, const float (&x)[kPackBlock],
+                                           uint32_t* __restrict__ row, uint32_t base, int b,
+                                           const float* __restrict__ thr, const unsigned char* __restrict__ qcell) {
 #pragma unroll
   for (int j = 0; j < kPackBlock; ++j) {
     const uint4 r = rs[j];
-    const uint32_t code = quant_code_b<B>(x[j], __uint_as_float(r.w), thr, qcell);
+    const uint32_t code = quant_code_b<B>(x[j], __uint_as_float(r.w), b, thr, qcell);
     const uint32_t off = r.z - base, w = off >> 5, sh = off & 31u;
     atomicOr(row + w, code << sh);
-    if constexpr (B > 1) {
-      if (sh > 32u - B) atomicOr(row + w + 1, code >> (32u - sh));
+    if constexpr (B != 1) {
+      if (sh + (uint32_t)b > 32u) atomicOr(row + w + 1, code >> (32u - sh));
     }
   }
 }
@@ -198,16 +203,10 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const __grid_constan
       for (int j = 0; j < kPackBlock; ++j) xn[j] = __ldcs(xu + (size_t)rs[e1 + j].x * g.n);
     }
     const uint4* blk = rs + e0;
-    switch (blk[0].y) {
-      case 1: pack_block<1>(blk, x, row, base, thr, qcell); break;
-      case 2: pack_block<2>(blk, x, row, base, thr, qcell); break;
-      case 3: pack_block<3>(blk, x, row, base, thr, qcell); break;
-      case 4: pack_block<4>(blk, x, row, base, thr, qcell); break;
-      case 5: pack_block<5>(blk, x, row, base, thr, qcell); break;
-      case 6: pack_block<6>(blk, x, row, base, thr, qcell); break;
-      case 7: pack_block<7>(blk, x, row, base, thr, qcell); break;
-      default: pack_block<8>(blk, x, row, base, thr, qcell); break;
-    }
+    const int b = (int)blk[0].y;
+    if (b == 1) pack_block<1>(blk, x, row, base, 1, thr, qcell);
+    else if (b == 2) pack_block<2>(blk, x, row, base, 2, thr, qcell);
+    else pack_block<0>(blk, x, row, base, b, thr, qcell);
 #pragma unroll
     for (int j = 0; j < kPackBlock; ++j) x[j] = xn[j];
   }
