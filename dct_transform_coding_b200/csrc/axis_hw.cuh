@@ -84,12 +84,13 @@ __host__ __device__ inline HwLayout hw_layout(int H, int W, int kind) {
 
 // Grid sizes of a launch.  HX, WX > 0 are exact lengths fixed at compile time (the common grids
 // get their own kernels: straight-line transforms, no bounds tests); 0 takes them from the Geom.
-template <int HX, int WX>
+// NX > 0 fixes the channel count n as well (constant strides: immediate address offsets).
+template <int HX, int WX, int NX = 0>
 struct Dims {
   static constexpr int hx = HX, wx = WX;
   int H, W, HW, n;
   __device__ __forceinline__ explicit Dims(const Geom& g)
-      : H(HX ? HX : g.H), W(WX ? WX : g.W), HW((HX ? HX : g.H) * (WX ? WX : g.W)), n(g.n) {}
+      : H(HX ? HX : g.H), W(WX ? WX : g.W), HW((HX ? HX : g.H) * (WX ? WX : g.W)), n(NX ? NX : g.n) {}
 };
 
 // Pencil transform of length L (= EXACT when EXACT > 0) from length class CLASS.
@@ -169,27 +170,27 @@ __device__ __forceinline__ void put_energy(const D& g, float2* t2, int kp, int l
 // packing kernel then quantizes the finished coefficients without transforming anything.
 // Slabs [ks0, ks1) of channel chunk `chunk` of unit u; called by every thread of the CTA.  EF: the
 // stores of X are marked evict-first in L2 (X is read again only by the packing kernel).
-template <int HC, int WC, int HX, int WX, bool EF>
+template <int HC, int WC, int HX, int WX, bool EF, int NX = 0>
 __device__ __forceinline__ void fdct_hw_slabs(const Geom& g, float* __restrict__ Y, float* __restrict__ partial, int u,
                                               int chunk, int ks0, int ks1, unsigned char* smem) {
-  const Dims<HX, WX> D(g);
+  const Dims<HX, WX, NX> D(g);
   const HwLayout L = hw_layout(D.H, D.W, kLayStats);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const int HP = row_pairs(D.H), WP = row_pairs(D.W);
-  float* yunit = Y + (size_t)u * g.S * D.HW * g.n + chunk * kChunk;
+  float* yunit = Y + (size_t)u * g.S * D.HW * D.n + chunk * kChunk;
   auto tile_of = [&](int ks) {
     return reinterpret_cast<float*>(smem + L.tile + (L.nbuf == 2 ? (ks & 1) : 0) * L.tile_bytes);
   };
 
-  issue_tile(D, yunit + (size_t)ks0 * D.HW * g.n, tile_of(ks0));
+  issue_tile(D, yunit + (size_t)ks0 * D.HW * D.n, tile_of(ks0));
   cp_async_commit();
   for (int ks = ks0; ks < ks1; ++ks) {
     float* tile = tile_of(ks);
-    float* yslab = yunit + (size_t)ks * D.HW * g.n + lane;
+    float* yslab = yunit + (size_t)ks * D.HW * D.n + lane;
     cp_async_wait_all();
     __syncthreads();  // slab ks is in place; every thread is done with slab ks - 1
     if (L.nbuf == 2 && ks + 1 < ks1) {
-      issue_tile(D, yunit + (size_t)(ks + 1) * D.HW * g.n, tile_of(ks + 1));
+      issue_tile(D, yunit + (size_t)(ks + 1) * D.HW * D.n, tile_of(ks + 1));
       cp_async_commit();
     }
     // DCT along H, in place, one column pair at a time per warp
@@ -203,28 +204,28 @@ __device__ __forceinline__ void fdct_hw_slabs(const Geom& g, float* __restrict__
       float2 x[WC];
       w_load_fdct<WC>(D, t2, kp, lane, x);
       const bool second = 2 * kp + 1 < D.H;
-      float* y0 = yslab + (size_t)(2 * kp * D.W) * g.n;
+      float* y0 = yslab + (size_t)(2 * kp * D.W) * D.n;
       if constexpr (EF) {
         const uint64_t pol = l2_evict_first();
 #pragma unroll
         for (int t = 0; t < WC; ++t)
           if (t < D.W) {
-            st_ef(y0 + (size_t)t * g.n, x[t].x, pol);
-            if (second) st_ef(y0 + (size_t)(D.W + t) * g.n, x[t].y, pol);
+            st_ef(y0 + (size_t)t * D.n, x[t].x, pol);
+            if (second) st_ef(y0 + (size_t)(D.W + t) * D.n, x[t].y, pol);
           }
       } else {
 #pragma unroll
         for (int t = 0; t < WC; ++t)
           if (t < D.W) {
-            y0[(size_t)t * g.n] = x[t].x;
-            if (second) y0[(size_t)(D.W + t) * g.n] = x[t].y;
+            y0[(size_t)t * D.n] = x[t].x;
+            if (second) y0[(size_t)(D.W + t) * D.n] = x[t].y;
           }
       }
       __syncwarp();   // the row pair is read before its energies overwrite it
       put_energy<WC>(D, t2, kp, lane, x);
     }
     __syncthreads();
-    float* dst = partial + ((size_t)u * g.nch + chunk) * g.N + (size_t)ks * D.HW;
+    float* dst = partial + ((size_t)u * (NX ? NX / kChunk : g.nch) + chunk) * g.N + (size_t)ks * D.HW;
     for (int p = threadIdx.x; p < HP * D.W; p += blockDim.x) {
       const int r = p / D.W, t = p - r * D.W;
       const float2* e = t2 + rp_index(Wp, r, t);
@@ -237,7 +238,7 @@ __device__ __forceinline__ void fdct_hw_slabs(const Geom& g, float* __restrict__
     }
     if (L.nbuf == 1 && ks + 1 < ks1) {
       __syncthreads();  // everyone is done with the only tile
-      issue_tile(D, yunit + (size_t)(ks + 1) * D.HW * g.n, tile_of(ks + 1));
+      issue_tile(D, yunit + (size_t)(ks + 1) * D.HW * D.n, tile_of(ks + 1));
       cp_async_commit();
     }
   }

@@ -56,11 +56,13 @@ __device__ __forceinline__ void stage_input(const Geom& g, const UnitDev& ud, in
 }
 
 // Forward pencils of a staged input tile: cell hw0 + warp -> Y[u][k_s][hw][c0 + lane], fp32.
-template <int L, int NC>
+// HWX, NX > 0 fix H*W and the channel count n at compile time (constant strides).
+template <int L, int NC, int HWX = 0, int NX = 0>
 __device__ __forceinline__ void fdct_s_cells(const Geom& g, int u, int hw0, int c0, const unsigned char* tile,
                                              bool fp32, float* __restrict__ Y) {
   const int lane = threadIdx.x & 31, hwl = threadIdx.x >> 5, hw = hw0 + hwl;
-  if (hw >= g.HW) return;
+  const int HW = HWX ? HWX : g.HW, n = NX ? NX : g.n;
+  if (hw >= HW) return;
   float v[L];
   if (fp32) {
     const float* t = reinterpret_cast<const float*>(tile) + hwl * 32 + lane;
@@ -72,8 +74,8 @@ __device__ __forceinline__ void fdct_s_cells(const Geom& g, int u, int hw0, int 
     for (int s = 0; s < L; ++s) v[s] = __bfloat162float(t[s * NC * 32]);
   }
   dct_exact<L, false>(v);
-  float* yo = Y + ((size_t)u * L * g.HW + hw) * g.n + c0 + lane;
-  const size_t kstep = (size_t)g.HW * g.n;
+  float* yo = Y + ((size_t)u * L * HW + hw) * n + c0 + lane;
+  const size_t kstep = (size_t)HW * n;
 #pragma unroll
   for (int k = 0; k < L; ++k) yo[k * kstep] = v[k];
 }

@@ -50,7 +50,8 @@ __host__ __device__ inline size_t fused_fwd_smem(int H, int W, bool fp32_in, int
   return hw > st ? hw : st;
 }
 
-template <int L, int HX, int WX>
+// NX: the channel count when fixed at compile time (the common 512 and 1024), else 0.
+template <int L, int HX, int WX, int NX>
 __global__ void __launch_bounds__(kFusedThreads, 3) fdct3_kernel(const __grid_constant__ Geom g,
                                                                  const __grid_constant__ UnitList ul,
                                                                  float* __restrict__ Y, float* __restrict__ partial,
@@ -76,7 +77,7 @@ __global__ void __launch_bounds__(kFusedThreads, 3) fdct3_kernel(const __grid_co
       cp_async_wait_all();
     }
     __syncthreads();
-    fdct_s_cells<L, kNC>(g, u, t * kNC, c0, smem + buf * tb, fp32, Y);
+    fdct_s_cells<L, kNC, HX * WX, NX>(g, u, t * kNC, c0, smem + buf * tb, fp32, Y);
     __syncthreads();   // the tile's buffer is free again
     if (nbuf == 2) buf ^= 1;
     else if (next) stage_input<L, kNC, true>(g, ud, (t + kCluster) * kNC, c0, esz, lg_cpr, smem);
@@ -85,7 +86,7 @@ __global__ void __launch_bounds__(kFusedThreads, 3) fdct3_kernel(const __grid_co
   // DCT along H and W on this CTA's range of slabs
   constexpr int spc = (L + kCluster - 1) / kCluster;
   const int ks0 = r * spc, ks1 = min(L, ks0 + spc);
-  if (ks0 < ks1) fdct_hw_slabs<16, 16, HX, WX, true>(g, Y, partial, u, chunk, ks0, ks1, smem);
+  if (ks0 < ks1) fdct_hw_slabs<16, 16, HX, WX, true, NX>(g, Y, partial, u, chunk, ks0, ks1, smem);
 }
 
 template <class K, class... Args>
@@ -117,8 +118,10 @@ cudaError_t launch_grid(const Geom& g, const UnitList& ul, int nu, float* buf, f
   int nbuf = 1;
   const size_t smem = fused_fwd_smem<L>(HX, WX, (g.flags & TACTKV_FP32_IO) != 0, &nbuf);
   if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
-  return launch_cluster(fdct3_kernel<L, HX, WX>, g, nu, smem, st, g, ul, buf, partial,
-                        input_pieces_lg(g, ul, g.unit0, nu));
+  const int lg_cpr = input_pieces_lg(g, ul, g.unit0, nu);
+  if (g.n == 1024) return launch_cluster(fdct3_kernel<L, HX, WX, 1024>, g, nu, smem, st, g, ul, buf, partial, lg_cpr);
+  if (g.n == 512) return launch_cluster(fdct3_kernel<L, HX, WX, 512>, g, nu, smem, st, g, ul, buf, partial, lg_cpr);
+  return launch_cluster(fdct3_kernel<L, HX, WX, 0>, g, nu, smem, st, g, ul, buf, partial, lg_cpr);
 }
 
 }  // namespace
