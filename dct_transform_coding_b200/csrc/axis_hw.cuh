@@ -151,18 +151,41 @@ __device__ __forceinline__ void w_load_fdct(const D& g, const float2* t2, int kp
     if (t < g.W) x[t] = t2[rp_index(Wp, kp, t) + lane];
   pencil<WC, D::wx, false>(x, g.W);
 }
-// Energies of row pair kp, written over its own (already read) elements: channel c of record
-// (kp, t) at rp_index(kp, t) + (c ^ (p & 15)) with p = kp*W + t, conflict-free for the 32 channels
-// writing a record and for the 16 records that a half warp reads at once.
-template <int WC, class D>
-__device__ __forceinline__ void put_energy(const D& g, float2* t2, int kp, int lane, const float2 (&x)[WC]) {
-  const int Wp = 2 * row_pairs(g.W);
+// Sums over the 32 lanes of the warp of 32 values per lane (recursive halving: at each step a
+// lane keeps half of its values and adds the partner lane's copy of that half); lane l returns the
+// total of value l.
+__device__ __forceinline__ float warp_transpose_sum(float (&v)[32], int lane) {
 #pragma unroll
-  for (int t = 0; t < WC; ++t)
-    if (t < g.W) {
-      const int p = kp * g.W + t;
-      t2[rp_index(Wp, kp, t) + (lane ^ (p & 15))] = __fmul2_rn(x[t], x[t]);
+  for (int h = 16; h >= 1; h >>= 1) {
+    const bool upper = lane & h;
+#pragma unroll
+    for (int i = 0; i < h; ++i) {
+      const float send = upper ? v[i] : v[i + h], keep = upper ? v[i + h] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, h);
     }
+  }
+  return v[0];
+}
+
+// Energies of row pair kp summed over the warp's 32 channels and stored to dst (the slab's bins):
+// the squares of rows 2kp and 2kp+1 go through the transpose sum 16 columns at a time, so that
+// lane l ends with column (l & 15) of row 2kp + (l >> 4) of that group of columns.
+template <int WC, class D>
+__device__ __forceinline__ void store_energy(const D& g, int kp, int lane, const float2 (&x)[WC], float* dst) {
+  const int row = 2 * kp + (lane >> 4);
+#pragma unroll
+  for (int t0 = 0; t0 < WC; t0 += 16) {
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float2 e = t0 + j < g.W ? __fmul2_rn(x[t0 + j], x[t0 + j]) : make_float2(0.f, 0.f);
+      v[j] = e.x;
+      v[16 + j] = e.y;
+    }
+    const float sum = warp_transpose_sum(v, lane);
+    const int t = t0 + (lane & 15);
+    if (t < g.W && row < g.H) dst[row * g.W + t] = sum;
+  }
 }
 
 // Pass 1 of compression: the 3D DCT is completed (H and W after the S pass) and written back over
@@ -197,9 +220,9 @@ __device__ __forceinline__ void fdct_hw_slabs(const Geom& g, float* __restrict__
     for (int wp = warp; wp < WP; wp += nwarps) h_pass_fwd<HC>(D, tile, 2 * wp, lane);
     __syncthreads();
     float2* t2 = reinterpret_cast<float2*>(tile);
-    const int Wp = 2 * WP;
     // DCT along W on row pair kp; the coefficients go back over the slab of Y (this CTA's own
-    // bytes), their squares over the row pair's own elements of the tile
+    // bytes), their squares summed over the 32 channels to the slab's bins of partial
+    float* dst = partial + ((size_t)u * (NX ? NX / kChunk : g.nch) + chunk) * g.N + (size_t)ks * D.HW;
     for (int kp = warp; kp < HP; kp += nwarps) {
       float2 x[WC];
       w_load_fdct<WC>(D, t2, kp, lane, x);
@@ -221,20 +244,7 @@ __device__ __forceinline__ void fdct_hw_slabs(const Geom& g, float* __restrict__
             if (second) y0[(size_t)(D.W + t) * D.n] = x[t].y;
           }
       }
-      __syncwarp();   // the row pair is read before its energies overwrite it
-      put_energy<WC>(D, t2, kp, lane, x);
-    }
-    __syncthreads();
-    float* dst = partial + ((size_t)u * (NX ? NX / kChunk : g.nch) + chunk) * g.N + (size_t)ks * D.HW;
-    for (int p = threadIdx.x; p < HP * D.W; p += blockDim.x) {
-      const int r = p / D.W, t = p - r * D.W;
-      const float2* e = t2 + rp_index(Wp, r, t);
-      const int sw15 = p & 15;
-      float2 acc = make_float2(0.f, 0.f);
-#pragma unroll 8
-      for (int c = 0; c < kChunk; ++c) acc = __fadd2_rn(acc, e[c ^ sw15]);
-      dst[2 * r * D.W + t] = acc.x;
-      if (2 * r + 1 < D.H) dst[(2 * r + 1) * D.W + t] = acc.y;
+      store_energy<WC>(D, kp, lane, x, dst);
     }
     if (L.nbuf == 1 && ks + 1 < ks1) {
       __syncthreads();  // everyone is done with the only tile
