@@ -482,7 +482,8 @@ __global__ void __launch_bounds__(256) decode_index_kernel(const __grid_constant
   if (ok && !raw) {
     // dense decoding records, one per (slab, row pair kp, column t) at ks*HP*W + kp*W + t:
     // {sigma of row 2kp, sigma of row 2kp+1, position << 8 | code mask of each row}; a bin without
-    // bits (and the padding row of an odd H) has sigma 0 and mask 0
+    // bits (and the padding row of an odd H) has sigma 0, mask 0 and a position inside its slab's
+    // span, so that the decoder may read its (empty) code like any other
     const float* sig = reinterpret_cast<const float*>(pay + g.off_sigma);
     const int HP = (g.H + 1) >> 1, RP = HP * g.W;
     uint32_t* urec32 = reinterpret_cast<uint32_t*>(recs + (size_t)u * g.N);
@@ -505,11 +506,11 @@ __global__ void __launch_bounds__(256) decode_index_kernel(const __grid_constant
         }
         pos += __shfl_sync(0xffffffffu, incl, 31);
       }
-      if (g.H & 1)   // the padding row H of the last row pair
+      if (g.H & 1)   // the padding row H of the last row pair: no bits, at the slab's first bit
         for (int t = lane; t < g.W; t += 32) {
           uint32_t* rec = urec32 + ((size_t)k * RP + (size_t)(HP - 1) * g.W + t) * 4;
           rec[1] = 0u;
-          rec[3] = 0u;
+          rec[3] = s_P[k] << 8;
         }
     }
   }

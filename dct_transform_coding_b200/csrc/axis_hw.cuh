@@ -65,7 +65,7 @@ __host__ __device__ inline HwLayout hw_layout(int H, int W, int kind) {
   L.bsl_stride = 0;
   const size_t bsl = 0;
   const size_t sig = 0;
-  const size_t lv = de ? kLmLvTotal * 4 : 0;
+  const size_t lv = de ? (kLmLvTotal + 1) * 4 : 0;   // a zero in front of the levels
   const size_t rest = words + meta + bsl + sig + lv + 256;
   L.nbuf = (de || 2 * L.tile_bytes + rest > kSmemBudget) ? 1 : 2;
   // every region starts on a 16-byte boundary (cp.async of 16 bytes, 16-byte record loads)
@@ -304,7 +304,7 @@ __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul,
     for (int e = threadIdx.x; e < RP; e += blockDim.x) cp_async16(rb + e, urecs + (size_t)ks * RP + e);
   };
   if (!raw) {
-    for (int i = threadIdx.x; i < kLmLvTotal; i += blockDim.x) lvs[i] = c_lm_levels[i];
+    for (int i = threadIdx.x; i <= kLmLvTotal; i += blockDim.x) lvs[i] = i ? c_lm_levels[i - 1] : 0.f;
     if (ok) issue_slab(ks0);
     cp_async_commit();
   }
@@ -335,21 +335,20 @@ __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul,
         for (int t = 0; t < WC; ++t)
           if (t < D.W) x[t] = make_float2(s[t], second ? s[D.W + t] : 0.f);
       } else {
+        // lvs1[-1] is the zero in front of the levels: a bin without bits (mask 0) reads it, so
+        // every code is read the same way, without a branch
+        const float* lvs1 = lvs + 1;
 #pragma unroll
         for (int t = 0; t < WC; ++t)
           if (t < D.W) {
             // record: sigma of each row, position << 8 | code mask of each row (mask 0: no bits)
             const uint4 m = rs[kp * D.W + t];
-            float l0 = 0.f, l1 = 0.f;
             const uint32_t k0 = m.z & 0xffu, k1 = m.w & 0xffu;
-            if (k0) {
-              const uint32_t off = (m.z >> 8) - base, w = off >> 5;
-              l0 = lvs[k0 - 1u + (__funnelshift_r(row[w], row[w + 1], off) & k0)];
-            }
-            if (k1) {
-              const uint32_t off = (m.w >> 8) - base, w = off >> 5;
-              l1 = lvs[k1 - 1u + (__funnelshift_r(row[w], row[w + 1], off) & k1)];
-            }
+            const uint32_t off0 = (m.z >> 8) - base, off1 = (m.w >> 8) - base;
+            const uint32_t* w0 = row + (off0 >> 5);
+            const uint32_t* w1 = row + (off1 >> 5);
+            const float l0 = lvs1[(int)(k0 + (__funnelshift_r(w0[0], w0[1], off0) & k0)) - 1];
+            const float l1 = lvs1[(int)(k1 + (__funnelshift_r(w1[0], w1[1], off1) & k1)) - 1];
             x[t] = __fmul2_rn(make_float2(l0, l1), make_float2(__uint_as_float(m.x), __uint_as_float(m.y)));
           }
       }
