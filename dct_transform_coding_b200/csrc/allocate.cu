@@ -481,14 +481,16 @@ __global__ void __launch_bounds__(256) decode_index_kernel(const __grid_constant
   }
   if (ok && !raw) {
     // dense decoding records, one per (slab, row pair kp, column t) at ks*HP*W + kp*W + t:
-    // {sigma of row 2kp, sigma of row 2kp+1, position << 8 | code mask of each row}; a bin without
-    // bits (and the padding row of an odd H) has sigma 0, mask 0 and a position inside its slab's
-    // span, so that the decoder may read its (empty) code like any other
+    // {sigma of row 2kp, sigma of row 2kp+1, offset << 8 | code mask of each row}, the offset of a
+    // code counted from the first bit of its slab's first stream word (P(k_s) rounded down to 32);
+    // a bin without bits (and the padding row of an odd H) has sigma 0, mask 0 and an offset
+    // inside its slab's span, so that the decoder may read its (empty) code like any other
     const float* sig = reinterpret_cast<const float*>(pay + g.off_sigma);
     const int HP = (g.H + 1) >> 1, RP = HP * g.W;
     uint32_t* urec32 = reinterpret_cast<uint32_t*>(recs + (size_t)u * g.N);
     for (int k = warp; k < g.S; k += nwarps) {
       uint32_t pos = s_P[k];
+      const uint32_t wbase = pos & ~31u;   // first bit of the slab's first stream word
       for (int i0 = 0; i0 < g.HW; i0 += 32) {
         const int j = i0 + lane, i = k * g.HW + j;
         const uint32_t v = j < g.HW ? b[i] : 0u;
@@ -502,7 +504,7 @@ __global__ void __launch_bounds__(256) decode_index_kernel(const __grid_constant
           const int kh = j / g.W, t = j - kh * g.W;
           uint32_t* rec = urec32 + ((size_t)k * RP + (size_t)(kh >> 1) * g.W + t) * 4;
           rec[kh & 1] = v ? __float_as_uint(sig[i]) : 0u;
-          rec[2 + (kh & 1)] = ((pos + incl - v) << 8) | ((1u << v) - 1u);
+          rec[2 + (kh & 1)] = ((pos + incl - v - wbase) << 8) | ((1u << v) - 1u);
         }
         pos += __shfl_sync(0xffffffffu, incl, 31);
       }
@@ -510,7 +512,7 @@ __global__ void __launch_bounds__(256) decode_index_kernel(const __grid_constant
         for (int t = lane; t < g.W; t += 32) {
           uint32_t* rec = urec32 + ((size_t)k * RP + (size_t)(HP - 1) * g.W + t) * 4;
           rec[1] = 0u;
-          rec[3] = s_P[k] << 8;
+          rec[3] = (s_P[k] - wbase) << 8;
         }
     }
   }

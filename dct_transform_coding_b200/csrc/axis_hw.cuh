@@ -263,9 +263,9 @@ __device__ __forceinline__ void fdct_hw_slabs(const Geom& g, float* __restrict__
 __device__ __forceinline__ int cp_index(int Wp, int h, int wp) { return (h * Wp + 2 * wp) * 16; }
 
 // Per slab: the stream words and the slab's dense records (per row pair and column: sigma and
-// stream position of the two rows' bins) arrive by cp.async, the next slab's meanwhile.  Warp kp
-// decodes rows 2kp and 2kp+1 in registers and runs the inverse DCT along W, writing column pairs;
-// then the inverse DCT along H runs on column pairs, into the fp32 volume V.
+// code offset within the slab's words of the two rows' bins) arrive by cp.async, the next slab's
+// meanwhile.  Warp kp decodes rows 2kp and 2kp+1 in registers and runs the inverse DCT along W,
+// writing column pairs; then the inverse DCT along H runs on column pairs, into the fp32 volume V.
 template <int HC, int WC, int HX, int WX, int MODE>
 __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul, float* __restrict__ V,
                                               const uint32_t* __restrict__ index, const uint4* __restrict__ recs, int u,
@@ -319,7 +319,6 @@ __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul,
     }
     // decode rows 2kp, 2kp+1 of warp kp (dequantize in registers) and run the inverse DCT along W;
     // column pairs go to the tile
-    const uint32_t base = ok && !raw ? (P[ks] & ~31u) : 0u;
     const uint4* rs = rbuf_of(ks);
     const uint32_t* row = sbuf_of(ks) + lane * L.words;   // this lane's channel stream
     for (int kp = warp; kp < HP; kp += nwarps) {
@@ -341,10 +340,10 @@ __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul,
 #pragma unroll
         for (int t = 0; t < WC; ++t)
           if (t < D.W) {
-            // record: sigma of each row, position << 8 | code mask of each row (mask 0: no bits)
+            // record: sigma of each row, offset << 8 | code mask of each row (mask 0: no bits)
             const uint4 m = rs[kp * D.W + t];
             const uint32_t k0 = m.z & 0xffu, k1 = m.w & 0xffu;
-            const uint32_t off0 = (m.z >> 8) - base, off1 = (m.w >> 8) - base;
+            const uint32_t off0 = m.z >> 8, off1 = m.w >> 8;   // from the slab's first word
             const uint32_t* w0 = row + (off0 >> 5);
             const uint32_t* w1 = row + (off1 >> 5);
             const float l0 = lvs1[(int)(k0 + (__funnelshift_r(w0[0], w0[1], off0) & k0)) - 1];

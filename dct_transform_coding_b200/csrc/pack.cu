@@ -84,9 +84,9 @@ __device__ __forceinline__ void pack_block(const uint4* __restrict__ rs, const f
                                            const float* __restrict__ thr, const unsigned char* __restrict__ qcell) {
 #pragma unroll
   for (int j = 0; j < kPackBlock; ++j) {
-    const uint4 r = rs[j];
-    const uint32_t code = quant_code_b<B>(x[j], __uint_as_float(r.w), b, thr, qcell);
-    const uint32_t off = r.z - base, w = off >> 5, sh = off & 31u;
+    const uint2 r = reinterpret_cast<const uint2*>(rs + j)[1];   // {stream position, 1/sigma}
+    const uint32_t code = quant_code_b<B>(x[j], __uint_as_float(r.y), b, thr, qcell);
+    const uint32_t off = r.x - base, w = off >> 5, sh = off & 31u;
     atomicOr(row + w, code << sh);
     if constexpr (B != 1) {
       if (sh + (uint32_t)b > 32u) atomicOr(row + w + 1, code >> (32u - sh));
