@@ -157,23 +157,6 @@ __device__ __forceinline__ void dct_exact(V* x) {
 
 __device__ __forceinline__ void set_status(unsigned int* status, unsigned int code) { atomicCAS(status, 0u, code); }
 
-__device__ __forceinline__ float load_one(const void* base, long long elem, bool fp32) {
-  if (fp32) return static_cast<const float*>(base)[elem];
-  return __bfloat162float(static_cast<const __nv_bfloat16*>(base)[elem]);
-}
-__device__ __forceinline__ void store_one(void* base, long long elem, float v, bool fp32) {
-  if (fp32) static_cast<float*>(base)[elem] = v;
-  else static_cast<__nv_bfloat16*>(base)[elem] = __float2bfloat16_rn(v);
-}
-__device__ __forceinline__ float2 load_pair(const void* base, long long elem, bool fp32) {
-  if (fp32) return *reinterpret_cast<const float2*>(static_cast<const float*>(base) + elem);
-  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(static_cast<const __nv_bfloat16*>(base) + elem));
-}
-__device__ __forceinline__ void store_pair(void* base, long long elem, float2 v, bool fp32) {
-  if (fp32) *reinterpret_cast<float2*>(static_cast<float*>(base) + elem) = v;
-  else *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(base) + elem) = __float22bfloat162_rn(v);
-}
-
 // Asynchronous global -> shared copies (LDGSTS): issued now, waited for with cp_async_wait_all.
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
@@ -185,8 +168,9 @@ __device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
-// Streams that pass through L2 once (the input, the finished coefficients, the output) are
-// marked evict-first, so that they give way to the fp32 volume that is read back soon after.
+// Streams that pass through L2 once (the input, the finished coefficients) are marked
+// evict-first in the fused forward kernel, so that they give way to the fp32 volume that is read
+// back soon after.
 __device__ __forceinline__ uint64_t l2_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(p));
@@ -204,10 +188,6 @@ __device__ __forceinline__ void cp_async4_ef(void* smem, const void* gmem, uint6
 }
 __device__ __forceinline__ void st_ef(float* p, float v, uint64_t pol) {
   asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;\n" ::"l"(p), "f"(v), "l"(pol) : "memory");
-}
-__device__ __forceinline__ void st_ef(__nv_bfloat16* p, __nv_bfloat16 v, uint64_t pol) {
-  asm volatile("st.global.L2::cache_hint.b16 [%0], %1, %2;\n" ::"l"(p), "h"(__bfloat16_as_ushort(v)), "l"(pol)
-               : "memory");
 }
 // Invalidate the 128-byte L2 line at p (global memory, 128-byte aligned) without writing it back,
 // for scratch data that nothing reads again; its contents become undefined.
