@@ -8,9 +8,11 @@
 // missing key or drops the smallest kept one, so the result is the set of the B largest keys
 // (ties to the lower bin index).  This kernel selects that set directly and exactly:
 //   * the B-th largest key K is found by radix selection on its fp64 bit pattern (patterns of
-//     positive doubles order like their values): a histogram of all keys' exponents, then 8-bit
-//     digits of the mantissa among the keys with K's exponent -- 8 passes; if any key would be
-//     subnormal, by bisection over the patterns instead;
+//     positive doubles order like their values): a histogram of all keys' exponents, then 11-bit
+//     digits of the mantissa among the keys with K's exponent.  Every key is a normal fp64
+//     number: a variance is an fp64 sum of float32 energies divided by n <= 2^16, so a positive
+//     one is at least 2^-149 / 2^16 = 2^-165, and its smallest key (4^-7 of it) 2^-179 lies far
+//     above the smallest normal double 2^-1022;
 //   * count(v) = #keys >= v is evaluated per bin from the fp64 exponent and mantissa fields
 //     (sigma^2 4^-k >= v  <=>  2k <= e(sigma^2) - e(v) - 1 + [m(sigma^2) >= m(v)]);
 //   * keys above K are all taken, keys equal to K are handed out in bin order until the budget
@@ -30,20 +32,11 @@ namespace {
 constexpr size_t kAllocSmemVar = 192 * 1024;   // variances kept in shared memory up to N = 24576 bins
 constexpr int kExpBuckets = 2048;                // biased exponents of fp64
 
-// Number of keys var * 4^-k (k = 0..7) that are >= v, exactly; var > 0, v >= 0.
+// Number of keys var * 4^-k (k = 0..7) that are >= v, exactly, for positive normal var and v (every
+// variance and every selection threshold here is normal, see the head of this file).
 __device__ __forceinline__ int key_count(double var, double v) {
   const unsigned long long a = __double_as_longlong(var), b = __double_as_longlong(v);
   const int ea = (int)(a >> 52), eb = (int)(b >> 52);
-  if (ea == 0 || eb == 0) {  // subnormal or zero operand: compare the keys directly (exact)
-    int c = 0;
-    double k = var;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      c += k >= v;
-      k *= 0.25;
-    }
-    return c;
-  }
   const int g = (a & 0xFFFFFFFFFFFFFull) >= (b & 0xFFFFFFFFFFFFFull);
   const int d = ea - eb - 1 + g;  // key k qualifies iff 2k <= d
   if (d < 0) return 0;
@@ -60,18 +53,6 @@ __device__ T block_sum(T v, T* s_red /* 32 entries */) {
   __syncthreads();
   T r = 0;
   for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r += s_red[w];
-  return r;
-}
-
-__device__ double block_max(double v, double* s_red) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
-  __syncthreads();
-  if (lane == 0) s_red[warp] = v;
-  __syncthreads();
-  double r = s_red[0];
-  for (int w = 1; w < (int)(blockDim.x >> 5); ++w) r = fmax(r, s_red[w]);
   return r;
 }
 
@@ -134,7 +115,6 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
                                                                  double* __restrict__ var_ws, bool var_in_smem,
                                                                  uint32_t* __restrict__ index, uint4* __restrict__ recs) {
   __shared__ long long s_ll[32];
-  __shared__ double s_d[32];
   __shared__ uint32_t s_scan[33];
   __shared__ uint32_t s_cnt[kAllocThreads];
   __shared__ uint32_t s_slab[kMaxSlabs];
@@ -143,7 +123,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
   __shared__ uint32_t s_NZ[kMaxSlabs + 1];
   __shared__ uint32_t s_bpos[kMaxN / kPackRecs + 1];
   __shared__ uint32_t s_hist[kExpBuckets], s_rev[kExpBuckets];
-  __shared__ int s_pick, s_emin;
+  __shared__ int s_pick;
   __shared__ uint32_t s_above, s_count;
   __shared__ unsigned long long s_mant;
   extern __shared__ __align__(16) unsigned char smem_var[];
@@ -159,10 +139,6 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
 
   // 1. sigma^2 (reduced over the channel chunks by reduce_var_kernel)
   long long act = 0;
-  double vmax = 0.0;
-  int emin = 2047;   // smallest biased exponent of a positive variance
-  if (threadIdx.x == 0) s_emin = 2047;
-  __syncthreads();
   const double* var_g = var_ws + (size_t)u * g.N;
   // the counting passes take bins interleaved across threads (bin i to thread i mod blockDim):
   // consecutive threads read consecutive variances, without bank conflicts
@@ -170,97 +146,76 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
     const double v = var_g[i];
     var[i] = v;
     act += v > 0.0;
-    vmax = fmax(vmax, v);
-    if (v > 0.0) emin = min(emin, (int)(__double_as_longlong(v) >> 52));
   }
-  atomicMin(&s_emin, emin);   // (block_sum synchronizes the block before s_emin is read)
   act = block_sum<long long>(act, s_ll);
-  vmax = block_max(vmax, s_d);
   const long long B = (long long)g.bits * g.N;
   const bool select = !raw && 8 * act > B;
 
   // 2. the B-th largest key K (counted with multiplicity): the largest pattern lo with
   // count(lo) >= B, so count(lo + 1) < B.  The keys of bin i are var_i * 4^-k: the mantissa of
-  // var_i with the exponents e_i - 2k.  When every key is a normal number (e_i >= 15), K is found by
-  // radix selection: K's exponent from the histogram of all keys' exponents (the histogram of the
-  // bins' exponents summed over the 8 shifts), then 11-bit digits of K's mantissa from the keys
-  // with that exponent (at most one per bin), until one key is left.  Otherwise (subnormal keys)
-  // by bisection over the 64-bit patterns, which order like the values.
+  // var_i with the exponents e_i - 2k (all normal numbers, see the head of this file).  K is found
+  // by radix selection: K's exponent from the histogram of all keys' exponents (the histogram of
+  // the bins' exponents summed over the 8 shifts), then 11-bit digits of K's mantissa from the
+  // keys with that exponent (at most one per bin), until one key is left.
   unsigned long long lo = 0, hi = 0;
   if (select) {
-    if (s_emin >= 15) {
-      for (int j = threadIdx.x; j < kExpBuckets; j += blockDim.x) s_hist[j] = 0;
-      __syncthreads();
-      const unsigned lt = (1u << (threadIdx.x & 31)) - 1u;
-      for (int i0 = 0; i0 < g.N; i0 += blockDim.x) {   // warp-uniform rounds: bins with one exponent
-        const int i = i0 + (int)threadIdx.x;           // are counted by one atomic per warp
-        const double x = i < g.N ? var[i] : 0.0;
-        const int e = x > 0.0 ? (int)(__double_as_longlong(x) >> 52) : -1;
-        const unsigned peers = __match_any_sync(0xffffffffu, e);
-        if (e >= 0 && (peers & lt) == 0u) atomicAdd(&s_hist[e], (uint32_t)__popc(peers));
-      }
-      __syncthreads();
-      for (int j = threadIdx.x; j < kExpBuckets; j += blockDim.x) {
-        uint32_t c = 0;
+    for (int j = threadIdx.x; j < kExpBuckets; j += blockDim.x) s_hist[j] = 0;
+    __syncthreads();
+    const unsigned lt = (1u << (threadIdx.x & 31)) - 1u;
+    for (int i0 = 0; i0 < g.N; i0 += blockDim.x) {   // warp-uniform rounds: bins with one exponent
+      const int i = i0 + (int)threadIdx.x;           // are counted by one atomic per warp
+      const double x = i < g.N ? var[i] : 0.0;
+      const int e = x > 0.0 ? (int)(__double_as_longlong(x) >> 52) : -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, e);
+      if (e >= 0 && (peers & lt) == 0u) atomicAdd(&s_hist[e], (uint32_t)__popc(peers));
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j < kExpBuckets; j += blockDim.x) {
+      uint32_t c = 0;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) c += j + 2 * k < kExpBuckets ? s_hist[j + 2 * k] : 0u;
-        s_rev[j] = c;   // keys with exponent j
+      for (int k = 0; k < 8; ++k) c += j + 2 * k < kExpBuckets ? s_hist[j + 2 * k] : 0u;
+      s_rev[j] = c;   // keys with exponent j
+    }
+    __syncthreads();
+    uint32_t above = 0, here = 0;
+    const int E = select_bucket(s_rev, kExpBuckets, (uint32_t)B, s_hist, s_scan, &s_pick, &s_above, &s_count,
+                                &above, &here);
+    uint32_t need = (uint32_t)B - above;      // K is the need-th largest key with exponent E
+    unsigned long long prefix = 0;            // K's leading mantissa bits selected so far
+    int done = 0;                             // how many of the 52 mantissa bits
+    while (done < 52) {
+      const int width = min(11, 52 - done), shift = 52 - done - width;
+      __syncthreads();
+      for (int j = threadIdx.x; j < (1 << width); j += blockDim.x) s_hist[j] = 0;
+      __syncthreads();
+      for (int i = threadIdx.x; i < g.N; i += blockDim.x) {
+        const unsigned long long bits = (unsigned long long)__double_as_longlong(var[i]);
+        const int d = (int)(bits >> 52) - E;   // (var[i] > 0: its sign bit is 0)
+        const unsigned long long m = bits & 0xFFFFFFFFFFFFFull;
+        if (var[i] > 0.0 && d >= 0 && d <= 14 && !(d & 1) && (m >> (shift + width)) == prefix)
+          atomicAdd(&s_hist[(m >> shift) & ((1u << width) - 1u)], 1u);
       }
       __syncthreads();
-      uint32_t above = 0, here = 0;
-      const int E = select_bucket(s_rev, kExpBuckets, (uint32_t)B, s_hist, s_scan, &s_pick, &s_above, &s_count,
-                                  &above, &here);
-      uint32_t need = (uint32_t)B - above;      // K is the need-th largest key with exponent E
-      unsigned long long prefix = 0;            // K's leading mantissa bits selected so far
-      int done = 0;                             // how many of the 52 mantissa bits
-      while (done < 52) {
-        const int width = min(11, 52 - done), shift = 52 - done - width;
-        __syncthreads();
-        for (int j = threadIdx.x; j < (1 << width); j += blockDim.x) s_hist[j] = 0;
-        __syncthreads();
+      uint32_t above_d = 0;
+      const int digit = select_bucket(s_hist, 1 << width, need, s_rev, s_scan, &s_pick, &s_above, &s_count,
+                                      &above_d, &here);
+      need -= above_d;
+      prefix = (prefix << width) | (unsigned long long)digit;
+      done += width;
+      if (here == 1u && done < 52) {   // a single key has these leading bits: it is K
         for (int i = threadIdx.x; i < g.N; i += blockDim.x) {
           const unsigned long long bits = (unsigned long long)__double_as_longlong(var[i]);
-          const int d = (int)(bits >> 52) - E;   // (var[i] > 0: its sign bit is 0)
+          const int d = (int)(bits >> 52) - E;
           const unsigned long long m = bits & 0xFFFFFFFFFFFFFull;
-          if (var[i] > 0.0 && d >= 0 && d <= 14 && !(d & 1) && (m >> (shift + width)) == prefix)
-            atomicAdd(&s_hist[(m >> shift) & ((1u << width) - 1u)], 1u);
+          if (var[i] > 0.0 && d >= 0 && d <= 14 && !(d & 1) && (m >> shift) == prefix) s_mant = m;
         }
         __syncthreads();
-        uint32_t above_d = 0;
-        const int digit = select_bucket(s_hist, 1 << width, need, s_rev, s_scan, &s_pick, &s_above, &s_count,
-                                        &above_d, &here);
-        need -= above_d;
-        prefix = (prefix << width) | (unsigned long long)digit;
-        done += width;
-        if (here == 1u && done < 52) {   // a single key has these leading bits: it is K
-          for (int i = threadIdx.x; i < g.N; i += blockDim.x) {
-            const unsigned long long bits = (unsigned long long)__double_as_longlong(var[i]);
-            const int d = (int)(bits >> 52) - E;
-            const unsigned long long m = bits & 0xFFFFFFFFFFFFFull;
-            if (var[i] > 0.0 && d >= 0 && d <= 14 && !(d & 1) && (m >> shift) == prefix) s_mant = m;
-          }
-          __syncthreads();
-          prefix = s_mant;
-          done = 52;
-        }
-      }
-      lo = ((unsigned long long)E << 52) | prefix;
-      hi = lo + 1ull;
-    } else {
-      hi = (unsigned long long)__double_as_longlong(vmax) + 1ull;   // above every key: count = 0 < B
-      while (hi - lo > 1) {                                         // count(+0) = 8 * act > B
-        const unsigned long long mid = lo + (hi - lo) / 2;
-        const double v = __longlong_as_double((long long)mid);
-        long long c = 0;
-        for (int i = threadIdx.x; i < g.N; i += blockDim.x) {
-          const double x = var[i];
-          if (x > 0.0) c += key_count(x, v);
-        }
-        c = block_sum<long long>(c, s_ll);
-        if (c >= B) lo = mid;
-        else hi = mid;
+        prefix = s_mant;
+        done = 52;
       }
     }
+    lo = ((unsigned long long)E << 52) | prefix;
+    hi = lo + 1ull;
   }
   const double v_lo = __longlong_as_double((long long)lo), v_hi = __longlong_as_double((long long)hi);
 
@@ -415,7 +370,8 @@ __global__ void __launch_bounds__(256) decode_index_kernel(const __grid_constant
                                                            const __grid_constant__ UnitList ul,
                                                            uint32_t* __restrict__ index, uint4* __restrict__ recs,
                                                            unsigned int* status) {
-  __shared__ int s_ok;
+  __shared__ int s_ok;    // header check: written by thread 0 before the first barrier, then only read
+  __shared__ int s_bad;   // allocation check: set by any thread, read after the next barriers
   __shared__ uint32_t s_slab[kMaxSlabs];
   __shared__ uint32_t s_nzslab[kMaxSlabs];
   __shared__ uint32_t s_P[kMaxSlabs + 1];
@@ -439,11 +395,15 @@ __global__ void __launch_bounds__(256) decode_index_kernel(const __grid_constant
            (long long)total == (long long)g.off_codes + (long long)g.n * cs && (long long)total <= g.capacity;
     }
     s_ok = ok;
+    s_bad = 0;
   }
   __syncthreads();
-  bool ok = s_ok;
+  // Every thread takes the same branch below: s_ok is not written again, and the allocation check
+  // reports through s_bad, which is read only after the barriers that follow every write to it.
+  const bool header_ok = s_ok;
+  bool ok = header_ok;
   const unsigned char* b = pay + kHeaderBytes;
-  if (ok && !raw) {
+  if (header_ok && !raw) {
     bool bad = false;
     for (int k = warp; k < g.S; k += nwarps) {
       uint32_t sum = 0, nz = 0;
@@ -460,14 +420,14 @@ __global__ void __launch_bounds__(256) decode_index_kernel(const __grid_constant
         s_nzslab[k] = nz;
       }
     }
-    if (bad) s_ok = 0;
+    if (bad) s_bad = 1;
     __syncthreads();
     if (warp == 0) slab_scan(s_slab, g.S, s_P);
     else if (warp == 1) slab_scan(s_nzslab, g.S, s_NZ);
     __syncthreads();
-    if (threadIdx.x == 0 && s_P[g.S] != reinterpret_cast<const uint32_t*>(pay)[10]) s_ok = 0;
+    if (threadIdx.x == 0 && s_P[g.S] != reinterpret_cast<const uint32_t*>(pay)[10]) s_bad = 1;
     __syncthreads();
-    ok = s_ok;
+    ok = s_bad == 0;
   }
   uint32_t* P = index + (size_t)u * unit_index_words(g.S);
   uint32_t* NZ = P + g.S + 2;
@@ -526,14 +486,19 @@ cudaError_t launch_decode_index(const Geom& g, const UnitList& ul, int nu, uint3
   return cudaGetLastError();
 }
 
-cudaError_t launch_allocate(const Geom& g, const UnitList& ul, int nu, const float* partial, double* var,
-                            uint32_t* index, uint4* recs, cudaStream_t st) {
+cudaError_t launch_allocate_from_var(const Geom& g, const UnitList& ul, int nu, double* var, uint32_t* index,
+                                     uint4* recs, cudaStream_t st) {
   const size_t var_bytes = (size_t)g.N * sizeof(double);
   const bool in_smem = var_bytes <= kAllocSmemVar;
   if (in_smem) cudaFuncSetAttribute(allocate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)var_bytes);
-  reduce_var_kernel<<<dim3((g.N + 255) / 256, nu), 256, 0, st>>>(g, partial, var);
   allocate_kernel<<<nu, kAllocThreads, in_smem ? var_bytes : 0, st>>>(g, ul, var, in_smem, index, recs);
   return cudaGetLastError();
+}
+
+cudaError_t launch_allocate(const Geom& g, const UnitList& ul, int nu, const float* partial, double* var,
+                            uint32_t* index, uint4* recs, cudaStream_t st) {
+  reduce_var_kernel<<<dim3((g.N + 255) / 256, nu), 256, 0, st>>>(g, partial, var);
+  return launch_allocate_from_var(g, ul, nu, var, index, recs, st);
 }
 
 }  // namespace tactkv

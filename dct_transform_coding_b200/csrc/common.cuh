@@ -83,6 +83,10 @@ void axis_hw_shape(int hcls, int wcls, const Geom& g, bool inverse, int mode, si
 // (N per unit), and zeroes the stream word at every P(k_s).
 cudaError_t launch_allocate(const Geom& g, const UnitList& ul, int nu, const float* partial, double* var,
                             uint32_t* index, uint4* recs, cudaStream_t st);
+// The allocation alone, on the fp64 variances var[u][bin] given in the workspace (which it
+// overwrites): the same kernel and outputs as launch_allocate without the variance reduction.
+cudaError_t launch_allocate_from_var(const Geom& g, const UnitList& ul, int nu, double* var, uint32_t* index,
+                                     uint4* recs, cudaStream_t st);
 // Quantization and packing of the finished coefficients X (workspace volume) into the payloads.
 cudaError_t launch_pack(const Geom& g, const UnitList& ul, int nu, const float* X, const uint4* recs,
                         const uint32_t* index, cudaStream_t st);

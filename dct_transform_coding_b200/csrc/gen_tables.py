@@ -1,8 +1,8 @@
 #!/usr/bin/env python3
 """Generate the CUDA library's fixed Lloyd-Max codebooks (build step; writes lloyd_max_tables.inc).
 
-TACT-KV quantizes every surviving bin coordinate with "a precomputed Lloyd-Max table at that
-bin's bit width" ("Methodology in Plain English", stage 4).  The codebook is the minimum-MSE
+TACT-KV quantizes every coordinate of a surviving bin with a fixed Lloyd-Max codebook chosen by
+the bin's bit width ("Methodology in Plain English", stage 4).  The codebook is the minimum-MSE
 scalar quantizer of a unit Gaussian with 2^b levels, b = 1..8: every level is the centroid of
 its cell and every threshold the midpoint of two neighbouring levels.
 

@@ -385,6 +385,35 @@ tactkv_status tactkv_compress_noalloc(const tactkv_unit* units, int n_units, str
   return compress_impl(units, n_units, ws, kNoAllocScratchBytes, stream, nullptr);
 }
 
+tactkv_status tactkv_allocate(const tactkv_unit* unit, const double* var, void* workspace, size_t workspace_bytes,
+                              struct CUstream_st* stream) {
+  t_launches = 0;
+  if (!unit || !var || !unit->payload) return TACTKV_INVALID_ARG;
+  Geom g;
+  tactkv_status st = make_geom(*unit, g);
+  if (st != TACTKV_OK) return st;
+  if (reinterpret_cast<uintptr_t>(unit->payload) % 16 || reinterpret_cast<uintptr_t>(var) % 8) return TACTKV_ALIGNMENT;
+  if (unit->payload_capacity < payload_bytes_geom(g)) return TACTKV_CAPACITY;
+  g.capacity = (long long)unit->payload_capacity;
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256 || workspace_bytes < kStatusBytes + unit_ws_bytes(g))
+    return TACTKV_WORKSPACE;
+  UnitList ul;
+  memset(&ul, 0, sizeof(ul));
+  ul.u[0].in = unit->kv_in;
+  ul.u[0].out = unit->kv_out;
+  ul.u[0].payload = static_cast<unsigned char*>(unit->payload);
+  ul.u[0].tok_stride = unit->token_stride;
+  ul.u[0].head_stride = unit->head_stride;
+  ul.u[0].layer = unit->layer;
+  ul.u[0].kv = unit->kv;
+  const WsView w = view(static_cast<unsigned char*>(workspace), g, 1);
+  if (cudaMemcpyAsync(w.var, var, sizeof(double) * g.N, cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
+    return TACTKV_CUDA;
+  t_launches = 1;
+  if (launch_allocate_from_var(g, ul, 1, w.var, w.index, w.recs, stream) != cudaSuccess) return TACTKV_CUDA;
+  return TACTKV_OK;
+}
+
 tactkv_status tactkv_device_status(void* workspace, size_t workspace_bytes, struct CUstream_st* stream) {
   if (!workspace || workspace_bytes < kStatusBytes) return TACTKV_WORKSPACE;
   unsigned int v = 0;

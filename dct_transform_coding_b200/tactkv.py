@@ -37,7 +37,7 @@ TACTKV_FP32_IO = 2
 HEADER_BYTES = 64
 EXPORTED = ("tactkv_payload_bytes", "tactkv_workspace_bytes", "tactkv_compress", "tactkv_decompress",
             "tactkv_compress_profiled", "tactkv_decompress_profiled", "tactkv_compress_noalloc",
-            "tactkv_device_status",
+            "tactkv_allocate", "tactkv_device_status",
             "tactkv_status_string", "tactkv_lloyd_max_table", "tactkv_format_version", "tactkv_last_launches")
 
 
@@ -67,6 +67,8 @@ for _name in ("tactkv_compress_profiled", "tactkv_decompress_profiled"):
                                      ctypes.POINTER(ctypes.c_void_p)]
 _lib.tactkv_compress_noalloc.restype = ctypes.c_int
 _lib.tactkv_compress_noalloc.argtypes = [_P, ctypes.c_int, ctypes.c_void_p]
+_lib.tactkv_allocate.restype = ctypes.c_int
+_lib.tactkv_allocate.argtypes = [_P, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
 _lib.tactkv_device_status.restype = ctypes.c_int
 _lib.tactkv_device_status.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
 _lib.tactkv_status_string.restype = ctypes.c_char_p
@@ -133,6 +135,30 @@ def tactkv_compress_noalloc(units, stream_ptr: int) -> int:
     calls that could overlap on the GPU."""
     arr = _as_array(units)
     return int(_lib.tactkv_compress_noalloc(arr, len(arr), ctypes.c_void_p(stream_ptr)))
+
+
+def tactkv_allocate(unit: tactkv_unit, var_ptr: int, workspace_ptr: int, workspace_bytes: int,
+                    stream_ptr: int) -> int:
+    """Stage 3 on given fp64 variances (device pointer var_ptr, N doubles): header, b[] and sigma[]
+    of unit.payload as compress would write them."""
+    return int(_lib.tactkv_allocate(ctypes.byref(unit), ctypes.c_void_p(var_ptr), ctypes.c_void_p(workspace_ptr),
+                                    workspace_bytes, ctypes.c_void_p(stream_ptr)))
+
+
+def allocate(var: torch.Tensor, S: int, H: int, W: int, bits: int, *, heads: int = 1, head_dim: int = 32,
+             stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Bit allocation of the fp64 variances var [S*H*W] (on the GPU): returns b [S*H*W] uint8."""
+    var = var.to(torch.float64).contiguous()
+    cap = payload_capacity(S, H, W, heads, head_dim, bits)
+    payload = torch.zeros(((cap + 15) // 16 * 16,), dtype=torch.uint8, device=var.device)
+    u = tactkv_unit(S=S, H=H, W=W, heads=heads, head_dim=head_dim, bits=bits, payload=payload.data_ptr(),
+                    payload_capacity=payload.numel(), token_stride=heads * head_dim, head_stride=head_dim)
+    ws = alloc_workspace([u], var.device)
+    st = tactkv_allocate(u, var.data_ptr(), ws.data_ptr(), ws.numel(), _stream_ptr(stream))
+    if st != TACTKV_OK:
+        raise TactkvError(st, "tactkv_allocate")
+    N = S * H * W
+    return payload[HEADER_BYTES:HEADER_BYTES + N]
 
 
 def tactkv_device_status(workspace_ptr: int, workspace_bytes: int, stream_ptr: int) -> int:

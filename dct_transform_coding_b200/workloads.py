@@ -3,9 +3,9 @@
 The TACT-KV pages evaluate on real CT / video KV caches that are not available here, so every
 input is a synthetic stand-in with the structure the method relies on: a visual K or V tensor of
 one layer, laid out on its (S, H, W) token grid ("Methodology in Plain English", stage 1 of the
-TACT-KV summary page), strongly correlated along all three axes ("strongly autocorrelated along
-all three spatial axes", same section) and heavy-tailed ("Main Findings", gain-shape bullet:
-post-DCT absmax/std 4.81 versus 3.01 for a Gaussian).
+TACT-KV summary page), correlated along each of the three axes (the same section names this
+as the redundancy the 3D transform removes) and heavy-tailed ("Main Findings", gain-shape
+bullet: post-DCT absmax/std 4.81 versus 3.01 for a Gaussian).
 
 Field recipe (per channel): iid innovations e, filtered along S, then H, then W by a stationary
 AR(1) recursion y[0] = e[0], y[t] = rho * y[t-1] + sqrt(1 - rho^2) * e[t]; innovations are

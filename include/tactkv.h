@@ -17,9 +17,10 @@
  * i = (k_s*H + k_h)*W + k_w, N = T bins.  Nominal budget: bits*N bit slots per channel.
  *
  * Memory.  Every pointer in a unit descriptor and the workspace are DEVICE pointers owned by
- * the caller.  The library allocates nothing, keeps no state other than constant tables in the
- * CUDA module, and is safe to call from several host threads on different streams provided
- * each call has its own workspace.  Calls are asynchronous on `stream`; a status other than
+ * the caller.  The library allocates nothing.  Its only state is the constant tables in the CUDA
+ * module and the fixed device scratch array of tactkv_compress_noalloc (below); every other entry
+ * point is safe to call from several host threads on different streams provided each call has
+ * its own workspace.  Calls are asynchronous on `stream`; a status other than
  * TACTKV_OK means nothing was launched for the failing group of units (earlier groups of the
  * same call may already be queued).  Errors found by the kernels (a corrupt payload) are
  * recorded in the workspace and read back with tactkv_device_status().
@@ -36,7 +37,7 @@
  *                       i's code, P_i = sum_{j<i} b_j; stream bit q is bit (q&7) of byte q>>3.
  *                       With TACTKV_NO_QUANT a stream holds the N float32 coefficients instead.
  * pad16(x) rounds x up to a multiple of 16.  The gain/rate part is the pages' sum(b_i*d + 32)
- * bits per layer; the b[] bytes are its "small index overhead".
+ * bits per layer; the b[] bytes are the index the pages add on top of it.
  */
 #ifndef TACTKV_H_
 #define TACTKV_H_
@@ -140,6 +141,19 @@ tactkv_status tactkv_decompress_profiled(const tactkv_unit* units, int n_units, 
    tactkv_compress. */
 tactkv_status tactkv_compress_noalloc(const tactkv_unit* units, int n_units,
                                       struct CUstream_st* stream);
+
+/* Stage 3 alone ("Methodology in Plain English", stage 3: reverse water-filling of the bit budget
+   bits*N over the bins, cap 8 bits): the allocation compress runs, applied to the variances the
+   caller gives instead of the ones compress measures.  var: DEVICE array of N = S*H*W doubles,
+   var[i] >= 0 the variance of bin i (8-byte aligned; not modified).  Writes into unit->payload
+   exactly what compress writes there from its own variances: the header, b[N] (the selection of
+   the B = bits*N largest keys var_i * 4^-k, k = 0..7, ties to the lower bin index, every active bin
+   at 8 bits when 8*#active <= B; b = 0 where var = 0), sigma[N] = float32(sqrt(var)) and the zero
+   padding; the code area is left unspecified.  Only the unit's shape, bits, flags, layer, kv,
+   payload and payload_capacity are read.  workspace: at least tactkv_workspace_bytes(unit, 1)
+   bytes, 256-byte aligned.  Asynchronous on `stream`; one kernel. */
+tactkv_status tactkv_allocate(const tactkv_unit* unit, const double* var, void* workspace,
+                              size_t workspace_bytes, struct CUstream_st* stream);
 
 /* Synchronizes `stream`, returns the first error the kernels recorded in `workspace` since the
    previous call (TACTKV_OK if none), and clears it. */

@@ -14,7 +14,7 @@ Transform for Compressing Volumetric KV Caches in Medical VLMs", ai.info), secti
 2. Transform (stage 2): orthonormal separable 3D DCT-II along S, H and W, per channel; the
    feature axis is not transformed.  Frequency bin i = (k_s*H + k_h)*W + k_w.
 3. Bit allocation (stage 3): per-bin variance sigma_i^2 = mean over the n channels of X[i,c]^2
-   (estimated on the fly per layer per sequence, "Key Contributions" item 3); reverse
+   (estimated afresh for every layer of every sequence, "Key Contributions" item 3); reverse
    water-filling b_i = max(0, 1/2 log2(sigma_i^2 / theta)), theta by bisection, b_i rounded to
    integers, a +-1 greedy correction to hit the budget, cap 8 bits, b_i = 0 drops the bin.
 4. Quantize (stage 4): gain-shape -- each bin is scaled by its own sigma_i and every coordinate
@@ -75,7 +75,8 @@ def _pad16(x: int) -> int:
 def dct_matrix(L: int) -> np.ndarray:
     """Orthonormal DCT-II matrix: C[k, t] = a_k cos(pi (2t+1) k / (2L)), a_0 = sqrt(1/L), a_k = sqrt(2/L).
 
-    Stage 2 of the methodology ("separable 3D DCT-II ... orthonormal and lossless on its own").
+    Stage 2 of the methodology: a separable 3D DCT-II whose basis is orthonormal, so the transform
+    alone loses nothing.
     """
     k = np.arange(L, dtype=np.float64)[:, None]
     t = np.arange(L, dtype=np.float64)[None, :]
@@ -143,8 +144,10 @@ def water_level(var: np.ndarray, B: float) -> float:
 def allocate_bits(var: np.ndarray, bits: int) -> np.ndarray:
     """Integer bits per bin by reverse water-filling with bisection and a +-1 greedy fix.
 
-    Stage 3 of the methodology: "a water level is found by bisection with a +-1 greedy
-    correction to hit the budget exactly.  Bits are capped at 8."  Budget B = bits * N.
+    Stage 3 of the methodology ("Methodology in Plain English" on the TACT-KV summary page): the
+    water level theta comes from a bisection, the continuous rates are rounded, and single-bit
+    greedy steps then bring the total exactly to the budget B = bits * N; no bin takes more than
+    8 bits.
     """
     var = np.asarray(var, dtype=np.float64)
     N = var.size
@@ -222,8 +225,8 @@ def _centroids(levels: np.ndarray):
 
 
 def lloyd_max(bits: int) -> Tuple[np.ndarray, np.ndarray]:
-    """Lloyd-Max quantizer of a unit Gaussian with 2^bits levels (stage 4: "precomputed Lloyd-Max
-    table"): levels are the centroids of their cells and thresholds the midpoints of adjacent
+    """Lloyd-Max quantizer of a unit Gaussian with 2^bits levels (stage 4: the fixed codebook of
+    each bit width): levels are the centroids of their cells and thresholds the midpoints of adjacent
     levels.  Lloyd's alternation is run from a companding start; because it converges slowly for
     many levels, Newton's method on the same two conditions finishes it.  Returns (levels,
     thresholds), increasing."""
@@ -410,10 +413,13 @@ def codes_of(payload) -> Tuple[np.ndarray, np.ndarray]:
 
 
 def threshold_distance(u: np.ndarray, bits: int) -> np.ndarray:
-    """Distance of u to the nearest decision threshold, relative to max(1, |t|) (fp64)."""
-    _, t = table(bits)
-    u = np.asarray(u, dtype=np.float64)[..., None]
-    return np.min(np.abs(u - t) / np.maximum(1.0, np.abs(t)), axis=-1)
+    """Distance of u to the nearest decision threshold t_j of the b-bit codebook, each distance
+    taken relative to max(1, |t_j|) (fp64).  This is the band of the code-parity rule: a code may
+    differ from the oracle's only where this distance is at most 1e-5 (the middle threshold 0 of
+    an even codebook gets the absolute distance)."""
+    thresholds_b = table(bits)[1]
+    gaps = np.abs(np.asarray(u, dtype=np.float64)[..., None] - thresholds_b)
+    return np.min(gaps / np.maximum(1.0, np.abs(thresholds_b)), axis=-1)
 
 
 def to_bf16(x: np.ndarray) -> np.ndarray:

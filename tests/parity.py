@@ -1,9 +1,10 @@
 """Parity checks of the CUDA codec against the CPU oracle (shared by the GPU tests and smoke()).
 
 Acceptance, per unit (the codec's stated tolerances, with the readings needed to apply them):
-* bit allocations equal the oracle's exactly.  A differing bin is tolerated only as a tie
-  artefact: its deciding key sigma^2 4^-k lies within 1e-6 (relative) of the oracle's selection
-  threshold, where fp32-vs-fp64 variance estimates may legitimately swap the order;
+* bit allocations equal the oracle's exactly, with no tolerance.  The report gives the relative
+  gap between the B-th and the (B+1)-th largest key sigma^2 4^-k of the oracle ("alloc_margin"):
+  the GPU's variances come from float32 coefficients, so a gap of the order of 1e-7 could let the
+  two sides order those keys differently; a failure names that case, it is not forgiven;
 * quantization codes equal the oracle's, except where the oracle's scaled coefficient
   u = X / sigma lies within 1e-5 * max(1, |t|) of a decision threshold t (distance taken in
   sigma-scaled units, because the middle threshold is 0);
@@ -19,7 +20,7 @@ from oracle import tactkv_oracle as O
 CODE_BAND = 1e-5
 RECON_TOL = 1e-3
 ROUNDTRIP_TOL = 1e-5
-TIE_TOL = 1e-6
+NEAR_TIE = 1e-6
 
 
 def rel_rms(a, b) -> float:
@@ -39,6 +40,17 @@ def selection_threshold(var: np.ndarray, bits: int) -> float:
     return float(np.partition(keys, keys.size - B)[keys.size - B])
 
 
+def allocation_margin(var: np.ndarray, bits: int) -> float:
+    """Relative gap (K_B - K_{B+1}) / K_B between the B-th and the (B+1)-th largest keys (inf when
+    every active bin saturates or no key is left out): how far the oracle's selection is from a tie."""
+    act = var > 0
+    B = bits * var.size
+    keys = np.sort((var[act][:, None] * 4.0 ** -np.arange(8)[None, :]).ravel())[::-1]
+    if 8 * int(act.sum()) <= B or keys.size <= B:
+        return np.inf
+    return float((keys[B - 1] - keys[B]) / keys[B - 1])
+
+
 def compare_unit(x: np.ndarray, gpu_payload: bytes, gpu_recon: np.ndarray, *, S, H, W, heads, head_dim, bits,
                  layer=0, kv=0, flags=0, io_round=O.to_bf16, report=None):
     """Check one unit.  x: the input exactly as the GPU saw it; gpu_recon: the GPU decode of gpu_payload."""
@@ -56,20 +68,20 @@ def compare_unit(x: np.ndarray, gpu_payload: bytes, gpu_recon: np.ndarray, *, S,
     sig_g = g["sigma"].astype(np.float64)
     big = var > 1e-12 * max(var.max(), 1e-300)
     assert np.all(np.abs(sig_g[big] - sig_o[big]) <= 2e-5 * sig_o[big]), "gain mismatch"
-    out = dict(tie_bins=0, code_mismatch_band=0, codes=0)
+    out = dict(alloc_margin=np.inf, code_mismatch_band=0, codes=0)
     if no_quant:
         Xg = g["streams"][:, :4 * N].copy().view("<f4").astype(np.float64).T
         assert rel_rms(Xg, info["X"]) <= ROUNDTRIP_TOL
     else:
         b_o, b_g = info["b"], g["b"]
+        out["alloc_margin"] = allocation_margin(var, bits)
         differ = np.nonzero(b_o != b_g)[0]
         if differ.size:
             thr = selection_threshold(var, bits)
-            for i in differ:
-                k = min(b_o[i], b_g[i])                     # the key that decides the extra bit
-                key = var[i] * 4.0 ** -k
-                assert abs(key / thr - 1) < TIE_TOL, f"allocation differs at bin {i}: {b_o[i]} vs {b_g[i]}"
-            out["tie_bins"] = int(differ.size)
+            near = sum(abs(var[i] * 4.0 ** -min(b_o[i], b_g[i]) / thr - 1) < NEAR_TIE for i in differ)
+            raise AssertionError(f"allocation differs at {differ.size} bins (first {differ[0]}: oracle "
+                                 f"{b_o[differ[0]]}, GPU {b_g[differ[0]]}); {near} of them decide a key within "
+                                 f"{NEAR_TIE} of the selection threshold (float32 vs fp64 near-tie)")
         assert b_g.sum() == g["code_bits"]
         _, codes_g = O.codes_of(gpu_payload)
         codes_o = info["codes"]

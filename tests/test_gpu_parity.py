@@ -255,6 +255,51 @@ def test_full_size_sampled_units(name, bits, pick):
     torch.cuda.empty_cache()
 
 
+# ------------------------------------------------------------------------------ exact ties ---
+def _gpu_allocation(var, grid, bits):
+    S, H, W = grid
+    v = torch.from_numpy(np.asarray(var, dtype=np.float64)).to(DEV)
+    b = T.allocate(v, S, H, W, bits)
+    torch.cuda.synchronize()
+    return b.cpu().numpy().astype(np.int64)
+
+
+@pytest.mark.parametrize("var,grid,bits,want", [
+    ([1.0, 1.0, 16.0], (1, 1, 3), 1, [1, 0, 2]),       # three keys equal to 1 for the last slot
+    ([1.0, 4.0, 4.0], (1, 1, 3), 1, [1, 1, 1]),
+    ([8.0, 2.0], (1, 1, 2), 1, [2, 0]),                # keys 8 4^-(k+1) = 2 4^-k tie at every k
+    ([8.0, 2.0], (1, 1, 2), 2, [3, 1]),
+    ([2.0, 8.0], (1, 1, 2), 1, [1, 1]),                # key 2 of bin 0 ties key 8/4 of bin 1: bin 0 wins
+    ([0.0, 5.0, 0.0, 5.0], (1, 2, 2), 3, [0, 6, 0, 6]),  # zero bins get nothing; budget 12 split evenly
+    ([3.0, 0.0, 1.0, 2.0], (1, 1, 4), 8, [8, 0, 8, 8]),  # every active bin saturates below the budget
+])
+def test_allocation_kernel_exact_on_planted_ties(var, grid, bits, want):
+    """Stage 3 ("Methodology in Plain English": the bisection, rounding and +-1 greedy steps up to
+    the budget, capped at 8 bits, ties to the lower bin index) on variances given to the library
+    directly, so the GPU and the oracle see the same fp64 numbers and exact ties are exact on both
+    sides.  Compared with no tolerance against the oracle and the brute-force top-B selection."""
+    var = np.asarray(var)
+    assert O.allocate_bits(var, bits).tolist() == want
+    assert O.allocate_bits_topk(var, bits).tolist() == want
+    assert _gpu_allocation(var, grid, bits).tolist() == want
+
+
+@pytest.mark.parametrize("grid,bits,seed", [((64, 16, 16), 1, 0), ((64, 16, 16), 2, 1), ((16, 16, 16), 4, 2),
+                                             ((32, 24, 24), 1, 3), ((7, 5, 9), 3, 4), ((64, 32, 32), 1, 5)])
+def test_allocation_kernel_exact_on_tie_heavy_variances(grid, bits, seed):
+    """Thousands of exact key ties: variances drawn from four mantissas times powers of 4 (so
+    sigma_i^2 4^-k of one bin equals that of many others), 10% of the bins empty.  The GPU's radix
+    selection and its in-order tie fill must give the oracle's allocation bit for bit."""
+    rng = np.random.default_rng(seed)
+    N = grid[0] * grid[1] * grid[2]
+    var = rng.choice([1.0, 1.5, 3.0, 0.75], N) * 4.0 ** rng.integers(-12, 12, N)
+    var[rng.random(N) < 0.1] = 0.0
+    b_gpu = _gpu_allocation(var, grid, bits)
+    b_o = O.allocate_bits(var, bits)
+    assert np.array_equal(b_gpu, b_o), np.nonzero(b_gpu != b_o)[0][:10]
+    assert b_gpu.sum() == bits * N
+
+
 # ------------------------------------------------------------------------------ error paths ---
 def test_corrupt_header_is_reported_and_zero_filled():
     S, H, W, heads, D = 8, 4, 4, 1, 32
@@ -272,6 +317,40 @@ def test_corrupt_header_is_reported_and_zero_filled():
     assert not out.any()
     # status is cleared once read; a good payload decodes cleanly afterwards
     T.decompress(pay, S, H, W, 2, heads=heads, head_dim=D, workspace=ws, check=True)
+
+
+def test_bit_width_above_8_is_reported_and_zero_filled():
+    """A payload whose header is intact but whose allocation holds a bit width of 9 (the sum of
+    the widths unchanged, so only the per-bin range check can catch it): the decoder's index
+    kernel must flag it, zero-fill that unit and decode the next unit of the batch normally."""
+    S, H, W, heads, D = 8, 4, 4, 1, 32
+    x = torch.stack([make_unit(S, H, W, heads, D, rho=(0.9, 0.9, 0.9), seed=s, device=DEV) for s in (2, 3)])
+    pay = T.compress(x, S, H, W, 2, layers=[0, 1])
+    bad = pay.clone()
+    b = bad[0, 64:64 + S * H * W].cpu().numpy().astype(np.int64)
+    i_hi = int(np.argmax(b))
+    donors = [j for j in np.argsort(-b) if j != i_hi and b[j] > 0]
+    need = 9 - int(b[i_hi])
+    for j in donors:                    # move bits from other bins so that the total is unchanged
+        take = min(need, int(b[j]))
+        b[j] -= take
+        need -= take
+        if need == 0:
+            break
+    assert need == 0
+    b[i_hi] = 9
+    bad[0, 64:64 + S * H * W] = torch.from_numpy(b.astype(np.uint8)).to(DEV)
+    units = T.make_units(None, S, H, W, 2, heads=heads, head_dim=D, payload=bad, out=torch.ones_like(x),
+                         layers=[0, 1], n_units=2)
+    ws = T.alloc_workspace(units, DEV)
+    out = torch.ones_like(x)
+    T.decompress(bad, S, H, W, 2, heads=heads, head_dim=D, out=out, layers=[0, 1], workspace=ws)
+    st = T.tactkv_device_status(ws.data_ptr(), ws.numel(), torch.cuda.current_stream().cuda_stream)
+    assert st == T.TACTKV_CORRUPT_PAYLOAD
+    assert not out[0].any()
+    good = T.decompress(pay, S, H, W, 2, heads=heads, head_dim=D, layers=[0, 1], check=True)
+    torch.cuda.synchronize()
+    assert torch.equal(out[1], good[1])
 
 
 def test_wrong_layer_is_rejected():

@@ -100,6 +100,19 @@ def test_workspace_checks_without_gpu(T):
     assert T.tactkv_compress(units, 1 << 20, need - 1, 0) == T.TACTKV_WORKSPACE
 
 
+def test_allocate_argument_checks_without_gpu(T):
+    u = _unit(T)
+    assert T.tactkv_allocate(u, 0, 1 << 20, 1 << 30, 0) == T.TACTKV_INVALID_ARG          # no variances
+    assert T.tactkv_allocate(_unit(T, payload=None), 4096, 1 << 20, 1 << 30, 0) == T.TACTKV_INVALID_ARG
+    assert T.tactkv_allocate(_unit(T, bits=9), 4096, 1 << 20, 1 << 30, 0) == T.TACTKV_INVALID_ARG
+    assert T.tactkv_allocate(_unit(T, S=17), 4096, 1 << 20, 1 << 30, 0) == T.TACTKV_UNSUPPORTED_SHAPE
+    assert T.tactkv_allocate(u, 4100, 1 << 20, 1 << 30, 0) == T.TACTKV_ALIGNMENT        # var not 8-aligned
+    assert T.tactkv_allocate(_unit(T, payload_capacity=100), 4096, 1 << 20, 1 << 30, 0) == T.TACTKV_CAPACITY
+    need = T.tactkv_workspace_bytes([u])
+    assert T.tactkv_allocate(u, 4096, 1 << 20, need - 1, 0) == T.TACTKV_WORKSPACE
+    assert T.tactkv_allocate(u, 4096, 0, need, 0) == T.TACTKV_WORKSPACE
+
+
 def test_decompress_checks_output_pointer(T):
     units = [_unit(T, kv_out=None)]
     assert T.tactkv_decompress(units, 1 << 20, 1 << 30, 0) == T.TACTKV_INVALID_ARG

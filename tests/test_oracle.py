@@ -2,8 +2,8 @@
 
 Each test checks the oracle against something other than itself: a closed form, a library
 routine that computes the same textbook transform, a brute-force search, a printed table, or
-an invariant the summary page states ("orthonormal and lossless on its own", "hit the budget
-exactly", "capped at 8", Theorem 1's 1/gamma).  A dropped term, a wrong sign or index, or a
+an invariant the summary page states (an orthonormal transform that alone loses nothing, an
+allocation that meets the budget exactly with at most 8 bits per bin, Theorem 1's 1/gamma).  A dropped term, a wrong sign or index, or a
 transposed operand anywhere in the oracle fails at least one of them.
 """
 import math
@@ -141,6 +141,43 @@ def test_quantize_decisions():
     assert list(codes) == [0, 1, 0, 1, 2, 2, 3, 3]
     # a threshold itself goes to the upper cell (decided in float32)
     assert O.quantize(np.array([np.float32(t2[2])]), 2)[0] == 3
+
+
+def _max1960_thresholds(golden_dir, bits):
+    with open(os.path.join(golden_dir, "lloyd_max_max1960.txt")) as f:
+        for line in f:
+            p = line.split()
+            if p and not line.startswith("#") and int(p[0]) == bits and p[1] == "thresholds":
+                return [float(v) for v in p[2:]]
+    raise KeyError(bits)
+
+
+def test_threshold_distance_hand_values(golden_dir):
+    """The code-parity band: distance from u to the NEAREST decision threshold t_j, divided by
+    max(1, |t_j|).  Pinned with thresholds printed by Max (1960) (4 significant digits, so every
+    expected value below is checked to a relative 1e-2, far tighter than any of the planted
+    alternatives: a squared divisor, the farthest threshold, the levels instead of thresholds)."""
+    t2 = _max1960_thresholds(golden_dir, 2)          # 0, 0.9816 (and -0.9816)
+    t3 = _max1960_thresholds(golden_dir, 3)          # 0, 0.5006, 1.050, 1.748
+    # the middle threshold 0 of an even codebook: the absolute distance
+    assert abs(O.threshold_distance(np.array([0.25]), 1)[0] - 0.25) < 1e-12
+    assert abs(O.threshold_distance(np.array([-0.3]), 1)[0] - 0.3) < 1e-12
+    assert abs(O.threshold_distance(np.array([0.01]), 2)[0] - 0.01) < 1e-12
+    # a threshold below 1 in magnitude: absolute distance as well
+    d = O.threshold_distance(np.array([t2[1] + 0.1, -(t2[1] + 0.1)]), 2)
+    assert np.allclose(d, 0.1, rtol=1e-2)
+    # a threshold above 1: the distance relative to |t_j| (not |t_j|^2)
+    d = O.threshold_distance(np.array([t3[3] + 0.2]), 3)[0]
+    assert abs(d / (0.2 / t3[3]) - 1) < 1e-2
+    # between two thresholds the nearer one counts: 0.75 lies 0.2494 above 0.5006 and 0.30 below
+    # 1.050 (0.2857 relative); the level 0.7560 in between is no decision boundary
+    d = O.threshold_distance(np.array([0.75]), 3)[0]
+    assert abs(d / (0.75 - t3[1]) - 1) < 1e-2
+    # far outside the table the outermost threshold decides: 3 bits, u = 5 -> (5 - 1.748) / 1.748
+    d = O.threshold_distance(np.array([5.0]), 3)[0]
+    assert abs(d / ((5.0 - t3[3]) / t3[3]) - 1) < 1e-2
+    # vectorised over any shape
+    assert O.threshold_distance(np.zeros((3, 4)), 2).shape == (3, 4)
 
 
 # ------------------------------------------------------------------------------ allocation ---

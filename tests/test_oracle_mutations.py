@@ -45,6 +45,13 @@ MUTATIONS = [
      "out[:, q >> 3] |= (bit << (7 - (q & 7))).astype(np.uint8)"),
     ("lloyd-max: thresholds not midpoints", "return y, 0.5 * (y[1:] + y[:-1])",
      "return y, 0.45 * (y[1:] + y[:-1])"),
+    ("code band: squared divisor", "return np.min(gaps / np.maximum(1.0, np.abs(thresholds_b)), axis=-1)",
+     "return np.min(gaps / np.maximum(1.0, np.abs(thresholds_b)) ** 2, axis=-1)"),
+    ("code band: farthest threshold", "return np.min(gaps / np.maximum(1.0, np.abs(thresholds_b)), axis=-1)",
+     "return np.max(gaps / np.maximum(1.0, np.abs(thresholds_b)), axis=-1)"),
+    ("code band: distance to the levels", "thresholds_b = table(bits)[1]", "thresholds_b = table(bits)[0]"),
+    ("code band: no relative scaling", "return np.min(gaps / np.maximum(1.0, np.abs(thresholds_b)), axis=-1)",
+     "return np.min(gaps, axis=-1)"),
 ]
 
 
