@@ -34,7 +34,7 @@ FALLBACK_HBM_GBS = 6650.0
 def parse_args():
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="med4b")
@@ -45,6 +45,8 @@ def parse_args():
     ap.add_argument("--e2e-groups", type=int, default=32, help="unit groups pipelined over streams in the e2e run")
     ap.add_argument("--e2e-streams", type=int, default=4, help="streams (each with a workspace) in the e2e run")
     ap.add_argument("--units", type=int, default=None, help="use only the first U units of the batch (profiling)")
+    ap.add_argument("--no-others", action="store_true", help="skip the other workloads' lines")
+    ap.add_argument("--other-units", type=int, default=128, help="units of each other workload measured")
     return ap.parse_args()
 
 
@@ -68,7 +70,7 @@ class ClockSampler:
         self.proc = None
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-lms", "200", "-i", gpu_id], stdout=subprocess.PIPE,
+                                          "-lms", "50", "-i", gpu_id], stdout=subprocess.PIPE,
                                          stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -112,25 +114,18 @@ def gpu_id_for_smi(dev_index: int) -> str:
         return vis.split(",")[dev_index] if vis else str(dev_index)
 
 
-def blas_threads() -> int:
-    try:
-        import numpy as np
-        from threadpoolctl import threadpool_info
-        np.dot(np.ones((64, 64)), np.ones((64, 64)))
-        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
-        return int(max(n)) if n else 1
-    except Exception:
-        return os.cpu_count() or 1
-
-
 def oracle_round_trip_seconds(x_np, w, bits, n_units=1):
-    """Time the CPU oracle (as it stands) compressing and decompressing n_units unit(s)."""
+    """Time the CPU oracle (as it stands) compressing and decompressing n_units unit(s), on one
+    host thread: its NumPy calls are held to a single BLAS/OpenMP thread, so the core count the
+    baseline reports (1) is the one it used."""
+    from threadpoolctl import threadpool_limits
     from oracle import tactkv_oracle as O
-    t = time.perf_counter()
-    for _ in range(n_units):
-        p = O.compress_unit(x_np, w.S, w.H, w.W, x_np.shape[1], x_np.shape[2], bits)
-        O.decompress_unit(p)
-    return time.perf_counter() - t
+    with threadpool_limits(limits=1):
+        t = time.perf_counter()
+        for _ in range(n_units):
+            p = O.compress_unit(x_np, w.S, w.H, w.W, x_np.shape[1], x_np.shape[2], bits)
+            O.decompress_unit(p)
+        return time.perf_counter() - t
 
 
 # ---------------------------------------------------------------------- multi-rank host logic ---
@@ -156,39 +151,44 @@ def job_gbs(world: int, bytes_per_rank: int, ms: float) -> float:
 
 # ---------------------------------------------------------------------------- reference arm ---
 def run_reference(args, w, bits, rank):
-    """The base contract's reference arm for this codec: the CPU oracle on the host cores."""
+    """The base contract's reference arm for this codec: the CPU oracle, as it stands, on the host.
+    Each step compresses and decompresses one whole unit of the workload (units taken in turn), or,
+    when K + W whole units would not end within about four minutes, the first channels of one."""
     if rank != 0:
         return
     import numpy as np
     import torch
-    from dct_transform_coding_b200.workloads import make_unit, unit_seed
-    sample_heads, D = 1, 32                                    # calibrate on 32 channels
-    seed = unit_seed(w, 0, 0, 0)
+    from dct_transform_coding_b200.workloads import make_workload_unit
 
-    def sample(hd):
-        x = make_unit(w.S, w.H, w.W, 1, hd, rho=w.rho, nu=w.nu, scale=w.scale, dtype=w.dtype, seed=seed)
+    all_units = list(w.units())
+
+    def unit(k, channels=None):
+        x = make_workload_unit(w, *all_units[k % len(all_units)])
+        if channels is not None:
+            x = x.reshape(x.shape[0], -1)[:, :channels].reshape(x.shape[0], 1, channels)
         return x.float().numpy().astype(np.float64) if w.dtype == torch.float32 else x.float().numpy()
 
-    t32 = oracle_round_trip_seconds(sample(D), w, bits)
-    budget = 120.0 / max(1, args.steps + args.warmup)
-    hd = 32
-    while hd * 2 <= w.channels and t32 * (hd * 2) / 32 <= budget:
-        hd *= 2
-    x = sample(hd)
-    for _ in range(args.warmup):
-        oracle_round_trip_seconds(x, w, bits)
-    times = [oracle_round_trip_seconds(x, w, bits) for _ in range(args.steps)]
+    t_unit = oracle_round_trip_seconds(unit(0), w, bits)
+    total = args.steps + args.warmup
+    channels = None
+    if t_unit * total > 240.0:
+        channels = 32
+        while channels * 2 <= w.channels and t_unit * total * channels * 2 / w.channels <= 240.0:
+            channels *= 2
+    for k in range(args.warmup):
+        oracle_round_trip_seconds(unit(k, channels), w, bits)
+    times = [oracle_round_trip_seconds(unit(args.warmup + k, channels), w, bits) for k in range(args.steps)]
     step = statistics.mean(times)
-    nbytes = w.tokens * hd * 2
+    nbytes = w.tokens * (channels or w.channels) * 2
     value = nbytes / step / 1e9
-    cores = blas_threads()
-    desc = (f"1 unit of {w.name} (sequence 0, layer 0, K) restricted to its first {hd} of {w.channels} "
-            f"channels ({w.S}x{w.H}x{w.W} grid, {bits} bit/elem), compress + decompress per step")
+    what = "one whole unit" if channels is None else f"the first {channels} of the {w.channels} channels of one unit"
+    desc = (f"{what} of {w.name} per step (units in turn from (sequence 0, layer 0, K); {w.S}x{w.H}x{w.W} grid, "
+            f"{bits} bit/elem), compress + decompress by the fp64 NumPy oracle on one host thread")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_of(w, bits),
-            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -251,12 +251,6 @@ def main():
         check(T.tactkv_decompress(du, ws.data_ptr(), ws.numel(), sp), "decompress")
         return n + T.tactkv_last_launches()
 
-    def profiled_step(cu_p, du_p, ev_c, ev_d):
-        check(T.tactkv_compress_profiled(cu_p, ws.data_ptr(), ws.numel(), sp, [e.cuda_event for e in ev_c]),
-              "compress")
-        check(T.tactkv_decompress_profiled(du_p, ws.data_ptr(), ws.numel(), sp, [e.cuda_event for e in ev_d]),
-              "decompress")
-
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
@@ -285,81 +279,175 @@ def main():
         elapsed_ms = max_over_ranks(elapsed_ms, dist, dev)
     ms_step = elapsed_ms / args.steps
 
-    # per-kernel attribution: separate profiled steps (the profiled entry points record an event at
-    # every kernel boundary); not part of the timed region above
-    # a call records the stage events again in every wave, so the profiled steps run one wave's
-    # worth of units (at most 256) and the times are scaled to the whole batch
-    n_sub = min(U, 256)
-    cu_p, du_p = cu[:n_sub], du[:n_sub]
-    scale = U / n_sub
-    n_prof = min(5, args.steps)
-    evs_c = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_prof)]
-    evs_d = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_prof)]
-    for e in [e for es in evs_c + evs_d for e in es]:
-        e.record(stream)   # torch creates the CUDA event on its first record
-    for k in range(n_prof):
-        profiled_step(cu_p, du_p, evs_c[k], evs_d[k])
-    torch.cuda.synchronize(dev)
-    # stages: the S and H/W passes alternate per group of units, so they are timed together
-    names_c = ["fdct_s+fdct_hw", "reduce_var+allocate", "pack"]
-    names_d = ["decode_index", "idct_hw+idct_s"]
-    kern = {n: scale * statistics.mean(evs_c[k][i].elapsed_time(evs_c[k][i + 1]) for k in range(n_prof))
-            for i, n in enumerate(names_c)}
-    kern.update({n: scale * statistics.mean(evs_d[k][i].elapsed_time(evs_d[k][i + 1]) for k in range(n_prof))
-                 for i, n in enumerate(names_d)})
-    ms_c = scale * statistics.mean(evs_c[k][0].elapsed_time(evs_c[k][3]) for k in range(n_prof))
-    ms_d = scale * statistics.mean(evs_d[k][0].elapsed_time(evs_d[k][2]) for k in range(n_prof))
+    prof = profile_stages(T, cu, du, ws, stream, U, min(5, args.steps))
 
     # bytes: payload sizes actually written (header field total_bytes)
     hdr = payload[:, :64].cpu().numpy()
     pay_bytes = int(sum(int.from_bytes(bytes(h[48:56]), "little") for h in hdr))
     in_bytes = U * Tk * heads * D * 2
-    alg_c = in_bytes + pay_bytes                     # read bf16 K/V, write payloads
-    alg_d = pay_bytes + in_bytes                     # read payloads, write bf16 K/V
     peak, peak_kind = measured_peaks()
     value = job_gbs(world, in_bytes, ms_step)
     if args.units:
         w = dataclasses.replace(w, sequences=1, layers=U, kv=(0,))   # describe what actually ran
-    achieved = (alg_c + alg_d) / (ms_step * 1e-3) / 1e9
-    dominant = max(kern, key=kern.get)
-    kernels = {n: {"ms": round(kern[n], 4), "share": round(kern[n] / (ms_c + ms_d), 4)} for n in kern}
-
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", f"{w.name}_step_dram_bytes.txt")
-    if os.path.exists(tpath):
-        for line in open(tpath):
-            if line.startswith("dram_bytes_per_step:"):
-                traffic = int(line.split(":")[1])
+    roofline = stage_roofline(prof, in_bytes, pay_bytes, U * w.tokens, ms_step, peak, peak_kind, w.name)
 
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "vs_baseline": None, "dtype": "f32", "io_dtype": "bf16", "data": "synthetic",
         "config": config_of(w, bits),
         # compress / decompress alone, from the profiled (one stream, kernel after kernel) steps
-        "compress_gbs": round(in_bytes / (ms_c * 1e-3) / 1e9, 2),
-        "decompress_gbs": round(in_bytes / (ms_d * 1e-3) / 1e9, 2),
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "kernel": "compress+decompress step",
-                     "algorithmic_bytes_per_step": alg_c + alg_d, "peak_kind": peak_kind,
-                     "compress_frac": round(alg_c / (ms_c * 1e-3) / 1e9 / peak, 4),
-                     "decompress_frac": round(alg_d / (ms_d * 1e-3) / 1e9 / peak, 4),
-                     "dominant_kernel": dominant},
-        "kernels": kernels,
+        "compress_gbs": round(in_bytes / (prof["compress_ms"] * 1e-3) / 1e9, 2),
+        "decompress_gbs": round(in_bytes / (prof["decompress_ms"] * 1e-3) / 1e9, 2),
+        "roofline": roofline,
+        "kernels": {n: {"ms": round(v, 4), "share": round(v / (prof["compress_ms"] + prof["decompress_ms"]), 4)}
+                    for n, v in prof["stages"].items()},
         "gpu_launches": launches,
         "clocks": clocks,
     }
 
     if not args.no_e2e:
         result["e2e"] = e2e_run(args, T, x, payload, out, cu, du, ws, stream, world)
+    del x, out, payload, ws
+    torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(w, bits, x)
+        result["cpu_baseline"] = cpu_baseline(wr, bits, args.units)
+    if rank == 0 and world == 1 and not args.no_others and not args.units:
+        result["other_workloads"] = other_workloads(T, args, w.name, dev, peak, peak_kind)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(result), flush=True)
+
+
+STAGES_C = ["forward", "allocate", "pack"]          # compress: DCTs with energies, allocation, packing
+STAGES_D = ["decode_index", "inverse"]              # decompress: payload index, decode + inverse DCTs
+
+
+def profile_stages(T, cu, du, ws, stream, U, n_prof):
+    """Per-stage device times of one step, from the profiled entry points (an event at every stage
+    boundary), outside the timed region.  A call records the stage events again in every wave, so
+    the profiled steps run one wave's worth of units (at most 256), scaled to the whole batch."""
+    import torch
+    n_sub = min(U, 256)
+    cu_p, du_p = cu[:n_sub], du[:n_sub]
+    scale = U / n_sub
+    evs_c = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_prof)]
+    evs_d = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_prof)]
+    for e in [e for es in evs_c + evs_d for e in es]:
+        e.record(stream)   # torch creates the CUDA event on its first record
+    sp = int(stream.cuda_stream)
+    for k in range(n_prof):
+        st = T.tactkv_compress_profiled(cu_p, ws.data_ptr(), ws.numel(), sp, [e.cuda_event for e in evs_c[k]])
+        if st != T.TACTKV_OK:
+            raise T.TactkvError(st, "compress")
+        st = T.tactkv_decompress_profiled(du_p, ws.data_ptr(), ws.numel(), sp, [e.cuda_event for e in evs_d[k]])
+        if st != T.TACTKV_OK:
+            raise T.TactkvError(st, "decompress")
+    torch.cuda.synchronize()
+    mean = statistics.mean
+    stages = {n: scale * mean(evs_c[k][i].elapsed_time(evs_c[k][i + 1]) for k in range(n_prof))
+              for i, n in enumerate(STAGES_C)}
+    stages.update({n: scale * mean(evs_d[k][i].elapsed_time(evs_d[k][i + 1]) for k in range(n_prof))
+                   for i, n in enumerate(STAGES_D)})
+    return {"stages": stages,
+            "compress_ms": scale * mean(evs_c[k][0].elapsed_time(evs_c[k][3]) for k in range(n_prof)),
+            "decompress_ms": scale * mean(evs_d[k][0].elapsed_time(evs_d[k][2]) for k in range(n_prof))}
+
+
+def stage_roofline(prof, in_bytes, pay_bytes, bins_x_units, ms_step, peak, peak_kind, name):
+    """Roofline of the dominant stage: its algorithmic bytes (what the method must move through HBM
+    in that stage) over its measured time.  forward reads the bf16 input; allocate writes the gains
+    and bit widths (5 B per bin) and the headers; pack writes the codes; decode_index reads gains
+    and widths; inverse reads the codes and writes the bf16 output.  The whole step's fraction
+    (both directions' algorithmic bytes over the timed step) is reported beside it."""
+    meta = 5 * bins_x_units
+    codes = max(0, pay_bytes - meta)
+    alg = {"forward": in_bytes, "allocate": meta, "pack": codes, "decode_index": meta, "inverse": codes + in_bytes}
+    stages = prof["stages"]
+    dom = max(stages, key=stages.get)
+    achieved = alg[dom] / (stages[dom] * 1e-3) / 1e9
+    step_achieved = 2 * (in_bytes + pay_bytes) / (ms_step * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": dram_traffic(name, dom),
+            "kernel": dom, "kernel_ms": round(stages[dom], 4), "algorithmic_bytes": alg[dom],
+            "peak_kind": peak_kind,
+            "step_achieved": round(step_achieved, 1), "step_frac": round(step_achieved / peak, 4),
+            "compress_frac": round((in_bytes + pay_bytes) / (prof["compress_ms"] * 1e-3) / 1e9 / peak, 4),
+            "decompress_frac": round((in_bytes + pay_bytes) / (prof["decompress_ms"] * 1e-3) / 1e9 / peak, 4)}
+
+
+def dram_traffic(name, stage):
+    """DRAM bytes (read + write) of one launch of the stage's kernel on this workload, from the ncu
+    summary in profiles/ (lines `stage <name>: <bytes>`), or None when none was taken at this build."""
+    path = os.path.join(ROOT, "profiles", f"{name}_dram_bytes.txt")
+    if not os.path.exists(path):
+        return None
+    for line in open(path):
+        if line.startswith(f"stage {stage}:"):
+            return int(line.split(":")[1])
+    return None
+
+
+def other_workloads(T, args, main_name, dev, peak, peak_kind):
+    """The other benchmark workloads in the same run: one wave of up to --other-units units of each
+    (the codec's cost is per unit, so a wave stands for the batch), 10 timed steps, no e2e."""
+    import torch
+    from dct_transform_coding_b200.workloads import WORKLOADS, make_batch
+    out = {}
+    for name, bits_list in (("tiny", None), ("med4b_b8", (1, 2, 4)), ("med32b", None), ("video", None)):
+        if name == main_name:
+            continue
+        w = WORKLOADS[name]
+        U = min(w.n_units, args.other_units)
+        x = make_batch(w, device=dev, units=list(range(U)))
+        all_units = list(w.units())[:U]
+        layers, kvs = [u[1] for u in all_units], [u[2] for u in all_units]
+        for bits in (bits_list or w.bits):
+            flags = T.TACTKV_FP32_IO if x.dtype == torch.float32 else 0
+            cap = T.payload_capacity(w.S, w.H, w.W, w.heads, w.head_dim, bits, flags)
+            payload = torch.zeros((U, (cap + 15) // 16 * 16), dtype=torch.uint8, device=dev)
+            y = torch.empty_like(x)
+            cu = T.make_units(x, w.S, w.H, w.W, bits, heads=w.heads, head_dim=w.head_dim, payload=payload,
+                              layers=layers, kvs=kvs, flags=flags)
+            du = T.make_units(None, w.S, w.H, w.W, bits, heads=w.heads, head_dim=w.head_dim, payload=payload,
+                              out=y, layers=layers, kvs=kvs, n_units=U, flags=flags)
+            ws = T.alloc_workspace(cu, dev)
+            stream = torch.cuda.current_stream(dev)
+            sp = int(stream.cuda_stream)
+
+            def step():
+                T.tactkv_compress(cu, ws.data_ptr(), ws.numel(), sp)
+                T.tactkv_decompress(du, ws.data_ptr(), ws.numel(), sp)
+
+            for _ in range(3):
+                step()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize(dev)
+            a.record(stream)
+            for _ in range(10):
+                step()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            st = T.tactkv_device_status(ws.data_ptr(), ws.numel(), sp)
+            if st != T.TACTKV_OK:
+                raise T.TactkvError(st, f"{name} device status")
+            ms = a.elapsed_time(b) / 10
+            prof = profile_stages(T, cu, du, ws, stream, U, 3)
+            hdr = payload[:, :64].cpu().numpy()
+            pay_bytes = int(sum(int.from_bytes(bytes(h[48:56]), "little") for h in hdr))
+            in_bytes = x.numel() * 2          # the metric's unit: bf16 bytes of K/V
+            rl = stage_roofline(prof, in_bytes, pay_bytes, U * w.tokens, ms, peak, peak_kind, name)
+            out[f"{name}@{bits}"] = {"units": U, "ms_per_step": round(ms, 4),
+                                     "value": round(in_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                                     "step_frac": rl["step_frac"], "dominant": rl["kernel"],
+                                     "dominant_frac": rl["frac"],
+                                     "stages_ms": {k: round(v, 4) for k, v in prof["stages"].items()}}
+            del payload, y, ws
+        del x
+        torch.cuda.empty_cache()
+    return out
 
 
 def e2e_run(args, T, x, payload, out, cu, du, ws, stream, world):
@@ -421,24 +509,27 @@ def e2e_run(args, T, x, payload, out, cu, du, ws, stream, world):
             "ms_per_step": round(ms, 3), "groups": len(bounds), "streams": len(streams)}
 
 
-def cpu_baseline(w, bits, x):
-    """The oracle as it stands on the host cores, on whole units of the same batch (bounded)."""
+def cpu_baseline(w, bits, n_units=None):
+    """The oracle as it stands, on one host thread, on whole units of the same workload (units
+    taken in order from the first, up to about 10 s of work)."""
     import numpy as np
-    cores = blas_threads()
-    xs = x[0].float().cpu().numpy()
-    t = oracle_round_trip_seconds(xs, w, bits)
-    n = 1
-    if t < 10.0:
-        extra = min(2, int(10.0 // max(t, 1e-3)))
-        if extra:
-            t += sum(oracle_round_trip_seconds(x[1 + i].float().cpu().numpy(), w, bits) for i in range(extra))
-            n += extra
-    nbytes = n * w.elements_per_unit * 2
-    del np
-    return {"value": round(nbytes / t / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"{n} whole unit(s) of {w.name} (layers 0.., K/V), compress + decompress, fp64 NumPy",
-            "seconds": round(t, 2)}
+    import torch
+    from dct_transform_coding_b200.workloads import make_workload_unit
+    all_units = list(w.units())[:n_units or None]
 
+    def unit(k):
+        x = make_workload_unit(w, *all_units[k % len(all_units)])
+        return x.float().numpy().astype(np.float64) if w.dtype == torch.float32 else x.float().numpy()
+
+    t = oracle_round_trip_seconds(unit(0), w, bits)
+    n = 1
+    while t < 10.0 and n < 3:
+        t += oracle_round_trip_seconds(unit(n), w, bits)
+        n += 1
+    nbytes = n * w.elements_per_unit * 2
+    return {"value": round(nbytes / t / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} whole unit(s) of {w.name} (units 0..{n - 1}), compress + decompress, fp64 NumPy "
+                      f"oracle on one host thread", "seconds": round(t, 2)}
 
 if __name__ == "__main__":
     main()

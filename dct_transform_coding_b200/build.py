@@ -52,7 +52,7 @@ def _compile(name, src, defs, ptxas_info):
 
 
 def build(verbose: bool = False, ptxas_info: bool = False, jobs: int = 0) -> str:
-    for gen in ("gen_dct.py", "gen_tables.py"):
+    for gen in ("gen_dct.py", "gen_tables.py", "gen_mma_tables.py"):
         subprocess.run([sys.executable, os.path.join(CSRC, gen)], check=True,
                        stdout=None if verbose else subprocess.DEVNULL)
     os.makedirs(OBJ, exist_ok=True)

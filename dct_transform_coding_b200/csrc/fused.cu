@@ -15,6 +15,13 @@
 // kernels.
 #include "axis_s.cuh"
 #include "axis_hw.cuh"
+#include "tc.cuh"
+#include "dct_limbs.inc"
+
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
 
 #ifndef TACTKV_FUSED_S
 #error "TACTKV_FUSED_S must be defined"
@@ -89,6 +96,159 @@ __global__ void __launch_bounds__(kFusedThreads, 3) fdct3_kernel(const __grid_co
   if (ks0 < ks1) fdct_hw_slabs<16, 16, HX, WX, true, NX>(g, Y, partial, u, chunk, ks0, ks1, smem);
 }
 
+// ------------------------------------------------------------- S pass on the tensor cores ---
+// The DCT along S of a tile of 4 grid cells x 32 channels is the product
+//     Y[(cell, c), k] = sum_s x[(cell, c), s] * C[k, s]
+// with M = 128 rows (cell, c), N = S columns k and K = S.  x is exact in bf16; C is carried as
+// three bf16 limbs (hi + mid + lo, fp32 accuracy), accumulated into one fp32 TMEM accumulator.
+//   A = the input tile, loaded by TMA as [cell][s][32 channels] bf16 with 64-byte swizzle: MN-major,
+//       32 channels of one cell per 64-byte row, 8 rows of consecutive s per 512-byte atom;
+//   B = a limb of C, [k][s] with s contiguous: K-major with 128-byte swizzle (rows padded to 64 s).
+// Thread (warp w, lane l) then reads row 32 (w % 4) + l (cell w % 4, channel l) of the tile, half
+// (w / 4) of its S columns, and stores them to Y[k][cell][c]: 128 contiguous bytes per warp store.
+constexpr int kTcCells = 4;               // grid cells per tile (M = 128)
+
+template <int L>
+struct TcS {
+  static_assert(L == 16 || L == 32 || L == 64, "S of the tensor-core pass");
+  static constexpr int kABytes = kTcCells * L * 64;      // one input tile
+  static constexpr int kBBytes = L * 128;                // one limb of C, rows padded to 128 bytes
+  static constexpr int kSmem = 3 * kBBytes + 2 * kABytes + 1024;   // + alignment slack
+  static constexpr int kCols = L < 32 ? 32 : L;          // TMEM columns (power of two >= 32)
+  static constexpr int kHalf = L / 2;                    // columns read per thread
+};
+
+template <int L>
+__device__ __forceinline__ const uint16_t* dct_limb_fwd() {
+  if constexpr (L == 16) return &kDctLimbFwd16[0][0][0];
+  else if constexpr (L == 32) return &kDctLimbFwd32[0][0][0];
+  else return &kDctLimbFwd64[0][0][0];
+}
+
+// S pass of one (unit u, chunk) on this CTA's tiles t = r, r + kCluster, ... into Y.  Returns
+// false (and records TACTKV_TIMEOUT) if a copy or an MMA did not complete; the caller still takes
+// part in every barrier of the cluster.  Called by every thread of the CTA.
+template <int L, int HWX>
+__device__ bool fdct_s_tc(const Geom& g, int u, int chunk, int r, const CUtensorMap* tmap, float* __restrict__ Y,
+                          unsigned char* smem, uint64_t* bars, uint32_t* tmem_slot, int nx, unsigned int* status) {
+  using P = TcS<L>;
+  constexpr int kTiles = (HWX + kTcCells - 1) / kTcCells;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c0 = chunk * kChunk, head = c0 / g.head_dim, d0 = c0 - head * g.head_dim;
+  const int uw = u - g.unit0;   // the tensor map's unit coordinate: the unit's place in the wave
+  unsigned char* sB = smem;
+  unsigned char* sA = smem + 3 * P::kBBytes;
+  uint64_t* tma_bar = bars;       // [2]
+  uint64_t* mma_bar = bars + 2;
+  const int mine = r < kTiles ? (kTiles - r + kCluster - 1) / kCluster : 0;
+
+  // B: the three limbs of C, swizzled (16-byte chunk j of row k at chunk j ^ (k & 7))
+  const uint16_t* tab = dct_limb_fwd<L>();
+  for (int e = tid; e < 3 * L * 8; e += blockDim.x) {
+    const int l = e / (L * 8), rem = e - l * (L * 8), k = rem >> 3, j = rem & 7;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (j * 8 < L) v = *reinterpret_cast<const uint4*>(tab + ((size_t)l * L + k) * L + j * 8);
+    *reinterpret_cast<uint4*>(sB + l * P::kBBytes + k * 128 + ((j ^ (k & 7)) << 4)) = v;
+  }
+  tc::fence_proxy_async();
+  if (tid == 0) {
+    tc::prefetch_tmap(tmap);
+    tc::mbar_init(&tma_bar[0], 1);
+    tc::mbar_init(&tma_bar[1], 1);
+    tc::mbar_init(mma_bar, 1);
+    tc::fence_mbar_init();
+  }
+  if (warp == 0) tc::tmem_alloc(tmem_slot, P::kCols);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  if (tid == 0)
+    for (int j = 0; j < 2 && j < mine; ++j) {
+      tc::mbar_expect_tx(&tma_bar[j], P::kABytes);
+      tc::tma_load_5d(sA + j * P::kABytes, tmap, &tma_bar[j], d0, head, 0, (r + kCluster * j) * kTcCells, uw);
+    }
+  constexpr uint32_t kIdesc = tc::idesc_bf16(128, L, true);
+  bool ok = true;
+  for (int j = 0; j < mine; ++j) {
+    const int b = j & 1, t = r + kCluster * j;
+    bool ok_t = true;
+    if (tid == 0) {
+      ok_t = tc::mbar_wait(&tma_bar[b], (j >> 1) & 1);
+      if (ok_t) {
+        tc::fence_after_sync();
+        const uint32_t a0 = tc::smem_u32(sA + b * P::kABytes), b0 = tc::smem_u32(sB);
+        bool acc = false;
+#pragma unroll
+        for (int l = 0; l < 3; ++l)
+#pragma unroll
+          for (int ks = 0; ks < L / 16; ++ks) {
+            const uint64_t da = tc::smem_desc(a0 + ks * 1024, L * 64, 512, 4);
+            const uint64_t db = tc::smem_desc(b0 + l * P::kBBytes + ks * 32, 16, 1024, 2);
+            tc::mma_bf16(tmem, da, db, kIdesc, acc);
+            acc = true;
+          }
+        tc::mma_commit(mma_bar);
+      }
+    }
+    ok_t = __syncthreads_and(ok_t) != 0;
+    if (ok_t) ok_t = __syncthreads_and(tc::mbar_wait(mma_bar, j & 1)) != 0;
+    if (!ok_t) {
+      // give the copies and MMAs still in flight a bounded time to land before the shared and
+      // tensor memory they target is released
+      if (tid == 0) {
+        for (int jj = j; jj < j + 2 && jj < mine; ++jj) tc::mbar_wait(&tma_bar[jj & 1], (jj >> 1) & 1);
+        tc::mbar_wait(mma_bar, j & 1);
+      }
+      __syncthreads();
+      ok = false;
+      break;
+    }
+    tc::fence_after_sync();
+    // the tile's shared memory is free again: load the tile after next into it
+    if (tid == 0 && j + 2 < mine) {
+      tc::mbar_expect_tx(&tma_bar[b], P::kABytes);
+      tc::tma_load_5d(sA + b * P::kABytes, tmap, &tma_bar[b], d0, head, 0, (t + 2 * kCluster) * kTcCells, uw);
+    }
+    const int q = warp & 3, half = warp >> 2, cell = t * kTcCells + q;
+    float v[P::kHalf];
+    tc::tmem_ld<P::kHalf>(tmem + ((uint32_t)(32 * q) << 16) + half * P::kHalf, v);
+    tc::tmem_ld_wait();
+    if (cell < HWX) {
+      float* yo = Y + (((size_t)u * L + half * P::kHalf) * HWX + cell) * nx + c0 + lane;
+#pragma unroll
+      for (int k = 0; k < P::kHalf; ++k) yo[(size_t)k * HWX * nx] = v[k];
+    }
+    tc::fence_before_sync();
+    __syncthreads();   // every thread has read the accumulator before the next tile's MMAs
+  }
+  if (!ok && tid == 0) atomicCAS(status, 0u, (unsigned int)TACTKV_TIMEOUT);
+  tc::fence_after_sync();
+  if (warp == 0) tc::tmem_free(tmem, P::kCols);
+  return ok;
+}
+
+// The fused forward kernel with the S pass on the tensor cores (bf16 input described by tmap).
+template <int L, int HX, int WX, int NX>
+__global__ void __launch_bounds__(kFusedThreads, 3) fdct3_tc_kernel(const __grid_constant__ Geom g,
+                                                                    const __grid_constant__ UnitList ul,
+                                                                    float* __restrict__ Y, float* __restrict__ partial,
+                                                                    const __grid_constant__ CUtensorMap tmap,
+                                                                    unsigned int* status) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  __shared__ __align__(8) uint64_t s_bars[3];
+  __shared__ uint32_t s_tmem;
+  unsigned char* smem =
+      smem_raw + ((1024 - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);   // 1024-byte aligned (swizzle atoms)
+  const int r = blockIdx.x, chunk = blockIdx.y, u = g.unit0 + blockIdx.z;
+  const bool ok = fdct_s_tc<L, HX * WX>(g, u, chunk, r, &tmap, Y, smem, s_bars, &s_tmem, NX ? NX : g.n, status);
+  cluster_barrier();   // the chunk's Y is complete
+  if (!ok) return;     // (after the cluster barrier: no CTA of the cluster waits for this one)
+  constexpr int spc = (L + kCluster - 1) / kCluster;
+  const int ks0 = r * spc, ks1 = min(L, ks0 + spc);
+  if (ks0 < ks1) fdct_hw_slabs<16, 16, HX, WX, true, NX>(g, Y, partial, u, chunk, ks0, ks1, smem);
+}
+
 template <class K, class... Args>
 cudaError_t launch_cluster(K kernel, const Geom& g, int nu, size_t smem, cudaStream_t st, Args... args) {
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -108,13 +268,66 @@ cudaError_t launch_cluster(K kernel, const Geom& g, int nu, size_t smem, cudaStr
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
+// Tensor map of the wave's bf16 inputs for the tensor-core S pass: 5-D (d, head, s, cell, unit),
+// box (32, 1, S, 4 cells, 1) with 64-byte swizzle, so that a box lands as [cell][s][32 channels].
+// Needs head_dim a multiple of 32 (a chunk inside one head), 16-byte aligned pointers and
+// strides, and the wave's units equally spaced in memory with equal strides (one map for all);
+// false otherwise (the caller then uses the cp.async S pass).
+bool make_input_map(const Geom& g, const UnitList& ul, int nu, CUtensorMap* map) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  if (!encode || (g.flags & TACTKV_FP32_IO) || g.head_dim % kChunk != 0) return false;
+  const UnitDev& a = ul.u[g.unit0];
+  const long long tok = a.tok_stride, hs = a.head_stride;
+  if (tok * 2 % 16 || hs * 2 % 16 || reinterpret_cast<uintptr_t>(a.in) % 16) return false;
+  long long ustride = 16;
+  if (nu > 1) ustride = static_cast<const char*>(ul.u[g.unit0 + 1].in) - static_cast<const char*>(a.in);
+  if (ustride <= 0 || ustride % 16) return false;
+  for (int i = 1; i < nu; ++i) {
+    const UnitDev& b = ul.u[g.unit0 + i];
+    if (b.tok_stride != tok || b.head_stride != hs ||
+        static_cast<const char*>(b.in) - static_cast<const char*>(a.in) != (long long)i * ustride)
+      return false;
+  }
+  const cuuint64_t dims[5] = {(cuuint64_t)g.head_dim, (cuuint64_t)g.heads, (cuuint64_t)g.S, (cuuint64_t)g.HW,
+                              (cuuint64_t)nu};
+  const cuuint64_t strides[4] = {(cuuint64_t)(hs * 2), (cuuint64_t)(g.HW * tok * 2), (cuuint64_t)(tok * 2),
+                                 (cuuint64_t)ustride};
+  const cuuint32_t box[5] = {(cuuint32_t)kChunk, 1u, (cuuint32_t)g.S, (cuuint32_t)kTcCells, 1u};
+  const cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(a.in), dims, strides, box,
+                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <int HX, int WX>
-cudaError_t launch_grid(const Geom& g, const UnitList& ul, int nu, float* buf, float* partial, cudaStream_t st) {
+cudaError_t launch_grid(const Geom& g, const UnitList& ul, int nu, float* buf, float* partial, unsigned int* status,
+                        cudaStream_t st) {
   constexpr int L = TACTKV_FUSED_S;
   const HwLayout Ls = hw_layout(HX, WX, kLayStats);
   const size_t regions[] = {Ls.tile, Ls.sbuf, Ls.meta, Ls.lv, Ls.tile_bytes};
   for (size_t x : regions)
     if (x % 16) return cudaErrorMisalignedAddress;   // never launch a misaligned layout
+#if TACTKV_FUSED_S >= 16
+  CUtensorMap map;
+  if (!tc_s_pass_disabled() && make_input_map(g, ul, nu, &map)) {
+    const size_t smem = std::max<size_t>(TcS<L>::kSmem, Ls.total + 1024);
+    if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
+    if (g.n == 1024)
+      return launch_cluster(fdct3_tc_kernel<L, HX, WX, 1024>, g, nu, smem, st, g, ul, buf, partial, map, status);
+    if (g.n == 512)
+      return launch_cluster(fdct3_tc_kernel<L, HX, WX, 512>, g, nu, smem, st, g, ul, buf, partial, map, status);
+    return launch_cluster(fdct3_tc_kernel<L, HX, WX, 0>, g, nu, smem, st, g, ul, buf, partial, map, status);
+  }
+#endif
   int nbuf = 1;
   const size_t smem = fused_fwd_smem<L>(HX, WX, (g.flags & TACTKV_FP32_IO) != 0, &nbuf);
   if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
@@ -131,11 +344,11 @@ cudaError_t launch_grid(const Geom& g, const UnitList& ul, int nu, float* buf, f
 // Fused forward transforms of one wave for the grids above (g.S == TACTKV_FUSED_S):
 // x -> X in buf, energies in partial; cudaErrorNotSupported for any other grid.
 cudaError_t TACTKV_CAT(launch_fused_, TACTKV_FUSED_S)(const Geom& g, const UnitList& ul, int nu, float* buf,
-                                                      float* partial, cudaStream_t st) {
+                                                      float* partial, unsigned int* status, cudaStream_t st) {
   if (g.S != TACTKV_FUSED_S) return cudaErrorNotSupported;
-  if (g.H == 16 && g.W == 16) return launch_grid<16, 16>(g, ul, nu, buf, partial, st);
-  if (g.H == 14 && g.W == 14) return launch_grid<14, 14>(g, ul, nu, buf, partial, st);
-  if (g.H == 8 && g.W == 8) return launch_grid<8, 8>(g, ul, nu, buf, partial, st);
+  if (g.H == 16 && g.W == 16) return launch_grid<16, 16>(g, ul, nu, buf, partial, status, st);
+  if (g.H == 14 && g.W == 14) return launch_grid<14, 14>(g, ul, nu, buf, partial, status, st);
+  if (g.H == 8 && g.W == 8) return launch_grid<8, 8>(g, ul, nu, buf, partial, status, st);
   return cudaErrorNotSupported;
 }
 

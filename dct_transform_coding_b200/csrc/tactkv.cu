@@ -9,6 +9,7 @@
 // wave runs the decoding index (allocate.cu: header checks, slab offsets), the inverse H/W pass
 // (dequantize + inverse DCT along W and H) and the inverse DCT along S.
 #include <algorithm>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -38,7 +39,7 @@ cudaError_t launch_axis_s(int cls, bool inverse, const Geom& g, const UnitList& 
 }
 
 #define TACTKV_DECL_FUSED(s) \
-  cudaError_t launch_fused_##s(const Geom&, const UnitList&, int, float*, float*, cudaStream_t);
+  cudaError_t launch_fused_##s(const Geom&, const UnitList&, int, float*, float*, unsigned int*, cudaStream_t);
 TACTKV_DECL_FUSED(8)
 TACTKV_DECL_FUSED(16)
 TACTKV_DECL_FUSED(32)
@@ -51,12 +52,13 @@ bool fused_grid(const Geom& g) {
   const bool s = g.S == 8 || g.S == 16 || g.S == 32 || g.S == 64;
   return s && ((g.H == 16 && g.W == 16) || (g.H == 14 && g.W == 14) || (g.H == 8 && g.W == 8));
 }
-cudaError_t launch_fused(const Geom& g, const UnitList& ul, int nu, float* buf, float* partial, cudaStream_t st) {
+cudaError_t launch_fused(const Geom& g, const UnitList& ul, int nu, float* buf, float* partial, unsigned int* status,
+                         cudaStream_t st) {
   switch (g.S) {
-    case 8: return launch_fused_8(g, ul, nu, buf, partial, st);
-    case 16: return launch_fused_16(g, ul, nu, buf, partial, st);
-    case 32: return launch_fused_32(g, ul, nu, buf, partial, st);
-    case 64: return launch_fused_64(g, ul, nu, buf, partial, st);
+    case 8: return launch_fused_8(g, ul, nu, buf, partial, status, st);
+    case 16: return launch_fused_16(g, ul, nu, buf, partial, status, st);
+    case 32: return launch_fused_32(g, ul, nu, buf, partial, status, st);
+    case 64: return launch_fused_64(g, ul, nu, buf, partial, status, st);
     default: return cudaErrorNotSupported;
   }
 }
@@ -75,6 +77,14 @@ void axis_hw_shape(int hcls, int wcls, const Geom& g, bool inverse, int mode, si
   if (hcls == 16) return axis_hw_shape_16_32(g, inverse, mode, smem, threads);
   if (wcls == 16) return axis_hw_shape_32_16(g, inverse, mode, smem, threads);
   return axis_hw_shape_32_32(g, inverse, mode, smem, threads);
+}
+
+bool tc_s_pass_disabled() {
+  static const bool off = [] {
+    const char* e = getenv("TACTKV_SIMT_S");
+    return e && e[0] == '1';
+  }();
+  return off;
 }
 
 namespace {
@@ -303,7 +313,8 @@ static tactkv_status compress_impl(const tactkv_unit* units, int n_units, void* 
                          mark(0);
                          if (fused_grid(g)) {
                            t_launches += 1;   // fdct3
-                           if (launch_fused(g, ul, nu, w.big, w.partial, st) != cudaSuccess) return TACTKV_CUDA;
+                           if (launch_fused(g, ul, nu, w.big, w.partial, w.status, st) != cudaSuccess)
+                             return TACTKV_CUDA;
                          } else {
                            t_launches += 2;   // fdct_s, fdct_hw
                            if (launch_axis_s(cs, false, g, ul, nu, w.big, st) != cudaSuccess) return TACTKV_CUDA;
@@ -434,6 +445,7 @@ const char* tactkv_status_string(tactkv_status s) {
     case TACTKV_CUDA: return "CUDA error";
     case TACTKV_WORKSPACE: return "workspace missing or too small";
     case TACTKV_SCRATCH_LIMIT: return "unit larger than the fixed scratch of tactkv_compress_noalloc";
+    case TACTKV_TIMEOUT: return "a kernel's bounded wait for a copy or a tensor-core operation expired";
     default: return "unknown status";
   }
 }

@@ -30,6 +30,7 @@ TACTKV_CORRUPT_PAYLOAD = 5
 TACTKV_CUDA = 6
 TACTKV_WORKSPACE = 7
 TACTKV_SCRATCH_LIMIT = 8
+TACTKV_TIMEOUT = 9
 
 TACTKV_NO_QUANT = 1
 TACTKV_FP32_IO = 2

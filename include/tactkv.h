@@ -60,7 +60,9 @@ typedef enum {
   TACTKV_CORRUPT_PAYLOAD = 5,    /* (device status) a payload header or allocation is invalid */
   TACTKV_CUDA = 6,               /* a CUDA launch or copy failed */
   TACTKV_WORKSPACE = 7,          /* workspace null or smaller than one unit needs */
-  TACTKV_SCRATCH_LIMIT = 8       /* a unit needs more scratch than tactkv_compress_noalloc has */
+  TACTKV_SCRATCH_LIMIT = 8,      /* a unit needs more scratch than tactkv_compress_noalloc has */
+  TACTKV_TIMEOUT = 9             /* (device status) a kernel's bounded wait on a tensor-memory copy
+                                    or a tensor-core operation expired; its outputs are undefined */
 } tactkv_status;
 
 /* flags */

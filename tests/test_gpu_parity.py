@@ -255,6 +255,39 @@ def test_full_size_sampled_units(name, bits, pick):
     torch.cuda.empty_cache()
 
 
+# ------------------------------------------------------- tensor-core and CUDA-core S passes ---
+@pytest.mark.parametrize("S,H,W", [(64, 16, 16), (32, 14, 14), (16, 8, 8)])
+def test_tensor_core_and_cuda_core_s_pass_both_match_the_oracle(S, H, W):
+    """The fused forward kernel runs its DCT along S on the tensor cores when one TMA tensor map
+    can describe the whole wave (units evenly spaced in memory), and on the CUDA cores otherwise.
+    The same three units are compressed both ways (the second time listed in reverse memory order,
+    which no single map describes) and both payloads must pass the oracle's acceptance rules."""
+    heads, D = 2, 64
+    x = torch.stack([make_unit(S, H, W, heads, D, rho=(0.9, 0.85, 0.85), nu=4.0, seed=70 + i, device=DEV)
+                     for i in range(3)])
+    pay_tc, y_tc = _round_trip(x, S, H, W, 2, layers=[0, 1, 2], kvs=[0, 0, 0])
+    cap = T.payload_capacity(S, H, W, heads, D, 2)
+    pay_sm = torch.zeros((3, (cap + 15) // 16 * 16), dtype=torch.uint8, device=DEV)
+    y_sm = torch.empty_like(x)
+    cu = T.make_units(x, S, H, W, 2, heads=heads, head_dim=D, payload=pay_sm, layers=[0, 1, 2], kvs=[0, 0, 0])
+    du = T.make_units(None, S, H, W, 2, heads=heads, head_dim=D, payload=pay_sm, out=y_sm, layers=[0, 1, 2],
+                      kvs=[0, 0, 0], n_units=3)
+    cu_rev = (T.tactkv_unit * 3)(*[cu[2 - i] for i in range(3)])
+    ws = T.alloc_workspace(cu, DEV)
+    sp = torch.cuda.current_stream().cuda_stream
+    assert T.tactkv_compress(cu_rev, ws.data_ptr(), ws.numel(), sp) == T.TACTKV_OK
+    assert T.tactkv_decompress(du, ws.data_ptr(), ws.numel(), sp) == T.TACTKV_OK
+    assert T.tactkv_device_status(ws.data_ptr(), ws.numel(), sp) == T.TACTKV_OK
+    torch.cuda.synchronize()
+    for i in range(3):
+        xi = x[i].double().cpu().numpy()
+        for pay, y in ((pay_tc, y_tc), (pay_sm, y_sm)):
+            compare_unit(xi, pay[i].cpu().numpy().tobytes(), y[i].double().cpu().numpy(), S=S, H=H, W=W,
+                         heads=heads, head_dim=D, bits=2, layer=i, kv=0)
+    # same allocation both ways (the code streams may differ only inside the parity band)
+    assert torch.equal(pay_tc[:, :64 + S * H * W], pay_sm[:, :64 + S * H * W])
+
+
 # ------------------------------------------------------------------------------ exact ties ---
 def _gpu_allocation(var, grid, bits):
     S, H, W = grid
