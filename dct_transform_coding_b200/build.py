@@ -33,6 +33,9 @@ UNITS = [
     ("fused_16", "fused.cu", ["-DTACTKV_FUSED_S=16"]),
     ("fused_32", "fused.cu", ["-DTACTKV_FUSED_S=32"]),
     ("fused_64", "fused.cu", ["-DTACTKV_FUSED_S=64"]),
+    ("fused_inv_16", "fused_inv.cu", ["-DTACTKV_FUSED_S=16"]),
+    ("fused_inv_32", "fused_inv.cu", ["-DTACTKV_FUSED_S=32"]),
+    ("fused_inv_64", "fused_inv.cu", ["-DTACTKV_FUSED_S=64"]),
     ("allocate", "allocate.cu", []),
     ("pack", "pack.cu", []),
     ("tactkv", "tactkv.cu", []),

@@ -266,10 +266,15 @@ __device__ __forceinline__ int cp_index(int Wp, int h, int wp) { return (h * Wp 
 // code offset within the slab's words of the two rows' bins) arrive by cp.async, the next slab's
 // meanwhile.  Warp kp decodes rows 2kp and 2kp+1 in registers and runs the inverse DCT along W,
 // writing column pairs; then the inverse DCT along H runs on column pairs, into the fp32 volume V.
-template <int HC, int WC, int HX, int WX, int MODE>
+// PAIRS: instead of fp32 V[u][k_s][cell][c], write the result as bf16 pairs for the tensor-core
+// inverse along S: V_hi[u][k_s][cell pair][c] = (bf16(v[2p]), bf16(v[2p+1])) over V (as
+// __nv_bfloat162) and the remainders V_lo = bf16(v - float(V_hi)) over Vlo (W even).  Together
+// they carry v to about 2^-17 relative.
+template <int HC, int WC, int HX, int WX, int MODE, bool PAIRS = false>
 __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul, float* __restrict__ V,
                                               const uint32_t* __restrict__ index, const uint4* __restrict__ recs, int u,
-                                              int chunk, int ks0, int ks1, unsigned char* smem) {
+                                              int chunk, int ks0, int ks1, unsigned char* smem,
+                                              __nv_bfloat162* __restrict__ Vlo = nullptr) {
   const Dims<HX, WX> D(g);
   constexpr bool raw = MODE == kRaw;
   const HwLayout L = hw_layout(D.H, D.W, kLayDecode);
@@ -370,15 +375,31 @@ __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul,
       for (int h = 0; h < HC; ++h)
         if (h < D.H) xh[h] = tile[cp_index(Wp, h, wp) + lane];
       pencil<HC, HX, true>(xh, D.H);
-      float* v = vunit + ((size_t)ks * D.HW + 2 * wp) * g.n;
-      const bool two = 2 * wp + 1 < D.W;
+      if constexpr (PAIRS) {
+        // pair (cell h*W + 2wp, cell h*W + 2wp + 1) = pair index h*(W/2) + wp
+        const size_t base = ((size_t)u * g.S + ks) * (D.HW / 2) * g.n + chunk * kChunk + lane;
+        __nv_bfloat162* vh = reinterpret_cast<__nv_bfloat162*>(V) + base + (size_t)wp * g.n;
+        __nv_bfloat162* vl = Vlo + base + (size_t)wp * g.n;
 #pragma unroll
-      for (int h = 0; h < HC; ++h)
-        if (h < D.H) {
-          float* cell = v + (size_t)h * D.W * g.n;
-          cell[0] = xh[h].x;
-          if (two) cell[g.n] = xh[h].y;
-        }
+        for (int h = 0; h < HC; ++h)
+          if (h < D.H) {
+            const __nv_bfloat162 hi = __floats2bfloat162_rn(xh[h].x, xh[h].y);
+            const float2 back = __bfloat1622float2(hi);
+            const size_t o = (size_t)h * (D.W / 2) * g.n;
+            vh[o] = hi;
+            vl[o] = __floats2bfloat162_rn(xh[h].x - back.x, xh[h].y - back.y);
+          }
+      } else {
+        float* v = vunit + ((size_t)ks * D.HW + 2 * wp) * g.n;
+        const bool two = 2 * wp + 1 < D.W;
+#pragma unroll
+        for (int h = 0; h < HC; ++h)
+          if (h < D.H) {
+            float* cell = v + (size_t)h * D.W * g.n;
+            cell[0] = xh[h].x;
+            if (two) cell[g.n] = xh[h].y;
+          }
+      }
     }
     if (L.nslot == 1 && ok && !raw && ks + 1 < ks1) {   // the single slot is free once the records are used
       issue_slab(ks + 1);

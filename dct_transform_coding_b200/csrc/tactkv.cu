@@ -45,6 +45,25 @@ TACTKV_DECL_FUSED(16)
 TACTKV_DECL_FUSED(32)
 TACTKV_DECL_FUSED(64)
 #undef TACTKV_DECL_FUSED
+#define TACTKV_DECL_FUSED_INV(s)                                                                            \
+  cudaError_t launch_fused_inv_##s(const Geom&, const UnitList&, int, float*, const uint32_t*, const uint4*, \
+                                   unsigned int*, cudaStream_t);
+TACTKV_DECL_FUSED_INV(16)
+TACTKV_DECL_FUSED_INV(32)
+TACTKV_DECL_FUSED_INV(64)
+#undef TACTKV_DECL_FUSED_INV
+
+// Decode and all three inverse DCTs in one launch (quantized payloads on the fused grids with S =
+// 16, 32 or 64); cudaErrorNotSupported where the separate inverse kernels must run instead.
+cudaError_t launch_fused_inv(const Geom& g, const UnitList& ul, int nu, float* big, const uint32_t* index,
+                             const uint4* recs, unsigned int* status, cudaStream_t st) {
+  switch (g.S) {
+    case 16: return launch_fused_inv_16(g, ul, nu, big, index, recs, status, st);
+    case 32: return launch_fused_inv_32(g, ul, nu, big, index, recs, status, st);
+    case 64: return launch_fused_inv_64(g, ul, nu, big, index, recs, status, st);
+    default: return cudaErrorNotSupported;
+  }
+}
 
 // Grids with a fused three-axis forward kernel (one launch for the S and H/W passes, the volume
 // kept in L2 between them).
@@ -350,11 +369,20 @@ static tactkv_status decompress_impl(const tactkv_unit* units, int n_units, void
                          if (launch_decode_index(g, ul, nu, w.index, w.recs, w.status, st) != cudaSuccess)
                            return TACTKV_CUDA;
                          mark(1);
-                         t_launches += 2;   // idct_hw, idct_s
-                         if (launch_axis_hw(ch, cw, true, mode, g, ul, nu, w.big, nullptr, w.index, w.recs,
-                                            slabs_per_cta(g, nu, true, mode), st) != cudaSuccess)
+                         const cudaError_t fe = fused_grid(g) ? launch_fused_inv(g, ul, nu, w.big, w.index, w.recs,
+                                                                                 w.status, st)
+                                                              : cudaErrorNotSupported;
+                         if (fe == cudaSuccess) {
+                           t_launches += 1;   // idct3 (decode, inverse H/W, inverse S)
+                         } else if (fe == cudaErrorNotSupported) {
+                           t_launches += 2;   // idct_hw, idct_s
+                           if (launch_axis_hw(ch, cw, true, mode, g, ul, nu, w.big, nullptr, w.index, w.recs,
+                                              slabs_per_cta(g, nu, true, mode), st) != cudaSuccess)
+                             return TACTKV_CUDA;
+                           if (launch_axis_s(cs, true, g, ul, nu, w.big, st) != cudaSuccess) return TACTKV_CUDA;
+                         } else {
                            return TACTKV_CUDA;
-                         if (launch_axis_s(cs, true, g, ul, nu, w.big, st) != cudaSuccess) return TACTKV_CUDA;
+                         }
                          mark(2);
                          return TACTKV_OK;
                        });

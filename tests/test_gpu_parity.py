@@ -288,6 +288,21 @@ def test_tensor_core_and_cuda_core_s_pass_both_match_the_oracle(S, H, W):
     assert torch.equal(pay_tc[:, :64 + S * H * W], pay_sm[:, :64 + S * H * W])
 
 
+@pytest.mark.parametrize("S,H,W,flags,dtype", [
+    (16, 8, 8, 0, torch.float32),     # fused decode on the tensor cores, float32 output
+    (32, 16, 16, 1, torch.bfloat16),  # NO_QUANT on a fused grid: the separate (exact) inverse kernels
+    (64, 14, 14, 1, torch.float32),
+])
+def test_fused_grid_output_variants(S, H, W, flags, dtype):
+    """The fused decode kernel writes bf16 or float32; NO_QUANT payloads keep the separate inverse
+    kernels (their round trip must stay within 1e-5), on the grids that have the fused kernels."""
+    heads, D = 1, 64
+    x = make_unit(S, H, W, heads, D, rho=(0.9, 0.85, 0.85), nu=4.0, seed=90 + S, dtype=dtype, device=DEV)[None]
+    reports, _, y = _check_batch(x, S, H, W, 3, flags=flags)
+    if flags:
+        assert rel_rms(y.double().cpu(), x.double().cpu()) <= 1e-5
+
+
 # ------------------------------------------------------------------------------ exact ties ---
 def _gpu_allocation(var, grid, bits):
     S, H, W = grid
