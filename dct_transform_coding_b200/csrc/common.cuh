@@ -25,7 +25,6 @@ constexpr size_t kStatusBytes = 256;       // status word at the start of the wo
 constexpr int kMaxHW = 1024;               // H*W limit of the H/W-axis kernels
 constexpr int kMaxSlabs = 64;              // S limit
 constexpr int kMaxN = kMaxSlabs * kMaxHW;  // bins per unit limit
-constexpr int kPackRecs = 1024;            // records per packing range (one CTA)
 
 enum HwMode { kStats = 0, kQuant = 1, kRaw = 2 };
 
@@ -83,8 +82,8 @@ cudaError_t launch_axis_hw(int hcls, int wcls, bool inverse, int mode, const Geo
                            float* partial, const uint32_t* index, const uint4* recs, int spc, cudaStream_t st);
 void axis_hw_shape(int hcls, int wcls, const Geom& g, bool inverse, int mode, size_t* smem, int* threads);
 // Per-unit bit allocation: writes b, sigma and the header into the payload, P and NZ into the
-// unit's index block, the records {bin, bits, P_i, 1/sigma_i} of the bins with bits into recs
-// (N per unit), and zeroes the stream word at every P(k_s).
+// unit's index block, and the records {bin, bits, P_i, 1/sigma_i} of the bins with bits into recs
+// (N per unit).
 cudaError_t launch_allocate(const Geom& g, const UnitList& ul, int nu, const float* partial, double* var,
                             uint32_t* index, uint4* recs, cudaStream_t st);
 // The allocation alone, on the fp64 variances var[u][bin] given in the workspace (which it

@@ -486,6 +486,46 @@ int tactkv_lloyd_max_table(int bits, double* levels, double* thresholds) {
   return L;
 }
 
+tactkv_status tactkv_occupancy(const void* payload, size_t bytes, tactkv_occupancy_t* out) {
+  if (!payload || !out || bytes < (size_t)kHeaderBytes) return TACTKV_INVALID_ARG;
+  const unsigned char* p = static_cast<const unsigned char*>(payload);
+  uint32_t h32[16];
+  memcpy(h32, p, sizeof(h32));
+  int32_t i32[16];
+  memcpy(i32, p, sizeof(i32));
+  if (h32[0] != kMagic || (h32[1] & 0xffffu) != (uint32_t)kVersion) return TACTKV_CORRUPT_PAYLOAD;
+  const long long S = i32[4], H = i32[5], W = i32[6], heads = i32[7], head_dim = i32[8];
+  if (S < 1 || H < 1 || W < 1 || heads < 1 || head_dim < 1) return TACTKV_CORRUPT_PAYLOAD;
+  const unsigned long long N = (unsigned long long)(S * H * W), n = (unsigned long long)(heads * head_dim);
+  if (bytes < (size_t)kHeaderBytes + N) return TACTKV_INVALID_ARG;
+  const bool raw = (h32[1] >> 16) & TACTKV_NO_QUANT;
+  unsigned long long code_bits = 0;
+  for (unsigned long long i = 0; i < N; ++i) {
+    const unsigned b = p[kHeaderBytes + i];
+    if (b > 8) return TACTKV_CORRUPT_PAYLOAD;
+    code_bits += b;
+  }
+  if (raw) code_bits = 32ull * N;
+  if (code_bits != h32[10]) return TACTKV_CORRUPT_PAYLOAD;
+  unsigned long long total = 0;
+  memcpy(&total, p + 48, sizeof(total));
+  out->bins = N;
+  out->channels = n;
+  out->code_bits = code_bits;
+  out->formula_bits = code_bits * n + 32ull * N;
+  out->index_bits = 8ull * N;
+  out->payload_bytes = total;
+  out->bits_per_element = 8.0 * (double)total / ((double)N * (double)n);
+  out->shrink_vs_bf16 = total ? 2.0 * (double)N * (double)n / (double)total : 0.0;
+  return TACTKV_OK;
+}
+
+int64_t tactkv_max_batch(uint64_t hbm_bytes, uint64_t fixed_bytes, uint64_t per_request_bytes) {
+  if (per_request_bytes == 0) return -1;
+  if (fixed_bytes >= hbm_bytes) return 0;
+  return (int64_t)((hbm_bytes - fixed_bytes) / per_request_bytes);
+}
+
 int tactkv_last_launches(void) { return t_launches; }
 
 int tactkv_format_version(void) { return kVersion; }

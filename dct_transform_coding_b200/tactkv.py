@@ -38,7 +38,7 @@ TACTKV_FP32_IO = 2
 HEADER_BYTES = 64
 EXPORTED = ("tactkv_payload_bytes", "tactkv_workspace_bytes", "tactkv_compress", "tactkv_decompress",
             "tactkv_compress_profiled", "tactkv_decompress_profiled", "tactkv_compress_noalloc",
-            "tactkv_allocate", "tactkv_device_status",
+            "tactkv_allocate", "tactkv_device_status", "tactkv_occupancy", "tactkv_max_batch",
             "tactkv_status_string", "tactkv_lloyd_max_table", "tactkv_format_version", "tactkv_last_launches")
 
 
@@ -52,6 +52,13 @@ class tactkv_unit(ctypes.Structure):
         ("token_stride", ctypes.c_int64), ("head_stride", ctypes.c_int64),
         ("payload", ctypes.c_void_p), ("payload_capacity", ctypes.c_size_t),
     ]
+
+
+class tactkv_occupancy_t(ctypes.Structure):
+    _fields_ = [("bins", ctypes.c_uint64), ("channels", ctypes.c_uint64), ("code_bits", ctypes.c_uint64),
+                ("formula_bits", ctypes.c_uint64), ("index_bits", ctypes.c_uint64),
+                ("payload_bytes", ctypes.c_uint64), ("bits_per_element", ctypes.c_double),
+                ("shrink_vs_bf16", ctypes.c_double)]
 
 
 _P = ctypes.POINTER(tactkv_unit)
@@ -72,6 +79,10 @@ _lib.tactkv_allocate.restype = ctypes.c_int
 _lib.tactkv_allocate.argtypes = [_P, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
 _lib.tactkv_device_status.restype = ctypes.c_int
 _lib.tactkv_device_status.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+_lib.tactkv_occupancy.restype = ctypes.c_int
+_lib.tactkv_occupancy.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(tactkv_occupancy_t)]
+_lib.tactkv_max_batch.restype = ctypes.c_int64
+_lib.tactkv_max_batch.argtypes = [ctypes.c_uint64, ctypes.c_uint64, ctypes.c_uint64]
 _lib.tactkv_status_string.restype = ctypes.c_char_p
 _lib.tactkv_status_string.argtypes = [ctypes.c_int]
 _lib.tactkv_lloyd_max_table.restype = ctypes.c_int
@@ -164,6 +175,31 @@ def allocate(var: torch.Tensor, S: int, H: int, W: int, bits: int, *, heads: int
 
 def tactkv_device_status(workspace_ptr: int, workspace_bytes: int, stream_ptr: int) -> int:
     return int(_lib.tactkv_device_status(ctypes.c_void_p(workspace_ptr), workspace_bytes, ctypes.c_void_p(stream_ptr)))
+
+
+def tactkv_occupancy(payload) -> dict:
+    """Occupancy of one payload (a host bytes-like object or a CPU uint8 tensor)."""
+    buf = bytes(payload.numpy().tobytes()) if isinstance(payload, torch.Tensor) else bytes(payload)
+    out = tactkv_occupancy_t()
+    st = int(_lib.tactkv_occupancy(ctypes.c_char_p(buf), len(buf), ctypes.byref(out)))
+    if st != TACTKV_OK:
+        raise TactkvError(st, "tactkv_occupancy")
+    return {name: getattr(out, name) for name, _ in tactkv_occupancy_t._fields_}
+
+
+def tactkv_max_batch(hbm_bytes: int, fixed_bytes: int, per_request_bytes: int) -> int:
+    return int(_lib.tactkv_max_batch(int(hbm_bytes), int(fixed_bytes), int(per_request_bytes)))
+
+
+def batch_capacity(hbm_bytes: int, fixed_bytes: int, payload_bytes_per_request: int, text_kv_bytes_per_request: int,
+                   visual_kv_bf16_bytes_per_request: int) -> dict:
+    """Decode batch that fits with the visual KV compressed versus kept in bf16 (the text KV stays
+    bf16 either way), and the per-request cache shrink."""
+    comp = payload_bytes_per_request + text_kv_bytes_per_request
+    full = visual_kv_bf16_bytes_per_request + text_kv_bytes_per_request
+    return {"batch_bf16": tactkv_max_batch(hbm_bytes, fixed_bytes, full),
+            "batch_compressed": tactkv_max_batch(hbm_bytes, fixed_bytes, comp),
+            "cache_shrink": full / comp if comp else float("inf")}
 
 
 def tactkv_status_string(status: int) -> str:

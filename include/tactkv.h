@@ -170,6 +170,32 @@ const char* tactkv_status_string(tactkv_status status);
    0 for bits outside 1..8.  Host-only; needs no GPU. */
 int tactkv_lloyd_max_table(int bits, double* levels, double* thresholds);
 
+/* Occupancy of one compressed unit ("Methodology in Plain English", stage 4: a layer's cache takes
+   sum_i (b_i * d + 32) bits plus a small index).  Here d is the number of channels sharing a
+   gain, n = heads*head_dim, and the index is the byte b_i of every bin. */
+typedef struct {
+  uint64_t bins;            /* N */
+  uint64_t channels;        /* n */
+  uint64_t code_bits;       /* sum_i b_i, the bits of one channel stream */
+  uint64_t formula_bits;    /* sum_i (b_i * n + 32): codes and gains */
+  uint64_t index_bits;      /* 8 * N: the bit widths */
+  uint64_t payload_bytes;   /* the payload's actual size (header, padding and alignment included) */
+  double bits_per_element;  /* 8 * payload_bytes / (N * n) */
+  double shrink_vs_bf16;    /* 2 * N * n / payload_bytes: size of the bf16 volume over the payload */
+} tactkv_occupancy_t;
+
+/* Reads a HOST copy of a payload (at least its header and b[] array: 64 + N bytes) and fills
+   *out.  Returns TACTKV_OK, TACTKV_INVALID_ARG (null pointers) or TACTKV_CORRUPT_PAYLOAD (bad
+   magic or version, a bit width above 8, or a code_bits field that disagrees with b[]).
+   Host-only; needs no GPU. */
+tactkv_status tactkv_occupancy(const void* payload, size_t bytes, tactkv_occupancy_t* out);
+
+/* Largest number of requests whose caches fit: floor((hbm_bytes - fixed_bytes) / per_request_bytes)
+   (0 when fixed_bytes >= hbm_bytes, -1 when per_request_bytes is 0).  fixed_bytes: what every
+   request shares (weights, activations, runtime reserve); per_request_bytes: one request's cache,
+   e.g. the sum of its units' payload_bytes plus its uncompressed text KV.  Host-only. */
+int64_t tactkv_max_batch(uint64_t hbm_bytes, uint64_t fixed_bytes, uint64_t per_request_bytes);
+
 /* Version of the payload format this library writes and reads. */
 int tactkv_format_version(void);
 

@@ -412,6 +412,25 @@ def codes_of(payload) -> Tuple[np.ndarray, np.ndarray]:
     return p["b"], _unpack_streams(p["streams"], p["b"])
 
 
+def occupancy_bits(b: np.ndarray, d: int) -> int:
+    """Stage 4's occupancy of one compressed layer: sum_i (b_i * d + 32) bits, d the channels that
+    share a gain (here all n = heads * head_dim channels of a bin), 32 bits for each bin's gain."""
+    b = np.asarray(b, dtype=np.int64)
+    return int(np.sum(b * int(d) + 32))
+
+
+def index_bits(N: int) -> int:
+    """The small index on top of the occupancy: one byte (the bit width) per bin."""
+    return 8 * int(N)
+
+
+def max_batch(hbm_bytes: int, fixed_bytes: int, per_request_bytes: int) -> int:
+    """Requests whose caches fit in what is left of the device memory after the shared part."""
+    if per_request_bytes <= 0:
+        return -1
+    return max(0, (int(hbm_bytes) - int(fixed_bytes)) // int(per_request_bytes))
+
+
 def threshold_distance(u: np.ndarray, bits: int) -> np.ndarray:
     """Distance of u to the nearest decision threshold t_j of the b-bit codebook, each distance
     taken relative to max(1, |t_j|) (fp64).  This is the band of the code-parity rule: a code may

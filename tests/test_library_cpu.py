@@ -155,3 +155,46 @@ def test_cell_table_code_lookup_equals_threshold_count(bits):
     code = c + (u >= padded[c]) + (u >= padded[c + 1])
     want = np.searchsorted(th32, u, side="right")
     assert np.array_equal(code, want)
+
+
+# ------------------------------------------------------------------- occupancy and capacity ---
+@pytest.mark.parametrize("bits", [1, 2, 4, 8])
+def test_occupancy_of_an_oracle_payload(T, bits):
+    """The library's occupancy report on a payload written by the oracle (no GPU needed)."""
+    S, H, W, heads, D = 4, 6, 5, 1, 32
+    x = np.random.default_rng(bits).standard_normal((S * H * W, heads, D))
+    p, info = O.compress_unit(x, S, H, W, heads, D, bits, return_info=True)
+    occ = T.tactkv_occupancy(p)
+    N, n = S * H * W, heads * D
+    assert occ["bins"] == N and occ["channels"] == n
+    assert occ["code_bits"] == int(info["b"].sum())
+    assert occ["formula_bits"] == O.occupancy_bits(info["b"], n)
+    assert occ["index_bits"] == O.index_bits(N)
+    assert occ["payload_bytes"] == len(p)
+    assert abs(occ["bits_per_element"] - 8 * len(p) / (N * n)) < 1e-12
+    assert abs(occ["shrink_vs_bf16"] - 2 * N * n / len(p)) < 1e-12
+
+
+def test_occupancy_rejects_corrupt_payloads(T):
+    S, H, W, heads, D = 4, 6, 5, 1, 32
+    p = bytearray(O.compress_unit(np.ones((S * H * W, heads, D)), S, H, W, heads, D, 2))
+    bad = bytearray(p)
+    bad[0] ^= 1                                      # magic
+    with pytest.raises(T.TactkvError):
+        T.tactkv_occupancy(bytes(bad))
+    bad = bytearray(p)
+    bad[64] = 9                                      # a bit width above 8
+    with pytest.raises(T.TactkvError):
+        T.tactkv_occupancy(bytes(bad))
+    bad = bytearray(p)
+    bad[64] = (bad[64] + 1) % 9 if bad[64] < 8 else 7  # widths no longer sum to the header's code_bits
+    with pytest.raises(T.TactkvError):
+        T.tactkv_occupancy(bytes(bad))
+
+
+def test_max_batch_and_capacity(T):
+    assert T.tactkv_max_batch(100, 30, 7) == O.max_batch(100, 30, 7) == 10
+    assert T.tactkv_max_batch(10, 20, 1) == 0 and T.tactkv_max_batch(10, 0, 0) == -1
+    cap = T.batch_capacity(hbm_bytes=1000, fixed_bytes=200, payload_bytes_per_request=10,
+                           text_kv_bytes_per_request=6, visual_kv_bf16_bytes_per_request=154)
+    assert cap == {"batch_bf16": 5, "batch_compressed": 50, "cache_shrink": 10.0}

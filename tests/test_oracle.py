@@ -325,3 +325,29 @@ def test_to_bf16_rounding():
     r = np.random.default_rng(3).standard_normal(10000).astype(np.float32).astype(np.float64)
     ref = torch.from_numpy(r.astype(np.float32)).to(torch.bfloat16).double().numpy()
     assert np.array_equal(O.to_bf16(r), ref)
+
+
+# ------------------------------------------------------------------- occupancy and capacity ---
+def test_occupancy_hand_example():
+    """Stage 4: sum_i (b_i d + 32) bits, plus one index byte per bin."""
+    assert O.occupancy_bits(np.array([2, 0, 3]), 2) == (2 * 2 + 32) + (0 + 32) + (3 * 2 + 32)
+    assert O.occupancy_bits(np.zeros(5, int), 128) == 5 * 32
+    assert O.index_bits(7) == 56
+
+
+def test_occupancy_bounds_the_payload():
+    """The payload holds exactly the occupancy and the index plus the header and 16-byte padding."""
+    S, H, W, heads, D = 4, 3, 5, 2, 16
+    x = RNG.standard_normal((S * H * W, heads, D))
+    for bits in (1, 3):
+        p, info = O.compress_unit(x, S, H, W, heads, D, bits, return_info=True)
+        N, n = S * H * W, heads * D
+        need_bits = O.occupancy_bits(info["b"], n) + O.index_bits(N)
+        assert 8 * len(p) >= need_bits
+        assert 8 * len(p) - need_bits < 8 * (64 + 16 + 16 + 16 * n)    # header and paddings only
+
+
+def test_max_batch_hand_values():
+    assert O.max_batch(100, 30, 7) == 10
+    assert O.max_batch(10, 20, 1) == 0
+    assert O.max_batch(10, 0, 0) == -1
