@@ -31,8 +31,16 @@ Readings taken where the pages are silent (each is listed in the design notes):
   (greatest sigma_i^2 * 4^-b_i, ties to the lowest index) one step at a time.
 * A code is the number of thresholds t_j <= u with u = X / sigma_i; the decision is taken in
   float32 (the precision of the CUDA kernels), ties go to the upper cell, outer cells saturate.
-* The fixed shared rotation of the shape vector named in stage 4 is not applied (the codec's
-  specification leaves it out).
+* The fixed shared rotation of the shape vector named in stage 4 is optional (FLAG_ROTATE, off by
+  default, as in the codec's specification).  Reading of "fixed shared orthogonal rotation": the
+  same orthogonal matrix R for every bin, layer and sequence, block-diagonal over groups of 32
+  consecutive channels, R_g = (1/sqrt(32)) H_32 D_g with H_32 the Sylvester-Hadamard matrix and D_g
+  a diagonal of signs drawn once from a counter-based SplitMix64 (see ``rotation_signs``).  It
+  acts on each bin's vector of n coefficients after the gain is measured (R is orthogonal, so the
+  gain is unchanged) and is undone after dequantization.
+* Ablation variants ("Main Findings": fewer transformed axes, uniform allocation), also flags:
+  FLAG_SKIP_S / _H / _W leave that axis untransformed (all three: no DCT); FLAG_UNIFORM gives every
+  bin with sigma^2 > 0 the nominal bits (b_i = bits) instead of water-filling.
 * Payload layout: see ``FORMAT`` below (the pages fix only its size, stage 4:
   sum_i (b_i * d + 32) bits plus a small index).
 """
@@ -60,6 +68,12 @@ from scipy.special import erfc, ndtri
 MAGIC = 0x31564B54          # bytes 'T','K','V','1'
 VERSION = 1
 FLAG_NO_QUANT = 1
+FLAG_SKIP_S = 4             # no DCT along S (ablation)
+FLAG_SKIP_H = 8             # no DCT along H
+FLAG_SKIP_W = 16            # no DCT along W
+FLAG_UNIFORM = 32           # uniform allocation: b_i = bits for every bin with sigma^2 > 0
+FLAG_ROTATE = 64            # fixed shared rotation of each bin's shape vector before quantization
+PAYLOAD_FLAGS = FLAG_NO_QUANT | FLAG_SKIP_S | FLAG_SKIP_H | FLAG_SKIP_W | FLAG_UNIFORM | FLAG_ROTATE
 HEADER_FMT = "<IHHiiiiiiiiIIQII"   # magic ver flags layer kv S H W heads head_dim bits codebits stride total r0 r1
 HEADER_BYTES = 64
 assert struct.calcsize(HEADER_FMT) == HEADER_BYTES
@@ -85,22 +99,77 @@ def dct_matrix(L: int) -> np.ndarray:
     return C
 
 
-def dct3(x: np.ndarray) -> np.ndarray:
-    """Forward separable 3D DCT-II of x[S, H, W, n] along the first three axes (fp64)."""
+def dct3(x: np.ndarray, axes=(True, True, True)) -> np.ndarray:
+    """Forward separable 3D DCT-II of x[S, H, W, n] along the first three axes (fp64); an axis whose
+    entry in `axes` is False is left untransformed (the ablations with fewer axes)."""
     S, H, W, _ = x.shape
-    y = np.einsum("ks,shwc->khwc", dct_matrix(S), x)
-    y = np.einsum("kh,shwc->skwc", dct_matrix(H), y)
-    y = np.einsum("kw,shwc->shkc", dct_matrix(W), y)
+    y = x
+    if axes[0]:
+        y = np.einsum("ks,shwc->khwc", dct_matrix(S), y)
+    if axes[1]:
+        y = np.einsum("kh,shwc->skwc", dct_matrix(H), y)
+    if axes[2]:
+        y = np.einsum("kw,shwc->shkc", dct_matrix(W), y)
     return y
 
 
-def idct3(X: np.ndarray) -> np.ndarray:
-    """Inverse of dct3: the transpose (DCT-III) along each axis."""
+def idct3(X: np.ndarray, axes=(True, True, True)) -> np.ndarray:
+    """Inverse of dct3: the transpose (DCT-III) along each transformed axis."""
     S, H, W, _ = X.shape
-    y = np.einsum("ks,khwc->shwc", dct_matrix(S), X)
-    y = np.einsum("kh,skwc->shwc", dct_matrix(H), y)
-    y = np.einsum("kw,shkc->shwc", dct_matrix(W), y)
+    y = X
+    if axes[0]:
+        y = np.einsum("ks,khwc->shwc", dct_matrix(S), y)
+    if axes[1]:
+        y = np.einsum("kh,skwc->shwc", dct_matrix(H), y)
+    if axes[2]:
+        y = np.einsum("kw,shkc->shwc", dct_matrix(W), y)
     return y
+
+
+def axes_of(flags: int):
+    return (not flags & FLAG_SKIP_S, not flags & FLAG_SKIP_H, not flags & FLAG_SKIP_W)
+
+
+# ----------------------------------------------------------------- shared shape rotation ---
+ROTATION_SEED = 0x544143544B56     # "TACTKV"
+ROTATION_GROUP = 32
+
+
+def splitmix64(seed: int, i: int) -> int:
+    """Output i (0, 1, ...) of the SplitMix64 generator (Steele, Lea and Flood, "Fast splittable
+    pseudorandom number generators", OOPSLA 2014) started from `seed`: state = seed + (i+1) gamma,
+    gamma = 0x9E3779B97F4A7C15, then the variant-13 finalizer of MurmurHash3."""
+    m = (1 << 64) - 1
+    z = (seed + (i + 1) * 0x9E3779B97F4A7C15) & m
+    z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & m
+    z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & m
+    return z ^ (z >> 31)
+
+
+def rotation_signs(n: int) -> np.ndarray:
+    """Sign of channel c: -1 when the top bit of SplitMix64 output c (seed ROTATION_SEED) is set."""
+    return np.array([-1.0 if splitmix64(ROTATION_SEED, c) >> 63 else 1.0 for c in range(n)])
+
+
+def hadamard(m: int) -> np.ndarray:
+    """Sylvester-Hadamard matrix of order m (a power of two): H[i, j] = (-1)^popcount(i & j)."""
+    i = np.arange(m)[:, None]
+    j = np.arange(m)[None, :]
+    pop = np.vectorize(lambda v: bin(int(v)).count("1"))(i & j)
+    return np.where(pop % 2 == 1, -1.0, 1.0)
+
+
+def rotation_matrix(n: int) -> np.ndarray:
+    """The fixed shared rotation R (n x n, orthogonal): block-diagonal over groups of 32 channels,
+    block g = H_32 diag(signs of its channels) / sqrt(32).  A bin's shape vector v becomes R v."""
+    if n % ROTATION_GROUP:
+        raise ValueError("the rotation acts on whole groups of 32 channels")
+    Hm = hadamard(ROTATION_GROUP) / math.sqrt(ROTATION_GROUP)
+    sg = rotation_signs(n)
+    R = np.zeros((n, n))
+    for g0 in range(0, n, ROTATION_GROUP):
+        R[g0:g0 + ROTATION_GROUP, g0:g0 + ROTATION_GROUP] = Hm * sg[None, g0:g0 + ROTATION_GROUP]
+    return R
 
 
 # -------------------------------------------------------------------------- bin variances ---
@@ -177,6 +246,13 @@ def allocate_bits(var: np.ndarray, bits: int) -> np.ndarray:
         i = idx[key == m].min()                     # ties -> lowest index
         b[i] += 1
     return b
+
+
+def allocate_uniform(var: np.ndarray, bits: int) -> np.ndarray:
+    """The uniform-allocation ablation ("Main Findings"): every bin with sigma^2 > 0 gets the nominal
+    bits, every other bin none."""
+    var = np.asarray(var, dtype=np.float64)
+    return np.where(var > 0, int(bits), 0).astype(np.int64)
 
 
 def allocate_bits_topk(var: np.ndarray, bits: int) -> np.ndarray:
@@ -331,16 +407,20 @@ def _unpack_streams(streams: np.ndarray, b: np.ndarray) -> np.ndarray:
 
 def compress_unit(x, S: int, H: int, W: int, heads: int, head_dim: int, bits: int,
                   layer: int = 0, kv: int = 0, no_quant: bool = False,
-                  return_info: bool = False):
-    """Compress one visual K or V, x[S*H*W, heads, head_dim] (any real dtype), to payload bytes."""
+                  return_info: bool = False, flags: int = 0):
+    """Compress one visual K or V, x[S*H*W, heads, head_dim] (any real dtype), to payload bytes.
+    flags: FLAG_SKIP_* (axes left untransformed), FLAG_UNIFORM, FLAG_ROTATE (see the head)."""
     n = heads * head_dim
     N = S * H * W
     if not 1 <= bits <= MAX_BITS:
         raise ValueError("bits must be 1..8")
+    flags = (int(flags) | (FLAG_NO_QUANT if no_quant else 0)) & PAYLOAD_FLAGS
+    no_quant = bool(flags & FLAG_NO_QUANT)
     xv = np.asarray(x, dtype=np.float64).reshape(S, H, W, n)
-    X = dct3(xv).reshape(N, n)
+    X = dct3(xv, axes_of(flags)).reshape(N, n)
     var = bin_variances(X)
     sig = stored_sigma(var)
+    Xq = X @ rotation_matrix(n).T if (flags & FLAG_ROTATE) and not no_quant else X   # row i: R X_i
     if no_quant:
         b = np.zeros(N, dtype=np.int64)
         lay = payload_layout(N, n, 32 * N, True)
@@ -349,23 +429,23 @@ def compress_unit(x, S: int, H: int, W: int, heads: int, head_dim: int, bits: in
         code_bits = 32 * N
         codes = None
     else:
-        b = allocate_bits(var, bits)
+        b = allocate_uniform(var, bits) if flags & FLAG_UNIFORM else allocate_bits(var, bits)
         code_bits = int(b.sum())
         lay = payload_layout(N, n, code_bits)
         codes = np.zeros((N, n), dtype=np.int64)
         for i in np.nonzero(b)[0]:
-            u = X[i] / np.float64(sig[i])
+            u = Xq[i] / np.float64(sig[i])
             codes[i] = quantize(u, int(b[i]))
         body = _pack_streams(codes, b, lay["chan_stride"])
     buf = bytearray(lay["total"])
-    struct.pack_into(HEADER_FMT, buf, 0, MAGIC, VERSION, FLAG_NO_QUANT if no_quant else 0,
+    struct.pack_into(HEADER_FMT, buf, 0, MAGIC, VERSION, flags,
                      layer, kv, S, H, W, heads, head_dim, bits, code_bits, lay["chan_stride"],
                      lay["total"], 0, 0)
     buf[lay["off_b"]:lay["off_b"] + N] = b.astype(np.uint8).tobytes()
     buf[lay["off_sigma"]:lay["off_sigma"] + 4 * N] = sig.astype("<f4").tobytes()
     buf[lay["off_codes"]:] = body.tobytes()
     if return_info:
-        return bytes(buf), dict(X=X, var=var, sigma=sig, b=b, codes=codes)
+        return bytes(buf), dict(X=X, Xq=Xq, var=var, sigma=sig, b=b, codes=codes)
     return bytes(buf)
 
 
@@ -402,7 +482,9 @@ def decompress_unit(payload) -> np.ndarray:
         X = np.zeros((N, n), dtype=np.float64)
         for i in np.nonzero(b)[0]:
             X[i] = np.float64(p["sigma"][i]) * dequantize(codes[i], int(b[i]))
-    x = idct3(X.reshape(p["S"], p["H"], p["W"], n))
+        if p["flags"] & FLAG_ROTATE:
+            X = X @ rotation_matrix(n)                  # row i: R^T (dequantized R X_i)
+    x = idct3(X.reshape(p["S"], p["H"], p["W"], n), axes_of(p["flags"]))
     return x.reshape(N, p["heads"], p["head_dim"])
 
 

@@ -351,3 +351,81 @@ def test_max_batch_hand_values():
     assert O.max_batch(100, 30, 7) == 10
     assert O.max_batch(10, 20, 1) == 0
     assert O.max_batch(10, 0, 0) == -1
+
+
+# ----------------------------------------------------- variants: rotation, axis mask, uniform ---
+def test_splitmix64_published_outputs():
+    """SplitMix64 (Steele, Lea and Flood 2014) from seed 0: the first three outputs of the
+    reference implementation (java.util.SplittableRandom's mix64 on the gamma sequence)."""
+    assert [O.splitmix64(0, i) for i in range(3)] == [0xE220A8397B1DCDAF, 0x6E789E6AA1B965F4, 0x06C45D188009454F]
+
+
+def test_hadamard_matches_scipy():
+    import scipy.linalg
+    for m in (1, 2, 8, 32):
+        assert np.array_equal(O.hadamard(m), scipy.linalg.hadamard(m))
+
+
+def test_rotation_is_orthogonal_block_diagonal_and_keeps_the_gain():
+    n = 96
+    R = O.rotation_matrix(n)
+    assert np.allclose(R @ R.T, np.eye(n), atol=1e-14, rtol=0)
+    assert np.allclose(np.abs(R[:32, :32]), 1 / math.sqrt(32), atol=0)
+    assert not R[:32, 32:].any() and not R[32:64, :32].any()          # groups of 32 channels
+    s = O.rotation_signs(n)
+    assert set(np.unique(s)) <= {-1.0, 1.0} and 20 < np.sum(s > 0) < 76
+    X = RNG.standard_normal((10, n))
+    assert np.allclose(O.bin_variances(X @ R.T), O.bin_variances(X), rtol=1e-13)   # gains unchanged
+
+
+def test_rotation_round_trip_and_gaussianization():
+    """With the rotation on, decompress(compress(x)) still reconstructs x (the decoder undoes R),
+    and a bin whose energy sits in one channel per group is spread over all 32 of them."""
+    S, H, W, heads, D = 2, 3, 4, 1, 64
+    x = RNG.standard_normal((S * H * W, heads, D))
+    p8 = O.compress_unit(x, S, H, W, heads, D, 8, flags=O.FLAG_ROTATE)
+    assert O.parse_payload(p8)["flags"] & O.FLAG_ROTATE
+    assert np.sqrt(np.mean((O.decompress_unit(p8) - x) ** 2)) < 0.02 * np.sqrt(np.mean(x ** 2))
+    e = np.zeros((1, 64))
+    e[0, 5] = 1.0
+    v = (e @ O.rotation_matrix(64).T)[0]
+    assert np.allclose(np.abs(v[:32]), 1 / math.sqrt(32)) and not v[32:].any()
+    # same allocation and gains as without the rotation; the codes differ
+    p0, i0 = O.compress_unit(x, S, H, W, heads, D, 2, return_info=True)
+    p1, i1 = O.compress_unit(x, S, H, W, heads, D, 2, return_info=True, flags=O.FLAG_ROTATE)
+    assert np.array_equal(i0["b"], i1["b"]) and np.array_equal(i0["sigma"], i1["sigma"])
+    assert not np.array_equal(i0["codes"], i1["codes"])
+
+
+@pytest.mark.parametrize("axes", [(True, False, False), (False, True, True), (False, False, True),
+                                  (False, False, False)])
+def test_axis_mask_matches_scipy_on_the_kept_axes(axes):
+    x = RNG.standard_normal((5, 6, 7, 3))
+    keep = tuple(a for a, k in zip((0, 1, 2), axes) if k)
+    ref = scipy.fft.dctn(x, type=2, norm="ortho", axes=keep) if keep else x
+    assert np.allclose(O.dct3(x, axes), ref, atol=1e-12, rtol=0)
+    assert np.allclose(O.idct3(ref, axes), x, atol=1e-12, rtol=0)
+    flags = (0 if axes[0] else O.FLAG_SKIP_S) | (0 if axes[1] else O.FLAG_SKIP_H) | (0 if axes[2] else O.FLAG_SKIP_W)
+    assert O.axes_of(flags) == axes
+
+
+def test_uniform_allocation_and_theorem1_through_the_codec():
+    """FLAG_UNIFORM gives every active bin the nominal bits; on Gaussian bins with spread variances
+    the distortion of the uniform payload over the water-filling payload approaches AM/GM of the
+    variances (Theorem 1) at a high rate."""
+    assert O.allocate_uniform(np.array([0.0, 2.0, 5.0]), 3).tolist() == [0, 3, 3]
+    rng = np.random.default_rng(11)
+    S, H, W, heads, D, bits = 4, 4, 4, 8, 250, 5
+    N, n = S * H * W, heads * D
+    var = 10.0 ** rng.uniform(-1, 1, N)
+    X = rng.standard_normal((N, n)) * np.sqrt(var)[:, None]
+    x = O.idct3(X.reshape(S, H, W, n)).reshape(N, heads, D)     # a field whose bins hold X
+    d = {}
+    for name, fl in (("uniform", O.FLAG_UNIFORM), ("wf", 0)):
+        p, info = O.compress_unit(x, S, H, W, heads, D, bits, return_info=True, flags=fl)
+        if fl:
+            assert np.all(info["b"] == bits)
+        d[name] = np.sum((O.decompress_unit(p) - x) ** 2)
+    v = O.bin_variances(X)
+    inv_gamma = np.mean(v) / math.exp(np.mean(np.log(v)))
+    assert abs(d["uniform"] / d["wf"] / inv_gamma - 1) < 0.1

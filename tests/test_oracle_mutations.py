@@ -49,6 +49,18 @@ MUTATIONS = [
      "return np.min(gaps / np.maximum(1.0, np.abs(thresholds_b)) ** 2, axis=-1)"),
     ("code band: farthest threshold", "return np.min(gaps / np.maximum(1.0, np.abs(thresholds_b)), axis=-1)",
      "return np.max(gaps / np.maximum(1.0, np.abs(thresholds_b)), axis=-1)"),
+    ("rotation: Hadamard sign from the wrong bits", "return np.where(pop % 2 == 1, -1.0, 1.0)",
+     "return np.where(pop % 3 == 1, -1.0, 1.0)"),
+    ("rotation: decoder does not undo it", "            X = X @ rotation_matrix(n)                  # row i",
+     "            X = X @ rotation_matrix(n).T                # row i"),
+    ("rotation: unnormalised", "Hm = hadamard(ROTATION_GROUP) / math.sqrt(ROTATION_GROUP)",
+     "Hm = hadamard(ROTATION_GROUP) / ROTATION_GROUP"),
+    ("splitmix: finalizer shift", "z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & m",
+     "z = ((z ^ (z >> 28)) * 0x94D049BB133111EB) & m"),
+    ("axis mask: H skipped when S is", "    if axes[1]:\n        y = np.einsum(\"kh,shwc->skwc\"",
+     "    if axes[0]:\n        y = np.einsum(\"kh,shwc->skwc\""),
+    ("uniform: nominal bits plus one", "return np.where(var > 0, int(bits), 0).astype(np.int64)",
+     "return np.where(var > 0, int(bits) + 1, 0).astype(np.int64)"),
     ("code band: distance to the levels", "thresholds_b = table(bits)[1]", "thresholds_b = table(bits)[0]"),
     ("code band: no relative scaling", "return np.min(gaps / np.maximum(1.0, np.abs(thresholds_b)), axis=-1)",
      "return np.min(gaps, axis=-1)"),
