@@ -147,7 +147,8 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
   }
   act = block_sum<long long>(act, s_ll);
   const long long B = (long long)g.bits * g.N;
-  const bool select = !raw && 8 * act > B;
+  const bool uniform = g.flags & TACTKV_UNIFORM_ALLOC;   // the ablation: bits for every active bin
+  const bool select = !raw && !uniform && 8 * act > B;
 
   // 2. the B-th largest key K (counted with multiplicity): the largest pattern lo with
   // count(lo) >= B, so count(lo + 1) < B.  The keys of bin i are var_i * 4^-k: the mantissa of
@@ -249,7 +250,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
     int b = 0;
     if (!raw && x > 0.0) {
       if (!select) {
-        b = 8;
+        b = uniform ? g.bits : 8;
       } else {
         b = key_count(x, v_hi);
         if (key_count(x, v_lo) > b) {
@@ -317,7 +318,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
     uint32_t* h32 = reinterpret_cast<uint32_t*>(pay);
     int32_t* i32 = reinterpret_cast<int32_t*>(pay);
     h32[0] = kMagic;
-    h32[1] = (uint32_t)kVersion | ((uint32_t)(g.flags & TACTKV_NO_QUANT) << 16);
+    h32[1] = (uint32_t)kVersion | ((uint32_t)(g.flags & kPayloadFlags) << 16);
     i32[2] = ud.layer;
     i32[3] = ud.kv;
     i32[4] = g.S;
@@ -363,7 +364,7 @@ __global__ void __launch_bounds__(256) decode_index_kernel(const __grid_constant
     const uint32_t ver_flags = h32[1], cb = h32[10], cs = h32[11];
     const unsigned long long total = *reinterpret_cast<const unsigned long long*>(pay + 48);
     bool ok = h32[0] == kMagic && (ver_flags & 0xffffu) == (uint32_t)kVersion &&
-              ((ver_flags >> 16) & TACTKV_NO_QUANT) == (raw ? TACTKV_NO_QUANT : 0u) && i32[2] == ud.layer &&
+              (ver_flags >> 16) == ((uint32_t)g.flags & kPayloadFlags) && i32[2] == ud.layer &&
               i32[3] == ud.kv && i32[4] == g.S && i32[5] == g.H && i32[6] == g.W && i32[7] == g.heads &&
               i32[8] == g.head_dim && i32[9] == g.bits;
     if (ok) {

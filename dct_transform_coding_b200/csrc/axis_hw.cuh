@@ -121,7 +121,7 @@ __device__ __forceinline__ int rp_index(int Wp, int kp, int w) { return ((2 * kp
 
 // Column pair (w0, w0+1): read, DCT along H, written back in place as row pairs.
 template <int HC, class D>
-__device__ __forceinline__ void h_pass_fwd(const D& g, float* tile, int w0, int lane) {
+__device__ __forceinline__ void h_pass_fwd(const D& g, float* tile, int w0, int lane, bool skip) {
   const int Wp = 2 * row_pairs(g.W), HP = row_pairs(g.H);
   float2 xh[HC];
 #pragma unroll
@@ -131,7 +131,7 @@ __device__ __forceinline__ void h_pass_fwd(const D& g, float* tile, int w0, int 
       xh[h] = make_float2(cell[0], cell[kChunk]);   // column W (odd W) is padding: read, never used
     }
   __syncwarp();   // the whole column pair is read before any lane rewrites it
-  pencil<HC, D::hx, false>(xh, g.H);
+  if (!skip) pencil<HC, D::hx, false>(xh, g.H);
   float2* t2 = reinterpret_cast<float2*>(tile);
 #pragma unroll
   for (int kp = 0; kp < (HC + 1) / 2; ++kp)
@@ -144,12 +144,13 @@ __device__ __forceinline__ void h_pass_fwd(const D& g, float* tile, int w0, int 
 }
 // Row pair kp -> DCT along W.
 template <int WC, class D>
-__device__ __forceinline__ void w_load_fdct(const D& g, const float2* t2, int kp, int lane, float2 (&x)[WC]) {
+__device__ __forceinline__ void w_load_fdct(const D& g, const float2* t2, int kp, int lane, float2 (&x)[WC],
+                                            bool skip) {
   const int Wp = 2 * row_pairs(g.W);
 #pragma unroll
   for (int t = 0; t < WC; ++t)
     if (t < g.W) x[t] = t2[rp_index(Wp, kp, t) + lane];
-  pencil<WC, D::wx, false>(x, g.W);
+  if (!skip) pencil<WC, D::wx, false>(x, g.W);
 }
 // Sums over the 32 lanes of the warp of 32 values per lane (recursive halving: at each step a
 // lane keeps half of its values and adds the partner lane's copy of that half); lane l returns the
@@ -217,7 +218,7 @@ __device__ __forceinline__ void fdct_hw_slabs(const Geom& g, float* __restrict__
       cp_async_commit();
     }
     // DCT along H, in place, one column pair at a time per warp
-    for (int wp = warp; wp < WP; wp += nwarps) h_pass_fwd<HC>(D, tile, 2 * wp, lane);
+    for (int wp = warp; wp < WP; wp += nwarps) h_pass_fwd<HC>(D, tile, 2 * wp, lane, g.flags & TACTKV_SKIP_H);
     __syncthreads();
     float2* t2 = reinterpret_cast<float2*>(tile);
     // DCT along W on row pair kp; the coefficients go back over the slab of Y (this CTA's own
@@ -225,7 +226,7 @@ __device__ __forceinline__ void fdct_hw_slabs(const Geom& g, float* __restrict__
     float* dst = partial + ((size_t)u * (NX ? NX / kChunk : g.nch) + chunk) * g.N + (size_t)ks * D.HW;
     for (int kp = warp; kp < HP; kp += nwarps) {
       float2 x[WC];
-      w_load_fdct<WC>(D, t2, kp, lane, x);
+      w_load_fdct<WC>(D, t2, kp, lane, x, g.flags & TACTKV_SKIP_W);
       const bool second = 2 * kp + 1 < D.H;
       float* y0 = yslab + (size_t)(2 * kp * D.W) * D.n;
       if constexpr (EF) {
@@ -283,6 +284,9 @@ __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul,
   const unsigned char* pay = ul.u[u].payload;
   const uint32_t* P = index + (size_t)u * unit_index_words(g.S);
   const bool ok = P[g.S + 1] != 0;   // the index kernel checked the header and the bit widths
+  // the shared rotation's inverse: sign of this lane's channel times 1/sqrt(32)
+  const bool rotate = !raw && (g.flags & TACTKV_ROTATE);
+  const float rot_scale = rotate ? rotation_sign((unsigned long long)(chunk * kChunk + lane)) * 0.17677669529663687f : 1.f;
   const uint32_t cstride = ok ? reinterpret_cast<const uint32_t*>(pay)[11] : 0u, sw = cstride / 4;
   const uint32_t* streams = reinterpret_cast<const uint32_t*>(pay + g.off_codes) + (size_t)chunk * kChunk * sw;
   const uint4* urecs = recs + (size_t)u * g.N;
@@ -356,7 +360,13 @@ __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul,
             x[t] = __fmul2_rn(make_float2(l0, l1), make_float2(__uint_as_float(m.x), __uint_as_float(m.y)));
           }
       }
-      pencil<WC, WX, true>(x, D.W);
+      if (rotate) {   // R^T = diag(s) H_32 / sqrt(32) across the warp's 32 channels, both rows
+#pragma unroll
+        for (int t = 0; t < WC; ++t)
+          if (t < D.W)
+            x[t] = make_float2(warp_wht(x[t].x, lane) * rot_scale, warp_wht(x[t].y, lane) * rot_scale);
+      }
+      if (!(g.flags & TACTKV_SKIP_W)) pencil<WC, WX, true>(x, D.W);
       const bool second = 2 * kp + 1 < D.H;
 #pragma unroll
       for (int wp = 0; wp < (WC + 1) / 2; ++wp)
@@ -374,7 +384,7 @@ __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul,
 #pragma unroll
       for (int h = 0; h < HC; ++h)
         if (h < D.H) xh[h] = tile[cp_index(Wp, h, wp) + lane];
-      pencil<HC, HX, true>(xh, D.H);
+      if (!(g.flags & TACTKV_SKIP_H)) pencil<HC, HX, true>(xh, D.H);
       if constexpr (PAIRS) {
         // pair (cell h*W + 2wp, cell h*W + 2wp + 1) = pair index h*(W/2) + wp
         const size_t base = ((size_t)u * g.S + ks) * (D.HW / 2) * g.n + chunk * kChunk + lane;

@@ -73,7 +73,7 @@ __device__ __forceinline__ void fdct_s_cells(const Geom& g, int u, int hw0, int 
 #pragma unroll
     for (int s = 0; s < L; ++s) v[s] = __bfloat162float(t[s * NC * 32]);
   }
-  dct_exact<L, false>(v);
+  if (!(g.flags & TACTKV_SKIP_S)) dct_exact<L, false>(v);
   float* yo = Y + ((size_t)u * L * HW + hw) * n + c0 + lane;
   const size_t kstep = (size_t)HW * n;
 #pragma unroll
@@ -116,7 +116,7 @@ __device__ __forceinline__ void idct_s_cells(const Geom& g, const UnitDev& ud, i
   const float* t = vtile + hwl * 32 + lane;
 #pragma unroll
   for (int k = 0; k < L; ++k) v[k] = t[k * NC * 32];
-  dct_exact<L, true>(v);
+  if (!(g.flags & TACTKV_SKIP_S)) dct_exact<L, true>(v);
   const int c = c0 + lane, head = c / g.head_dim, d = c - head * g.head_dim;
   const long long base = (long long)hw * ud.tok_stride + (long long)head * ud.head_stride + d;
   const long long sstep = (long long)g.HW * ud.tok_stride;

@@ -28,6 +28,12 @@ constexpr int kMaxN = kMaxSlabs * kMaxHW;  // bins per unit limit
 
 enum HwMode { kStats = 0, kQuant = 1, kRaw = 2 };
 
+// flags recorded in the payload header (everything but the I/O type)
+constexpr uint32_t kPayloadFlags =
+    TACTKV_NO_QUANT | TACTKV_SKIP_S | TACTKV_SKIP_H | TACTKV_SKIP_W | TACTKV_UNIFORM_ALLOC | TACTKV_ROTATE;
+constexpr uint32_t kAllFlags = kPayloadFlags | TACTKV_FP32_IO;
+constexpr unsigned long long kRotationSeed = 0x544143544B56ull;
+
 // ------------------------------------------------------------------------ launch descriptors ---
 struct UnitDev {
   const void* in;
@@ -163,6 +169,28 @@ __device__ __forceinline__ void dct_exact(V* x) {
 }
 
 __device__ __forceinline__ void set_status(unsigned int* status, unsigned int code) { atomicCAS(status, 0u, code); }
+
+// ------------------------------------------------------------------ shared shape rotation ---
+// Sign of channel c in the rotation: the top bit of output c of SplitMix64 (Steele, Lea and
+// Flood, OOPSLA 2014) started from kRotationSeed (state seed + (c+1) * gamma, then the variant-13
+// finalizer of MurmurHash3).
+__device__ __forceinline__ float rotation_sign(unsigned long long c) {
+  unsigned long long z = kRotationSeed + (c + 1ull) * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  z ^= z >> 31;
+  return (z >> 63) ? -1.f : 1.f;
+}
+// Walsh-Hadamard transform of the 32 lanes' values (Sylvester order: lane i gets
+// sum_j (-1)^popcount(i & j) v_j), unnormalised; every lane of the warp calls it.
+__device__ __forceinline__ float warp_wht(float v, int lane) {
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1) {
+    const float p = __shfl_xor_sync(0xffffffffu, v, h);
+    v = fmaf(v, (lane & h) ? -1.f : 1.f, p);   // lower lane: p + v; upper lane: p - v
+  }
+  return v;
+}
 
 // Asynchronous global -> shared copies (LDGSTS): issued now, waited for with cp_async_wait_all.
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {

@@ -283,7 +283,7 @@ bool make_input_map(const Geom& g, const UnitList& ul, int nu, CUtensorMap* map)
         q == cudaDriverEntryPointSuccess)
       encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
   });
-  if (!encode || (g.flags & TACTKV_FP32_IO) || g.head_dim % kChunk != 0) return false;
+  if (!encode || (g.flags & (TACTKV_FP32_IO | TACTKV_SKIP_S)) || g.head_dim % kChunk != 0) return false;
   const UnitDev& a = ul.u[g.unit0];
   const long long tok = a.tok_stride, hs = a.head_stride;
   if (tok * 2 % 16 || hs * 2 % 16 || reinterpret_cast<uintptr_t>(a.in) % 16) return false;

@@ -259,7 +259,8 @@ cudaError_t launch_grid(const Geom& g, const UnitList& ul, int nu, float* big, c
 cudaError_t TACTKV_CAT(launch_fused_inv_, TACTKV_FUSED_S)(const Geom& g, const UnitList& ul, int nu, float* big,
                                                           const uint32_t* index, const uint4* recs,
                                                           unsigned int* status, cudaStream_t st) {
-  if (g.S != TACTKV_FUSED_S || (g.flags & TACTKV_NO_QUANT) || tc_s_pass_disabled()) return cudaErrorNotSupported;
+  if (g.S != TACTKV_FUSED_S || (g.flags & (TACTKV_NO_QUANT | TACTKV_SKIP_S)) || tc_s_pass_disabled())
+    return cudaErrorNotSupported;
   if (g.H == 16 && g.W == 16) return launch_grid<16, 16>(g, ul, nu, big, index, recs, status, st);
   if (g.H == 14 && g.W == 14) return launch_grid<14, 14>(g, ul, nu, big, index, recs, status, st);
   if (g.H == 8 && g.W == 8) return launch_grid<8, 8>(g, ul, nu, big, index, recs, status, st);

@@ -91,6 +91,10 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const __grid_constan
   uint32_t* out = reinterpret_cast<uint32_t*>(pay + g.off_codes) + (size_t)(chunk * kChunk + lane) * sw;
   const float* xu = X + (size_t)u * g.N * g.n + chunk * kChunk + lane;
 
+  // the shared rotation R = H_32 diag(s) / sqrt(32) of each bin's 32 channels of this chunk
+  const bool rotate = g.flags & TACTKV_ROTATE;
+  const float rot_in = rotate ? rotation_sign((unsigned long long)(chunk * kChunk + lane)) : 1.f;
+
   const uint32_t A = rs[0].z;                                    // first bit of the range
   const uint32_t end_bit = r1 < nrec ? rs[r1 - r0].z : code_bits;
   const uint32_t first_word = (A + 31) >> 5;                     // words [first_word, stop_word) are ours
@@ -112,6 +116,11 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const __grid_constan
 #pragma unroll
     for (int j = 0; j < kBlock; ++j)
       if (e0 + j < m) x[j] = __ldcs(xu + (size_t)rs[e0 + j].x * g.n);
+    if (rotate) {
+#pragma unroll
+      for (int j = 0; j < kBlock; ++j)
+        if (e0 + j < m) x[j] = warp_wht(x[j] * rot_in, lane) * 0.17677669529663687f;
+    }
 #pragma unroll
     for (int j = 0; j < kBlock; ++j) {
       if (e0 + j >= m) break;

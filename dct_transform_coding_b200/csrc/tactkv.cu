@@ -110,7 +110,7 @@ namespace {
 
 tactkv_status make_geom(const tactkv_unit& u, Geom& g) {
   if (u.bits < 1 || u.bits > 8) return TACTKV_INVALID_ARG;
-  if (u.flags & ~(TACTKV_NO_QUANT | TACTKV_FP32_IO)) return TACTKV_INVALID_ARG;
+  if (u.flags & ~kAllFlags) return TACTKV_INVALID_ARG;
   if (u.S < 1 || u.H < 1 || u.W < 1 || u.heads < 1 || u.head_dim < 1) return TACTKV_INVALID_ARG;
   if (!supported_length(u.S) || !supported_length(u.H) || !supported_length(u.W)) return TACTKV_UNSUPPORTED_SHAPE;
   if (u.H > 32 || u.W > 32 || u.H * u.W > kMaxHW) return TACTKV_UNSUPPORTED_SHAPE;

@@ -34,6 +34,11 @@ TACTKV_TIMEOUT = 9
 
 TACTKV_NO_QUANT = 1
 TACTKV_FP32_IO = 2
+TACTKV_SKIP_S = 4
+TACTKV_SKIP_H = 8
+TACTKV_SKIP_W = 16
+TACTKV_UNIFORM_ALLOC = 32
+TACTKV_ROTATE = 64
 
 HEADER_BYTES = 64
 EXPORTED = ("tactkv_payload_bytes", "tactkv_workspace_bytes", "tactkv_compress", "tactkv_decompress",

@@ -26,7 +26,8 @@
  * recorded in the workspace and read back with tactkv_device_status().
  *
  * Payload format (version 1, little-endian), one self-describing blob per unit:
- *   [0, 64)             header: u32 magic 0x31564B54 ("TKV1"), u16 version = 1, u16 flags,
+ *   [0, 64)             header: u32 magic 0x31564B54 ("TKV1"), u16 version = 1, u16 flags (the
+ *                       unit's flags without TACTKV_FP32_IO),
  *                       i32 layer, kv, S, H, W, heads, head_dim, bits, u32 code_bits (sum b_i,
  *                       or 32*N with TACTKV_NO_QUANT), u32 chan_stride (bytes), u64 total_bytes,
  *                       u32 0, u32 0
@@ -68,6 +69,22 @@ typedef enum {
 /* flags */
 #define TACTKV_NO_QUANT 1u /* transform only: store float32 coefficients (lossless round trip) */
 #define TACTKV_FP32_IO  2u /* K/V are float32 instead of bfloat16 */
+/* Variants of the summary page's "Main Findings" ablations and of stage 4's shape rotation, all
+   recorded in the payload header (decompress must be given the same flags):
+     TACTKV_SKIP_S / _H / _W  no DCT along that axis (2-axis, 1-axis and no-DCT transforms);
+     TACTKV_UNIFORM_ALLOC     every bin with a nonzero variance gets the nominal bits (no
+                              water-filling; the total stays within the budget);
+     TACTKV_ROTATE            the fixed shared orthogonal rotation of each bin's shape vector before
+                              scalar quantization, undone after dequantization: block-diagonal over
+                              the 32-channel groups, H_32 diag(s) / sqrt(32) with H_32 the
+                              Sylvester-Hadamard matrix and s_c = -1 exactly when bit 63 of output c
+                              of SplitMix64 seeded with 0x544143544B56 is set (ignored with
+                              TACTKV_NO_QUANT).  Gains and allocation are unchanged by it. */
+#define TACTKV_SKIP_S        4u
+#define TACTKV_SKIP_H        8u
+#define TACTKV_SKIP_W       16u
+#define TACTKV_UNIFORM_ALLOC 32u
+#define TACTKV_ROTATE       64u
 
 typedef struct {
   int32_t layer;          /* recorded in the header, checked by decompress */
@@ -75,7 +92,7 @@ typedef struct {
   int32_t S, H, W;        /* token grid; lengths from the supported set below */
   int32_t heads, head_dim;/* n = heads*head_dim channels, n a multiple of 32, head_dim even */
   int32_t bits;           /* nominal bits per element, 1..8 */
-  uint32_t flags;         /* TACTKV_NO_QUANT | TACTKV_FP32_IO */
+  uint32_t flags;         /* TACTKV_NO_QUANT | TACTKV_FP32_IO | the variant flags above */
   const void* kv_in;      /* compress input: element (t, head, d) at
                              kv_in + t*token_stride + head*head_stride + d (elements) */
   void* kv_out;           /* decompress output, same indexing as kv_in */

@@ -54,13 +54,14 @@ def allocation_margin(var: np.ndarray, bits: int) -> float:
 def compare_unit(x: np.ndarray, gpu_payload: bytes, gpu_recon: np.ndarray, *, S, H, W, heads, head_dim, bits,
                  layer=0, kv=0, flags=0, io_round=O.to_bf16, report=None):
     """Check one unit.  x: the input exactly as the GPU saw it; gpu_recon: the GPU decode of gpu_payload."""
-    no_quant = bool(flags & 1)
-    p_o, info = O.compress_unit(x, S, H, W, heads, head_dim, bits, layer=layer, kv=kv, no_quant=no_quant,
-                                return_info=True)
+    pflags = flags & O.PAYLOAD_FLAGS
+    no_quant = bool(pflags & O.FLAG_NO_QUANT)
+    p_o, info = O.compress_unit(x, S, H, W, heads, head_dim, bits, layer=layer, kv=kv, return_info=True,
+                                flags=pflags)
     g = O.parse_payload(gpu_payload)
     assert (g["layer"], g["kv"], g["S"], g["H"], g["W"], g["heads"], g["head_dim"], g["bits"]) == \
         (layer, kv, S, H, W, heads, head_dim, bits)
-    assert bool(g["flags"] & 1) == no_quant
+    assert g["flags"] == pflags
     N = S * H * W
     var = info["var"]
     # gains: float32(sqrt(sigma^2)) from fp32 coefficients and fp64 sums
@@ -85,7 +86,7 @@ def compare_unit(x: np.ndarray, gpu_payload: bytes, gpu_recon: np.ndarray, *, S,
         assert b_g.sum() == g["code_bits"]
         _, codes_g = O.codes_of(gpu_payload)
         codes_o = info["codes"]
-        X = info["X"]
+        X = info["Xq"]                                  # the (rotated, when FLAG_ROTATE) coefficients coded
         same = np.nonzero((b_o == b_g) & (b_o > 0))[0]
         for i in same:
             bad = codes_g[i] != codes_o[i]

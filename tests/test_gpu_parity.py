@@ -303,6 +303,31 @@ def test_fused_grid_output_variants(S, H, W, flags, dtype):
         assert rel_rms(y.double().cpu(), x.double().cpu()) <= 1e-5
 
 
+# ---------------------------------------------------------------- ablation and rotation flags ---
+@pytest.mark.parametrize("shape", [(16, 16, 16, 2, 64), (5, 7, 6, 1, 96)], ids=["fused-grid", "ragged-grid"])
+@pytest.mark.parametrize("variant", ["no_dct", "hw_only", "s_only", "w_only", "uniform", "rotate",
+                                     "rotate_uniform_hw"])
+def test_variant_flags(shape, variant):
+    """The summary page's ablations ("Main Findings": fewer transformed axes, uniform allocation)
+    and stage 4's fixed shared rotation, as flags: payload, codes and reconstruction against the
+    oracle run with the same flags."""
+    flags = {"no_dct": T.TACTKV_SKIP_S | T.TACTKV_SKIP_H | T.TACTKV_SKIP_W, "hw_only": T.TACTKV_SKIP_S,
+             "s_only": T.TACTKV_SKIP_H | T.TACTKV_SKIP_W, "w_only": T.TACTKV_SKIP_S | T.TACTKV_SKIP_H,
+             "uniform": T.TACTKV_UNIFORM_ALLOC, "rotate": T.TACTKV_ROTATE,
+             "rotate_uniform_hw": T.TACTKV_ROTATE | T.TACTKV_UNIFORM_ALLOC | T.TACTKV_SKIP_S}[variant]
+    S, H, W, heads, D = shape
+    x = torch.stack([make_unit(S, H, W, heads, D, rho=(0.9, 0.85, 0.8), nu=4.0, seed=300 + i, device=DEV)
+                     for i in range(2)])
+    reports, pay, _ = _check_batch(x, S, H, W, 2, layers=[0, 1], kvs=[1, 1], flags=flags)
+    p = O.parse_payload(pay[0].cpu().numpy().tobytes())
+    assert p["flags"] == flags
+    if flags & T.TACTKV_UNIFORM_ALLOC:
+        assert set(np.unique(p["b"])) <= {0, 2}
+    # decoding with other flags than the payload's is refused
+    with pytest.raises(T.TactkvError):
+        T.decompress(pay, S, H, W, 2, heads=heads, head_dim=D, layers=[0, 1], kvs=[1, 1], flags=0, check=True)
+
+
 # ------------------------------------------------------------------------------ exact ties ---
 def _gpu_allocation(var, grid, bits):
     S, H, W = grid
