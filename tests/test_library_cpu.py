@@ -75,7 +75,7 @@ def _unit(T, **kw):
 
 @pytest.mark.parametrize("kw,status", [
     (dict(bits=0), "TACTKV_INVALID_ARG"), (dict(bits=9), "TACTKV_INVALID_ARG"),
-    (dict(flags=8), "TACTKV_INVALID_ARG"), (dict(S=0), "TACTKV_INVALID_ARG"),
+    (dict(flags=128), "TACTKV_INVALID_ARG"), (dict(S=0), "TACTKV_INVALID_ARG"),
     (dict(kv_in=None), "TACTKV_INVALID_ARG"), (dict(payload=None), "TACTKV_INVALID_ARG"),
     (dict(token_stride=0), "TACTKV_INVALID_ARG"),
     (dict(S=17), "TACTKV_UNSUPPORTED_SHAPE"), (dict(head_dim=30), "TACTKV_UNSUPPORTED_SHAPE"),
