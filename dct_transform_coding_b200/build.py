@@ -37,6 +37,7 @@ UNITS = [
     ("fused_inv_32", "fused_inv.cu", ["-DTACTKV_FUSED_S=32"]),
     ("fused_inv_64", "fused_inv.cu", ["-DTACTKV_FUSED_S=64"]),
     ("allocate", "allocate.cu", []),
+    ("attention", "attention.cu", []),
     ("pack", "pack.cu", []),
     ("tactkv", "tactkv.cu", []),
 ]

@@ -75,6 +75,7 @@ inline bool supported_length(int L) {
   }
 }
 inline int length_class(int L) { return L <= 16 ? 16 : (L <= 32 ? 32 : 64); }
+__host__ __device__ inline int length_class_dev(int L) { return L <= 16 ? 16 : (L <= 32 ? 32 : 64); }
 
 // TACTKV_SIMT_S=1 in the environment keeps the S-axis DCT of the fused forward kernel on the
 // CUDA cores (the cp.async form) instead of the tensor cores; read once per process.

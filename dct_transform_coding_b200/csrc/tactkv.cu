@@ -98,6 +98,13 @@ void axis_hw_shape(int hcls, int wcls, const Geom& g, bool inverse, int mode, si
   return axis_hw_shape_32_32(g, inverse, mode, smem, threads);
 }
 
+size_t attention_scores_smem(const Geom& g, int q_heads);
+size_t attention_values_smem(const Geom& g, int q_heads);
+cudaError_t launch_attention(const Geom& g, const UnitList& kl, const UnitList& vl, int nu, int q_heads,
+                             const uint32_t* kidx, const uint4* krec, const uint32_t* vidx, const uint4* vrec,
+                             const float* q, float* zp, float* part, float* out, float* m, float* l,
+                             cudaStream_t st);
+
 bool tc_s_pass_disabled() {
   static const bool off = [] {
     const char* e = getenv("TACTKV_SIMT_S");
@@ -450,6 +457,100 @@ tactkv_status tactkv_allocate(const tactkv_unit* unit, const double* var, void* 
     return TACTKV_CUDA;
   t_launches = 1;
   if (launch_allocate_from_var(g, ul, 1, w.var, w.index, w.recs, stream) != cudaSuccess) return TACTKV_CUDA;
+  return TACTKV_OK;
+}
+
+// ------------------------------------------------------------------ decode-time attention ---
+namespace {
+constexpr int kAttnMaxUnits = kMaxUnits / 2;   // K and V index blocks of one call share one launch
+
+struct AttnWs {
+  unsigned int* status;
+  uint32_t* index;   // 2 nu index blocks: K units, then V units
+  uint4* recs;       // 2 nu * N dense records
+  float* zp;         // nu * q_heads * N: z, then dct3(p)
+  float* part;       // nu * S * q_heads * head_dim
+  size_t total;
+};
+AttnWs attn_view(unsigned char* ws, const Geom& g, int nu, int q_heads) {
+  AttnWs a;
+  size_t off = kStatusBytes;
+  a.status = reinterpret_cast<unsigned int*>(ws);
+  a.index = reinterpret_cast<uint32_t*>(ws + off);
+  off += round256((size_t)2 * nu * unit_index_words(g.S) * 4);
+  a.recs = reinterpret_cast<uint4*>(ws + off);
+  off += round256((size_t)2 * nu * g.N * 16);
+  a.zp = reinterpret_cast<float*>(ws + off);
+  off += round256((size_t)nu * q_heads * g.N * 4);
+  a.part = reinterpret_cast<float*>(ws + off);
+  off += round256((size_t)nu * g.S * q_heads * g.head_dim * 4);
+  a.total = off;
+  return a;
+}
+tactkv_status attn_check(const tactkv_unit* k_units, const tactkv_unit* v_units, int n_units, int q_heads,
+                         Geom& g) {
+  if (n_units < 1 || n_units > kAttnMaxUnits || !k_units || !v_units) return TACTKV_INVALID_ARG;
+  tactkv_status st = make_geom(k_units[0], g);
+  if (st != TACTKV_OK) return st;
+  if ((g.flags & TACTKV_NO_QUANT) || q_heads < g.heads || q_heads % g.heads || q_heads / g.heads > 16 ||
+      g.head_dim % kChunk)
+    return TACTKV_UNSUPPORTED_SHAPE;
+  if ((size_t)g.N * 4 > 227 * 1024 || attention_scores_smem(g, q_heads) > 227 * 1024 ||
+      attention_values_smem(g, q_heads) > 227 * 1024)
+    return TACTKV_UNSUPPORTED_SHAPE;
+  long long cap = -1;
+  for (int i = 0; i < n_units; ++i)
+    for (const tactkv_unit* u : {&k_units[i], &v_units[i]}) {
+      if (!same_group(k_units[0], *u)) return TACTKV_INVALID_ARG;
+      if (!u->payload) return TACTKV_INVALID_ARG;
+      if (reinterpret_cast<uintptr_t>(u->payload) % 16) return TACTKV_ALIGNMENT;
+      if (u->payload_capacity < payload_bytes_geom(g)) return TACTKV_CAPACITY;
+      cap = cap < 0 ? (long long)u->payload_capacity : std::min(cap, (long long)u->payload_capacity);
+    }
+  g.capacity = cap;
+  return TACTKV_OK;
+}
+}  // namespace
+
+size_t tactkv_attention_workspace_bytes(const tactkv_unit* k_units, int n_units, int q_heads) {
+  Geom g;
+  if (!k_units || n_units < 1 || make_geom(k_units[0], g) != TACTKV_OK || q_heads < 1) return 0;
+  return attn_view(nullptr, g, n_units, q_heads).total;
+}
+
+tactkv_status tactkv_attention_decode(const tactkv_unit* k_units, const tactkv_unit* v_units, int n_units,
+                                      int q_heads, const float* q, float* out, float* m, float* l,
+                                      void* workspace, size_t workspace_bytes, struct CUstream_st* stream) {
+  t_launches = 0;
+  Geom g;
+  tactkv_status st = attn_check(k_units, v_units, n_units, q_heads, g);
+  if (st != TACTKV_OK) return st;
+  if (!q || !out || !m || !l) return TACTKV_INVALID_ARG;
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256) return TACTKV_WORKSPACE;
+  const AttnWs a = attn_view(static_cast<unsigned char*>(workspace), g, n_units, q_heads);
+  if (workspace_bytes < a.total) return TACTKV_WORKSPACE;
+  UnitList both, kl, vl;
+  memset(&both, 0, sizeof(both));
+  memset(&kl, 0, sizeof(kl));
+  memset(&vl, 0, sizeof(vl));
+  for (int i = 0; i < n_units; ++i) {
+    for (int side = 0; side < 2; ++side) {
+      const tactkv_unit& s = side ? v_units[i] : k_units[i];
+      UnitDev d;
+      memset(&d, 0, sizeof(d));
+      d.payload = static_cast<unsigned char*>(s.payload);
+      d.layer = s.layer;
+      d.kv = s.kv;
+      both.u[side * n_units + i] = d;
+      (side ? vl : kl).u[i] = d;
+    }
+  }
+  t_launches = 5;   // decode_index (K and V), scores, softmax, values, reduce
+  if (launch_decode_index(g, both, 2 * n_units, a.index, a.recs, a.status, stream) != cudaSuccess) return TACTKV_CUDA;
+  const size_t iw = unit_index_words(g.S);
+  if (launch_attention(g, kl, vl, n_units, q_heads, a.index, a.recs, a.index + n_units * iw,
+                       a.recs + (size_t)n_units * g.N, q, a.zp, a.part, out, m, l, stream) != cudaSuccess)
+    return TACTKV_CUDA;
   return TACTKV_OK;
 }
 

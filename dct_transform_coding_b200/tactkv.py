@@ -44,6 +44,7 @@ HEADER_BYTES = 64
 EXPORTED = ("tactkv_payload_bytes", "tactkv_workspace_bytes", "tactkv_compress", "tactkv_decompress",
             "tactkv_compress_profiled", "tactkv_decompress_profiled", "tactkv_compress_noalloc",
             "tactkv_allocate", "tactkv_device_status", "tactkv_occupancy", "tactkv_max_batch",
+            "tactkv_attention_workspace_bytes", "tactkv_attention_decode",
             "tactkv_status_string", "tactkv_lloyd_max_table", "tactkv_format_version", "tactkv_last_launches")
 
 
@@ -88,6 +89,12 @@ _lib.tactkv_occupancy.restype = ctypes.c_int
 _lib.tactkv_occupancy.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(tactkv_occupancy_t)]
 _lib.tactkv_max_batch.restype = ctypes.c_int64
 _lib.tactkv_max_batch.argtypes = [ctypes.c_uint64, ctypes.c_uint64, ctypes.c_uint64]
+_lib.tactkv_attention_workspace_bytes.restype = ctypes.c_size_t
+_lib.tactkv_attention_workspace_bytes.argtypes = [_P, ctypes.c_int, ctypes.c_int]
+_lib.tactkv_attention_decode.restype = ctypes.c_int
+_lib.tactkv_attention_decode.argtypes = [_P, _P, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                         ctypes.c_void_p]
 _lib.tactkv_status_string.restype = ctypes.c_char_p
 _lib.tactkv_status_string.argtypes = [ctypes.c_int]
 _lib.tactkv_lloyd_max_table.restype = ctypes.c_int
@@ -331,3 +338,38 @@ def decompress(payload: torch.Tensor, S: int, H: int, W: int, bits: int, *, head
         if ds != TACTKV_OK:
             raise TactkvError(ds, "tactkv_decompress (device)")
     return out
+
+
+def attention_decode(q: torch.Tensor, k_payload: torch.Tensor, v_payload: torch.Tensor, S: int, H: int, W: int,
+                     bits: int, *, heads: int, head_dim: int, layers=None, flags: int = 0,
+                     workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None,
+                     check: bool = False):
+    """One decode step of attention over compressed K/V: q [units, q_heads, head_dim] float32 on the
+    GPU, k_payload / v_payload [units, capacity] (compressed with kv 0 / 1).  Returns (out, m, l):
+    out [units, q_heads, head_dim] = softmax(q K^T / sqrt(head_dim)) V over the visual tokens, m and
+    l the scores' maximum and exp-sum per query head."""
+    U, q_heads, D = q.shape
+    q = q.contiguous().to(torch.float32)
+    ku = make_units(None, S, H, W, bits, heads=heads, head_dim=head_dim, payload=k_payload, layers=layers,
+                    kvs=[0] * U, flags=flags, n_units=U)
+    vu = make_units(None, S, H, W, bits, heads=heads, head_dim=head_dim, payload=v_payload, layers=layers,
+                    kvs=[1] * U, flags=flags, n_units=U)
+    out = torch.empty((U, q_heads, D), dtype=torch.float32, device=q.device)
+    m = torch.empty((U, q_heads), dtype=torch.float32, device=q.device)
+    l = torch.empty((U, q_heads), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        nbytes = int(_lib.tactkv_attention_workspace_bytes(ku, U, q_heads))
+        ws = torch.zeros(nbytes + 256, dtype=torch.uint8, device=q.device)
+        off = (-ws.data_ptr()) % 256
+        workspace = ws[off:off + nbytes]
+    st = int(_lib.tactkv_attention_decode(ku, vu, U, q_heads, ctypes.c_void_p(q.data_ptr()),
+                                          ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(m.data_ptr()),
+                                          ctypes.c_void_p(l.data_ptr()), ctypes.c_void_p(workspace.data_ptr()),
+                                          workspace.numel(), ctypes.c_void_p(_stream_ptr(stream))))
+    if st != TACTKV_OK:
+        raise TactkvError(st, "tactkv_attention_decode")
+    if check:
+        ds = tactkv_device_status(workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+        if ds != TACTKV_OK:
+            raise TactkvError(ds, "tactkv_attention_decode (device)")
+    return out, m, l

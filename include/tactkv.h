@@ -174,6 +174,27 @@ tactkv_status tactkv_compress_noalloc(const tactkv_unit* units, int n_units,
 tactkv_status tactkv_allocate(const tactkv_unit* unit, const double* var, void* workspace,
                               size_t workspace_bytes, struct CUstream_st* stream);
 
+/* One decode step of attention over compressed visual K/V (the paragraph after stage 4: decoding
+   runs inside the attention computation and the reconstructed cache never exists).  Unit i of
+   k_units / v_units is the K / V payload of one (sequence, layer); all 2*n_units descriptors have
+   the same shape, bits and flags (quantized, not TACTKV_NO_QUANT), and each unit's kv field must
+   match its payload.  Only the payload pointers and the shape fields are read.
+     q_heads   query heads, a multiple G of the K/V heads (G <= 16); query head j reads K/V head j/G;
+     q         DEVICE float32 [n_units][q_heads][head_dim], the decode step's queries;
+     out       DEVICE float32 [n_units][q_heads][head_dim]:
+                 out_j = sum_t softmax_t(q_j . K[t] / sqrt(head_dim)) V[t] over the S*H*W visual tokens;
+     m, l      DEVICE float32 [n_units][q_heads]: the scores' maximum and sum_t exp(score - m), so
+               that a caller can merge these tokens with its bf16 text tokens.
+   Limits: n_units <= 128, S*H*W <= 58112, head_dim a multiple of 32.  workspace: at least
+   tactkv_attention_workspace_bytes(k_units, n_units, q_heads) bytes, 256-byte aligned.  A corrupt
+   payload is recorded as TACTKV_CORRUPT_PAYLOAD (tactkv_device_status) and contributes no
+   tokens of its unit.  Asynchronous on `stream`; 5 kernels. */
+size_t tactkv_attention_workspace_bytes(const tactkv_unit* k_units, int n_units, int q_heads);
+tactkv_status tactkv_attention_decode(const tactkv_unit* k_units, const tactkv_unit* v_units, int n_units,
+                                      int q_heads, const float* q, float* out, float* m, float* l,
+                                      void* workspace, size_t workspace_bytes,
+                                      struct CUstream_st* stream);
+
 /* Synchronizes `stream`, returns the first error the kernels recorded in `workspace` since the
    previous call (TACTKV_OK if none), and clears it. */
 tactkv_status tactkv_device_status(void* workspace, size_t workspace_bytes,

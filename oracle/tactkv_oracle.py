@@ -488,6 +488,37 @@ def decompress_unit(payload) -> np.ndarray:
     return x.reshape(N, p["heads"], p["head_dim"])
 
 
+def attention_decode(q: np.ndarray, payload_k, payload_v):
+    """One decode step of attention over a compressed visual K/V (the paragraph after stage 4:
+    decoding can run inside the attention kernel, so the reconstructed cache never exists).
+
+    The plain definition on the decompressed cache: for query head j (q[j], of head_dim D) and its
+    key/value head j // G (G = query heads per K/V head),
+        s_j[t] = q_j . K[t] / sqrt(D),  m_j = max_t s_j[t],  l_j = sum_t exp(s_j[t] - m_j),
+        out_j  = sum_t exp(s_j[t] - m_j) V[t] / l_j,
+    over the unit's T = S*H*W visual tokens, K and V the fp64 reconstructions of the payloads.
+    Returns (out [Hq, D], m [Hq], l [Hq]); m and l let a caller merge these tokens with others."""
+    pk, pv = parse_payload(payload_k), parse_payload(payload_v)
+    K = decompress_unit(payload_k)            # [T, kv_heads, D]
+    V = decompress_unit(payload_v)
+    kv_heads, D = pk["heads"], pk["head_dim"]
+    assert (pv["heads"], pv["head_dim"]) == (kv_heads, D)
+    q = np.asarray(q, dtype=np.float64)
+    Hq = q.shape[0]
+    G = Hq // kv_heads
+    out = np.zeros((Hq, D))
+    m = np.zeros(Hq)
+    l = np.zeros(Hq)
+    for j in range(Hq):
+        h = j // G
+        sc = K[:, h, :] @ q[j] / math.sqrt(D)
+        m[j] = sc.max()
+        e = np.exp(sc - m[j])
+        l[j] = e.sum()
+        out[j] = e @ V[:, h, :] / l[j]
+    return out, m, l
+
+
 def codes_of(payload) -> Tuple[np.ndarray, np.ndarray]:
     """(b[N], codes[N, n]) decoded from a payload (for code-level parity checks)."""
     p = parse_payload(payload)

@@ -429,3 +429,45 @@ def test_uniform_allocation_and_theorem1_through_the_codec():
     v = O.bin_variances(X)
     inv_gamma = np.mean(v) / math.exp(np.mean(np.log(v)))
     assert abs(d["uniform"] / d["wf"] / inv_gamma - 1) < 0.1
+
+
+# ------------------------------------------------------------------- decode-time attention ---
+def test_attention_decode_matches_torch_sdpa():
+    """The oracle's attention over a compressed cache equals torch's scaled_dot_product_attention
+    (fp64, grouped query heads expanded) applied to the decompressed K and V."""
+    import torch
+    S, H, W, kv_heads, D, G = 4, 3, 5, 2, 32, 3
+    rng = np.random.default_rng(5)
+    k = rng.standard_normal((S * H * W, kv_heads, D))
+    v = rng.standard_normal((S * H * W, kv_heads, D))
+    pk = O.compress_unit(k, S, H, W, kv_heads, D, 3)
+    pv = O.compress_unit(v, S, H, W, kv_heads, D, 3, kv=1)
+    q = rng.standard_normal((kv_heads * G, D))
+    out, m, l = O.attention_decode(q, pk, pv)
+    K = torch.from_numpy(O.decompress_unit(pk)).permute(1, 0, 2).repeat_interleave(G, 0)   # [Hq, T, D]
+    V = torch.from_numpy(O.decompress_unit(pv)).permute(1, 0, 2).repeat_interleave(G, 0)
+    ref = torch.nn.functional.scaled_dot_product_attention(torch.from_numpy(q)[:, None, :], K, V)[:, 0, :]
+    assert np.allclose(out, ref.numpy(), atol=1e-12, rtol=1e-12)
+    s = torch.einsum("hd,htd->ht", torch.from_numpy(q), K) / math.sqrt(D)
+    assert np.allclose(m, s.max(dim=1).values.numpy(), atol=1e-12)
+    assert np.allclose(l, torch.exp(s - s.max(dim=1, keepdim=True).values).sum(1).numpy(), rtol=1e-12)
+
+
+def test_attention_decode_special_cases():
+    """A zero query attends uniformly (the output is the mean of the value rows, l = T); a query
+    that picks one token out by a large margin returns that token's value row."""
+    S, H, W, D = 2, 2, 4, 32
+    T = S * H * W
+    rng = np.random.default_rng(6)
+    v = rng.standard_normal((T, 1, D))
+    pv = O.compress_unit(v, S, H, W, 1, D, 8, kv=1)
+    Vh = O.decompress_unit(pv)[:, 0, :]
+    k = np.zeros((T, 1, D))
+    k[5, 0, 0] = 1.0
+    pk = O.compress_unit(k, S, H, W, 1, D, 8, no_quant=True)      # exact keys (float32 coefficients)
+    out, m, l = O.attention_decode(np.zeros((1, D)), pk, pv)
+    assert np.allclose(out[0], Vh.mean(axis=0), atol=1e-12) and abs(l[0] - T) < 1e-9
+    q = np.zeros((1, D))
+    q[0, 0] = 400.0 * math.sqrt(D)
+    out, m, l = O.attention_decode(q, pk, pv)
+    assert np.allclose(out[0], Vh[5], atol=1e-9) and abs(l[0] - 1) < 1e-9
