@@ -46,6 +46,8 @@ def parse_args():
     ap.add_argument("--e2e-streams", type=int, default=4, help="streams (each with a workspace) in the e2e run")
     ap.add_argument("--units", type=int, default=None, help="use only the first U units of the batch (profiling)")
     ap.add_argument("--no-others", action="store_true", help="skip the other workloads' lines")
+    ap.add_argument("--no-attention", action="store_true", help="skip the decode-time attention measurement")
+    ap.add_argument("--q-per-kv", type=int, default=2, help="query heads per K/V head in the attention step")
     ap.add_argument("--other-units", type=int, default=128, help="units of each other workload measured")
     return ap.parse_args()
 
@@ -306,6 +308,9 @@ def main():
         "clocks": clocks,
     }
 
+    if rank == 0 and not args.no_attention and len(set(kvs)) == 2:
+        result["attention_decode"] = attention_bench(T, w, bits, payload, out, du, ws, stream, layers, kvs, peak,
+                                                     peak_kind, q_per_kv=args.q_per_kv)
     if not args.no_e2e:
         result["e2e"] = e2e_run(args, T, x, payload, out, cu, du, ws, stream, world)
     del x, out, payload, ws
@@ -319,6 +324,54 @@ def main():
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(result), flush=True)
+
+
+def attention_bench(T, w, bits, payload, out, du, ws, stream, layers, kvs, peak, peak_kind, q_per_kv=2, iters=20):
+    """One decode step of attention for every layer of the batch, straight from the compressed K/V
+    (units with kv 0 / 1 of the same layer), against the same step done by decompressing the batch
+    to bf16 and running torch's scaled_dot_product_attention on it.  The roofline counts the bytes
+    the step must read (the K and V payloads, the queries) and write (outputs, m, l)."""
+    import torch
+    ki = [i for i, kv in enumerate(kvs) if kv == 0]
+    vi = [i for i, kv in enumerate(kvs) if kv == 1]
+    ki, vi = ki[:min(len(ki), len(vi), 128)], vi[:min(len(ki), len(vi), 128)]
+    U = len(ki)
+    dev = payload.device
+    Hq, D = w.heads * q_per_kv, w.head_dim
+    q = torch.randn((U, Hq, D), device=dev, generator=torch.Generator(device=dev).manual_seed(17))
+    pk, pv = payload[ki].contiguous(), payload[vi].contiguous()
+    lay = [layers[i] for i in ki]
+    T.attention_decode(q, pk, pv, w.S, w.H, w.W, bits, heads=w.heads, head_dim=D, layers=lay, check=True)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for _ in range(iters):
+        T.attention_decode(q, pk, pv, w.S, w.H, w.W, bits, heads=w.heads, head_dim=D, layers=lay)
+    ev[1].record(stream)
+    sp = int(stream.cuda_stream)
+    qh = q.to(torch.bfloat16)[:, :, None, :]
+    for _ in range(3):
+        T.tactkv_decompress(du, ws.data_ptr(), ws.numel(), sp)
+    ev[2].record(stream)
+    for _ in range(iters):
+        T.tactkv_decompress(du, ws.data_ptr(), ws.numel(), sp)
+        K = out[ki].permute(0, 2, 1, 3)             # [U, heads, T, D]
+        V = out[vi].permute(0, 2, 1, 3)
+        torch.nn.functional.scaled_dot_product_attention(qh, K, V, enable_gqa=True)
+    ev[3].record(stream)
+    torch.cuda.synchronize()
+    ms = ev[0].elapsed_time(ev[1]) / iters
+    ms_ref = ev[2].elapsed_time(ev[3]) / iters
+    hdr = torch.cat([pk, pv])[:, :64].cpu().numpy()
+    pay_bytes = int(sum(int.from_bytes(bytes(h[48:56]), "little") for h in hdr))
+    alg = pay_bytes + q.numel() * 4 + U * Hq * (D + 2) * 4
+    kv_bf16 = 2 * U * w.tokens * w.channels * 2
+    return {"layers": U, "q_heads": Hq, "ms_per_step": round(ms, 4),
+            "ms_decompress_then_sdpa": round(ms_ref, 4), "speedup": round(ms_ref / ms, 2),
+            "kv_bf16_bytes_served": kv_bf16, "value": round(kv_bf16 / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+            "roofline": {"bound": "hbm", "algorithmic_bytes": alg,
+                         "achieved": round(alg / (ms * 1e-3) / 1e9, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(alg / (ms * 1e-3) / 1e9 / peak, 4), "peak_kind": peak_kind}}
 
 
 STAGES_C = ["forward", "allocate", "pack"]          # compress: DCTs with energies, allocation, packing
