@@ -332,6 +332,7 @@ def attention_bench(T, w, bits, payload, out, du, ws, stream, layers, kvs, peak,
     to bf16 and running torch's scaled_dot_product_attention on it.  The roofline counts the bytes
     the step must read (the K and V payloads, the queries) and write (outputs, m, l)."""
     import torch
+    kvs = kvs[:payload.shape[0]]
     ki = [i for i, kv in enumerate(kvs) if kv == 0]
     vi = [i for i, kv in enumerate(kvs) if kv == 1]
     ki, vi = ki[:min(len(ki), len(vi), 128)], vi[:min(len(ki), len(vi), 128)]
