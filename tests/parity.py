@@ -8,7 +8,12 @@ Acceptance, per unit (the codec's stated tolerances, with the readings needed to
 * quantization codes equal the oracle's, except where the oracle's scaled coefficient
   u = X / sigma lies within 1e-5 * max(1, |t|) of a decision threshold t (distance taken in
   sigma-scaled units, because the middle threshold is 0);
-* reconstructions: ||y_gpu - y_oracle|| / ||y_oracle|| <= 1e-3, both rounded to the I/O type;
+* reconstructions: ||y_gpu - y_ref|| / ||y_ref|| <= 1e-3, both rounded to the I/O type, where y_ref
+  is the oracle's decode of the GPU's own payload (so the decoder is compared on identical codes).
+  The end-to-end figure against the oracle's own payload is asserted as well whenever the two
+  payloads hold identical codes; a code inside the band moves one coefficient by about one
+  quantization step, which in a small unit is alone above 1e-3 (one coefficient of 20,000 is
+  already a relative RMS near 7e-3), so with band codes present it is only reported;
 * with TACTKV_NO_QUANT the round trip matches the input within 1e-5 relative RMS.
 """
 from __future__ import annotations
@@ -99,7 +104,13 @@ def compare_unit(x: np.ndarray, gpu_payload: bytes, gpu_recon: np.ndarray, *, S,
     y_o = io_round(O.decompress_unit(p_o)).reshape(gpu_recon.shape)
     err = rel_rms(gpu_recon, y_o)
     out["recon_rel_rms"] = err
-    assert err <= (ROUNDTRIP_TOL if no_quant else RECON_TOL), f"reconstruction rel RMS {err}"
+    if no_quant or out["code_mismatch_band"] == 0:
+        assert err <= (ROUNDTRIP_TOL if no_quant else RECON_TOL), f"reconstruction rel RMS {err}"
+    if not no_quant:
+        y_same = io_round(O.decompress_unit(gpu_payload)).reshape(gpu_recon.shape)
+        err_same = rel_rms(gpu_recon, y_same)
+        out["decode_rel_rms"] = err_same
+        assert err_same <= RECON_TOL, f"decoder rel RMS {err_same} on the same payload"
     if report is not None:
         report.append(out)
     return out
