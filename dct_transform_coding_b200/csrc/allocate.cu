@@ -21,8 +21,10 @@
 //
 // The kernel also writes the first stream bit P(k_s) of every S slab (the same for every
 // channel) and the list of bins with bits (records {bin, bits, first stream bit, 1/sigma}, in bin
-// order) into the workspace, for the packing kernel.  decode_index_kernel rebuilds P from a
-// payload before decoding and checks the header and the bit widths.
+// order) into the workspace, and zeroes the stream word where each packing range of kPackRecs
+// records starts and the word of the last code bit: the packing kernel ORs the words it shares
+// with a neighbouring range into those.  decode_index_kernel rebuilds P from a payload before
+// decoding and checks the header and the bit widths.
 #include "common.cuh"
 
 namespace tactkv {
@@ -120,6 +122,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
   __shared__ uint32_t s_nzslab[kMaxSlabs];
   __shared__ uint32_t s_P[kMaxSlabs + 1];
   __shared__ uint32_t s_NZ[kMaxSlabs + 1];
+  __shared__ uint32_t s_bpos[kMaxN / kPackRecs + 1];
   __shared__ uint32_t s_hist[kExpBuckets], s_rev[kExpBuckets];
   __shared__ int s_pick;
   __shared__ uint32_t s_above, s_count;
@@ -309,9 +312,21 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
       const uint2 sb = reinterpret_cast<const uint2*>(var)[i];   // {sigma_i, b_i} of this thread's bins
       const uint32_t b = sb.y;
       if (b) {
+        if (slot % kPackRecs == 0) s_bpos[slot / kPackRecs] = pos;   // a packing range starts here
         urecs[slot++] = make_uint4((uint32_t)i, b, pos, __float_as_uint(__frcp_rn(__uint_as_float(sb.x))));
         pos += b;
       }
+    }
+    __syncthreads();
+    // zero the stream word where each packing range starts and the word holding the last code bit:
+    // neighbouring ranges OR their bits into them
+    const uint32_t sw = (uint32_t)(cstride / 4), nrec = s_NZ[g.S];
+    const uint32_t nb = (nrec + kPackRecs - 1) / kPackRecs;
+    uint32_t* words = reinterpret_cast<uint32_t*>(pay + g.off_codes);
+    for (uint32_t k = 0; k <= nb; ++k) {
+      const uint32_t w = (k < nb ? s_bpos[k] : s_P[g.S]) >> 5;
+      if (w < sw)
+        for (int c = threadIdx.x; c < g.n; c += blockDim.x) words[(size_t)c * sw + w] = 0u;
     }
   }
   if (threadIdx.x == 0) {

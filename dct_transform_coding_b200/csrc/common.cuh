@@ -25,6 +25,7 @@ constexpr size_t kStatusBytes = 256;       // status word at the start of the wo
 constexpr int kMaxHW = 1024;               // H*W limit of the H/W-axis kernels
 constexpr int kMaxSlabs = 64;              // S limit
 constexpr int kMaxN = kMaxSlabs * kMaxHW;  // bins per unit limit
+constexpr int kPackRecs = 1024;            // records per packing range (one CTA)
 
 enum HwMode { kStats = 0, kQuant = 1, kRaw = 2 };
 
@@ -78,8 +79,11 @@ inline int length_class(int L) { return L <= 16 ? 16 : (L <= 32 ? 32 : 64); }
 __host__ __device__ inline int length_class_dev(int L) { return L <= 16 ? 16 : (L <= 32 ? 32 : 64); }
 
 // TACTKV_SIMT_S=1 in the environment keeps the S-axis DCT of the fused forward kernel on the
-// CUDA cores (the cp.async form) instead of the tensor cores; read once per process.
+// CUDA cores (the cp.async form) instead of the tensor cores; TACTKV_FUSED_DECODE=1 decodes with
+// the single fused kernel (inverse S on the tensor cores) instead of the two inverse kernels.
+// Both are read once per process.
 bool tc_s_pass_disabled();
+bool fused_decode_enabled();
 
 
 // --------------------------------------------------------------------------------- launchers ---

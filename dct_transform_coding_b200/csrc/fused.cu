@@ -114,7 +114,7 @@ struct TcS {
   static constexpr int kABytes = kTcCells * L * 64;      // one input tile
   static constexpr int kBBytes = L * 128;                // one limb of C, rows padded to 128 bytes
   static constexpr int kSmem = 3 * kBBytes + 2 * kABytes + 1024;   // + alignment slack
-  static constexpr int kCols = L < 32 ? 32 : L;          // TMEM columns (power of two >= 32)
+  static constexpr int kCols = L < 32 ? 32 : L;          // TMEM columns of one accumulator (power of two >= 32)
   static constexpr int kHalf = L / 2;                    // columns read per thread
 };
 
@@ -125,9 +125,17 @@ __device__ __forceinline__ const uint16_t* dct_limb_fwd() {
   else return &kDctLimbFwd64[0][0][0];
 }
 
-// S pass of one (unit u, chunk) on this CTA's tiles t = r, r + kCluster, ... into Y.  Returns
-// false (and records TACTKV_TIMEOUT) if a copy or an MMA did not complete; the caller still takes
-// part in every barrier of the cluster.  Called by every thread of the CTA.
+// S pass of one (unit u, chunk) on this CTA's tiles t = r, r + kCluster, ... into Y, pipelined:
+//   warp 0 (one lane)  TMA producer and MMA issuer: the input tiles go through two shared-memory
+//                      stages, the products into two TMEM accumulators (64 columns each), so the
+//                      MMAs of a tile run while the epilogue drains the previous one;
+//   warps 4..7         epilogue: warp 4 + q reads lanes 32q.. (cell q of the tile) of a finished
+//                      accumulator, frees it, and stores the S values to Y;
+//   warps 1..3         idle until the H/W pass.
+// mbarriers: full[s] (TMA -> MMA, transaction bytes), done[a] (MMA commit -> epilogue and producer),
+// freed[a] (4 epilogue warps -> MMA).  Every wait is bounded; on expiry the CTA records
+// TACTKV_TIMEOUT, waits (bounded) for what is in flight, releases TMEM and returns false.  The
+// caller still takes part in every barrier of the cluster.  Called by every thread of the CTA.
 template <int L, int HWX>
 __device__ bool fdct_s_tc(const Geom& g, int u, int chunk, int r, const CUtensorMap* tmap, float* __restrict__ Y,
                           unsigned char* smem, uint64_t* bars, uint32_t* tmem_slot, int nx, unsigned int* status) {
@@ -138,8 +146,10 @@ __device__ bool fdct_s_tc(const Geom& g, int u, int chunk, int r, const CUtensor
   const int uw = u - g.unit0;   // the tensor map's unit coordinate: the unit's place in the wave
   unsigned char* sB = smem;
   unsigned char* sA = smem + 3 * P::kBBytes;
-  uint64_t* tma_bar = bars;       // [2]
-  uint64_t* mma_bar = bars + 2;
+  uint64_t* full = bars;          // [2]
+  uint64_t* done = bars + 2;      // [2]
+  uint64_t* freed = bars + 4;     // [2]
+  __shared__ int s_err;
   const int mine = r < kTiles ? (kTiles - r + kCluster - 1) / kCluster : 0;
 
   // B: the three limbs of C, swizzled (16-byte chunk j of row k at chunk j ^ (k & 7))
@@ -153,78 +163,105 @@ __device__ bool fdct_s_tc(const Geom& g, int u, int chunk, int r, const CUtensor
   tc::fence_proxy_async();
   if (tid == 0) {
     tc::prefetch_tmap(tmap);
-    tc::mbar_init(&tma_bar[0], 1);
-    tc::mbar_init(&tma_bar[1], 1);
-    tc::mbar_init(mma_bar, 1);
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&full[i], 1);
+      tc::mbar_init(&done[i], 1);
+      tc::mbar_init(&freed[i], 4);
+    }
     tc::fence_mbar_init();
+    s_err = 0;
   }
-  if (warp == 0) tc::tmem_alloc(tmem_slot, P::kCols);
+  if (warp == 0) tc::tmem_alloc(tmem_slot, 2 * P::kCols);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  if (tid == 0)
-    for (int j = 0; j < 2 && j < mine; ++j) {
-      tc::mbar_expect_tx(&tma_bar[j], P::kABytes);
-      tc::tma_load_5d(sA + j * P::kABytes, tmap, &tma_bar[j], d0, head, 0, (r + kCluster * j) * kTcCells, uw);
-    }
-  constexpr uint32_t kIdesc = tc::idesc_bf16(128, L, true);
-  bool ok = true;
-  for (int j = 0; j < mine; ++j) {
-    const int b = j & 1, t = r + kCluster * j;
-    bool ok_t = true;
-    if (tid == 0) {
-      ok_t = tc::mbar_wait(&tma_bar[b], (j >> 1) & 1);
-      if (ok_t) {
-        tc::fence_after_sync();
-        const uint32_t a0 = tc::smem_u32(sA + b * P::kABytes), b0 = tc::smem_u32(sB);
-        bool acc = false;
+
+  if (warp == 0 && lane == 0 && mine > 0) {
+    // ---- producer and MMA issuer
+    const uint64_t pol = l2_evict_first();
+    auto load = [&](int j) {
+      tc::mbar_expect_tx(&full[j & 1], P::kABytes);
+      tc::tma_load_5d_hint(sA + (j & 1) * P::kABytes, tmap, &full[j & 1], d0, head, 0,
+                           (r + kCluster * j) * kTcCells, uw, pol);
+    };
+    load(0);
+    if (mine > 1) load(1);
+    constexpr uint32_t kIdesc = tc::idesc_bf16(128, L, true);
+    bool ok = true;
+    for (int j = 0; j < mine && ok; ++j) {
+      const int st = j & 1;
+      if (j >= 2) ok = tc::mbar_wait(&freed[st], ((j - 2) >> 1) & 1);     // accumulator st drained
+      if (ok) ok = tc::mbar_wait(&full[st], (j >> 1) & 1);                 // tile j landed
+      if (!ok) break;
+      tc::fence_after_sync();
+      const uint32_t a0 = tc::smem_u32(sA + st * P::kABytes), b0 = tc::smem_u32(sB);
+      const uint32_t d = tmem + st * P::kCols;
+      bool acc = false;
 #pragma unroll
-        for (int l = 0; l < 3; ++l)
+      for (int l = 0; l < 3; ++l)
 #pragma unroll
-          for (int ks = 0; ks < L / 16; ++ks) {
-            const uint64_t da = tc::smem_desc(a0 + ks * 1024, L * 64, 512, 4);
-            const uint64_t db = tc::smem_desc(b0 + l * P::kBBytes + ks * 32, 16, 1024, 2);
-            tc::mma_bf16(tmem, da, db, kIdesc, acc);
-            acc = true;
-          }
-        tc::mma_commit(mma_bar);
+        for (int ks = 0; ks < L / 16; ++ks) {
+          tc::mma_bf16(d, tc::smem_desc(a0 + ks * 1024, L * 64, 512, 4),
+                       tc::smem_desc(b0 + l * P::kBBytes + ks * 32, 16, 1024, 2), kIdesc, acc);
+          acc = true;
+        }
+      tc::mma_commit(&done[st]);
+      // the stage of tile j - 1 is free once its MMAs completed: refill it with tile j + 1
+      if (j >= 1 && j + 1 < mine) {
+        ok = tc::mbar_wait(&done[(j - 1) & 1], ((j - 1) >> 1) & 1);
+        if (ok) load(j + 1);
       }
     }
-    ok_t = __syncthreads_and(ok_t) != 0;
-    if (ok_t) ok_t = __syncthreads_and(tc::mbar_wait(mma_bar, j & 1)) != 0;
-    if (!ok_t) {
-      // give the copies and MMAs still in flight a bounded time to land before the shared and
-      // tensor memory they target is released
-      if (tid == 0) {
-        for (int jj = j; jj < j + 2 && jj < mine; ++jj) tc::mbar_wait(&tma_bar[jj & 1], (jj >> 1) & 1);
-        tc::mbar_wait(mma_bar, j & 1);
+    if (!ok) {
+      s_err = 1;
+      // bounded waits for the copies and MMAs that may still be in flight
+      for (int i = 0; i < 2; ++i) {
+        tc::mbar_wait(&full[i], 0);
+        tc::mbar_wait(&done[i], 0);
       }
-      __syncthreads();
-      ok = false;
-      break;
     }
-    tc::fence_after_sync();
-    // the tile's shared memory is free again: load the tile after next into it
-    if (tid == 0 && j + 2 < mine) {
-      tc::mbar_expect_tx(&tma_bar[b], P::kABytes);
-      tc::tma_load_5d(sA + b * P::kABytes, tmap, &tma_bar[b], d0, head, 0, (t + 2 * kCluster) * kTcCells, uw);
-    }
-    const int q = warp & 3, half = warp >> 2, cell = t * kTcCells + q;
-    float v[P::kHalf];
-    tc::tmem_ld<P::kHalf>(tmem + ((uint32_t)(32 * q) << 16) + half * P::kHalf, v);
-    tc::tmem_ld_wait();
-    if (cell < HWX) {
-      float* yo = Y + (((size_t)u * L + half * P::kHalf) * HWX + cell) * nx + c0 + lane;
+  } else if (warp >= 4 && mine > 0) {
+    // ---- epilogue: warp 4 + q drains TMEM lanes 32q.. (cell q of each tile)
+    const int q = warp - 4;
+    for (int j = 0; j < mine; ++j) {
+      const int st = j & 1;
+      // (a warp vote keeps the warp converged for the .sync.aligned TMEM loads)
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(&done[st], (j >> 1) & 1))) {
+        s_err = 1;
+        break;
+      }
+      tc::fence_after_sync();
+      const int cell = (r + kCluster * j) * kTcCells + q;
+      float* yo = Y + ((size_t)u * L * HWX + cell) * nx + c0 + lane;
+      const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + st * P::kCols;
+      float v[P::kHalf];
+      tc::tmem_ld<P::kHalf>(taddr, v);
+      tc::tmem_ld_wait();
+      if (cell < HWX) {
 #pragma unroll
-      for (int k = 0; k < P::kHalf; ++k) yo[(size_t)k * HWX * nx] = v[k];
+        for (int k = 0; k < P::kHalf; ++k) yo[(size_t)k * HWX * nx] = v[k];
+      }
+      tc::tmem_ld<P::kHalf>(taddr + P::kHalf, v);
+      tc::tmem_ld_wait();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&freed[st]);   // the accumulator may take the next tile
+      if (cell < HWX) {
+#pragma unroll
+        for (int k = 0; k < P::kHalf; ++k) yo[(size_t)(P::kHalf + k) * HWX * nx] = v[k];
+      }
     }
-    tc::fence_before_sync();
-    __syncthreads();   // every thread has read the accumulator before the next tile's MMAs
   }
-  if (!ok && tid == 0) atomicCAS(status, 0u, (unsigned int)TACTKV_TIMEOUT);
+  tc::fence_before_sync();
+  __syncthreads();
   tc::fence_after_sync();
-  if (warp == 0) tc::tmem_free(tmem, P::kCols);
+  const bool ok = s_err == 0;
+  if (!ok && tid == 0) atomicCAS(status, 0u, (unsigned int)TACTKV_TIMEOUT);
+  if (warp == 0) {
+    __syncwarp();
+    tc::tmem_free(tmem, 2 * P::kCols);
+  }
   return ok;
 }
 
@@ -236,7 +273,7 @@ __global__ void __launch_bounds__(kFusedThreads, 3) fdct3_tc_kernel(const __grid
                                                                     const __grid_constant__ CUtensorMap tmap,
                                                                     unsigned int* status) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  __shared__ __align__(8) uint64_t s_bars[3];
+  __shared__ __align__(8) uint64_t s_bars[6];
   __shared__ uint32_t s_tmem;
   unsigned char* smem =
       smem_raw + ((1024 - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);   // 1024-byte aligned (swizzle atoms)

@@ -13,7 +13,9 @@
 //   A = a V tile, loaded by TMA as [cell pair][k][32 channels x 2 cells] bf16 with 128-byte swizzle:
 //       MN-major, one 128-byte row of 64 M-elements (channel, cell of the pair) per k;
 //   B = a limb of C^T, [s][k] with k contiguous: K-major with 128-byte swizzle.
-// Compiled once per S (TACTKV_FUSED_S = 16, 32, 64) for the grids 16x16, 14x14 and 8x8.
+// Compiled once per S (TACTKV_FUSED_S = 16, 32, 64) for the grids 16x16, 14x14 and 8x8.  Opt-in
+// (TACTKV_FUSED_DECODE=1): on B200 it measured slower than the two separate inverse kernels (its V
+// pairs left L2, and few CTAs of its 8-CTA clusters were resident at a time).
 #include "axis_hw.cuh"
 #include "tc.cuh"
 #include "dct_limbs.inc"
@@ -166,7 +168,10 @@ __device__ bool idct_s_tc(const Geom& g, const UnitDev& ud, int u, int chunk, in
   }
   if (!ok && tid == 0) atomicCAS(status, 0u, (unsigned int)TACTKV_TIMEOUT);
   tc::fence_after_sync();
-  if (warp == 0) tc::tmem_free(tmem, P::kCols);
+  if (warp == 0) {
+    __syncwarp();
+    tc::tmem_free(tmem, P::kCols);
+  }
   return ok;
 }
 
@@ -259,7 +264,7 @@ cudaError_t launch_grid(const Geom& g, const UnitList& ul, int nu, float* big, c
 cudaError_t TACTKV_CAT(launch_fused_inv_, TACTKV_FUSED_S)(const Geom& g, const UnitList& ul, int nu, float* big,
                                                           const uint32_t* index, const uint4* recs,
                                                           unsigned int* status, cudaStream_t st) {
-  if (g.S != TACTKV_FUSED_S || (g.flags & (TACTKV_NO_QUANT | TACTKV_SKIP_S)) || tc_s_pass_disabled())
+  if (g.S != TACTKV_FUSED_S || (g.flags & (TACTKV_NO_QUANT | TACTKV_SKIP_S)) || !fused_decode_enabled())
     return cudaErrorNotSupported;
   if (g.H == 16 && g.W == 16) return launch_grid<16, 16>(g, ul, nu, big, index, recs, status, st);
   if (g.H == 14 && g.W == 14) return launch_grid<14, 14>(g, ul, nu, big, index, recs, status, st);

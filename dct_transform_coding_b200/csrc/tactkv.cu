@@ -113,6 +113,14 @@ bool tc_s_pass_disabled() {
   return off;
 }
 
+bool fused_decode_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("TACTKV_FUSED_DECODE");
+    return e && e[0] == '1';
+  }();
+  return on;
+}
+
 namespace {
 
 tactkv_status make_geom(const tactkv_unit& u, Geom& g) {

@@ -328,6 +328,22 @@ def test_variant_flags(shape, variant):
         T.decompress(pay, S, H, W, 2, heads=heads, head_dim=D, layers=[0, 1], kvs=[1, 1], flags=0, check=True)
 
 
+def test_opt_in_fused_decode_kernel():
+    """The single-kernel decode (inverse S on the tensor cores; opt-in, TACTKV_FUSED_DECODE=1, read
+    once per process) on the fused-grid parity cases, in a child process."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, TACTKV_FUSED_DECODE="1")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-m", "pytest", "tests/test_gpu_parity.py", "-q", "-x", "-m", "gpu",
+                        "-p", "no:cacheprovider", "-k",
+                        "tensor_core_and_cuda_core or fused_grid_output or small_shapes or variant_flags or "
+                        "full_size_sampled_units and med4b-1"],
+                       cwd=root, env=env, capture_output=True, text=True, timeout=1200)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
+
+
 # ------------------------------------------------------------------------------ exact ties ---
 def _gpu_allocation(var, grid, bits):
     S, H, W = grid
