@@ -19,17 +19,18 @@ constexpr int kHwMinBlocks = (TACTKV_HCLASS == 16 && TACTKV_WCLASS == 16) ? 2 : 
 template <int HX>
 constexpr int hw_min_blocks_inv() { return (TACTKV_HCLASS == 16 && TACTKV_WCLASS == 16) ? (HX > 0 ? 3 : 2) : 1; }
 
-template <int HC, int WC, int HX, int WX>
+template <int HC, int WC, int HX, int WX, bool VAR>
 __global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) fdct_hw_kernel(const __grid_constant__ Geom g,
                                                                               const __grid_constant__ UnitList ul,
                                                                               float* __restrict__ Y,
                                                                               float* __restrict__ partial, int spc) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int ks0 = blockIdx.y * spc;
-  fdct_hw_slabs<HC, WC, HX, WX, false>(g, Y, partial, g.unit0 + blockIdx.z, blockIdx.x, ks0, min(g.S, ks0 + spc), smem);
+  fdct_hw_slabs<HC, WC, HX, WX, false, 0, VAR>(g, Y, partial, g.unit0 + blockIdx.z, blockIdx.x, ks0,
+                                               min(g.S, ks0 + spc), smem);
 }
 
-template <int HC, int WC, int HX, int WX, int MODE>
+template <int HC, int WC, int HX, int WX, int MODE, bool VAR>
 __global__ void __launch_bounds__(kMaxHwThreads, hw_min_blocks_inv<HX>()) idct_hw_kernel(const __grid_constant__ Geom g,
                                                                                          const __grid_constant__ UnitList ul,
                                                                                          float* __restrict__ V,
@@ -38,8 +39,8 @@ __global__ void __launch_bounds__(kMaxHwThreads, hw_min_blocks_inv<HX>()) idct_h
                                                                                          int spc) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int ks0 = blockIdx.y * spc;
-  idct_hw_slabs<HC, WC, HX, WX, MODE>(g, ul, V, index, recs, g.unit0 + blockIdx.z, blockIdx.x, ks0,
-                                      min(g.S, ks0 + spc), smem);
+  idct_hw_slabs<HC, WC, HX, WX, MODE, false, VAR>(g, ul, V, index, recs, g.unit0 + blockIdx.z, blockIdx.x, ks0,
+                                                  min(g.S, ks0 + spc), smem);
 }
 
 }  // namespace
@@ -65,11 +66,18 @@ cudaError_t launch_hw(bool inverse, int mode, const Geom& g, const UnitList& ul,
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);       \
     kern<<<grid, threads, sm, st>>>(__VA_ARGS__);                                      \
   } while (0)
+  const bool var = has_variant(g.flags);
   if (inverse) {
-    if (mode == kRaw) TACTKV_GO((idct_hw_kernel<H, W, HX, WX, kRaw>), g, ul, buf, slab_off, recs, spc);
-    else TACTKV_GO((idct_hw_kernel<H, W, HX, WX, kQuant>), g, ul, buf, slab_off, recs, spc);
+    if (mode == kRaw) {
+      if (var) TACTKV_GO((idct_hw_kernel<H, W, HX, WX, kRaw, true>), g, ul, buf, slab_off, recs, spc);
+      else TACTKV_GO((idct_hw_kernel<H, W, HX, WX, kRaw, false>), g, ul, buf, slab_off, recs, spc);
+    } else {
+      if (var) TACTKV_GO((idct_hw_kernel<H, W, HX, WX, kQuant, true>), g, ul, buf, slab_off, recs, spc);
+      else TACTKV_GO((idct_hw_kernel<H, W, HX, WX, kQuant, false>), g, ul, buf, slab_off, recs, spc);
+    }
   } else {
-    TACTKV_GO((fdct_hw_kernel<H, W, HX, WX>), g, ul, buf, partial, spc);
+    if (var) TACTKV_GO((fdct_hw_kernel<H, W, HX, WX, true>), g, ul, buf, partial, spc);
+    else TACTKV_GO((fdct_hw_kernel<H, W, HX, WX, false>), g, ul, buf, partial, spc);
   }
 #undef TACTKV_GO
   return cudaGetLastError();

@@ -194,7 +194,7 @@ __device__ __forceinline__ void store_energy(const D& g, int kp, int lane, const
 // packing kernel then quantizes the finished coefficients without transforming anything.
 // Slabs [ks0, ks1) of channel chunk `chunk` of unit u; called by every thread of the CTA.  EF: the
 // stores of X are marked evict-first in L2 (X is read again only by the packing kernel).
-template <int HC, int WC, int HX, int WX, bool EF, int NX = 0>
+template <int HC, int WC, int HX, int WX, bool EF, int NX = 0, bool VAR = false>
 __device__ __forceinline__ void fdct_hw_slabs(const Geom& g, float* __restrict__ Y, float* __restrict__ partial, int u,
                                               int chunk, int ks0, int ks1, unsigned char* smem) {
   const Dims<HX, WX, NX> D(g);
@@ -218,7 +218,7 @@ __device__ __forceinline__ void fdct_hw_slabs(const Geom& g, float* __restrict__
       cp_async_commit();
     }
     // DCT along H, in place, one column pair at a time per warp
-    for (int wp = warp; wp < WP; wp += nwarps) h_pass_fwd<HC>(D, tile, 2 * wp, lane, g.flags & TACTKV_SKIP_H);
+    for (int wp = warp; wp < WP; wp += nwarps) h_pass_fwd<HC>(D, tile, 2 * wp, lane, VAR && (g.flags & TACTKV_SKIP_H));
     __syncthreads();
     float2* t2 = reinterpret_cast<float2*>(tile);
     // DCT along W on row pair kp; the coefficients go back over the slab of Y (this CTA's own
@@ -226,7 +226,7 @@ __device__ __forceinline__ void fdct_hw_slabs(const Geom& g, float* __restrict__
     float* dst = partial + ((size_t)u * (NX ? NX / kChunk : g.nch) + chunk) * g.N + (size_t)ks * D.HW;
     for (int kp = warp; kp < HP; kp += nwarps) {
       float2 x[WC];
-      w_load_fdct<WC>(D, t2, kp, lane, x, g.flags & TACTKV_SKIP_W);
+      w_load_fdct<WC>(D, t2, kp, lane, x, VAR && (g.flags & TACTKV_SKIP_W));
       const bool second = 2 * kp + 1 < D.H;
       float* y0 = yslab + (size_t)(2 * kp * D.W) * D.n;
       if constexpr (EF) {
@@ -271,7 +271,7 @@ __device__ __forceinline__ int cp_index(int Wp, int h, int wp) { return (h * Wp 
 // inverse along S: V_hi[u][k_s][cell pair][c] = (bf16(v[2p]), bf16(v[2p+1])) over V (as
 // __nv_bfloat162) and the remainders V_lo = bf16(v - float(V_hi)) over Vlo (W even).  Together
 // they carry v to about 2^-17 relative.
-template <int HC, int WC, int HX, int WX, int MODE, bool PAIRS = false>
+template <int HC, int WC, int HX, int WX, int MODE, bool PAIRS = false, bool VAR = false>
 __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul, float* __restrict__ V,
                                               const uint32_t* __restrict__ index, const uint4* __restrict__ recs, int u,
                                               int chunk, int ks0, int ks1, unsigned char* smem,
@@ -284,8 +284,8 @@ __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul,
   const unsigned char* pay = ul.u[u].payload;
   const uint32_t* P = index + (size_t)u * unit_index_words(g.S);
   const bool ok = P[g.S + 1] != 0;   // the index kernel checked the header and the bit widths
-  // the shared rotation's inverse: sign of this lane's channel times 1/sqrt(32)
-  const bool rotate = !raw && (g.flags & TACTKV_ROTATE);
+  // the shared rotation's inverse (variant kernels only): sign of this lane's channel / sqrt(32)
+  const bool rotate = VAR && MODE == kQuant && (g.flags & TACTKV_ROTATE);
   const float rot_scale = rotate ? rotation_sign((unsigned long long)(chunk * kChunk + lane)) * 0.17677669529663687f : 1.f;
   const uint32_t cstride = ok ? reinterpret_cast<const uint32_t*>(pay)[11] : 0u, sw = cstride / 4;
   const uint32_t* streams = reinterpret_cast<const uint32_t*>(pay + g.off_codes) + (size_t)chunk * kChunk * sw;
@@ -366,7 +366,7 @@ __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul,
           if (t < D.W)
             x[t] = make_float2(warp_wht(x[t].x, lane) * rot_scale, warp_wht(x[t].y, lane) * rot_scale);
       }
-      if (!(g.flags & TACTKV_SKIP_W)) pencil<WC, WX, true>(x, D.W);
+      if (!VAR || !(g.flags & TACTKV_SKIP_W)) pencil<WC, WX, true>(x, D.W);
       const bool second = 2 * kp + 1 < D.H;
 #pragma unroll
       for (int wp = 0; wp < (WC + 1) / 2; ++wp)
@@ -384,7 +384,7 @@ __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul,
 #pragma unroll
       for (int h = 0; h < HC; ++h)
         if (h < D.H) xh[h] = tile[cp_index(Wp, h, wp) + lane];
-      if (!(g.flags & TACTKV_SKIP_H)) pencil<HC, HX, true>(xh, D.H);
+      if (!VAR || !(g.flags & TACTKV_SKIP_H)) pencil<HC, HX, true>(xh, D.H);
       if constexpr (PAIRS) {
         // pair (cell h*W + 2wp, cell h*W + 2wp + 1) = pair index h*(W/2) + wp
         const size_t base = ((size_t)u * g.S + ks) * (D.HW / 2) * g.n + chunk * kChunk + lane;

@@ -21,7 +21,7 @@ constexpr int kThreads = STile<kCells>::kThreads;
 constexpr int kMinBlocks = 4;
 
 // Forward: x (bf16 or fp32, strided) -> Y[u][k_s][hw][c] fp32.
-template <int L>
+template <int L, bool VAR>
 __global__ void __launch_bounds__(kThreads, kMinBlocks) fdct_s_kernel(const __grid_constant__ Geom g,
                                                                       const __grid_constant__ UnitList ul,
                                                                       float* __restrict__ Y, int lg_cpr) {
@@ -31,11 +31,11 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) fdct_s_kernel(const __gr
   stage_input<L, kCells, false>(g, ul.u[u], hw0, c0, fp32 ? 4 : 2, lg_cpr, tile);
   cp_async_wait_all();
   __syncthreads();
-  fdct_s_cells<L, kCells>(g, u, hw0, c0, tile, fp32, Y);
+  fdct_s_cells<L, kCells, 0, 0, VAR>(g, u, hw0, c0, tile, fp32, Y);
 }
 
 // Inverse: V[u][k_s][hw][c] fp32 -> x_hat (bf16, rounded to nearest even, or fp32), strided.
-template <int L>
+template <int L, bool VAR>
 __global__ void __launch_bounds__(kThreads, kMinBlocks) idct_s_kernel(const __grid_constant__ Geom g,
                                                                       const __grid_constant__ UnitList ul,
                                                                       const float* __restrict__ V) {
@@ -45,19 +45,23 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) idct_s_kernel(const __gr
   cp_async_wait_all();
   __syncthreads();
   drop_volume<L, kCells>(g, u, hw0, c0, V);
-  idct_s_cells<L, kCells>(g, ul.u[u], hw0, c0, vtile);
+  idct_s_cells<L, kCells, VAR>(g, ul.u[u], hw0, c0, vtile);
 }
 
 template <int L>
 cudaError_t launch_len(bool inverse, const Geom& g, const UnitList& ul, int nu, float* buf, cudaStream_t st) {
   const dim3 grid(g.n / 32, (g.HW + kCells - 1) / kCells, nu);
   const bool fp32 = g.flags & TACTKV_FP32_IO;
+  const bool var = has_variant(g.flags);
   if (inverse) {
     const size_t sm = (size_t)L * kCells * 32 * 4;
-    idct_s_kernel<L><<<grid, kThreads, sm, st>>>(g, ul, buf);
+    if (var) idct_s_kernel<L, true><<<grid, kThreads, sm, st>>>(g, ul, buf);
+    else idct_s_kernel<L, false><<<grid, kThreads, sm, st>>>(g, ul, buf);
   } else {
     const size_t sm = (size_t)L * kCells * 32 * (fp32 ? 4 : 2);
-    fdct_s_kernel<L><<<grid, kThreads, sm, st>>>(g, ul, buf, input_pieces_lg(g, ul, g.unit0, nu));
+    const int lg = input_pieces_lg(g, ul, g.unit0, nu);
+    if (var) fdct_s_kernel<L, true><<<grid, kThreads, sm, st>>>(g, ul, buf, lg);
+    else fdct_s_kernel<L, false><<<grid, kThreads, sm, st>>>(g, ul, buf, lg);
   }
   return cudaGetLastError();
 }

@@ -57,7 +57,7 @@ __device__ __forceinline__ void stage_input(const Geom& g, const UnitDev& ud, in
 
 // Forward pencils of a staged input tile: cell hw0 + warp -> Y[u][k_s][hw][c0 + lane], fp32.
 // HWX, NX > 0 fix H*W and the channel count n at compile time (constant strides).
-template <int L, int NC, int HWX = 0, int NX = 0>
+template <int L, int NC, int HWX = 0, int NX = 0, bool VAR = false>
 __device__ __forceinline__ void fdct_s_cells(const Geom& g, int u, int hw0, int c0, const unsigned char* tile,
                                              bool fp32, float* __restrict__ Y) {
   const int lane = threadIdx.x & 31, hwl = threadIdx.x >> 5, hw = hw0 + hwl;
@@ -73,7 +73,7 @@ __device__ __forceinline__ void fdct_s_cells(const Geom& g, int u, int hw0, int 
 #pragma unroll
     for (int s = 0; s < L; ++s) v[s] = __bfloat162float(t[s * NC * 32]);
   }
-  if (!(g.flags & TACTKV_SKIP_S)) dct_exact<L, false>(v);
+  if (!VAR || !(g.flags & TACTKV_SKIP_S)) dct_exact<L, false>(v);
   float* yo = Y + ((size_t)u * L * HW + hw) * n + c0 + lane;
   const size_t kstep = (size_t)HW * n;
 #pragma unroll
@@ -108,7 +108,7 @@ __device__ __forceinline__ void drop_volume(const Geom& g, int u, int hw0, int c
 
 // Inverse pencils of a staged volume tile: cell hw0 + warp -> x_hat (bf16, rounded to nearest
 // even, or fp32), strided.
-template <int L, int NC>
+template <int L, int NC, bool VAR = false>
 __device__ __forceinline__ void idct_s_cells(const Geom& g, const UnitDev& ud, int hw0, int c0, const float* vtile) {
   const int lane = threadIdx.x & 31, hwl = threadIdx.x >> 5, hw = hw0 + hwl;
   if (hw >= g.HW) return;
@@ -116,7 +116,7 @@ __device__ __forceinline__ void idct_s_cells(const Geom& g, const UnitDev& ud, i
   const float* t = vtile + hwl * 32 + lane;
 #pragma unroll
   for (int k = 0; k < L; ++k) v[k] = t[k * NC * 32];
-  if (!(g.flags & TACTKV_SKIP_S)) dct_exact<L, true>(v);
+  if (!VAR || !(g.flags & TACTKV_SKIP_S)) dct_exact<L, true>(v);
   const int c = c0 + lane, head = c / g.head_dim, d = c - head * g.head_dim;
   const long long base = (long long)hw * ud.tok_stride + (long long)head * ud.head_stride + d;
   const long long sstep = (long long)g.HW * ud.tok_stride;

@@ -34,6 +34,11 @@ constexpr uint32_t kPayloadFlags =
     TACTKV_NO_QUANT | TACTKV_SKIP_S | TACTKV_SKIP_H | TACTKV_SKIP_W | TACTKV_UNIFORM_ALLOC | TACTKV_ROTATE;
 constexpr uint32_t kAllFlags = kPayloadFlags | TACTKV_FP32_IO;
 constexpr unsigned long long kRotationSeed = 0x544143544B56ull;
+// Variant flags (axis skips, shared rotation): kernels take a compile-time VAR switch and carry the
+// code for them only when it is set, so that the default kernels keep their register budgets.
+constexpr uint32_t kVariantFlags = TACTKV_SKIP_S | TACTKV_SKIP_H | TACTKV_SKIP_W | TACTKV_ROTATE;
+inline bool has_variant(int flags) { return (flags & kVariantFlags) != 0; }
+__host__ __device__ inline bool has_variant_dev(int flags) { return (flags & kVariantFlags) != 0; }
 
 // ------------------------------------------------------------------------ launch descriptors ---
 struct UnitDev {
@@ -78,11 +83,11 @@ inline bool supported_length(int L) {
 inline int length_class(int L) { return L <= 16 ? 16 : (L <= 32 ? 32 : 64); }
 __host__ __device__ inline int length_class_dev(int L) { return L <= 16 ? 16 : (L <= 32 ? 32 : 64); }
 
-// TACTKV_SIMT_S=1 in the environment keeps the S-axis DCT of the fused forward kernel on the
-// CUDA cores (the cp.async form) instead of the tensor cores; TACTKV_FUSED_DECODE=1 decodes with
-// the single fused kernel (inverse S on the tensor cores) instead of the two inverse kernels.
-// Both are read once per process.
-bool tc_s_pass_disabled();
+// Opt-in tensor-core forms (both measured slower on B200 than the default CUDA-core kernels):
+// TACTKV_TC_S=1 in the environment runs the S-axis DCT of the fused forward kernel on the tensor
+// cores; TACTKV_FUSED_DECODE=1 decodes with the single fused kernel (inverse S on the tensor cores)
+// instead of the two inverse kernels.  Both are read once per process.
+bool tc_s_pass_enabled();
 bool fused_decode_enabled();
 
 

@@ -58,7 +58,7 @@ __host__ __device__ inline size_t fused_fwd_smem(int H, int W, bool fp32_in, int
 }
 
 // NX: the channel count when fixed at compile time (the common 512 and 1024), else 0.
-template <int L, int HX, int WX, int NX>
+template <int L, int HX, int WX, int NX, bool VAR>
 __global__ void __launch_bounds__(kFusedThreads, 3) fdct3_kernel(const __grid_constant__ Geom g,
                                                                  const __grid_constant__ UnitList ul,
                                                                  float* __restrict__ Y, float* __restrict__ partial,
@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(kFusedThreads, 3) fdct3_kernel(const __grid_co
       cp_async_wait_all();
     }
     __syncthreads();
-    fdct_s_cells<L, kNC, HX * WX, NX>(g, u, t * kNC, c0, smem + buf * tb, fp32, Y);
+    fdct_s_cells<L, kNC, HX * WX, NX, VAR>(g, u, t * kNC, c0, smem + buf * tb, fp32, Y);
     __syncthreads();   // the tile's buffer is free again
     if (nbuf == 2) buf ^= 1;
     else if (next) stage_input<L, kNC, true>(g, ud, (t + kCluster) * kNC, c0, esz, lg_cpr, smem);
@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(kFusedThreads, 3) fdct3_kernel(const __grid_co
   // DCT along H and W on this CTA's range of slabs
   constexpr int spc = (L + kCluster - 1) / kCluster;
   const int ks0 = r * spc, ks1 = min(L, ks0 + spc);
-  if (ks0 < ks1) fdct_hw_slabs<16, 16, HX, WX, true, NX>(g, Y, partial, u, chunk, ks0, ks1, smem);
+  if (ks0 < ks1) fdct_hw_slabs<16, 16, HX, WX, true, NX, VAR>(g, Y, partial, u, chunk, ks0, ks1, smem);
 }
 
 // ------------------------------------------------------------- S pass on the tensor cores ---
@@ -320,7 +320,7 @@ bool make_input_map(const Geom& g, const UnitList& ul, int nu, CUtensorMap* map)
         q == cudaDriverEntryPointSuccess)
       encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
   });
-  if (!encode || (g.flags & (TACTKV_FP32_IO | TACTKV_SKIP_S)) || g.head_dim % kChunk != 0) return false;
+  if (!encode || (g.flags & TACTKV_FP32_IO) || has_variant(g.flags) || g.head_dim % kChunk != 0) return false;
   const UnitDev& a = ul.u[g.unit0];
   const long long tok = a.tok_stride, hs = a.head_stride;
   if (tok * 2 % 16 || hs * 2 % 16 || reinterpret_cast<uintptr_t>(a.in) % 16) return false;
@@ -355,7 +355,7 @@ cudaError_t launch_grid(const Geom& g, const UnitList& ul, int nu, float* buf, f
     if (x % 16) return cudaErrorMisalignedAddress;   // never launch a misaligned layout
 #if TACTKV_FUSED_S >= 16
   CUtensorMap map;
-  if (!tc_s_pass_disabled() && make_input_map(g, ul, nu, &map)) {
+  if (tc_s_pass_enabled() && make_input_map(g, ul, nu, &map)) {
     const size_t smem = std::max<size_t>(TcS<L>::kSmem, Ls.total + 1024);
     if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
     if (g.n == 1024)
@@ -369,9 +369,13 @@ cudaError_t launch_grid(const Geom& g, const UnitList& ul, int nu, float* buf, f
   const size_t smem = fused_fwd_smem<L>(HX, WX, (g.flags & TACTKV_FP32_IO) != 0, &nbuf);
   if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
   const int lg_cpr = input_pieces_lg(g, ul, g.unit0, nu);
-  if (g.n == 1024) return launch_cluster(fdct3_kernel<L, HX, WX, 1024>, g, nu, smem, st, g, ul, buf, partial, lg_cpr);
-  if (g.n == 512) return launch_cluster(fdct3_kernel<L, HX, WX, 512>, g, nu, smem, st, g, ul, buf, partial, lg_cpr);
-  return launch_cluster(fdct3_kernel<L, HX, WX, 0>, g, nu, smem, st, g, ul, buf, partial, lg_cpr);
+  if (has_variant(g.flags))
+    return launch_cluster(fdct3_kernel<L, HX, WX, 0, true>, g, nu, smem, st, g, ul, buf, partial, lg_cpr);
+  if (g.n == 1024)
+    return launch_cluster(fdct3_kernel<L, HX, WX, 1024, false>, g, nu, smem, st, g, ul, buf, partial, lg_cpr);
+  if (g.n == 512)
+    return launch_cluster(fdct3_kernel<L, HX, WX, 512, false>, g, nu, smem, st, g, ul, buf, partial, lg_cpr);
+  return launch_cluster(fdct3_kernel<L, HX, WX, 0, false>, g, nu, smem, st, g, ul, buf, partial, lg_cpr);
 }
 
 }  // namespace

@@ -191,7 +191,12 @@ __global__ void __launch_bounds__(kThreads, 3) idct3_tc_kernel(const __grid_cons
   const int r = blockIdx.x, chunk = blockIdx.y, u = g.unit0 + blockIdx.z;
   constexpr int spc = (L + kCluster - 1) / kCluster;
   const int ks0 = r * spc, ks1 = min(L, ks0 + spc);
-  if (ks0 < ks1) idct_hw_slabs<16, 16, HX, WX, kQuant, true>(g, ul, Vhi, index, recs, u, chunk, ks0, ks1, smem, Vlo);
+  if (ks0 < ks1) {
+    if (has_variant_dev(g.flags))
+      idct_hw_slabs<16, 16, HX, WX, kQuant, true, true>(g, ul, Vhi, index, recs, u, chunk, ks0, ks1, smem, Vlo);
+    else
+      idct_hw_slabs<16, 16, HX, WX, kQuant, true, false>(g, ul, Vhi, index, recs, u, chunk, ks0, ks1, smem, Vlo);
+  }
   cluster_barrier();   // the chunk's V is complete
   idct_s_tc<L, HX * WX>(g, ul.u[u], u, chunk, r, &mhi, &mlo, smem, s_bars, &s_tmem, status);
 }
@@ -264,7 +269,8 @@ cudaError_t launch_grid(const Geom& g, const UnitList& ul, int nu, float* big, c
 cudaError_t TACTKV_CAT(launch_fused_inv_, TACTKV_FUSED_S)(const Geom& g, const UnitList& ul, int nu, float* big,
                                                           const uint32_t* index, const uint4* recs,
                                                           unsigned int* status, cudaStream_t st) {
-  if (g.S != TACTKV_FUSED_S || (g.flags & (TACTKV_NO_QUANT | TACTKV_SKIP_S)) || !fused_decode_enabled())
+  if (g.S != TACTKV_FUSED_S || (g.flags & (TACTKV_NO_QUANT | TACTKV_SKIP_S | TACTKV_SKIP_H | TACTKV_SKIP_W)) ||
+      !fused_decode_enabled())
     return cudaErrorNotSupported;
   if (g.H == 16 && g.W == 16) return launch_grid<16, 16>(g, ul, nu, big, index, recs, status, st);
   if (g.H == 14 && g.W == 14) return launch_grid<14, 14>(g, ul, nu, big, index, recs, status, st);

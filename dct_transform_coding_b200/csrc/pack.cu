@@ -97,6 +97,9 @@ __device__ __forceinline__ void pack_block(const uint4* __restrict__ rs, const f
   }
 }
 
+// VAR: the payload has variant flags (the shared rotation), a compile-time switch so that the
+// default kernel keeps its register budget.
+template <bool VAR>
 __global__ void __launch_bounds__(kPackThreads) pack_kernel(const __grid_constant__ Geom g,
                                                             const __grid_constant__ UnitList ul,
                                                             const float* __restrict__ X, const uint4* __restrict__ recs,
@@ -188,7 +191,7 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const __grid_constan
   __syncthreads();
 
   uint32_t* row = sbuf + lane * L.words;
-  const bool rotate = g.flags & TACTKV_ROTATE;
+  const bool rotate = VAR && (g.flags & TACTKV_ROTATE);
   const float rot_in = rotate ? rotation_sign((unsigned long long)(chunk * kChunk + lane)) : 1.f;
   // blocks of kPackBlock records per warp; the next block's coefficients are loaded while this
   // one is quantized
@@ -269,10 +272,11 @@ cudaError_t launch_pack(const Geom& g, const UnitList& ul, int nu, const float* 
     pack_raw_kernel<<<dim3(g.nch, g.S, nu), kPackThreads, 0, st>>>(g, ul, X, spc);
   } else {
     const PackLayout L = pack_layout();
-    cudaFuncSetAttribute(pack_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
+    auto kernel = has_variant(g.flags) ? pack_kernel<true> : pack_kernel<false>;
+    cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
     // ranges of kPackRecs records; a unit has at most N records, CTAs past its last record exit
     const dim3 grid(g.nch, (g.N + kPackRecs - 1) / kPackRecs, nu);
-    pack_kernel<<<grid, kPackThreads, L.total, st>>>(g, ul, X, recs, index);
+    kernel<<<grid, kPackThreads, L.total, st>>>(g, ul, X, recs, index);
   }
   return cudaGetLastError();
 }

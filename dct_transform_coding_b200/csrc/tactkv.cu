@@ -105,12 +105,12 @@ cudaError_t launch_attention(const Geom& g, const UnitList& kl, const UnitList& 
                              const float* q, float* zp, float* part, float* out, float* m, float* l,
                              cudaStream_t st);
 
-bool tc_s_pass_disabled() {
-  static const bool off = [] {
-    const char* e = getenv("TACTKV_SIMT_S");
+bool tc_s_pass_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("TACTKV_TC_S");
     return e && e[0] == '1';
   }();
-  return off;
+  return on;
 }
 
 bool fused_decode_enabled() {

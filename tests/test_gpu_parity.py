@@ -258,10 +258,11 @@ def test_full_size_sampled_units(name, bits, pick):
 # ------------------------------------------------------- tensor-core and CUDA-core S passes ---
 @pytest.mark.parametrize("S,H,W", [(64, 16, 16), (32, 14, 14), (16, 8, 8)])
 def test_tensor_core_and_cuda_core_s_pass_both_match_the_oracle(S, H, W):
-    """The fused forward kernel runs its DCT along S on the tensor cores when one TMA tensor map
-    can describe the whole wave (units evenly spaced in memory), and on the CUDA cores otherwise.
-    The same three units are compressed both ways (the second time listed in reverse memory order,
-    which no single map describes) and both payloads must pass the oracle's acceptance rules."""
+    """With TACTKV_TC_S=1 the fused forward kernel runs its DCT along S on the tensor cores when
+    one TMA tensor map can describe the whole wave (units evenly spaced in memory), and on the CUDA
+    cores otherwise.  The same three units are compressed both ways (the second time listed in
+    reverse memory order, which no single map describes) and both payloads must pass the oracle's
+    acceptance rules (without the variable both runs take the CUDA-core form)."""
     heads, D = 2, 64
     x = torch.stack([make_unit(S, H, W, heads, D, rho=(0.9, 0.85, 0.85), nu=4.0, seed=70 + i, device=DEV)
                      for i in range(3)])
@@ -328,13 +329,14 @@ def test_variant_flags(shape, variant):
         T.decompress(pay, S, H, W, 2, heads=heads, head_dim=D, layers=[0, 1], kvs=[1, 1], flags=0, check=True)
 
 
-def test_opt_in_fused_decode_kernel():
-    """The single-kernel decode (inverse S on the tensor cores; opt-in, TACTKV_FUSED_DECODE=1, read
-    once per process) on the fused-grid parity cases, in a child process."""
+def test_opt_in_tensor_core_kernels():
+    """The opt-in tensor-core forms, read once per process: the forward kernel's DCT along S on
+    tcgen05 (TACTKV_TC_S=1) and the single-kernel decode with the inverse S on tcgen05
+    (TACTKV_FUSED_DECODE=1), on the fused-grid parity cases, in a child process."""
     import os
     import subprocess
     import sys
-    env = dict(os.environ, TACTKV_FUSED_DECODE="1")
+    env = dict(os.environ, TACTKV_TC_S="1", TACTKV_FUSED_DECODE="1")
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     r = subprocess.run([sys.executable, "-m", "pytest", "tests/test_gpu_parity.py", "-q", "-x", "-m", "gpu",
                         "-p", "no:cacheprovider", "-k",
