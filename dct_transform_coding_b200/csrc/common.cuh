@@ -89,6 +89,7 @@ __host__ __device__ inline int length_class_dev(int L) { return L <= 16 ? 16 : (
 // instead of the two inverse kernels.  Both are read once per process.
 bool tc_s_pass_enabled();
 bool fused_decode_enabled();
+bool pack_seq_enabled();   // TACTKV_PACK_SEQ=1: the sequential bit-string packer
 
 
 // --------------------------------------------------------------------------------- launchers ---

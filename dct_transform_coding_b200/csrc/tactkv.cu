@@ -113,6 +113,14 @@ bool tc_s_pass_enabled() {
   return on;
 }
 
+bool pack_seq_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("TACTKV_PACK_SEQ");
+    return e && e[0] == '1';
+  }();
+  return on;
+}
+
 bool fused_decode_enabled() {
   static const bool on = [] {
     const char* e = getenv("TACTKV_FUSED_DECODE");

@@ -336,7 +336,7 @@ def test_opt_in_tensor_core_kernels():
     import os
     import subprocess
     import sys
-    env = dict(os.environ, TACTKV_TC_S="1", TACTKV_FUSED_DECODE="1")
+    env = dict(os.environ, TACTKV_TC_S="1", TACTKV_FUSED_DECODE="1", TACTKV_PACK_SEQ="1")
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     r = subprocess.run([sys.executable, "-m", "pytest", "tests/test_gpu_parity.py", "-q", "-x", "-m", "gpu",
                         "-p", "no:cacheprovider", "-k",
