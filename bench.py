@@ -376,7 +376,7 @@ def attention_bench(T, w, bits, payload, out, du, ws, stream, layers, kvs, peak,
 
 
 STAGES_C = ["forward", "allocate", "pack"]          # compress: DCTs with energies, allocation, packing
-STAGES_D = ["decode_index", "inverse"]              # decompress: payload index, decode + inverse DCTs
+STAGES_D = ["decode_index", "idct_hw", "idct_s"]    # decompress: payload index, decode + inverse W/H, inverse S
 
 
 def profile_stages(T, cu, du, ws, stream, U, n_prof):
@@ -388,7 +388,7 @@ def profile_stages(T, cu, du, ws, stream, U, n_prof):
     cu_p, du_p = cu[:n_sub], du[:n_sub]
     scale = U / n_sub
     evs_c = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_prof)]
-    evs_d = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_prof)]
+    evs_d = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_prof)]
     for e in [e for es in evs_c + evs_d for e in es]:
         e.record(stream)   # torch creates the CUDA event on its first record
     sp = int(stream.cuda_stream)
@@ -407,18 +407,21 @@ def profile_stages(T, cu, du, ws, stream, U, n_prof):
                    for i, n in enumerate(STAGES_D)})
     return {"stages": stages,
             "compress_ms": scale * mean(evs_c[k][0].elapsed_time(evs_c[k][3]) for k in range(n_prof)),
-            "decompress_ms": scale * mean(evs_d[k][0].elapsed_time(evs_d[k][2]) for k in range(n_prof))}
+            "decompress_ms": scale * mean(evs_d[k][0].elapsed_time(evs_d[k][3]) for k in range(n_prof))}
 
 
 def stage_roofline(prof, in_bytes, pay_bytes, bins_x_units, ms_step, peak, peak_kind, name):
-    """Roofline of the dominant stage: its algorithmic bytes (what the method must move through HBM
-    in that stage) over its measured time.  forward reads the bf16 input; allocate writes the gains
-    and bit widths (5 B per bin) and the headers; pack writes the codes; decode_index reads gains
-    and widths; inverse reads the codes and writes the bf16 output.  The whole step's fraction
-    (both directions' algorithmic bytes over the timed step) is reported beside it."""
+    """Roofline of the dominant kernel (each stage below is one kernel, reduce_var + allocate aside):
+    its algorithmic bytes (what the method itself must move through HBM in that kernel) over its
+    measured time.  forward (the three forward DCTs) reads the bf16 input; allocate writes the gains
+    and bit widths (5 B per bin) and the headers; pack writes the codes; decode_index reads gains and
+    widths; idct_hw (decoding with the inverse DCTs along W and H) reads the codes; idct_s (the
+    inverse DCT along S) writes the bf16 output.  The whole step's fraction (both directions'
+    algorithmic bytes over the timed step) is reported beside it."""
     meta = 5 * bins_x_units
     codes = max(0, pay_bytes - meta)
-    alg = {"forward": in_bytes, "allocate": meta, "pack": codes, "decode_index": meta, "inverse": codes + in_bytes}
+    alg = {"forward": in_bytes, "allocate": meta, "pack": codes, "decode_index": meta, "idct_hw": codes,
+           "idct_s": in_bytes}
     stages = prof["stages"]
     dom = max(stages, key=stages.get)
     achieved = alg[dom] / (stages[dom] * 1e-3) / 1e9

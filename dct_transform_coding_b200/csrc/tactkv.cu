@@ -397,16 +397,18 @@ static tactkv_status decompress_impl(const tactkv_unit* units, int n_units, void
                                                               : cudaErrorNotSupported;
                          if (fe == cudaSuccess) {
                            t_launches += 1;   // idct3 (decode, inverse H/W, inverse S)
+                           mark(2);
                          } else if (fe == cudaErrorNotSupported) {
                            t_launches += 2;   // idct_hw, idct_s
                            if (launch_axis_hw(ch, cw, true, mode, g, ul, nu, w.big, nullptr, w.index, w.recs,
                                               slabs_per_cta(g, nu, true, mode), st) != cudaSuccess)
                              return TACTKV_CUDA;
+                           mark(2);
                            if (launch_axis_s(cs, true, g, ul, nu, w.big, st) != cudaSuccess) return TACTKV_CUDA;
                          } else {
                            return TACTKV_CUDA;
                          }
-                         mark(2);
+                         mark(3);
                          return TACTKV_OK;
                        });
 }

@@ -147,7 +147,7 @@ def tactkv_compress_profiled(units, workspace_ptr: int, workspace_bytes: int, st
 
 
 def tactkv_decompress_profiled(units, workspace_ptr: int, workspace_bytes: int, stream_ptr: int, events) -> int:
-    """events: sequence of 3 cudaEvent_t handles or None."""
+    """events: sequence of 4 cudaEvent_t handles or None."""
     arr = _as_array(units)
     return int(_lib.tactkv_decompress_profiled(arr, len(arr), ctypes.c_void_p(workspace_ptr), workspace_bytes,
                                                ctypes.c_void_p(stream_ptr), _events_array(events)))

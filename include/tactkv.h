@@ -136,7 +136,9 @@ tactkv_status tactkv_decompress(const tactkv_unit* units, int n_units, void* wor
    compress:   0 before the transforms, 1 after the DCTs along S and along H and W (with the
                energy sums) of every unit, 2 after the allocation, 3 after quantization and
                packing.
-   decompress: 0 before the payload index, 1 after it, 2 after the inverse DCTs of every unit. */
+   decompress: 0 before the payload index, 1 after it, 2 after the inverse DCT along W and H
+               (with the decoding), 3 after the inverse DCT along S (with the single-kernel decode
+               2 and 3 mark the same point). */
 tactkv_status tactkv_compress_profiled(const tactkv_unit* units, int n_units, void* workspace,
                                        size_t workspace_bytes, struct CUstream_st* stream,
                                        void* const* events);
