@@ -41,6 +41,12 @@ Readings taken where the pages are silent (each is listed in the design notes):
 * Ablation variants ("Main Findings": fewer transformed axes, uniform allocation), also flags:
   FLAG_SKIP_S / _H / _W leave that axis untransformed (all three: no DCT); FLAG_UNIFORM gives every
   bin with sigma^2 > 0 the nominal bits (b_i = bits) instead of water-filling.
+* Per-head gains (FLAG_HEAD_GAIN, off by default).  Stage 4 counts Sum(b_i * d + 32) bits with d
+  the head dimension of the pages' models ("Main Findings" quotes absmax-to-std "at d=256"), which
+  reads as one gain-shape vector, with its own 32-bit gain, per (bin, head).  With the flag, bin i
+  of head h is scaled by g[h, i] = float32(sqrt(mean over the head's head_dim channels of
+  X[i, c]^2)) and dequantized with it; a zero gain scales by 0 (every coordinate is then 0).  The
+  bit allocation still uses the pooled sigma_i^2 of all channels, so b_i is shared by the heads.
 * Payload layout: see ``FORMAT`` below (the pages fix only its size, stage 4:
   sum_i (b_i * d + 32) bits plus a small index).
 """
@@ -59,6 +65,7 @@ from scipy.special import erfc, ndtri
 #   [0, 64)                     header, see HEADER_FMT
 #   [64, 64 + pad16(N))         uint8  b[N]        bits of each frequency bin (0..8)
 #   [off_sigma, +pad16(4N))     float32 sigma[N]   stored gain of each bin
+#                               (FLAG_HEAD_GAIN: float32 sigma[heads][N], pad16(4 * heads * N))
 #   [off_codes, ...)            n channel streams, channel c at off_codes + c * chan_stride
 #       quantized:   stream bit P_i + k holds bit k (LSB first) of bin i's code, with
 #                    P_i = sum_{j<i} b_j; stream bit q is bit (q & 7) of byte (q >> 3);
@@ -73,7 +80,9 @@ FLAG_SKIP_H = 8             # no DCT along H
 FLAG_SKIP_W = 16            # no DCT along W
 FLAG_UNIFORM = 32           # uniform allocation: b_i = bits for every bin with sigma^2 > 0
 FLAG_ROTATE = 64            # fixed shared rotation of each bin's shape vector before quantization
-PAYLOAD_FLAGS = FLAG_NO_QUANT | FLAG_SKIP_S | FLAG_SKIP_H | FLAG_SKIP_W | FLAG_UNIFORM | FLAG_ROTATE
+FLAG_HEAD_GAIN = 128        # one gain per (bin, head) instead of one per bin
+PAYLOAD_FLAGS = (FLAG_NO_QUANT | FLAG_SKIP_S | FLAG_SKIP_H | FLAG_SKIP_W | FLAG_UNIFORM | FLAG_ROTATE |
+                 FLAG_HEAD_GAIN)
 HEADER_FMT = "<IHHiiiiiiiiIIQII"   # magic ver flags layer kv S H W heads head_dim bits codebits stride total r0 r1
 HEADER_BYTES = 64
 assert struct.calcsize(HEADER_FMT) == HEADER_BYTES
@@ -365,19 +374,35 @@ def dequantize(code: np.ndarray, bits: int) -> np.ndarray:
 
 
 # ------------------------------------------------------------------------------ payload -----
-def payload_layout(N: int, n: int, code_bits: int, no_quant: bool = False) -> Dict[str, int]:
+def payload_layout(N: int, n: int, code_bits: int, no_quant: bool = False, gains: int = 1) -> Dict[str, int]:
+    """Byte offsets of the payload's parts; gains = gain vectors of N floats (heads with
+    FLAG_HEAD_GAIN, else 1)."""
     off_sigma = HEADER_BYTES + _pad16(N)
-    off_codes = off_sigma + _pad16(4 * N)
+    off_codes = off_sigma + _pad16(4 * N * gains)
     stride = _pad16(4 * N) if no_quant else _pad16((code_bits + 7) // 8)
     return dict(off_b=HEADER_BYTES, off_sigma=off_sigma, off_codes=off_codes, chan_stride=stride,
                 total=off_codes + n * stride)
 
 
 def payload_capacity(S: int, H: int, W: int, heads: int, head_dim: int, bits: int,
-                     no_quant: bool = False) -> int:
+                     no_quant: bool = False, flags: int = 0) -> int:
     """Worst-case payload size: sum_i b_i <= bits * N."""
     N = S * H * W
-    return payload_layout(N, heads * head_dim, bits * N, no_quant)["total"]
+    no_quant = no_quant or bool(flags & FLAG_NO_QUANT)
+    return payload_layout(N, heads * head_dim, 32 * N if no_quant else bits * N, no_quant,
+                          _gain_vectors(flags, heads))["total"]
+
+
+def _gain_vectors(flags: int, heads: int) -> int:
+    return heads if (flags & FLAG_HEAD_GAIN) and not (flags & FLAG_NO_QUANT) else 1
+
+
+def head_gains(X: np.ndarray, heads: int, head_dim: int) -> np.ndarray:
+    """Per-head gains g[h, i] = float32(sqrt(mean over head h's channels of X[i, c]^2)) (the
+    per-head reading of stage 4's gain-shape vectors), as fp64 values of float32 numbers."""
+    X = np.asarray(X, dtype=np.float64)
+    hv = np.mean(X.reshape(X.shape[0], heads, head_dim) ** 2, axis=2).T     # [heads, N]
+    return stored_sigma(hv)
 
 
 def _pack_streams(codes: np.ndarray, b: np.ndarray, stride: int) -> np.ndarray:
@@ -409,7 +434,8 @@ def compress_unit(x, S: int, H: int, W: int, heads: int, head_dim: int, bits: in
                   layer: int = 0, kv: int = 0, no_quant: bool = False,
                   return_info: bool = False, flags: int = 0):
     """Compress one visual K or V, x[S*H*W, heads, head_dim] (any real dtype), to payload bytes.
-    flags: FLAG_SKIP_* (axes left untransformed), FLAG_UNIFORM, FLAG_ROTATE (see the head)."""
+    flags: FLAG_SKIP_* (axes left untransformed), FLAG_UNIFORM, FLAG_ROTATE, FLAG_HEAD_GAIN (see
+    the head)."""
     n = heads * head_dim
     N = S * H * W
     if not 1 <= bits <= MAX_BITS:
@@ -431,10 +457,15 @@ def compress_unit(x, S: int, H: int, W: int, heads: int, head_dim: int, bits: in
     else:
         b = allocate_uniform(var, bits) if flags & FLAG_UNIFORM else allocate_bits(var, bits)
         code_bits = int(b.sum())
-        lay = payload_layout(N, n, code_bits)
+        if flags & FLAG_HEAD_GAIN:
+            sig = head_gains(X, heads, head_dim)                            # [heads, N]
+        lay = payload_layout(N, n, code_bits, gains=_gain_vectors(flags, heads))
         codes = np.zeros((N, n), dtype=np.int64)
         for i in np.nonzero(b)[0]:
-            u = Xq[i] / np.float64(sig[i])
+            # the gain of every channel of bin i: the bin's, or its head's (0 where a head is silent)
+            g = np.repeat(sig[:, i], head_dim) if flags & FLAG_HEAD_GAIN else np.full(n, sig[i])
+            g = g.astype(np.float64)
+            u = np.divide(Xq[i], g, out=np.zeros(n), where=g > 0)
             codes[i] = quantize(u, int(b[i]))
         body = _pack_streams(codes, b, lay["chan_stride"])
     buf = bytearray(lay["total"])
@@ -442,7 +473,8 @@ def compress_unit(x, S: int, H: int, W: int, heads: int, head_dim: int, bits: in
                      layer, kv, S, H, W, heads, head_dim, bits, code_bits, lay["chan_stride"],
                      lay["total"], 0, 0)
     buf[lay["off_b"]:lay["off_b"] + N] = b.astype(np.uint8).tobytes()
-    buf[lay["off_sigma"]:lay["off_sigma"] + 4 * N] = sig.astype("<f4").tobytes()
+    sig_bytes = np.ascontiguousarray(sig, dtype="<f4").tobytes()
+    buf[lay["off_sigma"]:lay["off_sigma"] + len(sig_bytes)] = sig_bytes
     buf[lay["off_codes"]:] = body.tobytes()
     if return_info:
         return bytes(buf), dict(X=X, Xq=Xq, var=var, sigma=sig, b=b, codes=codes)
@@ -458,11 +490,14 @@ def parse_payload(payload) -> Dict:
         raise ValueError("not a TACT-KV payload")
     N = S * H * W
     n = heads * head_dim
-    lay = payload_layout(N, n, code_bits, bool(flags & FLAG_NO_QUANT))
+    gains = _gain_vectors(flags, heads)
+    lay = payload_layout(N, n, code_bits, bool(flags & FLAG_NO_QUANT), gains)
     if lay["chan_stride"] != stride or lay["total"] != total or len(buf) < total:
         raise ValueError("inconsistent payload header")
     b = np.frombuffer(buf, np.uint8, N, lay["off_b"]).astype(np.int64)
-    sig = np.frombuffer(buf, "<f4", N, lay["off_sigma"]).copy()
+    sig = np.frombuffer(buf, "<f4", N * gains, lay["off_sigma"]).copy()
+    if (flags & FLAG_HEAD_GAIN) and not (flags & FLAG_NO_QUANT):
+        sig = sig.reshape(gains, N)                     # [heads, N]
     streams = np.frombuffer(buf, np.uint8, n * stride, lay["off_codes"]).reshape(n, stride)
     return dict(flags=flags, layer=layer, kv=kv, S=S, H=H, W=W, heads=heads, head_dim=head_dim,
                 bits=bits, code_bits=code_bits, b=b, sigma=sig, streams=streams, N=N, n=n)
@@ -481,7 +516,11 @@ def decompress_unit(payload) -> np.ndarray:
         codes = _unpack_streams(p["streams"], b)
         X = np.zeros((N, n), dtype=np.float64)
         for i in np.nonzero(b)[0]:
-            X[i] = np.float64(p["sigma"][i]) * dequantize(codes[i], int(b[i]))
+            if p["flags"] & FLAG_HEAD_GAIN:
+                g = np.repeat(p["sigma"][:, i].astype(np.float64), p["head_dim"])
+            else:
+                g = np.float64(p["sigma"][i])
+            X[i] = g * dequantize(codes[i], int(b[i]))
         if p["flags"] & FLAG_ROTATE:
             X = X @ rotation_matrix(n)                  # row i: R^T (dequantized R X_i)
     x = idct3(X.reshape(p["S"], p["H"], p["W"], n), axes_of(p["flags"]))
@@ -525,11 +564,13 @@ def codes_of(payload) -> Tuple[np.ndarray, np.ndarray]:
     return p["b"], _unpack_streams(p["streams"], p["b"])
 
 
-def occupancy_bits(b: np.ndarray, d: int) -> int:
-    """Stage 4's occupancy of one compressed layer: sum_i (b_i * d + 32) bits, d the channels that
-    share a gain (here all n = heads * head_dim channels of a bin), 32 bits for each bin's gain."""
+def occupancy_bits(b: np.ndarray, d: int, vectors: int = 1) -> int:
+    """Stage 4's occupancy of one compressed layer: sum over the gain-shape vectors of
+    (b_i * d + 32) bits, d the channels that share a gain and 32 bits for the gain.  By default a
+    bin is one vector of all n = heads * head_dim channels (d = n); with per-head gains each bin
+    holds `vectors` = heads vectors of d = head_dim channels."""
     b = np.asarray(b, dtype=np.int64)
-    return int(np.sum(b * int(d) + 32))
+    return int(vectors) * int(np.sum(b * int(d) + 32))
 
 
 def index_bits(N: int) -> int:

@@ -431,6 +431,59 @@ def test_uniform_allocation_and_theorem1_through_the_codec():
     assert abs(d["uniform"] / d["wf"] / inv_gamma - 1) < 0.1
 
 
+# -------------------------------------------------------------------------- per-head gains ---
+def test_head_gain_one_head_is_the_pooled_gain():
+    """With a single head the per-head gain is the bin's pooled gain: same b, gains, codes and
+    reconstruction as the default payload; only the header's flag differs."""
+    S, H, W, heads, D = 2, 4, 4, 1, 64
+    x = RNG.standard_normal((S * H * W, heads, D))
+    p0, i0 = O.compress_unit(x, S, H, W, heads, D, 3, return_info=True)
+    p1, i1 = O.compress_unit(x, S, H, W, heads, D, 3, return_info=True, flags=O.FLAG_HEAD_GAIN)
+    assert np.array_equal(i0["b"], i1["b"]) and np.array_equal(i0["codes"], i1["codes"])
+    assert np.array_equal(O.parse_payload(p1)["sigma"], O.parse_payload(p0)["sigma"][None])
+    assert np.array_equal(O.decompress_unit(p0), O.decompress_unit(p1))
+    assert p0[:6] == p1[:6] and p0[8:] == p1[8:] and p1[6:8] != p0[6:8]
+
+
+def test_head_gain_scaled_copy_of_a_head():
+    """Gain-shape per head: head 1 = 4 x head 0 (exact in fp64) gives gains g1 = 4 g0 exactly and the
+    very codes of head 0, and reconstructs to 4 x head 0's reconstruction; one gain per bin would
+    quantize head 1 on another scale (different codes)."""
+    S, H, W, D, bits = 2, 4, 4, 32, 3
+    x0 = RNG.standard_normal((S * H * W, 1, D))
+    x = np.concatenate([x0, 4.0 * x0], axis=1)
+    p, info = O.compress_unit(x, S, H, W, 2, D, bits, return_info=True, flags=O.FLAG_HEAD_GAIN)
+    g = O.parse_payload(p)["sigma"]
+    assert g.shape == (2, S * H * W) and np.array_equal(g[1], 4 * g[0])
+    act = info["b"] > 0
+    assert np.array_equal(info["codes"][act][:, D:], info["codes"][act][:, :D])
+    y = O.decompress_unit(p)
+    assert np.array_equal(y[:, 1], 4 * y[:, 0])
+    _, pooled = O.compress_unit(x, S, H, W, 2, D, bits, return_info=True)
+    assert not np.array_equal(pooled["codes"][act][:, D:], pooled["codes"][act][:, :D])
+
+
+def test_head_gain_silent_head_and_occupancy():
+    """A head whose channels are all zero gets zero gains and an exactly zero reconstruction, the
+    other head's gains are those of its own channels; the payload carries heads x N gains, and the
+    stage-4 occupancy counts one 32-bit gain per (bin, head)."""
+    S, H, W, D, bits = 2, 2, 4, 32, 2
+    N = S * H * W
+    x = np.concatenate([RNG.standard_normal((N, 1, D)), np.zeros((N, 1, D))], axis=1)
+    p, info = O.compress_unit(x, S, H, W, 2, D, bits, return_info=True, flags=O.FLAG_HEAD_GAIN)
+    g = O.parse_payload(p)["sigma"]
+    assert not g[1].any()
+    assert np.array_equal(g[0], np.sqrt(np.mean(info["X"][:, :D] ** 2, axis=1)).astype(np.float32))
+    y = O.decompress_unit(p)
+    assert not y[:, 1].any() and np.sqrt(np.mean((y[:, 0] - x[:, 0]) ** 2)) < 0.5
+    # gains region: pad16(4 * heads * N) bytes; the codes follow it
+    lay = O.payload_layout(N, 2 * D, int(info["b"].sum()), gains=2)
+    assert lay["off_codes"] - lay["off_sigma"] == 4 * 2 * N and len(p) == lay["total"]
+    b = info["b"]
+    assert O.occupancy_bits(b, D, 2) == int(np.sum(b) * 2 * D + 32 * 2 * N)
+    assert O.occupancy_bits(b, 2 * D) == int(np.sum(b) * 2 * D + 32 * N)
+
+
 # ------------------------------------------------------------------- decode-time attention ---
 def test_attention_decode_matches_torch_sdpa():
     """The oracle's attention over a compressed cache equals torch's scaled_dot_product_attention

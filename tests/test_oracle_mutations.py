@@ -61,6 +61,13 @@ MUTATIONS = [
      "    if axes[0]:\n        y = np.einsum(\"kh,shwc->skwc\""),
     ("uniform: nominal bits plus one", "return np.where(var > 0, int(bits), 0).astype(np.int64)",
      "return np.where(var > 0, int(bits) + 1, 0).astype(np.int64)"),
+    ("head gain: heads and channels transposed",
+     "hv = np.mean(X.reshape(X.shape[0], heads, head_dim) ** 2, axis=2).T",
+     "hv = np.mean(X.reshape(X.shape[0], head_dim, heads) ** 2, axis=1).T"),
+    ("head gain: pooled over all heads", "g = np.repeat(sig[:, i], head_dim) if flags & FLAG_HEAD_GAIN",
+     "g = np.repeat(np.sqrt(np.mean(sig[:, i].astype(np.float64) ** 2)), n) if flags & FLAG_HEAD_GAIN"),
+    ("head gain: decoder uses head 0's gain", "g = np.repeat(p[\"sigma\"][:, i].astype(np.float64), p[\"head_dim\"])",
+     "g = np.repeat(p[\"sigma\"][0, i].astype(np.float64), p[\"heads\"] * p[\"head_dim\"])"),
     ("code band: distance to the levels", "thresholds_b = table(bits)[1]", "thresholds_b = table(bits)[0]"),
     ("code band: no relative scaling", "return np.min(gaps / np.maximum(1.0, np.abs(thresholds_b)), axis=-1)",
      "return np.min(gaps, axis=-1)"),
