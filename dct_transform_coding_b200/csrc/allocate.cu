@@ -58,16 +58,34 @@ __device__ T block_sum(T v, T* s_red /* 32 entries */) {
 }
 
 // sigma_i^2 = (1/n) sum over the channel chunks of the fp32 per-chunk energy sums, in fp64 and
-// in a fixed order; one thread per bin across the whole GPU.
-__global__ void __launch_bounds__(256) reduce_var_kernel(const __grid_constant__ Geom g, const float* __restrict__ partial,
+// in a fixed order; one thread per bin across the whole GPU.  With per-head gains the same sums,
+// restarted at every head's first chunk, give the gains float32(sqrt(sum / head_dim)) of bin i in
+// every head, written straight into the payload's sigma[head][bin].
+__global__ void __launch_bounds__(256) reduce_var_kernel(const __grid_constant__ Geom g,
+                                                         const __grid_constant__ UnitList ul,
+                                                         const float* __restrict__ partial,
                                                          double* __restrict__ var_ws) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   const int u = blockIdx.y;
   if (i >= g.N) return;
   const float* p = partial + (size_t)u * g.nch * g.N + i;
   double acc = 0.0;
+  if (head_gains_on(g.flags)) {
+    float* gains = reinterpret_cast<float*>(ul.u[u].payload + g.off_sigma) + i;
+    const int cph = g.head_dim / kChunk;   // chunks of a head
+    for (int h = 0; h < g.heads; ++h) {
+      double acc_h = 0.0;
+      for (int q = h * cph; q < (h + 1) * cph; ++q) {
+        const double v = (double)__ldcs(p + (size_t)q * g.N);
+        acc += v;
+        acc_h += v;
+      }
+      gains[(size_t)h * g.N] = (float)sqrt(acc_h / (double)g.head_dim);
+    }
+  } else {
 #pragma unroll 8
-  for (int q = 0; q < g.nch; ++q) acc += (double)__ldcs(p + (size_t)q * g.N);
+    for (int q = 0; q < g.nch; ++q) acc += (double)__ldcs(p + (size_t)q * g.N);
+  }
   var_ws[(size_t)u * g.N + i] = acc / (double)g.n;
 }
 
@@ -264,7 +282,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
     }
     pay[kHeaderBytes + i] = (unsigned char)b;
     const float sg = (float)sqrt(x);
-    reinterpret_cast<float*>(pay + g.off_sigma)[i] = sg;
+    if (!head_gains_on(g.flags)) reinterpret_cast<float*>(pay + g.off_sigma)[i] = sg;   // (else: per head, written)
     reinterpret_cast<uint2*>(var)[i] = make_uint2(__float_as_uint(sg), (uint32_t)b);   // for the records
     code_bits_local += b;
     slab_sum += b;
@@ -281,7 +299,8 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
   }
   // zero padding after the b[] and sigma[] arrays
   for (int i = kHeaderBytes + g.N + threadIdx.x; i < g.off_sigma; i += blockDim.x) pay[i] = 0;
-  for (int i = g.off_sigma + 4 * g.N + threadIdx.x; i < g.off_codes; i += blockDim.x) pay[i] = 0;
+  for (int i = g.off_sigma + 4 * g.N * gain_vectors(g.flags, g.heads) + threadIdx.x; i < g.off_codes; i += blockDim.x)
+    pay[i] = 0;
   const long long code_bits = raw ? 32LL * g.N : block_sum<long long>(code_bits_local, s_ll);
   const long long cstride = pad16((code_bits + 7) / 8);
   // slab offsets P(k_s) and record offsets NZ(k_s), and a zero in the stream word at every P(k_s)
@@ -490,7 +509,7 @@ cudaError_t launch_allocate_from_var(const Geom& g, const UnitList& ul, int nu, 
 
 cudaError_t launch_allocate(const Geom& g, const UnitList& ul, int nu, const float* partial, double* var,
                             uint32_t* index, uint4* recs, cudaStream_t st) {
-  reduce_var_kernel<<<dim3((g.N + 255) / 256, nu), 256, 0, st>>>(g, partial, var);
+  reduce_var_kernel<<<dim3((g.N + 255) / 256, nu), 256, 0, st>>>(g, ul, partial, var);
   return launch_allocate_from_var(g, ul, nu, var, index, recs, st);
 }
 

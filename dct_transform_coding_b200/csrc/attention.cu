@@ -28,9 +28,29 @@ constexpr int kAttnThreads = 256;
 constexpr int kMaxG = 16;                   // query heads per K/V head
 constexpr float kInvSqrt32 = 0.17677669529663687f;
 
-// Stage the slab's dense decoding records in shared memory and list the slab's bins that have
-// bits (in bin order): act[a] = bin index j, actrec[a] = {sigma, offset << 8 | code mask} of that
-// bin.  Returns the count.  Called by every thread; ends with a barrier.
+// Words of a channel stream held per slab in shared memory: the most a slab can span (8 bits per
+// bin, from any bit of its first word), two zero words for the look-ahead of the code reads, and
+// an odd count, so that 32 lanes reading 32 channels' rows at one offset hit 32 banks.
+__host__ __device__ inline int attn_word_stride(int HW) { return ((8 * HW + 31) / 32 + 3) | 1; }
+__host__ __device__ inline int pad32(int x) { return (x + 31) / 32 * 32; }
+
+// Copy the words of slab ks of the D channel streams from `row0` (channel 0's stream, word P(ks)
+// >> 5) into words[c][stride], asynchronously, with the two look-ahead words zeroed.  Every thread.
+__device__ __forceinline__ void stage_words(const uint32_t* __restrict__ row0, uint32_t sw, int D, int nw, int stride,
+                                            uint32_t* __restrict__ words) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  for (int c = warp; c < D; c += nwarps)
+    for (int w = lane; w < nw + 2; w += 32) {
+      if (w < nw) cp_async4(words + c * stride + w, row0 + (size_t)c * sw + w);
+      else words[c * stride + w] = 0u;
+    }
+  cp_async_commit();
+}
+
+// Stage the slab's dense decoding records and list the slab's bins that have bits (in bin order):
+// act[a] = bin index j, actrec[a] = {sigma, offset << 8 | code mask} of that bin, for a < count;
+// actrec is then zero up to the next multiple of 32 (a zero record decodes to 0).  Returns the
+// count.  Called by every thread; ends with a barrier.
 __device__ int stage_active(const uint4* __restrict__ srec, int HW, int W, uint2* __restrict__ actrec,
                             int* __restrict__ act, int* s_count, int* s_warp) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
@@ -65,38 +85,67 @@ __device__ int stage_active(const uint4* __restrict__ srec, int HW, int W, uint2
     }
     __syncthreads();
   }
-  return *s_count;
+  const int na = *s_count;
+  for (int a = na + (int)threadIdx.x; a < pad32(na); a += blockDim.x) actrec[a] = make_uint2(0u, 0u);
+  __syncthreads();
+  return na;
 }
 
-// Code of a bin with bits (record {sigma, offset << 8 | mask}) in this lane's channel stream
-// `row` (the slab's first word); only words that hold some of its bits are read.
-__device__ __forceinline__ uint32_t read_code(const uint32_t* __restrict__ row, uint32_t mk) {
-  const uint32_t k = mk & 0xffu, off = mk >> 8;
+// Dequantized coefficient of a bin (record {sigma, offset << 8 | mask}) in a channel's staged row
+// (the slab's first word on); a zero record gives 0 through the zero in front of the levels.
+__device__ __forceinline__ float decode_staged(const uint32_t* __restrict__ row, uint2 r, const float* lvs1) {
+  const uint32_t k = r.y & 0xffu, off = r.y >> 8;
   const uint32_t* w = row + (off >> 5);
-  const uint32_t lo = __ldg(w), hi = (off & 31u) + (uint32_t)__popc(k) > 32u ? __ldg(w + 1) : 0u;
-  return __funnelshift_r(lo, hi, off) & k;
+  const uint32_t code = __funnelshift_r(w[0], w[1], off) & k;
+  return __uint_as_float(r.x) * lvs1[(int)(k + code) - 1];
 }
 
-// z_j[i] for the G query heads of K/V head h over the bins of slab ks.  Warp w handles the channel
-// groups w, w + 8, ... of the head (lane = channel); each warp's per-bin sums over its 32 channels
-// go to its own row of s_part and are added up in warp order (deterministic).
-__global__ void __launch_bounds__(kAttnThreads) attn_scores_kernel(const __grid_constant__ Geom g,
-                                                                   const __grid_constant__ UnitList ul,
-                                                                   const uint32_t* __restrict__ index,
-                                                                   const uint4* __restrict__ recs,
-                                                                   const float* __restrict__ q, int q_heads,
-                                                                   float* __restrict__ z) {
+// With per-head gains: the staged records of the active bins take head h's gains instead of the
+// bins' (sigma[h][bin] in the payload).  Every thread; the caller synchronizes before use.
+__device__ __forceinline__ void head_gain_records(const Geom& g, const unsigned char* pay, int h, int ks, int na,
+                                                  uint2* actrec, const int* act) {
+  const float* hg = reinterpret_cast<const float*>(pay + g.off_sigma) + (size_t)h * g.N + (size_t)ks * g.HW;
+  for (int a = threadIdx.x; a < na; a += blockDim.x) actrec[a].x = __float_as_uint(hg[act[a]]);
+}
+
+// z_j[i] for the G query heads of K/V head h over the bins of slab ks.  The slab's words of the
+// head's D channel streams are staged in shared memory.  The warps work in pairs on batches of 32
+// active bins (pair p takes batches p, p + 4, ...); warp w of the pair takes the channel groups
+// cg = w, w + 2, ... (lane = channel within a group) and, for two query heads at a time, accumulates
+// q_j[d] X_K[i, d] over them in registers, sums over its 32 lanes (transpose sum: lane l ends with
+// active bin a0 + l), and the second warp's sums are added to the first's through shared memory.
+// z of the bins without bits is 0.
+constexpr int kScoreThreads = 256;
+constexpr int kScorePairs = kScoreThreads / 64;
+__global__ void __launch_bounds__(kScoreThreads) attn_scores_kernel(const __grid_constant__ Geom g,
+                                                                    const __grid_constant__ UnitList ul,
+                                                                    const uint32_t* __restrict__ index,
+                                                                    const uint4* __restrict__ recs,
+                                                                    const float* __restrict__ q, int q_heads,
+                                                                    float* __restrict__ z) {
   extern __shared__ __align__(16) float sh[];
   __shared__ int s_count, s_warp[32];
+  __shared__ float s_red[kScorePairs][2][32];
   const int ks = blockIdx.x, h = blockIdx.y, u = blockIdx.z;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  const int G = q_heads / g.heads, D = g.head_dim, HW = g.HW;
-  float* lvs1 = sh + 1;                             // a zero in front of the levels
-  float* qs = sh + (kLmLvTotal + 1 + 3) / 4 * 4;    // [G][D], rotated when the payload is
-  float* s_part = qs + G * D;                       // [nwarps][G][HW], by active-bin index
-  uint2* actrec = reinterpret_cast<uint2*>(s_part + (size_t)nwarps * G * HW);   // [HW]
-  int* act = reinterpret_cast<int*>(actrec + HW);                                 // [HW]
+  const int G = q_heads / g.heads, D = g.head_dim, HW = g.HW, stride = attn_word_stride(HW);
+  float* lvs1 = sh + 1;                                        // a zero in front of the levels
+  float* qs = sh + (kLmLvTotal + 1 + 3) / 4 * 4;               // [G][D], rotated when the payload is
+  float* zs = qs + G * D;                                      // [G][HW]
+  uint2* actrec = reinterpret_cast<uint2*>(zs + (G * HW + 1) / 2 * 2);   // [pad32(HW)]
+  int* act = reinterpret_cast<int*>(actrec + pad32(HW));                 // [HW]
+  uint32_t* words = reinterpret_cast<uint32_t*>(act + pad32(HW));        // [D][stride]
+  const uint32_t* P = index + (size_t)u * unit_index_words(g.S);
+  const bool ok = P[g.S + 1] != 0;
+  const unsigned char* pay = ul.u[u].payload;
+  if (ok) {
+    const uint32_t p0 = P[ks], p1 = P[ks + 1], sw = reinterpret_cast<const uint32_t*>(pay)[11] / 4;
+    const int nw = (int)(((p0 & 31u) + (p1 - p0) + 31) >> 5);
+    stage_words(reinterpret_cast<const uint32_t*>(pay + g.off_codes) + (size_t)h * D * sw + (p0 >> 5), sw, D, nw,
+                stride, words);
+  }
   for (int i = threadIdx.x; i <= kLmLvTotal; i += blockDim.x) sh[i] = i ? c_lm_levels[i - 1] : 0.f;
+  for (int i = threadIdx.x; i < G * HW; i += blockDim.x) zs[i] = 0.f;
   const float* qu = q + ((size_t)u * q_heads + (size_t)h * G) * D;
   const bool rotate = g.flags & TACTKV_ROTATE;
   for (int gg = warp; gg < G * (D / 32); gg += nwarps) {   // (query head, channel group) per warp
@@ -105,64 +154,52 @@ __global__ void __launch_bounds__(kAttnThreads) attn_scores_kernel(const __grid_
     if (rotate) v = warp_wht(v * rotation_sign((unsigned long long)(h * D + d)), lane) * kInvSqrt32;
     qs[gq * D + d] = v;
   }
-  for (int i = threadIdx.x; i < nwarps * G * HW; i += blockDim.x) s_part[i] = 0.f;
-  const uint32_t* P = index + (size_t)u * unit_index_words(g.S);
-  const bool ok = P[g.S + 1] != 0;
-  const unsigned char* pay = ul.u[u].payload;
   const uint4* srec = recs + (size_t)u * g.N + (size_t)ks * ((g.H + 1) / 2) * g.W;
   const int na = ok ? stage_active(srec, HW, g.W, actrec, act, &s_count, s_warp) : 0;
-  if (!ok) __syncthreads();
-  if (na > 0) {
-    const uint32_t sw = reinterpret_cast<const uint32_t*>(pay)[11] / 4, w0 = P[ks] >> 5;
-    const uint32_t* streams = reinterpret_cast<const uint32_t*>(pay + g.off_codes);
-    float* mine = s_part + (size_t)warp * G * HW;
-    for (int cg = warp; cg < D / 32; cg += nwarps) {
-      const int d = cg * 32 + lane;
-      const uint32_t* row = streams + (size_t)(h * D + d) * sw + w0;
-      for (int a0 = 0; a0 < na; a0 += 32) {
-        float val[32];
-#pragma unroll
-        for (int b = 0; b < 32; ++b) {
-          val[b] = 0.f;
-          if (a0 + b < na) {
-            const uint2 r = actrec[a0 + b];
-            const uint32_t k = r.y & 0xffu;
-            val[b] = __uint_as_float(r.x) * lvs1[(int)(k + read_code(row, r.y)) - 1];
-          }
-        }
-        for (int gq = 0; gq < G; ++gq) {
-          const float qd = qs[gq * D + d];
-          float t[32];
-#pragma unroll
-          for (int b = 0; b < 32; ++b) t[b] = val[b] * qd;
-          // sum over the warp's 32 channels: lane l ends with active bin a0 + l
-#pragma unroll
-          for (int hh = 16; hh >= 1; hh >>= 1) {
-            const bool upper = lane & hh;
-#pragma unroll
-            for (int i = 0; i < hh; ++i) {
-              const float send = upper ? t[i] : t[i + hh], keep = upper ? t[i + hh] : t[i];
-              t[i] = keep + __shfl_xor_sync(0xffffffffu, send, hh);
-            }
-          }
-          if (a0 + lane < na) mine[gq * HW + a0 + lane] += t[0];
-        }
-      }
-    }
-  }
+  if (head_gains_on(g.flags)) head_gain_records(g, pay, h, ks, na, actrec, act);
+  cp_async_wait_all();
   __syncthreads();
   const float scale = rsqrtf((float)D);
-  float* zu = z + ((size_t)u * q_heads + (size_t)h * G) * g.N + (size_t)ks * HW;
-  for (int i = threadIdx.x; i < G * HW; i += blockDim.x) {   // bins without bits: z = 0
-    const int gq = i / HW, j = i - gq * HW;
-    zu[(size_t)gq * g.N + j] = 0.f;
+  const int pair = warp >> 1, half = warp & 1;
+  const int rounds = (na + kScorePairs * 32 - 1) / (kScorePairs * 32);   // the same for every warp
+  for (int it = 0; it < rounds; ++it) {
+    const int a0 = (it * kScorePairs + pair) * 32;
+    for (int gp = 0; gp < G; gp += 2) {
+      const bool two = gp + 1 < G;
+      float s0 = 0.f, s1 = 0.f;
+      if (a0 < na) {
+        float acc0[32], acc1[32];
+#pragma unroll
+        for (int b = 0; b < 32; ++b) acc0[b] = acc1[b] = 0.f;
+        for (int d = half * 32 + lane; d < D; d += 64) {
+          const uint32_t* row = words + d * stride;
+          const float q0 = qs[gp * D + d], q1 = two ? qs[(gp + 1) * D + d] : 0.f;
+#pragma unroll
+          for (int b = 0; b < 32; ++b) {
+            const float x = decode_staged(row, actrec[a0 + b], lvs1);
+            acc0[b] = fmaf(x, q0, acc0[b]);
+            acc1[b] = fmaf(x, q1, acc1[b]);
+          }
+        }
+        s0 = warp_transpose_sum(acc0, lane);
+        s1 = warp_transpose_sum(acc1, lane);
+        if (half) {
+          s_red[pair][0][lane] = s0;
+          s_red[pair][1][lane] = s1;
+        }
+      }
+      __syncthreads();
+      if (!half && a0 + lane < na) {
+        zs[gp * HW + act[a0 + lane]] = (s0 + s_red[pair][0][lane]) * scale;
+        if (two) zs[(gp + 1) * HW + act[a0 + lane]] = (s1 + s_red[pair][1][lane]) * scale;
+      }
+      __syncthreads();
+    }
   }
-  __syncthreads();
-  for (int i = threadIdx.x; i < G * na; i += blockDim.x) {
-    const int gq = i / na, a = i - gq * na;
-    float acc = 0.f;
-    for (int w = 0; w < nwarps; ++w) acc += s_part[((size_t)w * G + gq) * HW + a];
-    zu[(size_t)gq * g.N + act[a]] = acc * scale;
+  float* zu = z + ((size_t)u * q_heads + (size_t)h * G) * g.N + (size_t)ks * HW;
+  for (int i = threadIdx.x; i < G * HW; i += blockDim.x) {
+    const int gq = i / HW, j = i - gq * HW;
+    zu[(size_t)gq * g.N + j] = zs[i];
   }
 }
 
@@ -197,15 +234,21 @@ __device__ void pencils_any(float* vol, int L, int count, int stride, int step_o
     else pencils<0, 64, INV>(vol, L, count, stride, step_outer, inner);
   }
 }
+// Row length of the score volume in shared memory: W rounded up to an odd count, so that the 32
+// lanes of a warp, each on its own row of the pass along W, hit 32 different banks.
+__host__ __device__ inline int vol_row(int W) { return W | 1; }
+__host__ __device__ inline size_t softmax_smem(const Geom& g) { return (size_t)g.S * g.H * vol_row(g.W) * 4; }
+
+// vol[s][h][w] at (s*H + h)*Wr + w, Wr = vol_row(W).
 template <bool INV, int SX, int HX, int WX>
 __device__ void dct3_volume(float* vol, const Geom& g) {
-  const int S = g.S, H = g.H, W = g.W;
-  // along W: pencils (s, h), contiguous; along H: (s, w), stride W; along S: (h, w), stride H*W
-  if (!(g.flags & TACTKV_SKIP_W)) pencils_any<WX, INV>(vol, W, S * H, 1, W, 1);
+  const int S = g.S, H = g.H, W = g.W, Wr = vol_row(W);
+  // along W: pencils (s, h), contiguous; along H: (s, w), stride Wr; along S: (h, w), stride H*Wr
+  if (!(g.flags & TACTKV_SKIP_W)) pencils_any<WX, INV>(vol, W, S * H, 1, Wr, 1);
   __syncthreads();
-  if (!(g.flags & TACTKV_SKIP_H)) pencils_any<HX, INV>(vol, H, S * W, W, H * W, W);
+  if (!(g.flags & TACTKV_SKIP_H)) pencils_any<HX, INV>(vol, H, S * W, Wr, H * Wr, W);
   __syncthreads();
-  if (!(g.flags & TACTKV_SKIP_S)) pencils_any<SX, INV>(vol, S, H * W, H * W, 0, H * W);
+  if (!(g.flags & TACTKV_SKIP_S)) pencils_any<SX, INV>(vol, S, H * W, H * Wr, Wr, W);
   __syncthreads();
 }
 
@@ -235,22 +278,24 @@ __global__ void __launch_bounds__(kSoftmaxThreads) attn_softmax_kernel(const __g
   __shared__ float red[32];
   const int j = blockIdx.x, u = blockIdx.y;
   float* zg = zp + ((size_t)u * q_heads + j) * g.N;
-  for (int i = threadIdx.x; i < g.N; i += blockDim.x) vol[i] = zg[i];
+  const int W = g.W, Wr = vol_row(W);
+  auto at = [&](int i) { return (i / W) * Wr + (i - (i / W) * W); };   // bin i -> its padded place
+  for (int i = threadIdx.x; i < g.N; i += blockDim.x) vol[at(i)] = zg[i];
   __syncthreads();
   dct3_volume<true, SX, HX, WX>(vol, g);
   float mx = -INFINITY;
-  for (int i = threadIdx.x; i < g.N; i += blockDim.x) mx = fmaxf(mx, vol[i]);
+  for (int i = threadIdx.x; i < g.N; i += blockDim.x) mx = fmaxf(mx, vol[at(i)]);
   mx = block_reduce(mx, red, true);
   float sum = 0.f;
   for (int i = threadIdx.x; i < g.N; i += blockDim.x) {
-    const float e = __expf(vol[i] - mx);
-    vol[i] = e;
+    const float e = __expf(vol[at(i)] - mx);
+    vol[at(i)] = e;
     sum += e;
   }
   sum = block_reduce(sum, red, false);
   __syncthreads();
   dct3_volume<false, SX, HX, WX>(vol, g);
-  for (int i = threadIdx.x; i < g.N; i += blockDim.x) zg[i] = vol[i];
+  for (int i = threadIdx.x; i < g.N; i += blockDim.x) zg[i] = vol[at(i)];
   if (threadIdx.x == 0) {
     m_out[(size_t)u * q_heads + j] = mx;
     l_out[(size_t)u * q_heads + j] = sum;
@@ -259,7 +304,10 @@ __global__ void __launch_bounds__(kSoftmaxThreads) attn_softmax_kernel(const __g
 
 // part[u][ks][j][d] = sum over the bins i of slab ks of dct3(p_j)[i] * X_V[i, hD + d] (rotated
 // domain when the payload is); thread = channel, G accumulators each, no reduction across threads.
-// Only bins with bits are visited; their weights dct3(p_j)[i] * sigma_i are formed once per CTA.
+// The slab's words of the head's channel streams are staged in shared memory, and only bins with
+// bits are visited; their weights dct3(p_j)[i] * sigma_i are formed once per CTA.  GM: the most
+// query heads per K/V head the instance handles (4 keeps the accumulators few).
+template <int GM>
 __global__ void __launch_bounds__(kAttnThreads) attn_values_kernel(const __grid_constant__ Geom g,
                                                                    const __grid_constant__ UnitList ul,
                                                                    const uint32_t* __restrict__ index,
@@ -269,40 +317,52 @@ __global__ void __launch_bounds__(kAttnThreads) attn_values_kernel(const __grid_
   extern __shared__ __align__(16) float sh[];
   __shared__ int s_count, s_warp[32];
   const int ks = blockIdx.x, h = blockIdx.y, u = blockIdx.z;
-  const int G = q_heads / g.heads, D = g.head_dim, HW = g.HW;
+  const int G = q_heads / g.heads, D = g.head_dim, HW = g.HW, stride = attn_word_stride(HW);
   float* lvs1 = sh + 1;
   float* wt = sh + (kLmLvTotal + 1 + 3) / 4 * 4;        // [HW][G]: weight of active bin a for head g
-  uint2* actrec = reinterpret_cast<uint2*>(wt + ((size_t)G * HW + 1) / 2 * 2);   // 8-byte aligned
-  int* act = reinterpret_cast<int*>(actrec + HW);
-  for (int i = threadIdx.x; i <= kLmLvTotal; i += blockDim.x) sh[i] = i ? c_lm_levels[i - 1] : 0.f;
+  uint2* actrec = reinterpret_cast<uint2*>(wt + ((size_t)G * HW + 1) / 2 * 2);   // [pad32(HW)], 8-byte aligned
+  int* act = reinterpret_cast<int*>(actrec + pad32(HW));                         // [HW]
+  uint32_t* words = reinterpret_cast<uint32_t*>(act + pad32(HW));                // [D][stride]
   const uint32_t* P = index + (size_t)u * unit_index_words(g.S);
   const bool ok = P[g.S + 1] != 0;
   const unsigned char* pay = ul.u[u].payload;
+  if (ok) {
+    const uint32_t p0 = P[ks], p1 = P[ks + 1], sw = reinterpret_cast<const uint32_t*>(pay)[11] / 4;
+    const int nw = (int)(((p0 & 31u) + (p1 - p0) + 31) >> 5);
+    stage_words(reinterpret_cast<const uint32_t*>(pay + g.off_codes) + (size_t)h * D * sw + (p0 >> 5), sw, D, nw,
+                stride, words);
+  }
+  for (int i = threadIdx.x; i <= kLmLvTotal; i += blockDim.x) sh[i] = i ? c_lm_levels[i - 1] : 0.f;
   const uint4* srec = recs + (size_t)u * g.N + (size_t)ks * ((g.H + 1) / 2) * g.W;
   const int na = ok ? stage_active(srec, HW, g.W, actrec, act, &s_count, s_warp) : 0;
-  if (!ok) __syncthreads();
+  if (head_gains_on(g.flags)) {
+    head_gain_records(g, pay, h, ks, na, actrec, act);
+    __syncthreads();
+  }
   for (int i = threadIdx.x; i < G * na; i += blockDim.x) {
     const int a = i / G, gq = i - a * G;
     wt[i] = ptil[((size_t)u * q_heads + (size_t)h * G + gq) * g.N + (size_t)ks * HW + act[a]] *
             __uint_as_float(actrec[a].x);
   }
+  cp_async_wait_all();
   __syncthreads();
-  const uint32_t sw = ok ? reinterpret_cast<const uint32_t*>(pay)[11] / 4 : 0u, w0 = P[ks] >> 5;
-  const uint32_t* streams = reinterpret_cast<const uint32_t*>(pay + g.off_codes);
   for (int d = threadIdx.x; d < D; d += blockDim.x) {
-    float acc[kMaxG];
+    float acc[GM];
 #pragma unroll
-    for (int gq = 0; gq < kMaxG; ++gq) acc[gq] = 0.f;
-    const uint32_t* row = streams + (size_t)(h * D + d) * sw + w0;
+    for (int gq = 0; gq < GM; ++gq) acc[gq] = 0.f;
+    const uint32_t* row = words + d * stride;
     for (int a = 0; a < na; ++a) {
-      const uint32_t mk = actrec[a].y;
-      const float lv = lvs1[(int)((mk & 0xffu) + read_code(row, mk)) - 1];
+      const uint2 r = actrec[a];
+      const uint32_t k = r.y & 0xffu, off = r.y >> 8;
+      const uint32_t* w = row + (off >> 5);
+      const float lv = lvs1[(int)(k + (__funnelshift_r(w[0], w[1], off) & k)) - 1];
 #pragma unroll
-      for (int gq = 0; gq < kMaxG; ++gq)
+      for (int gq = 0; gq < GM; ++gq)
         if (gq < G) acc[gq] = fmaf(wt[a * G + gq], lv, acc[gq]);
     }
-    for (int gq = 0; gq < G; ++gq)
-      part[(((size_t)u * g.S + ks) * q_heads + (size_t)h * G + gq) * D + d] = acc[gq];
+#pragma unroll
+    for (int gq = 0; gq < GM; ++gq)
+      if (gq < G) part[(((size_t)u * g.S + ks) * q_heads + (size_t)h * G + gq) * D + d] = acc[gq];
   }
 }
 
@@ -331,20 +391,25 @@ __global__ void __launch_bounds__(kAttnThreads) attn_reduce_kernel(const __grid_
 
 size_t attention_scores_smem(const Geom& g, int q_heads) {
   const int G = q_heads / g.heads;
-  return (size_t)((kLmLvTotal + 1 + 3) / 4 * 4 + G * g.head_dim + (kAttnThreads / 32) * G * g.HW) * 4 +
-         (size_t)g.HW * 12;
+  return (size_t)((kLmLvTotal + 1 + 3) / 4 * 4 + G * g.head_dim + (G * g.HW + 1) / 2 * 2) * 4 +
+         (size_t)pad32(g.HW) * 12 + (size_t)g.head_dim * attn_word_stride(g.HW) * 4;
 }
+size_t attention_softmax_smem(const Geom& g) { return softmax_smem(g); }
 size_t attention_values_smem(const Geom& g, int q_heads) {
   const int G = q_heads / g.heads;
-  return (size_t)((kLmLvTotal + 1 + 3) / 4 * 4 + (G * g.HW + 1) / 2 * 2) * 4 + (size_t)g.HW * 12;
+  return (size_t)((kLmLvTotal + 1 + 3) / 4 * 4 + (G * g.HW + 1) / 2 * 2) * 4 + (size_t)pad32(g.HW) * 12 +
+         (size_t)g.head_dim * attn_word_stride(g.HW) * 4;
 }
+
+// One thread per channel of the head (head_dim is a multiple of 32), at most kAttnThreads.
+inline int values_threads(int D) { return D < kAttnThreads ? D : kAttnThreads; }
 
 cudaError_t launch_attention(const Geom& g, const UnitList& kl, const UnitList& vl, int nu, int q_heads,
                              const uint32_t* kidx, const uint4* krec, const uint32_t* vidx, const uint4* vrec,
                              const float* q, float* zp, float* part, float* out, float* m, float* l,
                              cudaStream_t st) {
   const size_t s1 = attention_scores_smem(g, q_heads), s3 = attention_values_smem(g, q_heads);
-  const size_t s2 = (size_t)g.N * 4;
+  const size_t s2 = softmax_smem(g);
   if (s1 > 227 * 1024 || s2 > 227 * 1024 || s3 > 227 * 1024 || q_heads / g.heads > kMaxG)
     return cudaErrorInvalidConfiguration;
   cudaFuncSetAttribute(attn_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1);
@@ -355,10 +420,11 @@ cudaError_t launch_attention(const Geom& g, const UnitList& kl, const UnitList& 
   else if (g.S == 32 && g.H == 24 && g.W == 24) softmax = attn_softmax_kernel<32, 24, 24>;
   else if (g.S == 8 && g.H == 8 && g.W == 8) softmax = attn_softmax_kernel<8, 8, 8>;
   cudaFuncSetAttribute(softmax, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2);
-  cudaFuncSetAttribute(attn_values_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s3);
-  attn_scores_kernel<<<dim3(g.S, g.heads, nu), kAttnThreads, s1, st>>>(g, kl, kidx, krec, q, q_heads, zp);
+  auto values = q_heads / g.heads <= 4 ? attn_values_kernel<4> : attn_values_kernel<kMaxG>;
+  cudaFuncSetAttribute(values, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s3);
+  attn_scores_kernel<<<dim3(g.S, g.heads, nu), kScoreThreads, s1, st>>>(g, kl, kidx, krec, q, q_heads, zp);
   softmax<<<dim3(q_heads, nu), kSoftmaxThreads, s2, st>>>(g, zp, m, l, q_heads);
-  attn_values_kernel<<<dim3(g.S, g.heads, nu), kAttnThreads, s3, st>>>(g, vl, vidx, vrec, zp, q_heads, part);
+  values<<<dim3(g.S, g.heads, nu), values_threads(g.head_dim), s3, st>>>(g, vl, vidx, vrec, zp, q_heads, part);
   attn_reduce_kernel<<<dim3(q_heads, nu), kAttnThreads, 0, st>>>(g, part, l, q_heads, out);
   return cudaGetLastError();
 }

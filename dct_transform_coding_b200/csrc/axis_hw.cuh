@@ -152,22 +152,6 @@ __device__ __forceinline__ void w_load_fdct(const D& g, const float2* t2, int kp
     if (t < g.W) x[t] = t2[rp_index(Wp, kp, t) + lane];
   if (!skip) pencil<WC, D::wx, false>(x, g.W);
 }
-// Sums over the 32 lanes of the warp of 32 values per lane (recursive halving: at each step a
-// lane keeps half of its values and adds the partner lane's copy of that half); lane l returns the
-// total of value l.
-__device__ __forceinline__ float warp_transpose_sum(float (&v)[32], int lane) {
-#pragma unroll
-  for (int h = 16; h >= 1; h >>= 1) {
-    const bool upper = lane & h;
-#pragma unroll
-    for (int i = 0; i < h; ++i) {
-      const float send = upper ? v[i] : v[i + h], keep = upper ? v[i + h] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, h);
-    }
-  }
-  return v[0];
-}
-
 // Energies of row pair kp summed over the warp's 32 channels and stored to dst (the slab's bins):
 // the squares of rows 2kp and 2kp+1 go through the transpose sum 16 columns at a time, so that
 // lane l ends with column (l & 15) of row 2kp + (l >> 4) of that group of columns.
@@ -286,6 +270,10 @@ __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul,
   const bool ok = P[g.S + 1] != 0;   // the index kernel checked the header and the bit widths
   // the shared rotation's inverse (variant kernels only): sign of this lane's channel / sqrt(32)
   const bool rotate = VAR && MODE == kQuant && (g.flags & TACTKV_ROTATE);
+  // per-head gains (variant kernels only): this chunk's head's sigma[bin], else the records' gains
+  const float* hgain = (VAR && MODE == kQuant && head_gains_on(g.flags))
+                           ? reinterpret_cast<const float*>(pay + g.off_sigma) + (size_t)(chunk * kChunk / g.head_dim) * g.N
+                           : nullptr;
   const float rot_scale = rotate ? rotation_sign((unsigned long long)(chunk * kChunk + lane)) * 0.17677669529663687f : 1.f;
   const uint32_t cstride = ok ? reinterpret_cast<const uint32_t*>(pay)[11] : 0u, sw = cstride / 4;
   const uint32_t* streams = reinterpret_cast<const uint32_t*>(pay + g.off_codes) + (size_t)chunk * kChunk * sw;
@@ -357,7 +345,13 @@ __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul,
             const uint32_t* w1 = row + (off1 >> 5);
             const float l0 = lvs1[(int)(k0 + (__funnelshift_r(w0[0], w0[1], off0) & k0)) - 1];
             const float l1 = lvs1[(int)(k1 + (__funnelshift_r(w1[0], w1[1], off1) & k1)) - 1];
-            x[t] = __fmul2_rn(make_float2(l0, l1), make_float2(__uint_as_float(m.x), __uint_as_float(m.y)));
+            float s0 = __uint_as_float(m.x), s1 = __uint_as_float(m.y);
+            if (VAR && hgain) {   // (a row without bits keeps its gain 0; the padding row reads nothing)
+              const size_t i0 = (size_t)ks * D.HW + (size_t)(2 * kp) * D.W + t;
+              s0 = k0 ? __ldg(hgain + i0) : 0.f;
+              s1 = k1 ? __ldg(hgain + i0 + D.W) : 0.f;
+            }
+            x[t] = __fmul2_rn(make_float2(l0, l1), make_float2(s0, s1));
           }
       }
       if (rotate) {   // R^T = diag(s) H_32 / sqrt(32) across the warp's 32 channels, both rows

@@ -30,13 +30,14 @@ constexpr int kPackRecs = 1024;            // records per packing range (one CTA
 enum HwMode { kStats = 0, kQuant = 1, kRaw = 2 };
 
 // flags recorded in the payload header (everything but the I/O type)
-constexpr uint32_t kPayloadFlags =
-    TACTKV_NO_QUANT | TACTKV_SKIP_S | TACTKV_SKIP_H | TACTKV_SKIP_W | TACTKV_UNIFORM_ALLOC | TACTKV_ROTATE;
+constexpr uint32_t kPayloadFlags = TACTKV_NO_QUANT | TACTKV_SKIP_S | TACTKV_SKIP_H | TACTKV_SKIP_W |
+                                   TACTKV_UNIFORM_ALLOC | TACTKV_ROTATE | TACTKV_HEAD_GAIN;
 constexpr uint32_t kAllFlags = kPayloadFlags | TACTKV_FP32_IO;
 constexpr unsigned long long kRotationSeed = 0x544143544B56ull;
-// Variant flags (axis skips, shared rotation): kernels take a compile-time VAR switch and carry the
-// code for them only when it is set, so that the default kernels keep their register budgets.
-constexpr uint32_t kVariantFlags = TACTKV_SKIP_S | TACTKV_SKIP_H | TACTKV_SKIP_W | TACTKV_ROTATE;
+// Variant flags (axis skips, shared rotation, per-head gains): kernels take a compile-time VAR
+// switch and carry the code for them only when it is set, so that the default kernels keep their
+// register budgets.
+constexpr uint32_t kVariantFlags = TACTKV_SKIP_S | TACTKV_SKIP_H | TACTKV_SKIP_W | TACTKV_ROTATE | TACTKV_HEAD_GAIN;
 inline bool has_variant(int flags) { return (flags & kVariantFlags) != 0; }
 __host__ __device__ inline bool has_variant_dev(int flags) { return (flags & kVariantFlags) != 0; }
 
@@ -59,6 +60,13 @@ struct Geom {
 };
 
 __host__ __device__ inline long long pad16(long long x) { return (x + 15) / 16 * 16; }
+
+// Gain vectors of N floats in a payload: one per head with TACTKV_HEAD_GAIN on a quantized
+// payload (sigma[head][bin]), else one (sigma[bin]).
+__host__ __device__ inline bool head_gains_on(int flags) {
+  return (flags & TACTKV_HEAD_GAIN) && !(flags & TACTKV_NO_QUANT);
+}
+__host__ __device__ inline int gain_vectors(int flags, int heads) { return head_gains_on(flags) ? heads : 1; }
 
 // Per-unit index block in the workspace: P(k_s) for k_s = 0..S (first stream bit of each slab,
 // P(S) = code_bits), the decoder's ok flag, then NZ(k_s) for k_s = 0..S (first record of each slab
@@ -89,7 +97,6 @@ __host__ __device__ inline int length_class_dev(int L) { return L <= 16 ? 16 : (
 // instead of the two inverse kernels.  Both are read once per process.
 bool tc_s_pass_enabled();
 bool fused_decode_enabled();
-bool pack_seq_enabled();   // TACTKV_PACK_SEQ=1: the sequential bit-string packer
 
 
 // --------------------------------------------------------------------------------- launchers ---
@@ -180,6 +187,22 @@ __device__ __forceinline__ void dct_exact(V* x) {
 }
 
 __device__ __forceinline__ void set_status(unsigned int* status, unsigned int code) { atomicCAS(status, 0u, code); }
+
+// Sums over the 32 lanes of the warp of 32 values per lane (recursive halving: at each step a
+// lane keeps half of its values and adds the partner lane's copy of that half); lane l returns the
+// total of value l.
+__device__ __forceinline__ float warp_transpose_sum(float (&v)[32], int lane) {
+#pragma unroll
+  for (int h = 16; h >= 1; h >>= 1) {
+    const bool upper = lane & h;
+#pragma unroll
+    for (int i = 0; i < h; ++i) {
+      const float send = upper ? v[i] : v[i + h], keep = upper ? v[i + h] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, h);
+    }
+  }
+  return v[0];
+}
 
 // ------------------------------------------------------------------ shared shape rotation ---
 // Sign of channel c in the rotation: the top bit of output c of SplitMix64 (Steele, Lea and

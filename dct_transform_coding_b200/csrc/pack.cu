@@ -19,7 +19,8 @@
 // words first).  The CTA with the last record also writes the zero padding of the channel streams.
 //
 // With TACTKV_ROTATE every record's 32 coefficients (one bin, the CTA's 32 channels) are first
-// rotated by R = H_32 diag(s) / sqrt(32) across the warp (sign, Walsh-Hadamard, scale).
+// rotated by R = H_32 diag(s) / sqrt(32) across the warp (sign, Walsh-Hadamard, scale).  With
+// TACTKV_HEAD_GAIN the scale of a record is the reciprocal of its bin's gain in the CTA's head.
 //
 // NO_QUANT (raw) copies X into the channel streams as float32.
 #include "common.cuh"
@@ -136,6 +137,15 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const __grid_constan
     const int e = q * kPackThreads + (int)threadIdx.x;
     mine[q] = e < m ? urecs[r0 + e] : make_uint4(0u, 0u, 0u, 0u);
   }
+  if (VAR && head_gains_on(g.flags)) {   // 1/gain of the CTA's head (0 for a zero gain: u = 0)
+    const float* hg = reinterpret_cast<const float*>(pay + g.off_sigma) + (size_t)(chunk * kChunk / g.head_dim) * g.N;
+#pragma unroll
+    for (int q = 0; q < kPer; ++q)
+      if (mine[q].y) {
+        const float gh = hg[mine[q].x];
+        mine[q].w = gh > 0.f ? __float_as_uint(__frcp_rn(gh)) : 0u;
+      }
+  }
   if (threadIdx.x < 9 * kWarps) (&s_cnt[0][0])[threadIdx.x] = 0u;
   for (int i = threadIdx.x; i < TACTKV_THR_PAD_TOTAL; i += kPackThreads) thr[i] = c_thr_pad[i];
   for (int i = threadIdx.x; i < 6 * TACTKV_Q_CELLS; i += kPackThreads) qcell[i] = c_qcell[i];
@@ -241,118 +251,6 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const __grid_constan
   }
 }
 
-// ------------------------------------------------------------------ sequential bit strings ---
-// A second packer (selected with TACTKV_PACK_SEQ=1 while it is measured against the one above).
-// A warp owns kSeqRange consecutive records of one (unit, chunk), lane = channel.  The codes of
-// consecutive records are consecutive bits of every channel stream, so each lane ORs its codes
-// into a 64-bit register at offsets taken from the records' own stream positions (the only serial
-// chain is a few integer operations on warp-uniform values) and stores a word as soon as it is
-// complete.  The warp owns the words whose first bit lies in its range: it drops the bits in front
-// of its first owned word and finishes its last one from the next range's first records, so every
-// word is written once, by a plain store; nothing is cleared beforehand and nothing is atomic.
-constexpr int kSeqRange = 128;            // records per warp
-constexpr int kSeqExtra = 32;             // records staged past the range (a word holds < 32 codes)
-
-struct SeqLayout {
-  size_t rec, thr, qcell, total;
-};
-__host__ __device__ inline SeqLayout seq_layout() {
-  SeqLayout L;
-  auto p16 = [](size_t x) { return (x + 15) / 16 * 16; };
-  size_t o = 0;
-  L.rec = o; o += p16((size_t)(kPackThreads / 32) * (kSeqRange + kSeqExtra) * 16);
-  L.thr = o; o += p16((size_t)TACTKV_THR_PAD_TOTAL * 4);
-  L.qcell = o; o += p16((size_t)6 * TACTKV_Q_CELLS);
-  L.total = o;
-  return L;
-}
-
-__device__ __forceinline__ uint32_t quant_code_any(float x, float inv_sigma, int b, const float* __restrict__ thr,
-                                                   const unsigned char* __restrict__ qcell) {
-  if (b == 1) return quant_code_b<1>(x, inv_sigma, 1, thr, qcell);
-  if (b == 2) return quant_code_b<2>(x, inv_sigma, 2, thr, qcell);
-  return quant_code_b<0>(x, inv_sigma, b, thr, qcell);
-}
-
-template <bool VAR>
-__global__ void __launch_bounds__(kPackThreads) pack_seq_kernel(const __grid_constant__ Geom g,
-                                                                const __grid_constant__ UnitList ul,
-                                                                const float* __restrict__ X,
-                                                                const uint4* __restrict__ recs,
-                                                                const uint32_t* __restrict__ index) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  const SeqLayout L = seq_layout();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int chunk = blockIdx.x, u = blockIdx.z;
-  const uint32_t* P = index + (size_t)u * unit_index_words(g.S);
-  const uint32_t nrec = P[2 * g.S + 2], code_bits = P[g.S];
-  const uint4* urecs = recs + (size_t)u * g.N;
-  float* thr = reinterpret_cast<float*>(smem + L.thr);
-  unsigned char* qcell = smem + L.qcell;
-  uint4* rs = reinterpret_cast<uint4*>(smem + L.rec) + warp * (kSeqRange + kSeqExtra);
-  for (int i = threadIdx.x; i < TACTKV_THR_PAD_TOTAL; i += kPackThreads) thr[i] = c_thr_pad[i];
-  for (int i = threadIdx.x; i < 6 * TACTKV_Q_CELLS; i += kPackThreads) qcell[i] = c_qcell[i];
-  const uint32_t r0 = (blockIdx.y * (kPackThreads / 32) + warp) * kSeqRange;
-  const uint32_t r1 = min(nrec, r0 + kSeqRange);
-  const int staged = r0 < nrec ? (int)min((uint32_t)(kSeqRange + kSeqExtra), nrec - r0) : 0;
-  for (int e = lane; e < staged; e += 32) rs[e] = urecs[r0 + e];
-  __syncthreads();
-  if (r0 >= nrec) return;
-  __syncwarp();
-  unsigned char* pay = ul.u[u].payload;
-  const uint32_t sw = reinterpret_cast<const uint32_t*>(pay)[11] / 4;
-  uint32_t* out = reinterpret_cast<uint32_t*>(pay + g.off_codes) + (size_t)(chunk * kChunk + lane) * sw;
-  const float* xu = X + (size_t)u * g.N * g.n + chunk * kChunk + lane;
-  const bool rotate = VAR && (g.flags & TACTKV_ROTATE);
-  const float rot_in = rotate ? rotation_sign((unsigned long long)(chunk * kChunk + lane)) : 1.f;
-
-  const uint32_t A = rs[0].z;                                    // first bit of the range
-  const uint32_t end_bit = r1 < nrec ? rs[r1 - r0].z : code_bits;
-  const uint32_t first_word = (A + 31) >> 5;                     // words [first_word, ..) are ours
-  const uint32_t stop_bit = min(code_bits, ((end_bit + 31) >> 5) << 5);
-  int extra = 0;                                                 // next-range records that finish our last word
-  if (r1 < nrec) {
-    const uint32_t k = r1 - r0 + lane;
-    extra = __popc(__ballot_sync(0xffffffffu, (int)k < staged && rs[k].z < stop_bit));
-  }
-  const int m = (int)(r1 - r0) + extra;
-
-  unsigned long long acc = 0;
-  uint32_t w = A >> 5;            // the word acc's low half belongs to
-  float x[kPackBlock], xn[kPackBlock];
-#pragma unroll
-  for (int j = 0; j < kPackBlock; ++j) x[j] = j < m ? __ldcs(xu + (size_t)rs[j].x * g.n) : 0.f;
-  for (int e0 = 0; e0 < m; e0 += kPackBlock) {
-    const int e1 = e0 + kPackBlock;
-#pragma unroll
-    for (int j = 0; j < kPackBlock; ++j) xn[j] = e1 + j < m ? __ldcs(xu + (size_t)rs[e1 + j].x * g.n) : 0.f;
-    if (rotate) {
-#pragma unroll
-      for (int j = 0; j < kPackBlock; ++j) x[j] = warp_wht(x[j] * rot_in, lane) * 0.17677669529663687f;
-    }
-#pragma unroll
-    for (int j = 0; j < kPackBlock; ++j) {
-      if (e0 + j < m) {
-        const uint4 r = rs[e0 + j];
-        const int b = (int)r.y;
-        const uint32_t rel = r.z - (w << 5);                     // < 32: words are stored as they fill
-        acc |= (unsigned long long)quant_code_any(x[j], __uint_as_float(r.w), b, thr, qcell) << rel;
-        if (rel + (uint32_t)b >= 32u) {
-          if (w >= first_word) out[w] = (uint32_t)acc;
-          acc >>= 32;
-          ++w;
-        }
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < kPackBlock; ++j) x[j] = xn[j];
-  }
-  const uint32_t last_end = rs[m - 1].z + rs[m - 1].y;           // first bit after the last code
-  if (last_end > (w << 5) && w >= first_word && (w << 5) < stop_bit) out[w] = (uint32_t)acc;   // the streams' last word
-  if (r1 == nrec)   // zero padding of the streams after the last code bit
-    for (uint32_t z = (code_bits + 31) >> 5; z < sw; ++z) out[z] = 0u;
-}
-
 // NO_QUANT: the float32 coefficients of every bin into the channel streams (stream c holds X[i, c]
 // at byte 4i), then the zero padding up to the channel stride.
 __global__ void __launch_bounds__(kPackThreads) pack_raw_kernel(const __grid_constant__ Geom g,
@@ -383,14 +281,6 @@ cudaError_t launch_pack(const Geom& g, const UnitList& ul, int nu, const float* 
     const int spc = 1;
     pack_raw_kernel<<<dim3(g.nch, g.S, nu), kPackThreads, 0, st>>>(g, ul, X, spc);
   } else {
-    if (pack_seq_enabled()) {
-      const SeqLayout L = seq_layout();
-      auto kernel = has_variant(g.flags) ? pack_seq_kernel<true> : pack_seq_kernel<false>;
-      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
-      const dim3 grid(g.nch, (g.N + (kPackThreads / 32) * kSeqRange - 1) / ((kPackThreads / 32) * kSeqRange), nu);
-      kernel<<<grid, kPackThreads, L.total, st>>>(g, ul, X, recs, index);
-      return cudaGetLastError();
-    }
     const PackLayout L = pack_layout();
     auto kernel = has_variant(g.flags) ? pack_kernel<true> : pack_kernel<false>;
     cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);

@@ -100,6 +100,7 @@ void axis_hw_shape(int hcls, int wcls, const Geom& g, bool inverse, int mode, si
 
 size_t attention_scores_smem(const Geom& g, int q_heads);
 size_t attention_values_smem(const Geom& g, int q_heads);
+size_t attention_softmax_smem(const Geom& g);
 cudaError_t launch_attention(const Geom& g, const UnitList& kl, const UnitList& vl, int nu, int q_heads,
                              const uint32_t* kidx, const uint4* krec, const uint32_t* vidx, const uint4* vrec,
                              const float* q, float* zp, float* part, float* out, float* m, float* l,
@@ -108,14 +109,6 @@ cudaError_t launch_attention(const Geom& g, const UnitList& kl, const UnitList& 
 bool tc_s_pass_enabled() {
   static const bool on = [] {
     const char* e = getenv("TACTKV_TC_S");
-    return e && e[0] == '1';
-  }();
-  return on;
-}
-
-bool pack_seq_enabled() {
-  static const bool on = [] {
-    const char* e = getenv("TACTKV_PACK_SEQ");
     return e && e[0] == '1';
   }();
   return on;
@@ -139,6 +132,8 @@ tactkv_status make_geom(const tactkv_unit& u, Geom& g) {
   if (u.H > 32 || u.W > 32 || u.H * u.W > kMaxHW) return TACTKV_UNSUPPORTED_SHAPE;
   const long long n = (long long)u.heads * u.head_dim;
   if (n % kChunk != 0 || u.head_dim % 2 != 0 || n > (1 << 16)) return TACTKV_UNSUPPORTED_SHAPE;
+  // per-head gains: every 32-channel chunk lies inside one head
+  if (head_gains_on((int)u.flags) && u.head_dim % kChunk != 0) return TACTKV_UNSUPPORTED_SHAPE;
   const long long N = (long long)u.S * u.H * u.W;
   g.S = u.S;
   g.H = u.H;
@@ -153,7 +148,7 @@ tactkv_status make_geom(const tactkv_unit& u, Geom& g) {
   g.bits = u.bits;
   g.flags = (int)u.flags;
   g.off_sigma = (int)(kHeaderBytes + pad16(g.N));
-  g.off_codes = (int)(g.off_sigma + pad16(4LL * g.N));
+  g.off_codes = (int)(g.off_sigma + pad16(4LL * g.N * gain_vectors(g.flags, g.heads)));
   g.capacity = 0;
   g.unit0 = 0;
   return TACTKV_OK;
@@ -456,6 +451,7 @@ tactkv_status tactkv_allocate(const tactkv_unit* unit, const double* var, void* 
   Geom g;
   tactkv_status st = make_geom(*unit, g);
   if (st != TACTKV_OK) return st;
+  if (head_gains_on(g.flags)) return TACTKV_INVALID_ARG;   // per-head gains need the channels, not variances
   if (reinterpret_cast<uintptr_t>(unit->payload) % 16 || reinterpret_cast<uintptr_t>(var) % 8) return TACTKV_ALIGNMENT;
   if (unit->payload_capacity < payload_bytes_geom(g)) return TACTKV_CAPACITY;
   g.capacity = (long long)unit->payload_capacity;
@@ -513,7 +509,7 @@ tactkv_status attn_check(const tactkv_unit* k_units, const tactkv_unit* v_units,
   if ((g.flags & TACTKV_NO_QUANT) || q_heads < g.heads || q_heads % g.heads || q_heads / g.heads > 16 ||
       g.head_dim % kChunk)
     return TACTKV_UNSUPPORTED_SHAPE;
-  if ((size_t)g.N * 4 > 227 * 1024 || attention_scores_smem(g, q_heads) > 227 * 1024 ||
+  if (attention_softmax_smem(g) > 227 * 1024 || attention_scores_smem(g, q_heads) > 227 * 1024 ||
       attention_values_smem(g, q_heads) > 227 * 1024)
     return TACTKV_UNSUPPORTED_SHAPE;
   long long cap = -1;
@@ -631,7 +627,8 @@ tactkv_status tactkv_occupancy(const void* payload, size_t bytes, tactkv_occupan
   out->bins = N;
   out->channels = n;
   out->code_bits = code_bits;
-  out->formula_bits = code_bits * n + 32ull * N;
+  // one 32-bit gain per gain-shape vector: per bin, or per (bin, head) with per-head gains
+  out->formula_bits = code_bits * n + 32ull * N * (unsigned long long)gain_vectors((int)(h32[1] >> 16), (int)heads);
   out->index_bits = 8ull * N;
   out->payload_bytes = total;
   out->bits_per_element = 8.0 * (double)total / ((double)N * (double)n);

@@ -39,6 +39,7 @@ TACTKV_SKIP_H = 8
 TACTKV_SKIP_W = 16
 TACTKV_UNIFORM_ALLOC = 32
 TACTKV_ROTATE = 64
+TACTKV_HEAD_GAIN = 128
 
 HEADER_BYTES = 64
 EXPORTED = ("tactkv_payload_bytes", "tactkv_workspace_bytes", "tactkv_compress", "tactkv_decompress",

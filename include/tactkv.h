@@ -32,7 +32,8 @@
  *                       or 32*N with TACTKV_NO_QUANT), u32 chan_stride (bytes), u64 total_bytes,
  *                       u32 0, u32 0
  *   [64, +pad16(N))     u8 b[N]          bits of every bin (0..8; 0 = dropped)
- *   then pad16(4N)      f32 sigma[N]     gain of every bin, float32(sqrt(sigma^2))
+ *   then pad16(4N)      f32 sigma[N]     gain of every bin, float32(sqrt(sigma^2)); with
+ *                       TACTKV_HEAD_GAIN pad16(4*heads*N) bytes, f32 sigma[heads][N]
  *   then n streams      channel c at offset off_codes + c*chan_stride, chan_stride =
  *                       pad16(ceil(code_bits/8)); stream bit P_i + k is bit k (LSB first) of bin
  *                       i's code, P_i = sum_{j<i} b_j; stream bit q is bit (q&7) of byte q>>3.
@@ -79,12 +80,20 @@ typedef enum {
                               the 32-channel groups, H_32 diag(s) / sqrt(32) with H_32 the
                               Sylvester-Hadamard matrix and s_c = -1 exactly when bit 63 of output c
                               of SplitMix64 seeded with 0x544143544B56 is set (ignored with
-                              TACTKV_NO_QUANT).  Gains and allocation are unchanged by it. */
+                              TACTKV_NO_QUANT).  Gains and allocation are unchanged by it;
+     TACTKV_HEAD_GAIN         one gain per (bin, head) instead of one per bin: the gain-shape
+                              vectors of stage 4 are a bin's head_dim coordinates in one head
+                              (the d of stage 4's occupancy sum), each scaled by
+                              float32(sqrt(mean over the head's channels of X^2)) and decoded with
+                              it (a zero gain scales by 0).  The bit allocation still uses the
+                              variance pooled over all channels.  Needs head_dim a multiple of 32;
+                              the payload then holds sigma[heads][N] (ignored with TACTKV_NO_QUANT). */
 #define TACTKV_SKIP_S        4u
 #define TACTKV_SKIP_H        8u
 #define TACTKV_SKIP_W       16u
 #define TACTKV_UNIFORM_ALLOC 32u
 #define TACTKV_ROTATE       64u
+#define TACTKV_HEAD_GAIN   128u
 
 typedef struct {
   int32_t layer;          /* recorded in the header, checked by decompress */
@@ -171,7 +180,8 @@ tactkv_status tactkv_compress_noalloc(const tactkv_unit* units, int n_units,
    the B = bits*N largest keys var_i * 4^-k, k = 0..7, ties to the lower bin index, every active bin
    at 8 bits when 8*#active <= B; b = 0 where var = 0), sigma[N] = float32(sqrt(var)) and the zero
    padding; the code area is left unspecified.  Only the unit's shape, bits, flags, layer, kv,
-   payload and payload_capacity are read.  workspace: at least tactkv_workspace_bytes(unit, 1)
+   payload and payload_capacity are read.  TACTKV_HEAD_GAIN is refused (TACTKV_INVALID_ARG): its
+   gains come from the channels, which this call does not see.  workspace: at least tactkv_workspace_bytes(unit, 1)
    bytes, 256-byte aligned.  Asynchronous on `stream`; one kernel. */
 tactkv_status tactkv_allocate(const tactkv_unit* unit, const double* var, void* workspace,
                               size_t workspace_bytes, struct CUstream_st* stream);
@@ -187,7 +197,10 @@ tactkv_status tactkv_allocate(const tactkv_unit* unit, const double* var, void* 
                  out_j = sum_t softmax_t(q_j . K[t] / sqrt(head_dim)) V[t] over the S*H*W visual tokens;
      m, l      DEVICE float32 [n_units][q_heads]: the scores' maximum and sum_t exp(score - m), so
                that a caller can merge these tokens with its bf16 text tokens.
-   Limits: n_units <= 128, S*H*W <= 58112, head_dim a multiple of 32.  workspace: at least
+   Limits: n_units <= 128, head_dim a multiple of 32, and shared memory for one slab's stream words
+   of a head (head_dim * ((8*H*W + 31)/32 + 3, rounded up to odd) 4-byte words) and for the score
+   volume (S*H*(W rounded up to odd) floats) within 227 KB each; other shapes return
+   TACTKV_UNSUPPORTED_SHAPE (every benchmark grid fits).  workspace: at least
    tactkv_attention_workspace_bytes(k_units, n_units, q_heads) bytes, 256-byte aligned.  A corrupt
    payload is recorded as TACTKV_CORRUPT_PAYLOAD (tactkv_device_status) and contributes no
    tokens of its unit.  Asynchronous on `stream`; 5 kernels. */
@@ -211,13 +224,14 @@ const char* tactkv_status_string(tactkv_status status);
 int tactkv_lloyd_max_table(int bits, double* levels, double* thresholds);
 
 /* Occupancy of one compressed unit ("Methodology in Plain English", stage 4: a layer's cache takes
-   sum_i (b_i * d + 32) bits plus a small index).  Here d is the number of channels sharing a
-   gain, n = heads*head_dim, and the index is the byte b_i of every bin. */
+   sum_i (b_i * d + 32) bits plus a small index).  The sum runs over the gain-shape vectors: one per
+   bin with d = n = heads*head_dim, or, with TACTKV_HEAD_GAIN, one per (bin, head) with
+   d = head_dim.  The index is the byte b_i of every bin. */
 typedef struct {
   uint64_t bins;            /* N */
   uint64_t channels;        /* n */
   uint64_t code_bits;       /* sum_i b_i, the bits of one channel stream */
-  uint64_t formula_bits;    /* sum_i (b_i * n + 32): codes and gains */
+  uint64_t formula_bits;    /* sum_i (b_i * n + 32 * gains per bin): codes and gains */
   uint64_t index_bits;      /* 8 * N: the bit widths */
   uint64_t payload_bytes;   /* the payload's actual size (header, padding and alignment included) */
   double bits_per_element;  /* 8 * payload_bytes / (N * n) */

@@ -70,9 +70,11 @@ def compare_unit(x: np.ndarray, gpu_payload: bytes, gpu_recon: np.ndarray, *, S,
     N = S * H * W
     var = info["var"]
     # gains: float32(sqrt(sigma^2)) from fp32 coefficients and fp64 sums
+    # (per-head gains: [heads, N], each head's gains against the same relative floor)
     sig_o = info["sigma"].astype(np.float64)
     sig_g = g["sigma"].astype(np.float64)
-    big = var > 1e-12 * max(var.max(), 1e-300)
+    assert sig_g.shape == sig_o.shape
+    big = sig_o > 1e-6 * max(sig_o.max(), 1e-300)
     assert np.all(np.abs(sig_g[big] - sig_o[big]) <= 2e-5 * sig_o[big]), "gain mismatch"
     out = dict(alloc_margin=np.inf, code_mismatch_band=0, codes=0)
     if no_quant:
@@ -97,7 +99,8 @@ def compare_unit(x: np.ndarray, gpu_payload: bytes, gpu_recon: np.ndarray, *, S,
             bad = codes_g[i] != codes_o[i]
             out["codes"] += codes_o.shape[1]
             if bad.any():
-                u = X[i, bad] / sig_o[i]
+                gain = np.repeat(sig_o[:, i], head_dim) if sig_o.ndim == 2 else np.full(X.shape[1], sig_o[i])
+                u = np.divide(X[i, bad], gain[bad], out=np.zeros(int(bad.sum())), where=gain[bad] > 0)
                 d = O.threshold_distance(u, int(b_o[i]))
                 assert np.all(d <= CODE_BAND), f"code mismatch outside the band at bin {i}: {d.max()}"
                 out["code_mismatch_band"] += int(bad.sum())

@@ -52,13 +52,14 @@ def _run(S, H, W, heads, D, G, bits, flags=0, units=2, qscale=1.0, seed=0):
     (16, 16, 16, 2, 64, 4, 1),
     (5, 7, 6, 2, 32, 3, 3),        # ragged grid
     (64, 16, 16, 4, 256, 2, 1),    # the 4B-class medical layout (one layer)
+    (4, 24, 24, 2, 128, 4, 2),     # the 32B-class slab (24 x 24 cells, 128 channels per head)
 ])
 def test_attention_matches_oracle(S, H, W, heads, D, G, bits):
     _run(S, H, W, heads, D, G, bits)
 
 
-@pytest.mark.parametrize("flags", [T.TACTKV_ROTATE if torch.cuda.is_available() else 64,
-                                   (T.TACTKV_SKIP_S | T.TACTKV_UNIFORM_ALLOC) if torch.cuda.is_available() else 36])
+@pytest.mark.parametrize("flags", [64, 4 | 32, 128, 128 | 64],
+                         ids=["rotate", "skip_s_uniform", "head_gain", "head_gain_rotate"])
 def test_attention_with_variant_flags(flags):
     _run(16, 8, 8, 2, 64, 2, 2, flags=flags, seed=5)
 

@@ -305,17 +305,18 @@ def test_fused_grid_output_variants(S, H, W, flags, dtype):
 
 
 # ---------------------------------------------------------------- ablation and rotation flags ---
-@pytest.mark.parametrize("shape", [(16, 16, 16, 2, 64), (5, 7, 6, 1, 96)], ids=["fused-grid", "ragged-grid"])
+@pytest.mark.parametrize("shape", [(16, 16, 16, 2, 64), (5, 7, 6, 3, 32)], ids=["fused-grid", "ragged-grid"])
 @pytest.mark.parametrize("variant", ["no_dct", "hw_only", "s_only", "w_only", "uniform", "rotate",
-                                     "rotate_uniform_hw"])
+                                     "rotate_uniform_hw", "head_gain", "head_gain_rotate"])
 def test_variant_flags(shape, variant):
-    """The summary page's ablations ("Main Findings": fewer transformed axes, uniform allocation)
-    and stage 4's fixed shared rotation, as flags: payload, codes and reconstruction against the
-    oracle run with the same flags."""
+    """The summary page's ablations ("Main Findings": fewer transformed axes, uniform allocation),
+    stage 4's fixed shared rotation and per-head gains, as flags: payload, codes and reconstruction
+    against the oracle run with the same flags."""
     flags = {"no_dct": T.TACTKV_SKIP_S | T.TACTKV_SKIP_H | T.TACTKV_SKIP_W, "hw_only": T.TACTKV_SKIP_S,
              "s_only": T.TACTKV_SKIP_H | T.TACTKV_SKIP_W, "w_only": T.TACTKV_SKIP_S | T.TACTKV_SKIP_H,
              "uniform": T.TACTKV_UNIFORM_ALLOC, "rotate": T.TACTKV_ROTATE,
-             "rotate_uniform_hw": T.TACTKV_ROTATE | T.TACTKV_UNIFORM_ALLOC | T.TACTKV_SKIP_S}[variant]
+             "rotate_uniform_hw": T.TACTKV_ROTATE | T.TACTKV_UNIFORM_ALLOC | T.TACTKV_SKIP_S,
+             "head_gain": T.TACTKV_HEAD_GAIN, "head_gain_rotate": T.TACTKV_HEAD_GAIN | T.TACTKV_ROTATE}[variant]
     S, H, W, heads, D = shape
     x = torch.stack([make_unit(S, H, W, heads, D, rho=(0.9, 0.85, 0.8), nu=4.0, seed=300 + i, device=DEV)
                      for i in range(2)])
@@ -329,6 +330,20 @@ def test_variant_flags(shape, variant):
         T.decompress(pay, S, H, W, 2, heads=heads, head_dim=D, layers=[0, 1], kvs=[1, 1], flags=0, check=True)
 
 
+def test_head_gain_scaled_copy_of_a_head():
+    """Per-head gains on the GPU: head 1 = 4 x head 0 (exact in bf16 and in every float32 step)
+    gives head 1 exactly 4 x head 0's gains and exactly head 0's codes, on a fused grid."""
+    S, H, W, D = 16, 16, 16, 64
+    x0 = make_unit(S, H, W, 1, D, rho=(0.9, 0.85, 0.85), nu=4.0, seed=77, device=DEV)
+    x = torch.cat([x0, x0 * 4], dim=1)[None]
+    reports, pay, _ = _check_batch(x, S, H, W, 3, flags=T.TACTKV_HEAD_GAIN)
+    p = O.parse_payload(pay[0].cpu().numpy().tobytes())
+    assert p["sigma"].shape == (2, S * H * W) and np.array_equal(p["sigma"][1], 4 * p["sigma"][0])
+    b, codes = O.codes_of(pay[0].cpu().numpy().tobytes())
+    act = b > 0
+    assert np.array_equal(codes[act][:, D:], codes[act][:, :D])
+
+
 def test_opt_in_tensor_core_kernels():
     """The opt-in tensor-core forms, read once per process: the forward kernel's DCT along S on
     tcgen05 (TACTKV_TC_S=1) and the single-kernel decode with the inverse S on tcgen05
@@ -336,7 +351,7 @@ def test_opt_in_tensor_core_kernels():
     import os
     import subprocess
     import sys
-    env = dict(os.environ, TACTKV_TC_S="1", TACTKV_FUSED_DECODE="1", TACTKV_PACK_SEQ="1")
+    env = dict(os.environ, TACTKV_TC_S="1", TACTKV_FUSED_DECODE="1")
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     r = subprocess.run([sys.executable, "-m", "pytest", "tests/test_gpu_parity.py", "-q", "-x", "-m", "gpu",
                         "-p", "no:cacheprovider", "-k",

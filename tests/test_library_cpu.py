@@ -52,11 +52,13 @@ def test_codebook_rejects_bad_bits(T):
 
 @pytest.mark.parametrize("shape,bits,flags", [((64, 16, 16, 4, 256), 1, 0), ((32, 24, 24, 8, 128), 1, 0),
                                               ((64, 14, 14, 4, 128), 4, 0), ((8, 8, 8, 1, 64), 2, 0),
-                                              ((8, 8, 8, 1, 64), 2, 1), ((5, 7, 3, 2, 32), 8, 0)])
+                                              ((8, 8, 8, 1, 64), 2, 1), ((5, 7, 3, 2, 32), 8, 0),
+                                              ((64, 16, 16, 4, 256), 1, 128), ((5, 7, 3, 2, 32), 3, 128),
+                                              ((8, 8, 8, 2, 64), 2, 129)])
 def test_payload_capacity_matches_oracle_layout(T, shape, bits, flags):
     S, H, W, heads, D = shape
     cap = T.payload_capacity(S, H, W, heads, D, bits, flags)
-    assert cap == O.payload_capacity(S, H, W, heads, D, bits, no_quant=bool(flags & 1))
+    assert cap == O.payload_capacity(S, H, W, heads, D, bits, flags=flags)
 
 
 def test_unsupported_shapes_report_zero_capacity(T):
@@ -75,7 +77,8 @@ def _unit(T, **kw):
 
 @pytest.mark.parametrize("kw,status", [
     (dict(bits=0), "TACTKV_INVALID_ARG"), (dict(bits=9), "TACTKV_INVALID_ARG"),
-    (dict(flags=128), "TACTKV_INVALID_ARG"), (dict(S=0), "TACTKV_INVALID_ARG"),
+    (dict(flags=256), "TACTKV_INVALID_ARG"), (dict(S=0), "TACTKV_INVALID_ARG"),
+    (dict(flags=128, heads=2, head_dim=48), "TACTKV_UNSUPPORTED_SHAPE"),   # per-head gains: head_dim % 32
     (dict(kv_in=None), "TACTKV_INVALID_ARG"), (dict(payload=None), "TACTKV_INVALID_ARG"),
     (dict(token_stride=0), "TACTKV_INVALID_ARG"),
     (dict(S=17), "TACTKV_UNSUPPORTED_SHAPE"), (dict(head_dim=30), "TACTKV_UNSUPPORTED_SHAPE"),
@@ -111,6 +114,8 @@ def test_allocate_argument_checks_without_gpu(T):
     need = T.tactkv_workspace_bytes([u])
     assert T.tactkv_allocate(u, 4096, 1 << 20, need - 1, 0) == T.TACTKV_WORKSPACE
     assert T.tactkv_allocate(u, 4096, 0, need, 0) == T.TACTKV_WORKSPACE
+    # per-head gains come from the channels, which the given variances do not carry
+    assert T.tactkv_allocate(_unit(T, flags=128), 4096, 1 << 20, 1 << 30, 0) == T.TACTKV_INVALID_ARG
 
 
 def test_decompress_checks_output_pointer(T):
@@ -173,6 +178,18 @@ def test_occupancy_of_an_oracle_payload(T, bits):
     assert occ["payload_bytes"] == len(p)
     assert abs(occ["bits_per_element"] - 8 * len(p) / (N * n)) < 1e-12
     assert abs(occ["shrink_vs_bf16"] - 2 * N * n / len(p)) < 1e-12
+
+
+def test_occupancy_with_per_head_gains(T):
+    """With per-head gains the stage-4 sum runs over (bin, head) vectors of head_dim channels: one
+    32-bit gain per bin and head."""
+    S, H, W, heads, D = 4, 6, 5, 3, 32
+    x = np.random.default_rng(3).standard_normal((S * H * W, heads, D))
+    p, info = O.compress_unit(x, S, H, W, heads, D, 2, return_info=True, flags=O.FLAG_HEAD_GAIN)
+    occ = T.tactkv_occupancy(p)
+    assert occ["formula_bits"] == O.occupancy_bits(info["b"], D, heads)
+    assert occ["payload_bytes"] == len(p)
+    assert occ["formula_bits"] - O.occupancy_bits(info["b"], heads * D) == 32 * (heads - 1) * S * H * W
 
 
 def test_occupancy_rejects_corrupt_payloads(T):
