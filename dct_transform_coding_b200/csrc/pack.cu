@@ -79,6 +79,13 @@ __device__ __forceinline__ uint32_t quant_code_b(float x, float inv_sigma, int b
   }
 }
 
+// OR into a shared-memory word without reading the old value back (a reduction, not an atomic
+// with a result): nothing waits for it, so consecutive codes of a warp do not stall on each other.
+__device__ __forceinline__ void red_or_shared(uint32_t* p, uint32_t v) {
+  asm volatile("red.shared.or.b32 [%0], %1;\n" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))), "r"(v)
+               : "memory");
+}
+
 // One block of kPackBlock records, all of width b (= B when B > 0): quantize x[] and OR the codes
 // into the row (a code of more than one bit may straddle into the next word).  The records, the
 // word row and the tables do not overlap, so the record loads need not wait for the atomics.
@@ -91,9 +98,9 @@ __device__ __forceinline__ void pack_block(const uint4* __restrict__ rs, const f
     const uint2 r = reinterpret_cast<const uint2*>(rs + j)[1];   // {stream position, 1/sigma}
     const uint32_t code = quant_code_b<B>(x[j], __uint_as_float(r.y), b, thr, qcell);
     const uint32_t off = r.x - base, w = off >> 5, sh = off & 31u;
-    atomicOr(row + w, code << sh);
+    red_or_shared(row + w, code << sh);
     if constexpr (B != 1) {
-      if (sh + (uint32_t)b > 32u) atomicOr(row + w + 1, code >> (32u - sh));
+      if (sh + (uint32_t)b > 32u) red_or_shared(row + w + 1, code >> (32u - sh));
     }
   }
 }
