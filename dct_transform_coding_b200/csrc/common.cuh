@@ -97,7 +97,6 @@ __host__ __device__ inline int length_class_dev(int L) { return L <= 16 ? 16 : (
 // instead of the two inverse kernels.  Both are read once per process.
 bool tc_s_pass_enabled();
 bool fused_decode_enabled();
-bool unit_waves_enabled();   // TACTKV_UNIT_WAVES=1: inverse kernels one unit at a time (measurement)
 
 
 // --------------------------------------------------------------------------------- launchers ---

@@ -89,18 +89,24 @@ __device__ __forceinline__ void red_or_shared(uint32_t* p, uint32_t v) {
 // One block of kPackBlock records, all of width b (= B when B > 0): quantize x[] and OR the codes
 // into the row (a code of more than one bit may straddle into the next word).  The records, the
 // word row and the tables do not overlap, so the record loads need not wait for the atomics.
+// In three phases -- the block's records, then its codes, then the ORs -- so that the loads of one
+// phase are all in flight together instead of each waiting behind the previous record's OR.
 template <int B>
 __device__ __forceinline__ void pack_block(const uint4* __restrict__ rs, const float (&x)[kPackBlock],
                                            uint32_t* __restrict__ row, uint32_t base, int b,
                                            const float* __restrict__ thr, const unsigned char* __restrict__ qcell) {
+  uint2 r[kPackBlock];
+#pragma unroll
+  for (int j = 0; j < kPackBlock; ++j) r[j] = reinterpret_cast<const uint2*>(rs + j)[1];   // {position, 1/sigma}
+  uint32_t code[kPackBlock];
+#pragma unroll
+  for (int j = 0; j < kPackBlock; ++j) code[j] = quant_code_b<B>(x[j], __uint_as_float(r[j].y), b, thr, qcell);
 #pragma unroll
   for (int j = 0; j < kPackBlock; ++j) {
-    const uint2 r = reinterpret_cast<const uint2*>(rs + j)[1];   // {stream position, 1/sigma}
-    const uint32_t code = quant_code_b<B>(x[j], __uint_as_float(r.y), b, thr, qcell);
-    const uint32_t off = r.x - base, w = off >> 5, sh = off & 31u;
-    red_or_shared(row + w, code << sh);
+    const uint32_t off = r[j].x - base, w = off >> 5, sh = off & 31u;
+    red_or_shared(row + w, code[j] << sh);
     if constexpr (B != 1) {
-      if (sh + (uint32_t)b > 32u) red_or_shared(row + w + 1, code >> (32u - sh));
+      if (sh + (uint32_t)b > 32u) red_or_shared(row + w + 1, code[j] >> (32u - sh));
     }
   }
 }
@@ -108,7 +114,7 @@ __device__ __forceinline__ void pack_block(const uint4* __restrict__ rs, const f
 // VAR: the payload has variant flags (the shared rotation), a compile-time switch so that the
 // default kernel keeps its register budget.
 template <bool VAR>
-__global__ void __launch_bounds__(kPackThreads) pack_kernel(const __grid_constant__ Geom g,
+__global__ void __launch_bounds__(kPackThreads, 4) pack_kernel(const __grid_constant__ Geom g,
                                                             const __grid_constant__ UnitList ul,
                                                             const float* __restrict__ X, const uint4* __restrict__ recs,
                                                             const uint32_t* __restrict__ index) {

@@ -114,14 +114,6 @@ bool tc_s_pass_enabled() {
   return on;
 }
 
-bool unit_waves_enabled() {
-  static const bool on = [] {
-    const char* e = getenv("TACTKV_UNIT_WAVES");
-    return e && e[0] == '1';
-  }();
-  return on;
-}
-
 bool fused_decode_enabled() {
   static const bool on = [] {
     const char* e = getenv("TACTKV_FUSED_DECODE");
@@ -400,19 +392,6 @@ static tactkv_status decompress_impl(const tactkv_unit* units, int n_units, void
                                                               : cudaErrorNotSupported;
                          if (fe == cudaSuccess) {
                            t_launches += 1;   // idct3 (decode, inverse H/W, inverse S)
-                           mark(2);
-                         } else if (fe == cudaErrorNotSupported && unit_waves_enabled()) {
-                           // one unit at a time: its V is read back by idct_s while it is still in L2
-                           const int spc1 = slabs_per_cta(g, 1, true, mode);
-                           for (int k = 0; k < nu; ++k) {
-                             Geom g1 = g;
-                             g1.unit0 = k;
-                             t_launches += 2;
-                             if (launch_axis_hw(ch, cw, true, mode, g1, ul, 1, w.big, nullptr, w.index, w.recs, spc1,
-                                                st) != cudaSuccess)
-                               return TACTKV_CUDA;
-                             if (launch_axis_s(cs, true, g1, ul, 1, w.big, st) != cudaSuccess) return TACTKV_CUDA;
-                           }
                            mark(2);
                          } else if (fe == cudaErrorNotSupported) {
                            t_launches += 2;   // idct_hw, idct_s
