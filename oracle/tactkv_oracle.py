@@ -32,7 +32,7 @@ Readings taken where the pages are silent (each is listed in the design notes):
 * A code is the number of thresholds t_j <= u with u = X / sigma_i; the decision is taken in
   float32 (the precision of the CUDA kernels), ties go to the upper cell, outer cells saturate.
 * The fixed shared rotation of the shape vector named in stage 4 is optional (FLAG_ROTATE, off by
-  default, as in the codec's specification).  Reading of "fixed shared orthogonal rotation": the
+  default, as in the codec's specification).  Reading of the fixed, shared orthogonal rotation: the
   same orthogonal matrix R for every bin, layer and sequence, block-diagonal over groups of 32
   consecutive channels, R_g = (1/sqrt(32)) H_32 D_g with H_32 the Sylvester-Hadamard matrix and D_g
   a diagonal of signs drawn once from a counter-based SplitMix64 (see ``rotation_signs``).  It
