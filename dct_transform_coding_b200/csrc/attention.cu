@@ -270,14 +270,26 @@ __device__ float block_reduce(float v, float* red, bool is_max) {
 // Per query head: scores = idct3(z), p = exp(scores - max), l = sum p, then dct3(p) over z's place.
 // SX, HX, WX > 0: the grid's lengths fixed at compile time (the benchmark grids), 0: any grid.
 constexpr int kSoftmaxThreads = 512;
+// A unit whose K or V payload failed the index checks contributes no tokens: p = 0, m = -inf, l = 0.
 template <int SX, int HX, int WX>
 __global__ void __launch_bounds__(kSoftmaxThreads) attn_softmax_kernel(const __grid_constant__ Geom g,
+                                                                    const uint32_t* __restrict__ kidx,
+                                                                    const uint32_t* __restrict__ vidx,
                                                                     float* __restrict__ zp, float* __restrict__ m_out,
                                                                     float* __restrict__ l_out, int q_heads) {
   extern __shared__ __align__(16) float vol[];
   __shared__ float red[32];
   const int j = blockIdx.x, u = blockIdx.y;
   float* zg = zp + ((size_t)u * q_heads + j) * g.N;
+  const size_t iw = (size_t)unit_index_words(g.S);
+  if (kidx[u * iw + g.S + 1] == 0u || vidx[u * iw + g.S + 1] == 0u) {   // the same for the whole CTA
+    for (int i = threadIdx.x; i < g.N; i += blockDim.x) zg[i] = 0.f;
+    if (threadIdx.x == 0) {
+      m_out[(size_t)u * q_heads + j] = -INFINITY;
+      l_out[(size_t)u * q_heads + j] = 0.f;
+    }
+    return;
+  }
   const int W = g.W, Wr = vol_row(W);
   auto at = [&](int i) { return (i / W) * Wr + (i - (i / W) * W); };   // bin i -> its padded place
   for (int i = threadIdx.x; i < g.N; i += blockDim.x) vol[at(i)] = zg[i];
@@ -373,7 +385,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_reduce_kernel(const __grid_
                                                                    const float* __restrict__ l_in, int q_heads,
                                                                    float* __restrict__ out) {
   const int j = blockIdx.x, u = blockIdx.y, D = g.head_dim, G = q_heads / g.heads, h = j / G;
-  const float inv_l = 1.f / l_in[(size_t)u * q_heads + j];
+  const float lj = l_in[(size_t)u * q_heads + j];
+  const float inv_l = lj > 0.f ? 1.f / lj : 0.f;   // l = 0: a unit without tokens (corrupt payload)
   const bool rotate = g.flags & TACTKV_ROTATE;
   const int lane = threadIdx.x & 31;
   for (int d0 = 0; d0 < D; d0 += blockDim.x) {
@@ -423,7 +436,7 @@ cudaError_t launch_attention(const Geom& g, const UnitList& kl, const UnitList& 
   auto values = q_heads / g.heads <= 4 ? attn_values_kernel<4> : attn_values_kernel<kMaxG>;
   cudaFuncSetAttribute(values, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s3);
   attn_scores_kernel<<<dim3(g.S, g.heads, nu), kScoreThreads, s1, st>>>(g, kl, kidx, krec, q, q_heads, zp);
-  softmax<<<dim3(q_heads, nu), kSoftmaxThreads, s2, st>>>(g, zp, m, l, q_heads);
+  softmax<<<dim3(q_heads, nu), kSoftmaxThreads, s2, st>>>(g, kidx, vidx, zp, m, l, q_heads);
   values<<<dim3(g.S, g.heads, nu), values_threads(g.head_dim), s3, st>>>(g, vl, vidx, vrec, zp, q_heads, part);
   attn_reduce_kernel<<<dim3(q_heads, nu), kAttnThreads, 0, st>>>(g, part, l, q_heads, out);
   return cudaGetLastError();

@@ -36,9 +36,8 @@ constexpr int kFusedThreads = STile<kNC>::kThreads;
 static_assert(kFusedThreads == kMaxHwThreads, "the H/W pieces run with the same block");
 
 // Every thread of every CTA of the cluster: global writes before it are visible to the cluster's
-// reads after it.
+// reads after it (release and acquire at cluster scope; the reads are ordinary cp.async copies).
 __device__ __forceinline__ void cluster_barrier() {
-  __threadfence();
   asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
   asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
 }

@@ -53,8 +53,10 @@ __device__ __forceinline__ const uint16_t* dct_limb_inv() {
   else return &kDctLimbInv64[0][0][0];
 }
 
+// Every thread of every CTA of the cluster: its global writes before it (ordinary stores) are
+// visible after it to the cluster's reads, the tensor-memory copies (async proxy) included.
 __device__ __forceinline__ void cluster_barrier() {
-  __threadfence();
+  asm volatile("fence.proxy.async.global;\n" ::: "memory");
   asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
   asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
 }

@@ -186,6 +186,10 @@ def allocate(var: torch.Tensor, S: int, H: int, W: int, bits: int, *, heads: int
     return payload[HEADER_BYTES:HEADER_BYTES + N]
 
 
+def tactkv_attention_workspace_bytes(k_units, n_units: int, q_heads: int) -> int:
+    return int(_lib.tactkv_attention_workspace_bytes(_as_array(k_units), n_units, q_heads))
+
+
 def tactkv_device_status(workspace_ptr: int, workspace_bytes: int, stream_ptr: int) -> int:
     return int(_lib.tactkv_device_status(ctypes.c_void_p(workspace_ptr), workspace_bytes, ctypes.c_void_p(stream_ptr)))
 
@@ -359,7 +363,7 @@ def attention_decode(q: torch.Tensor, k_payload: torch.Tensor, v_payload: torch.
     m = torch.empty((U, q_heads), dtype=torch.float32, device=q.device)
     l = torch.empty((U, q_heads), dtype=torch.float32, device=q.device)
     if workspace is None:
-        nbytes = int(_lib.tactkv_attention_workspace_bytes(ku, U, q_heads))
+        nbytes = tactkv_attention_workspace_bytes(ku, U, q_heads)
         ws = torch.zeros(nbytes + 256, dtype=torch.uint8, device=q.device)
         off = (-ws.data_ptr()) % 256
         workspace = ws[off:off + nbytes]

@@ -203,7 +203,8 @@ tactkv_status tactkv_allocate(const tactkv_unit* unit, const double* var, void* 
    TACTKV_UNSUPPORTED_SHAPE (every benchmark grid fits).  workspace: at least
    tactkv_attention_workspace_bytes(k_units, n_units, q_heads) bytes, 256-byte aligned.  A corrupt
    payload is recorded as TACTKV_CORRUPT_PAYLOAD (tactkv_device_status) and contributes no
-   tokens of its unit.  Asynchronous on `stream`; 5 kernels. */
+   tokens of its unit: out = 0, m = -inf and l = 0 for that unit's query heads.  Asynchronous on
+   `stream`; 5 kernels. */
 size_t tactkv_attention_workspace_bytes(const tactkv_unit* k_units, int n_units, int q_heads);
 tactkv_status tactkv_attention_decode(const tactkv_unit* k_units, const tactkv_unit* v_units, int n_units,
                                       int q_heads, const float* q, float* out, float* m, float* l,

@@ -67,3 +67,32 @@ def test_attention_with_variant_flags(flags):
 def test_attention_sharp_scores():
     """Large query norms make the softmax nearly one-hot: the max-subtraction must hold up."""
     _run(8, 8, 8, 1, 64, 2, 4, qscale=8.0, seed=11)
+
+
+def test_attention_corrupt_unit_contributes_no_tokens():
+    """A unit whose K (or V) payload is corrupt is reported as TACTKV_CORRUPT_PAYLOAD and contributes
+    no tokens (out = 0, m = -inf, l = 0); the other units of the call are unaffected."""
+    S, H, W, heads, D, G, bits, units = 8, 8, 8, 1, 64, 2, 2, 3
+    k = torch.stack([make_unit(S, H, W, heads, D, rho=(0.9, 0.85, 0.85), nu=4.0, seed=40 + i, device=DEV)
+                     for i in range(units)])
+    v = torch.stack([make_unit(S, H, W, heads, D, rho=(0.9, 0.85, 0.85), nu=4.0, seed=50 + i, device=DEV)
+                     for i in range(units)])
+    layers = list(range(units))
+    pk = T.compress(k, S, H, W, bits, layers=layers, kvs=[0] * units)
+    pv = T.compress(v, S, H, W, bits, layers=layers, kvs=[1] * units)
+    pk[1, 0] ^= 1                                   # unit 1: K magic broken
+    pv[2, 64] = 9                                   # unit 2: a V bit width above 8
+    q = torch.randn((units, heads * G, D), generator=torch.Generator(DEV).manual_seed(7), device=DEV)
+    ku = T.make_units(None, S, H, W, bits, heads=heads, head_dim=D, payload=pk, layers=layers, kvs=[0] * units,
+                      n_units=units)
+    nbytes = T.tactkv_attention_workspace_bytes(ku, units, heads * G)
+    ws = torch.zeros(nbytes + 256, dtype=torch.uint8, device=DEV)
+    off = (-ws.data_ptr()) % 256
+    ws = ws[off:off + nbytes]
+    out, m, l = T.attention_decode(q, pk, pv, S, H, W, bits, heads=heads, head_dim=D, layers=layers, workspace=ws)
+    assert T.tactkv_device_status(ws.data_ptr(), ws.numel(), 0) == T.TACTKV_CORRUPT_PAYLOAD
+    for i in (1, 2):
+        assert not out[i].any() and not l[i].any() and torch.all(torch.isneginf(m[i]))
+    o_ref, m_ref, l_ref = O.attention_decode(q[0].double().cpu().numpy(), pk[0].cpu().numpy().tobytes(),
+                                             pv[0].cpu().numpy().tobytes())
+    assert np.max(np.abs(out[0].double().cpu().numpy() - o_ref)) <= TOL * np.max(np.abs(o_ref))
