@@ -29,6 +29,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "KV compress+decompress GB/s (bf16 input) and % of B200 HBM roofline"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0     # B200 HBM3e nominal, reported beside the measured copy peak
 
 
 def parse_args():
@@ -426,11 +427,15 @@ def stage_roofline(prof, in_bytes, pay_bytes, bins_x_units, ms_step, peak, peak_
     dom = max(stages, key=stages.get)
     achieved = alg[dom] / (stages[dom] * 1e-3) / 1e9
     step_achieved = 2 * (in_bytes + pay_bytes) / (ms_step * 1e-3) / 1e9
+    traffic = dram_traffic(name, dom)
     return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-            "frac": round(achieved / peak, 4), "traffic": dram_traffic(name, dom),
+            "frac": round(achieved / peak, 4), "traffic": traffic,
+            "traffic_gbs": round(traffic / (stages[dom] * 1e-3) / 1e9, 1) if traffic else None,
+            "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
             "kernel": dom, "kernel_ms": round(stages[dom], 4), "algorithmic_bytes": alg[dom],
             "peak_kind": peak_kind,
             "step_achieved": round(step_achieved, 1), "step_frac": round(step_achieved / peak, 4),
+            "step_frac_of_nominal_8tbs": round(step_achieved / NOMINAL_HBM_GBS, 4),
             "compress_frac": round((in_bytes + pay_bytes) / (prof["compress_ms"] * 1e-3) / 1e9 / peak, 4),
             "decompress_frac": round((in_bytes + pay_bytes) / (prof["decompress_ms"] * 1e-3) / 1e9 / peak, 4)}
 

@@ -106,6 +106,8 @@ __global__ void __launch_bounds__(kFusedThreads, 3) fdct3_kernel(const __grid_co
 // Thread (warp w, lane l) then reads row 32 (w % 4) + l (cell w % 4, channel l) of the tile, half
 // (w / 4) of its S columns, and stores them to Y[k][cell][c]: 128 contiguous bytes per warp store.
 constexpr int kTcCells = 4;               // grid cells per tile (M = 128)
+constexpr int kTcEpilogueWarps = 8;       // warps 0..7 drain the accumulators; warp 8 produces
+constexpr int kTcThreads = 32 * (kTcEpilogueWarps + 1);
 
 template <int L>
 struct TcS {
@@ -125,14 +127,14 @@ __device__ __forceinline__ const uint16_t* dct_limb_fwd() {
 }
 
 // S pass of one (unit u, chunk) on this CTA's tiles t = r, r + kCluster, ... into Y, pipelined:
-//   warp 0 (one lane)  TMA producer and MMA issuer: the input tiles go through two shared-memory
+//   warp 8 (one lane)  TMA producer and MMA issuer: the input tiles go through two shared-memory
 //                      stages, the products into two TMEM accumulators (64 columns each), so the
 //                      MMAs of a tile run while the epilogue drains the previous one;
-//   warps 4..7         epilogue: warp 4 + q reads lanes 32q.. (cell q of the tile) of a finished
-//                      accumulator, frees it, and stores the S values to Y;
-//   warps 1..3         idle until the H/W pass.
+//   warps 0..7         epilogue: warp w reads lanes 32 (w % 4).. (cell w % 4 of the tile) and half
+//                      w / 4 of the S columns of a finished accumulator, frees it, and stores those
+//                      S values to Y.
 // mbarriers: full[s] (TMA -> MMA, transaction bytes), done[a] (MMA commit -> epilogue and producer),
-// freed[a] (4 epilogue warps -> MMA).  Every wait is bounded; on expiry the CTA records
+// freed[a] (8 epilogue warps -> MMA).  Every wait is bounded; on expiry the CTA records
 // TACTKV_TIMEOUT, waits (bounded) for what is in flight, releases TMEM and returns false.  The
 // caller still takes part in every barrier of the cluster.  Called by every thread of the CTA.
 template <int L, int HWX>
@@ -165,7 +167,7 @@ __device__ bool fdct_s_tc(const Geom& g, int u, int chunk, int r, const CUtensor
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&full[i], 1);
       tc::mbar_init(&done[i], 1);
-      tc::mbar_init(&freed[i], 4);
+      tc::mbar_init(&freed[i], kTcEpilogueWarps);
     }
     tc::fence_mbar_init();
     s_err = 0;
@@ -176,7 +178,7 @@ __device__ bool fdct_s_tc(const Geom& g, int u, int chunk, int r, const CUtensor
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0 && lane == 0 && mine > 0) {
+  if (warp == kTcEpilogueWarps && lane == 0 && mine > 0) {
     // ---- producer and MMA issuer
     const uint64_t pol = l2_evict_first();
     auto load = [&](int j) {
@@ -220,9 +222,10 @@ __device__ bool fdct_s_tc(const Geom& g, int u, int chunk, int r, const CUtensor
         tc::mbar_wait(&done[i], 0);
       }
     }
-  } else if (warp >= 4 && mine > 0) {
-    // ---- epilogue: warp 4 + q drains TMEM lanes 32q.. (cell q of each tile)
-    const int q = warp - 4;
+  } else if (warp < kTcEpilogueWarps && mine > 0) {
+    // ---- epilogue: warp w drains TMEM lanes 32 (w % 4).. (cell w % 4 of each tile), columns of
+    //      half w / 4
+    const int q = warp & 3, half = warp >> 2;
     for (int j = 0; j < mine; ++j) {
       const int st = j & 1;
       // (a warp vote keeps the warp converged for the .sync.aligned TMEM loads)
@@ -232,23 +235,17 @@ __device__ bool fdct_s_tc(const Geom& g, int u, int chunk, int r, const CUtensor
       }
       tc::fence_after_sync();
       const int cell = (r + kCluster * j) * kTcCells + q;
-      float* yo = Y + ((size_t)u * L * HWX + cell) * nx + c0 + lane;
-      const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + st * P::kCols;
+      float* yo = Y + ((size_t)u * L * HWX + cell) * nx + c0 + lane + (size_t)half * P::kHalf * HWX * nx;
+      const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + st * P::kCols + half * P::kHalf;
       float v[P::kHalf];
       tc::tmem_ld<P::kHalf>(taddr, v);
-      tc::tmem_ld_wait();
-      if (cell < HWX) {
-#pragma unroll
-        for (int k = 0; k < P::kHalf; ++k) yo[(size_t)k * HWX * nx] = v[k];
-      }
-      tc::tmem_ld<P::kHalf>(taddr + P::kHalf, v);
       tc::tmem_ld_wait();
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&freed[st]);   // the accumulator may take the next tile
       if (cell < HWX) {
 #pragma unroll
-        for (int k = 0; k < P::kHalf; ++k) yo[(size_t)(P::kHalf + k) * HWX * nx] = v[k];
+        for (int k = 0; k < P::kHalf; ++k) yo[(size_t)k * HWX * nx] = v[k];
       }
     }
   }
@@ -266,7 +263,7 @@ __device__ bool fdct_s_tc(const Geom& g, int u, int chunk, int r, const CUtensor
 
 // The fused forward kernel with the S pass on the tensor cores (bf16 input described by tmap).
 template <int L, int HX, int WX, int NX>
-__global__ void __launch_bounds__(kFusedThreads, 3) fdct3_tc_kernel(const __grid_constant__ Geom g,
+__global__ void __launch_bounds__(kTcThreads, 3) fdct3_tc_kernel(const __grid_constant__ Geom g,
                                                                     const __grid_constant__ UnitList ul,
                                                                     float* __restrict__ Y, float* __restrict__ partial,
                                                                     const __grid_constant__ CUtensorMap tmap,
@@ -286,12 +283,12 @@ __global__ void __launch_bounds__(kFusedThreads, 3) fdct3_tc_kernel(const __grid
 }
 
 template <class K, class... Args>
-cudaError_t launch_cluster(K kernel, const Geom& g, int nu, size_t smem, cudaStream_t st, Args... args) {
+cudaError_t launch_cluster(K kernel, int threads, const Geom& g, int nu, size_t smem, cudaStream_t st, Args... args) {
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(kCluster, g.nch, nu);
-  cfg.blockDim = dim3(kFusedThreads, 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute at[1];
@@ -358,10 +355,10 @@ cudaError_t launch_grid(const Geom& g, const UnitList& ul, int nu, float* buf, f
     const size_t smem = std::max<size_t>(TcS<L>::kSmem, Ls.total + 1024);
     if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
     if (g.n == 1024)
-      return launch_cluster(fdct3_tc_kernel<L, HX, WX, 1024>, g, nu, smem, st, g, ul, buf, partial, map, status);
+      return launch_cluster(fdct3_tc_kernel<L, HX, WX, 1024>, kTcThreads, g, nu, smem, st, g, ul, buf, partial, map, status);
     if (g.n == 512)
-      return launch_cluster(fdct3_tc_kernel<L, HX, WX, 512>, g, nu, smem, st, g, ul, buf, partial, map, status);
-    return launch_cluster(fdct3_tc_kernel<L, HX, WX, 0>, g, nu, smem, st, g, ul, buf, partial, map, status);
+      return launch_cluster(fdct3_tc_kernel<L, HX, WX, 512>, kTcThreads, g, nu, smem, st, g, ul, buf, partial, map, status);
+    return launch_cluster(fdct3_tc_kernel<L, HX, WX, 0>, kTcThreads, g, nu, smem, st, g, ul, buf, partial, map, status);
   }
 #endif
   int nbuf = 1;
@@ -369,12 +366,12 @@ cudaError_t launch_grid(const Geom& g, const UnitList& ul, int nu, float* buf, f
   if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
   const int lg_cpr = input_pieces_lg(g, ul, g.unit0, nu);
   if (has_variant(g.flags))
-    return launch_cluster(fdct3_kernel<L, HX, WX, 0, true>, g, nu, smem, st, g, ul, buf, partial, lg_cpr);
+    return launch_cluster(fdct3_kernel<L, HX, WX, 0, true>, kFusedThreads, g, nu, smem, st, g, ul, buf, partial, lg_cpr);
   if (g.n == 1024)
-    return launch_cluster(fdct3_kernel<L, HX, WX, 1024, false>, g, nu, smem, st, g, ul, buf, partial, lg_cpr);
+    return launch_cluster(fdct3_kernel<L, HX, WX, 1024, false>, kFusedThreads, g, nu, smem, st, g, ul, buf, partial, lg_cpr);
   if (g.n == 512)
-    return launch_cluster(fdct3_kernel<L, HX, WX, 512, false>, g, nu, smem, st, g, ul, buf, partial, lg_cpr);
-  return launch_cluster(fdct3_kernel<L, HX, WX, 0, false>, g, nu, smem, st, g, ul, buf, partial, lg_cpr);
+    return launch_cluster(fdct3_kernel<L, HX, WX, 512, false>, kFusedThreads, g, nu, smem, st, g, ul, buf, partial, lg_cpr);
+  return launch_cluster(fdct3_kernel<L, HX, WX, 0, false>, kFusedThreads, g, nu, smem, st, g, ul, buf, partial, lg_cpr);
 }
 
 }  // namespace
