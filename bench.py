@@ -543,10 +543,12 @@ def e2e_run(args, T, x, payload, out, cu, du, ws, stream, world):
             sp = int(s.cuda_stream)
             with torch.cuda.stream(s):
                 x[a:b].copy_(xh[a:b], non_blocking=True)
-                T.tactkv_compress(cu[a:b], wsg.data_ptr(), wsg.numel(), sp)
+                st = T.tactkv_compress(cu[a:b], wsg.data_ptr(), wsg.numel(), sp)
                 ph[a:b].copy_(payload[a:b], non_blocking=True)
-                T.tactkv_decompress(du[a:b], wsg.data_ptr(), wsg.numel(), sp)
+                st = st or T.tactkv_decompress(du[a:b], wsg.data_ptr(), wsg.numel(), sp)
                 oh[a:b].copy_(out[a:b], non_blocking=True)
+                if st != T.TACTKV_OK:
+                    raise T.TactkvError(st, "e2e step")
         for s in streams:
             done = torch.cuda.Event()
             done.record(s)
