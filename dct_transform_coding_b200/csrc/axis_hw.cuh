@@ -334,25 +334,53 @@ __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul,
         // lvs1[-1] is the zero in front of the levels: a bin without bits (mask 0) reads it, so
         // every code is read the same way, without a branch
         const float* lvs1 = lvs + 1;
+        const uint4* rr = rs + kp * D.W;   // record: sigma of each row, offset << 8 | code mask of each row
+        // The row pair's bins are consecutive in the stream: from the first bin's offset to the
+        // last bin's offset plus its bits.  When those bits lie in two stream words (most row
+        // pairs at low rates), both words are read once and every code is shifted out of them.
+        const uint32_t start = rr[0].z >> 8;
+        const uint32_t last = D.H > 2 * kp + 1 ? rr[D.W - 1].w : rr[D.W - 1].z;
+        const uint32_t end = (last >> 8) + (uint32_t)__popc(last & 0xffu);
+        const uint32_t base = start & ~31u;
+        if (end <= base + 64u) {
+          const unsigned long long win = ((unsigned long long)row[(base >> 5) + 1] << 32) | row[base >> 5];
 #pragma unroll
-        for (int t = 0; t < WC; ++t)
-          if (t < D.W) {
-            // record: sigma of each row, offset << 8 | code mask of each row (mask 0: no bits)
-            const uint4 m = rs[kp * D.W + t];
-            const uint32_t k0 = m.z & 0xffu, k1 = m.w & 0xffu;
-            const uint32_t off0 = m.z >> 8, off1 = m.w >> 8;   // from the slab's first word
-            const uint32_t* w0 = row + (off0 >> 5);
-            const uint32_t* w1 = row + (off1 >> 5);
-            const float l0 = lvs1[(int)(k0 + (__funnelshift_r(w0[0], w0[1], off0) & k0)) - 1];
-            const float l1 = lvs1[(int)(k1 + (__funnelshift_r(w1[0], w1[1], off1) & k1)) - 1];
-            float s0 = __uint_as_float(m.x), s1 = __uint_as_float(m.y);
-            if (VAR && hgain) {   // (a row without bits keeps its gain 0; the padding row reads nothing)
-              const size_t i0 = (size_t)ks * D.HW + (size_t)(2 * kp) * D.W + t;
-              s0 = k0 ? __ldg(hgain + i0) : 0.f;
-              s1 = k1 ? __ldg(hgain + i0 + D.W) : 0.f;
+          for (int t = 0; t < WC; ++t)
+            if (t < D.W) {
+              const uint4 m = rr[t];
+              const uint32_t k0 = m.z & 0xffu, k1 = m.w & 0xffu;
+              // (a code's shift is below 64; the padding row's record, mask 0, may point elsewhere)
+              const uint32_t c0 = (uint32_t)(win >> (((m.z >> 8) - base) & 63u)) & k0;
+              const uint32_t c1 = (uint32_t)(win >> (((m.w >> 8) - base) & 63u)) & k1;
+              const float l0 = lvs1[(int)(k0 + c0) - 1], l1 = lvs1[(int)(k1 + c1) - 1];
+              float s0 = __uint_as_float(m.x), s1 = __uint_as_float(m.y);
+              if (VAR && hgain) {   // (a row without bits keeps its gain 0; the padding row reads nothing)
+                const size_t i0 = (size_t)ks * D.HW + (size_t)(2 * kp) * D.W + t;
+                s0 = k0 ? __ldg(hgain + i0) : 0.f;
+                s1 = k1 ? __ldg(hgain + i0 + D.W) : 0.f;
+              }
+              x[t] = __fmul2_rn(make_float2(l0, l1), make_float2(s0, s1));
             }
-            x[t] = __fmul2_rn(make_float2(l0, l1), make_float2(s0, s1));
-          }
+        } else {
+#pragma unroll
+          for (int t = 0; t < WC; ++t)
+            if (t < D.W) {
+              const uint4 m = rr[t];
+              const uint32_t k0 = m.z & 0xffu, k1 = m.w & 0xffu;
+              const uint32_t off0 = m.z >> 8, off1 = m.w >> 8;   // from the slab's first word
+              const uint32_t* w0 = row + (off0 >> 5);
+              const uint32_t* w1 = row + (off1 >> 5);
+              const float l0 = lvs1[(int)(k0 + (__funnelshift_r(w0[0], w0[1], off0) & k0)) - 1];
+              const float l1 = lvs1[(int)(k1 + (__funnelshift_r(w1[0], w1[1], off1) & k1)) - 1];
+              float s0 = __uint_as_float(m.x), s1 = __uint_as_float(m.y);
+              if (VAR && hgain) {
+                const size_t i0 = (size_t)ks * D.HW + (size_t)(2 * kp) * D.W + t;
+                s0 = k0 ? __ldg(hgain + i0) : 0.f;
+                s1 = k1 ? __ldg(hgain + i0 + D.W) : 0.f;
+              }
+              x[t] = __fmul2_rn(make_float2(l0, l1), make_float2(s0, s1));
+            }
+        }
       }
       if (rotate) {   // R^T = diag(s) H_32 / sqrt(32) across the warp's 32 channels, both rows
 #pragma unroll
