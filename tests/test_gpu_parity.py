@@ -344,6 +344,31 @@ def test_head_gain_scaled_copy_of_a_head():
     assert np.array_equal(codes[act][:, D:], codes[act][:, :D])
 
 
+@pytest.mark.parametrize("shape,bits,flags", [((16, 16, 16, 2, 64), 2, 0), ((5, 7, 6, 3, 32), 8, 0),
+                                              ((16, 16, 16, 2, 64), 3, 64 | 128)],
+                         ids=["fused-grid-2b", "ragged-8b", "fused-grid-rotate-headgain"])
+def test_canaries_around_payloads_and_outputs(shape, bits, flags):
+    """Compress writes exactly the payload's total_bytes (the bytes after it in a larger buffer keep
+    their canary), and decompress into a strided view leaves the gaps between heads untouched."""
+    S, H, W, heads, D = shape
+    U = 2
+    x = torch.stack([make_unit(S, H, W, heads, D, rho=(0.9, 0.85, 0.8), nu=4.0, seed=500 + i, device=DEV)
+                     for i in range(U)])
+    cap = T.payload_capacity(S, H, W, heads, D, bits, flags)
+    pay = torch.full((U, cap + 272), 0xA5, dtype=torch.uint8, device=DEV)
+    T.compress(x, S, H, W, bits, layers=[0, 1], kvs=[0, 0], flags=flags, payload=pay)
+    big = torch.full((U, S * H * W, heads, D + 8), 7.0, dtype=torch.bfloat16, device=DEV)
+    T.decompress(pay, S, H, W, bits, heads=heads, head_dim=D, layers=[0, 1], kvs=[0, 0], flags=flags,
+                 out=big[..., :D], check=True)
+    torch.cuda.synchronize()
+    for i in range(U):
+        buf = pay[i].cpu().numpy()
+        total = int.from_bytes(buf[48:56].tobytes(), "little")
+        assert total <= cap and np.all(buf[total:] == 0xA5)
+        assert total == len(O.compress_unit(x[i].double().cpu().numpy(), S, H, W, heads, D, bits, flags=flags))
+    assert torch.all(big[..., D:] == 7.0)
+
+
 def test_opt_in_tensor_core_kernels():
     """The opt-in tensor-core forms, read once per process: the forward kernel's DCT along S on
     tcgen05 (TACTKV_TC_S=1) and the single-kernel decode with the inverse S on tcgen05

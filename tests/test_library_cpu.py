@@ -192,6 +192,25 @@ def test_occupancy_with_per_head_gains(T):
     assert occ["formula_bits"] - O.occupancy_bits(info["b"], heads * D) == 32 * (heads - 1) * S * H * W
 
 
+@pytest.mark.parametrize("flags", [0, 128])
+def test_payload_size_is_the_occupancy_formula_plus_header_index_and_padding(T, flags):
+    """Stage 4's relation on real payloads: the payload's bytes are the formula's bits (codes and
+    32-bit gains), the 64-byte header, one byte of bit width per bin, and nothing but the padding
+    of each part to 16 bytes."""
+    def pad16(v):
+        return (v + 15) // 16 * 16
+    S, H, W, heads, D = 3, 5, 6, 2, 32
+    N, n = S * H * W, heads * D
+    for bits in (1, 3, 8):
+        x = np.random.default_rng(bits).standard_normal((N, heads, D))
+        p = O.compress_unit(x, S, H, W, heads, D, bits, flags=flags)
+        occ = T.tactkv_occupancy(p)
+        g = heads if flags & 128 else 1
+        stride = pad16((occ["code_bits"] + 7) // 8)
+        padding_bits = 8 * (pad16(N) - N) + 8 * (pad16(4 * N * g) - 4 * N * g) + n * (8 * stride - occ["code_bits"])
+        assert 8 * occ["payload_bytes"] == 8 * 64 + occ["index_bits"] + occ["formula_bits"] + padding_bits
+
+
 def test_occupancy_rejects_corrupt_payloads(T):
     S, H, W, heads, D = 4, 6, 5, 1, 32
     p = bytearray(O.compress_unit(np.ones((S * H * W, heads, D)), S, H, W, heads, D, 2))
