@@ -269,10 +269,10 @@ __device__ float block_reduce(float v, float* red, bool is_max) {
 
 // Per query head: scores = idct3(z), p = exp(scores - max), l = sum p, then dct3(p) over z's place.
 // SX, HX, WX > 0: the grid's lengths fixed at compile time (the benchmark grids), 0: any grid.
-constexpr int kSoftmaxThreads = 512;
+constexpr int kSoftmaxThreads = 256;
 // A unit whose K or V payload failed the index checks contributes no tokens: p = 0, m = -inf, l = 0.
 template <int SX, int HX, int WX>
-__global__ void __launch_bounds__(kSoftmaxThreads) attn_softmax_kernel(const __grid_constant__ Geom g,
+__global__ void __launch_bounds__(kSoftmaxThreads, 2) attn_softmax_kernel(const __grid_constant__ Geom g,
                                                                     const uint32_t* __restrict__ kidx,
                                                                     const uint32_t* __restrict__ vidx,
                                                                     float* __restrict__ zp, float* __restrict__ m_out,
