@@ -14,8 +14,8 @@
 // by code specialised for 1 bit, 2 bits, or 3 and more bits by table); while it quantizes one
 // block, the 16 coefficient rows (128 bytes each) of its next block are in flight.  For a record
 // it computes u = X * (1/sigma) and the code, and ORs the code into the channel's word row at its
-// stream position.  The span's words are then stored once; its first and last words may hold bits
-// of the neighbouring ranges and are ORed into the payload atomically (the allocation zeroes those
+// stream position (a shared-memory reduction).  The span's words are then stored once; its first and
+// last words may hold bits of the neighbouring ranges and are ORed into the payload atomically (the allocation zeroes those
 // words first).  The CTA with the last record also writes the zero padding of the channel streams.
 //
 // With TACTKV_ROTATE every record's 32 coefficients (one bin, the CTA's 32 channels) are first
@@ -87,10 +87,9 @@ __device__ __forceinline__ void red_or_shared(uint32_t* p, uint32_t v) {
 }
 
 // One block of kPackBlock records, all of width b (= B when B > 0): quantize x[] and OR the codes
-// into the row (a code of more than one bit may straddle into the next word).  The records, the
-// word row and the tables do not overlap, so the record loads need not wait for the atomics.
-// In three phases -- the block's records, then its codes, then the ORs -- so that the loads of one
-// phase are all in flight together instead of each waiting behind the previous record's OR.
+// into the row (a code of more than one bit may straddle into the next word).  In three phases --
+// the block's records, then its codes, then the ORs -- so that the loads of one phase are all in
+// flight together instead of each waiting behind the previous record's OR.
 template <int B>
 __device__ __forceinline__ void pack_block(const uint4* __restrict__ rs, const float (&x)[kPackBlock],
                                            uint32_t* __restrict__ row, uint32_t base, int b,
