@@ -371,6 +371,8 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
 }
 
 // ----------------------------------------------------------------------------- decode index ---
+constexpr int kDecodeIndexThreads = 1024;   // a warp per slab (S <= 64): two slabs per warp at most
+
 // One CTA per unit: the header must describe exactly the unit the caller asked for, every bit
 // width must be <= 8 and their sum must equal the header's code_bits; then P(k_s), NZ(k_s) and the
 // decoding records are rebuilt from the payload (one warp per slab, a scan gives every bin's stream
@@ -378,7 +380,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
 // kernel's warp for a row pair reads its two rows' bins in order: sigma and position << 8 | code
 // mask for each of the two rows.  The 32 chunk CTAs that decode a bin do no index arithmetic of
 // their own.
-__global__ void __launch_bounds__(256) decode_index_kernel(const __grid_constant__ Geom g,
+__global__ void __launch_bounds__(kDecodeIndexThreads) decode_index_kernel(const __grid_constant__ Geom g,
                                                            const __grid_constant__ UnitList ul,
                                                            uint32_t* __restrict__ index, uint4* __restrict__ recs,
                                                            unsigned int* status) {
@@ -494,7 +496,7 @@ __global__ void __launch_bounds__(256) decode_index_kernel(const __grid_constant
 
 cudaError_t launch_decode_index(const Geom& g, const UnitList& ul, int nu, uint32_t* index, uint4* recs,
                                 unsigned int* status, cudaStream_t st) {
-  decode_index_kernel<<<nu, 256, 0, st>>>(g, ul, index, recs, status);
+  decode_index_kernel<<<nu, kDecodeIndexThreads, 0, st>>>(g, ul, index, recs, status);
   return cudaGetLastError();
 }
 
