@@ -15,9 +15,9 @@ namespace {
 // Register budget: class-16 pencils fit two CTAs of 256 threads per SM; class-32 float2 pencils
 // need more than 128 registers.
 constexpr int kHwMinBlocks = (TACTKV_HCLASS == 16 && TACTKV_WCLASS == 16) ? 2 : 1;
-// The exact-size class-16 inverse kernels fit 80 registers without spilling: three CTAs per SM.
+// The exact-size class-16 inverse kernels fit 64 registers without spilling: four CTAs per SM.
 template <int HX>
-constexpr int hw_min_blocks_inv() { return (TACTKV_HCLASS == 16 && TACTKV_WCLASS == 16) ? (HX > 0 ? 3 : 2) : 1; }
+constexpr int hw_min_blocks_inv() { return (TACTKV_HCLASS == 16 && TACTKV_WCLASS == 16) ? (HX > 0 ? 4 : 2) : 1; }
 
 template <int HC, int WC, int HX, int WX, bool VAR>
 __global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) fdct_hw_kernel(const __grid_constant__ Geom g,
