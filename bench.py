@@ -45,6 +45,9 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--e2e-groups", type=int, default=32, help="unit groups pipelined over streams in the e2e run")
     ap.add_argument("--e2e-streams", type=int, default=4, help="streams (each with a workspace) in the e2e run")
+    ap.add_argument("--streams", type=int, default=1,
+                    help="streams of the timed step: the batch goes in that many unit groups, one per stream "
+                         "(each with its own workspace), joined at the end of every step")
     ap.add_argument("--units", type=int, default=None, help="use only the first U units of the batch (profiling)")
     ap.add_argument("--no-others", action="store_true", help="skip the other workloads' lines")
     ap.add_argument("--no-attention", action="store_true", help="skip the decode-time attention measurement")
@@ -248,11 +251,34 @@ def main():
         if st != T.TACTKV_OK:
             raise T.TactkvError(st, what)
 
+    n_str = max(1, min(args.streams, U))
+    groups = [(U * k // n_str, U * (k + 1) // n_str) for k in range(n_str)]
+    side = [torch.cuda.Stream(dev) for _ in range(n_str)] if n_str > 1 else []
+    side_ws = [T.alloc_workspace(cu[a:b], dev) for a, b in groups] if n_str > 1 else []
+
     def step():
-        check(T.tactkv_compress(cu, ws.data_ptr(), ws.numel(), sp), "compress")
-        n = T.tactkv_last_launches()
-        check(T.tactkv_decompress(du, ws.data_ptr(), ws.numel(), sp), "decompress")
-        return n + T.tactkv_last_launches()
+        if n_str == 1:
+            check(T.tactkv_compress(cu, ws.data_ptr(), ws.numel(), sp), "compress")
+            n = T.tactkv_last_launches()
+            check(T.tactkv_decompress(du, ws.data_ptr(), ws.numel(), sp), "decompress")
+            return n + T.tactkv_last_launches()
+        # groups of units on their own streams: one group's forward transforms (bound by data
+        # movement) can overlap another's decoding (bound by instructions)
+        start = torch.cuda.Event()
+        start.record(stream)
+        n = 0
+        for (a, b), s_, w_ in zip(groups, side, side_ws):
+            s_.wait_event(start)
+            spg = int(s_.cuda_stream)
+            check(T.tactkv_compress(cu[a:b], w_.data_ptr(), w_.numel(), spg), "compress")
+            n += T.tactkv_last_launches()
+            check(T.tactkv_decompress(du[a:b], w_.data_ptr(), w_.numel(), spg), "decompress")
+            n += T.tactkv_last_launches()
+        for s_ in side:
+            done = torch.cuda.Event()
+            done.record(s_)
+            stream.wait_event(done)
+        return n
 
     for _ in range(args.warmup):
         step()
