@@ -12,15 +12,15 @@
 namespace tactkv {
 namespace {
 
-// Register budget: class-16 pencils fit two CTAs of 256 threads per SM; class-32 float2 pencils
-// need more than 128 registers.
+// Register budget: class-16 pencils fit two CTAs of 256 threads per SM; the generic class-32
+// float2 pencils need more than 128 registers, the exact 24 x 24 ones fit two CTAs per SM.
 constexpr int kHwMinBlocks = (TACTKV_HCLASS == 16 && TACTKV_WCLASS == 16) ? 2 : 1;
 // The exact-size class-16 inverse kernels fit 64 registers without spilling: four CTAs per SM.
 template <int HX>
-constexpr int hw_min_blocks_inv() { return (TACTKV_HCLASS == 16 && TACTKV_WCLASS == 16) ? (HX > 0 ? 4 : 2) : 1; }
+constexpr int hw_min_blocks_inv() { return (TACTKV_HCLASS == 16 && TACTKV_WCLASS == 16) ? (HX > 0 ? 4 : 2) : (HX > 0 ? 2 : 1); }
 
 template <int HC, int WC, int HX, int WX, bool VAR>
-__global__ void __launch_bounds__(kMaxHwThreads, kHwMinBlocks) fdct_hw_kernel(const __grid_constant__ Geom g,
+__global__ void __launch_bounds__(kMaxHwThreads, (HX > 0 ? 2 : kHwMinBlocks)) fdct_hw_kernel(const __grid_constant__ Geom g,
                                                                               const __grid_constant__ UnitList ul,
                                                                               float* __restrict__ Y,
                                                                               float* __restrict__ partial, int spc) {

@@ -61,7 +61,8 @@ __host__ __device__ inline HwLayout hw_layout(int H, int W, int kind) {
   const size_t words1 = (size_t)32 * L.words * 4, meta1 = (size_t)HW * 16;
   // the exact-size decode kernels of the common grids run four CTAs per SM: one slot then leaves
   // room for the fourth, which hides more latency than the prefetched slot did (measured on B200)
-  const bool four_per_sm = (H == 16 && W == 16) || (H == 14 && W == 14) || (H == 8 && W == 8);
+  // likewise two CTAs per SM for the exact 24 x 24 kernels (one slot or tile buffer each)
+  const bool four_per_sm = (H == 16 && W == 16) || (H == 14 && W == 14) || (H == 8 && W == 8) || (H == 24 && W == 24);
   L.nslot = (de && (four_per_sm || (size_t)(2 * HP) * (2 * WP) * 128 + 2 * (words1 + meta1) + kLmLvTotal * 4 + 256 >
                                        kSmemBudget))
                 ? 1
@@ -73,7 +74,7 @@ __host__ __device__ inline HwLayout hw_layout(int H, int W, int kind) {
   const size_t sig = 0;
   const size_t lv = de ? (kLmLvTotal + 1) * 4 : 0;   // a zero in front of the levels
   const size_t rest = words + meta + bsl + sig + lv + 256;
-  L.nbuf = (de || 2 * L.tile_bytes + rest > kSmemBudget) ? 1 : 2;
+  L.nbuf = (de || (H == 24 && W == 24) || 2 * L.tile_bytes + rest > kSmemBudget) ? 1 : 2;
   // every region starts on a 16-byte boundary (cp.async of 16 bytes, 16-byte record loads)
   auto p16 = [](size_t x) { return (x + 15) / 16 * 16; };
   size_t o = 0;
