@@ -10,8 +10,8 @@
 // only the clusters in flight hold Y lines, and the streams that pass through once (the input and
 // the finished coefficients X) are marked evict-first so that they give way to it.
 //
-// The common grids (16x16, 14x14, 8x8) with S = 8, 16, 32 or 64 have a fused kernel; this file is
-// compiled once per S (TACTKV_FUSED_S).  Other shapes use the separate S-axis and H/W-axis
+// The common grids (16x16, 14x14, 8x8 with S = 8, 16, 32 or 64, and 24x24 with S up to 32) have a
+// fused kernel; this file is compiled once per S (TACTKV_FUSED_S).  Other shapes use the separate S-axis and H/W-axis
 // kernels.
 #include "axis_s.cuh"
 #include "axis_hw.cuh"
@@ -56,9 +56,14 @@ __host__ __device__ inline size_t fused_fwd_smem(int H, int W, bool fp32_in, int
   return hw > st ? hw : st;
 }
 
+// Pencil length class of an H or W length, and CTAs per SM: the 16-class grids fit 80 registers
+// (three CTAs), the 24 x 24 grid's 32-class float2 pencils 128 (two CTAs).
+__host__ __device__ constexpr int hw_class(int x) { return x > 16 ? 32 : 16; }
+__host__ __device__ constexpr int fused_min_blocks(int hx) { return hx > 16 ? 2 : 3; }
+
 // NX: the channel count when fixed at compile time (the common 512 and 1024), else 0.
 template <int L, int HX, int WX, int NX, bool VAR>
-__global__ void __launch_bounds__(kFusedThreads, 3) fdct3_kernel(const __grid_constant__ Geom g,
+__global__ void __launch_bounds__(kFusedThreads, fused_min_blocks(HX)) fdct3_kernel(const __grid_constant__ Geom g,
                                                                  const __grid_constant__ UnitList ul,
                                                                  float* __restrict__ Y, float* __restrict__ partial,
                                                                  int lg_cpr) {
@@ -92,7 +97,8 @@ __global__ void __launch_bounds__(kFusedThreads, 3) fdct3_kernel(const __grid_co
   // DCT along H and W on this CTA's range of slabs
   constexpr int spc = (L + kCluster - 1) / kCluster;
   const int ks0 = r * spc, ks1 = min(L, ks0 + spc);
-  if (ks0 < ks1) fdct_hw_slabs<16, 16, HX, WX, true, NX, VAR>(g, Y, partial, u, chunk, ks0, ks1, smem);
+  if (ks0 < ks1)
+    fdct_hw_slabs<hw_class(HX), hw_class(WX), HX, WX, true, NX, VAR>(g, Y, partial, u, chunk, ks0, ks1, smem);
 }
 
 // ------------------------------------------------------------- S pass on the tensor cores ---
@@ -350,6 +356,7 @@ cudaError_t launch_grid(const Geom& g, const UnitList& ul, int nu, float* buf, f
   for (size_t x : regions)
     if (x % 16) return cudaErrorMisalignedAddress;   // never launch a misaligned layout
 #if TACTKV_FUSED_S >= 16
+  if constexpr (HX <= 16) {   // (the tensor-core form covers the 16-class grids)
   CUtensorMap map;
   if (tc_s_pass_enabled() && make_input_map(g, ul, nu, &map)) {
     const size_t smem = std::max<size_t>(TcS<L>::kSmem, Ls.total + 1024);
@@ -359,6 +366,7 @@ cudaError_t launch_grid(const Geom& g, const UnitList& ul, int nu, float* buf, f
     if (g.n == 512)
       return launch_cluster(fdct3_tc_kernel<L, HX, WX, 512>, kTcThreads, g, nu, smem, st, g, ul, buf, partial, map, status);
     return launch_cluster(fdct3_tc_kernel<L, HX, WX, 0>, kTcThreads, g, nu, smem, st, g, ul, buf, partial, map, status);
+  }
   }
 #endif
   int nbuf = 1;
@@ -386,6 +394,9 @@ cudaError_t TACTKV_CAT(launch_fused_, TACTKV_FUSED_S)(const Geom& g, const UnitL
   if (g.H == 16 && g.W == 16) return launch_grid<16, 16>(g, ul, nu, buf, partial, status, st);
   if (g.H == 14 && g.W == 14) return launch_grid<14, 14>(g, ul, nu, buf, partial, status, st);
   if (g.H == 8 && g.W == 8) return launch_grid<8, 8>(g, ul, nu, buf, partial, status, st);
+#if TACTKV_FUSED_S <= 32
+  if (g.H == 24 && g.W == 24) return launch_grid<24, 24>(g, ul, nu, buf, partial, status, st);
+#endif
   return cudaErrorNotSupported;
 }
 

@@ -69,7 +69,8 @@ cudaError_t launch_fused_inv(const Geom& g, const UnitList& ul, int nu, float* b
 // kept in L2 between them).
 bool fused_grid(const Geom& g) {
   const bool s = g.S == 8 || g.S == 16 || g.S == 32 || g.S == 64;
-  return s && ((g.H == 16 && g.W == 16) || (g.H == 14 && g.W == 14) || (g.H == 8 && g.W == 8));
+  return s && ((g.H == 16 && g.W == 16) || (g.H == 14 && g.W == 14) || (g.H == 8 && g.W == 8) ||
+               (g.H == 24 && g.W == 24 && g.S <= 32));
 }
 cudaError_t launch_fused(const Geom& g, const UnitList& ul, int nu, float* buf, float* partial, unsigned int* status,
                          cudaStream_t st) {

@@ -257,7 +257,8 @@ int tactkv_format_version(void);
 /* Number of kernels that the calling host thread's most recent tactkv_compress*,
    tactkv_decompress* call launched, over all its waves (0 after a call that failed before
    launching).  A compress wave launches 4 kernels when its grid has a fused three-axis forward
-   transform kernel (H x W = 16 x 16, 14 x 14 or 8 x 8 with S = 8, 16, 32 or 64) and 5 otherwise;
+   transform kernel (H x W = 16 x 16, 14 x 14 or 8 x 8 with S = 8, 16, 32 or 64, 24 x 24 with S = 8, 16
+   or 32) and 5 otherwise;
    a decompress wave launches 3. */
 int tactkv_last_launches(void);
 

@@ -68,6 +68,8 @@ def test_tiny_config_fp32_io():
     ((8, 14, 14, 1, 64), 3),    # fused three-axis kernels: S = 8 on the 14 x 14 grid
     ((32, 8, 8, 2, 32), 2),     # fused, S = 32 on the 8 x 8 grid
     ((64, 8, 8, 1, 32), 1),     # fused, S = 64 on the 8 x 8 grid
+    ((16, 24, 24, 2, 64), 2),   # fused, S = 16 on the 24 x 24 grid (32-class H/W pencils)
+    ((32, 24, 24, 1, 32), 1),   # fused, S = 32 on the 24 x 24 grid (the 32B-class medical layout)
 ])
 def test_small_shapes_bf16(shape, bits):
     S, H, W, heads, D = shape
@@ -293,6 +295,7 @@ def test_tensor_core_and_cuda_core_s_pass_both_match_the_oracle(S, H, W):
     (16, 8, 8, 0, torch.float32),     # fused decode on the tensor cores, float32 output
     (32, 16, 16, 1, torch.bfloat16),  # NO_QUANT on a fused grid: the separate (exact) inverse kernels
     (64, 14, 14, 1, torch.float32),
+    (32, 24, 24, 0, torch.float32),   # fused forward on the 24 x 24 grid, float32 output
 ])
 def test_fused_grid_output_variants(S, H, W, flags, dtype):
     """The fused decode kernel writes bf16 or float32; NO_QUANT payloads keep the separate inverse
