@@ -15,10 +15,13 @@
 // pairs, writes the finished coefficients X back over the slab in global memory and sums X^2 over
 // the 32 channels into partial[u][chunk][bin].
 //
-// Inverse (idct_hw), per slab: the slab's stream words arrive by cp.async (next slab prefetched);
-// per-bin records give each bin's bits, gain and stream position; warp j decodes rows 2j and 2j+1
-// (unpack + dequantize in registers), runs the inverse DCT along W and writes column pairs; then
-// runs the inverse DCT along H on column pair j and stores the result into the fp32 volume V.
+// Inverse (idct_hw), per slab: the slab's stream words arrive by cp.async (the next slab's
+// meanwhile where there is room for a second slot; the common grids keep one slot and run more CTAs
+// per SM instead); per-bin records give each bin's bits, gain and stream position; warp j decodes
+// rows 2j and 2j+1 (unpack + dequantize in registers: a row whose codes fit in two stream words is
+// read once and its codes shifted out of that 64-bit window), runs the inverse DCT along W and
+// writes column pairs; then runs the inverse DCT along H on column pair j and stores the result into
+// the fp32 volume V.
 #pragma once
 #include "common.cuh"
 #include "lloyd_max_tables.inc"
