@@ -70,6 +70,8 @@ def test_tiny_config_fp32_io():
     ((64, 8, 8, 1, 32), 1),     # fused, S = 64 on the 8 x 8 grid
     ((16, 24, 24, 2, 64), 2),   # fused, S = 16 on the 24 x 24 grid (32-class H/W pencils)
     ((32, 24, 24, 1, 32), 1),   # fused, S = 32 on the 24 x 24 grid (the 32B-class medical layout)
+    ((8, 24, 24, 1, 64), 4),    # fused, S = 8 on the 24 x 24 grid (one slab per CTA of the cluster)
+    ((64, 24, 24, 1, 32), 2),   # S = 64 on the 24 x 24 grid: the separate transform kernels
 ])
 def test_small_shapes_bf16(shape, bits):
     S, H, W, heads, D = shape
