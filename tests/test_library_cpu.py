@@ -134,6 +134,52 @@ def _gen_tables():
     return mod
 
 
+def _csrc_module(name):
+    import importlib.util
+    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                        "dct_transform_coding_b200", "csrc", name + ".py")
+    spec = importlib.util.spec_from_file_location(name, path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+@pytest.mark.parametrize("L", [1, 2, 3, 5, 7, 8, 14, 16, 20, 24, 28, 32, 40, 48, 56, 64])
+def test_generated_pencil_programs_match_scipy(L):
+    """The library's generated DCT programs (forward and its transpose), evaluated in float64 and in
+    float32, against scipy's orthonormal DCT-II / DCT-III: exact to rounding in float64, and within a
+    few float32 ulps of the largest coefficient in float32 (the accuracy the codes rely on)."""
+    import scipy.fft
+    G = _csrc_module("gen_dct")
+    g, outs = G.build_forward(L)
+    tg, touts = G.transpose_graph(g, outs)
+    x = np.random.default_rng(L).standard_normal((L, 64))
+    ref_f = scipy.fft.dct(x, type=2, norm="ortho", axis=0)
+    ref_i = scipy.fft.idct(x, type=2, norm="ortho", axis=0)
+    assert np.max(np.abs(G.evaluate(g, outs, x) - ref_f)) < 1e-12
+    assert np.max(np.abs(G.evaluate(tg, touts, x) - ref_i)) < 1e-12
+    f32 = G.evaluate(g, outs, x.astype(np.float32), dtype=np.float32).astype(np.float64)
+    assert np.max(np.abs(f32 - ref_f)) < 16 * np.finfo(np.float32).eps * np.max(np.abs(ref_f))
+
+
+@pytest.mark.parametrize("L", [16, 32, 64])
+def test_tensor_core_limbs_rebuild_the_dct_matrix(L):
+    """The three bf16 limbs of the DCT matrix used by the tensor-core S pass: each limb exactly a
+    bfloat16 value, their sum equal to scipy's orthonormal DCT-II matrix within 2^-24, and the
+    rounding to bfloat16 ties to even."""
+    import scipy.fft
+    G = _csrc_module("gen_mma_tables")
+    C = scipy.fft.dct(np.eye(L), type=2, norm="ortho", axis=0)
+    parts = G.limbs(G.dct_matrix(L))
+    for p in parts:
+        assert np.array_equal(p, p.astype(np.float32).astype(np.float64))
+        for v in p.ravel()[:64]:
+            G.bf16_bits(float(v))              # raises unless the low 16 bits of the float32 are 0
+    assert np.max(np.abs(parts[0] + parts[1] + parts[2] - C)) <= 2.0 ** -24
+    assert G.round_bf16(1.0 + 2.0 ** -8) == 1.0 and G.round_bf16(1.0 + 3 * 2.0 ** -8) == 1.0 + 2 ** -6
+    assert G.round_bf16(-(1.0 + 2.0 ** -8 + 2.0 ** -20)) == -(1.0 + 2.0 ** -7)
+
+
 @pytest.mark.parametrize("bits", range(3, 9))
 def test_cell_table_code_lookup_equals_threshold_count(bits):
     """The kernels' code lookup for b >= 3 (cell of u, table count, two compares), emulated in
