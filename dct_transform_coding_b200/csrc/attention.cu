@@ -28,6 +28,8 @@ namespace {
 constexpr int kAttnThreads = 256;
 constexpr int kMaxG = 16;                   // query heads per K/V head
 constexpr float kInvSqrt32 = 0.17677669529663687f;
+constexpr int kLv0Floats = TACTKV_LV0_VEC * 4;   // the levels behind a zero, in whole 16-byte vectors
+static_assert(kLv0Floats >= kLmLvTotal + 1, "level table");
 
 // Words of a channel stream held per slab in shared memory: the most a slab can span (8 bits per
 // bin, from any bit of its first word), two zero words for the look-ahead of the code reads, and
@@ -131,7 +133,7 @@ __global__ void __launch_bounds__(kScoreThreads) attn_scores_kernel(const __grid
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const int G = q_heads / g.heads, D = g.head_dim, HW = g.HW, stride = attn_word_stride(HW);
   float* lvs1 = sh + 1;                                        // a zero in front of the levels
-  float* qs = sh + (kLmLvTotal + 1 + 3) / 4 * 4;               // [G][D], rotated when the payload is
+  float* qs = sh + kLv0Floats;               // [G][D], rotated when the payload is
   float* zs = qs + G * D;                                      // [G][HW]
   uint2* actrec = reinterpret_cast<uint2*>(zs + (G * HW + 1) / 2 * 2);   // [pad32(HW)]
   int* act = reinterpret_cast<int*>(actrec + pad32(HW));                 // [HW]
@@ -145,7 +147,7 @@ __global__ void __launch_bounds__(kScoreThreads) attn_scores_kernel(const __grid
     stage_words(reinterpret_cast<const uint32_t*>(pay + g.off_codes) + (size_t)h * D * sw + (p0 >> 5), sw, D, nw,
                 stride, words);
   }
-  for (int i = threadIdx.x; i <= kLmLvTotal; i += blockDim.x) sh[i] = i ? c_lm_levels[i - 1] : 0.f;
+  copy_vec16(sh, g_lm_levels0, TACTKV_LV0_VEC);
   for (int i = threadIdx.x; i < G * HW; i += blockDim.x) zs[i] = 0.f;
   const float* qu = q + ((size_t)u * q_heads + (size_t)h * G) * D;
   const bool rotate = g.flags & TACTKV_ROTATE;
@@ -332,7 +334,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_values_kernel(const __grid_
   const int ks = blockIdx.x, h = blockIdx.y, u = blockIdx.z;
   const int G = q_heads / g.heads, D = g.head_dim, HW = g.HW, stride = attn_word_stride(HW);
   float* lvs1 = sh + 1;
-  float* wt = sh + (kLmLvTotal + 1 + 3) / 4 * 4;        // [HW][G]: weight of active bin a for head g
+  float* wt = sh + kLv0Floats;        // [HW][G]: weight of active bin a for head g
   uint2* actrec = reinterpret_cast<uint2*>(wt + ((size_t)G * HW + 1) / 2 * 2);   // [pad32(HW)], 8-byte aligned
   int* act = reinterpret_cast<int*>(actrec + pad32(HW));                         // [HW]
   uint32_t* words = reinterpret_cast<uint32_t*>(act + pad32(HW));                // [D][stride]
@@ -345,7 +347,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_values_kernel(const __grid_
     stage_words(reinterpret_cast<const uint32_t*>(pay + g.off_codes) + (size_t)h * D * sw + (p0 >> 5), sw, D, nw,
                 stride, words);
   }
-  for (int i = threadIdx.x; i <= kLmLvTotal; i += blockDim.x) sh[i] = i ? c_lm_levels[i - 1] : 0.f;
+  copy_vec16(sh, g_lm_levels0, TACTKV_LV0_VEC);
   const uint4* srec = recs + (size_t)u * g.N + (size_t)ks * ((g.H + 1) / 2) * g.W;
   const int na = ok ? stage_active(srec, HW, g.W, actrec, act, &s_count, s_warp) : 0;
   if (head_gains_on(g.flags)) {
@@ -405,13 +407,13 @@ __global__ void __launch_bounds__(kAttnThreads) attn_reduce_kernel(const __grid_
 
 size_t attention_scores_smem(const Geom& g, int q_heads) {
   const int G = q_heads / g.heads;
-  return (size_t)((kLmLvTotal + 1 + 3) / 4 * 4 + G * g.head_dim + (G * g.HW + 1) / 2 * 2) * 4 +
+  return (size_t)(kLv0Floats + G * g.head_dim + (G * g.HW + 1) / 2 * 2) * 4 +
          (size_t)pad32(g.HW) * 12 + (size_t)g.head_dim * attn_word_stride(g.HW) * 4;
 }
 size_t attention_softmax_smem(const Geom& g) { return softmax_smem(g); }
 size_t attention_values_smem(const Geom& g, int q_heads) {
   const int G = q_heads / g.heads;
-  return (size_t)((kLmLvTotal + 1 + 3) / 4 * 4 + (G * g.HW + 1) / 2 * 2) * 4 + (size_t)pad32(g.HW) * 12 +
+  return (size_t)(kLv0Floats + (G * g.HW + 1) / 2 * 2) * 4 + (size_t)pad32(g.HW) * 12 +
          (size_t)g.head_dim * attn_word_stride(g.HW) * 4;
 }
 

@@ -25,6 +25,7 @@
 #pragma once
 #include "common.cuh"
 #include "lloyd_max_tables.inc"
+static_assert(TACTKV_LV0_VEC * 4 >= tactkv::kLmLvTotal + 1, "level table");
 
 namespace tactkv {
 namespace {
@@ -75,7 +76,7 @@ __host__ __device__ inline HwLayout hw_layout(int H, int W, int kind) {
   L.bsl_stride = 0;
   const size_t bsl = 0;
   const size_t sig = 0;
-  const size_t lv = de ? (kLmLvTotal + 1) * 4 : 0;   // a zero in front of the levels
+  const size_t lv = de ? (size_t)TACTKV_LV0_VEC * 16 : 0;   // a zero in front of the levels
   const size_t rest = words + meta + bsl + sig + lv + 256;
   L.nbuf = (de || (H == 24 && W == 24) || 2 * L.tile_bytes + rest > kSmemBudget) ? 1 : 2;
   // every region starts on a 16-byte boundary (cp.async of 16 bytes, 16-byte record loads)
@@ -311,7 +312,7 @@ __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul,
     for (int e = threadIdx.x; e < RP; e += blockDim.x) cp_async16(rb + e, urecs + (size_t)ks * RP + e);
   };
   if (!raw) {
-    for (int i = threadIdx.x; i <= kLmLvTotal; i += blockDim.x) lvs[i] = i ? c_lm_levels[i - 1] : 0.f;
+    for (int i = threadIdx.x; i < TACTKV_LV0_VEC; i += blockDim.x) cp_async16(lvs + 4 * i, g_lm_levels0 + 4 * i);
     if (ok) issue_slab(ks0);
     cp_async_commit();
   }

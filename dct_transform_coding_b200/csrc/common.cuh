@@ -237,6 +237,14 @@ __device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+// A table of n 16-byte vectors from global memory into shared memory, vector i by thread i (mod the
+// block), one load each: copied out of constant memory instead, a warp's 32 different addresses
+// would be served one after another.
+__device__ __forceinline__ void copy_vec16(void* smem, const void* gmem, int n) {
+  uint4* d = reinterpret_cast<uint4*>(smem);
+  const uint4* s = reinterpret_cast<const uint4*>(gmem);
+  for (int i = threadIdx.x; i < n; i += blockDim.x) d[i] = __ldg(s + i);
+}
 // Streams that pass through L2 once (the input, the finished coefficients) are marked
 // evict-first in the fused forward kernel, so that they give way to the fp32 volume that is read
 // back soon after.

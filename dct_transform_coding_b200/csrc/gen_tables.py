@@ -187,6 +187,24 @@ def generate() -> str:
     lines += ["  " + ", ".join(lit(v) for v in pad_all[i:i + 4]) + "," for i in range(0, len(pad_all), 4)]
     lines += ["};", "static __constant__ unsigned char c_qcell[] = {"]
     lines += ["  " + ", ".join(str(v) for v in qtab[i:i + 32]) + "," for i in range(0, len(qtab), 32)]
+    lines += ["};"]
+    # The same tables in global memory, 16-byte aligned and padded to whole 16-byte vectors, for
+    # kernels that copy them to shared memory: thread i reads vector i, where a copy out of
+    # constant memory would serialise the warp's 32 different addresses.  The levels get a zero
+    # in front (index 0 stands for "no bits").
+    lv0 = [0.0] + [f32v(v) for v in lv_all]
+    lv0 += [0.0] * (-len(lv0) % 4)
+    thr16 = pad_all + [math.inf] * (-len(pad_all) % 4)
+    q16 = qtab + [0] * (-len(qtab) % 16)
+    lines += [f"#define TACTKV_LV0_VEC {len(lv0) // 4}",
+              f"#define TACTKV_THR_VEC {len(thr16) // 4}",
+              f"#define TACTKV_QCELL_VEC {len(q16) // 16}",
+              "static __device__ __align__(16) const float g_lm_levels0[] = {"]
+    lines += ["  " + ", ".join(lit(v) for v in lv0[i:i + 4]) + "," for i in range(0, len(lv0), 4)]
+    lines += ["};", "static __device__ __align__(16) const float g_thr_pad[] = {"]
+    lines += ["  " + ", ".join(lit(v) for v in thr16[i:i + 4]) + "," for i in range(0, len(thr16), 4)]
+    lines += ["};", "static __device__ __align__(16) const unsigned char g_qcell[] = {"]
+    lines += ["  " + ", ".join(str(v) for v in q16[i:i + 32]) + "," for i in range(0, len(q16), 32)]
     lines += ["};", "#endif", ""]
     return "\n".join(lines)
 

@@ -48,8 +48,8 @@ __host__ __device__ inline PackLayout pack_layout() {
   size_t o = 0;
   L.rec = o; o += p16((size_t)kPackRecSlots * 16);
   L.sbuf = o; o += p16((size_t)kChunk * L.words * 4);
-  L.thr = o; o += p16((size_t)TACTKV_THR_PAD_TOTAL * 4);
-  L.qcell = o; o += p16((size_t)6 * TACTKV_Q_CELLS);
+  L.thr = o; o += (size_t)TACTKV_THR_VEC * 16;
+  L.qcell = o; o += (size_t)TACTKV_QCELL_VEC * 16;
   L.total = o;
   return L;
 }
@@ -159,8 +159,8 @@ __global__ void __launch_bounds__(kPackThreads, 4) pack_kernel(const __grid_cons
       }
   }
   if (threadIdx.x < 9 * kWarps) (&s_cnt[0][0])[threadIdx.x] = 0u;
-  for (int i = threadIdx.x; i < TACTKV_THR_PAD_TOTAL; i += kPackThreads) thr[i] = c_thr_pad[i];
-  for (int i = threadIdx.x; i < 6 * TACTKV_Q_CELLS; i += kPackThreads) qcell[i] = c_qcell[i];
+  copy_vec16(thr, g_thr_pad, TACTKV_THR_VEC);
+  copy_vec16(qcell, g_qcell, TACTKV_QCELL_VEC);
   // bit span [A, B) of the range; its words from word A >> 5 on are assembled in shared memory
   const uint32_t A = m > 0 ? urecs[r0].z : code_bits;
   const uint32_t B = r1 < nrec ? urecs[r1].z : code_bits;

@@ -208,6 +208,35 @@ def test_cell_table_code_lookup_equals_threshold_count(bits):
     assert np.array_equal(code, want)
 
 
+def _c_array(text, name):
+    """The initialiser of the C array `name` in generated source, as a list of numbers."""
+    import re
+    body = re.search(r"\b" + name + r"\[\] = \{(.*?)\};", text, re.S).group(1)
+    vals = []
+    for tok in body.replace("\n", " ").split(","):
+        tok = tok.strip()
+        if tok:
+            vals.append(np.inf if tok == "INFINITY" else float(tok.rstrip("f")))
+    return vals
+
+
+def test_global_table_copies_match_the_constant_tables():
+    """The 16-byte-vector copies of the codebook tables that kernels stage into shared memory: the
+    levels behind a leading zero, the padded thresholds and the code cells, each equal to its
+    constant-memory table and padded to whole 16-byte vectors."""
+    G = _gen_tables()
+    text = G.generate()
+    lv, lv0 = _c_array(text, "c_lm_levels"), _c_array(text, "g_lm_levels0")
+    thr, thr16 = _c_array(text, "c_thr_pad"), _c_array(text, "g_thr_pad")
+    q, q16 = _c_array(text, "c_qcell"), _c_array(text, "g_qcell")
+    assert len(lv) == 510 and lv0[0] == 0.0 and lv0[1:len(lv) + 1] == lv and len(lv0) % 4 == 0
+    assert all(v == 0.0 for v in lv0[len(lv) + 1:])
+    assert thr16[:len(thr)] == thr and len(thr16) % 4 == 0 and all(np.isinf(thr16[len(thr):]))
+    assert q16[:len(q)] == q and len(q16) % 16 == 0
+    for name, vals, per in (("LV0", lv0, 4), ("THR", thr16, 4), ("QCELL", q16, 16)):
+        assert f"#define TACTKV_{name}_VEC {len(vals) // per}" in text
+
+
 # ------------------------------------------------------------------- occupancy and capacity ---
 @pytest.mark.parametrize("bits", [1, 2, 4, 8])
 def test_occupancy_of_an_oracle_payload(T, bits):
