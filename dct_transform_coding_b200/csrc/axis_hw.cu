@@ -30,7 +30,8 @@ __global__ void __launch_bounds__(kMaxHwThreads, (HX > 0 ? 2 : kHwMinBlocks)) fd
                                                min(g.S, ks0 + spc), smem);
 }
 
-template <int HC, int WC, int HX, int WX, int MODE, bool VAR>
+// NX: the channel count when fixed at compile time (512 or 1024, the exact grids' plain decode), else 0.
+template <int HC, int WC, int HX, int WX, int MODE, bool VAR, int NX = 0>
 __global__ void __launch_bounds__(kMaxHwThreads, hw_min_blocks_inv<HX>()) idct_hw_kernel(const __grid_constant__ Geom g,
                                                                                          const __grid_constant__ UnitList ul,
                                                                                          float* __restrict__ V,
@@ -39,8 +40,8 @@ __global__ void __launch_bounds__(kMaxHwThreads, hw_min_blocks_inv<HX>()) idct_h
                                                                                          int spc) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int ks0 = blockIdx.y * spc;
-  idct_hw_slabs<HC, WC, HX, WX, MODE, false, VAR>(g, ul, V, index, recs, g.unit0 + blockIdx.z, blockIdx.x, ks0,
-                                                  min(g.S, ks0 + spc), smem);
+  idct_hw_slabs<HC, WC, HX, WX, MODE, false, VAR, NX>(g, ul, V, index, recs, g.unit0 + blockIdx.z, blockIdx.x, ks0,
+                                                      min(g.S, ks0 + spc), smem);
 }
 
 }  // namespace
@@ -73,6 +74,8 @@ cudaError_t launch_hw(bool inverse, int mode, const Geom& g, const UnitList& ul,
       else TACTKV_GO((idct_hw_kernel<H, W, HX, WX, kRaw, false>), g, ul, buf, slab_off, recs, spc);
     } else {
       if (var) TACTKV_GO((idct_hw_kernel<H, W, HX, WX, kQuant, true>), g, ul, buf, slab_off, recs, spc);
+      else if (HX > 0 && g.n == 1024) TACTKV_GO((idct_hw_kernel<H, W, HX, WX, kQuant, false, HX ? 1024 : 0>), g, ul, buf, slab_off, recs, spc);
+      else if (HX > 0 && g.n == 512) TACTKV_GO((idct_hw_kernel<H, W, HX, WX, kQuant, false, HX ? 512 : 0>), g, ul, buf, slab_off, recs, spc);
       else TACTKV_GO((idct_hw_kernel<H, W, HX, WX, kQuant, false>), g, ul, buf, slab_off, recs, spc);
     }
   } else {

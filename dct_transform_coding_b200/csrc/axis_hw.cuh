@@ -266,12 +266,12 @@ __device__ __forceinline__ int cp_index(int Wp, int h, int wp) { return (h * Wp 
 // inverse along S: V_hi[u][k_s][cell pair][c] = (bf16(v[2p]), bf16(v[2p+1])) over V (as
 // __nv_bfloat162) and the remainders V_lo = bf16(v - float(V_hi)) over Vlo (W even).  Together
 // they carry v to about 2^-17 relative.
-template <int HC, int WC, int HX, int WX, int MODE, bool PAIRS = false, bool VAR = false>
+template <int HC, int WC, int HX, int WX, int MODE, bool PAIRS = false, bool VAR = false, int NX = 0>
 __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul, float* __restrict__ V,
                                               const uint32_t* __restrict__ index, const uint4* __restrict__ recs, int u,
                                               int chunk, int ks0, int ks1, unsigned char* smem,
                                               __nv_bfloat162* __restrict__ Vlo = nullptr) {
-  const Dims<HX, WX> D(g);
+  const Dims<HX, WX, NX> D(g);
   constexpr bool raw = MODE == kRaw;
   const HwLayout L = hw_layout(D.H, D.W, kLayDecode);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
@@ -316,7 +316,7 @@ __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul,
     if (ok) issue_slab(ks0);
     cp_async_commit();
   }
-  float* vunit = V + (size_t)u * g.S * D.HW * g.n + chunk * kChunk + lane;
+  float* vunit = V + (size_t)u * g.S * D.HW * D.n + chunk * kChunk + lane;
 
   for (int ks = ks0; ks < ks1; ++ks) {
     cp_async_wait_all();
@@ -434,14 +434,14 @@ __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul,
             vl[o] = __floats2bfloat162_rn(xh[h].x - back.x, xh[h].y - back.y);
           }
       } else {
-        float* v = vunit + ((size_t)ks * D.HW + 2 * wp) * g.n;
+        float* v = vunit + ((size_t)ks * D.HW + 2 * wp) * D.n;
         const bool two = 2 * wp + 1 < D.W;
 #pragma unroll
         for (int h = 0; h < HC; ++h)
           if (h < D.H) {
-            float* cell = v + (size_t)h * D.W * g.n;
+            float* cell = v + (size_t)h * D.W * D.n;
             cell[0] = xh[h].x;
-            if (two) cell[g.n] = xh[h].y;
+            if (two) cell[D.n] = xh[h].y;
           }
       }
     }

@@ -72,6 +72,8 @@ def test_tiny_config_fp32_io():
     ((32, 24, 24, 1, 32), 1),   # fused, S = 32 on the 24 x 24 grid (the 32B-class medical layout)
     ((8, 24, 24, 1, 64), 4),    # fused, S = 8 on the 24 x 24 grid (one slab per CTA of the cluster)
     ((64, 24, 24, 1, 32), 2),   # S = 64 on the 24 x 24 grid: the separate transform kernels
+    ((8, 16, 16, 2, 256), 2),   # 512 channels: the decode kernel with its channel count fixed
+    ((8, 8, 8, 4, 256), 3),     # 1024 channels on the 8 x 8 grid, likewise
 ])
 def test_small_shapes_bf16(shape, bits):
     S, H, W, heads, D = shape
