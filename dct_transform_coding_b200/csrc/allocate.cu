@@ -21,9 +21,7 @@
 //
 // The kernel also writes the first stream bit P(k_s) of every S slab (the same for every
 // channel) and the list of bins with bits (records {bin, bits, first stream bit, 1/sigma}, in bin
-// order) into the workspace, and zeroes the stream word where each packing range of kPackRecs
-// records starts and the word of the last code bit: the packing kernel ORs the words it shares
-// with a neighbouring range into those.  decode_index_kernel rebuilds P from a payload before
+// order) into the workspace.  decode_index_kernel rebuilds P from a payload before
 // decoding and checks the header and the bit widths.
 #include "common.cuh"
 
@@ -140,7 +138,6 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
   __shared__ uint32_t s_nzslab[kMaxSlabs];
   __shared__ uint32_t s_P[kMaxSlabs + 1];
   __shared__ uint32_t s_NZ[kMaxSlabs + 1];
-  __shared__ uint32_t s_bpos[kMaxN / kPackRecs + 1];
   __shared__ uint32_t s_hist[kExpBuckets], s_rev[kExpBuckets];
   __shared__ int s_pick;
   __shared__ uint32_t s_above, s_count;
@@ -303,8 +300,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
     pay[i] = 0;
   const long long code_bits = raw ? 32LL * g.N : block_sum<long long>(code_bits_local, s_ll);
   const long long cstride = pad16((code_bits + 7) / 8);
-  // slab offsets P(k_s) and record offsets NZ(k_s), and a zero in the stream word at every P(k_s)
-  // of every channel
+  // slab offsets P(k_s) and record offsets NZ(k_s)
   __syncthreads();
   if (threadIdx.x < 32) slab_scan(s_slab, g.S, s_P);
   else if (threadIdx.x < 64) slab_scan(s_nzslab, g.S, s_NZ);
@@ -331,21 +327,9 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const __grid_co
       const uint2 sb = reinterpret_cast<const uint2*>(var)[i];   // {sigma_i, b_i} of this thread's bins
       const uint32_t b = sb.y;
       if (b) {
-        if (slot % kPackRecs == 0) s_bpos[slot / kPackRecs] = pos;   // a packing range starts here
         urecs[slot++] = make_uint4((uint32_t)i, b, pos, __float_as_uint(__frcp_rn(__uint_as_float(sb.x))));
         pos += b;
       }
-    }
-    __syncthreads();
-    // zero the stream word where each packing range starts and the word holding the last code bit:
-    // neighbouring ranges OR their bits into them
-    const uint32_t sw = (uint32_t)(cstride / 4), nrec = s_NZ[g.S];
-    const uint32_t nb = (nrec + kPackRecs - 1) / kPackRecs;
-    uint32_t* words = reinterpret_cast<uint32_t*>(pay + g.off_codes);
-    for (uint32_t k = 0; k <= nb; ++k) {
-      const uint32_t w = (k < nb ? s_bpos[k] : s_P[g.S]) >> 5;
-      if (w < sw)
-        for (int c = threadIdx.x; c < g.n; c += blockDim.x) words[(size_t)c * sw + w] = 0u;
     }
   }
   if (threadIdx.x == 0) {

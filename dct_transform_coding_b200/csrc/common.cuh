@@ -25,7 +25,8 @@ constexpr size_t kStatusBytes = 256;       // status word at the start of the wo
 constexpr int kMaxHW = 1024;               // H*W limit of the H/W-axis kernels
 constexpr int kMaxSlabs = 64;              // S limit
 constexpr int kMaxN = kMaxSlabs * kMaxHW;  // bins per unit limit
-constexpr int kPackRecs = 1024;            // records per packing range (one CTA)
+// Records per packing range (one CTA) when a lane packs four channels; 4 * kPackRecs when it packs one.
+constexpr int kPackRecs = 256;
 
 enum HwMode { kStats = 0, kQuant = 1, kRaw = 2 };
 

@@ -212,12 +212,17 @@ def test_cross_decode_oracle_payload_on_gpu():
     assert rel_rms(y[0].double().cpu().numpy(), ref) <= 1e-3
 
 
-def test_payload_bytes_match_oracle_format():
+@pytest.mark.parametrize("shape,bits", [
+    ((8, 8, 8, 1, 64), 2),     # two chunks: one channel per lane, one packing range
+    ((8, 8, 8, 4, 32), 2),     # four chunks: four channels per lane, ranges of 256 records
+    ((16, 8, 8, 4, 32), 1),    # likewise, more ranges at 1 bit
+])
+def test_payload_bytes_match_oracle_format(shape, bits):
     """Where allocations and codes agree, the GPU payload is byte-identical to the oracle's."""
-    S, H, W, heads, D = 8, 8, 8, 1, 64
+    S, H, W, heads, D = shape
     x = make_unit(S, H, W, heads, D, rho=(0.9, 0.9, 0.9), nu=4.0, seed=21, device=DEV)[None]
-    pay, _ = _round_trip(x, S, H, W, 2, layers=[0], kvs=[0])
-    p_o, info = O.compress_unit(x[0].double().cpu().numpy(), S, H, W, heads, D, 2, return_info=True)
+    pay, _ = _round_trip(x, S, H, W, bits, layers=[0], kvs=[0])
+    p_o, info = O.compress_unit(x[0].double().cpu().numpy(), S, H, W, heads, D, bits, return_info=True)
     g = pay[0].cpu().numpy().tobytes()[:len(p_o)]
     po = np.frombuffer(p_o, np.uint8)
     gg = np.frombuffer(g, np.uint8)
@@ -228,6 +233,30 @@ def test_payload_bytes_match_oracle_format():
     _, codes_g = O.codes_of(g)
     if np.array_equal(codes_g, info["codes"]):
         assert np.array_equal(gg[lay["off_codes"]:], po[lay["off_codes"]:])
+
+
+@pytest.mark.parametrize("bits,flags", [(1, 0), (4, 0), (2, 64)])
+def test_payload_independent_of_buffer_contents(bits, flags):
+    """The packer clears the bit fields it owns in the stream words it shares with a neighbouring
+    range instead of relying on zeroed memory: payload buffers filled with zeros, with ones and
+    with random bytes give the same payload.  A benchmark-size unit (many packing ranges); flags 64
+    (the rotation) takes the one-channel-per-lane packer."""
+    S, H, W, heads, D = 64, 16, 16, 4, 256
+    x = make_unit(S, H, W, heads, D, rho=(0.85, 0.9, 0.9), nu=4.0, seed=5 + bits, device=DEV)[None]
+    cap = T.payload_capacity(S, H, W, heads, D, bits, flags)
+    cap = (cap + 15) // 16 * 16
+    fills = [torch.zeros((1, cap), dtype=torch.uint8, device=DEV),
+             torch.full((1, cap), 255, dtype=torch.uint8, device=DEV),
+             torch.randint(0, 256, (1, cap), dtype=torch.uint8, device=DEV,
+                           generator=torch.Generator(device=DEV).manual_seed(bits))]
+    outs = []
+    for buf in fills:
+        T.compress(x, S, H, W, bits, layers=[0], kvs=[0], flags=flags, payload=buf)
+        torch.cuda.synchronize()
+        outs.append(buf[0].cpu().numpy().tobytes())
+    used = T.tactkv_occupancy(outs[0])["payload_bytes"]
+    assert used > 0
+    assert outs[1][:used] == outs[0][:used] and outs[2][:used] == outs[0][:used]
 
 
 # ------------------------------------------------------------------------------- full sizes ---
