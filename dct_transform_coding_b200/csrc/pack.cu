@@ -178,7 +178,8 @@ __global__ void __launch_bounds__(kPackThreads, 4) pack_kernel(const __grid_cons
     mine[q] = e < m ? urecs[r0 + e] : make_uint4(0u, 0u, 0u, 0u);
   }
   if (VAR && head_gains_on(g.flags)) {   // 1/gain of the CTA's head (0 for a zero gain: u = 0)
-    const float* hg = reinterpret_cast<const float*>(pay + g.off_sigma) + (size_t)(chunk0 * kChunk / g.head_dim) * g.N;
+    const float* hg =
+        reinterpret_cast<const float*>(pay + g.off_sigma) + (size_t)(chunk0 * kChunk / g.head_dim) * g.N;
 #pragma unroll
     for (int q = 0; q < kPer; ++q)
       if (mine[q].y) {
@@ -212,9 +213,20 @@ __global__ void __launch_bounds__(kPackThreads, 4) pack_kernel(const __grid_cons
     __syncwarp();
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    uint32_t run = 0;
-    for (int b = 1; b <= 8; ++b) {
+  if (warp == 0) {   // lane b - 1: width b's first slot (groups padded to whole blocks), its warps' slots
+    const int b = lane + 1;
+    uint32_t tot = 0;
+    if (lane < 8)
+      for (int w = 0; w < kWarps; ++w) tot += s_cnt[b][w];
+    const uint32_t padded = (tot + PB - 1) / PB * PB;
+    uint32_t incl = padded;
+#pragma unroll
+    for (int d = 1; d < 8; d <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += v;
+    }
+    if (lane < 8) {
+      uint32_t run = incl - padded;
       s_grp[b] = run;
       for (int w = 0; w < kWarps; ++w) {
         const uint32_t c = s_cnt[b][w];
@@ -222,9 +234,8 @@ __global__ void __launch_bounds__(kPackThreads, 4) pack_kernel(const __grid_cons
         run += c;
       }
       s_fill[b] = run;
-      run = (run + PB - 1) / PB * PB;
     }
-    s_grp[9] = run;
+    if (lane == 7) s_grp[9] = incl;
   }
   __syncthreads();
 #pragma unroll
@@ -342,7 +353,8 @@ cudaError_t launch_pack(const Geom& g, const UnitList& ul, int nu, const float* 
     pack_raw_kernel<<<dim3(g.nch, g.S, nu), kPackThreads, 0, st>>>(g, ul, X, spc);
   } else {
     // four channels per lane where the chunks come in fours, else one; a unit has at most N
-    // records, CTAs past its last record exit
+    // records, CTAs past its last record exit (measured: a CTA looping over two ranges, to launch
+    // fewer CTAs without work, was slower)
     auto go = [&](auto kernel, int cpl, size_t smem, int recs_per_cta) {
       cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       const dim3 grid(g.nch / cpl, (g.N + recs_per_cta - 1) / recs_per_cta, nu);
