@@ -412,6 +412,12 @@ __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul,
         }
     }
     __syncthreads();
+    // the words and records of slab ks are used up: with a single slot, the next slab's load
+    // starts now and overlaps the pass along H and the stores
+    if (L.nslot == 1 && ok && !raw && ks + 1 < ks1) {
+      issue_slab(ks + 1);
+      cp_async_commit();
+    }
     // inverse DCT along H on column pair wp; store to V
     for (int wp = warp; wp < WP; wp += nwarps) {
       float2 xh[HC];
@@ -444,10 +450,6 @@ __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul,
             if (two) cell[D.n] = xh[h].y;
           }
       }
-    }
-    if (L.nslot == 1 && ok && !raw && ks + 1 < ks1) {   // the single slot is free once the records are used
-      issue_slab(ks + 1);
-      cp_async_commit();
     }
   }
   cp_async_wait_all();
