@@ -293,7 +293,7 @@ __global__ void __launch_bounds__(kSoftmaxThreads, 2) attn_softmax_kernel(const 
     }
     return;
   }
-  const int W = g.W, Wr = vol_row(W);
+  const int W = WX ? WX : g.W, Wr = vol_row(W);   // (a division by a constant on the exact grids)
   auto at = [&](int i) { return (i / W) * Wr + (i - (i / W) * W); };   // bin i -> its padded place
   for (int i = threadIdx.x; i < g.N; i += blockDim.x) vol[at(i)] = zg[i];
   __syncthreads();
@@ -395,8 +395,19 @@ __global__ void __launch_bounds__(kAttnThreads) attn_reduce_kernel(const __grid_
   for (int d0 = 0; d0 < D; d0 += blockDim.x) {
     const int d = d0 + threadIdx.x;
     float acc = 0.f;
-    if (d < D)
-      for (int ks = 0; ks < g.S; ++ks) acc += part[(((size_t)u * g.S + ks) * q_heads + j) * D + d];
+    if (d < D) {   // in slab order; the loads of 16 slabs are issued before their sums
+      const float* pp = part + ((size_t)u * g.S * q_heads + j) * D + d;
+      const size_t st = (size_t)q_heads * D;
+      int ks = 0;
+      for (; ks + 16 <= g.S; ks += 16) {
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = pp[(size_t)(ks + i) * st];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc += v[i];
+      }
+      for (; ks < g.S; ++ks) acc += pp[(size_t)ks * st];
+    }
     if (rotate)   // R^T y = diag(s) H y / sqrt(32); D is a multiple of 32, so whole warps take part
       acc = warp_wht(acc, lane) * kInvSqrt32 * rotation_sign((unsigned long long)(h * D + (d < D ? d : 0)));
     if (d < D) out[((size_t)u * q_heads + j) * D + d] = acc * inv_l;
