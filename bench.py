@@ -355,9 +355,11 @@ def main():
 
 def attention_bench(T, w, bits, payload, out, du, ws, stream, layers, kvs, peak, peak_kind, q_per_kv=2, iters=20):
     """One decode step of attention for every layer of the batch, straight from the compressed K/V
-    (units with kv 0 / 1 of the same layer), against the same step done by decompressing the batch
-    to bf16 and running torch's scaled_dot_product_attention on it.  The roofline counts the bytes
-    the step must read (the K and V payloads, the queries) and write (outputs, m, l)."""
+    (units with kv 0 / 1 of the same layer), against the same step done by decompressing K and V to
+    bf16, straight into the [layers, heads, tokens, head_dim] layout SDPA takes (through the output
+    strides), and running torch's scaled_dot_product_attention on them; both warmed up first.  The
+    roofline counts the bytes the step must read (the K and V payloads, the queries) and write
+    (outputs, m, l)."""
     import torch
     kvs = kvs[:payload.shape[0]]
     ki = [i for i, kv in enumerate(kvs) if kv == 0]
@@ -378,14 +380,26 @@ def attention_bench(T, w, bits, payload, out, du, ws, stream, layers, kvs, peak,
     ev[1].record(stream)
     sp = int(stream.cuda_stream)
     qh = q.to(torch.bfloat16)[:, :, None, :]
+    Kb = torch.empty((U, w.heads, w.tokens, D), dtype=torch.bfloat16, device=dev)   # [U, heads, T, D]
+    Vb = torch.empty_like(Kb)
+    dk = T.make_units(None, w.S, w.H, w.W, bits, heads=w.heads, head_dim=D, payload=pk,
+                      out=Kb.permute(0, 2, 1, 3), layers=lay, kvs=[0] * U)
+    dv = T.make_units(None, w.S, w.H, w.W, bits, heads=w.heads, head_dim=D, payload=pv,
+                      out=Vb.permute(0, 2, 1, 3), layers=lay, kvs=[1] * U)
+
+    def baseline():
+        for units in (dk, dv):
+            st = T.tactkv_decompress(units, ws.data_ptr(), ws.numel(), sp)
+            if st != T.TACTKV_OK:
+                raise T.TactkvError(st, "attention baseline")
+        with torch.cuda.stream(stream):
+            torch.nn.functional.scaled_dot_product_attention(qh, Kb, Vb, enable_gqa=True)
+
     for _ in range(3):
-        T.tactkv_decompress(du, ws.data_ptr(), ws.numel(), sp)
+        baseline()
     ev[2].record(stream)
     for _ in range(iters):
-        T.tactkv_decompress(du, ws.data_ptr(), ws.numel(), sp)
-        K = out[ki].permute(0, 2, 1, 3)             # [U, heads, T, D]
-        V = out[vi].permute(0, 2, 1, 3)
-        torch.nn.functional.scaled_dot_product_attention(qh, K, V, enable_gqa=True)
+        baseline()
     ev[3].record(stream)
     torch.cuda.synchronize()
     ms = ev[0].elapsed_time(ev[1]) / iters

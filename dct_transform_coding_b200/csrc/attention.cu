@@ -366,6 +366,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_values_kernel(const __grid_
 #pragma unroll
     for (int gq = 0; gq < GM; ++gq) acc[gq] = 0.f;
     const uint32_t* row = words + d * stride;
+    // four bins' loads in flight at a time; the sums keep their order
+#pragma unroll 4
     for (int a = 0; a < na; ++a) {
       const uint2 r = actrec[a];
       const uint32_t k = r.y & 0xffu, off = r.y >> 8;
