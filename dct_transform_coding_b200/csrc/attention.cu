@@ -31,10 +31,16 @@ constexpr float kInvSqrt32 = 0.17677669529663687f;
 constexpr int kLv0Floats = TACTKV_LV0_VEC * 4;   // the levels behind a zero, in whole 16-byte vectors
 static_assert(kLv0Floats >= kLmLvTotal + 1, "level table");
 
-// Words of a channel stream held per slab in shared memory: the most a slab can span (8 bits per
-// bin, from any bit of its first word), two zero words for the look-ahead of the code reads, and
-// an odd count, so that 32 lanes reading 32 channels' rows at one offset hit 32 banks.
-__host__ __device__ inline int attn_word_stride(int HW) { return ((8 * HW + 31) / 32 + 3) | 1; }
+// Words of a channel stream held per slab in shared memory: what a slab spans at 2 * bits + 2 bits
+// per bin (at most 8), from any bit of its first word, two zero words for the look-ahead of the
+// code reads, and an odd count, so that 32 lanes reading 32 channels' rows at one offset hit 32
+// banks.  A slab whose codes span more (its bins hold far more than the average bits) is decoded
+// from the payload in global memory instead.  Sizing the rows for the call's rate rather than for
+// 8 bits per bin leaves room for more CTAs per SM.
+__host__ __device__ inline int attn_cap_bits(int bits) { return 2 * bits + 2 < 8 ? 2 * bits + 2 : 8; }
+__host__ __device__ inline int attn_word_stride(int HW, int bits) {
+  return ((attn_cap_bits(bits) * HW + 31) / 32 + 3) | 1;
+}
 __host__ __device__ inline int pad32(int x) { return (x + 31) / 32 * 32; }
 
 // Copy the words of slab ks of the D channel streams from `row0` (channel 0's stream, word P(ks)
@@ -94,13 +100,24 @@ __device__ int stage_active(const uint4* __restrict__ srec, int HW, int W, uint2
   return na;
 }
 
-// Dequantized coefficient of a bin (record {sigma, offset << 8 | mask}) in a channel's staged row
-// (the slab's first word on); a zero record gives 0 through the zero in front of the levels.
-__device__ __forceinline__ float decode_staged(const uint32_t* __restrict__ row, uint2 r, const float* lvs1) {
-  const uint32_t k = r.y & 0xffu, off = r.y >> 8;
+// Codebook level of a bin's code (record word y = offset << 8 | mask) in a channel's row from the
+// slab's first word on: staged in shared memory (GLOBAL false: two zero words after the slab make
+// the second word always readable) or the payload's stream itself (GLOBAL true: the second word is
+// read only when the code reaches into it, so nothing past the stream is touched).  A bin without
+// bits (mask 0) gives the zero in front of the levels.
+template <bool GLOBAL>
+__device__ __forceinline__ float level_at(const uint32_t* __restrict__ row, uint32_t y, const float* lvs1) {
+  const uint32_t k = y & 0xffu, off = y >> 8;
   const uint32_t* w = row + (off >> 5);
-  const uint32_t code = __funnelshift_r(w[0], w[1], off) & k;
-  return __uint_as_float(r.x) * lvs1[(int)(k + code) - 1];
+  uint32_t lo, hi;
+  if constexpr (GLOBAL) {
+    lo = __ldg(w);
+    hi = (off & 31u) + (uint32_t)__popc(k) > 32u ? __ldg(w + 1) : 0u;   // uniform across the warp
+  } else {
+    lo = w[0];
+    hi = w[1];
+  }
+  return lvs1[(int)(k + (__funnelshift_r(lo, hi, off) & k)) - 1];
 }
 
 // With per-head gains: the staged records of the active bins take head h's gains instead of the
@@ -112,28 +129,35 @@ __device__ __forceinline__ void head_gain_records(const Geom& g, const unsigned 
 }
 
 // z_j[i] for the G query heads of K/V head h over the bins of slab ks.  The slab's words of the
-// head's D channel streams are staged in shared memory.  The warps work in pairs on batches of 32
-// active bins (pair p takes batches p, p + 4, ...); warp w of the pair takes the channel groups
-// cg = w, w + 2, ... (lane = channel within a group) and, for two query heads at a time, accumulates
-// q_j[d] X_K[i, d] over them in registers, sums over its 32 lanes (transpose sum: lane l ends with
-// active bin a0 + l), and the second warp's sums are added to the first's through shared memory.
+// head's D channel streams are staged in shared memory when they fit (else read from the payload).
+// The warps work in pairs on batches of 16 active bins (pair p takes batches p, p + 4, ...); warp
+// w of the pair takes the channel groups cg = w, w + 2, ... (lane = channel within a group) and,
+// for two query heads at a time, accumulates q_j[d] X_K[i, d] over them in registers (32 sums: two
+// heads x 16 bins), sums over its 32 lanes (transpose sum: lane l ends with head l >> 4 and active
+// bin a0 + (l & 15)), and the second warp's sums are added to the first's through shared memory.
 // z of the bins without bits is 0.
 constexpr int kScoreThreads = 256;
 constexpr int kScorePairs = kScoreThreads / 64;
-__global__ void __launch_bounds__(kScoreThreads) attn_scores_kernel(const __grid_constant__ Geom g,
-                                                                    const __grid_constant__ UnitList ul,
-                                                                    const uint32_t* __restrict__ index,
-                                                                    const uint4* __restrict__ recs,
-                                                                    const float* __restrict__ q, int q_heads,
-                                                                    float* __restrict__ z) {
+constexpr int kScoreBatch = 16;
+template <bool B>
+struct BoolTag {
+  static constexpr bool value = B;
+};
+
+__global__ void __launch_bounds__(kScoreThreads, 3) attn_scores_kernel(const __grid_constant__ Geom g,
+                                                                       const __grid_constant__ UnitList ul,
+                                                                       const uint32_t* __restrict__ index,
+                                                                       const uint4* __restrict__ recs,
+                                                                       const float* __restrict__ q, int q_heads,
+                                                                       float* __restrict__ z) {
   extern __shared__ __align__(16) float sh[];
   __shared__ int s_count, s_warp[32];
-  __shared__ float s_red[kScorePairs][2][32];
+  __shared__ float s_red[kScorePairs][32];
   const int ks = blockIdx.x, h = blockIdx.y, u = blockIdx.z;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  const int G = q_heads / g.heads, D = g.head_dim, HW = g.HW, stride = attn_word_stride(HW);
+  const int G = q_heads / g.heads, D = g.head_dim, HW = g.HW, stride = attn_word_stride(HW, g.bits);
   float* lvs1 = sh + 1;                                        // a zero in front of the levels
-  float* qs = sh + kLv0Floats;               // [G][D], rotated when the payload is
+  float* qs = sh + kLv0Floats;                                 // [G][D], rotated when the payload is
   float* zs = qs + G * D;                                      // [G][HW]
   uint2* actrec = reinterpret_cast<uint2*>(zs + (G * HW + 1) / 2 * 2);   // [pad32(HW)]
   int* act = reinterpret_cast<int*>(actrec + pad32(HW));                 // [HW]
@@ -141,12 +165,12 @@ __global__ void __launch_bounds__(kScoreThreads) attn_scores_kernel(const __grid
   const uint32_t* P = index + (size_t)u * unit_index_words(g.S);
   const bool ok = P[g.S + 1] != 0;
   const unsigned char* pay = ul.u[u].payload;
-  if (ok) {
-    const uint32_t p0 = P[ks], p1 = P[ks + 1], sw = reinterpret_cast<const uint32_t*>(pay)[11] / 4;
-    const int nw = (int)(((p0 & 31u) + (p1 - p0) + 31) >> 5);
-    stage_words(reinterpret_cast<const uint32_t*>(pay + g.off_codes) + (size_t)h * D * sw + (p0 >> 5), sw, D, nw,
-                stride, words);
-  }
+  const uint32_t p0 = ok ? P[ks] : 0u, p1 = ok ? P[ks + 1] : 0u;
+  const uint32_t sw = ok ? reinterpret_cast<const uint32_t*>(pay)[11] / 4 : 0u;
+  const int nw = (int)(((p0 & 31u) + (p1 - p0) + 31) >> 5);
+  const bool staged = nw + 2 <= stride;                        // the same for the whole CTA
+  const uint32_t* streams = reinterpret_cast<const uint32_t*>(pay + g.off_codes) + (size_t)h * D * sw + (p0 >> 5);
+  if (ok && staged) stage_words(streams, sw, D, nw, stride, words);
   copy_vec16(sh, g_lm_levels0, TACTKV_LV0_VEC);
   for (int i = threadIdx.x; i < G * HW; i += blockDim.x) zs[i] = 0.f;
   const float* qu = q + ((size_t)u * q_heads + (size_t)h * G) * D;
@@ -164,41 +188,41 @@ __global__ void __launch_bounds__(kScoreThreads) attn_scores_kernel(const __grid
   __syncthreads();
   const float scale = rsqrtf((float)D);
   const int pair = warp >> 1, half = warp & 1;
-  const int rounds = (na + kScorePairs * 32 - 1) / (kScorePairs * 32);   // the same for every warp
-  for (int it = 0; it < rounds; ++it) {
-    const int a0 = (it * kScorePairs + pair) * 32;
-    for (int gp = 0; gp < G; gp += 2) {
-      const bool two = gp + 1 < G;
-      float s0 = 0.f, s1 = 0.f;
-      if (a0 < na) {
-        float acc0[32], acc1[32];
+  const int rounds = (na + kScorePairs * kScoreBatch - 1) / (kScorePairs * kScoreBatch);   // the same for every warp
+  auto batches = [&](auto global) {
+    constexpr bool kGlobal = decltype(global)::value;
+    for (int it = 0; it < rounds; ++it) {
+      const int a0 = (it * kScorePairs + pair) * kScoreBatch;
+      for (int gp = 0; gp < G; gp += 2) {
+        const bool two = gp + 1 < G;
+        float s = 0.f;
+        if (a0 < na) {
+          float acc[2 * kScoreBatch];   // [head gp, gp + 1][bin a0 ..]
 #pragma unroll
-        for (int b = 0; b < 32; ++b) acc0[b] = acc1[b] = 0.f;
-        for (int d = half * 32 + lane; d < D; d += 64) {
-          const uint32_t* row = words + d * stride;
-          const float q0 = qs[gp * D + d], q1 = two ? qs[(gp + 1) * D + d] : 0.f;
+          for (int b = 0; b < 2 * kScoreBatch; ++b) acc[b] = 0.f;
+          for (int d = half * 32 + lane; d < D; d += 64) {
+            const uint32_t* row = kGlobal ? streams + (size_t)d * sw : words + d * stride;
+            const float q0 = qs[gp * D + d], q1 = two ? qs[(gp + 1) * D + d] : 0.f;
 #pragma unroll
-          for (int b = 0; b < 32; ++b) {
-            const float x = decode_staged(row, actrec[a0 + b], lvs1);
-            acc0[b] = fmaf(x, q0, acc0[b]);
-            acc1[b] = fmaf(x, q1, acc1[b]);
+            for (int b = 0; b < kScoreBatch; ++b) {
+              const uint2 r = actrec[a0 + b];   // {sigma, offset << 8 | mask}
+              const float x = __uint_as_float(r.x) * level_at<kGlobal>(row, r.y, lvs1);
+              acc[b] = fmaf(x, q0, acc[b]);
+              acc[kScoreBatch + b] = fmaf(x, q1, acc[kScoreBatch + b]);
+            }
           }
+          s = warp_transpose_sum(acc, lane);
+          if (half) s_red[pair][lane] = s;
         }
-        s0 = warp_transpose_sum(acc0, lane);
-        s1 = warp_transpose_sum(acc1, lane);
-        if (half) {
-          s_red[pair][0][lane] = s0;
-          s_red[pair][1][lane] = s1;
-        }
+        __syncthreads();
+        const int a = a0 + (lane & (kScoreBatch - 1)), gq = gp + (lane >> 4);
+        if (!half && a0 < na && a < na && (gq == gp || two)) zs[gq * HW + act[a]] = (s + s_red[pair][lane]) * scale;
+        __syncthreads();
       }
-      __syncthreads();
-      if (!half && a0 + lane < na) {
-        zs[gp * HW + act[a0 + lane]] = (s0 + s_red[pair][0][lane]) * scale;
-        if (two) zs[(gp + 1) * HW + act[a0 + lane]] = (s1 + s_red[pair][1][lane]) * scale;
-      }
-      __syncthreads();
     }
-  }
+  };
+  if (staged) batches(BoolTag<false>{});
+  else batches(BoolTag<true>{});
   float* zu = z + ((size_t)u * q_heads + (size_t)h * G) * g.N + (size_t)ks * HW;
   for (int i = threadIdx.x; i < G * HW; i += blockDim.x) {
     const int gq = i / HW, j = i - gq * HW;
@@ -332,7 +356,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_values_kernel(const __grid_
   extern __shared__ __align__(16) float sh[];
   __shared__ int s_count, s_warp[32];
   const int ks = blockIdx.x, h = blockIdx.y, u = blockIdx.z;
-  const int G = q_heads / g.heads, D = g.head_dim, HW = g.HW, stride = attn_word_stride(HW);
+  const int G = q_heads / g.heads, D = g.head_dim, HW = g.HW, stride = attn_word_stride(HW, g.bits);
   float* lvs1 = sh + 1;
   float* wt = sh + kLv0Floats;        // [HW][G]: weight of active bin a for head g
   uint2* actrec = reinterpret_cast<uint2*>(wt + ((size_t)G * HW + 1) / 2 * 2);   // [pad32(HW)], 8-byte aligned
@@ -341,12 +365,12 @@ __global__ void __launch_bounds__(kAttnThreads) attn_values_kernel(const __grid_
   const uint32_t* P = index + (size_t)u * unit_index_words(g.S);
   const bool ok = P[g.S + 1] != 0;
   const unsigned char* pay = ul.u[u].payload;
-  if (ok) {
-    const uint32_t p0 = P[ks], p1 = P[ks + 1], sw = reinterpret_cast<const uint32_t*>(pay)[11] / 4;
-    const int nw = (int)(((p0 & 31u) + (p1 - p0) + 31) >> 5);
-    stage_words(reinterpret_cast<const uint32_t*>(pay + g.off_codes) + (size_t)h * D * sw + (p0 >> 5), sw, D, nw,
-                stride, words);
-  }
+  const uint32_t p0 = ok ? P[ks] : 0u, p1 = ok ? P[ks + 1] : 0u;
+  const uint32_t sw = ok ? reinterpret_cast<const uint32_t*>(pay)[11] / 4 : 0u;
+  const int nw = (int)(((p0 & 31u) + (p1 - p0) + 31) >> 5);
+  const bool staged = nw + 2 <= stride;                        // the same for the whole CTA
+  const uint32_t* streams = reinterpret_cast<const uint32_t*>(pay + g.off_codes) + (size_t)h * D * sw + (p0 >> 5);
+  if (ok && staged) stage_words(streams, sw, D, nw, stride, words);
   copy_vec16(sh, g_lm_levels0, TACTKV_LV0_VEC);
   const uint4* srec = recs + (size_t)u * g.N + (size_t)ks * ((g.H + 1) / 2) * g.W;
   const int na = ok ? stage_active(srec, HW, g.W, actrec, act, &s_count, s_warp) : 0;
@@ -361,26 +385,28 @@ __global__ void __launch_bounds__(kAttnThreads) attn_values_kernel(const __grid_
   }
   cp_async_wait_all();
   __syncthreads();
-  for (int d = threadIdx.x; d < D; d += blockDim.x) {
-    float acc[GM];
+  auto channels = [&](auto global) {
+    constexpr bool kGlobal = decltype(global)::value;
+    for (int d = threadIdx.x; d < D; d += blockDim.x) {
+      float acc[GM];
 #pragma unroll
-    for (int gq = 0; gq < GM; ++gq) acc[gq] = 0.f;
-    const uint32_t* row = words + d * stride;
-    // four bins' loads in flight at a time; the sums keep their order
+      for (int gq = 0; gq < GM; ++gq) acc[gq] = 0.f;
+      const uint32_t* row = kGlobal ? streams + (size_t)d * sw : words + d * stride;
+      // four bins' loads in flight at a time; the sums keep their order
 #pragma unroll 4
-    for (int a = 0; a < na; ++a) {
-      const uint2 r = actrec[a];
-      const uint32_t k = r.y & 0xffu, off = r.y >> 8;
-      const uint32_t* w = row + (off >> 5);
-      const float lv = lvs1[(int)(k + (__funnelshift_r(w[0], w[1], off) & k)) - 1];
+      for (int a = 0; a < na; ++a) {
+        const float lv = level_at<kGlobal>(row, actrec[a].y, lvs1);   // (sigma is in the weights)
+#pragma unroll
+        for (int gq = 0; gq < GM; ++gq)
+          if (gq < G) acc[gq] = fmaf(wt[a * G + gq], lv, acc[gq]);
+      }
 #pragma unroll
       for (int gq = 0; gq < GM; ++gq)
-        if (gq < G) acc[gq] = fmaf(wt[a * G + gq], lv, acc[gq]);
+        if (gq < G) part[(((size_t)u * g.S + ks) * q_heads + (size_t)h * G + gq) * D + d] = acc[gq];
     }
-#pragma unroll
-    for (int gq = 0; gq < GM; ++gq)
-      if (gq < G) part[(((size_t)u * g.S + ks) * q_heads + (size_t)h * G + gq) * D + d] = acc[gq];
-  }
+  };
+  if (staged) channels(BoolTag<false>{});
+  else channels(BoolTag<true>{});
 }
 
 // out[u][j][d] = (R^T) sum over slabs, in slab order, of part / l (blockDim a multiple of 32;
@@ -421,13 +447,13 @@ __global__ void __launch_bounds__(kAttnThreads) attn_reduce_kernel(const __grid_
 size_t attention_scores_smem(const Geom& g, int q_heads) {
   const int G = q_heads / g.heads;
   return (size_t)(kLv0Floats + G * g.head_dim + (G * g.HW + 1) / 2 * 2) * 4 +
-         (size_t)pad32(g.HW) * 12 + (size_t)g.head_dim * attn_word_stride(g.HW) * 4;
+         (size_t)pad32(g.HW) * 12 + (size_t)g.head_dim * attn_word_stride(g.HW, g.bits) * 4;
 }
 size_t attention_softmax_smem(const Geom& g) { return softmax_smem(g); }
 size_t attention_values_smem(const Geom& g, int q_heads) {
   const int G = q_heads / g.heads;
   return (size_t)(kLv0Floats + (G * g.HW + 1) / 2 * 2) * 4 + (size_t)pad32(g.HW) * 12 +
-         (size_t)g.head_dim * attn_word_stride(g.HW) * 4;
+         (size_t)g.head_dim * attn_word_stride(g.HW, g.bits) * 4;
 }
 
 // One thread per channel of the head (head_dim is a multiple of 32), at most kAttnThreads.

@@ -198,8 +198,9 @@ tactkv_status tactkv_allocate(const tactkv_unit* unit, const double* var, void* 
      m, l      DEVICE float32 [n_units][q_heads]: the scores' maximum and sum_t exp(score - m), so
                that a caller can merge these tokens with its bf16 text tokens.
    Limits: n_units <= 128, head_dim a multiple of 32, and shared memory for one slab's stream words
-   of a head (head_dim * ((8*H*W + 31)/32 + 3, rounded up to odd) 4-byte words) and for the score
-   volume (S*H*(W rounded up to odd) floats) within 227 KB each; other shapes return
+   of a head (head_dim * ((c*H*W + 31)/32 + 3, rounded up to odd) 4-byte words, c = min(8, 2*bits + 2)
+   bits per bin; a slab whose codes span more is decoded from the payload directly) and for the
+   score volume (S*H*(W rounded up to odd) floats) within 227 KB each; other shapes return
    TACTKV_UNSUPPORTED_SHAPE (every benchmark grid fits).  workspace: at least
    tactkv_attention_workspace_bytes(k_units, n_units, q_heads) bytes, 256-byte aligned.  A corrupt
    payload is recorded as TACTKV_CORRUPT_PAYLOAD (tactkv_device_status) and contributes no

@@ -23,11 +23,12 @@ DEV = "cuda:0"
 TOL = 1e-4
 
 
-def _run(S, H, W, heads, D, G, bits, flags=0, units=2, qscale=1.0, seed=0):
-    k = torch.stack([make_unit(S, H, W, heads, D, rho=(0.9, 0.85, 0.85), nu=4.0, seed=seed + 2 * i, device=DEV)
-                     for i in range(units)])
-    v = torch.stack([make_unit(S, H, W, heads, D, rho=(0.9, 0.85, 0.85), nu=4.0, seed=seed + 2 * i + 1, device=DEV)
-                     for i in range(units)])
+def _run(S, H, W, heads, D, G, bits, flags=0, units=2, qscale=1.0, seed=0, k=None, v=None):
+    if k is None:
+        k = torch.stack([make_unit(S, H, W, heads, D, rho=(0.9, 0.85, 0.85), nu=4.0, seed=seed + 2 * i, device=DEV)
+                         for i in range(units)])
+        v = torch.stack([make_unit(S, H, W, heads, D, rho=(0.9, 0.85, 0.85), nu=4.0, seed=seed + 2 * i + 1,
+                                   device=DEV) for i in range(units)])
     layers = list(range(units))
     pk = T.compress(k, S, H, W, bits, layers=layers, kvs=[0] * units, flags=flags)
     pv = T.compress(v, S, H, W, bits, layers=layers, kvs=[1] * units, flags=flags)
@@ -53,6 +54,7 @@ def _run(S, H, W, heads, D, G, bits, flags=0, units=2, qscale=1.0, seed=0):
     (5, 7, 6, 2, 32, 3, 3),        # ragged grid
     (64, 16, 16, 4, 256, 2, 1),    # the 4B-class medical layout (one layer)
     (4, 24, 24, 2, 128, 4, 2),     # the 32B-class slab (24 x 24 cells, 128 channels per head)
+    (8, 8, 8, 1, 64, 8, 2),        # eight query heads per K/V head (the wide values kernel)
 ])
 def test_attention_matches_oracle(S, H, W, heads, D, G, bits):
     _run(S, H, W, heads, D, G, bits)
@@ -62,6 +64,25 @@ def test_attention_matches_oracle(S, H, W, heads, D, G, bits):
                          ids=["rotate", "skip_s_uniform", "head_gain", "head_gain_rotate"])
 def test_attention_with_variant_flags(flags):
     _run(16, 8, 8, 2, 64, 2, 2, flags=flags, seed=5)
+
+
+def test_attention_reads_slabs_too_wide_to_stage():
+    """A slab whose codes span more stream words than the shared-memory rows hold (sized for
+    2 * bits + 2 bits per bin) is decoded from the payload in global memory.  K and V constant along
+    S put the whole budget into the first slab: 8 bits per bin there at 2 bits per element over 4
+    slabs, 64 words per channel against rows of 51."""
+    S, H, W, heads, D, G, bits, units = 4, 16, 16, 2, 64, 2, 2, 2
+    gen = torch.Generator(device=DEV).manual_seed(23)
+
+    def flat_along_s():
+        one = torch.randn((units, 1, H * W, heads, D), generator=gen, device=DEV)
+        return one.expand(units, S, H * W, heads, D).reshape(units, S * H * W, heads, D).to(torch.bfloat16)
+
+    k, v = flat_along_s(), flat_along_s()
+    _run(S, H, W, heads, D, G, bits, units=units, k=k, v=v, seed=23)
+    pk = T.compress(k, S, H, W, bits, layers=[0, 1], kvs=[0, 0])
+    b = O.parse_payload(pk[0].cpu().numpy().tobytes())["b"].reshape(S, H * W)
+    assert b[0].sum() == 8 * H * W and b[1:].sum() == 0   # the first slab takes every bit
 
 
 def test_attention_sharp_scores():
