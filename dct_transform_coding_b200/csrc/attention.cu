@@ -144,7 +144,7 @@ struct BoolTag {
   static constexpr bool value = B;
 };
 
-__global__ void __launch_bounds__(kScoreThreads, 3) attn_scores_kernel(const __grid_constant__ Geom g,
+__global__ void __launch_bounds__(kScoreThreads, 4) attn_scores_kernel(const __grid_constant__ Geom g,
                                                                        const __grid_constant__ UnitList ul,
                                                                        const uint32_t* __restrict__ index,
                                                                        const uint4* __restrict__ recs,
