@@ -319,7 +319,20 @@ __global__ void __launch_bounds__(kSoftmaxThreads, 2) attn_softmax_kernel(const 
   }
   const int W = WX ? WX : g.W, Wr = vol_row(W);   // (a division by a constant on the exact grids)
   auto at = [&](int i) { return (i / W) * Wr + (i - (i / W) * W); };   // bin i -> its padded place
-  for (int i = threadIdx.x; i < g.N; i += blockDim.x) vol[at(i)] = zg[i];
+  constexpr int kBatch = 8;   // loads of z in flight per thread before their stores
+  for (int i0 = threadIdx.x; i0 < g.N; i0 += kBatch * blockDim.x) {
+    float t[kBatch];
+#pragma unroll
+    for (int r = 0; r < kBatch; ++r) {
+      const int i = i0 + r * (int)blockDim.x;
+      t[r] = i < g.N ? zg[i] : 0.f;
+    }
+#pragma unroll
+    for (int r = 0; r < kBatch; ++r) {
+      const int i = i0 + r * (int)blockDim.x;
+      if (i < g.N) vol[at(i)] = t[r];
+    }
+  }
   __syncthreads();
   dct3_volume<true, SX, HX, WX>(vol, g);
   float mx = -INFINITY;
