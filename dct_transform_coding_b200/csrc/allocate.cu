@@ -439,8 +439,10 @@ __global__ void __launch_bounds__(kDecodeIndexThreads) decode_index_kernel(const
   }
   if (ok && !raw) {
     // dense decoding records, one per (slab, row pair kp, column t) at ks*HP*W + kp*W + t:
-    // {sigma of row 2kp, sigma of row 2kp+1, offset << 8 | code mask of each row}, the offset of a
-    // code counted from the first bit of its slab's first stream word (P(k_s) rounded down to 32);
+    // {sigma of row 2kp, sigma of row 2kp+1, shift << 26 | offset << 8 | code mask of each row}, the
+    // offset (18 bits) of a code counted from the first bit of its slab's first stream word (P(k_s)
+    // rounded down to 32), the shift (6 bits) counted from the first bit of the stream word that
+    // holds the row's first code (the decoder's 64-bit window when the row's codes fit in it);
     // a bin without bits (and the padding row of an odd H) has sigma 0, mask 0 and an offset
     // inside its slab's span, so that the decoder may read its (empty) code like any other
     const float* sig = reinterpret_cast<const float*>(pay + g.off_sigma);
@@ -472,6 +474,26 @@ __global__ void __launch_bounds__(kDecodeIndexThreads) decode_index_kernel(const
           rec[1] = 0u;
           rec[3] = (s_P[k] - wbase) << 8;
         }
+      // the shifts: columns t > 0 from their row's first code (column 0, not yet changed), then
+      // column 0 itself
+      __syncwarp();
+      for (int e = lane; e < RP; e += 32) {
+        const int kp = e / g.W;
+        if (e == kp * g.W) continue;
+        uint32_t* rec = urec32 + ((size_t)k * RP + e) * 4;
+        const uint32_t* first = urec32 + ((size_t)k * RP + (size_t)kp * g.W) * 4;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const uint32_t y = rec[2 + r], base = (first[2 + r] >> 8) & 0x3ffe0u;
+          rec[2 + r] = y | (((((y >> 8) & 0x3ffffu) - base) & 63u) << 26);
+        }
+      }
+      __syncwarp();
+      for (int kp = lane; kp < HP; kp += 32) {
+        uint32_t* rec = urec32 + ((size_t)k * RP + (size_t)kp * g.W) * 4;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) rec[2 + r] |= ((rec[2 + r] >> 8) & 31u) << 26;
+      }
     }
   }
 }

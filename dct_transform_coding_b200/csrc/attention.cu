@@ -72,6 +72,7 @@ __device__ int stage_active(const uint4* __restrict__ srec, int HW, int W, uint2
       const int kh = j / W, t = j - kh * W;
       const uint4 m = srec[(kh >> 1) * W + t];
       r = (kh & 1) ? make_uint2(m.y, m.w) : make_uint2(m.x, m.z);
+      r.y &= 0x03ffffffu;   // offset << 8 | mask (the decoder's window shift dropped)
     }
     const bool has = (r.y & 0xffu) != 0u;
     const unsigned bal = __ballot_sync(0xffffffffu, has);

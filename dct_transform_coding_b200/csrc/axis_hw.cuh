@@ -345,14 +345,16 @@ __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul,
         // lvs1[-1] is the zero in front of the levels: a bin without bits (mask 0) reads it, so
         // every code is read the same way, without a branch
         const float* lvs1 = lvs + 1;
-        const uint4* rr = rs + kp * D.W;   // record: sigma of each row, offset << 8 | code mask of each row
+        // record: sigma of each row, shift << 26 | offset << 8 | code mask of each row
+        const uint4* rr = rs + kp * D.W;
         // Each row's bins are consecutive in the stream: from its first bin's offset to its last
         // bin's offset plus its bits.  When each row's bits lie in two stream words (most rows at
-        // 1-3 bits per element), those words are read once and every code is shifted out of them.
+        // 1-3 bits per element), those words are read once and every code is shifted out of them
+        // by the shift its record carries.
         const uint4 mf = rr[0], ml = rr[D.W - 1];
-        const uint32_t base0 = (mf.z >> 8) & ~31u, base1 = (mf.w >> 8) & ~31u;
-        const uint32_t end0 = (ml.z >> 8) + (uint32_t)__popc(ml.z & 0xffu);
-        const uint32_t end1 = (ml.w >> 8) + (uint32_t)__popc(ml.w & 0xffu);
+        const uint32_t base0 = (mf.z >> 8) & 0x3ffe0u, base1 = (mf.w >> 8) & 0x3ffe0u;
+        const uint32_t end0 = ((ml.z >> 8) & 0x3ffffu) + (uint32_t)__popc(ml.z & 0xffu);
+        const uint32_t end1 = ((ml.w >> 8) & 0x3ffffu) + (uint32_t)__popc(ml.w & 0xffu);
         if (end0 <= base0 + 64u && end1 <= base1 + 64u) {
           const unsigned long long win0 = ((unsigned long long)row[(base0 >> 5) + 1] << 32) | row[base0 >> 5];
           const unsigned long long win1 = ((unsigned long long)row[(base1 >> 5) + 1] << 32) | row[base1 >> 5];
@@ -361,9 +363,9 @@ __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul,
             if (t < D.W) {
               const uint4 m = rr[t];
               const uint32_t k0 = m.z & 0xffu, k1 = m.w & 0xffu;
-              // (a code's shift is below 64; a bin without bits has mask 0 whatever its shift)
-              const uint32_t c0 = (uint32_t)(win0 >> (((m.z >> 8) - base0) & 63u)) & k0;
-              const uint32_t c1 = (uint32_t)(win1 >> (((m.w >> 8) - base1) & 63u)) & k1;
+              // (a bin without bits has mask 0 whatever its shift)
+              const uint32_t c0 = (uint32_t)(win0 >> (m.z >> 26)) & k0;
+              const uint32_t c1 = (uint32_t)(win1 >> (m.w >> 26)) & k1;
               const float l0 = lvs1[(int)(k0 + c0) - 1], l1 = lvs1[(int)(k1 + c1) - 1];
               float s0 = __uint_as_float(m.x), s1 = __uint_as_float(m.y);
               if (VAR && hgain) {   // (a row without bits keeps its gain 0; the padding row reads nothing)
@@ -379,7 +381,8 @@ __device__ __forceinline__ void idct_hw_slabs(const Geom& g, const UnitList& ul,
             if (t < D.W) {
               const uint4 m = rr[t];
               const uint32_t k0 = m.z & 0xffu, k1 = m.w & 0xffu;
-              const uint32_t off0 = m.z >> 8, off1 = m.w >> 8;   // from the slab's first word
+              // offsets from the slab's first word
+              const uint32_t off0 = (m.z >> 8) & 0x3ffffu, off1 = (m.w >> 8) & 0x3ffffu;
               const uint32_t* w0 = row + (off0 >> 5);
               const uint32_t* w1 = row + (off1 >> 5);
               const float l0 = lvs1[(int)(k0 + (__funnelshift_r(w0[0], w0[1], off0) & k0)) - 1];
