@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(kPackThreads, 4) pack_kernel(const __grid_cons
   uint32_t* words_out = reinterpret_cast<uint32_t*>(pay + g.off_codes) + (size_t)chunk0 * kChunk * sw;
 
   // Thread t holds records t, t + 256, ... of the range (empty slots past m have width 0).
-  constexpr int kPer = R / kPackThreads;
+  constexpr int kPer = (R + kPackThreads - 1) / kPackThreads;
   uint4 mine[kPer];
 #pragma unroll
   for (int q = 0; q < kPer; ++q) {
@@ -354,7 +354,7 @@ cudaError_t launch_pack(const Geom& g, const UnitList& ul, int nu, const float* 
   } else {
     // four channels per lane where the chunks come in fours, else one; a unit has at most N
     // records, CTAs past its last record exit (measured: a CTA looping over two ranges, to launch
-    // fewer CTAs without work, was slower)
+    // fewer CTAs without work, was slower; so were eight channels per lane, ranges of 128 records)
     auto go = [&](auto kernel, int cpl, size_t smem, int recs_per_cta) {
       cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       const dim3 grid(g.nch / cpl, (g.N + recs_per_cta - 1) / recs_per_cta, nu);

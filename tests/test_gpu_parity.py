@@ -216,6 +216,7 @@ def test_cross_decode_oracle_payload_on_gpu():
     ((8, 8, 8, 1, 64), 2),     # two chunks: one channel per lane, one packing range
     ((8, 8, 8, 4, 32), 2),     # four chunks: four channels per lane, ranges of 256 records
     ((16, 8, 8, 4, 32), 1),    # likewise, more ranges at 1 bit
+    ((16, 8, 8, 8, 32), 2),    # eight chunks: two CTAs of four channels per lane side by side
 ])
 def test_payload_bytes_match_oracle_format(shape, bits):
     """Where allocations and codes agree, the GPU payload is byte-identical to the oracle's."""
