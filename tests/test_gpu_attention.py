@@ -55,6 +55,7 @@ def _run(S, H, W, heads, D, G, bits, flags=0, units=2, qscale=1.0, seed=0, k=Non
     (64, 16, 16, 4, 256, 2, 1),    # the 4B-class medical layout (one layer)
     (4, 24, 24, 2, 128, 4, 2),     # the 32B-class slab (24 x 24 cells, 128 channels per head)
     (8, 8, 8, 1, 64, 8, 2),        # eight query heads per K/V head (the wide values kernel)
+    (8, 32, 32, 1, 256, 2, 1),     # the largest slab, 256 channels: rows fit only at a low rate
 ])
 def test_attention_matches_oracle(S, H, W, heads, D, G, bits):
     _run(S, H, W, heads, D, G, bits)

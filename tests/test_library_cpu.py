@@ -118,6 +118,32 @@ def test_allocate_argument_checks_without_gpu(T):
     assert T.tactkv_allocate(_unit(T, flags=128), 4096, 1 << 20, 1 << 30, 0) == T.TACTKV_INVALID_ARG
 
 
+def _attention_status(T, S, H, W, heads, D, bits, q_heads, flags=0):
+    """tactkv_attention_decode's host checks only: fake device pointers and a null workspace, so a
+    call that passes the shape checks stops at TACTKV_WORKSPACE before anything is launched."""
+    ku = (T.tactkv_unit * 1)(_unit(T, S=S, H=H, W=W, heads=heads, head_dim=D, bits=bits, flags=flags, kv=0,
+                                   payload_capacity=1 << 40))
+    vu = (T.tactkv_unit * 1)(_unit(T, S=S, H=H, W=W, heads=heads, head_dim=D, bits=bits, flags=flags, kv=1,
+                                   payload_capacity=1 << 40))
+    p = ctypes.c_void_p(4096)
+    return int(T._lib.tactkv_attention_decode(ku, vu, 1, q_heads, p, p, p, p, None, 0, None))
+
+
+@pytest.mark.parametrize("shape,bits,q_heads,flags,status", [
+    ((64, 16, 16, 4, 256), 1, 8, 0, "TACTKV_WORKSPACE"),       # the benchmark layer: supported
+    ((64, 16, 16, 4, 256), 1, 8, 1, "TACTKV_UNSUPPORTED_SHAPE"),   # NO_QUANT payloads
+    ((64, 16, 16, 4, 256), 1, 6, 0, "TACTKV_UNSUPPORTED_SHAPE"),   # q_heads not a multiple of heads
+    ((8, 8, 8, 1, 64), 2, 17, 0, "TACTKV_UNSUPPORTED_SHAPE"),      # more than 16 query heads per K/V head
+    # the stream-word rows are sized for min(8, 2*bits + 2) bits per bin: a 32 x 32 slab of 256
+    # channels fits at 1 bit per element (131 words per channel) but not at 4 (259 words, 265 KB)
+    ((8, 32, 32, 1, 256), 1, 2, 0, "TACTKV_WORKSPACE"),
+    ((8, 32, 32, 1, 256), 4, 2, 0, "TACTKV_UNSUPPORTED_SHAPE"),
+])
+def test_attention_shape_checks_without_gpu(T, shape, bits, q_heads, flags, status):
+    S, H, W, heads, D = shape
+    assert _attention_status(T, S, H, W, heads, D, bits, q_heads, flags) == getattr(T, status)
+
+
 def test_decompress_checks_output_pointer(T):
     units = [_unit(T, kv_out=None)]
     assert T.tactkv_decompress(units, 1 << 20, 1 << 30, 0) == T.TACTKV_INVALID_ARG
