@@ -7,8 +7,9 @@
 // chunks, range of records); lane l of a warp packs channel l of each of its CPL chunks, so every
 // decision about a record is uniform across the warp and only the coefficient values differ.  CPL
 // is 4 on the default path (a record's position, width and gain are read and turned into a word and
-// a shift once for four channels; ranges of kPackRecs records) and 1 for the variant kernels
-// (ranges of 4 * kPackRecs).  Bins without bits are never read.
+// a shift once for four channels; ranges of kPackRecs records) and 1 for the variant kernels and for
+// channel counts whose chunks do not come in fours (ranges of 4 * kPackRecs).  Bins without bits are
+// never read.
 //
 // The CTA clears the word rows of its bit span in shared memory and puts its records there grouped
 // by bit width (records are independent of each other: each carries its stream position), each
