@@ -17,8 +17,9 @@
  * i = (k_s*H + k_h)*W + k_w, N = T bins.  Nominal budget: bits*N bit slots per channel.
  *
  * Memory.  Every pointer in a unit descriptor and the workspace are DEVICE pointers owned by
- * the caller.  The library allocates nothing.  Its only state is the constant tables in the CUDA
- * module and the fixed device scratch array of tactkv_compress_noalloc (below); every other entry
+ * the caller.  The library allocates nothing.  Its only state is the read-only tables in the CUDA
+ * module (constant memory, and 16-byte-aligned copies in global memory that kernels stage into
+ * shared memory) and the fixed device scratch array of tactkv_compress_noalloc (below); every other entry
  * point is safe to call from several host threads on different streams provided each call has
  * its own workspace.  Calls are asynchronous on `stream`; a status other than
  * TACTKV_OK means nothing was launched for the failing group of units (earlier groups of the
