@@ -196,13 +196,25 @@ def generate() -> str:
     lv0 += [0.0] * (-len(lv0) % 4)
     thr16 = pad_all + [math.inf] * (-len(pad_all) % 4)
     q16 = qtab + [0] * (-len(qtab) % 16)
+    # for b >= 3, the pair (t_c, t_{c+1}) of padded thresholds for every count c = 0 .. 2^b - 1,
+    # width b's pairs from pair 2^b - 8 on: the two compares after the cell lookup take one load
+    pairs = []
+    for b in range(3, 9):
+        o = (1 << b) + b - 3
+        assert len(pairs) == 2 * ((1 << b) - 8)
+        for c in range(1 << b):
+            pairs += [pad_all[o + c], pad_all[o + c + 1]]
+    pairs += [math.inf] * (-len(pairs) % 4)
     lines += [f"#define TACTKV_LV0_VEC {len(lv0) // 4}",
               f"#define TACTKV_THR_VEC {len(thr16) // 4}",
+              f"#define TACTKV_THR_PAIR_VEC {len(pairs) // 4}",
               f"#define TACTKV_QCELL_VEC {len(q16) // 16}",
               "static __device__ __align__(16) const float g_lm_levels0[] = {"]
     lines += ["  " + ", ".join(lit(v) for v in lv0[i:i + 4]) + "," for i in range(0, len(lv0), 4)]
     lines += ["};", "static __device__ __align__(16) const float g_thr_pad[] = {"]
     lines += ["  " + ", ".join(lit(v) for v in thr16[i:i + 4]) + "," for i in range(0, len(thr16), 4)]
+    lines += ["};", "static __device__ __align__(16) const float g_thr_pairs[] = {"]
+    lines += ["  " + ", ".join(lit(v) for v in pairs[i:i + 4]) + "," for i in range(0, len(pairs), 4)]
     lines += ["};", "static __device__ __align__(16) const unsigned char g_qcell[] = {"]
     lines += ["  " + ", ".join(str(v) for v in q16[i:i + 32]) + "," for i in range(0, len(q16), 32)]
     lines += ["};", "#endif", ""]

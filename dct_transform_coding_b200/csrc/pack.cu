@@ -49,11 +49,8 @@ template <int CPL>
 __host__ __device__ constexpr int pack_pad_word() { return (8 * pack_recs<CPL>() + 31) / 32 + 1; }
 static_assert(pack_pad_word<1>() + 2 <= pack_words<1>() && pack_pad_word<4>() + 2 <= pack_words<4>(), "rows");
 
-// Thresholds of width b padded with two +inf, stored for b = 1, 2, ... in turn.
-__device__ __forceinline__ int thr_pad_offset(int b) { return (1 << b) + b - 3; }
-
 struct PackLayout {
-  size_t rec, sbuf, thr, qcell, total;
+  size_t rec, sbuf, thr2, qcell, total;
 };
 // A range's records grouped by bit width, each group padded to whole blocks; then the word rows of
 // the CPL * 32 channels and the codebook tables.
@@ -64,7 +61,7 @@ __host__ __device__ inline PackLayout pack_layout() {
   size_t o = 0;
   L.rec = o; o += p16((size_t)(pack_recs<CPL>() + 8 * pack_block<CPL>()) * 16);
   L.sbuf = o; o += p16((size_t)CPL * kChunk * pack_words<CPL>() * 4);
-  L.thr = o; o += (size_t)TACTKV_THR_VEC * 16;
+  L.thr2 = o; o += (size_t)TACTKV_THR_PAIR_VEC * 16;
   L.qcell = o; o += (size_t)TACTKV_QCELL_VEC * 16;
   L.total = o;
   return L;
@@ -75,9 +72,11 @@ __host__ __device__ inline PackLayout pack_layout() {
 // the sign test, which needs no gain (1/sigma is positive and finite, so u >= 0 exactly when
 // x >= 0); b = 2: three compares against {-t, 0, t}; b >= 3: the cell of u in a uniform grid gives
 // the count c of thresholds below the cell, and two compares finish it (a cell holds at most two
-// thresholds; the thresholds are padded with +inf).
+// thresholds; the thresholds are padded with +inf), against the pair (t_c, t_{c+1}) read in one
+// load (pair 2^b - 8 + c).  The cell index saturates: the conversion to unsigned takes values
+// below the grid to 0, min() those above it to the last cell.
 template <int B>
-__device__ __forceinline__ uint32_t quant_code_b(float x, float inv_sigma, int b, const float* __restrict__ thr,
+__device__ __forceinline__ uint32_t quant_code_b(float x, float inv_sigma, int b, const float2* __restrict__ thr2,
                                                  const unsigned char* __restrict__ qcell) {
   if constexpr (B == 1) {
     return x >= 0.f;
@@ -86,11 +85,10 @@ __device__ __forceinline__ uint32_t quant_code_b(float x, float inv_sigma, int b
     if constexpr (B == 2) {
       return (uint32_t)(u >= -TACTKV_LM_T2) + (uint32_t)(u >= 0.f) + (uint32_t)(u >= TACTKV_LM_T2);
     } else {
-      int j = __float2int_rd(fmaf(u, TACTKV_Q_SCALE, TACTKV_Q_OFFSET));
-      j = min(max(j, 0), TACTKV_Q_CELLS - 1);
+      const uint32_t j = min(__float2uint_rd(fmaf(u, TACTKV_Q_SCALE, TACTKV_Q_OFFSET)), TACTKV_Q_CELLS - 1u);
       const uint32_t c = qcell[(b - 3) * TACTKV_Q_CELLS + j];
-      const float* t = thr + thr_pad_offset(b) + c;
-      return c + (uint32_t)(u >= t[0]) + (uint32_t)(u >= t[1]);
+      const float2 t = thr2[(1 << b) - 8 + c];
+      return c + (uint32_t)(u >= t.x) + (uint32_t)(u >= t.y);
     }
   }
 }
@@ -110,7 +108,7 @@ __device__ __forceinline__ void red_or_shared(uint32_t* p, uint32_t v) {
 template <int B, int CPL, int PB>
 __device__ __forceinline__ void pack_block(const uint4* __restrict__ rs, const float (&x)[PB][CPL],
                                            uint32_t* __restrict__ row, uint32_t base, int b,
-                                           const float* __restrict__ thr, const unsigned char* __restrict__ qcell) {
+                                           const float2* __restrict__ thr2, const unsigned char* __restrict__ qcell) {
   constexpr int kRowStride = kChunk * pack_words<CPL>();
   uint2 r[PB];
 #pragma unroll
@@ -119,7 +117,7 @@ __device__ __forceinline__ void pack_block(const uint4* __restrict__ rs, const f
 #pragma unroll
   for (int j = 0; j < PB; ++j)
 #pragma unroll
-    for (int k = 0; k < CPL; ++k) code[j][k] = quant_code_b<B>(x[j][k], __uint_as_float(r[j].y), b, thr, qcell);
+    for (int k = 0; k < CPL; ++k) code[j][k] = quant_code_b<B>(x[j][k], __uint_as_float(r[j].y), b, thr2, qcell);
 #pragma unroll
   for (int j = 0; j < PB; ++j) {
     const uint32_t off = r[j].x - base, w = off >> 5, sh = off & 31u;
@@ -165,7 +163,7 @@ __global__ void __launch_bounds__(kPackThreads, 4) pack_kernel(const __grid_cons
   const float* xu = X + (size_t)u * g.N * g.n + chunk0 * kChunk + lane;
   uint4* rs = reinterpret_cast<uint4*>(smem + L.rec);
   uint32_t* sbuf = reinterpret_cast<uint32_t*>(smem + L.sbuf);
-  float* thr = reinterpret_cast<float*>(smem + L.thr);
+  float2* thr2 = reinterpret_cast<float2*>(smem + L.thr2);
   unsigned char* qcell = smem + L.qcell;
   const uint32_t cstride = reinterpret_cast<const uint32_t*>(pay)[11], sw = cstride / 4;
   uint32_t* words_out = reinterpret_cast<uint32_t*>(pay + g.off_codes) + (size_t)chunk0 * kChunk * sw;
@@ -189,7 +187,7 @@ __global__ void __launch_bounds__(kPackThreads, 4) pack_kernel(const __grid_cons
       }
   }
   if (threadIdx.x < 9 * kWarps) (&s_cnt[0][0])[threadIdx.x] = 0u;
-  copy_vec16(thr, g_thr_pad, TACTKV_THR_VEC);
+  copy_vec16(thr2, g_thr_pairs, TACTKV_THR_PAIR_VEC);
   copy_vec16(qcell, g_qcell, TACTKV_QCELL_VEC);
   // bit span [A, B) of the range; its words from word A >> 5 on are assembled in shared memory
   const uint32_t A = m > 0 ? urecs[r0].z : code_bits;
@@ -285,9 +283,9 @@ __global__ void __launch_bounds__(kPackThreads, 4) pack_kernel(const __grid_cons
     }
     const uint4* blk = rs + e0;
     const int b = (int)blk[0].y;
-    if (b == 1) pack_block<1, CPL, PB>(blk, x, row, base, 1, thr, qcell);
-    else if (b == 2) pack_block<2, CPL, PB>(blk, x, row, base, 2, thr, qcell);
-    else pack_block<0, CPL, PB>(blk, x, row, base, b, thr, qcell);
+    if (b == 1) pack_block<1, CPL, PB>(blk, x, row, base, 1, thr2, qcell);
+    else if (b == 2) pack_block<2, CPL, PB>(blk, x, row, base, 2, thr2, qcell);
+    else pack_block<0, CPL, PB>(blk, x, row, base, b, thr2, qcell);
 #pragma unroll
     for (int j = 0; j < PB; ++j)
 #pragma unroll

@@ -248,8 +248,9 @@ def _c_array(text, name):
 
 def test_global_table_copies_match_the_constant_tables():
     """The 16-byte-vector copies of the codebook tables that kernels stage into shared memory: the
-    levels behind a leading zero, the padded thresholds and the code cells, each equal to its
-    constant-memory table and padded to whole 16-byte vectors."""
+    levels behind a leading zero, the padded thresholds, the threshold pairs the packer compares
+    against after its cell lookup, and the code cells, each equal to its constant-memory table and
+    padded to whole 16-byte vectors."""
     G = _gen_tables()
     text = G.generate()
     lv, lv0 = _c_array(text, "c_lm_levels"), _c_array(text, "g_lm_levels0")
@@ -259,7 +260,15 @@ def test_global_table_copies_match_the_constant_tables():
     assert all(v == 0.0 for v in lv0[len(lv) + 1:])
     assert thr16[:len(thr)] == thr and len(thr16) % 4 == 0 and all(np.isinf(thr16[len(thr):]))
     assert q16[:len(q)] == q and len(q16) % 16 == 0
-    for name, vals, per in (("LV0", lv0, 4), ("THR", thr16, 4), ("QCELL", q16, 16)):
+    # the pairs (t_c, t_c+1) of each width b >= 3 from pair 2^b - 8 on, c = 0 .. 2^b - 1
+    pairs = _c_array(text, "g_thr_pairs")
+    for b in range(3, 9):
+        o = (1 << b) + b - 3          # width b's first threshold among the padded ones
+        for c in range(1 << b):
+            p = (1 << b) - 8 + c
+            assert pairs[2 * p] == thr[o + c] and pairs[2 * p + 1] == thr[o + c + 1]
+    assert np.isinf(thr[(1 << 8) + 8 - 3 + 255]) and np.isinf(pairs[2 * (504 - 1) + 1])
+    for name, vals, per in (("LV0", lv0, 4), ("THR", thr16, 4), ("THR_PAIR", pairs, 4), ("QCELL", q16, 16)):
         assert f"#define TACTKV_{name}_VEC {len(vals) // per}" in text
 
 
