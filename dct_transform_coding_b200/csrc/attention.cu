@@ -8,8 +8,9 @@
 //   output   o_j    = sum_t p_j[t] V[t]    = sum_i dct3(p_j)[i] X_V[i, hD + d]
 // with p_j[t] = exp(s_j[t] - m_j), m_j = max_t s_j[t], l_j = sum_t p_j[t], and out_j = o_j / l_j
 // (query head j uses K/V head h = j / G).  Only bins with bits are decoded, from each slab's words
-// of the payloads' channel streams staged in shared memory; the volumes of T values per query head
-// are transformed in shared memory.  A unit whose K or V payload fails the index checks contributes
+// of the payloads' channel streams staged in shared memory (read from the payload directly when a
+// slab's codes span more than the rows, sized for the call's rate, hold); the volumes of T values
+// per query head are transformed in shared memory.  A unit whose K or V payload fails the index checks contributes
 // no tokens (out 0, m -inf, l 0).  With the shared rotation R (per 32-channel group), X = R^T X' for the coded X': the
 // query is rotated (q . R^T x' = (R q) . x') and the output rotated back at the end.
 //
