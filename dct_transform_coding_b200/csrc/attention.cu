@@ -10,9 +10,10 @@
 // (query head j uses K/V head h = j / G).  Only bins with bits are decoded, from each slab's words
 // of the payloads' channel streams staged in shared memory (read from the payload directly when a
 // slab's codes span more than the rows, sized for the call's rate, hold); the volumes of T values
-// per query head are transformed in shared memory.  A unit whose K or V payload fails the index checks contributes
-// no tokens (out 0, m -inf, l 0).  With the shared rotation R (per 32-channel group), X = R^T X' for the coded X': the
-// query is rotated (q . R^T x' = (R q) . x') and the output rotated back at the end.
+// per query head are transformed in shared memory.  A unit whose K or V payload fails the index
+// checks contributes no tokens (out 0, m -inf, l 0).  With the shared rotation R (per 32-channel
+// group), X = R^T X' for the coded X': the query is rotated (q . R^T x' = (R q) . x') and the
+// output rotated back at the end.
 //
 // Kernels (one launch each, all units of a call share one shape):
 //   decode_index   (allocate.cu) the K and V payloads' checks, slab offsets and dense records;
